@@ -1,0 +1,186 @@
+"""fp64 CPU oracle for SS2D (CrossScan -> S6 selective scan -> CrossMerge).
+
+TEST INFRASTRUCTURE ONLY.  This package is the checker that the CUDA library
+is compared against.  It shares no code with the CUDA path; only the tests,
+``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` may use it.
+
+Sources of the arithmetic (restated, not copied):
+
+* "VMamba: Visual State Space Model", section "2D Selective Scan (SS2D) for
+  visual data" and Fig. 2: CrossScan unfolds the map along four paths, one S6
+  block per path, CrossMerge sums the four results back into the map.
+* "vision mamba-yolov8", section "2. Vmamba module code", ``selective_scan_ref``:
+  the S6 recurrence with softplus step size and grouped B/C.
+
+The numerical work lives in ``ss2d_oracle.c`` (plain loops, double precision);
+this module compiles it with gcc on first use and marshals numpy arrays.
+Inputs may be any real dtype; they are converted to float64 exactly
+(bf16 / fp32 values are representable in fp64).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "ss2d_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+K_PATHS = 4
+
+
+def build(force: bool = False) -> str:
+    """Compile ``ss2d_oracle.c`` into ``liboracle.so`` (gcc, -O2, OpenMP)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-fno-fast-math",
+               "-ffp-contract=off", _SRC, "-o", tmp, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB_PATH)
+            P = ctypes.POINTER(ctypes.c_double)
+            l = ctypes.c_long
+            lib.oracle_path_pixel.argtypes = [ctypes.c_int, l, l, l]
+            lib.oracle_path_pixel.restype = l
+            lib.oracle_cross_scan.argtypes = [l, l, l, l, P, P]
+            lib.oracle_cross_merge.argtypes = [l, l, l, l, P, P]
+            lib.oracle_selective_scan_fwd.argtypes = [l, l, l, l, l, P, P, P, P, P, P, P,
+                                                      ctypes.c_int, P, P]
+            lib.oracle_selective_scan_bwd.argtypes = [l, l, l, l, l, P, P, P, P, P, P, P,
+                                                      ctypes.c_int, P, P, P, P, P, P, P, P]
+            lib.oracle_ss2d_forward.argtypes = [l, l, l, l, l, P, P, P, P, P, P, P, ctypes.c_int, P]
+            lib.oracle_ss2d_backward.argtypes = [l, l, l, l, l, P, P, P, P, P, P, P, ctypes.c_int,
+                                                 P, P, P, P, P, P, P, P]
+            lib.oracle_num_threads.restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def _f64(a):
+    """Contiguous float64 copy of an array-like (torch tensors included)."""
+    if a is None:
+        return None
+    if hasattr(a, "detach"):  # torch tensor: exact upcast on the host
+        a = a.detach().to("cpu").double().numpy()
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def path_pixel(k: int, l: int, H: int, W: int) -> int:
+    """Pixel index h*W+w visited at step l of path k."""
+    return int(_load().oracle_path_pixel(int(k), int(l), int(H), int(W)))
+
+
+def cross_scan(x):
+    """x (B, D, H, W) -> xs (B, 4, D, H*W)."""
+    x = _f64(x)
+    Bn, Dn, H, W = x.shape
+    xs = np.empty((Bn, K_PATHS, Dn, H * W), dtype=np.float64)
+    _load().oracle_cross_scan(Bn, Dn, H, W, _ptr(x), _ptr(xs))
+    return xs
+
+
+def cross_merge(ys, H: int, W: int):
+    """ys (B, 4, D, H*W) -> y (B, D, H, W), summed as (y0 + y2) + (y1 + y3)."""
+    ys = _f64(ys)
+    Bn, K, Dn, L = ys.shape
+    assert K == K_PATHS and L == H * W
+    y = np.empty((Bn, Dn, H, W), dtype=np.float64)
+    _load().oracle_cross_merge(Bn, Dn, H, W, _ptr(ys), _ptr(y))
+    return y
+
+
+def selective_scan_fwd(u, delta, A, B, C, D=None, delta_bias=None, delta_softplus=False,
+                       return_last_state=False):
+    """S6 forward.  u, delta (Bn, Ch, L); A (Ch, N); B, C (Bn, G, N, L); D, delta_bias (Ch)."""
+    u, delta, A, B, C = (_f64(t) for t in (u, delta, A, B, C))
+    D, delta_bias = _f64(D), _f64(delta_bias)
+    Bn, Ch, L = u.shape
+    N = A.shape[1]
+    G = B.shape[1]
+    assert delta.shape == u.shape and A.shape == (Ch, N) and B.shape == (Bn, G, N, L)
+    assert C.shape == B.shape and Ch % G == 0
+    out = np.empty_like(u)
+    last = np.empty((Bn, Ch, N), dtype=np.float64) if return_last_state else None
+    _load().oracle_selective_scan_fwd(Bn, Ch, L, N, G, _ptr(u), _ptr(delta), _ptr(A), _ptr(B),
+                                      _ptr(C), _ptr(D), _ptr(delta_bias), int(bool(delta_softplus)),
+                                      _ptr(out), _ptr(last))
+    return (out, last) if return_last_state else out
+
+
+def selective_scan_bwd(u, delta, A, B, C, D, delta_bias, delta_softplus, dout):
+    """S6 backward.  Returns dict du, ddelta, dA, dB, dC, dD, ddelta_bias (None when absent)."""
+    u, delta, A, B, C, dout = (_f64(t) for t in (u, delta, A, B, C, dout))
+    D, delta_bias = _f64(D), _f64(delta_bias)
+    Bn, Ch, L = u.shape
+    N = A.shape[1]
+    G = B.shape[1]
+    du = np.empty_like(u)
+    ddelta = np.empty_like(u)
+    dA = np.empty_like(A)
+    dB = np.empty_like(B)
+    dC = np.empty_like(C)
+    dD = np.empty(Ch, dtype=np.float64) if D is not None else None
+    dbias = np.empty(Ch, dtype=np.float64) if delta_bias is not None else None
+    _load().oracle_selective_scan_bwd(Bn, Ch, L, N, G, _ptr(u), _ptr(delta), _ptr(A), _ptr(B),
+                                      _ptr(C), _ptr(D), _ptr(delta_bias), int(bool(delta_softplus)),
+                                      _ptr(dout), _ptr(du), _ptr(ddelta), _ptr(dA), _ptr(dB),
+                                      _ptr(dC), _ptr(dD), _ptr(dbias))
+    return dict(du=du, ddelta=ddelta, dA=dA, dB=dB, dC=dC, dD=dD, ddelta_bias=dbias)
+
+
+def ss2d_forward(x, delta, A, B, C, D=None, delta_bias=None, delta_softplus=True):
+    """Full SS2D forward.  x (Bn, D, H, W) -> y (Bn, D, H, W)."""
+    x, delta, A, B, C = (_f64(t) for t in (x, delta, A, B, C))
+    D, delta_bias = _f64(D), _f64(delta_bias)
+    Bn, Dn, H, W = x.shape
+    N = A.shape[1]
+    assert delta.shape == (Bn, K_PATHS * Dn, H * W) and A.shape == (K_PATHS * Dn, N)
+    assert B.shape == (Bn, K_PATHS, N, H * W) and C.shape == B.shape
+    y = np.empty_like(x)
+    _load().oracle_ss2d_forward(Bn, Dn, H, W, N, _ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C),
+                                _ptr(D), _ptr(delta_bias), int(bool(delta_softplus)), _ptr(y))
+    return y
+
+
+def ss2d_backward(x, delta, A, B, C, D, delta_bias, delta_softplus, dy):
+    """Full SS2D backward.  Returns dict dx, ddelta, dA, dB, dC, dD, ddelta_bias."""
+    x, delta, A, B, C, dy = (_f64(t) for t in (x, delta, A, B, C, dy))
+    D, delta_bias = _f64(D), _f64(delta_bias)
+    Bn, Dn, H, W = x.shape
+    N = A.shape[1]
+    dx = np.empty_like(x)
+    ddelta = np.empty_like(delta)
+    dA = np.empty_like(A)
+    dB = np.empty_like(B)
+    dC = np.empty_like(C)
+    dD = np.empty(K_PATHS * Dn, dtype=np.float64) if D is not None else None
+    dbias = np.empty(K_PATHS * Dn, dtype=np.float64) if delta_bias is not None else None
+    _load().oracle_ss2d_backward(Bn, Dn, H, W, N, _ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C),
+                                 _ptr(D), _ptr(delta_bias), int(bool(delta_softplus)), _ptr(dy),
+                                 _ptr(dx), _ptr(ddelta), _ptr(dA), _ptr(dB), _ptr(dC), _ptr(dD),
+                                 _ptr(dbias))
+    return dict(dx=dx, ddelta=ddelta, dA=dA, dB=dB, dC=dC, dD=dD, ddelta_bias=dbias)
