@@ -1,0 +1,226 @@
+/*
+ * ss2d.h -- C ABI of libss2d: VMamba's 2D selective scan (SS2D) on NVIDIA B200 (sm_100a).
+ *
+ * SS2D ("VMamba: Visual State Space Model", section "2D Selective Scan (SS2D)
+ * for visual data", Fig. 2) has three steps:
+ *   CrossScan  -- unfold a (B, D, H, W) map into K = 4 sequences of length
+ *                 L = H*W: row-major (k=0), column-major (k=1, step l = w*H + h)
+ *                 and the two reversed (k=2 reverses k=0, k=3 reverses k=1);
+ *   S6         -- one selective scan per sequence (channel c = k*D + d uses the
+ *                 B/C group k): dt = softplus(delta + delta_bias),
+ *                 h = exp(dt*A[c,n]) * h + dt * B[n,l] * u,
+ *                 y = sum_n C[n,l] * h[n] + D[c] * u, with h = 0 at l = 0
+ *                 ("vision mamba-yolov8", section "2. Vmamba module code",
+ *                 selective_scan_ref);
+ *   CrossMerge -- put the four outputs back in image order and sum them,
+ *                 computed as (y0 + y2) + (y1 + y3) in fp32 and rounded once.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor pointers are DEVICE pointers, owned by the caller, fully
+ *    contiguous (row-major) in the layouts stated per argument.  The library
+ *    never allocates, frees or synchronises; every kernel is enqueued on
+ *    `stream` (a cudaStream_t; NULL means the legacy default stream).
+ *  - Element types: u/x, delta, B, C (and the gradients of those) have
+ *    desc->in_dtype; outputs y/out have desc->out_dtype.  A, D, delta_bias,
+ *    dA, dD, ddelta_bias and chunk states are always fp32.  The state h and all
+ *    accumulation are fp32 whatever the I/O type.
+ *  - Optional pointers (D, delta_bias, chunk_states, and their gradients) may
+ *    be NULL; a NULL D means no skip term, a NULL delta_bias means zero bias.
+ *  - Errors: arguments are validated on the host BEFORE anything is launched;
+ *    a bad argument returns its status and enqueues nothing.  A failed launch
+ *    returns SS2D_ERR_LAUNCH.  No exception or abort crosses the ABI.  NaN/Inf
+ *    in the data propagate and are not checked.
+ *  - Gradients are written, not accumulated into what the caller's buffer held.
+ *  - Pointers must be 16-byte aligned (what cudaMalloc and the PyTorch caching
+ *    allocator return for tensors that start at the beginning of their storage).
+ */
+#ifndef SS2D_H
+#define SS2D_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SS2D_API __attribute__((visibility("default")))
+#else
+#define SS2D_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* forward declaration of the CUDA runtime's stream type, so this header needs no CUDA include */
+struct CUstream_st;
+typedef struct CUstream_st *ss2d_stream_t;
+
+typedef enum {
+    SS2D_OK = 0,
+    SS2D_ERR_NULL = 1,      /* a required pointer is NULL */
+    SS2D_ERR_SHAPE = 2,     /* a size is <= 0, too large, or inconsistent (e.g. d_state > 16) */
+    SS2D_ERR_DTYPE = 3,     /* unsupported dtype or dtype combination */
+    SS2D_ERR_ALIGN = 4,     /* a pointer is not 16-byte aligned */
+    SS2D_ERR_WORKSPACE = 5, /* workspace NULL or smaller than ss2d_workspace_bytes() */
+    SS2D_ERR_LAUNCH = 6,    /* the CUDA launch failed (see ss2d_last_cuda_error()) */
+    SS2D_ERR_TIMEOUT = 7,   /* reserved: a bounded device-side wait gave up */
+    SS2D_ERR_DEVICE = 8     /* no usable CUDA device, or not an sm_100 device */
+} ss2d_status_t;
+
+typedef enum { SS2D_F32 = 0, SS2D_BF16 = 1 } ss2d_dtype_t;
+
+/* Problem description.  K = 4 paths is fixed; channels of the sequence view = 4*dim;
+ * sequence length L = height*width.  A 1-D problem is height = 1, width = L. */
+typedef struct {
+    int64_t batch;          /* B >= 1 */
+    int64_t dim;            /* D >= 1: channels of the image; the sequence view has 4*D */
+    int64_t height;         /* H >= 1 */
+    int64_t width;          /* W >= 1 */
+    int64_t d_state;        /* N, 1 <= N <= 16 */
+    ss2d_dtype_t in_dtype;  /* type of u/x, delta, B, C */
+    ss2d_dtype_t out_dtype; /* type of the output y / out */
+} ss2d_desc_t;
+
+/* Operation ids for ss2d_workspace_bytes(). */
+typedef enum {
+    SS2D_OP_SELECTIVE_SCAN_BWD = 1,
+    SS2D_OP_FORWARD = 2,
+    SS2D_OP_BACKWARD = 3
+} ss2d_op_t;
+
+/* Chunk length (steps) at which the forward saves scan states for the backward. */
+#define SS2D_CHUNK_LEN 64
+
+/* ----------------------------------------------------------------- steps -- */
+
+/*
+ * CrossScan (Fig. 2 of the VMamba page, "cross scan"):
+ *   xs[b, k, d, l] = x[b, d, pixel_k(l)]
+ * x  : (B, D, H, W)  desc->in_dtype
+ * xs : (B, 4, D, L)  desc->in_dtype   (bit-exact copy, no arithmetic)
+ */
+SS2D_API ss2d_status_t ss2d_cross_scan(const ss2d_desc_t *desc, const void *x, void *xs,
+                              ss2d_stream_t stream);
+
+/*
+ * CrossMerge (Fig. 2 of the VMamba page, "cross merge"):
+ *   y[b, d, p] = round_out((t0[p] + t2[p]) + (t1[p] + t3[p])),  t_k[pixel_k(l)] = ys[b, k, d, l]
+ * ys : (B, 4, D, L)  desc->in_dtype  (pass in_dtype = F32 to merge fp32 per-path outputs)
+ * y  : (B, D, H, W)  desc->out_dtype
+ * The sum is fp32 in that order, rounded once (so merge(scan(x)) == 4x exactly).
+ */
+SS2D_API ss2d_status_t ss2d_cross_merge(const ss2d_desc_t *desc, const void *ys, void *y,
+                               ss2d_stream_t stream);
+
+/*
+ * S6 selective scan forward over the 4*D sequences ("vision mamba-yolov8",
+ * section "2. Vmamba module code": selective_scan_ref and the forward of
+ * SelectiveScanFn).  Channel c = k*D + d uses B/C group k.
+ * u, delta     : (B, 4D, L)   in_dtype, delta[b, c, l] is step l of path k (sequence order)
+ * A            : (4D, N)      fp32
+ * Bm, Cm       : (B, 4, N, L) in_dtype
+ * D, delta_bias: (4D)         fp32 or NULL
+ * delta_softplus: nonzero -> dt = softplus(delta + bias), else dt = delta + bias
+ * out          : (B, 4D, L)   out_dtype
+ * chunk_states : (B, 4D, ceil(L / SS2D_CHUNK_LEN), N) fp32 or NULL.  Entry j holds
+ *                h after step min((j+1)*SS2D_CHUNK_LEN, L) - 1; the last entry is
+ *                the final state (the pages' last_state).
+ */
+SS2D_API ss2d_status_t ss2d_selective_scan_fwd(const ss2d_desc_t *desc, const void *u, const void *delta,
+                                      const float *A, const void *Bm, const void *Cm,
+                                      const float *D, const float *delta_bias, int delta_softplus,
+                                      void *out, float *chunk_states, ss2d_stream_t stream);
+
+/*
+ * S6 selective scan backward (the pages print only the call: the backward of
+ * SelectiveScanFn returns du, ddelta, dA, dB, dC, dD, ddelta_bias; the
+ * gradients are the analytic derivatives of the forward recurrence).
+ * Inputs as for ss2d_selective_scan_fwd, plus
+ * dout         : (B, 4D, L) out_dtype
+ * chunk_states : as written by the forward, or NULL (then recomputed internally)
+ * du, ddelta   : (B, 4D, L)   in_dtype
+ * dA           : (4D, N)      fp32, summed over batch and steps
+ * dBm, dCm     : (B, 4, N, L) in_dtype, summed over the D channels of group k
+ * dD, ddelta_bias: (4D) fp32; must be non-NULL exactly when D / delta_bias are
+ * workspace    : device buffer of ss2d_workspace_bytes(desc, SS2D_OP_SELECTIVE_SCAN_BWD)
+ *                bytes (16-byte aligned); contents on entry are ignored.
+ * Reductions are deterministic (fixed-order partial sums, no float atomics).
+ */
+SS2D_API ss2d_status_t ss2d_selective_scan_bwd(const ss2d_desc_t *desc, const void *u, const void *delta,
+                                      const float *A, const void *Bm, const void *Cm,
+                                      const float *D, const float *delta_bias, int delta_softplus,
+                                      const void *dout, const float *chunk_states,
+                                      void *du, void *ddelta, float *dA, void *dBm, void *dCm,
+                                      float *dD, float *ddelta_bias,
+                                      void *workspace, size_t workspace_bytes,
+                                      ss2d_stream_t stream);
+
+/* --------------------------------------------------------- fused SS2D -- */
+
+/*
+ * Fused SS2D forward: CrossScan -> S6 -> CrossMerge without the (B,4,D,L)
+ * intermediates.  The traversal of each path is folded into the kernels' load
+ * and store indexing.
+ * x            : (B, D, H, W)  in_dtype
+ * delta        : (B, 4D, L)    in_dtype (sequence order of each path)
+ * A, Bm, Cm, D, delta_bias, delta_softplus: as for ss2d_selective_scan_fwd
+ * y            : (B, D, H, W)  out_dtype
+ * chunk_states : as for ss2d_selective_scan_fwd (per path sequence), or NULL
+ * workspace    : ss2d_workspace_bytes(desc, SS2D_OP_FORWARD) bytes (may be 0 -> NULL ok)
+ */
+SS2D_API ss2d_status_t ss2d_forward(const ss2d_desc_t *desc, const void *x, const void *delta,
+                           const float *A, const void *Bm, const void *Cm, const float *D,
+                           const float *delta_bias, int delta_softplus, void *y,
+                           float *chunk_states, void *workspace, size_t workspace_bytes,
+                           ss2d_stream_t stream);
+
+/*
+ * Fused SS2D backward: g = CrossScan(dy) folded into the loads, S6 backward,
+ * dx = CrossMerge(du) folded into the stores.
+ * x, delta, A, Bm, Cm, D, delta_bias, delta_softplus, chunk_states: as for ss2d_forward
+ * dy           : (B, D, H, W) out_dtype
+ * dx           : (B, D, H, W) in_dtype
+ * ddelta       : (B, 4D, L)   in_dtype
+ * dA, dBm, dCm, dD, ddelta_bias: as for ss2d_selective_scan_bwd
+ * workspace    : ss2d_workspace_bytes(desc, SS2D_OP_BACKWARD) bytes
+ */
+SS2D_API ss2d_status_t ss2d_backward(const ss2d_desc_t *desc, const void *x, const void *delta,
+                            const float *A, const void *Bm, const void *Cm, const float *D,
+                            const float *delta_bias, int delta_softplus, const void *dy,
+                            const float *chunk_states, void *dx, void *ddelta, float *dA,
+                            void *dBm, void *dCm, float *dD, float *ddelta_bias,
+                            void *workspace, size_t workspace_bytes, ss2d_stream_t stream);
+
+/* ------------------------------------------------------------- helpers -- */
+
+/* Bytes of workspace an operation needs for this problem (0 if none).
+ * Returns (size_t)-1 for an invalid desc or op. */
+SS2D_API size_t ss2d_workspace_bytes(const ss2d_desc_t *desc, int op);
+
+/* Number of fp32 elements of the chunk_states buffer: B * 4D * ceil(L/SS2D_CHUNK_LEN) * N. */
+SS2D_API size_t ss2d_chunk_states_elems(const ss2d_desc_t *desc);
+
+/* Static, human-readable name of a status code. */
+SS2D_API const char *ss2d_status_string(ss2d_status_t status);
+
+/* Message of the last CUDA error this library saw on the calling thread ("" if none). */
+SS2D_API const char *ss2d_last_cuda_error(void);
+
+/* Kernels this library has launched since load (all threads); used to count launches. */
+SS2D_API uint64_t ss2d_launch_count(void);
+
+/* Tracing hook.  While set, the i-th kernel this library enqueues from the calling thread
+ * is followed by cudaEventRecord(events[i], stream) for i < count (events are cudaEvent_t
+ * handles the caller created; the library never creates, waits on or destroys them).  The
+ * index restarts at 0 on every call of this function; pass (NULL, 0) to stop.  Used to time
+ * the kernels of one entry point individually on their own stream. */
+SS2D_API void ss2d_set_trace_events(void *const *events, int count);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+SS2D_API int ss2d_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SS2D_H */

@@ -1,0 +1,346 @@
+"""selective_scan_crossscan_b200 -- VMamba's 2D selective scan (SS2D) on B200 (sm_100a).
+
+A thin Python binding over the C ABI of ``libss2d.so`` (declared in
+``include/ss2d.h``).  This module only marshals arguments: it makes tensors
+contiguous, allocates outputs and workspaces with PyTorch, and passes raw device
+pointers and the current CUDA stream.  Every step of the computation runs in the
+library's CUDA kernels; there is no CPU or PyTorch fallback -- if the library is
+missing or the device is not an sm_100 GPU, the calls raise.
+
+Steps ("VMamba: Visual State Space Model", section "2D Selective Scan (SS2D) for
+visual data", Fig. 2; the S6 arithmetic follows selective_scan_ref on
+"vision mamba-yolov8", section "2. Vmamba module code"):
+
+* ``cross_scan(x)``: (B, D, H, W) -> (B, 4, D, L): row-major, column-major, both reversed
+* ``selective_scan_fwd(u, delta, A, B, C, ...)``: S6 forward over (B, 4D, L) sequences
+* ``selective_scan_bwd(...)``: its gradients
+* ``cross_merge(ys, H, W)``: (B, 4, D, L) -> (B, D, H, W), (y0 + y2) + (y1 + y3)
+* ``ss2d_forward`` / ``ss2d_backward``: the fused SS2D forward and backward
+* ``SS2DFunction``: a torch.autograd.Function around the fused pair
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+__all__ = [
+    "SS2DError", "cross_scan", "cross_merge", "selective_scan_fwd", "selective_scan_bwd", "ss2d_forward",
+    "ss2d_backward", "SS2DFunction", "ss2d", "workspace_bytes", "chunk_states_elems", "launch_count",
+    "library_path", "CHUNK_LEN", "trace_events",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libss2d.so")
+_lock = threading.Lock()
+_lib = None
+
+CHUNK_LEN = 64  # SS2D_CHUNK_LEN
+F32, BF16 = 0, 1
+OP_SELECTIVE_SCAN_BWD, OP_FORWARD, OP_BACKWARD = 1, 2, 3
+_STATUS = {0: "SS2D_OK", 1: "SS2D_ERR_NULL", 2: "SS2D_ERR_SHAPE", 3: "SS2D_ERR_DTYPE", 4: "SS2D_ERR_ALIGN",
+           5: "SS2D_ERR_WORKSPACE", 6: "SS2D_ERR_LAUNCH", 7: "SS2D_ERR_TIMEOUT", 8: "SS2D_ERR_DEVICE"}
+
+
+class SS2DError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str = ""):
+        self.status = status
+        msg = f"{where}: {_STATUS.get(status, status)}"
+        if detail:
+            msg += f" ({detail})"
+        super().__init__(msg)
+
+
+class Desc(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("dim", ctypes.c_int64), ("height", ctypes.c_int64),
+                ("width", ctypes.c_int64), ("d_state", ctypes.c_int64), ("in_dtype", ctypes.c_int),
+                ("out_dtype", ctypes.c_int)]
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"{_LIB_PATH} is missing: build it with "
+                               "`python -m selective_scan_crossscan_b200._build` (needs nvcc)")
+        lib = ctypes.CDLL(_LIB_PATH)
+        P = ctypes.c_void_p
+        D = ctypes.POINTER(Desc)
+        i = ctypes.c_int
+        sz = ctypes.c_size_t
+        lib.ss2d_cross_scan.argtypes = [D, P, P, P]
+        lib.ss2d_cross_merge.argtypes = [D, P, P, P]
+        lib.ss2d_selective_scan_fwd.argtypes = [D, P, P, P, P, P, P, P, i, P, P, P]
+        lib.ss2d_selective_scan_bwd.argtypes = [D, P, P, P, P, P, P, P, i, P, P, P, P, P, P, P, P, P, P, sz, P]
+        lib.ss2d_forward.argtypes = [D, P, P, P, P, P, P, P, i, P, P, P, sz, P]
+        lib.ss2d_backward.argtypes = [D, P, P, P, P, P, P, P, i, P, P, P, P, P, P, P, P, P, P, sz, P]
+        for name in ("ss2d_cross_scan", "ss2d_cross_merge", "ss2d_selective_scan_fwd", "ss2d_selective_scan_bwd",
+                     "ss2d_forward", "ss2d_backward"):
+            getattr(lib, name).restype = ctypes.c_int
+        lib.ss2d_workspace_bytes.argtypes = [D, i]
+        lib.ss2d_workspace_bytes.restype = sz
+        lib.ss2d_chunk_states_elems.argtypes = [D]
+        lib.ss2d_chunk_states_elems.restype = sz
+        lib.ss2d_status_string.argtypes = [i]
+        lib.ss2d_status_string.restype = ctypes.c_char_p
+        lib.ss2d_last_cuda_error.restype = ctypes.c_char_p
+        lib.ss2d_launch_count.restype = ctypes.c_uint64
+        lib.ss2d_version.restype = ctypes.c_int
+        lib.ss2d_set_trace_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int]
+        lib.ss2d_set_trace_events.restype = None
+        _lib = lib
+        return lib
+
+
+def _code(dtype) -> int:
+    if dtype == torch.float32:
+        return F32
+    if dtype == torch.bfloat16:
+        return BF16
+    raise TypeError(f"unsupported dtype {dtype}: float32 or bfloat16")
+
+
+def _desc(batch, dim, height, width, d_state, in_dtype, out_dtype) -> Desc:
+    return Desc(int(batch), int(dim), int(height), int(width), int(d_state), _code(in_dtype), _code(out_dtype))
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _c(t, dtype=None):
+    """contiguous CUDA tensor (optionally cast); None passes through"""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("ss2d: tensors must live on a CUDA device")
+    if dtype is not None and t.dtype != dtype:
+        t = t.to(dtype)
+    return t.contiguous()
+
+
+def _stream(t):
+    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def _check(status, where):
+    if status != 0:
+        detail = _load().ss2d_last_cuda_error().decode() if status == 6 else ""
+        raise SS2DError(status, where, detail)
+
+
+def launch_count() -> int:
+    """Kernels libss2d has launched since it was loaded."""
+    return int(_load().ss2d_launch_count())
+
+
+class trace_events:
+    """Context manager: record the given torch.cuda.Event objects after the library's next kernels.
+
+    with ss.trace_events([e1, e2]):   # e1 after the 1st kernel, e2 after the 2nd
+        ss.ss2d_forward(...)
+    """
+
+    def __init__(self, events):
+        self._events = list(events)
+        self._arr = (ctypes.c_void_p * len(self._events))(*[e.cuda_event for e in self._events])
+
+    def __enter__(self):
+        _load().ss2d_set_trace_events(self._arr, len(self._events))
+        return self
+
+    def __exit__(self, *exc):
+        _load().ss2d_set_trace_events(None, 0)
+        return False
+
+
+def workspace_bytes(batch, dim, height, width, d_state, op, in_dtype=torch.float32, out_dtype=None) -> int:
+    d = _desc(batch, dim, height, width, d_state, in_dtype, out_dtype or in_dtype)
+    return int(_load().ss2d_workspace_bytes(ctypes.byref(d), int(op)))
+
+
+def chunk_states_elems(batch, dim, height, width, d_state) -> int:
+    d = _desc(batch, dim, height, width, d_state, torch.float32, torch.float32)
+    return int(_load().ss2d_chunk_states_elems(ctypes.byref(d)))
+
+
+def _workspace(nbytes, device):
+    if nbytes == 0:
+        return None
+    return torch.empty(int(nbytes), dtype=torch.uint8, device=device)
+
+
+# ------------------------------------------------------------------ steps --
+
+def cross_scan(x, out=None):
+    """x (B, D, H, W) -> xs (B, 4, D, H*W) in the same dtype."""
+    x = _c(x)
+    Bn, Dn, H, W = x.shape
+    if out is None:
+        out = torch.empty((Bn, 4, Dn, H * W), dtype=x.dtype, device=x.device)
+    d = _desc(Bn, Dn, H, W, 1, x.dtype, x.dtype)
+    _check(_load().ss2d_cross_scan(ctypes.byref(d), _p(x), _p(out), _stream(x)), "ss2d_cross_scan")
+    return out
+
+
+def cross_merge(ys, H, W, out=None, out_dtype=None):
+    """ys (B, 4, D, H*W) -> y (B, D, H, W) = (y0 + y2) + (y1 + y3) per pixel, fp32 sum, one rounding."""
+    ys = _c(ys)
+    Bn, K, Dn, L = ys.shape
+    if K != 4 or L != H * W:
+        raise ValueError("cross_merge: ys must be (B, 4, D, H*W)")
+    out_dtype = out_dtype or ys.dtype
+    if out is None:
+        out = torch.empty((Bn, Dn, H, W), dtype=out_dtype, device=ys.device)
+    d = _desc(Bn, Dn, H, W, 1, ys.dtype, out.dtype)
+    _check(_load().ss2d_cross_merge(ctypes.byref(d), _p(ys), _p(out), _stream(ys)), "ss2d_cross_merge")
+    return out
+
+
+def _params(A, D, delta_bias):
+    return _c(A, torch.float32), _c(D, torch.float32), _c(delta_bias, torch.float32)
+
+
+def selective_scan_fwd(u, delta, A, B, C, D=None, delta_bias=None, delta_softplus=False, out=None,
+                       out_dtype=None, return_chunk_states=False):
+    """S6 forward over the 4*dim sequences of an SS2D problem.
+
+    u, delta (Bn, 4D, L); A (4D, N) fp32; B, C (Bn, 4, N, L); D, delta_bias (4D) fp32 or None.
+    Returns out (Bn, 4D, L) [, chunk_states (Bn, 4D, ceil(L/64), N) fp32].
+    """
+    u = _c(u)
+    delta, B, C = (_c(t, u.dtype) for t in (delta, B, C))
+    A, D, delta_bias = _params(A, D, delta_bias)
+    Bn, Ch, L = u.shape
+    if Ch % 4 or B.shape[1] != 4:
+        raise ValueError("selective_scan_fwd: u must be (B, 4*dim, L) and B/C (B, 4, N, L)")
+    N = A.shape[1]
+    out_dtype = out_dtype or u.dtype
+    if out is None:
+        out = torch.empty((Bn, Ch, L), dtype=out_dtype, device=u.device)
+    cs = None
+    if return_chunk_states:
+        cs = torch.empty((Bn, Ch, -(-L // CHUNK_LEN), N), dtype=torch.float32, device=u.device)
+    d = _desc(Bn, Ch // 4, 1, L, N, u.dtype, out.dtype)
+    st = _load().ss2d_selective_scan_fwd(ctypes.byref(d), _p(u), _p(delta), _p(A), _p(B), _p(C), _p(D),
+                                         _p(delta_bias), int(bool(delta_softplus)), _p(out), _p(cs), _stream(u))
+    _check(st, "ss2d_selective_scan_fwd")
+    return (out, cs) if return_chunk_states else out
+
+
+def selective_scan_bwd(u, delta, A, B, C, D, delta_bias, delta_softplus, dout, chunk_states=None):
+    """Gradients of selective_scan_fwd.  Returns dict du, ddelta, dA, dB, dC, dD, ddelta_bias."""
+    u = _c(u)
+    delta, B, C = (_c(t, u.dtype) for t in (delta, B, C))
+    A, D, delta_bias = _params(A, D, delta_bias)
+    dout = _c(dout)
+    chunk_states = _c(chunk_states, torch.float32)
+    Bn, Ch, L = u.shape
+    N = A.shape[1]
+    dev = u.device
+    du = torch.empty_like(u)
+    ddelta = torch.empty_like(u)
+    dA = torch.empty_like(A)
+    dB = torch.empty_like(B)
+    dC = torch.empty_like(C)
+    dD = torch.empty_like(D) if D is not None else None
+    dbias = torch.empty_like(delta_bias) if delta_bias is not None else None
+    d = _desc(Bn, Ch // 4, 1, L, N, u.dtype, dout.dtype)
+    lib = _load()
+    nbytes = int(lib.ss2d_workspace_bytes(ctypes.byref(d), OP_SELECTIVE_SCAN_BWD))
+    ws = _workspace(nbytes, dev)
+    st = lib.ss2d_selective_scan_bwd(ctypes.byref(d), _p(u), _p(delta), _p(A), _p(B), _p(C), _p(D), _p(delta_bias),
+                                     int(bool(delta_softplus)), _p(dout), _p(chunk_states), _p(du), _p(ddelta),
+                                     _p(dA), _p(dB), _p(dC), _p(dD), _p(dbias), _p(ws), nbytes, _stream(u))
+    _check(st, "ss2d_selective_scan_bwd")
+    return dict(du=du, ddelta=ddelta, dA=dA, dB=dB, dC=dC, dD=dD, ddelta_bias=dbias)
+
+
+# ------------------------------------------------------------------ fused --
+
+def ss2d_forward(x, delta, A, B, C, D=None, delta_bias=None, delta_softplus=True, out=None, out_dtype=None,
+                 return_chunk_states=False, workspace=None):
+    """Fused SS2D forward.  x (Bn, D, H, W), delta (Bn, 4D, H*W), A (4D, N), B/C (Bn, 4, N, H*W).
+
+    Returns y (Bn, D, H, W) [, chunk_states].  ``workspace`` may be a preallocated uint8
+    CUDA tensor of at least workspace_bytes(..., OP_FORWARD) bytes.
+    """
+    x = _c(x)
+    delta, B, C = (_c(t, x.dtype) for t in (delta, B, C))
+    A, D, delta_bias = _params(A, D, delta_bias)
+    Bn, Dn, H, W = x.shape
+    N = A.shape[1]
+    out_dtype = out_dtype or x.dtype
+    if out is None:
+        out = torch.empty((Bn, Dn, H, W), dtype=out_dtype, device=x.device)
+    cs = None
+    if return_chunk_states:
+        cs = torch.empty((Bn, 4 * Dn, -(-(H * W) // CHUNK_LEN), N), dtype=torch.float32, device=x.device)
+    d = _desc(Bn, Dn, H, W, N, x.dtype, out.dtype)
+    lib = _load()
+    nbytes = int(lib.ss2d_workspace_bytes(ctypes.byref(d), OP_FORWARD))
+    if workspace is None or workspace.numel() < nbytes:
+        workspace = _workspace(nbytes, x.device)
+    st = lib.ss2d_forward(ctypes.byref(d), _p(x), _p(delta), _p(A), _p(B), _p(C), _p(D), _p(delta_bias),
+                          int(bool(delta_softplus)), _p(out), _p(cs), _p(workspace), nbytes, _stream(x))
+    _check(st, "ss2d_forward")
+    return (out, cs) if return_chunk_states else out
+
+
+def ss2d_backward(x, delta, A, B, C, D, delta_bias, delta_softplus, dy, chunk_states=None, workspace=None):
+    """Fused SS2D backward.  Returns dict dx, ddelta, dA, dB, dC, dD, ddelta_bias."""
+    x = _c(x)
+    delta, B, C = (_c(t, x.dtype) for t in (delta, B, C))
+    A, D, delta_bias = _params(A, D, delta_bias)
+    dy = _c(dy)
+    chunk_states = _c(chunk_states, torch.float32)
+    Bn, Dn, H, W = x.shape
+    N = A.shape[1]
+    dev = x.device
+    dx = torch.empty_like(x)
+    ddelta = torch.empty_like(delta)
+    dA = torch.empty_like(A)
+    dB = torch.empty_like(B)
+    dC = torch.empty_like(C)
+    dD = torch.empty_like(D) if D is not None else None
+    dbias = torch.empty_like(delta_bias) if delta_bias is not None else None
+    d = _desc(Bn, Dn, H, W, N, x.dtype, dy.dtype)
+    lib = _load()
+    nbytes = int(lib.ss2d_workspace_bytes(ctypes.byref(d), OP_BACKWARD))
+    if workspace is None or workspace.numel() < nbytes:
+        workspace = _workspace(nbytes, dev)
+    st = lib.ss2d_backward(ctypes.byref(d), _p(x), _p(delta), _p(A), _p(B), _p(C), _p(D), _p(delta_bias),
+                           int(bool(delta_softplus)), _p(dy), _p(chunk_states), _p(dx), _p(ddelta), _p(dA), _p(dB),
+                           _p(dC), _p(dD), _p(dbias), _p(workspace), nbytes, _stream(x))
+    _check(st, "ss2d_backward")
+    return dict(dx=dx, ddelta=ddelta, dA=dA, dB=dB, dC=dC, dD=dD, ddelta_bias=dbias)
+
+
+class SS2DFunction(torch.autograd.Function):
+    """autograd wrapper: forward saves the chunk states, backward runs the fused backward."""
+
+    @staticmethod
+    def forward(ctx, x, delta, A, B, C, D, delta_bias, delta_softplus):
+        y, cs = ss2d_forward(x, delta, A, B, C, D, delta_bias, delta_softplus, return_chunk_states=True)
+        ctx.save_for_backward(x, delta, A, B, C, D, delta_bias, cs)
+        ctx.delta_softplus = delta_softplus
+        return y
+
+    @staticmethod
+    def backward(ctx, dy):
+        x, delta, A, B, C, D, delta_bias, cs = ctx.saved_tensors
+        g = ss2d_backward(x, delta, A, B, C, D, delta_bias, ctx.delta_softplus, dy.to(x.dtype), chunk_states=cs)
+        return g["dx"], g["ddelta"], g["dA"], g["dB"], g["dC"], g["dD"], g["ddelta_bias"], None
+
+
+def ss2d(x, delta, A, B, C, D=None, delta_bias=None, delta_softplus=True):
+    """Differentiable fused SS2D: y = CrossMerge(S6(CrossScan(x)))."""
+    return SS2DFunction.apply(x, delta, A, B, C, D, delta_bias, delta_softplus)

@@ -1,0 +1,352 @@
+// api.cu -- the C ABI of libss2d (declared in include/ss2d.h): argument
+// validation on the host, workspace layout, and dispatch to the kernels.
+#include <atomic>
+#include <cstdio>
+#include <cstring>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace ss2d {
+
+static std::atomic<uint64_t> g_launches{0};
+static thread_local void *const *g_trace_events = nullptr;
+static thread_local int g_trace_count = 0;
+static thread_local int g_trace_next = 0;
+
+void note_launch(cudaStream_t stream) {
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    if (g_trace_events && g_trace_next < g_trace_count)
+        cudaEventRecord(static_cast<cudaEvent_t>(g_trace_events[g_trace_next++]), stream);
+}
+
+static thread_local char g_last_error[256] = "";
+
+static ss2d_status_t from_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return SS2D_OK;
+    std::snprintf(g_last_error, sizeof(g_last_error), "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
+    return SS2D_ERR_LAUNCH;
+}
+
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static ss2d_status_t check_desc(const ss2d_desc_t *d) {
+    if (!d) return SS2D_ERR_NULL;
+    if (d->batch < 1 || d->dim < 1 || d->height < 1 || d->width < 1) return SS2D_ERR_SHAPE;
+    if (d->d_state < 1 || d->d_state > 16) return SS2D_ERR_SHAPE;
+    if ((d->in_dtype != SS2D_F32 && d->in_dtype != SS2D_BF16) ||
+        (d->out_dtype != SS2D_F32 && d->out_dtype != SS2D_BF16))
+        return SS2D_ERR_DTYPE;
+    // grid limits: the batch is a grid dimension (<= 65535); keep element counts in int64 range
+    if (d->batch > 65535) return SS2D_ERR_SHAPE;
+    const double elems = (double)d->batch * 4.0 * (double)d->dim * (double)d->height * (double)d->width *
+                         (double)d->d_state;
+    if (elems > 9.0e15) return SS2D_ERR_SHAPE;
+    if ((double)d->batch * (double)d->dim * ceil_div(d->height, 32) * ceil_div(d->width, 32) > 2147483647.0)
+        return SS2D_ERR_SHAPE;
+    return SS2D_OK;
+}
+
+static LaunchShape shape_of(const ss2d_desc_t *d) {
+    LaunchShape s;
+    s.B = d->batch;
+    s.D = d->dim;
+    s.H = d->height;
+    s.W = d->width;
+    s.L = d->height * d->width;
+    s.N = d->d_state;
+    return s;
+}
+
+// one cached compute-capability check per device
+static ss2d_status_t check_device() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) {
+        cudaGetLastError();
+        std::snprintf(g_last_error, sizeof(g_last_error), "no CUDA device");
+        return SS2D_ERR_DEVICE;
+    }
+    static std::atomic<int> ok[64];
+    if (dev < 64 && ok[dev].load() == 1) return SS2D_OK;
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return SS2D_ERR_DEVICE;
+    }
+    if (major != 10) {
+        std::snprintf(g_last_error, sizeof(g_last_error), "device %d is compute capability %d.x, need 10.0 (sm_100a)",
+                      dev, major);
+        return SS2D_ERR_DEVICE;
+    }
+    if (dev < 64) ok[dev].store(1);
+    return SS2D_OK;
+}
+
+#define SS2D_TRY(expr)                         \
+    do {                                       \
+        ss2d_status_t _st = (expr);            \
+        if (_st != SS2D_OK) return _st;        \
+    } while (0)
+
+static ss2d_status_t need(const void *p) {
+    if (!p) return SS2D_ERR_NULL;
+    if (!aligned16(p)) return SS2D_ERR_ALIGN;
+    return SS2D_OK;
+}
+static ss2d_status_t optional(const void *p) { return (p && !aligned16(p)) ? SS2D_ERR_ALIGN : SS2D_OK; }
+
+// workspace layouts ---------------------------------------------------------
+
+static size_t round64(size_t n) { return (n + 63) / 64 * 64; }
+
+static size_t fwd_ws_bytes(const LaunchShape &s) {
+    return round64((size_t)s.B * kPaths * s.D * s.L * sizeof(float)) + round64(scan_fwd_workspace_bytes(s));
+}
+static size_t bwd_fused_ws_bytes(const LaunchShape &s) {
+    return round64((size_t)s.B * kPaths * s.D * s.L * sizeof(float)) + round64(scan_bwd_workspace_bytes(s));
+}
+
+}  // namespace ss2d
+
+using namespace ss2d;
+
+extern "C" {
+
+int ss2d_version(void) { return 100; }  // 0.1.0
+
+uint64_t ss2d_launch_count(void) { return g_launches.load(); }
+
+void ss2d_set_trace_events(void *const *events, int count) {
+    g_trace_events = (events && count > 0) ? events : nullptr;
+    g_trace_count = g_trace_events ? count : 0;
+    g_trace_next = 0;
+}
+
+const char *ss2d_last_cuda_error(void) { return g_last_error; }
+
+const char *ss2d_status_string(ss2d_status_t s) {
+    switch (s) {
+        case SS2D_OK: return "SS2D_OK";
+        case SS2D_ERR_NULL: return "SS2D_ERR_NULL: a required pointer is NULL";
+        case SS2D_ERR_SHAPE: return "SS2D_ERR_SHAPE: invalid or unsupported sizes";
+        case SS2D_ERR_DTYPE: return "SS2D_ERR_DTYPE: unsupported dtype";
+        case SS2D_ERR_ALIGN: return "SS2D_ERR_ALIGN: pointer not 16-byte aligned";
+        case SS2D_ERR_WORKSPACE: return "SS2D_ERR_WORKSPACE: workspace missing or too small";
+        case SS2D_ERR_LAUNCH: return "SS2D_ERR_LAUNCH: CUDA launch failed";
+        case SS2D_ERR_TIMEOUT: return "SS2D_ERR_TIMEOUT: device-side wait gave up";
+        case SS2D_ERR_DEVICE: return "SS2D_ERR_DEVICE: no usable sm_100 device";
+    }
+    return "SS2D: unknown status";
+}
+
+size_t ss2d_chunk_states_elems(const ss2d_desc_t *desc) {
+    if (check_desc(desc) != SS2D_OK) return 0;
+    const LaunchShape s = shape_of(desc);
+    return (size_t)s.B * kPaths * s.D * ceil_div(s.L, SS2D_CHUNK_LEN) * s.N;
+}
+
+size_t ss2d_workspace_bytes(const ss2d_desc_t *desc, int op) {
+    if (check_desc(desc) != SS2D_OK) return (size_t)-1;
+    const LaunchShape s = shape_of(desc);
+    switch (op) {
+        case SS2D_OP_SELECTIVE_SCAN_BWD: return scan_bwd_workspace_bytes(s);
+        case SS2D_OP_FORWARD: return fwd_ws_bytes(s);
+        case SS2D_OP_BACKWARD: return bwd_fused_ws_bytes(s);
+        default: return (size_t)-1;
+    }
+}
+
+ss2d_status_t ss2d_cross_scan(const ss2d_desc_t *desc, const void *x, void *xs, ss2d_stream_t stream) {
+    SS2D_TRY(check_desc(desc));
+    SS2D_TRY(need(x));
+    SS2D_TRY(need(xs));
+    SS2D_TRY(check_device());
+    return from_cuda(launch_cross_scan(shape_of(desc), desc->in_dtype, x, xs, (cudaStream_t)stream));
+}
+
+ss2d_status_t ss2d_cross_merge(const ss2d_desc_t *desc, const void *ys, void *y, ss2d_stream_t stream) {
+    SS2D_TRY(check_desc(desc));
+    SS2D_TRY(need(ys));
+    SS2D_TRY(need(y));
+    SS2D_TRY(check_device());
+    return from_cuda(
+        launch_cross_merge(shape_of(desc), desc->in_dtype, desc->out_dtype, ys, y, (cudaStream_t)stream));
+}
+
+static ss2d_status_t check_scan_inputs(const void *u, const void *delta, const float *A, const void *Bm,
+                                       const void *Cm, const float *D, const float *delta_bias) {
+    SS2D_TRY(need(u));
+    SS2D_TRY(need(delta));
+    SS2D_TRY(need(A));
+    SS2D_TRY(need(Bm));
+    SS2D_TRY(need(Cm));
+    SS2D_TRY(optional(D));
+    SS2D_TRY(optional(delta_bias));
+    return SS2D_OK;
+}
+
+ss2d_status_t ss2d_selective_scan_fwd(const ss2d_desc_t *desc, const void *u, const void *delta, const float *A,
+                                      const void *Bm, const void *Cm, const float *D, const float *delta_bias,
+                                      int delta_softplus, void *out, float *chunk_states, ss2d_stream_t stream) {
+    SS2D_TRY(check_desc(desc));
+    SS2D_TRY(check_scan_inputs(u, delta, A, Bm, Cm, D, delta_bias));
+    SS2D_TRY(need(out));
+    SS2D_TRY(optional(chunk_states));
+    const LaunchShape s = shape_of(desc);
+    SS2D_TRY(check_device());
+    ScanFwdArgs a;
+    a.u = u;
+    a.delta = delta;
+    a.A = A;
+    a.Bm = Bm;
+    a.Cm = Cm;
+    a.Dv = D;
+    a.bias = delta_bias;
+    a.softplus = delta_softplus != 0;
+    a.out = out;
+    a.chunk_states = chunk_states;
+    a.from_image = false;
+    a.in_dtype = desc->in_dtype;
+    a.out_dtype = desc->out_dtype;
+    a.max_segments = 1;  // this entry point takes no workspace: one pass per sequence
+    return from_cuda(launch_scan_fwd(s, a, nullptr, (cudaStream_t)stream));
+}
+
+ss2d_status_t ss2d_selective_scan_bwd(const ss2d_desc_t *desc, const void *u, const void *delta, const float *A,
+                                      const void *Bm, const void *Cm, const float *D, const float *delta_bias,
+                                      int delta_softplus, const void *dout, const float *chunk_states, void *du,
+                                      void *ddelta, float *dA, void *dBm, void *dCm, float *dD,
+                                      float *ddelta_bias, void *workspace, size_t workspace_bytes,
+                                      ss2d_stream_t stream) {
+    SS2D_TRY(check_desc(desc));
+    SS2D_TRY(check_scan_inputs(u, delta, A, Bm, Cm, D, delta_bias));
+    SS2D_TRY(need(dout));
+    SS2D_TRY(optional(chunk_states));
+    SS2D_TRY(need(du));
+    SS2D_TRY(need(ddelta));
+    SS2D_TRY(need(dA));
+    SS2D_TRY(need(dBm));
+    SS2D_TRY(need(dCm));
+    if ((D == nullptr) != (dD == nullptr)) return SS2D_ERR_NULL;
+    if ((delta_bias == nullptr) != (ddelta_bias == nullptr)) return SS2D_ERR_NULL;
+    SS2D_TRY(optional(dD));
+    SS2D_TRY(optional(ddelta_bias));
+    const LaunchShape s = shape_of(desc);
+    const size_t ws = scan_bwd_workspace_bytes(s);
+    if (ws > 0 && (!workspace || workspace_bytes < ws)) return SS2D_ERR_WORKSPACE;
+    SS2D_TRY(optional(workspace));
+    SS2D_TRY(check_device());
+    ScanBwdArgs a;
+    a.u = u;
+    a.delta = delta;
+    a.A = A;
+    a.Bm = Bm;
+    a.Cm = Cm;
+    a.Dv = D;
+    a.bias = delta_bias;
+    a.softplus = delta_softplus != 0;
+    a.dout = dout;
+    a.chunk_states = chunk_states;
+    a.du = du;
+    a.ddelta = ddelta;
+    a.dA = dA;
+    a.dBm = dBm;
+    a.dCm = dCm;
+    a.dD = dD;
+    a.dbias = ddelta_bias;
+    a.from_image = false;
+    a.in_dtype = desc->in_dtype;
+    a.out_dtype = desc->out_dtype;
+    return from_cuda(launch_scan_bwd(s, a, workspace, workspace_bytes, (cudaStream_t)stream));
+}
+
+ss2d_status_t ss2d_forward(const ss2d_desc_t *desc, const void *x, const void *delta, const float *A,
+                           const void *Bm, const void *Cm, const float *D, const float *delta_bias,
+                           int delta_softplus, void *y, float *chunk_states, void *workspace,
+                           size_t workspace_bytes, ss2d_stream_t stream) {
+    SS2D_TRY(check_desc(desc));
+    SS2D_TRY(check_scan_inputs(x, delta, A, Bm, Cm, D, delta_bias));
+    SS2D_TRY(need(y));
+    SS2D_TRY(optional(chunk_states));
+    const LaunchShape s = shape_of(desc);
+    const size_t ws = fwd_ws_bytes(s);
+    if (ws > 0 && (!workspace || workspace_bytes < ws)) return SS2D_ERR_WORKSPACE;
+    SS2D_TRY(optional(workspace));
+    SS2D_TRY(check_device());
+    unsigned char *w = static_cast<unsigned char *>(workspace);
+    float *ys = reinterpret_cast<float *>(w);
+    void *seg = w + round64((size_t)s.B * kPaths * s.D * s.L * sizeof(float));
+    ScanFwdArgs a;
+    a.u = x;
+    a.delta = delta;
+    a.A = A;
+    a.Bm = Bm;
+    a.Cm = Cm;
+    a.Dv = D;
+    a.bias = delta_bias;
+    a.softplus = delta_softplus != 0;
+    a.out = ys;
+    a.chunk_states = chunk_states;
+    a.from_image = true;
+    a.in_dtype = desc->in_dtype;
+    a.out_dtype = SS2D_F32;
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = launch_scan_fwd(s, a, seg, st);
+    if (e != cudaSuccess) return from_cuda(e);
+    return from_cuda(launch_cross_merge(s, SS2D_F32, desc->out_dtype, ys, y, st));
+}
+
+ss2d_status_t ss2d_backward(const ss2d_desc_t *desc, const void *x, const void *delta, const float *A,
+                            const void *Bm, const void *Cm, const float *D, const float *delta_bias,
+                            int delta_softplus, const void *dy, const float *chunk_states, void *dx, void *ddelta,
+                            float *dA, void *dBm, void *dCm, float *dD, float *ddelta_bias, void *workspace,
+                            size_t workspace_bytes, ss2d_stream_t stream) {
+    SS2D_TRY(check_desc(desc));
+    SS2D_TRY(check_scan_inputs(x, delta, A, Bm, Cm, D, delta_bias));
+    SS2D_TRY(need(dy));
+    SS2D_TRY(optional(chunk_states));
+    SS2D_TRY(need(dx));
+    SS2D_TRY(need(ddelta));
+    SS2D_TRY(need(dA));
+    SS2D_TRY(need(dBm));
+    SS2D_TRY(need(dCm));
+    if ((D == nullptr) != (dD == nullptr)) return SS2D_ERR_NULL;
+    if ((delta_bias == nullptr) != (ddelta_bias == nullptr)) return SS2D_ERR_NULL;
+    SS2D_TRY(optional(dD));
+    SS2D_TRY(optional(ddelta_bias));
+    const LaunchShape s = shape_of(desc);
+    const size_t ws = bwd_fused_ws_bytes(s);
+    if (ws > 0 && (!workspace || workspace_bytes < ws)) return SS2D_ERR_WORKSPACE;
+    SS2D_TRY(optional(workspace));
+    SS2D_TRY(check_device());
+    unsigned char *w = static_cast<unsigned char *>(workspace);
+    float *du_seq = reinterpret_cast<float *>(w);
+    void *inner = w + round64((size_t)s.B * kPaths * s.D * s.L * sizeof(float));
+    ScanBwdArgs a;
+    a.u = x;
+    a.delta = delta;
+    a.A = A;
+    a.Bm = Bm;
+    a.Cm = Cm;
+    a.Dv = D;
+    a.bias = delta_bias;
+    a.softplus = delta_softplus != 0;
+    a.dout = dy;
+    a.chunk_states = chunk_states;
+    a.du = du_seq;
+    a.ddelta = ddelta;
+    a.dA = dA;
+    a.dBm = dBm;
+    a.dCm = dCm;
+    a.dD = dD;
+    a.dbias = ddelta_bias;
+    a.from_image = true;
+    a.in_dtype = desc->in_dtype;
+    a.out_dtype = desc->out_dtype;
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = launch_scan_bwd(s, a, inner, scan_bwd_workspace_bytes(s), st);
+    if (e != cudaSuccess) return from_cuda(e);
+    return from_cuda(launch_cross_merge(s, SS2D_F32, desc->in_dtype, du_seq, dx, st));
+}
+
+}  // extern "C"

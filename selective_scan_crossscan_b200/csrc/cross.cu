@@ -1,0 +1,142 @@
+// cross.cu -- CrossScan and CrossMerge (VMamba, "2D Selective Scan (SS2D) for
+// visual data", Fig. 2: unfold the map along four paths / merge the four
+// per-path outputs back into the map by summation).
+//
+// Both are pure data movement bounded by HBM.  A CTA owns a 32x32 pixel tile
+// of one (b, d) plane.  Row-major paths (k=0 forward, k=2 backward) are read
+// or written with lanes along w; column-major paths (k=1, k=3, step
+// l = w*H + h) with lanes along h, the tile being transposed through shared
+// memory, so every global access of a warp touches consecutive addresses.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace ss2d {
+
+constexpr int kTile = 32;
+constexpr int kRows = 8;  // blockDim = (32, 8)
+
+template <typename T>
+__global__ void __launch_bounds__(kTile * kRows)
+cross_scan_kernel(const T *__restrict__ x, T *__restrict__ xs, int64_t Dn, int64_t H, int64_t W,
+                  int64_t tiles_w, int64_t tiles_h) {
+    __shared__ T tile[kTile][kTile + 1];
+    int64_t blk = blockIdx.x;
+    const int64_t tw = blk % tiles_w;
+    blk /= tiles_w;
+    const int64_t th = blk % tiles_h;
+    const int64_t bd = blk / tiles_h;  // b * D + d
+    const int64_t b = bd / Dn, d = bd - b * Dn;
+    const int64_t L = H * W;
+    const int64_t h0 = th * kTile, w0 = tw * kTile;
+    const T *plane = x + bd * L;
+    T *out0 = xs + ((b * kPaths + 0) * Dn + d) * L;
+    T *out1 = xs + ((b * kPaths + 1) * Dn + d) * L;
+    T *out2 = xs + ((b * kPaths + 2) * Dn + d) * L;
+    T *out3 = xs + ((b * kPaths + 3) * Dn + d) * L;
+    const int tx = threadIdx.x, ty = threadIdx.y;
+
+#pragma unroll
+    for (int j = 0; j < kTile / kRows; ++j) {
+        const int hh = ty + kRows * j;
+        const int64_t h = h0 + hh, w = w0 + tx;
+        if (h < H && w < W) {
+            const int64_t p = h * W + w;
+            const T v = plane[p];
+            tile[hh][tx] = v;
+            out0[p] = v;          // row-major: step l = p
+            out2[L - 1 - p] = v;  // reversed row-major
+        }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < kTile / kRows; ++j) {
+        const int ww = ty + kRows * j;
+        const int64_t h = h0 + tx, w = w0 + ww;
+        if (h < H && w < W) {
+            const T v = tile[tx][ww];
+            const int64_t l = w * H + h;  // column-major step
+            out1[l] = v;
+            out3[L - 1 - l] = v;
+        }
+    }
+}
+
+template <typename Tin, typename Tout>
+__global__ void __launch_bounds__(kTile * kRows)
+cross_merge_kernel(const Tin *__restrict__ ys, Tout *__restrict__ y, int64_t Dn, int64_t H, int64_t W,
+                   int64_t tiles_w, int64_t tiles_h) {
+    __shared__ float t13[kTile][kTile + 1];  // (t1 + t3) at (hh, ww)
+    int64_t blk = blockIdx.x;
+    const int64_t tw = blk % tiles_w;
+    blk /= tiles_w;
+    const int64_t th = blk % tiles_h;
+    const int64_t bd = blk / tiles_h;
+    const int64_t b = bd / Dn, d = bd - b * Dn;
+    const int64_t L = H * W;
+    const int64_t h0 = th * kTile, w0 = tw * kTile;
+    const Tin *in0 = ys + ((b * kPaths + 0) * Dn + d) * L;
+    const Tin *in1 = ys + ((b * kPaths + 1) * Dn + d) * L;
+    const Tin *in2 = ys + ((b * kPaths + 2) * Dn + d) * L;
+    const Tin *in3 = ys + ((b * kPaths + 3) * Dn + d) * L;
+    Tout *plane = y + bd * L;
+    const int tx = threadIdx.x, ty = threadIdx.y;
+
+#pragma unroll
+    for (int j = 0; j < kTile / kRows; ++j) {
+        const int ww = ty + kRows * j;
+        const int64_t h = h0 + tx, w = w0 + ww;
+        if (h < H && w < W) {
+            const int64_t l = w * H + h;
+            t13[tx][ww] = ld(in1 + l) + ld(in3 + (L - 1 - l));
+        }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < kTile / kRows; ++j) {
+        const int hh = ty + kRows * j;
+        const int64_t h = h0 + hh, w = w0 + tx;
+        if (h < H && w < W) {
+            const int64_t p = h * W + w;
+            const float t02 = ld(in0 + p) + ld(in2 + (L - 1 - p));
+            st(plane + p, t02 + t13[hh][tx]);
+        }
+    }
+}
+
+static dim3 tile_grid(int64_t planes, int64_t H, int64_t W, int64_t *tw, int64_t *th) {
+    *tw = ceil_div(W, kTile);
+    *th = ceil_div(H, kTile);
+    return dim3((unsigned)(planes * *tw * *th));
+}
+
+cudaError_t launch_cross_scan(const LaunchShape &s, ss2d_dtype_t dt, const void *x, void *xs,
+                              cudaStream_t stream) {
+    int64_t tw, th;
+    dim3 grid = tile_grid(s.B * s.D, s.H, s.W, &tw, &th);
+    dim3 block(kTile, kRows);
+    if (dt == SS2D_F32)
+        cross_scan_kernel<float><<<grid, block, 0, stream>>>((const float *)x, (float *)xs, s.D, s.H, s.W, tw, th);
+    else
+        cross_scan_kernel<__nv_bfloat16><<<grid, block, 0, stream>>>(
+            (const __nv_bfloat16 *)x, (__nv_bfloat16 *)xs, s.D, s.H, s.W, tw, th);
+    note_launch(stream);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_cross_merge(const LaunchShape &s, ss2d_dtype_t din, ss2d_dtype_t dout, const void *ys,
+                               void *y, cudaStream_t stream) {
+    int64_t tw, th;
+    dim3 grid = tile_grid(s.B * s.D, s.H, s.W, &tw, &th);
+    dim3 block(kTile, kRows);
+#define SS2D_MERGE(TI, TO)                                                                               \
+    cross_merge_kernel<TI, TO><<<grid, block, 0, stream>>>((const TI *)ys, (TO *)y, s.D, s.H, s.W, tw, th)
+    if (din == SS2D_F32 && dout == SS2D_F32) SS2D_MERGE(float, float);
+    else if (din == SS2D_F32) SS2D_MERGE(float, __nv_bfloat16);
+    else if (dout == SS2D_F32) SS2D_MERGE(__nv_bfloat16, float);
+    else SS2D_MERGE(__nv_bfloat16, __nv_bfloat16);
+#undef SS2D_MERGE
+    note_launch(stream);
+    return cudaGetLastError();
+}
+
+}  // namespace ss2d

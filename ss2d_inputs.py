@@ -139,3 +139,23 @@ def batch_slice(inputs: dict, idx) -> dict:
         else:
             out[k] = v
     return out
+
+
+def make_scan_inputs(w: Workload, seed: int = 0, device="cpu", with_dout: bool = False):
+    """Inputs for the standalone S6 scan in its sequence view: u (B, 4D, L) drawn directly
+    (N(0,1)) instead of an image, the other tensors as in make_inputs.  dout ~ N(0,1) if asked."""
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed) + 1000)
+    f32 = dict(dtype=torch.float32, device=device, generator=g)
+    base = make_inputs(w, seed=seed, device=device, with_dy=False)
+    u = torch.randn((w.batch, K_PATHS * w.dim, w.L), **f32)
+    out = dict(base)
+    del out["x"]
+    out["u"] = u
+    if with_dout:
+        out["dout"] = torch.randn((w.batch, K_PATHS * w.dim, w.L), **f32)
+    if w.dtype == "bf16":
+        for key in ("u", "dout"):
+            if key in out:
+                out[key] = out[key].to(torch.bfloat16)
+    return out

@@ -1,0 +1,374 @@
+"""GPU parity: the CUDA library (called through its C ABI via the binding) against the fp64 oracle.
+
+Bars (element by element on the same seeded inputs):
+  * CrossScan / CrossMerge index maps: bit-exact;
+  * fp32 forward: |y - y_ref| <= 1e-4 * (1 + |y_ref|);
+  * fp32 gradients: relative L2 error <= 1e-4;
+  * bf16 inputs: relative L2 error <= 1e-2 against the oracle fed the same bf16-rounded values.
+Full-size workloads are compared on sampled batch items (batch items are independent, so
+the oracle on a batch slice is exact for those items).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import selective_scan_crossscan_b200 as ss
+import ss2d_inputs
+
+pytestmark = pytest.mark.gpu
+
+FWD_TOL = 1e-4
+GRAD_TOL = 1e-4
+BF16_TOL = 1e-2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    assert torch.cuda.is_available(), "the gpu tests need a CUDA device"
+    from selective_scan_crossscan_b200 import _build
+    _build.build()
+    oracle.build()
+    torch.cuda.set_device(0)
+
+
+def _np(t):
+    return t.detach().to("cpu").double().numpy()
+
+
+def _dev(inp):
+    return {k: v.cuda() for k, v in inp.items()}
+
+
+def assert_fwd_close(y, ref, what=""):
+    y = _np(y) if torch.is_tensor(y) else y
+    err = np.abs(y - ref)
+    bound = FWD_TOL * (1.0 + np.abs(ref))
+    worst = np.max(err - bound)
+    assert worst <= 0, f"{what}: max excess {worst:.3e}, max err {err.max():.3e}"
+
+
+def rel_l2(a, ref):
+    a = _np(a) if torch.is_tensor(a) else a
+    return float(np.linalg.norm((a - ref).ravel()) / max(np.linalg.norm(ref.ravel()), 1e-300))
+
+
+def assert_rel_l2(a, ref, tol, what=""):
+    r = rel_l2(a, ref)
+    assert r <= tol, f"{what}: rel L2 {r:.3e} > {tol}"
+
+
+# ------------------------------------------------------------ cross scan/merge
+
+SHAPES = [(1, 8, 8, 8), (2, 3, 5, 7), (2, 4, 33, 65), (1, 2, 1, 1), (3, 5, 14, 14), (1, 3, 1, 37), (1, 2, 40, 3)]
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("shape", SHAPES)
+def test_cross_scan_bit_exact(shape, dtype):
+    g = torch.Generator().manual_seed(1)
+    x = torch.randn(shape, generator=g).to(dtype)
+    xs = ss.cross_scan(x.cuda())
+    ref = oracle.cross_scan(x)
+    assert xs.dtype == dtype
+    np.testing.assert_array_equal(_np(xs), ref)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("shape", SHAPES)
+def test_merge_of_scan_is_exactly_four_x(shape, dtype):
+    g = torch.Generator().manual_seed(2)
+    x = torch.randn(shape, generator=g).to(dtype).cuda()
+    y = ss.cross_merge(ss.cross_scan(x), shape[2], shape[3])
+    assert torch.equal(y, 4 * x)
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+def test_cross_merge_index_map_bit_exact(shape):
+    # integer-valued tags keep every fp32 sum exact, so any misplaced element shows
+    Bn, Dn, H, W = shape
+    g = torch.Generator().manual_seed(3)
+    ys = torch.randint(-1000, 1000, (Bn, 4, Dn, H * W), generator=g).float()
+    y = ss.cross_merge(ys.cuda(), H, W)
+    np.testing.assert_array_equal(_np(y), oracle.cross_merge(ys, H, W))
+
+
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_cross_merge_random_values(out_dtype):
+    Bn, Dn, H, W = 2, 3, 9, 11
+    g = torch.Generator().manual_seed(4)
+    ys = torch.randn((Bn, 4, Dn, H * W), generator=g)
+    y = ss.cross_merge(ys.cuda(), H, W, out_dtype=out_dtype)
+    ref = oracle.cross_merge(ys, H, W)
+    tol = 1e-6 if out_dtype == torch.float32 else 8e-3
+    np.testing.assert_allclose(_np(y), ref, rtol=tol, atol=tol)
+
+
+# --------------------------------------------------------------- S6 forward
+
+def _scan_case(Bn, Dn, H, W, N, dtype="f32", seed=0):
+    w = ss2d_inputs.custom(Bn, Dn, H, W, N, dtype=dtype)
+    return w, ss2d_inputs.make_scan_inputs(w, seed=seed, with_dout=True)
+
+
+SCAN_CASES = [(1, 8, 8, 8, 4), (2, 70, 5, 7, 16), (1, 3, 1, 1, 3), (2, 16, 3, 45, 8), (1, 64, 9, 15, 1),
+              (1, 5, 16, 20, 16), (3, 2, 2, 2, 5)]
+
+
+@pytest.mark.parametrize("case", SCAN_CASES)
+def test_selective_scan_fwd_parity(case):
+    w, inp = _scan_case(*case)
+    d = _dev(inp)
+    y = ss.selective_scan_fwd(d["u"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["delta_bias"], True)
+    ref = oracle.selective_scan_fwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"],
+                                    inp["delta_bias"], True)
+    assert_fwd_close(y, ref, str(case))
+
+
+@pytest.mark.parametrize("opts", [dict(D=False, bias=True, sp=True), dict(D=True, bias=False, sp=True),
+                                  dict(D=False, bias=False, sp=False)])
+def test_selective_scan_fwd_optional_inputs(opts):
+    w, inp = _scan_case(2, 8, 6, 6, 8, seed=5)
+    if not opts["sp"]:
+        inp["delta"] = inp["delta"].abs() * 0.5 + 0.01  # positive step sizes without softplus
+    D = inp["D"] * 0.5 if opts["D"] else None
+    bias = inp["delta_bias"] if opts["bias"] else None
+    d = _dev(inp)
+    y = ss.selective_scan_fwd(d["u"], d["delta"], d["A"], d["B"], d["C"], None if D is None else D.cuda(),
+                              None if bias is None else bias.cuda(), opts["sp"])
+    ref = oracle.selective_scan_fwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], D, bias, opts["sp"])
+    assert_fwd_close(y, ref, str(opts))
+
+
+def test_selective_scan_fwd_chunk_states():
+    # chunk j holds h after step min(64 (j+1), L) - 1: the oracle's last state on the truncated sequence
+    w, inp = _scan_case(1, 4, 10, 20, 16, seed=6)  # L = 200 -> 4 chunks, ragged last one
+    d = _dev(inp)
+    y, cs = ss.selective_scan_fwd(d["u"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["delta_bias"], True,
+                                  return_chunk_states=True)
+    assert cs.shape == (1, 16, 4, 16)
+    for j, end in enumerate([64, 128, 192, 200]):
+        _, last = oracle.selective_scan_fwd(inp["u"][..., :end], inp["delta"][..., :end], inp["A"],
+                                            inp["B"][..., :end], inp["C"][..., :end], inp["D"], inp["delta_bias"],
+                                            True, return_last_state=True)
+        assert_rel_l2(cs[:, :, j], last, 1e-5, f"chunk {j}")
+
+
+def test_selective_scan_fwd_bf16():
+    w, inp = _scan_case(2, 16, 7, 7, 16, dtype="bf16", seed=7)
+    d = _dev(inp)
+    y = ss.selective_scan_fwd(d["u"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["delta_bias"], True)
+    assert y.dtype == torch.bfloat16
+    ref = oracle.selective_scan_fwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"],
+                                    inp["delta_bias"], True)
+    assert_rel_l2(y, ref, BF16_TOL)
+
+
+# -------------------------------------------------------------- S6 backward
+
+BWD_NAMES = [("du", "du"), ("ddelta", "ddelta"), ("dA", "dA"), ("dB", "dB"), ("dC", "dC"), ("dD", "dD"),
+             ("ddelta_bias", "ddelta_bias")]
+
+
+@pytest.mark.parametrize("case", [(1, 8, 8, 8, 4), (2, 40, 5, 7, 16), (1, 3, 1, 1, 3), (1, 33, 4, 50, 8),
+                                  (2, 4, 3, 43, 16)])
+@pytest.mark.parametrize("with_states", [False, True])
+def test_selective_scan_bwd_parity(case, with_states):
+    w, inp = _scan_case(*case, seed=8)
+    d = _dev(inp)
+    cs = None
+    if with_states:
+        _, cs = ss.selective_scan_fwd(d["u"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["delta_bias"], True,
+                                      return_chunk_states=True)
+    g = ss.selective_scan_bwd(d["u"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["delta_bias"], True, d["dout"],
+                              chunk_states=cs)
+    ref = oracle.selective_scan_bwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"],
+                                    inp["delta_bias"], True, inp["dout"])
+    for name, rname in BWD_NAMES:
+        assert_rel_l2(g[name], ref[rname], GRAD_TOL, f"{case} {name}")
+
+
+def test_selective_scan_bwd_without_optional():
+    w, inp = _scan_case(1, 8, 6, 11, 8, seed=9)
+    d = _dev(inp)
+    g = ss.selective_scan_bwd(d["u"], d["delta"], d["A"], d["B"], d["C"], None, None, True, d["dout"])
+    assert g["dD"] is None and g["ddelta_bias"] is None
+    ref = oracle.selective_scan_bwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], None, None, True,
+                                    inp["dout"])
+    for name in ("du", "ddelta", "dA", "dB", "dC"):
+        assert_rel_l2(g[name], ref[name], GRAD_TOL, name)
+
+
+# ------------------------------------------------------------- fused SS2D
+
+FUSED_CASES = [(1, 8, 8, 8, 4), (2, 6, 5, 9, 16), (1, 70, 12, 11, 16), (1, 8, 64, 64, 16), (2, 3, 1, 1, 2),
+               (1, 4, 3, 100, 8)]
+
+
+@pytest.mark.parametrize("case", FUSED_CASES)
+def test_ss2d_forward_parity(case):
+    Bn, Dn, H, W, N = case
+    w = ss2d_inputs.custom(Bn, Dn, H, W, N)
+    inp = ss2d_inputs.make_inputs(w, seed=10)
+    d = _dev(inp)
+    y = ss.ss2d_forward(d["x"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["delta_bias"], True)
+    ref = oracle.ss2d_forward(inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"], inp["delta_bias"],
+                              True)
+    assert_fwd_close(y, ref, str(case))
+
+
+def test_ss2d_forward_tiny_workload():
+    w = ss2d_inputs.workload(0)
+    inp = ss2d_inputs.make_inputs(w, seed=0)
+    d = _dev(inp)
+    y, cs = ss.ss2d_forward(d["x"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["delta_bias"], True,
+                            return_chunk_states=True)
+    ref = oracle.ss2d_forward(inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"], inp["delta_bias"],
+                              True)
+    assert_fwd_close(y, ref, "tiny")
+    # the last chunk state is the final state of each of the 4*D path sequences
+    xs = oracle.cross_scan(inp["x"]).reshape(1, 32, 64)
+    _, last = oracle.selective_scan_fwd(xs, inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"], inp["delta_bias"],
+                                        True, return_last_state=True)
+    assert_rel_l2(cs[:, :, -1], last, 1e-5, "last state")
+
+
+def test_ss2d_forward_bf16():
+    w = ss2d_inputs.custom(2, 16, 14, 14, 16, dtype="bf16", a_init="s4d_real")
+    inp = ss2d_inputs.make_inputs(w, seed=11)
+    d = _dev(inp)
+    y = ss.ss2d_forward(d["x"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["delta_bias"], True)
+    assert y.dtype == torch.bfloat16
+    ref = oracle.ss2d_forward(inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"], inp["delta_bias"],
+                              True)
+    assert_rel_l2(y, ref, BF16_TOL)
+
+
+def test_unfused_pipeline_equals_fused():
+    w = ss2d_inputs.custom(2, 8, 7, 9, 16)
+    d = _dev(ss2d_inputs.make_inputs(w, seed=12))
+    y = ss.ss2d_forward(d["x"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["delta_bias"], True)
+    xs = ss.cross_scan(d["x"]).reshape(2, 32, 63)
+    ys = ss.selective_scan_fwd(xs, d["delta"], d["A"], d["B"], d["C"], d["D"], d["delta_bias"], True)
+    y2 = ss.cross_merge(ys.reshape(2, 4, 8, 63), 7, 9)
+    assert torch.equal(y, y2)
+
+
+def test_forward_is_deterministic():
+    w = ss2d_inputs.custom(2, 20, 16, 16, 16)
+    d = _dev(ss2d_inputs.make_inputs(w, seed=13))
+    y1 = ss.ss2d_forward(d["x"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["delta_bias"], True)
+    y2 = ss.ss2d_forward(d["x"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["delta_bias"], True)
+    assert torch.equal(y1, y2)
+
+
+SS2D_BWD_NAMES = [("dx", "dx"), ("ddelta", "ddelta"), ("dA", "dA"), ("dB", "dB"), ("dC", "dC"), ("dD", "dD"),
+                  ("ddelta_bias", "ddelta_bias")]
+
+
+@pytest.mark.parametrize("case", [(1, 8, 8, 8, 4), (2, 6, 5, 9, 16), (1, 40, 9, 10, 16), (1, 3, 1, 1, 2),
+                                  (1, 4, 10, 20, 8)])
+@pytest.mark.parametrize("with_states", [False, True])
+def test_ss2d_backward_parity(case, with_states):
+    Bn, Dn, H, W, N = case
+    w = ss2d_inputs.custom(Bn, Dn, H, W, N)
+    inp = ss2d_inputs.make_inputs(w, seed=14, with_dy=True)
+    d = _dev(inp)
+    cs = None
+    if with_states:
+        _, cs = ss.ss2d_forward(d["x"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["delta_bias"], True,
+                                return_chunk_states=True)
+    g = ss.ss2d_backward(d["x"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["delta_bias"], True, d["dy"],
+                         chunk_states=cs)
+    ref = oracle.ss2d_backward(inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"], inp["delta_bias"],
+                               True, inp["dy"])
+    for name, rname in SS2D_BWD_NAMES:
+        assert_rel_l2(g[name], ref[rname], GRAD_TOL, f"{case} {name}")
+
+
+def test_ss2d_backward_bf16():
+    w = ss2d_inputs.custom(1, 8, 12, 12, 16, dtype="bf16", a_init="s4d_real")
+    inp = ss2d_inputs.make_inputs(w, seed=15, with_dy=True)
+    d = _dev(inp)
+    g = ss.ss2d_backward(d["x"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["delta_bias"], True, d["dy"])
+    ref = oracle.ss2d_backward(inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"], inp["delta_bias"],
+                               True, inp["dy"])
+    for name, rname in SS2D_BWD_NAMES:
+        assert_rel_l2(g[name], ref[rname], BF16_TOL, name)
+
+
+def test_autograd_function_matches_backward():
+    w = ss2d_inputs.custom(1, 4, 6, 7, 8)
+    inp = ss2d_inputs.make_inputs(w, seed=16, with_dy=True)
+    d = _dev(inp)
+    leaves = {k: d[k].clone().requires_grad_(True) for k in ("x", "delta", "A", "B", "C", "D", "delta_bias")}
+    y = ss.ss2d(leaves["x"], leaves["delta"], leaves["A"], leaves["B"], leaves["C"], leaves["D"],
+                leaves["delta_bias"], True)
+    y.backward(d["dy"])
+    ref = oracle.ss2d_backward(inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"], inp["delta_bias"],
+                               True, inp["dy"])
+    for k, rname in (("x", "dx"), ("delta", "ddelta"), ("A", "dA"), ("B", "dB"), ("C", "dC"), ("D", "dD"),
+                     ("delta_bias", "ddelta_bias")):
+        assert_rel_l2(leaves[k].grad, ref[rname], GRAD_TOL, k)
+
+
+def test_launch_counter_counts_fused_forward():
+    w = ss2d_inputs.custom(1, 8, 8, 8, 4)
+    d = _dev(ss2d_inputs.make_inputs(w, seed=17))
+    before = ss.launch_count()
+    ss.ss2d_forward(d["x"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["delta_bias"], True)
+    torch.cuda.synchronize()
+    assert ss.launch_count() - before >= 2
+
+
+# ---------------------------------------------------- full-size workloads
+
+def _full_forward_check(index, items):
+    w = ss2d_inputs.workload(index)
+    inp = ss2d_inputs.make_inputs(w, seed=index, device="cuda", with_dy=False)
+    y = ss.ss2d_forward(inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"], inp["delta_bias"], True)
+    torch.cuda.synchronize()
+    sl = ss2d_inputs.batch_slice(inp, items)
+    ref = oracle.ss2d_forward(sl["x"], sl["delta"], sl["A"], sl["B"], sl["C"], sl["D"], sl["delta_bias"], True)
+    got = y[items]
+    if w.dtype == "f32":
+        assert_fwd_close(got, ref, w.name)
+    else:
+        assert_rel_l2(got, ref, BF16_TOL, w.name)
+
+
+def test_full_size_vmamba_t_stage1_fp32():
+    _full_forward_check(1, [0, 64, 127])
+
+
+def test_full_size_vmamba_stage3_bf16():
+    _full_forward_check(2, [0, 64, 127])
+
+
+def test_full_size_highres_bf16():
+    _full_forward_check(3, [0, 4, 7])
+
+
+def test_full_size_fwd_bwd_fp32():
+    w = ss2d_inputs.workload(4)
+    inp = ss2d_inputs.make_inputs(w, seed=4, device="cuda", with_dy=True)
+    y, cs = ss.ss2d_forward(inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"], inp["delta_bias"], True,
+                            return_chunk_states=True)
+    g = ss.ss2d_backward(inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"], inp["delta_bias"], True,
+                         inp["dy"], chunk_states=cs)
+    torch.cuda.synchronize()
+    items = [0, 16, 31]
+    sl = ss2d_inputs.batch_slice(inp, items)
+    ref_y = oracle.ss2d_forward(sl["x"], sl["delta"], sl["A"], sl["B"], sl["C"], sl["D"], sl["delta_bias"], True)
+    assert_fwd_close(y[items], ref_y, "c4 fwd")
+    ref = oracle.ss2d_backward(sl["x"], sl["delta"], sl["A"], sl["B"], sl["C"], sl["D"], sl["delta_bias"], True,
+                               sl["dy"])
+    # per-item gradients compare directly; dA, dD, ddelta_bias sum over the whole batch, so they are
+    # checked on the full batch through the identity with per-item sums below
+    for name in ("dx", "ddelta", "dB", "dC"):
+        assert_rel_l2(g[name][items], ref[name], GRAD_TOL, f"c4 {name}")
+    # batch-summed parameter gradients: oracle over the whole batch would cost minutes; instead
+    # check them on the three items with a separate GPU call restricted to those items
+    g3 = ss.ss2d_backward(sl["x"], sl["delta"], sl["A"], sl["B"], sl["C"], sl["D"], sl["delta_bias"], True, sl["dy"])
+    for name in ("dA", "dD", "ddelta_bias"):
+        assert_rel_l2(g3[name], ref[name], GRAD_TOL, f"c4 items {name}")
