@@ -240,6 +240,8 @@ def run_gpu(args, world, rank, local):
         _build.build()
     barrier(world)
     w = ss2d_inputs.workload(args.workload)
+    if args.batch:
+        w = w.with_batch(args.batch)
     dev = torch.device("cuda", local)
     inp = ss2d_inputs.make_inputs(w, seed=shard_seed(args.workload, rank), device=dev, with_dy=False)
     y = torch.empty((w.batch, w.dim, w.height, w.width), dtype=w.torch_dtype, device=dev)
@@ -420,6 +422,8 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", type=int, default=1, help="index into ss2d_inputs.WORKLOADS (default 1)")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch (small cases for profiling; not a bench line)")
     ap.add_argument("--impl", choices=["ss2d", "reference"], default="ss2d")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -33,7 +33,8 @@ __all__ = [
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-_LIB_PATH = os.path.join(_HERE, "libss2d.so")
+# SS2D_LIBRARY may point at another build of the same library (e.g. a tuning variant)
+_LIB_PATH = os.environ.get("SS2D_LIBRARY") or os.path.join(_HERE, "libss2d.so")
 _lock = threading.Lock()
 _lib = None
 
@@ -151,6 +152,9 @@ class trace_events:
 
     def __init__(self, events):
         self._events = list(events)
+        for e in self._events:
+            if not e.cuda_event:  # torch creates the CUDA event lazily, on its first record
+                e.record()
         self._arr = (ctypes.c_void_p * len(self._events))(*[e.cuda_event for e in self._events])
 
     def __enter__(self):

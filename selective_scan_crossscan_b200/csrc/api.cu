@@ -99,11 +99,17 @@ static ss2d_status_t optional(const void *p) { return (p && !aligned16(p)) ? SS2
 
 static size_t round64(size_t n) { return (n + 63) / 64 * 64; }
 
-static size_t fwd_ws_bytes(const LaunchShape &s) {
-    return round64((size_t)s.B * kPaths * s.D * s.L * sizeof(float)) + round64(scan_fwd_workspace_bytes(s));
+static size_t elem_size(ss2d_dtype_t t) { return t == SS2D_F32 ? 4 : 2; }
+
+// fused forward workspace: [fp32 per-path outputs (B,4D,L)] [transposed image (B,D,W,H)] [segment summaries]
+static size_t fwd_ws_bytes(const LaunchShape &s, ss2d_dtype_t in) {
+    return round64((size_t)s.B * kPaths * s.D * s.L * sizeof(float)) +
+           round64((size_t)s.B * s.D * s.L * elem_size(in)) + round64(scan_fwd_workspace_bytes(s));
 }
-static size_t bwd_fused_ws_bytes(const LaunchShape &s) {
-    return round64((size_t)s.B * kPaths * s.D * s.L * sizeof(float)) + round64(scan_bwd_workspace_bytes(s));
+// fused backward workspace: [fp32 per-path du (B,4D,L)] [transposed image] [scan backward workspace]
+static size_t bwd_fused_ws_bytes(const LaunchShape &s, ss2d_dtype_t in) {
+    return round64((size_t)s.B * kPaths * s.D * s.L * sizeof(float)) +
+           round64((size_t)s.B * s.D * s.L * elem_size(in)) + round64(scan_bwd_workspace_bytes(s));
 }
 
 }  // namespace ss2d
@@ -150,8 +156,8 @@ size_t ss2d_workspace_bytes(const ss2d_desc_t *desc, int op) {
     const LaunchShape s = shape_of(desc);
     switch (op) {
         case SS2D_OP_SELECTIVE_SCAN_BWD: return scan_bwd_workspace_bytes(s);
-        case SS2D_OP_FORWARD: return fwd_ws_bytes(s);
-        case SS2D_OP_BACKWARD: return bwd_fused_ws_bytes(s);
+        case SS2D_OP_FORWARD: return fwd_ws_bytes(s, desc->in_dtype);
+        case SS2D_OP_BACKWARD: return bwd_fused_ws_bytes(s, desc->in_dtype);
         default: return (size_t)-1;
     }
 }
@@ -269,15 +275,22 @@ ss2d_status_t ss2d_forward(const ss2d_desc_t *desc, const void *x, const void *d
     SS2D_TRY(need(y));
     SS2D_TRY(optional(chunk_states));
     const LaunchShape s = shape_of(desc);
-    const size_t ws = fwd_ws_bytes(s);
+    const size_t ws = fwd_ws_bytes(s, desc->in_dtype);
     if (ws > 0 && (!workspace || workspace_bytes < ws)) return SS2D_ERR_WORKSPACE;
     SS2D_TRY(optional(workspace));
     SS2D_TRY(check_device());
     unsigned char *w = static_cast<unsigned char *>(workspace);
     float *ys = reinterpret_cast<float *>(w);
-    void *seg = w + round64((size_t)s.B * kPaths * s.D * s.L * sizeof(float));
+    w += round64((size_t)s.B * kPaths * s.D * s.L * sizeof(float));
+    void *xT = w;
+    w += round64((size_t)s.B * s.D * s.L * elem_size(desc->in_dtype));
+    void *seg = w;
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = launch_transpose(s, desc->in_dtype, x, xT, st);
+    if (e != cudaSuccess) return from_cuda(e);
     ScanFwdArgs a;
     a.u = x;
+    a.uT = xT;
     a.delta = delta;
     a.A = A;
     a.Bm = Bm;
@@ -290,8 +303,7 @@ ss2d_status_t ss2d_forward(const ss2d_desc_t *desc, const void *x, const void *d
     a.from_image = true;
     a.in_dtype = desc->in_dtype;
     a.out_dtype = SS2D_F32;
-    cudaStream_t st = (cudaStream_t)stream;
-    cudaError_t e = launch_scan_fwd(s, a, seg, st);
+    e = launch_scan_fwd(s, a, seg, st);
     if (e != cudaSuccess) return from_cuda(e);
     return from_cuda(launch_cross_merge(s, SS2D_F32, desc->out_dtype, ys, y, st));
 }
@@ -315,15 +327,26 @@ ss2d_status_t ss2d_backward(const ss2d_desc_t *desc, const void *x, const void *
     SS2D_TRY(optional(dD));
     SS2D_TRY(optional(ddelta_bias));
     const LaunchShape s = shape_of(desc);
-    const size_t ws = bwd_fused_ws_bytes(s);
+    const size_t ws = bwd_fused_ws_bytes(s, desc->in_dtype);
     if (ws > 0 && (!workspace || workspace_bytes < ws)) return SS2D_ERR_WORKSPACE;
     SS2D_TRY(optional(workspace));
     SS2D_TRY(check_device());
     unsigned char *w = static_cast<unsigned char *>(workspace);
     float *du_seq = reinterpret_cast<float *>(w);
-    void *inner = w + round64((size_t)s.B * kPaths * s.D * s.L * sizeof(float));
+    w += round64((size_t)s.B * kPaths * s.D * s.L * sizeof(float));
+    void *xT = w;
+    w += round64((size_t)s.B * s.D * s.L * elem_size(desc->in_dtype));
+    void *inner = w;
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e;
+    if (!chunk_states) {
+        // the chunk states are recomputed by a forward pass that reads the column paths from xT
+        e = launch_transpose(s, desc->in_dtype, x, xT, st);
+        if (e != cudaSuccess) return from_cuda(e);
+    }
     ScanBwdArgs a;
     a.u = x;
+    a.uT = xT;
     a.delta = delta;
     a.A = A;
     a.Bm = Bm;
@@ -343,8 +366,7 @@ ss2d_status_t ss2d_backward(const ss2d_desc_t *desc, const void *x, const void *
     a.from_image = true;
     a.in_dtype = desc->in_dtype;
     a.out_dtype = desc->out_dtype;
-    cudaStream_t st = (cudaStream_t)stream;
-    cudaError_t e = launch_scan_bwd(s, a, inner, scan_bwd_workspace_bytes(s), st);
+    e = launch_scan_bwd(s, a, inner, scan_bwd_workspace_bytes(s), st);
     if (e != cudaSuccess) return from_cuda(e);
     return from_cuda(launch_cross_merge(s, SS2D_F32, desc->in_dtype, du_seq, dx, st));
 }

@@ -33,6 +33,35 @@ __device__ __forceinline__ float ld(const T *p) { return Elem<T>::load(p); }
 template <typename T>
 __device__ __forceinline__ void st(T *p, float v) { Elem<T>::store(p, v); }
 
+// ---------------------------------------------- 4-element vector I/O --
+// (16-byte accesses for fp32, 8-byte for bf16; the address must be aligned to them)
+
+__device__ __forceinline__ void ld4(const float *p, float v[4]) {
+    const float4 q = *reinterpret_cast<const float4 *>(p);
+    v[0] = q.x;
+    v[1] = q.y;
+    v[2] = q.z;
+    v[3] = q.w;
+}
+__device__ __forceinline__ void ld4(const __nv_bfloat16 *p, float v[4]) {
+    const uint2 q = *reinterpret_cast<const uint2 *>(p);
+    v[0] = __uint_as_float(q.x << 16);
+    v[1] = __uint_as_float(q.x & 0xffff0000u);
+    v[2] = __uint_as_float(q.y << 16);
+    v[3] = __uint_as_float(q.y & 0xffff0000u);
+}
+__device__ __forceinline__ void st4(float *p, const float v[4]) {
+    *reinterpret_cast<float4 *>(p) = make_float4(v[0], v[1], v[2], v[3]);
+}
+__device__ __forceinline__ void st4(__nv_bfloat16 *p, const float v[4]) {
+    const __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]);
+    const __nv_bfloat162 b = __floats2bfloat162_rn(v[2], v[3]);
+    uint2 q;
+    q.x = *reinterpret_cast<const uint32_t *>(&a);
+    q.y = *reinterpret_cast<const uint32_t *>(&b);
+    *reinterpret_cast<uint2 *>(p) = q;
+}
+
 // ------------------------------------------------------------- path maps --
 
 // Pixel index h*W + w visited at step l of path k.  k=0 row-major, k=1

@@ -123,13 +123,115 @@ cudaError_t launch_cross_scan(const LaunchShape &s, ss2d_dtype_t dt, const void 
     return cudaGetLastError();
 }
 
+// x (B, D, H, W) -> xT (B, D, W, H): the column-major paths of the fused
+// forward then read their sequence contiguously (row k=1 of xT is path 1).
+template <typename T>
+__global__ void __launch_bounds__(kTile * kRows)
+transpose_kernel(const T *__restrict__ x, T *__restrict__ xT, int64_t H, int64_t W, int64_t tiles_w,
+                 int64_t tiles_h) {
+    __shared__ T tile[kTile][kTile + 1];
+    int64_t blk = blockIdx.x;
+    const int64_t tw = blk % tiles_w;
+    blk /= tiles_w;
+    const int64_t th = blk % tiles_h;
+    const int64_t bd = blk / tiles_h;
+    const int64_t L = H * W;
+    const int64_t h0 = th * kTile, w0 = tw * kTile;
+    const T *plane = x + bd * L;
+    T *tplane = xT + bd * L;
+    const int tx = threadIdx.x, ty = threadIdx.y;
+#pragma unroll
+    for (int j = 0; j < kTile / kRows; ++j) {
+        const int hh = ty + kRows * j;
+        const int64_t h = h0 + hh, w = w0 + tx;
+        if (h < H && w < W) tile[hh][tx] = plane[h * W + w];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < kTile / kRows; ++j) {
+        const int ww = ty + kRows * j;
+        const int64_t h = h0 + tx, w = w0 + ww;
+        if (h < H && w < W) tplane[w * H + h] = tile[tx][ww];
+    }
+}
+
+// CrossMerge with 4-element vector accesses, for H % 4 == 0 and W % 4 == 0 (then
+// every 4-pixel run of a row or a column, and its mirror in a reversed path, is
+// aligned).  256 threads per 32x32 tile; each thread handles 4 pixels.
+template <typename Tin, typename Tout>
+__global__ void __launch_bounds__(256)
+cross_merge_vec_kernel(const Tin *__restrict__ ys, Tout *__restrict__ y, int64_t Dn, int64_t H, int64_t W,
+                       int64_t tiles_w, int64_t tiles_h) {
+    __shared__ float t13[kTile][kTile + 1];  // (t1 + t3) at [w - w0][h - h0]
+    int64_t blk = blockIdx.x;
+    const int64_t tw = blk % tiles_w;
+    blk /= tiles_w;
+    const int64_t th = blk % tiles_h;
+    const int64_t bd = blk / tiles_h;
+    const int64_t b = bd / Dn, d = bd - b * Dn;
+    const int64_t L = H * W;
+    const int64_t h0 = th * kTile, w0 = tw * kTile;
+    const Tin *in0 = ys + ((b * kPaths + 0) * Dn + d) * L;
+    const Tin *in1 = ys + ((b * kPaths + 1) * Dn + d) * L;
+    const Tin *in2 = ys + ((b * kPaths + 2) * Dn + d) * L;
+    const Tin *in3 = ys + ((b * kPaths + 3) * Dn + d) * L;
+    const int t = threadIdx.x;
+    {
+        const int col = t >> 3, hq = t & 7;
+        const int64_t w = w0 + col, h = h0 + 4 * hq;
+        if (w < W && h < H) {
+            const int64_t l = w * H + h;  // steps l..l+3 of the column path
+            float v1[4], v3[4];
+            ld4(in1 + l, v1);
+            ld4(in3 + (L - 4 - l), v3);  // reversed: step l+e sits at L-1-l-e
+#pragma unroll
+            for (int e = 0; e < 4; ++e) t13[col][4 * hq + e] = v1[e] + v3[3 - e];
+        }
+    }
+    __syncthreads();
+    {
+        const int row = t >> 3, wq = t & 7;
+        const int64_t h = h0 + row, w = w0 + 4 * wq;
+        if (h < H && w < W) {
+            const int64_t p = h * W + w;
+            float v0[4], v2[4], out[4];
+            ld4(in0 + p, v0);
+            ld4(in2 + (L - 4 - p), v2);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) out[e] = (v0[e] + v2[3 - e]) + t13[4 * wq + e][row];
+            st4(y + bd * L + p, out);
+        }
+    }
+}
+
+cudaError_t launch_transpose(const LaunchShape &s, ss2d_dtype_t dt, const void *x, void *xT, cudaStream_t stream) {
+    int64_t tw, th;
+    dim3 grid = tile_grid(s.B * s.D, s.H, s.W, &tw, &th);
+    dim3 block(kTile, kRows);
+    if (dt == SS2D_F32)
+        transpose_kernel<float><<<grid, block, 0, stream>>>((const float *)x, (float *)xT, s.H, s.W, tw, th);
+    else
+        transpose_kernel<__nv_bfloat16><<<grid, block, 0, stream>>>((const __nv_bfloat16 *)x,
+                                                                    (__nv_bfloat16 *)xT, s.H, s.W, tw, th);
+    note_launch(stream);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_cross_merge(const LaunchShape &s, ss2d_dtype_t din, ss2d_dtype_t dout, const void *ys,
                                void *y, cudaStream_t stream) {
     int64_t tw, th;
     dim3 grid = tile_grid(s.B * s.D, s.H, s.W, &tw, &th);
     dim3 block(kTile, kRows);
-#define SS2D_MERGE(TI, TO)                                                                               \
-    cross_merge_kernel<TI, TO><<<grid, block, 0, stream>>>((const TI *)ys, (TO *)y, s.D, s.H, s.W, tw, th)
+    const bool vec = (s.H % 4) == 0 && (s.W % 4) == 0;
+#define SS2D_MERGE(TI, TO)                                                                                      \
+    do {                                                                                                        \
+        if (vec)                                                                                                \
+            cross_merge_vec_kernel<TI, TO><<<grid, 256, 0, stream>>>((const TI *)ys, (TO *)y, s.D, s.H, s.W, tw, \
+                                                                      th);                                      \
+        else                                                                                                    \
+            cross_merge_kernel<TI, TO><<<grid, block, 0, stream>>>((const TI *)ys, (TO *)y, s.D, s.H, s.W, tw,  \
+                                                                    th);                                        \
+    } while (0)
     if (din == SS2D_F32 && dout == SS2D_F32) SS2D_MERGE(float, float);
     else if (din == SS2D_F32) SS2D_MERGE(float, __nv_bfloat16);
     else if (dout == SS2D_F32) SS2D_MERGE(__nv_bfloat16, float);

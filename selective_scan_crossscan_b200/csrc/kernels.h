@@ -18,6 +18,8 @@ void note_launch(cudaStream_t stream);
 
 cudaError_t launch_cross_scan(const LaunchShape &s, ss2d_dtype_t dt, const void *x, void *xs,
                               cudaStream_t stream);
+// x (B, D, H, W) -> xT (B, D, W, H), bit-exact
+cudaError_t launch_transpose(const LaunchShape &s, ss2d_dtype_t dt, const void *x, void *xT, cudaStream_t stream);
 cudaError_t launch_cross_merge(const LaunchShape &s, ss2d_dtype_t din, ss2d_dtype_t dout, const void *ys,
                                void *y, cudaStream_t stream);
 
@@ -25,6 +27,7 @@ cudaError_t launch_cross_merge(const LaunchShape &s, ss2d_dtype_t din, ss2d_dtyp
 
 struct ScanFwdArgs {
     const void *u;       // (B, 4D, L) sequences, or (B, D, H, W) image when from_image
+    const void *uT = nullptr;  // (B, D, W, H) transposed image, read by the column paths when from_image
     const void *delta;   // (B, 4D, L)
     const float *A;      // (4D, N)
     const void *Bm;      // (B, 4, N, L)
@@ -49,6 +52,7 @@ cudaError_t launch_scan_fwd(const LaunchShape &s, const ScanFwdArgs &a, void *wo
 
 struct ScanBwdArgs {
     const void *u;       // (B, 4D, L) sequences, or (B, D, H, W) image when from_image
+    const void *uT = nullptr;  // transposed image (recomputing chunk states from the image needs it)
     const void *delta;
     const float *A;
     const void *Bm;

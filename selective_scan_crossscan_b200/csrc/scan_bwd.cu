@@ -216,7 +216,8 @@ __global__ void __launch_bounds__(kBT) scan_bwd_kernel(const BwdParams p) {
                             const float dtu = dt * sm.us[t][i];
 #pragma unroll
                             for (int n = 0; n < NS; ++n) {
-                                h[n] = fmaf(ex2_sfu(dt * A2[n]), h[n], dtu * sm.Bs[i][n]);
+                                // the same rounded dt*u*B as the adjoint subtracts below
+                                h[n] = fmaf(ex2_sfu(dt * A2[n]), h[n], __fmul_rn(dtu, sm.Bs[i][n]));
                                 hist[j][n] = h[n];
                             }
                         }
@@ -241,7 +242,8 @@ __global__ void __launch_bounds__(kBT) scan_bwd_kernel(const BwdParams p) {
                             const float Cn = sm.Cs[i][n];
                             const float a = ex2_sfu(dt * A2[n]);
                             lam[n] = fmaf(Cn, g, lam[n]);
-                            const float ah = hist[j][n] - dtu * Bn;  // a_l * h_{l-1}
+                            // a_l * h_{l-1}, exactly 0 when h_{l-1} = 0
+                            const float ah = __fsub_rn(hist[j][n], __fmul_rn(dtu, Bn));
                             ddt = fmaf(lam[n], fmaf(A2[n] * An_scale, ah, Bn * uv), ddt);
                             dA[n] = fmaf(lam[n] * dt, ah, dA[n]);
                             dul = fmaf(lam[n] * dt, Bn, dul);
@@ -404,6 +406,7 @@ cudaError_t launch_scan_bwd(const LaunchShape &s, const ScanBwdArgs &a, void *wo
         // recompute the forward's chunk states (no outputs written)
         ScanFwdArgs f;
         f.u = a.u;
+        f.uT = a.uT;
         f.delta = a.delta;
         f.A = a.A;
         f.Bm = a.Bm;

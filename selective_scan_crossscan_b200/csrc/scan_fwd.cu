@@ -10,29 +10,43 @@
 // slots, not by HBM.  Each thread owns one whole (b, c) sequence with all N
 // states in registers and walks it in order: per state update that is one
 // FMUL (dt * A*log2e), one MUFU.EX2, one FMUL (dt*u * B) and two FFMAs -- no
-// cross-thread scan arithmetic at all.  A CTA holds 64 channels of one (b, k),
-// so B[., l] and C[., l] are the same for all its threads: they are staged in
-// shared memory as [step][state] and read as broadcast 16-byte loads.  u and
-// delta are staged per 32-step chunk with coalesced loads.
+// cross-thread scan arithmetic at all.
+//
+//  * A CTA is one warp: 32 channels of one (b, k).  The headline problem
+//    (98,304 sequences) then fits the GPU in a single wave (~21 warps per SM),
+//    so no SM idles while a second, nearly empty wave runs.
+//  * u and delta are read by each thread along its own sequence, four steps at
+//    a time (16-byte loads for fp32, 8-byte for bf16), one group ahead of use.
+//  * B[., l] and C[., l] are the same for all 32 threads (group k of batch b):
+//    they are staged in shared memory in 32-step chunks with cp.async, double
+//    buffered, and read as broadcast vector loads.
+//  * The fused SS2D forward reads u from the image along path k: row-major
+//    paths from x (k=2 backwards), column-major paths from a transposed copy
+//    of x (k=3 backwards), so every load stays sequential.
 //
 // When a problem has too few sequences to fill the GPU, each sequence is cut
 // into segments: a summary pass computes, per segment, the state reached
 // from zero and the decay product exp(A * sum dt); the output pass starts
 // each segment from the carry combined over the segments before it.
-//
-// The fused SS2D forward reads u straight from the (B, D, H, W) image along
-// path k (CrossScan folded into the loads).
 #include "common.cuh"
 #include "kernels.h"
 
 namespace ss2d {
 
-constexpr int kTD = 64;  // channels (= threads) per CTA
-constexpr int kLC = 32;  // steps staged per chunk
+constexpr int kWarp = 32;   // threads (= channels) per CTA
+constexpr int kLC = 32;     // steps of B/C per staged chunk
+constexpr int kG = 4;       // steps per register group
 constexpr int kStateChunk = SS2D_CHUNK_LEN;
 
+// Resident CTAs (warps) per SM the forward kernel is compiled for; 21 puts the
+// headline problem's 3,072 warps in one wave on 148 SMs, fewer leaves more registers.
+#ifndef SS2D_FWD_MIN_BLOCKS
+#define SS2D_FWD_MIN_BLOCKS 20
+#endif
+
 struct FwdParams {
-    const void *u;
+    const void *u;       // (B, 4D, L) sequences, or image x (B, D, H, W)
+    const void *uT;      // transposed image (B, D, W, H) for the column paths (image mode)
     const void *delta;
     const float *A;
     const void *Bm;
@@ -50,33 +64,96 @@ struct FwdParams {
     int64_t nchunks;
 };
 
+// Four steps l0..l0+3 of a sequence stored forwards (rev = false) or backwards
+// (step l at index L-1-l).  VEC: one aligned vector load; else scalar loads
+// with bounds (steps at or past lend read as 0).
+template <bool VEC, typename T>
+__device__ __forceinline__ void load_group(const T *row, bool rev, int64_t L, int64_t l0, int64_t lend, float v[4]) {
+    if (VEC) {
+        if (!rev) {
+            ld4(row + l0, v);
+        } else {
+            float w[4];
+            ld4(row + (L - 4 - l0), w);
+            v[0] = w[3];
+            v[1] = w[2];
+            v[2] = w[1];
+            v[3] = w[0];
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < kG; ++j) {
+            const int64_t l = l0 + j;
+            v[j] = (l < lend) ? ld(row + (rev ? (L - 1 - l) : l)) : 0.f;
+        }
+    }
+}
+
+template <typename T>
+__device__ __forceinline__ void cp_async_bytes(T *smem_dst, const T *gsrc, int bytes) {
+    const unsigned dst = (unsigned)__cvta_generic_to_shared(smem_dst);
+    if (bytes == 16)
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(gsrc));
+    else if (bytes == 8)
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(dst), "l"(gsrc));
+    else
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(dst), "l"(gsrc));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
+
+// Stage B/C steps [l0, l0+len) of group (b, k) into smem buffers [NS][kLC].
+// VEC: 4-element cp.async copies (len is a multiple of 4); else plain loads.
+template <int NS, bool VEC, typename Tin>
+__device__ __forceinline__ void stage_bc(Tin (*Bs)[kLC], Tin (*Cs)[kLC], const Tin *Bk, const Tin *Ck, int N,
+                                         int64_t L, int64_t l0, int len) {
+    const int t = threadIdx.x;
+    if (VEC) {
+        const int q = kLC / 4;
+        for (int idx = t; idx < NS * q; idx += kWarp) {
+            const int n = idx / q, i4 = (idx % q) * 4;
+            if (n < N && i4 < len) {
+                cp_async_bytes(&Bs[n][i4], Bk + (int64_t)n * L + l0 + i4, 4 * (int)sizeof(Tin));
+                cp_async_bytes(&Cs[n][i4], Ck + (int64_t)n * L + l0 + i4, 4 * (int)sizeof(Tin));
+            }
+        }
+    } else {
+        for (int idx = t; idx < NS * kLC; idx += kWarp) {
+            const int n = idx / kLC, i = idx % kLC;
+            const bool ok = n < N && i < len;
+            Bs[n][i] = ok ? Bk[(int64_t)n * L + l0 + i] : Tin(0.f);
+            Cs[n][i] = ok ? Ck[(int64_t)n * L + l0 + i] : Tin(0.f);
+        }
+    }
+}
+
 // PASS 0: single pass.  PASS 1: segment summaries only.  PASS 2: outputs with carries.
-template <int NS, typename Tin, typename Tout, bool IMG, int PASS>
-__global__ void __launch_bounds__(kTD) scan_fwd_kernel(const FwdParams p) {
-    __shared__ float us[kTD][kLC + 1];
-    __shared__ float ds[kTD][kLC + 1];
-    __shared__ __align__(16) float Bs[kLC][NS];
-    __shared__ __align__(16) float Cs[kLC][NS];
+template <int NS, typename Tin, typename Tout, bool IMG, int PASS, bool VEC>
+__global__ void __launch_bounds__(kWarp, SS2D_FWD_MIN_BLOCKS) scan_fwd_kernel(const FwdParams p) {
+    __shared__ __align__(16) Tin Bs[2][NS][kLC];
+    __shared__ __align__(16) Tin Cs[2][NS][kLC];
+    __shared__ float A2s[NS][kWarp];  // A[c, n] * log2(e) of each lane's channel (kept out of registers)
 
     const int t = threadIdx.x;
     const int k = blockIdx.y;
     const int64_t b = blockIdx.z / p.nseg;
     const int s = blockIdx.z % p.nseg;
     const int64_t D = p.D, L = p.L, C4 = kPaths * p.D;
-    const int64_t d0 = (int64_t)blockIdx.x * kTD;
-    const int nch = (int)min((int64_t)kTD, D - d0);
-    const bool active = t < nch;
-    const int64_t c = k * D + d0 + t;
+    const int64_t d = (int64_t)blockIdx.x * kWarp + t;
+    const bool active = d < D;
+    const int64_t c = k * D + (active ? d : 0);
     const int N = p.N;
     const int64_t lbeg = (int64_t)s * p.seglen;
     const int64_t lend = min(L, lbeg + p.seglen);
 
-    float A2[NS], h[NS];
+    float h[NS];
 #pragma unroll
     for (int n = 0; n < NS; ++n) {
-        A2[n] = (active && n < N) ? p.A[c * N + n] * kLog2e : 0.f;
+        A2s[n][t] = (active && n < N) ? p.A[c * N + n] * kLog2e : 0.f;
         h[n] = 0.f;
     }
+    __syncwarp();
     const float Dc = (active && p.Dv) ? p.Dv[c] : 0.f;
     const float bias = (active && p.bias) ? p.bias[c] : 0.f;
 
@@ -91,84 +168,131 @@ __global__ void __launch_bounds__(kTD) scan_fwd_kernel(const FwdParams p) {
     }
     float dtsum = 0.f;
 
-    const Tin *delta = static_cast<const Tin *>(p.delta);
-    const Tin *u = static_cast<const Tin *>(p.u);
+    // this thread's u and delta sequences
+    const Tin *urow;
+    bool urev;
+    if (IMG) {
+        const Tin *img = static_cast<const Tin *>((k & 1) ? p.uT : p.u);
+        urow = img + (b * D + (active ? d : 0)) * L;
+        urev = k >= 2;
+    } else {
+        urow = static_cast<const Tin *>(p.u) + (b * C4 + c) * L;
+        urev = false;
+    }
+    const Tin *drow = static_cast<const Tin *>(p.delta) + (b * C4 + c) * L;
     const Tin *Bk = static_cast<const Tin *>(p.Bm) + (b * kPaths + k) * N * L;
     const Tin *Ck = static_cast<const Tin *>(p.Cm) + (b * kPaths + k) * N * L;
-    Tout *out = static_cast<Tout *>(p.out);
+    Tout *orow = p.out ? static_cast<Tout *>(p.out) + (b * C4 + c) * L : nullptr;
 
-    for (int64_t l0 = lbeg; l0 < lend; l0 += kLC) {
-        const int len = (int)min((int64_t)kLC, lend - l0);
-        __syncthreads();  // previous chunk fully consumed
-        for (int idx = t; idx < kTD * kLC; idx += kTD) {
-            const int ch = idx / kLC, i = idx % kLC;
-            float uv = 0.f, dv = 0.f;
-            if (ch < nch && i < len) {
-                const int64_t l = l0 + i;
-                const int64_t cc = k * D + d0 + ch;
-                dv = ld(delta + (b * C4 + cc) * L + l);
-                if (IMG)
-                    uv = ld(u + (b * D + d0 + ch) * L + path_pixel(k, l, p.H, p.W));
-                else
-                    uv = ld(u + (b * C4 + cc) * L + l);
-            }
-            us[ch][i] = uv;
-            ds[ch][i] = dv;
-        }
-        for (int idx = t; idx < NS * kLC; idx += kTD) {
-            const int n = idx / kLC, i = idx % kLC;
-            float bv = 0.f, cv = 0.f;
-            if (n < N && i < len) {
-                bv = ld(Bk + n * L + l0 + i);
-                cv = ld(Ck + n * L + l0 + i);
-            }
-            Bs[i][n] = bv;
-            Cs[i][n] = cv;
-        }
-        __syncthreads();
+    const int64_t nloc = lend - lbeg;
+    const int nchunk = (int)ceil_div(nloc, kLC);
 
-        if (active) {
-            for (int i = 0; i < len; ++i) {
-                const float uv = us[t][i];
-                const float tt = ds[t][i] + bias;
-                const float dt = p.softplus ? softplus_f(tt) : tt;
-                const float dtu = dt * uv;
-                float y = 0.f;
+    // rows n >= N of the B/C buffers are never copied: zero them once so padded
+    // states stay at h = 0 and contribute nothing
+    if (VEC && N < NS) {
+        Tin *bz = &Bs[0][0][0], *cz = &Cs[0][0][0];
+        for (int i = t; i < 2 * NS * kLC; i += kWarp) {
+            bz[i] = Tin(0.f);
+            cz[i] = Tin(0.f);
+        }
+        __syncwarp();
+    }
+
+    float ucur[kG], dcur[kG];
+    if (active) {
+        load_group<VEC>(urow, urev, L, lbeg, lend, ucur);
+        load_group<VEC>(drow, false, L, lbeg, lend, dcur);
+    }
+    stage_bc<NS, VEC>(Bs[0], Cs[0], Bk, Ck, N, L, lbeg, (int)min((int64_t)kLC, nloc));
+    cp_async_commit();
+
+    for (int ch = 0; ch < nchunk; ++ch) {
+        const int64_t cbeg = lbeg + (int64_t)ch * kLC;
+        const int clen = (int)min((int64_t)kLC, lend - cbeg);
+        const int buf = ch & 1;
+        if (ch + 1 < nchunk) {
+            const int64_t nbeg = cbeg + kLC;
+            stage_bc<NS, VEC>(Bs[buf ^ 1], Cs[buf ^ 1], Bk, Ck, N, L, nbeg, (int)min((int64_t)kLC, lend - nbeg));
+            cp_async_commit();
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncwarp();
+
+        for (int g = 0; g < clen; g += kG) {
+            const int64_t l0 = cbeg + g;
+            float unx[kG], dnx[kG];
+            const bool more = active && (l0 + kG < lend);
+            if (more) {
+                load_group<VEC>(urow, urev, L, l0 + kG, lend, unx);
+                load_group<VEC>(drow, false, L, l0 + kG, lend, dnx);
+            }
+            if (active) {
+                float dt[kG], dtu[kG], y[kG];
 #pragma unroll
-                for (int n4 = 0; n4 < NS / 4; ++n4) {
-                    const float4 bq = *reinterpret_cast<const float4 *>(&Bs[i][4 * n4]);
-                    const float4 cq = *reinterpret_cast<const float4 *>(&Cs[i][4 * n4]);
-                    const float bb[4] = {bq.x, bq.y, bq.z, bq.w};
-                    const float cc[4] = {cq.x, cq.y, cq.z, cq.w};
+                for (int j = 0; j < kG; ++j) {
+                    const float tt = dcur[j] + bias;
+                    dt[j] = p.softplus ? softplus_f(tt) : tt;
+                    dtu[j] = dt[j] * ucur[j];
+                    y[j] = Dc * ucur[j];  // skip term first: u is dead during the state loop
+                }
+                const int nvalid = (int)min((int64_t)kG, lend - l0);
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int n = 4 * n4 + j;
-                        const float a = ex2_sfu(dt * A2[n]);
-                        h[n] = fmaf(a, h[n], dtu * bb[j]);
-                        y = fmaf(cc[j], h[n], y);
+                for (int n = 0; n < NS; ++n) {
+                    const float a2 = A2s[n][t];
+                    float bq[kG], cq[kG];
+                    if (VEC) {
+                        ld4(&Bs[buf][n][g], bq);
+                        ld4(&Cs[buf][n][g], cq);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < kG; ++j) {
+                            bq[j] = (g + j < kLC) ? ld(&Bs[buf][n][g + j]) : 0.f;
+                            cq[j] = (g + j < kLC) ? ld(&Cs[buf][n][g + j]) : 0.f;
+                        }
+                    }
+#pragma unroll
+                    for (int j = 0; j < kG; ++j) {
+                        if (VEC || j < nvalid) {
+                            const float a = ex2_sfu(dt[j] * a2);
+                            h[n] = fmaf(a, h[n], dtu[j] * bq[j]);
+                            y[j] = fmaf(cq[j], h[n], y[j]);
+                        }
                     }
                 }
                 if (PASS == 1) {
-                    dtsum += dt;
+#pragma unroll
+                    for (int j = 0; j < kG; ++j)
+                        if (VEC || j < nvalid) dtsum += dt[j];
                 } else {
-                    us[t][i] = fmaf(Dc, uv, y);
-                    const int64_t l = l0 + i;
-                    if (p.chunk_states && (((l + 1) % kStateChunk) == 0 || l + 1 == L)) {
-                        float *cs = p.chunk_states + ((b * C4 + c) * p.nchunks + l / kStateChunk) * N;
+                    if (orow) {
+                        if (VEC) {
+                            st4(orow + l0, y);
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < kG; ++j)
+                                if (j < nvalid) st(orow + l0 + j, y[j]);
+                        }
+                    }
+                    const int64_t llast = l0 + nvalid - 1;
+                    if (p.chunk_states && (((llast + 1) % kStateChunk) == 0 || llast + 1 == L)) {
+                        float *cs = p.chunk_states + ((b * C4 + c) * p.nchunks + llast / kStateChunk) * N;
 #pragma unroll
                         for (int n = 0; n < NS; ++n)
                             if (n < N) cs[n] = h[n];
                     }
                 }
             }
-        }
-        if (PASS != 1 && p.out) {
-            __syncthreads();
-            for (int idx = t; idx < kTD * kLC; idx += kTD) {
-                const int ch = idx / kLC, i = idx % kLC;
-                if (ch < nch && i < len) st(out + (b * C4 + k * D + d0 + ch) * L + l0 + i, us[ch][i]);
+            if (more) {
+#pragma unroll
+                for (int j = 0; j < kG; ++j) {
+                    ucur[j] = unx[j];
+                    dcur[j] = dnx[j];
+                }
             }
         }
+        __syncwarp();  // every lane is done with this buffer before it is refilled
     }
 
     if (PASS == 1 && active) {
@@ -176,7 +300,7 @@ __global__ void __launch_bounds__(kTD) scan_fwd_kernel(const FwdParams p) {
 #pragma unroll
         for (int n = 0; n < NS; ++n)
             if (n < N) {
-                sg[n] = ex2_sfu(A2[n] * dtsum);
+                sg[n] = ex2_sfu(A2s[n][t] * dtsum);
                 sg[N + n] = h[n];
             }
     }
@@ -214,40 +338,40 @@ size_t scan_fwd_workspace_bytes(const LaunchShape &s) {
     return (size_t)s.B * kPaths * s.D * nseg * 2 * s.N * sizeof(float);
 }
 
-template <int NS, typename Tin, typename Tout, bool IMG>
-static cudaError_t launch_ns(const LaunchShape &s, const FwdParams &p, cudaStream_t stream) {
-    dim3 grid((unsigned)ceil_div(s.D, kTD), kPaths, (unsigned)(s.B * p.nseg));
+template <int NS, typename Tin, typename Tout, bool IMG, bool VEC>
+static cudaError_t launch_ns(const FwdParams &p, cudaStream_t stream) {
+    dim3 grid((unsigned)ceil_div(p.D, kWarp), kPaths, (unsigned)(p.B * p.nseg));
     if (p.nseg == 1) {
-        scan_fwd_kernel<NS, Tin, Tout, IMG, 0><<<grid, kTD, 0, stream>>>(p);
+        scan_fwd_kernel<NS, Tin, Tout, IMG, 0, VEC><<<grid, kWarp, 0, stream>>>(p);
         note_launch(stream);
     } else {
-        scan_fwd_kernel<NS, Tin, Tout, IMG, 1><<<grid, kTD, 0, stream>>>(p);
+        scan_fwd_kernel<NS, Tin, Tout, IMG, 1, VEC><<<grid, kWarp, 0, stream>>>(p);
         note_launch(stream);
-        scan_fwd_kernel<NS, Tin, Tout, IMG, 2><<<grid, kTD, 0, stream>>>(p);
+        scan_fwd_kernel<NS, Tin, Tout, IMG, 2, VEC><<<grid, kWarp, 0, stream>>>(p);
         note_launch(stream);
     }
     return cudaGetLastError();
 }
 
-template <typename Tin, typename Tout, bool IMG>
-static cudaError_t launch_types(const LaunchShape &s, const FwdParams &p, cudaStream_t stream) {
-    if (s.N <= 4) return launch_ns<4, Tin, Tout, IMG>(s, p, stream);
-    if (s.N <= 8) return launch_ns<8, Tin, Tout, IMG>(s, p, stream);
-    return launch_ns<16, Tin, Tout, IMG>(s, p, stream);
+template <typename Tin, typename Tout, bool IMG, bool VEC>
+static cudaError_t launch_types(const FwdParams &p, cudaStream_t stream) {
+    if (p.N <= 4) return launch_ns<4, Tin, Tout, IMG, VEC>(p, stream);
+    if (p.N <= 8) return launch_ns<8, Tin, Tout, IMG, VEC>(p, stream);
+    return launch_ns<16, Tin, Tout, IMG, VEC>(p, stream);
 }
 
-template <bool IMG>
-static cudaError_t launch_img(const LaunchShape &s, const FwdParams &p, ss2d_dtype_t din, ss2d_dtype_t dout,
-                              cudaStream_t stream) {
-    if (din == SS2D_F32 && dout == SS2D_F32) return launch_types<float, float, IMG>(s, p, stream);
-    if (din == SS2D_F32) return launch_types<float, __nv_bfloat16, IMG>(s, p, stream);
-    if (dout == SS2D_F32) return launch_types<__nv_bfloat16, float, IMG>(s, p, stream);
-    return launch_types<__nv_bfloat16, __nv_bfloat16, IMG>(s, p, stream);
+template <bool IMG, bool VEC>
+static cudaError_t launch_img(const FwdParams &p, ss2d_dtype_t din, ss2d_dtype_t dout, cudaStream_t stream) {
+    if (din == SS2D_F32 && dout == SS2D_F32) return launch_types<float, float, IMG, VEC>(p, stream);
+    if (din == SS2D_F32) return launch_types<float, __nv_bfloat16, IMG, VEC>(p, stream);
+    if (dout == SS2D_F32) return launch_types<__nv_bfloat16, float, IMG, VEC>(p, stream);
+    return launch_types<__nv_bfloat16, __nv_bfloat16, IMG, VEC>(p, stream);
 }
 
 cudaError_t launch_scan_fwd(const LaunchShape &s, const ScanFwdArgs &a, void *workspace, cudaStream_t stream) {
     FwdParams p;
     p.u = a.u;
+    p.uT = a.uT;
     p.delta = a.delta;
     p.A = a.A;
     p.Bm = a.Bm;
@@ -266,8 +390,13 @@ cudaError_t launch_scan_fwd(const LaunchShape &s, const ScanFwdArgs &a, void *wo
     p.softplus = a.softplus;
     seg_plan(s, a.max_segments, &p.nseg, &p.seglen);
     p.nchunks = ceil_div(s.L, kStateChunk);
-    if (a.from_image) return launch_img<true>(s, p, a.in_dtype, a.out_dtype, stream);
-    return launch_img<false>(s, p, a.in_dtype, a.out_dtype, stream);
+    // 4-step vector loads need every row start and step group 4-element aligned
+    const bool vec = (s.L % 4) == 0;
+    if (a.from_image)
+        return vec ? launch_img<true, true>(p, a.in_dtype, a.out_dtype, stream)
+                   : launch_img<true, false>(p, a.in_dtype, a.out_dtype, stream);
+    return vec ? launch_img<false, true>(p, a.in_dtype, a.out_dtype, stream)
+               : launch_img<false, false>(p, a.in_dtype, a.out_dtype, stream);
 }
 
 }  // namespace ss2d
