@@ -243,15 +243,27 @@ def run_gpu(args, world, rank, local):
     if args.batch:
         w = w.with_batch(args.batch)
     dev = torch.device("cuda", local)
-    inp = ss2d_inputs.make_inputs(w, seed=shard_seed(args.workload, rank), device=dev, with_dy=False)
+    inp = ss2d_inputs.make_inputs(w, seed=shard_seed(args.workload, rank), device=dev, with_dy=args.backward)
     y = torch.empty((w.batch, w.dim, w.height, w.width), dtype=w.torch_dtype, device=dev)
     nbytes = ss.workspace_bytes(w.batch, w.dim, w.height, w.width, w.d_state, ss.OP_FORWARD, w.torch_dtype)
     ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step():
-        ss.ss2d_forward(inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"], inp["delta_bias"], True,
-                        out=y, workspace=ws)
+    if args.backward:
+        nb = ss.workspace_bytes(w.batch, w.dim, w.height, w.width, w.d_state, ss.OP_BACKWARD, w.torch_dtype)
+        wsb = torch.empty(max(nb, 1), dtype=torch.uint8, device=dev)
+        cs = torch.empty((w.batch, 4 * w.dim, -(-w.L // ss.CHUNK_LEN), w.d_state), dtype=torch.float32, device=dev)
+
+        def step():
+            # forward keeping the chunk states, then the fused backward from them
+            ss.ss2d_forward(inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"], inp["delta_bias"],
+                            True, out=y, workspace=ws, chunk_states_out=cs)
+            ss.ss2d_backward(inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"], inp["delta_bias"],
+                             True, inp["dy"], chunk_states=cs, workspace=wsb)
+    else:
+        def step():
+            ss.ss2d_forward(inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"], inp["delta_bias"],
+                            True, out=y, workspace=ws)
 
     # kernels per step (to size the trace-event list)
     before = ss.launch_count()
@@ -314,7 +326,7 @@ def run_gpu(args, world, rank, local):
     sfu_achieved = w.updates / (dom_ms / 1e3) / 1e9  # one exp(dt*A) per state update
     traffic = recorded_traffic(w.name)
 
-    e2e = run_e2e(args, w, inp, dev, stream, world, rank) if not args.no_e2e else None
+    e2e = run_e2e(args, w, inp, dev, stream, world, rank) if not (args.no_e2e or args.backward) else None
 
     result = {
         "metric": METRIC,
@@ -332,6 +344,7 @@ def run_gpu(args, world, rank, local):
         "config": {"workload": w.name, "batch_per_gpu": w.batch, "global_batch": w.batch * world, "dim": w.dim,
                    "height": w.height, "width": w.width, "d_state": w.d_state, "paths": 4,
                    "parallelism": f"batch shards x{world}, no collective",
+                   "pass": "forward + backward" if args.backward else "forward",
                    "l2": f"inputs {alg_bytes / 1e9:.2f} GB > 126 MB L2, no flush needed"},
         "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved_gbs / hbm_peak, "traffic": traffic,
@@ -425,6 +438,8 @@ def main(argv=None):
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (small cases for profiling; not a bench line)")
     ap.add_argument("--impl", choices=["ss2d", "reference"], default="ss2d")
+    ap.add_argument("--backward", action="store_true",
+                    help="time forward (keeping chunk states) + fused backward per step")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="time budget of the CPU oracle sample")

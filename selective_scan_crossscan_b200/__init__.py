@@ -271,7 +271,7 @@ def selective_scan_bwd(u, delta, A, B, C, D, delta_bias, delta_softplus, dout, c
 # ------------------------------------------------------------------ fused --
 
 def ss2d_forward(x, delta, A, B, C, D=None, delta_bias=None, delta_softplus=True, out=None, out_dtype=None,
-                 return_chunk_states=False, workspace=None):
+                 return_chunk_states=False, workspace=None, chunk_states_out=None):
     """Fused SS2D forward.  x (Bn, D, H, W), delta (Bn, 4D, H*W), A (4D, N), B/C (Bn, 4, N, H*W).
 
     Returns y (Bn, D, H, W) [, chunk_states].  ``workspace`` may be a preallocated uint8
@@ -285,8 +285,8 @@ def ss2d_forward(x, delta, A, B, C, D=None, delta_bias=None, delta_softplus=True
     out_dtype = out_dtype or x.dtype
     if out is None:
         out = torch.empty((Bn, Dn, H, W), dtype=out_dtype, device=x.device)
-    cs = None
-    if return_chunk_states:
+    cs = chunk_states_out
+    if return_chunk_states and cs is None:
         cs = torch.empty((Bn, 4 * Dn, -(-(H * W) // CHUNK_LEN), N), dtype=torch.float32, device=x.device)
     d = _desc(Bn, Dn, H, W, N, x.dtype, out.dtype)
     lib = _load()

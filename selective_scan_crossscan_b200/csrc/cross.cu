@@ -204,7 +204,69 @@ cross_merge_vec_kernel(const Tin *__restrict__ ys, Tout *__restrict__ y, int64_t
     }
 }
 
+// Small planes (L <= kSmallPlane): a tile would leave most threads idle, so a CTA
+// handles whole planes instead.  Transpose: the CTA's planes are one contiguous
+// block in both x and xT; it is staged in shared memory and written back in
+// output order, so both global passes are fully coalesced.
+constexpr int kSmallPlane = 1024;
+constexpr int kSmallElems = 4096;  // elements staged per CTA
+
+template <typename T>
+__global__ void __launch_bounds__(256)
+transpose_small_kernel(const T *__restrict__ x, T *__restrict__ xT, int64_t planes, int H, int W) {
+    __shared__ T buf[kSmallElems];
+    const int L = H * W;
+    const int ppb = kSmallElems / L;
+    const int64_t p0 = (int64_t)blockIdx.x * ppb;
+    const int np = (int)min((int64_t)ppb, planes - p0);
+    const int n = np * L;
+    const T *src = x + p0 * L;
+    T *dst = xT + p0 * L;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) buf[i] = src[i];
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const int q = i / L, m = i - q * L;  // output position m = w*H + h of plane q
+        const int w = m / H, h = m - w * H;
+        dst[i] = buf[q * L + h * W + w];
+    }
+}
+
+// CrossMerge for small planes: one thread per output pixel; the four per-path
+// planes of a (b, d) span at most 4 KB each, so the column-order gathers stay in cache.
+template <typename Tin, typename Tout>
+__global__ void __launch_bounds__(256)
+cross_merge_small_kernel(const Tin *__restrict__ ys, Tout *__restrict__ y, int64_t Dn, int H, int W,
+                         int64_t total) {
+    const int64_t L = (int64_t)H * W;
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
+         e += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t bd = e / L;
+        const int p = (int)(e - bd * L);
+        const int64_t b = bd / Dn, d = bd - b * Dn;
+        const int h = p / W, w = p - h * W;
+        const int64_t lc = (int64_t)w * H + h;
+        const Tin *base = ys + (b * kPaths * Dn + d) * L;
+        const int64_t stride = Dn * L;  // between paths
+        const float t02 = ld(base + p) + ld(base + 2 * stride + (L - 1 - p));
+        const float t13 = ld(base + stride + lc) + ld(base + 3 * stride + (L - 1 - lc));
+        st(y + e, t02 + t13);
+    }
+}
+
 cudaError_t launch_transpose(const LaunchShape &s, ss2d_dtype_t dt, const void *x, void *xT, cudaStream_t stream) {
+    if (s.L <= kSmallPlane) {
+        const int64_t planes = s.B * s.D;
+        const int ppb = kSmallElems / (int)s.L;
+        const unsigned grid = (unsigned)ceil_div(planes, ppb);
+        if (dt == SS2D_F32)
+            transpose_small_kernel<float><<<grid, 256, 0, stream>>>((const float *)x, (float *)xT, planes, (int)s.H,
+                                                                    (int)s.W);
+        else
+            transpose_small_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
+                (const __nv_bfloat16 *)x, (__nv_bfloat16 *)xT, planes, (int)s.H, (int)s.W);
+        note_launch(stream);
+        return cudaGetLastError();
+    }
     int64_t tw, th;
     dim3 grid = tile_grid(s.B * s.D, s.H, s.W, &tw, &th);
     dim3 block(kTile, kRows);
@@ -223,9 +285,16 @@ cudaError_t launch_cross_merge(const LaunchShape &s, ss2d_dtype_t din, ss2d_dtyp
     dim3 grid = tile_grid(s.B * s.D, s.H, s.W, &tw, &th);
     dim3 block(kTile, kRows);
     const bool vec = (s.H % 4) == 0 && (s.W % 4) == 0;
+    const bool small = s.L <= kSmallPlane && !vec;
+    const int64_t total = s.B * s.D * s.L;
+    const int64_t small_blocks = ceil_div(total, 256);
+    const unsigned small_grid = (unsigned)(small_blocks < 148 * 32 ? small_blocks : 148 * 32);
 #define SS2D_MERGE(TI, TO)                                                                                      \
     do {                                                                                                        \
-        if (vec)                                                                                                \
+        if (small)                                                                                              \
+            cross_merge_small_kernel<TI, TO><<<small_grid, 256, 0, stream>>>((const TI *)ys, (TO *)y, s.D,       \
+                                                                            (int)s.H, (int)s.W, total);         \
+        else if (vec)                                                                                           \
             cross_merge_vec_kernel<TI, TO><<<grid, 256, 0, stream>>>((const TI *)ys, (TO *)y, s.D, s.H, s.W, tw, \
                                                                       th);                                      \
         else                                                                                                    \

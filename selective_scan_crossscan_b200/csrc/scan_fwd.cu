@@ -41,7 +41,7 @@ constexpr int kStateChunk = SS2D_CHUNK_LEN;
 // Resident CTAs (warps) per SM the forward kernel is compiled for; 21 puts the
 // headline problem's 3,072 warps in one wave on 148 SMs, fewer leaves more registers.
 #ifndef SS2D_FWD_MIN_BLOCKS
-#define SS2D_FWD_MIN_BLOCKS 20
+#define SS2D_FWD_MIN_BLOCKS 12
 #endif
 
 struct FwdParams {
@@ -129,60 +129,69 @@ __device__ __forceinline__ void stage_bc(Tin (*Bs)[kLC], Tin (*Cs)[kLC], const T
 }
 
 // PASS 0: single pass.  PASS 1: segment summaries only.  PASS 2: outputs with carries.
-template <int NS, typename Tin, typename Tout, bool IMG, int PASS, bool VEC>
+// SEQ sequences per thread: lane t of the CTA owns channels d0 + t + 32*s, s < SEQ, so
+// the B/C loads are shared by SEQ sequences and the independent chains interleave.
+template <int NS, int SEQ, typename Tin, typename Tout, bool IMG, int PASS, bool VEC>
 __global__ void __launch_bounds__(kWarp, SS2D_FWD_MIN_BLOCKS) scan_fwd_kernel(const FwdParams p) {
     __shared__ __align__(16) Tin Bs[2][NS][kLC];
     __shared__ __align__(16) Tin Cs[2][NS][kLC];
-    __shared__ float A2s[NS][kWarp];  // A[c, n] * log2(e) of each lane's channel (kept out of registers)
+    __shared__ float2 A2s[SEQ][NS][kWarp];  // (A[c,n]*log2 e) twice per lane's channel (kept out of registers)
 
     const int t = threadIdx.x;
     const int k = blockIdx.y;
     const int64_t b = blockIdx.z / p.nseg;
-    const int s = blockIdx.z % p.nseg;
+    const int sg_i = blockIdx.z % p.nseg;
     const int64_t D = p.D, L = p.L, C4 = kPaths * p.D;
-    const int64_t d = (int64_t)blockIdx.x * kWarp + t;
-    const bool active = d < D;
-    const int64_t c = k * D + (active ? d : 0);
+    const int64_t d0 = (int64_t)blockIdx.x * (kWarp * SEQ) + t;  // channel of sequence 0
     const int N = p.N;
-    const int64_t lbeg = (int64_t)s * p.seglen;
+    const int64_t lbeg = (int64_t)sg_i * p.seglen;
     const int64_t lend = min(L, lbeg + p.seglen);
 
-    float h[NS];
+    bool active[SEQ];
+    int64_t c[SEQ];
+    float h[SEQ][NS], Dc[SEQ], bias[SEQ], dtsum[SEQ];
 #pragma unroll
-    for (int n = 0; n < NS; ++n) {
-        A2s[n][t] = (active && n < N) ? p.A[c * N + n] * kLog2e : 0.f;
-        h[n] = 0.f;
-    }
-    __syncwarp();
-    const float Dc = (active && p.Dv) ? p.Dv[c] : 0.f;
-    const float bias = (active && p.bias) ? p.bias[c] : 0.f;
-
-    if (PASS == 2 && active) {
-        // carry into this segment: fold the summaries of the segments before it
-        const float *sg = p.seg + (b * C4 + c) * (int64_t)p.nseg * 2 * N;
-        for (int s2 = 0; s2 < s; ++s2) {
+    for (int q = 0; q < SEQ; ++q) {
+        const int64_t d = d0 + kWarp * q;
+        active[q] = d < D;
+        c[q] = k * D + (active[q] ? d : 0);
+        Dc[q] = (active[q] && p.Dv) ? p.Dv[c[q]] : 0.f;
+        bias[q] = (active[q] && p.bias) ? p.bias[c[q]] : 0.f;
+        dtsum[q] = 0.f;
 #pragma unroll
-            for (int n = 0; n < NS; ++n)
-                if (n < N) h[n] = fmaf(sg[(s2 * 2 + 0) * N + n], h[n], sg[(s2 * 2 + 1) * N + n]);
+        for (int n = 0; n < NS; ++n) {
+            const float a2 = (active[q] && n < N) ? p.A[c[q] * N + n] * kLog2e : 0.f;
+            A2s[q][n][t] = make_float2(a2, a2);
+            h[q][n] = 0.f;
+        }
+        if (PASS == 2 && active[q]) {
+            // carry into this segment: fold the summaries of the segments before it
+            const float *sg = p.seg + (b * C4 + c[q]) * (int64_t)p.nseg * 2 * N;
+            for (int s2 = 0; s2 < sg_i; ++s2) {
+#pragma unroll
+                for (int n = 0; n < NS; ++n)
+                    if (n < N) h[q][n] = fmaf(sg[(s2 * 2 + 0) * N + n], h[q][n], sg[(s2 * 2 + 1) * N + n]);
+            }
         }
     }
-    float dtsum = 0.f;
+    __syncwarp();
 
-    // this thread's u and delta sequences
+    // sequence 0's rows; sequence q sits 32*q rows further in every (.., channel, L) tensor
+    const int64_t qstride = (int64_t)kWarp * L;
     const Tin *urow;
     bool urev;
     if (IMG) {
         const Tin *img = static_cast<const Tin *>((k & 1) ? p.uT : p.u);
-        urow = img + (b * D + (active ? d : 0)) * L;
+        urow = img + (b * D + (active[0] ? d0 : 0)) * L;
         urev = k >= 2;
     } else {
-        urow = static_cast<const Tin *>(p.u) + (b * C4 + c) * L;
+        urow = static_cast<const Tin *>(p.u) + (b * C4 + c[0]) * L;
         urev = false;
     }
-    const Tin *drow = static_cast<const Tin *>(p.delta) + (b * C4 + c) * L;
+    const Tin *drow = static_cast<const Tin *>(p.delta) + (b * C4 + c[0]) * L;
     const Tin *Bk = static_cast<const Tin *>(p.Bm) + (b * kPaths + k) * N * L;
     const Tin *Ck = static_cast<const Tin *>(p.Cm) + (b * kPaths + k) * N * L;
-    Tout *orow = p.out ? static_cast<Tout *>(p.out) + (b * C4 + c) * L : nullptr;
+    Tout *orow = p.out ? static_cast<Tout *>(p.out) + (b * C4 + c[0]) * L : nullptr;
 
     const int64_t nloc = lend - lbeg;
     const int nchunk = (int)ceil_div(nloc, kLC);
@@ -198,11 +207,13 @@ __global__ void __launch_bounds__(kWarp, SS2D_FWD_MIN_BLOCKS) scan_fwd_kernel(co
         __syncwarp();
     }
 
-    float ucur[kG], dcur[kG];
-    if (active) {
-        load_group<VEC>(urow, urev, L, lbeg, lend, ucur);
-        load_group<VEC>(drow, false, L, lbeg, lend, dcur);
-    }
+    float ucur[SEQ][kG], dcur[SEQ][kG];
+#pragma unroll
+    for (int q = 0; q < SEQ; ++q)
+        if (active[q]) {
+            load_group<VEC>(urow + q * qstride, urev, L, lbeg, lend, ucur[q]);
+            load_group<VEC>(drow + q * qstride, false, L, lbeg, lend, dcur[q]);
+        }
     stage_bc<NS, VEC>(Bs[0], Cs[0], Bk, Ck, N, L, lbeg, (int)min((int64_t)kLC, nloc));
     cp_async_commit();
 
@@ -222,87 +233,118 @@ __global__ void __launch_bounds__(kWarp, SS2D_FWD_MIN_BLOCKS) scan_fwd_kernel(co
 
         for (int g = 0; g < clen; g += kG) {
             const int64_t l0 = cbeg + g;
-            float unx[kG], dnx[kG];
-            const bool more = active && (l0 + kG < lend);
-            if (more) {
-                load_group<VEC>(urow, urev, L, l0 + kG, lend, unx);
-                load_group<VEC>(drow, false, L, l0 + kG, lend, dnx);
-            }
-            if (active) {
-                float dt[kG], dtu[kG], y[kG];
+            const int nvalid = (int)min((int64_t)kG, lend - l0);
+            float unx[SEQ][kG], dnx[SEQ][kG];
+            const bool more = l0 + kG < lend;
 #pragma unroll
-                for (int j = 0; j < kG; ++j) {
-                    const float tt = dcur[j] + bias;
-                    dt[j] = p.softplus ? softplus_f(tt) : tt;
-                    dtu[j] = dt[j] * ucur[j];
-                    y[j] = Dc * ucur[j];  // skip term first: u is dead during the state loop
+            for (int q = 0; q < SEQ; ++q)
+                if (more && active[q]) {
+                    load_group<VEC>(urow + q * qstride, urev, L, l0 + kG, lend, unx[q]);
+                    load_group<VEC>(drow + q * qstride, false, L, l0 + kG, lend, dnx[q]);
                 }
-                const int nvalid = (int)min((int64_t)kG, lend - l0);
+
+            // per sequence: step sizes, dt*u and the skip term, steps (0,1) and (2,3) packed (f32x2)
+            float2 dt01[SEQ], dt23[SEQ], dtu01[SEQ], dtu23[SEQ], y01[SEQ], y23[SEQ];
 #pragma unroll
-                for (int n = 0; n < NS; ++n) {
-                    const float a2 = A2s[n][t];
-                    float bq[kG], cq[kG];
-                    if (VEC) {
-                        ld4(&Bs[buf][n][g], bq);
-                        ld4(&Cs[buf][n][g], cq);
-                    } else {
+            for (int q = 0; q < SEQ; ++q) {
+                const float2 t01 = make_float2(dcur[q][0] + bias[q], dcur[q][1] + bias[q]);
+                const float2 t23 = make_float2(dcur[q][2] + bias[q], dcur[q][3] + bias[q]);
+                dt01[q] = p.softplus ? softplus_f2(t01) : t01;
+                dt23[q] = p.softplus ? softplus_f2(t23) : t23;
+                if (!VEC && nvalid < kG) {
+                    // steps past the end keep h unchanged: dt = 0 gives decay 1 and input 0
+                    if (nvalid < 2) dt01[q].y = 0.f;
+                    if (nvalid < 3) dt23[q].x = 0.f;
+                    dt23[q].y = 0.f;
+                }
+                const float2 u01 = make_float2(ucur[q][0], ucur[q][1]);
+                const float2 u23 = make_float2(ucur[q][2], ucur[q][3]);
+                dtu01[q] = __fmul2_rn(dt01[q], u01);
+                dtu23[q] = __fmul2_rn(dt23[q], u23);
+                // skip term first: u is not needed during the state loop
+                y01[q] = __fmul2_rn(make_float2(Dc[q], Dc[q]), u01);
+                y23[q] = __fmul2_rn(make_float2(Dc[q], Dc[q]), u23);
+            }
 #pragma unroll
-                        for (int j = 0; j < kG; ++j) {
-                            bq[j] = (g + j < kLC) ? ld(&Bs[buf][n][g + j]) : 0.f;
-                            cq[j] = (g + j < kLC) ? ld(&Cs[buf][n][g + j]) : 0.f;
-                        }
-                    }
+            for (int n = 0; n < NS; ++n) {
+                float bq[kG], cq[kG];
+                if (VEC) {
+                    ld4(&Bs[buf][n][g], bq);
+                    ld4(&Cs[buf][n][g], cq);
+                } else {
 #pragma unroll
                     for (int j = 0; j < kG; ++j) {
-                        if (VEC || j < nvalid) {
-                            const float a = ex2_sfu(dt[j] * a2);
-                            h[n] = fmaf(a, h[n], dtu[j] * bq[j]);
-                            y[j] = fmaf(cq[j], h[n], y[j]);
-                        }
+                        bq[j] = (g + j < kLC) ? ld(&Bs[buf][n][g + j]) : 0.f;
+                        cq[j] = (g + j < kLC) ? ld(&Cs[buf][n][g + j]) : 0.f;
                     }
                 }
-                if (PASS == 1) {
+                const float2 b01v = make_float2(bq[0], bq[1]), b23v = make_float2(bq[2], bq[3]);
+                const float2 c01v = make_float2(cq[0], cq[1]), c23v = make_float2(cq[2], cq[3]);
 #pragma unroll
-                    for (int j = 0; j < kG; ++j)
-                        if (VEC || j < nvalid) dtsum += dt[j];
+                for (int q = 0; q < SEQ; ++q) {
+                    const float2 a2 = A2s[q][n][t];
+                    const float2 x01 = __fmul2_rn(dt01[q], a2), x23 = __fmul2_rn(dt23[q], a2);
+                    const float2 b01 = __fmul2_rn(dtu01[q], b01v), b23 = __fmul2_rn(dtu23[q], b23v);
+                    const float h0 = fmaf(ex2_sfu(x01.x), h[q][n], b01.x);
+                    const float h1 = fmaf(ex2_sfu(x01.y), h0, b01.y);
+                    const float h2 = fmaf(ex2_sfu(x23.x), h1, b23.x);
+                    const float h3 = fmaf(ex2_sfu(x23.y), h2, b23.y);
+                    h[q][n] = h3;
+                    y01[q] = __ffma2_rn(c01v, make_float2(h0, h1), y01[q]);
+                    y23[q] = __ffma2_rn(c23v, make_float2(h2, h3), y23[q]);
+                }
+            }
+#pragma unroll
+            for (int q = 0; q < SEQ; ++q) {
+                if (!active[q]) continue;
+                if (PASS == 1) {
+                    dtsum[q] += (dt01[q].x + dt01[q].y) + (dt23[q].x + dt23[q].y);
                 } else {
+                    const float y[kG] = {y01[q].x, y01[q].y, y23[q].x, y23[q].y};
                     if (orow) {
+                        Tout *o = orow + q * qstride;
                         if (VEC) {
-                            st4(orow + l0, y);
+                            st4(o + l0, y);
                         } else {
 #pragma unroll
                             for (int j = 0; j < kG; ++j)
-                                if (j < nvalid) st(orow + l0 + j, y[j]);
+                                if (j < nvalid) st(o + l0 + j, y[j]);
                         }
                     }
                     const int64_t llast = l0 + nvalid - 1;
                     if (p.chunk_states && (((llast + 1) % kStateChunk) == 0 || llast + 1 == L)) {
-                        float *cs = p.chunk_states + ((b * C4 + c) * p.nchunks + llast / kStateChunk) * N;
+                        float *cs = p.chunk_states + ((b * C4 + c[q]) * p.nchunks + llast / kStateChunk) * N;
 #pragma unroll
                         for (int n = 0; n < NS; ++n)
-                            if (n < N) cs[n] = h[n];
+                            if (n < N) cs[n] = h[q][n];
                     }
                 }
             }
             if (more) {
 #pragma unroll
-                for (int j = 0; j < kG; ++j) {
-                    ucur[j] = unx[j];
-                    dcur[j] = dnx[j];
-                }
+                for (int q = 0; q < SEQ; ++q)
+#pragma unroll
+                    for (int j = 0; j < kG; ++j) {
+                        ucur[q][j] = unx[q][j];
+                        dcur[q][j] = dnx[q][j];
+                    }
             }
         }
         __syncwarp();  // every lane is done with this buffer before it is refilled
     }
 
-    if (PASS == 1 && active) {
-        float *sg = p.seg + ((b * C4 + c) * (int64_t)p.nseg + s) * 2 * N;
+    if (PASS == 1) {
 #pragma unroll
-        for (int n = 0; n < NS; ++n)
-            if (n < N) {
-                sg[n] = ex2_sfu(A2s[n][t] * dtsum);
-                sg[N + n] = h[n];
-            }
+        for (int q = 0; q < SEQ; ++q) {
+            if (!active[q]) continue;
+            float *sg = p.seg + ((b * C4 + c[q]) * (int64_t)p.nseg + sg_i) * 2 * N;
+#pragma unroll
+            for (int n = 0; n < NS; ++n)
+                if (n < N) {
+                    sg[n] = ex2_sfu(A2s[q][n][t].x * dtsum[q]);
+                    sg[N + n] = h[q][n];
+                }
+        }
     }
 }
 
@@ -338,16 +380,22 @@ size_t scan_fwd_workspace_bytes(const LaunchShape &s) {
     return (size_t)s.B * kPaths * s.D * nseg * 2 * s.N * sizeof(float);
 }
 
+// sequences per thread (see scan_fwd_kernel)
+#ifndef SS2D_FWD_SEQ
+#define SS2D_FWD_SEQ 1
+#endif
+
 template <int NS, typename Tin, typename Tout, bool IMG, bool VEC>
 static cudaError_t launch_ns(const FwdParams &p, cudaStream_t stream) {
-    dim3 grid((unsigned)ceil_div(p.D, kWarp), kPaths, (unsigned)(p.B * p.nseg));
+    constexpr int SEQ = SS2D_FWD_SEQ;
+    dim3 grid((unsigned)ceil_div(p.D, kWarp * SEQ), kPaths, (unsigned)(p.B * p.nseg));
     if (p.nseg == 1) {
-        scan_fwd_kernel<NS, Tin, Tout, IMG, 0, VEC><<<grid, kWarp, 0, stream>>>(p);
+        scan_fwd_kernel<NS, SEQ, Tin, Tout, IMG, 0, VEC><<<grid, kWarp, 0, stream>>>(p);
         note_launch(stream);
     } else {
-        scan_fwd_kernel<NS, Tin, Tout, IMG, 1, VEC><<<grid, kWarp, 0, stream>>>(p);
+        scan_fwd_kernel<NS, SEQ, Tin, Tout, IMG, 1, VEC><<<grid, kWarp, 0, stream>>>(p);
         note_launch(stream);
-        scan_fwd_kernel<NS, Tin, Tout, IMG, 2, VEC><<<grid, kWarp, 0, stream>>>(p);
+        scan_fwd_kernel<NS, SEQ, Tin, Tout, IMG, 2, VEC><<<grid, kWarp, 0, stream>>>(p);
         note_launch(stream);
     }
     return cudaGetLastError();
