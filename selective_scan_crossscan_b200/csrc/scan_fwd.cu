@@ -34,14 +34,14 @@
 namespace ss2d {
 
 constexpr int kWarp = 32;   // threads (= channels) per CTA
-constexpr int kLC = 32;     // steps of B/C per staged chunk
+constexpr int kLC = 16;     // steps staged per chunk (B/C, u, delta)
 constexpr int kG = 4;       // steps per register group
 constexpr int kStateChunk = SS2D_CHUNK_LEN;
 
 // Resident CTAs (warps) per SM the forward kernel is compiled for; 21 puts the
 // headline problem's 3,072 warps in one wave on 148 SMs, fewer leaves more registers.
 #ifndef SS2D_FWD_MIN_BLOCKS
-#define SS2D_FWD_MIN_BLOCKS 12
+#define SS2D_FWD_MIN_BLOCKS 16
 #endif
 
 struct FwdParams {
@@ -64,36 +64,11 @@ struct FwdParams {
     int64_t nchunks;
 };
 
-// Four steps l0..l0+3 of a sequence stored forwards (rev = false) or backwards
-// (step l at index L-1-l).  VEC: one aligned vector load; else scalar loads
-// with bounds (steps at or past lend read as 0).
-template <bool VEC, typename T>
-__device__ __forceinline__ void load_group(const T *row, bool rev, int64_t L, int64_t l0, int64_t lend, float v[4]) {
-    if (VEC) {
-        if (!rev) {
-            ld4(row + l0, v);
-        } else {
-            float w[4];
-            ld4(row + (L - 4 - l0), w);
-            v[0] = w[3];
-            v[1] = w[2];
-            v[2] = w[1];
-            v[3] = w[0];
-        }
-    } else {
-#pragma unroll
-        for (int j = 0; j < kG; ++j) {
-            const int64_t l = l0 + j;
-            v[j] = (l < lend) ? ld(row + (rev ? (L - 1 - l) : l)) : 0.f;
-        }
-    }
-}
-
 template <typename T>
 __device__ __forceinline__ void cp_async_bytes(T *smem_dst, const T *gsrc, int bytes) {
     const unsigned dst = (unsigned)__cvta_generic_to_shared(smem_dst);
     if (bytes == 16)
-        asm volatile("cp.async.ca.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(gsrc));
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(gsrc));
     else if (bytes == 8)
         asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(dst), "l"(gsrc));
     else
@@ -103,95 +78,117 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
 
-// Stage B/C steps [l0, l0+len) of group (b, k) into smem buffers [NS][kLC].
-// VEC: 4-element cp.async copies (len is a multiple of 4); else plain loads.
+// Shared-memory staging of one chunk (kLC steps):
+//  * B/C of group (b, k): [NS][kLC], shared by the 32 lanes;
+//  * each lane's u and delta rows: [32][kRow], rows padded to kRow elements so
+//    the per-lane 4-step vector reads hit distinct banks.  A reversed u row
+//    (paths 2, 3) is copied in memory order: step cbeg+i sits at kLC-1-i.
+template <typename Tin, int NS>
+struct FwdStage {
+    static constexpr int kRow = kLC + 4;
+    Tin B[NS][kLC];
+    Tin C[NS][kLC];
+    Tin U[kWarp][kRow];
+    Tin Dl[kWarp][kRow];
+};
+
+// Issue the copies of chunk [cbeg, cbeg+len).  VEC: 4-element cp.async pieces
+// (len is then a multiple of 4); else plain loads (synchronous).
 template <int NS, bool VEC, typename Tin>
-__device__ __forceinline__ void stage_bc(Tin (*Bs)[kLC], Tin (*Cs)[kLC], const Tin *Bk, const Tin *Ck, int N,
-                                         int64_t L, int64_t l0, int len) {
+__device__ __forceinline__ void stage_chunk(FwdStage<Tin, NS> &st, const Tin *Bk, const Tin *Ck, int N, int64_t L,
+                                            const Tin *urow, bool urev, const Tin *drow, bool active, int64_t cbeg,
+                                            int len) {
     const int t = threadIdx.x;
+    constexpr int kBytes = 4 * (int)sizeof(Tin);
     if (VEC) {
-        const int q = kLC / 4;
+        constexpr int q = kLC / 4;
         for (int idx = t; idx < NS * q; idx += kWarp) {
             const int n = idx / q, i4 = (idx % q) * 4;
             if (n < N && i4 < len) {
-                cp_async_bytes(&Bs[n][i4], Bk + (int64_t)n * L + l0 + i4, 4 * (int)sizeof(Tin));
-                cp_async_bytes(&Cs[n][i4], Ck + (int64_t)n * L + l0 + i4, 4 * (int)sizeof(Tin));
+                cp_async_bytes(&st.B[n][i4], Bk + (int64_t)n * L + cbeg + i4, kBytes);
+                cp_async_bytes(&st.C[n][i4], Ck + (int64_t)n * L + cbeg + i4, kBytes);
+            }
+        }
+        if (active) {
+#pragma unroll
+            for (int i4 = 0; i4 < kLC; i4 += 4) {
+                if (i4 < len) {
+                    cp_async_bytes(&st.Dl[t][i4], drow + cbeg + i4, kBytes);
+                    if (!urev)
+                        cp_async_bytes(&st.U[t][i4], urow + cbeg + i4, kBytes);
+                    else  // steps cbeg+i4 .. +3 live at memory L-1-cbeg-i4-3 .. L-1-cbeg-i4
+                        cp_async_bytes(&st.U[t][kLC - 4 - i4], urow + (L - cbeg - 4 - i4), kBytes);
+                }
             }
         }
     } else {
         for (int idx = t; idx < NS * kLC; idx += kWarp) {
             const int n = idx / kLC, i = idx % kLC;
             const bool ok = n < N && i < len;
-            Bs[n][i] = ok ? Bk[(int64_t)n * L + l0 + i] : Tin(0.f);
-            Cs[n][i] = ok ? Ck[(int64_t)n * L + l0 + i] : Tin(0.f);
+            st.B[n][i] = ok ? Bk[(int64_t)n * L + cbeg + i] : Tin(0.f);
+            st.C[n][i] = ok ? Ck[(int64_t)n * L + cbeg + i] : Tin(0.f);
+        }
+        for (int i = 0; i < kLC; ++i) {
+            const bool ok = active && i < len;
+            const int64_t l = cbeg + i;
+            st.Dl[t][i] = ok ? drow[l] : Tin(0.f);
+            st.U[t][urev ? (kLC - 1 - i) : i] = ok ? urow[urev ? (L - 1 - l) : l] : Tin(0.f);
         }
     }
 }
 
 // PASS 0: single pass.  PASS 1: segment summaries only.  PASS 2: outputs with carries.
-// SEQ sequences per thread: lane t of the CTA owns channels d0 + t + 32*s, s < SEQ, so
-// the B/C loads are shared by SEQ sequences and the independent chains interleave.
-template <int NS, int SEQ, typename Tin, typename Tout, bool IMG, int PASS, bool VEC>
+template <int NS, typename Tin, typename Tout, bool IMG, int PASS, bool VEC>
 __global__ void __launch_bounds__(kWarp, SS2D_FWD_MIN_BLOCKS) scan_fwd_kernel(const FwdParams p) {
-    __shared__ __align__(16) Tin Bs[2][NS][kLC];
-    __shared__ __align__(16) Tin Cs[2][NS][kLC];
-    __shared__ float2 A2s[SEQ][NS][kWarp];  // (A[c,n]*log2 e) twice per lane's channel (kept out of registers)
+    __shared__ __align__(16) FwdStage<Tin, NS> stage[2];
+    __shared__ float A2s[NS][kWarp];  // A[c, n] * log2(e) of each lane's channel (kept out of registers)
 
     const int t = threadIdx.x;
     const int k = blockIdx.y;
     const int64_t b = blockIdx.z / p.nseg;
-    const int sg_i = blockIdx.z % p.nseg;
+    const int sgi = blockIdx.z % p.nseg;
     const int64_t D = p.D, L = p.L, C4 = kPaths * p.D;
-    const int64_t d0 = (int64_t)blockIdx.x * (kWarp * SEQ) + t;  // channel of sequence 0
+    const int64_t d = (int64_t)blockIdx.x * kWarp + t;
+    const bool active = d < D;
+    const int64_t c = k * D + (active ? d : 0);
     const int N = p.N;
-    const int64_t lbeg = (int64_t)sg_i * p.seglen;
+    const int64_t lbeg = (int64_t)sgi * p.seglen;
     const int64_t lend = min(L, lbeg + p.seglen);
 
-    bool active[SEQ];
-    int64_t c[SEQ];
-    float h[SEQ][NS], Dc[SEQ], bias[SEQ], dtsum[SEQ];
+    float h[NS];
 #pragma unroll
-    for (int q = 0; q < SEQ; ++q) {
-        const int64_t d = d0 + kWarp * q;
-        active[q] = d < D;
-        c[q] = k * D + (active[q] ? d : 0);
-        Dc[q] = (active[q] && p.Dv) ? p.Dv[c[q]] : 0.f;
-        bias[q] = (active[q] && p.bias) ? p.bias[c[q]] : 0.f;
-        dtsum[q] = 0.f;
+    for (int n = 0; n < NS; ++n) {
+        A2s[n][t] = (active && n < N) ? p.A[c * N + n] * kLog2e : 0.f;
+        h[n] = 0.f;
+    }
+    const float Dc = (active && p.Dv) ? p.Dv[c] : 0.f;
+    const float bias = (active && p.bias) ? p.bias[c] : 0.f;
+    if (PASS == 2 && active) {
+        // carry into this segment: fold the summaries of the segments before it
+        const float *sg = p.seg + (b * C4 + c) * (int64_t)p.nseg * 2 * N;
+        for (int s2 = 0; s2 < sgi; ++s2) {
 #pragma unroll
-        for (int n = 0; n < NS; ++n) {
-            const float a2 = (active[q] && n < N) ? p.A[c[q] * N + n] * kLog2e : 0.f;
-            A2s[q][n][t] = make_float2(a2, a2);
-            h[q][n] = 0.f;
-        }
-        if (PASS == 2 && active[q]) {
-            // carry into this segment: fold the summaries of the segments before it
-            const float *sg = p.seg + (b * C4 + c[q]) * (int64_t)p.nseg * 2 * N;
-            for (int s2 = 0; s2 < sg_i; ++s2) {
-#pragma unroll
-                for (int n = 0; n < NS; ++n)
-                    if (n < N) h[q][n] = fmaf(sg[(s2 * 2 + 0) * N + n], h[q][n], sg[(s2 * 2 + 1) * N + n]);
-            }
+            for (int n = 0; n < NS; ++n)
+                if (n < N) h[n] = fmaf(sg[(s2 * 2 + 0) * N + n], h[n], sg[(s2 * 2 + 1) * N + n]);
         }
     }
-    __syncwarp();
+    float dtsum = 0.f;
 
-    // sequence 0's rows; sequence q sits 32*q rows further in every (.., channel, L) tensor
-    const int64_t qstride = (int64_t)kWarp * L;
+    // this lane's u and delta sequences
     const Tin *urow;
     bool urev;
     if (IMG) {
         const Tin *img = static_cast<const Tin *>((k & 1) ? p.uT : p.u);
-        urow = img + (b * D + (active[0] ? d0 : 0)) * L;
+        urow = img + (b * D + (active ? d : 0)) * L;
         urev = k >= 2;
     } else {
-        urow = static_cast<const Tin *>(p.u) + (b * C4 + c[0]) * L;
+        urow = static_cast<const Tin *>(p.u) + (b * C4 + c) * L;
         urev = false;
     }
-    const Tin *drow = static_cast<const Tin *>(p.delta) + (b * C4 + c[0]) * L;
+    const Tin *drow = static_cast<const Tin *>(p.delta) + (b * C4 + c) * L;
     const Tin *Bk = static_cast<const Tin *>(p.Bm) + (b * kPaths + k) * N * L;
     const Tin *Ck = static_cast<const Tin *>(p.Cm) + (b * kPaths + k) * N * L;
-    Tout *orow = p.out ? static_cast<Tout *>(p.out) + (b * C4 + c[0]) * L : nullptr;
+    Tout *orow = p.out ? static_cast<Tout *>(p.out) + (b * C4 + c) * L : nullptr;
 
     const int64_t nloc = lend - lbeg;
     const int nchunk = (int)ceil_div(nloc, kLC);
@@ -199,22 +196,15 @@ __global__ void __launch_bounds__(kWarp, SS2D_FWD_MIN_BLOCKS) scan_fwd_kernel(co
     // rows n >= N of the B/C buffers are never copied: zero them once so padded
     // states stay at h = 0 and contribute nothing
     if (VEC && N < NS) {
-        Tin *bz = &Bs[0][0][0], *cz = &Cs[0][0][0];
-        for (int i = t; i < 2 * NS * kLC; i += kWarp) {
-            bz[i] = Tin(0.f);
-            cz[i] = Tin(0.f);
-        }
-        __syncwarp();
+        for (int sb = 0; sb < 2; ++sb)
+            for (int i = t; i < NS * kLC; i += kWarp) {
+                (&stage[sb].B[0][0])[i] = Tin(0.f);
+                (&stage[sb].C[0][0])[i] = Tin(0.f);
+            }
     }
+    __syncwarp();
 
-    float ucur[SEQ][kG], dcur[SEQ][kG];
-#pragma unroll
-    for (int q = 0; q < SEQ; ++q)
-        if (active[q]) {
-            load_group<VEC>(urow + q * qstride, urev, L, lbeg, lend, ucur[q]);
-            load_group<VEC>(drow + q * qstride, false, L, lbeg, lend, dcur[q]);
-        }
-    stage_bc<NS, VEC>(Bs[0], Cs[0], Bk, Ck, N, L, lbeg, (int)min((int64_t)kLC, nloc));
+    stage_chunk<NS, VEC>(stage[0], Bk, Ck, N, L, urow, urev, drow, active, lbeg, (int)min((int64_t)kLC, nloc));
     cp_async_commit();
 
     for (int ch = 0; ch < nchunk; ++ch) {
@@ -223,128 +213,116 @@ __global__ void __launch_bounds__(kWarp, SS2D_FWD_MIN_BLOCKS) scan_fwd_kernel(co
         const int buf = ch & 1;
         if (ch + 1 < nchunk) {
             const int64_t nbeg = cbeg + kLC;
-            stage_bc<NS, VEC>(Bs[buf ^ 1], Cs[buf ^ 1], Bk, Ck, N, L, nbeg, (int)min((int64_t)kLC, lend - nbeg));
+            stage_chunk<NS, VEC>(stage[buf ^ 1], Bk, Ck, N, L, urow, urev, drow, active, nbeg,
+                                 (int)min((int64_t)kLC, lend - nbeg));
             cp_async_commit();
             cp_async_wait<1>();
         } else {
             cp_async_wait<0>();
         }
         __syncwarp();
+        const FwdStage<Tin, NS> &sm = stage[buf];
 
-        for (int g = 0; g < clen; g += kG) {
-            const int64_t l0 = cbeg + g;
-            const int nvalid = (int)min((int64_t)kG, lend - l0);
-            float unx[SEQ][kG], dnx[SEQ][kG];
-            const bool more = l0 + kG < lend;
-#pragma unroll
-            for (int q = 0; q < SEQ; ++q)
-                if (more && active[q]) {
-                    load_group<VEC>(urow + q * qstride, urev, L, l0 + kG, lend, unx[q]);
-                    load_group<VEC>(drow + q * qstride, false, L, l0 + kG, lend, dnx[q]);
-                }
-
-            // per sequence: step sizes, dt*u and the skip term, steps (0,1) and (2,3) packed (f32x2)
-            float2 dt01[SEQ], dt23[SEQ], dtu01[SEQ], dtu23[SEQ], y01[SEQ], y23[SEQ];
-#pragma unroll
-            for (int q = 0; q < SEQ; ++q) {
-                const float2 t01 = make_float2(dcur[q][0] + bias[q], dcur[q][1] + bias[q]);
-                const float2 t23 = make_float2(dcur[q][2] + bias[q], dcur[q][3] + bias[q]);
-                dt01[q] = p.softplus ? softplus_f2(t01) : t01;
-                dt23[q] = p.softplus ? softplus_f2(t23) : t23;
-                if (!VEC && nvalid < kG) {
-                    // steps past the end keep h unchanged: dt = 0 gives decay 1 and input 0
-                    if (nvalid < 2) dt01[q].y = 0.f;
-                    if (nvalid < 3) dt23[q].x = 0.f;
-                    dt23[q].y = 0.f;
-                }
-                const float2 u01 = make_float2(ucur[q][0], ucur[q][1]);
-                const float2 u23 = make_float2(ucur[q][2], ucur[q][3]);
-                dtu01[q] = __fmul2_rn(dt01[q], u01);
-                dtu23[q] = __fmul2_rn(dt23[q], u23);
-                // skip term first: u is not needed during the state loop
-                y01[q] = __fmul2_rn(make_float2(Dc[q], Dc[q]), u01);
-                y23[q] = __fmul2_rn(make_float2(Dc[q], Dc[q]), u23);
-            }
-#pragma unroll
-            for (int n = 0; n < NS; ++n) {
-                float bq[kG], cq[kG];
+        if (active) {
+            for (int g = 0; g < clen; g += kG) {
+                const int64_t l0 = cbeg + g;
+                const int nvalid = (int)min((int64_t)kG, lend - l0);
+                float uv[kG], dv[kG];
                 if (VEC) {
-                    ld4(&Bs[buf][n][g], bq);
-                    ld4(&Cs[buf][n][g], cq);
+                    ld4(&sm.Dl[t][g], dv);
+                    if (!urev) {
+                        ld4(&sm.U[t][g], uv);
+                    } else {
+                        float w[kG];
+                        ld4(&sm.U[t][kLC - 4 - g], w);
+                        uv[0] = w[3];
+                        uv[1] = w[2];
+                        uv[2] = w[1];
+                        uv[3] = w[0];
+                    }
                 } else {
 #pragma unroll
                     for (int j = 0; j < kG; ++j) {
-                        bq[j] = (g + j < kLC) ? ld(&Bs[buf][n][g + j]) : 0.f;
-                        cq[j] = (g + j < kLC) ? ld(&Cs[buf][n][g + j]) : 0.f;
+                        dv[j] = (g + j < kLC) ? ld(&sm.Dl[t][g + j]) : 0.f;
+                        uv[j] = (g + j < kLC) ? ld(&sm.U[t][urev ? (kLC - 1 - g - j) : (g + j)]) : 0.f;
                     }
                 }
-                const float2 b01v = make_float2(bq[0], bq[1]), b23v = make_float2(bq[2], bq[3]);
-                const float2 c01v = make_float2(cq[0], cq[1]), c23v = make_float2(cq[2], cq[3]);
+                // step pairs (0,1) and (2,3) ride the packed fp32 pipe (f32x2)
+                const float2 t01 = make_float2(dv[0] + bias, dv[1] + bias);
+                const float2 t23 = make_float2(dv[2] + bias, dv[3] + bias);
+                float2 dt01 = p.softplus ? softplus_f2(t01) : t01;
+                float2 dt23 = p.softplus ? softplus_f2(t23) : t23;
+                if (!VEC && nvalid < kG) {
+                    // steps past the end keep h unchanged: dt = 0 gives decay 1 and input 0
+                    if (nvalid < 2) dt01.y = 0.f;
+                    if (nvalid < 3) dt23.x = 0.f;
+                    dt23.y = 0.f;
+                }
+                const float2 u01 = make_float2(uv[0], uv[1]), u23 = make_float2(uv[2], uv[3]);
+                const float2 dtu01 = __fmul2_rn(dt01, u01), dtu23 = __fmul2_rn(dt23, u23);
+                // skip term first: u is not needed during the state loop
+                float2 y01 = __fmul2_rn(make_float2(Dc, Dc), u01);
+                float2 y23 = __fmul2_rn(make_float2(Dc, Dc), u23);
 #pragma unroll
-                for (int q = 0; q < SEQ; ++q) {
-                    const float2 a2 = A2s[q][n][t];
-                    const float2 x01 = __fmul2_rn(dt01[q], a2), x23 = __fmul2_rn(dt23[q], a2);
-                    const float2 b01 = __fmul2_rn(dtu01[q], b01v), b23 = __fmul2_rn(dtu23[q], b23v);
-                    const float h0 = fmaf(ex2_sfu(x01.x), h[q][n], b01.x);
+                for (int n = 0; n < NS; ++n) {
+                    const float a2s = A2s[n][t];
+                    const float2 a2 = make_float2(a2s, a2s);
+                    float bq[kG], cq[kG];
+                    if (VEC) {
+                        ld4(&sm.B[n][g], bq);
+                        ld4(&sm.C[n][g], cq);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < kG; ++j) {
+                            bq[j] = (g + j < kLC) ? ld(&sm.B[n][g + j]) : 0.f;
+                            cq[j] = (g + j < kLC) ? ld(&sm.C[n][g + j]) : 0.f;
+                        }
+                    }
+                    const float2 x01 = __fmul2_rn(dt01, a2), x23 = __fmul2_rn(dt23, a2);
+                    const float2 b01 = __fmul2_rn(dtu01, make_float2(bq[0], bq[1]));
+                    const float2 b23 = __fmul2_rn(dtu23, make_float2(bq[2], bq[3]));
+                    const float h0 = fmaf(ex2_sfu(x01.x), h[n], b01.x);
                     const float h1 = fmaf(ex2_sfu(x01.y), h0, b01.y);
                     const float h2 = fmaf(ex2_sfu(x23.x), h1, b23.x);
                     const float h3 = fmaf(ex2_sfu(x23.y), h2, b23.y);
-                    h[q][n] = h3;
-                    y01[q] = __ffma2_rn(c01v, make_float2(h0, h1), y01[q]);
-                    y23[q] = __ffma2_rn(c23v, make_float2(h2, h3), y23[q]);
+                    h[n] = h3;
+                    y01 = __ffma2_rn(make_float2(cq[0], cq[1]), make_float2(h0, h1), y01);
+                    y23 = __ffma2_rn(make_float2(cq[2], cq[3]), make_float2(h2, h3), y23);
                 }
-            }
-#pragma unroll
-            for (int q = 0; q < SEQ; ++q) {
-                if (!active[q]) continue;
                 if (PASS == 1) {
-                    dtsum[q] += (dt01[q].x + dt01[q].y) + (dt23[q].x + dt23[q].y);
+                    dtsum += (dt01.x + dt01.y) + (dt23.x + dt23.y);
                 } else {
-                    const float y[kG] = {y01[q].x, y01[q].y, y23[q].x, y23[q].y};
+                    const float y[kG] = {y01.x, y01.y, y23.x, y23.y};
                     if (orow) {
-                        Tout *o = orow + q * qstride;
                         if (VEC) {
-                            st4(o + l0, y);
+                            st4(orow + l0, y);
                         } else {
 #pragma unroll
                             for (int j = 0; j < kG; ++j)
-                                if (j < nvalid) st(o + l0 + j, y[j]);
+                                if (j < nvalid) st(orow + l0 + j, y[j]);
                         }
                     }
                     const int64_t llast = l0 + nvalid - 1;
                     if (p.chunk_states && (((llast + 1) % kStateChunk) == 0 || llast + 1 == L)) {
-                        float *cs = p.chunk_states + ((b * C4 + c[q]) * p.nchunks + llast / kStateChunk) * N;
+                        float *cs = p.chunk_states + ((b * C4 + c) * p.nchunks + llast / kStateChunk) * N;
 #pragma unroll
                         for (int n = 0; n < NS; ++n)
-                            if (n < N) cs[n] = h[q][n];
+                            if (n < N) cs[n] = h[n];
                     }
                 }
-            }
-            if (more) {
-#pragma unroll
-                for (int q = 0; q < SEQ; ++q)
-#pragma unroll
-                    for (int j = 0; j < kG; ++j) {
-                        ucur[q][j] = unx[q][j];
-                        dcur[q][j] = dnx[q][j];
-                    }
             }
         }
         __syncwarp();  // every lane is done with this buffer before it is refilled
     }
 
-    if (PASS == 1) {
+    if (PASS == 1 && active) {
+        float *sg = p.seg + ((b * C4 + c) * (int64_t)p.nseg + sgi) * 2 * N;
 #pragma unroll
-        for (int q = 0; q < SEQ; ++q) {
-            if (!active[q]) continue;
-            float *sg = p.seg + ((b * C4 + c[q]) * (int64_t)p.nseg + sg_i) * 2 * N;
-#pragma unroll
-            for (int n = 0; n < NS; ++n)
-                if (n < N) {
-                    sg[n] = ex2_sfu(A2s[q][n][t].x * dtsum[q]);
-                    sg[N + n] = h[q][n];
-                }
-        }
+        for (int n = 0; n < NS; ++n)
+            if (n < N) {
+                sg[n] = ex2_sfu(A2s[n][t] * dtsum);
+                sg[N + n] = h[n];
+            }
     }
 }
 
@@ -380,22 +358,16 @@ size_t scan_fwd_workspace_bytes(const LaunchShape &s) {
     return (size_t)s.B * kPaths * s.D * nseg * 2 * s.N * sizeof(float);
 }
 
-// sequences per thread (see scan_fwd_kernel)
-#ifndef SS2D_FWD_SEQ
-#define SS2D_FWD_SEQ 1
-#endif
-
 template <int NS, typename Tin, typename Tout, bool IMG, bool VEC>
 static cudaError_t launch_ns(const FwdParams &p, cudaStream_t stream) {
-    constexpr int SEQ = SS2D_FWD_SEQ;
-    dim3 grid((unsigned)ceil_div(p.D, kWarp * SEQ), kPaths, (unsigned)(p.B * p.nseg));
+    dim3 grid((unsigned)ceil_div(p.D, kWarp), kPaths, (unsigned)(p.B * p.nseg));
     if (p.nseg == 1) {
-        scan_fwd_kernel<NS, SEQ, Tin, Tout, IMG, 0, VEC><<<grid, kWarp, 0, stream>>>(p);
+        scan_fwd_kernel<NS, Tin, Tout, IMG, 0, VEC><<<grid, kWarp, 0, stream>>>(p);
         note_launch(stream);
     } else {
-        scan_fwd_kernel<NS, SEQ, Tin, Tout, IMG, 1, VEC><<<grid, kWarp, 0, stream>>>(p);
+        scan_fwd_kernel<NS, Tin, Tout, IMG, 1, VEC><<<grid, kWarp, 0, stream>>>(p);
         note_launch(stream);
-        scan_fwd_kernel<NS, SEQ, Tin, Tout, IMG, 2, VEC><<<grid, kWarp, 0, stream>>>(p);
+        scan_fwd_kernel<NS, Tin, Tout, IMG, 2, VEC><<<grid, kWarp, 0, stream>>>(p);
         note_launch(stream);
     }
     return cudaGetLastError();
