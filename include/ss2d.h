@@ -89,7 +89,7 @@ typedef enum {
 } ss2d_op_t;
 
 /* Chunk length (steps) at which the forward saves scan states for the backward. */
-#define SS2D_CHUNK_LEN 64
+#define SS2D_CHUNK_LEN 16
 
 /* ----------------------------------------------------------------- steps -- */
 

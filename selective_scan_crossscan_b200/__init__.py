@@ -38,7 +38,7 @@ _LIB_PATH = os.environ.get("SS2D_LIBRARY") or os.path.join(_HERE, "libss2d.so")
 _lock = threading.Lock()
 _lib = None
 
-CHUNK_LEN = 64  # SS2D_CHUNK_LEN
+CHUNK_LEN = 16  # SS2D_CHUNK_LEN
 F32, BF16 = 0, 1
 OP_SELECTIVE_SCAN_BWD, OP_FORWARD, OP_BACKWARD = 1, 2, 3
 _STATUS = {0: "SS2D_OK", 1: "SS2D_ERR_NULL", 2: "SS2D_ERR_SHAPE", 3: "SS2D_ERR_DTYPE", 4: "SS2D_ERR_ALIGN",

@@ -106,10 +106,11 @@ static size_t fwd_ws_bytes(const LaunchShape &s, ss2d_dtype_t in) {
     return round64((size_t)s.B * kPaths * s.D * s.L * sizeof(float)) +
            round64((size_t)s.B * s.D * s.L * elem_size(in)) + round64(scan_fwd_workspace_bytes(s));
 }
-// fused backward workspace: [fp32 per-path du (B,4D,L)] [transposed image] [scan backward workspace]
-static size_t bwd_fused_ws_bytes(const LaunchShape &s, ss2d_dtype_t in) {
+// fused backward workspace: [fp32 per-path du (B,4D,L)] [transposed x] [transposed dy] [scan backward workspace]
+static size_t bwd_fused_ws_bytes(const LaunchShape &s, ss2d_dtype_t in, ss2d_dtype_t out) {
     return round64((size_t)s.B * kPaths * s.D * s.L * sizeof(float)) +
-           round64((size_t)s.B * s.D * s.L * elem_size(in)) + round64(scan_bwd_workspace_bytes(s));
+           round64((size_t)s.B * s.D * s.L * elem_size(in)) + round64((size_t)s.B * s.D * s.L * elem_size(out)) +
+           round64(scan_bwd_workspace_bytes(s));
 }
 
 }  // namespace ss2d
@@ -157,7 +158,7 @@ size_t ss2d_workspace_bytes(const ss2d_desc_t *desc, int op) {
     switch (op) {
         case SS2D_OP_SELECTIVE_SCAN_BWD: return scan_bwd_workspace_bytes(s);
         case SS2D_OP_FORWARD: return fwd_ws_bytes(s, desc->in_dtype);
-        case SS2D_OP_BACKWARD: return bwd_fused_ws_bytes(s, desc->in_dtype);
+        case SS2D_OP_BACKWARD: return bwd_fused_ws_bytes(s, desc->in_dtype, desc->out_dtype);
         default: return (size_t)-1;
     }
 }
@@ -327,7 +328,7 @@ ss2d_status_t ss2d_backward(const ss2d_desc_t *desc, const void *x, const void *
     SS2D_TRY(optional(dD));
     SS2D_TRY(optional(ddelta_bias));
     const LaunchShape s = shape_of(desc);
-    const size_t ws = bwd_fused_ws_bytes(s, desc->in_dtype);
+    const size_t ws = bwd_fused_ws_bytes(s, desc->in_dtype, desc->out_dtype);
     if (ws > 0 && (!workspace || workspace_bytes < ws)) return SS2D_ERR_WORKSPACE;
     SS2D_TRY(optional(workspace));
     SS2D_TRY(check_device());
@@ -336,17 +337,19 @@ ss2d_status_t ss2d_backward(const ss2d_desc_t *desc, const void *x, const void *
     w += round64((size_t)s.B * kPaths * s.D * s.L * sizeof(float));
     void *xT = w;
     w += round64((size_t)s.B * s.D * s.L * elem_size(desc->in_dtype));
+    void *dyT = w;
+    w += round64((size_t)s.B * s.D * s.L * elem_size(desc->out_dtype));
     void *inner = w;
     cudaStream_t st = (cudaStream_t)stream;
-    cudaError_t e;
-    if (!chunk_states) {
-        // the chunk states are recomputed by a forward pass that reads the column paths from xT
-        e = launch_transpose(s, desc->in_dtype, x, xT, st);
-        if (e != cudaSuccess) return from_cuda(e);
-    }
+    // the column-major paths read x and dy from transposed copies, so every load is a contiguous row
+    cudaError_t e = launch_transpose(s, desc->in_dtype, x, xT, st);
+    if (e != cudaSuccess) return from_cuda(e);
+    e = launch_transpose(s, desc->out_dtype, dy, dyT, st);
+    if (e != cudaSuccess) return from_cuda(e);
     ScanBwdArgs a;
     a.u = x;
     a.uT = xT;
+    a.doutT = dyT;
     a.delta = delta;
     a.A = A;
     a.Bm = Bm;

@@ -61,6 +61,7 @@ struct ScanBwdArgs {
     const float *bias;
     int softplus;
     const void *dout;          // (B, 4D, L), or (B, D, H, W) image when from_image
+    const void *doutT = nullptr;  // transposed dout image (column paths when from_image)
     const float *chunk_states; // or null
     void *du;                  // (B, 4D, L) in_dtype, or fp32 when from_image (merged afterwards)
     void *ddelta;

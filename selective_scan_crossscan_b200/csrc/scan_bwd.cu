@@ -12,45 +12,57 @@
 //   dB[n,l] += lambda[n] dt_l u_l
 //   du_l     = g_l D + sum_n lambda[n] dt_l B[n,l]
 //   ddelta_l = ddt_l * sigmoid(delta_l + bias)   (softplus) or ddt_l
-// and a_l h_{l-1} = h_l - dt_l B_l u_l, so the terms need h_l, not h_{l-1}.
+// and a_l h_{l-1} = h_l - dt_l B_l u_l, so the adjoint needs h_l, not h_{l-1}.
 //
-// Design: one thread per (b, c) sequence with all N states in registers, as
-// in the forward.  A CTA is one warp: 32 channels of one (b, k).  The
-// sequence is walked backwards in 32-step halves of the forward's 64-step
-// state chunks.  Per half: the states are recomputed forward from the chunk
-// state, keeping a checkpoint every 4 steps in shared memory; then, for each
-// 4-step block from last to first, the block's states are recomputed into
-// registers and the adjoint walks back through them.  dB/dC sum over the
-// channels of the group: each step's 2N contributions are transposed through
-// shared memory and summed by the lanes (fixed order), one CTA partial per
-// (b, k, tile); a second kernel sums the partials over tiles (and dA, dD,
-// ddelta_bias over the batch) in a fixed order -- no float atomics.
+// Design (B200).  Two lanes share one (b, c) sequence, each holding half of
+// the N states in registers, so a warp covers 16 channels of one (b, k) and a
+// CTA of four warps 64 channels.  The sequence is walked backwards in 16-step
+// blocks, each starting from a state the forward saved (chunk states every 16
+// steps):
+//   1. the block's u, delta, dout, B, C are staged in shared memory, and a
+//      pre-pass computes dt, dt*u and d softplus/d delta once per
+//      (channel, step), the two lanes of a channel splitting the steps;
+//   2. the states are recomputed forwards keeping a checkpoint every 4 steps;
+//   3. for each 4-step sub-block, last to first, the states h_l and decays a_l
+//      are recomputed into registers and the adjoint walks back through them
+//      (two exponentials per state update in all).
+// All per-state arithmetic runs on packed state pairs (f32x2).  dB/dC sum over
+// the channels of the group: two steps' contributions of every lane are
+// transposed through shared memory (128-bit stores) and each lane sums one of
+// the 2N outputs over the warp's 16 channels for both steps at once
+// (64-bit loads, packed adds); the four warps' sums are added in a fixed order
+// and written as one partial per (b, k, 64-channel tile); a second kernel sums
+// the partials over tiles, and dA, dD, ddelta_bias over the batch, in a fixed
+// order -- no float atomics, deterministic results.
 #include "common.cuh"
 #include "kernels.h"
 
 namespace ss2d {
 
-constexpr int kBT = 32;    // channels (= threads) per CTA
-constexpr int kBH = 32;    // steps per staged half chunk
-constexpr int kSub = 4;    // steps per register block
-constexpr int kNCk = kBH / kSub;
-constexpr int kChunk = SS2D_CHUNK_LEN;  // 64, the forward's state-chunk length
-static_assert(kChunk == 2 * kBH, "backward walks each state chunk as two halves");
+constexpr int kWarps = 4;                 // warps per CTA
+constexpr int kChPerWarp = 16;            // channels per warp (two lanes each)
+constexpr int kChPerCta = kWarps * kChPerWarp;
+constexpr int kBlk = SS2D_CHUNK_LEN;      // steps per block = forward state-chunk length
+constexpr int kSub = 4;                   // steps per register sub-block
+constexpr int kNSub = kBlk / kSub;
+static_assert(kBlk == 16, "the backward walks 16-step blocks");
 
 struct BwdParams {
-    const void *u;
+    const void *u;      // (B, 4D, L) sequences, or image x (B, D, H, W)
+    const void *uT;     // transposed image (image mode, column paths)
     const void *delta;
     const float *A;
     const void *Bm;
     const void *Cm;
     const float *Dv;
     const float *bias;
-    const void *dout;
-    const float *cs;   // (B, 4D, nchunks, N)
+    const void *dout;   // (B, 4D, L), or image dy (B, D, H, W)
+    const void *doutT;  // transposed dy (image mode, column paths)
+    const float *cs;    // (B, 4D, nchunks, N)
     void *du;
     void *ddelta;
-    float *part_bc;    // (B, 4, ntiles, 2N, L)
-    float *part_p;     // (B, 4D, N + 2): dA (N), dD, ddelta_bias partials
+    float *part_bc;     // (B, 4, ntiles, 2N, L)
+    float *part_p;      // (B, 4D, N + 2): dA (N), dD, ddelta_bias partials
     int64_t B, D, H, W, L;
     int N;
     int softplus;
@@ -59,242 +71,280 @@ struct BwdParams {
 };
 
 template <int NS>
-struct BwdSmem {
-    float us[kBT][kBH + 1];
-    float ds[kBT][kBH + 1];   // delta, overwritten by ddelta
-    float gs[kBT][kBH + 1];   // dout, overwritten by du
-    float Bs[kBH][NS];
-    float Cs[kBH][NS];
-    float ck[kBT][kNCk * NS + 4];     // checkpoints, padded rows
-    float red[kBT][2 * NS + 1];       // per-step transpose for the channel sum
-    float bct[kBH][2 * NS];           // channel sums of the half: [step][dB n | dC n]
+struct BwdWarpSmem {
+    static constexpr int HS = NS / 2;  // states per lane
+    static constexpr int kRow = kBlk + 1;
+    float U[kChPerWarp][kRow];
+    float DT[kChPerWarp][kRow];
+    float DTU[kChPerWarp][kRow];
+    float SG[kChPerWarp][kRow];  // delta, then d softplus / d delta, then ddelta
+    float G[kChPerWarp][kRow];   // dout, then du
+    float Bs[kBlk][NS + 4];      // B[., l] with the states contiguous (16-byte aligned rows)
+    float Cs[kBlk][NS + 4];
+    float ck[32][kNSub][HS];     // per-lane state checkpoints
+    float red[kChPerWarp][4 * NS + 4];  // [channel][output o][2 steps]
+    float bct[kBlk][2 * NS];     // channel sums of this warp: [step][dB n | dC n]
 };
 
 template <int NS, typename Tin, typename Tg, bool IMG>
-__device__ __forceinline__ void stage_half(BwdSmem<NS> &sm, const BwdParams &p, int64_t b, int k, int64_t d0,
-                                           int nch, int64_t l0, int len) {
-    const int t = threadIdx.x;
+__device__ __forceinline__ void stage_block(BwdWarpSmem<NS> &sm, const BwdParams &p, int64_t b, int k,
+                                            int64_t dw0, int nch, int64_t l0, int len) {
+    const int lane = threadIdx.x & 31;
     const int64_t D = p.D, L = p.L, C4 = kPaths * p.D;
-    const Tin *u = static_cast<const Tin *>(p.u);
-    const Tin *delta = static_cast<const Tin *>(p.delta);
-    const Tg *g = static_cast<const Tg *>(p.dout);
-    for (int idx = t; idx < kBT * kBH; idx += kBT) {
-        const int ch = idx / kBH, i = idx % kBH;
+    const bool rev = IMG && k >= 2;
+    for (int idx = lane; idx < kChPerWarp * kBlk; idx += 32) {
+        const int ci = idx / kBlk, i = idx % kBlk;
         float uv = 0.f, dv = 0.f, gv = 0.f;
-        if (ch < nch && i < len) {
+        if (ci < nch && i < len) {
             const int64_t l = l0 + i;
-            const int64_t cc = k * D + d0 + ch;
-            dv = ld(delta + (b * C4 + cc) * L + l);
+            const int64_t cc = k * D + dw0 + ci;
+            dv = ld(static_cast<const Tin *>(p.delta) + (b * C4 + cc) * L + l);
             if (IMG) {
-                const int64_t pix = (b * D + d0 + ch) * L + path_pixel(k, l, p.H, p.W);
-                uv = ld(u + pix);
-                gv = ld(g + pix);
+                const int64_t row = (b * D + dw0 + ci) * L;
+                const int64_t m = rev ? (L - 1 - l) : l;
+                const Tin *ub = static_cast<const Tin *>((k & 1) ? p.uT : p.u);
+                const Tg *gb = static_cast<const Tg *>((k & 1) ? p.doutT : p.dout);
+                uv = ld(ub + row + m);
+                gv = ld(gb + row + m);
             } else {
-                uv = ld(u + (b * C4 + cc) * L + l);
-                gv = ld(g + (b * C4 + cc) * L + l);
+                uv = ld(static_cast<const Tin *>(p.u) + (b * C4 + cc) * L + l);
+                gv = ld(static_cast<const Tg *>(p.dout) + (b * C4 + cc) * L + l);
             }
         }
-        sm.us[ch][i] = uv;
-        sm.ds[ch][i] = dv;
-        sm.gs[ch][i] = gv;
+        sm.U[ci][i] = uv;
+        sm.SG[ci][i] = dv;
+        sm.G[ci][i] = gv;
     }
     const Tin *Bk = static_cast<const Tin *>(p.Bm) + (b * kPaths + k) * p.N * L;
     const Tin *Ck = static_cast<const Tin *>(p.Cm) + (b * kPaths + k) * p.N * L;
-    for (int idx = t; idx < NS * kBH; idx += kBT) {
-        const int n = idx / kBH, i = idx % kBH;
-        float bv = 0.f, cv = 0.f;
-        if (n < p.N && i < len) {
-            bv = ld(Bk + n * L + l0 + i);
-            cv = ld(Ck + n * L + l0 + i);
-        }
-        sm.Bs[i][n] = bv;
-        sm.Cs[i][n] = cv;
+    for (int idx = lane; idx < NS * kBlk; idx += 32) {
+        const int n = idx / kBlk, i = idx % kBlk;
+        const bool ok = n < p.N && i < len;
+        sm.Bs[i][n] = ok ? ld(Bk + (int64_t)n * L + l0 + i) : 0.f;
+        sm.Cs[i][n] = ok ? ld(Ck + (int64_t)n * L + l0 + i) : 0.f;
     }
 }
 
 template <int NS, typename Tin, typename Tg, typename Tdu, bool IMG>
-__global__ void __launch_bounds__(kBT) scan_bwd_kernel(const BwdParams p) {
+__global__ void __launch_bounds__(32 * kWarps) scan_bwd_kernel(const BwdParams p) {
+    constexpr int HS = NS / 2;
+    constexpr int HP = HS / 2;  // state pairs per lane
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    BwdSmem<NS> &sm = *reinterpret_cast<BwdSmem<NS> *>(smem_raw);
+    BwdWarpSmem<NS> *wsm = reinterpret_cast<BwdWarpSmem<NS> *>(smem_raw);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    BwdWarpSmem<NS> &sm = wsm[warp];
 
-    const int t = threadIdx.x;
+    const int ci = lane >> 1, hf = lane & 1;  // channel within the warp, state half
     const int k = blockIdx.y;
     const int64_t b = blockIdx.z;
     const int64_t D = p.D, L = p.L, C4 = kPaths * p.D;
-    const int64_t d0 = (int64_t)blockIdx.x * kBT;
-    const int nch = (int)min((int64_t)kBT, D - d0);
-    const bool active = t < nch;
-    const int64_t c = k * D + d0 + t;
+    const int64_t dc0 = (int64_t)blockIdx.x * kChPerCta;  // first channel of the CTA
+    const int64_t dw0 = dc0 + warp * kChPerWarp;           // first channel of this warp
+    const int nch = (int)max((int64_t)0, min((int64_t)kChPerWarp, D - dw0));
+    const bool active = ci < nch;
+    const int64_t c = k * D + (active ? dw0 + ci : 0);
     const int N = p.N;
+    const int n0 = hf * HS;  // first state of this lane
 
-    float A2[NS], lam[NS], dA[NS];
+    float2 A2[HP], Aln[HP], lam[HP], dA[HP];
 #pragma unroll
-    for (int n = 0; n < NS; ++n) {
-        A2[n] = (active && n < N) ? p.A[c * N + n] * kLog2e : 0.f;
-        lam[n] = 0.f;
-        dA[n] = 0.f;
+    for (int q = 0; q < HP; ++q) {
+        const int na = n0 + 2 * q, nb = na + 1;
+        const float aa = (active && na < N) ? p.A[c * N + na] : 0.f;
+        const float ab = (active && nb < N) ? p.A[c * N + nb] : 0.f;
+        A2[q] = make_float2(aa * kLog2e, ab * kLog2e);
+        Aln[q] = make_float2(aa, ab);
+        lam[q] = make_float2(0.f, 0.f);
+        dA[q] = make_float2(0.f, 0.f);
     }
-    const float An_scale = kLn2;  // A = A2 * ln2
     const float Dc = (active && p.Dv) ? p.Dv[c] : 0.f;
     const float bias = (active && p.bias) ? p.bias[c] : 0.f;
     float dD = 0.f, dbias = 0.f;
 
     Tdu *du_out = static_cast<Tdu *>(p.du);
     Tin *dd_out = static_cast<Tin *>(p.ddelta);
-    float *pbc = p.part_bc + ((b * kPaths + k) * p.ntiles + blockIdx.x) * (int64_t)(2 * N) * L;
+    const int nblk = (int)ceil_div(L, kBlk);
 
-    for (int64_t J = p.nchunks - 1; J >= 0; --J) {
-        const int64_t cbeg = J * kChunk;
-        const int clen = (int)min((int64_t)kChunk, L - cbeg);
-        float hJ[NS];
+    for (int blk = nblk - 1; blk >= 0; --blk) {
+        const int64_t l0 = (int64_t)blk * kBlk;
+        const int len = (int)min((int64_t)kBlk, L - l0);
+        __syncwarp();
+        stage_block<NS, Tin, Tg, IMG>(sm, p, b, k, dw0, nch, l0, len);
+        __syncwarp();
+        // pre-pass: dt, dt*u, d softplus / d delta for each (channel, step), lanes hf split the steps
+        for (int i = hf * (kBlk / 2); i < (hf + 1) * (kBlk / 2); ++i) {
+            const float tt = sm.SG[ci][i] + bias;
+            float dt, sg;
+            if (p.softplus) {
+                const float z = ex2_sfu(-fabsf(tt) * kLog2e);  // e^{-|t|}
+                dt = softplus_f(tt);
+                const float r = __frcp_rn(1.f + z);
+                sg = tt >= 0.f ? r : z * r;  // sigmoid(t)
+            } else {
+                dt = tt;
+                sg = 1.f;
+            }
+            if (i >= len) dt = 0.f;  // past the end: decay 1, no input
+            sm.DT[ci][i] = dt;
+            sm.DTU[ci][i] = dt * sm.U[ci][i];
+            sm.SG[ci][i] = sg;
+        }
+        __syncwarp();
+
+        // level 1: checkpoint every kSub steps, from the state the forward saved before this block
         {
-            const float *src = (J > 0 && active) ? p.cs + ((b * C4 + c) * p.nchunks + (J - 1)) * N : nullptr;
+            float2 h[HP];
+            const float *src = (blk > 0 && active) ? p.cs + ((b * C4 + c) * p.nchunks + (blk - 1)) * N : nullptr;
 #pragma unroll
-            for (int n = 0; n < NS; ++n) hJ[n] = (src && n < N) ? src[n] : 0.f;
-        }
-        const int nhalf = clen > kBH ? 2 : 1;
-        float hmid[NS];
-        if (nhalf == 2) {
-            // state after the first half: run it forward once
-            __syncthreads();
-            stage_half<NS, Tin, Tg, IMG>(sm, p, b, k, d0, nch, cbeg, kBH);
-            __syncthreads();
-#pragma unroll
-            for (int n = 0; n < NS; ++n) hmid[n] = hJ[n];
-            if (active) {
-                for (int i = 0; i < kBH; ++i) {
-                    const float tt = sm.ds[t][i] + bias;
-                    const float dt = p.softplus ? softplus_f(tt) : tt;
-                    const float dtu = dt * sm.us[t][i];
-#pragma unroll
-                    for (int n = 0; n < NS; ++n)
-                        hmid[n] = fmaf(ex2_sfu(dt * A2[n]), hmid[n], dtu * sm.Bs[i][n]);
-                }
+            for (int q = 0; q < HP; ++q) {
+                const int na = n0 + 2 * q;
+                h[q] = make_float2((src && na < N) ? src[na] : 0.f, (src && na + 1 < N) ? src[na + 1] : 0.f);
             }
-        }
-        for (int half = nhalf - 1; half >= 0; --half) {
-            const int64_t l0 = cbeg + half * kBH;
-            const int len = (int)min((int64_t)kBH, L - l0);
-            __syncthreads();
-            stage_half<NS, Tin, Tg, IMG>(sm, p, b, k, d0, nch, l0, len);
-            __syncthreads();
-            const int nsub = (len + kSub - 1) / kSub;
-
-            // level 1: checkpoints every kSub steps
-            if (active) {
-                float h[NS];
+            for (int s = 0; s < kNSub; ++s) {
 #pragma unroll
-                for (int n = 0; n < NS; ++n) h[n] = (half == 1) ? hmid[n] : hJ[n];
-                for (int q = 0; q < nsub; ++q) {
+                for (int q = 0; q < HP; ++q) *reinterpret_cast<float2 *>(&sm.ck[lane][s][2 * q]) = h[q];
+                for (int i = s * kSub; i < s * kSub + kSub && i < len; ++i) {
+                    const float dt = sm.DT[ci][i], dtu = sm.DTU[ci][i];
 #pragma unroll
-                    for (int n = 0; n < NS; ++n) sm.ck[t][q * NS + n] = h[n];
-                    for (int i = q * kSub; i < min(len, q * kSub + kSub); ++i) {
-                        const float tt = sm.ds[t][i] + bias;
-                        const float dt = p.softplus ? softplus_f(tt) : tt;
-                        const float dtu = dt * sm.us[t][i];
-#pragma unroll
-                        for (int n = 0; n < NS; ++n) h[n] = fmaf(ex2_sfu(dt * A2[n]), h[n], dtu * sm.Bs[i][n]);
+                    for (int q = 0; q < HP; ++q) {
+                        const float2 bb = *reinterpret_cast<const float2 *>(&sm.Bs[i][n0 + 2 * q]);
+                        const float2 x = __fmul2_rn(make_float2(dt, dt), A2[q]);
+                        const float2 a = make_float2(ex2_sfu(x.x), ex2_sfu(x.y));
+                        h[q] = __ffma2_rn(a, h[q], __fmul2_rn(make_float2(dtu, dtu), bb));
                     }
                 }
             }
+        }
 
-            // level 2 + adjoint walk, 4-step blocks from last to first
-            for (int q = nsub - 1; q >= 0; --q) {
-                const int i0 = q * kSub;
-                const int cnt = min(kSub, len - i0);
-                float hist[kSub][NS];
-                if (active) {
-                    float h[NS];
+        // level 2 + adjoint walk, 4-step sub-blocks from last to first
+        const int nsub = (len + kSub - 1) / kSub;
+        for (int s = nsub - 1; s >= 0; --s) {
+            const int i0 = s * kSub;
+            const int cnt = min(kSub, len - i0);
+            float2 hist[kSub][HP], dec[kSub][HP];
+            {
+                float2 h[HP];
 #pragma unroll
-                    for (int n = 0; n < NS; ++n) h[n] = sm.ck[t][q * NS + n];
+                for (int q = 0; q < HP; ++q) h[q] = *reinterpret_cast<const float2 *>(&sm.ck[lane][s][2 * q]);
 #pragma unroll
-                    for (int j = 0; j < kSub; ++j) {
-                        if (j < cnt) {
-                            const int i = i0 + j;
-                            const float tt = sm.ds[t][i] + bias;
-                            const float dt = p.softplus ? softplus_f(tt) : tt;
-                            const float dtu = dt * sm.us[t][i];
+                for (int j = 0; j < kSub; ++j) {
+                    const int i = i0 + j;  // steps past the end have dt = 0: decay 1, no input
+                    const float dt = sm.DT[ci][i], dtu = sm.DTU[ci][i];
 #pragma unroll
-                            for (int n = 0; n < NS; ++n) {
-                                // the same rounded dt*u*B as the adjoint subtracts below
-                                h[n] = fmaf(ex2_sfu(dt * A2[n]), h[n], __fmul_rn(dtu, sm.Bs[i][n]));
-                                hist[j][n] = h[n];
-                            }
+                    for (int q = 0; q < HP; ++q) {
+                        const float2 bb = *reinterpret_cast<const float2 *>(&sm.Bs[i][n0 + 2 * q]);
+                        const float2 x = __fmul2_rn(make_float2(dt, dt), A2[q]);
+                        dec[j][q] = make_float2(ex2_sfu(x.x), ex2_sfu(x.y));
+                        h[q] = __ffma2_rn(dec[j][q], h[q], __fmul2_rn(make_float2(dtu, dtu), bb));
+                        hist[j][q] = h[q];
+                    }
+                }
+            }
+            // the adjoint, two steps at a time (jp, jp-1)
+            for (int jp = cnt - 1; jp >= 0; jp -= 2) {
+                float2 vb[2][HP], vc[2][HP];  // dB, dC contributions of the two steps
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int j = jp - e;
+#pragma unroll
+                    for (int q = 0; q < HP; ++q) {
+                        vb[e][q] = make_float2(0.f, 0.f);
+                        vc[e][q] = make_float2(0.f, 0.f);
+                    }
+                    if (j < 0) continue;
+#pragma unroll
+                    for (int jj = 0; jj < kSub; ++jj) {
+                        if (jj != j) continue;  // registers need compile-time indices
+                        const int i = i0 + jj;
+                        const float g = sm.G[ci][i], dt = sm.DT[ci][i], dtu = sm.DTU[ci][i];
+                        const float uv = sm.U[ci][i];
+                        float2 ddt2 = make_float2(0.f, 0.f), du2 = make_float2(0.f, 0.f);
+#pragma unroll
+                        for (int q = 0; q < HP; ++q) {
+                            const float2 bb = *reinterpret_cast<const float2 *>(&sm.Bs[i][n0 + 2 * q]);
+                            const float2 cc = *reinterpret_cast<const float2 *>(&sm.Cs[i][n0 + 2 * q]);
+                            lam[q] = __ffma2_rn(cc, make_float2(g, g), lam[q]);
+                            const float2 bt = __fmul2_rn(make_float2(dtu, dtu), bb);  // as in the recompute
+                            const float2 ah = __ffma2_rn(bt, make_float2(-1.f, -1.f), hist[jj][q]);  // a_l h_{l-1}
+                            const float2 inner = __ffma2_rn(Aln[q], ah, __fmul2_rn(make_float2(uv, uv), bb));
+                            ddt2 = __ffma2_rn(lam[q], inner, ddt2);
+                            const float2 ldt = __fmul2_rn(lam[q], make_float2(dt, dt));
+                            dA[q] = __ffma2_rn(ldt, ah, dA[q]);
+                            du2 = __ffma2_rn(ldt, bb, du2);
+                            vb[e][q] = __fmul2_rn(lam[q], make_float2(dtu, dtu));
+                            vc[e][q] = __fmul2_rn(make_float2(g, g), hist[jj][q]);
+                            lam[q] = __fmul2_rn(lam[q], dec[jj][q]);
+                        }
+                        float ddt = ddt2.x + ddt2.y, dul = du2.x + du2.y;
+                        ddt += __shfl_xor_sync(0xffffffffu, ddt, 1);  // the other half of the states
+                        dul += __shfl_xor_sync(0xffffffffu, dul, 1);
+                        if (hf == 0 && active) {
+                            const float dd = ddt * sm.SG[ci][i];
+                            dbias += dd;
+                            dD = fmaf(g, uv, dD);
+                            sm.SG[ci][i] = dd;
+                            sm.G[ci][i] = fmaf(g, Dc, dul);
                         }
                     }
                 }
+                // transpose the two steps' contributions: red[ci][o][e], o = state (dB) or NS + state (dC)
 #pragma unroll
-                for (int j = kSub - 1; j >= 0; --j) {
-                    if (j >= cnt) continue;  // uniform across the warp
-                    const int i = i0 + j;
-                    float ddt = 0.f;
-                    if (active) {
-                        const float uv = sm.us[t][i];
-                        const float g = sm.gs[t][i];
-                        const float tt = sm.ds[t][i] + bias;
-                        const float dt = p.softplus ? softplus_f(tt) : tt;
-                        const float dtu = dt * uv;
-                        float dul = g * Dc;
-                        dD = fmaf(g, uv, dD);
-#pragma unroll
-                        for (int n = 0; n < NS; ++n) {
-                            const float Bn = sm.Bs[i][n];
-                            const float Cn = sm.Cs[i][n];
-                            const float a = ex2_sfu(dt * A2[n]);
-                            lam[n] = fmaf(Cn, g, lam[n]);
-                            // a_l * h_{l-1}, exactly 0 when h_{l-1} = 0
-                            const float ah = __fsub_rn(hist[j][n], __fmul_rn(dtu, Bn));
-                            ddt = fmaf(lam[n], fmaf(A2[n] * An_scale, ah, Bn * uv), ddt);
-                            dA[n] = fmaf(lam[n] * dt, ah, dA[n]);
-                            dul = fmaf(lam[n] * dt, Bn, dul);
-                            sm.red[t][n] = lam[n] * dtu;          // dB contribution
-                            sm.red[t][NS + n] = g * hist[j][n];    // dC contribution
-                            lam[n] *= a;
-                        }
-                        const float dd = p.softplus ? ddt * sigmoid_f(tt) : ddt;
-                        dbias += dd;
-                        sm.ds[t][i] = dd;
-                        sm.gs[t][i] = dul;
-                    } else {
-#pragma unroll
-                        for (int n = 0; n < 2 * NS; ++n) sm.red[t][n] = 0.f;
-                    }
-                    __syncwarp();
-                    // lane v < 2N sums contribution v over the 32 channels, in lane order
-                    if (t < 2 * NS) {
-                        float s = 0.f;
-#pragma unroll 8
-                        for (int r = 0; r < kBT; ++r) s += sm.red[r][t];
-                        sm.bct[i][t] = s;
-                    }
-                    __syncwarp();
+                for (int q = 0; q < HP; ++q) {
+                    const int o = n0 + 2 * q;
+                    *reinterpret_cast<float4 *>(&sm.red[ci][2 * o]) =
+                        make_float4(vb[0][q].x, vb[1][q].x, vb[0][q].y, vb[1][q].y);
+                    *reinterpret_cast<float4 *>(&sm.red[ci][2 * (NS + o)]) =
+                        make_float4(vc[0][q].x, vc[1][q].x, vc[0][q].y, vc[1][q].y);
                 }
-            }
-            __syncthreads();
-            // write du, ddelta and the dB/dC partial of this half
-            for (int idx = t; idx < kBT * kBH; idx += kBT) {
-                const int ch = idx / kBH, i = idx % kBH;
-                if (ch < nch && i < len) {
-                    const int64_t cc = k * D + d0 + ch;
-                    st(du_out + (b * C4 + cc) * L + l0 + i, sm.gs[ch][i]);
-                    st(dd_out + (b * C4 + cc) * L + l0 + i, sm.ds[ch][i]);
+                __syncwarp();
+                if (lane < 2 * NS) {  // lane = output o: sum over the warp's channels, both steps at once
+                    float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+                    for (int r = 0; r < kChPerWarp; ++r)
+                        acc = __fadd2_rn(acc, *reinterpret_cast<const float2 *>(&sm.red[r][2 * lane]));
+                    sm.bct[i0 + jp][lane] = acc.x;
+                    if (jp - 1 >= 0) sm.bct[i0 + jp - 1][lane] = acc.y;
                 }
-            }
-            for (int idx = t; idx < 2 * N * kBH; idx += kBT) {
-                const int v = idx / kBH, i = idx % kBH;
-                const int col = v < N ? v : NS + (v - N);
-                if (i < len) pbc[(int64_t)v * L + l0 + i] = sm.bct[i][col];
+                __syncwarp();
             }
         }
+        __syncthreads();  // all four warps' channel sums of this block are in shared memory
+
+        // outputs of the block: du, ddelta of each warp's channels; dB/dC partial of the CTA
+        for (int idx = lane; idx < kChPerWarp * kBlk; idx += 32) {
+            const int cw = idx / kBlk, i = idx % kBlk;
+            if (cw < nch && i < len) {
+                const int64_t cc = k * D + dw0 + cw;
+                st(du_out + (b * C4 + cc) * L + l0 + i, sm.G[cw][i]);
+                st(dd_out + (b * C4 + cc) * L + l0 + i, sm.SG[cw][i]);
+            }
+        }
+        float *pbc = p.part_bc + ((b * kPaths + k) * p.ntiles + blockIdx.x) * (int64_t)(2 * N) * L;
+        for (int idx = threadIdx.x; idx < 2 * N * kBlk; idx += 32 * kWarps) {
+            const int v = idx / kBlk, i = idx % kBlk;
+            const int col = v < N ? v : NS + (v - N);
+            if (i < len) {
+                float s = 0.f;
+#pragma unroll
+                for (int w = 0; w < kWarps; ++w) s += wsm[w].bct[i][col];
+                pbc[(int64_t)v * L + l0 + i] = s;
+            }
+        }
+        __syncthreads();  // bct is rewritten by the next block
     }
 
     if (active) {
         float *pp = p.part_p + (b * C4 + c) * (N + 2);
 #pragma unroll
-        for (int n = 0; n < NS; ++n)
-            if (n < N) pp[n] = dA[n];
-        pp[N] = dD;
-        pp[N + 1] = dbias;
+        for (int q = 0; q < HP; ++q) {
+            const int na = n0 + 2 * q;
+            if (na < N) pp[na] = dA[q].x;
+            if (na + 1 < N) pp[na + 1] = dA[q].y;
+        }
+        if (hf == 0) {
+            pp[N] = dD;
+            pp[N + 1] = dbias;
+        }
     }
 }
 
@@ -336,10 +386,10 @@ __global__ void bwd_reduce_params_kernel(const float *__restrict__ part_p, float
 
 // ---------------------------------------------------------------- launch --
 
-static int bwd_tiles(const LaunchShape &s) { return (int)ceil_div(s.D, kBT); }
+static int bwd_tiles(const LaunchShape &s) { return (int)ceil_div(s.D, kChPerCta); }
 
 size_t scan_bwd_workspace_bytes(const LaunchShape &s) {
-    const size_t nchunks = (size_t)ceil_div(s.L, kChunk);
+    const size_t nchunks = (size_t)ceil_div(s.L, kBlk);
     size_t bytes = 0;
     auto add = [&](size_t n) { bytes += (n + 63) / 64 * 64; };
     add((size_t)s.B * kPaths * bwd_tiles(s) * 2 * s.N * s.L * sizeof(float));  // part_bc
@@ -351,12 +401,12 @@ size_t scan_bwd_workspace_bytes(const LaunchShape &s) {
 
 template <int NS, typename Tin, typename Tg, typename Tdu, bool IMG>
 static cudaError_t launch_bwd_t(const LaunchShape &s, const BwdParams &p, cudaStream_t stream) {
-    const size_t smem = sizeof(BwdSmem<NS>);
+    const size_t smem = sizeof(BwdWarpSmem<NS>) * kWarps;
     auto kern = scan_bwd_kernel<NS, Tin, Tg, Tdu, IMG>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)bwd_tiles(s), kPaths, (unsigned)s.B);
-    kern<<<grid, kBT, smem, stream>>>(p);
+    kern<<<grid, 32 * kWarps, smem, stream>>>(p);
     note_launch(stream);
     return cudaGetLastError();
 }
@@ -387,7 +437,7 @@ static cudaError_t launch_bwd_types(const LaunchShape &s, const BwdParams &p, ss
 cudaError_t launch_scan_bwd(const LaunchShape &s, const ScanBwdArgs &a, void *workspace, size_t ws_bytes,
                             cudaStream_t stream) {
     (void)ws_bytes;
-    const int64_t nchunks = ceil_div(s.L, kChunk);
+    const int64_t nchunks = ceil_div(s.L, kBlk);
     unsigned char *ws = static_cast<unsigned char *>(workspace);
     size_t off = 0;
     auto take = [&](size_t n) {
@@ -426,6 +476,7 @@ cudaError_t launch_scan_bwd(const LaunchShape &s, const ScanBwdArgs &a, void *wo
 
     BwdParams p;
     p.u = a.u;
+    p.uT = a.uT;
     p.delta = a.delta;
     p.A = a.A;
     p.Bm = a.Bm;
@@ -433,6 +484,7 @@ cudaError_t launch_scan_bwd(const LaunchShape &s, const ScanBwdArgs &a, void *wo
     p.Dv = a.Dv;
     p.bias = a.bias;
     p.dout = a.dout;
+    p.doutT = a.doutT;
     p.cs = cs;
     p.du = a.du;
     p.ddelta = a.ddelta;

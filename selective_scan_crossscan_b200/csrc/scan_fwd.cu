@@ -43,6 +43,11 @@ constexpr int kStateChunk = SS2D_CHUNK_LEN;
 #ifndef SS2D_FWD_MIN_BLOCKS
 #define SS2D_FWD_MIN_BLOCKS 16
 #endif
+// 1: A*log2(e) per (lane, state) lives in shared memory (fewer registers);
+// 0: in registers (fewer shared-memory loads)
+#ifndef SS2D_FWD_A2_SMEM
+#define SS2D_FWD_A2_SMEM 1
+#endif
 
 struct FwdParams {
     const void *u;       // (B, 4D, L) sequences, or image x (B, D, H, W)
@@ -141,7 +146,13 @@ __device__ __forceinline__ void stage_chunk(FwdStage<Tin, NS> &st, const Tin *Bk
 template <int NS, typename Tin, typename Tout, bool IMG, int PASS, bool VEC>
 __global__ void __launch_bounds__(kWarp, SS2D_FWD_MIN_BLOCKS) scan_fwd_kernel(const FwdParams p) {
     __shared__ __align__(16) FwdStage<Tin, NS> stage[2];
+#if SS2D_FWD_A2_SMEM
     __shared__ float A2s[NS][kWarp];  // A[c, n] * log2(e) of each lane's channel (kept out of registers)
+#define SS2D_A2(n) A2s[n][t]
+#else
+    float A2r[NS];
+#define SS2D_A2(n) A2r[n]
+#endif
 
     const int t = threadIdx.x;
     const int k = blockIdx.y;
@@ -158,7 +169,7 @@ __global__ void __launch_bounds__(kWarp, SS2D_FWD_MIN_BLOCKS) scan_fwd_kernel(co
     float h[NS];
 #pragma unroll
     for (int n = 0; n < NS; ++n) {
-        A2s[n][t] = (active && n < N) ? p.A[c * N + n] * kLog2e : 0.f;
+        SS2D_A2(n) = (active && n < N) ? p.A[c * N + n] * kLog2e : 0.f;
         h[n] = 0.f;
     }
     const float Dc = (active && p.Dv) ? p.Dv[c] : 0.f;
@@ -265,7 +276,7 @@ __global__ void __launch_bounds__(kWarp, SS2D_FWD_MIN_BLOCKS) scan_fwd_kernel(co
                 float2 y23 = __fmul2_rn(make_float2(Dc, Dc), u23);
 #pragma unroll
                 for (int n = 0; n < NS; ++n) {
-                    const float a2s = A2s[n][t];
+                    const float a2s = SS2D_A2(n);
                     const float2 a2 = make_float2(a2s, a2s);
                     float bq[kG], cq[kG];
                     if (VEC) {
@@ -320,11 +331,13 @@ __global__ void __launch_bounds__(kWarp, SS2D_FWD_MIN_BLOCKS) scan_fwd_kernel(co
 #pragma unroll
         for (int n = 0; n < NS; ++n)
             if (n < N) {
-                sg[n] = ex2_sfu(A2s[n][t] * dtsum);
+                sg[n] = ex2_sfu(SS2D_A2(n) * dtsum);
                 sg[N + n] = h[n];
             }
     }
 }
+
+#undef SS2D_A2
 
 // Segment plan: how many segments each sequence is cut into, and their length
 // (a multiple of the state-chunk length).  One segment means a single pass.

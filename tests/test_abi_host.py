@@ -103,9 +103,9 @@ def test_valid_call_without_gpu_reports_device_error(lib):
 
 
 def test_workspace_and_chunk_state_sizes(lib):
-    # chunk states: B * 4D * ceil(L / 64) * N fp32
-    assert lib.ss2d_chunk_states_elems(_d(B=2, D=3, H=5, W=13, N=7)) == 2 * 12 * 2 * 7
-    assert lib.ss2d_chunk_states_elems(_d(B=1, D=8, H=8, W=8, N=4)) == 32 * 1 * 4
+    # chunk states: B * 4D * ceil(L / 16) * N fp32
+    assert lib.ss2d_chunk_states_elems(_d(B=2, D=3, H=5, W=13, N=7)) == 2 * 12 * 5 * 7
+    assert lib.ss2d_chunk_states_elems(_d(B=1, D=8, H=8, W=8, N=4)) == 32 * 4 * 4
     # the fused forward keeps one fp32 value per sequence step
     assert lib.ss2d_workspace_bytes(_d(B=2, D=3, H=5, W=13, N=7), ss.OP_FORWARD) >= 2 * 12 * 65 * 4
     assert lib.ss2d_workspace_bytes(_d(), 99) == ctypes.c_size_t(-1).value

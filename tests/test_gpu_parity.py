@@ -148,13 +148,13 @@ def test_selective_scan_fwd_optional_inputs(opts):
 
 
 def test_selective_scan_fwd_chunk_states():
-    # chunk j holds h after step min(64 (j+1), L) - 1: the oracle's last state on the truncated sequence
-    w, inp = _scan_case(1, 4, 10, 20, 16, seed=6)  # L = 200 -> 4 chunks, ragged last one
+    # chunk j holds h after step min(16 (j+1), L) - 1: the oracle's last state on the truncated sequence
+    w, inp = _scan_case(1, 4, 10, 20, 16, seed=6)  # L = 200 -> 13 chunks, ragged last one
     d = _dev(inp)
     y, cs = ss.selective_scan_fwd(d["u"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["delta_bias"], True,
                                   return_chunk_states=True)
-    assert cs.shape == (1, 16, 4, 16)
-    for j, end in enumerate([64, 128, 192, 200]):
+    assert cs.shape == (1, 16, 13, 16)
+    for j, end in [(0, 16), (5, 96), (11, 192), (12, 200)]:
         _, last = oracle.selective_scan_fwd(inp["u"][..., :end], inp["delta"][..., :end], inp["A"],
                                             inp["B"][..., :end], inp["C"][..., :end], inp["D"], inp["delta_bias"],
                                             True, return_last_state=True)
@@ -251,14 +251,21 @@ def test_ss2d_forward_bf16():
     assert_rel_l2(y, ref, BF16_TOL)
 
 
-def test_unfused_pipeline_equals_fused():
-    w = ss2d_inputs.custom(2, 8, 7, 9, 16)
+@pytest.mark.parametrize("H,W", [(4, 8), (7, 9)])
+def test_unfused_pipeline_equals_fused(H, W):
+    # single pass on both sides (L <= 32): bit-identical; longer sequences of a small problem are
+    # split into segments by the fused forward, whose carries round differently: within 1e-5
+    w = ss2d_inputs.custom(2, 8, H, W, 16)
+    L = H * W
     d = _dev(ss2d_inputs.make_inputs(w, seed=12))
     y = ss.ss2d_forward(d["x"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["delta_bias"], True)
-    xs = ss.cross_scan(d["x"]).reshape(2, 32, 63)
+    xs = ss.cross_scan(d["x"]).reshape(2, 32, L)
     ys = ss.selective_scan_fwd(xs, d["delta"], d["A"], d["B"], d["C"], d["D"], d["delta_bias"], True)
-    y2 = ss.cross_merge(ys.reshape(2, 4, 8, 63), 7, 9)
-    assert torch.equal(y, y2)
+    y2 = ss.cross_merge(ys.reshape(2, 4, 8, L), H, W)
+    if L <= 32:
+        assert torch.equal(y, y2)
+    else:
+        torch.testing.assert_close(y, y2, rtol=1e-5, atol=1e-5)
 
 
 def test_forward_is_deterministic():
