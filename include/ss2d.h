@@ -191,6 +191,33 @@ SS2D_API ss2d_status_t ss2d_backward(const ss2d_desc_t *desc, const void *x, con
                             void *dBm, void *dCm, float *dD, float *ddelta_bias,
                             void *workspace, size_t workspace_bytes, ss2d_stream_t stream);
 
+/*
+ * S6 selective scan forward that allocates nothing and takes no workspace.
+ * The pages have no counterpart: this is an addition of this library.
+ *
+ * Some callers cannot allocate device memory when they call: a serving loop
+ * whose memory plan is fixed at start-up, or a host program that links only
+ * this C library and has no device allocator to provide a workspace.  Arguments,
+ * layouts and results are those of ss2d_selective_scan_fwd; unlike it, when a
+ * problem has too few sequences to fill the GPU (fewer than ~76k), the scan
+ * splits every sequence into up to 32 segments, keeping the per-segment
+ * summaries (B * 4D * segments * 2N fp32) in a 16 MiB static device buffer
+ * inside the library.
+ *  - A problem whose summaries exceed 16 MiB returns SS2D_ERR_SHAPE before any
+ *    launch (ss2d_last_cuda_error() says how many bytes it needed).
+ *  - Every GPU that loads the library holds the 16 MiB buffer until exit.
+ *  - The first call on each device looks up the buffer's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture on the device.
+ *  - All calls on a device share the buffer: calls that can overlap on the GPU
+ *    (other streams, unordered host threads) race and give wrong results.  Each
+ *    call writes every entry before reading it, so nothing needs clearing.
+ */
+SS2D_API ss2d_status_t ss2d_selective_scan_fwd_noalloc(const ss2d_desc_t *desc, const void *u, const void *delta,
+                                                       const float *A, const void *Bm, const void *Cm,
+                                                       const float *D, const float *delta_bias, int delta_softplus,
+                                                       void *out, float *chunk_states, ss2d_stream_t stream);
+
 /* ------------------------------------------------------------- helpers -- */
 
 /* Bytes of workspace an operation needs for this problem (0 if none).

@@ -1,6 +1,7 @@
 // api.cu -- the C ABI of libss2d (declared in include/ss2d.h): argument
 // validation on the host, workspace layout, and dispatch to the kernels.
 #include <atomic>
+#include <cstdarg>
 #include <cstdio>
 #include <cstring>
 
@@ -375,3 +376,29 @@ ss2d_status_t ss2d_backward(const ss2d_desc_t *desc, const void *x, const void *
 }
 
 }  // extern "C"
+
+namespace ss2d {
+
+// the argument checks of ss2d_selective_scan_fwd, for entry points defined elsewhere
+ss2d_status_t check_scan_fwd_args(const ss2d_desc_t *desc, const void *u, const void *delta, const float *A,
+                                  const void *Bm, const void *Cm, const float *D, const float *delta_bias,
+                                  const void *out, const float *chunk_states) {
+    SS2D_TRY(check_desc(desc));
+    SS2D_TRY(check_scan_inputs(u, delta, A, Bm, Cm, D, delta_bias));
+    SS2D_TRY(need(out));
+    SS2D_TRY(optional(chunk_states));
+    return SS2D_OK;
+}
+
+ss2d_status_t device_usable() { return check_device(); }
+
+ss2d_status_t status_from_cuda(cudaError_t e) { return from_cuda(e); }
+
+void set_error_message(const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    std::vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+    va_end(ap);
+}
+
+}  // namespace ss2d

@@ -75,6 +75,14 @@ struct ScanBwdArgs {
 };
 
 size_t scan_bwd_workspace_bytes(const LaunchShape &s);
+
+// Helpers of the C-ABI layer (api.cu) for entry points defined in other files.
+ss2d_status_t check_scan_fwd_args(const ss2d_desc_t *desc, const void *u, const void *delta, const float *A,
+                                  const void *Bm, const void *Cm, const float *D, const float *delta_bias,
+                                  const void *out, const float *chunk_states);
+ss2d_status_t device_usable();
+ss2d_status_t status_from_cuda(cudaError_t e);
+void set_error_message(const char *fmt, ...);
 cudaError_t launch_scan_bwd(const LaunchShape &s, const ScanBwdArgs &a, void *workspace, size_t ws_bytes,
                             cudaStream_t stream);
 
