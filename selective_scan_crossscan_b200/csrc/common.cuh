@@ -133,6 +133,38 @@ __device__ __forceinline__ float2 softplus_f2(float2 t) {
     return __ffma2_rn(z, q, make_float2(fmaxf(t.x, 0.f), fmaxf(t.y, 0.f)));
 }
 
+// 2^x for two values on the FMA pipe (packed f32x2), to take exponentials off the
+// SFU: Cody-Waite split x = j + f with j = rint(x) (magic-number rounding) and
+// f in [-1/2, 1/2], 2^f by a degree-5 polynomial fitted to 2^f on [-1/2, 1/2]
+// (Chebyshev least squares weighted for relative error; maximum relative error
+// 2.2e-7 in fp32, about that of the SFU's approximation), then j added to the
+// exponent field.  Arguments are clamped below at -125 (results under 2^-125
+// are returned as ~2^-125 instead of flushing to zero: both are negligible
+// against O(1) terms).
+constexpr float kEx2C0 = 1.0000001192092896f;
+constexpr float kEx2C1 = 0.6931469440460205f;
+constexpr float kEx2C2 = 0.24022121727466583f;
+constexpr float kEx2C3 = 0.05550742521882057f;
+constexpr float kEx2C4 = 0.009675459936261177f;
+constexpr float kEx2C5 = 0.0013266970636323094f;
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
+
+__device__ __forceinline__ float2 ex2_poly2(float2 x) {
+    x = make_float2(fmaxf(x.x, -125.f), fmaxf(x.y, -125.f));
+    const float2 t = __fadd2_rn(x, make_float2(kRoundMagic, kRoundMagic));      // low bits hold rint(x)
+    const float2 j = __fadd2_rn(t, make_float2(-kRoundMagic, -kRoundMagic));    // rint(x) as a float
+    const float2 f = __ffma2_rn(j, make_float2(-1.f, -1.f), x);                  // x - rint(x), exact
+    float2 q = make_float2(kEx2C5, kEx2C5);
+    q = __ffma2_rn(q, f, make_float2(kEx2C4, kEx2C4));
+    q = __ffma2_rn(q, f, make_float2(kEx2C3, kEx2C3));
+    q = __ffma2_rn(q, f, make_float2(kEx2C2, kEx2C2));
+    q = __ffma2_rn(q, f, make_float2(kEx2C1, kEx2C1));
+    q = __ffma2_rn(q, f, make_float2(kEx2C0, kEx2C0));
+    // t's bit pattern is 0x4B400000 + rint(x); shifted by 23 only rint(x) lands in the exponent field
+    return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
+                       __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
+}
+
 // d softplus / dt = sigmoid(t)
 __device__ __forceinline__ float sigmoid_f(float t) {
     return 1.f / (1.f + ex2_sfu(-t * kLog2e));

@@ -34,7 +34,11 @@
 namespace ss2d {
 
 constexpr int kWarp = 32;   // threads (= channels) per CTA
-constexpr int kLC = 16;     // steps staged per chunk (B/C, u, delta)
+// steps staged per chunk (B/C, u, delta); shorter chunks use less shared memory per CTA
+#ifndef SS2D_FWD_LC
+#define SS2D_FWD_LC 16
+#endif
+constexpr int kLC = SS2D_FWD_LC;
 constexpr int kG = 4;       // steps per register group
 constexpr int kStateChunk = SS2D_CHUNK_LEN;
 
@@ -42,6 +46,15 @@ constexpr int kStateChunk = SS2D_CHUNK_LEN;
 // headline problem's 3,072 warps in one wave on 148 SMs, fewer leaves more registers.
 #ifndef SS2D_FWD_MIN_BLOCKS
 #define SS2D_FWD_MIN_BLOCKS 16
+#endif
+// Of every 16 states, how many take their exponentials from the FMA-pipe
+// polynomial (ex2_poly2) instead of the SFU, to balance the two pipes.
+#ifndef SS2D_FWD_POLY_STATES
+#define SS2D_FWD_POLY_STATES 0
+#endif
+// 1: the y readout sums even and odd states in two accumulators (shorter chains)
+#ifndef SS2D_FWD_YSPLIT
+#define SS2D_FWD_YSPLIT 0
 #endif
 // 1: A*log2(e) per (lane, state) lives in shared memory (fewer registers);
 // 0: in registers (fewer shared-memory loads)
@@ -271,9 +284,11 @@ __global__ void __launch_bounds__(kWarp, SS2D_FWD_MIN_BLOCKS) scan_fwd_kernel(co
                 }
                 const float2 u01 = make_float2(uv[0], uv[1]), u23 = make_float2(uv[2], uv[3]);
                 const float2 dtu01 = __fmul2_rn(dt01, u01), dtu23 = __fmul2_rn(dt23, u23);
-                // skip term first: u is not needed during the state loop
+                // skip term first: u is not needed during the state loop.  Even and odd
+                // states accumulate separately, halving the dependent chain of adds.
                 float2 y01 = __fmul2_rn(make_float2(Dc, Dc), u01);
                 float2 y23 = __fmul2_rn(make_float2(Dc, Dc), u23);
+                float2 z01 = make_float2(0.f, 0.f), z23 = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int n = 0; n < NS; ++n) {
                     const float a2s = SS2D_A2(n);
@@ -292,13 +307,30 @@ __global__ void __launch_bounds__(kWarp, SS2D_FWD_MIN_BLOCKS) scan_fwd_kernel(co
                     const float2 x01 = __fmul2_rn(dt01, a2), x23 = __fmul2_rn(dt23, a2);
                     const float2 b01 = __fmul2_rn(dtu01, make_float2(bq[0], bq[1]));
                     const float2 b23 = __fmul2_rn(dtu23, make_float2(bq[2], bq[3]));
-                    const float h0 = fmaf(ex2_sfu(x01.x), h[n], b01.x);
-                    const float h1 = fmaf(ex2_sfu(x01.y), h0, b01.y);
-                    const float h2 = fmaf(ex2_sfu(x23.x), h1, b23.x);
-                    const float h3 = fmaf(ex2_sfu(x23.y), h2, b23.y);
+                    float2 e01, e23;
+                    if (n >= NS - (SS2D_FWD_POLY_STATES * NS) / 16) {  // FMA-pipe exponentials
+                        e01 = ex2_poly2(x01);
+                        e23 = ex2_poly2(x23);
+                    } else {
+                        e01 = make_float2(ex2_sfu(x01.x), ex2_sfu(x01.y));
+                        e23 = make_float2(ex2_sfu(x23.x), ex2_sfu(x23.y));
+                    }
+                    const float h0 = fmaf(e01.x, h[n], b01.x);
+                    const float h1 = fmaf(e01.y, h0, b01.y);
+                    const float h2 = fmaf(e23.x, h1, b23.x);
+                    const float h3 = fmaf(e23.y, h2, b23.y);
                     h[n] = h3;
-                    y01 = __ffma2_rn(make_float2(cq[0], cq[1]), make_float2(h0, h1), y01);
-                    y23 = __ffma2_rn(make_float2(cq[2], cq[3]), make_float2(h2, h3), y23);
+                    if (SS2D_FWD_YSPLIT && (n & 1)) {
+                        z01 = __ffma2_rn(make_float2(cq[0], cq[1]), make_float2(h0, h1), z01);
+                        z23 = __ffma2_rn(make_float2(cq[2], cq[3]), make_float2(h2, h3), z23);
+                    } else {
+                        y01 = __ffma2_rn(make_float2(cq[0], cq[1]), make_float2(h0, h1), y01);
+                        y23 = __ffma2_rn(make_float2(cq[2], cq[3]), make_float2(h2, h3), y23);
+                    }
+                }
+                if (SS2D_FWD_YSPLIT) {
+                    y01 = __fadd2_rn(y01, z01);
+                    y23 = __fadd2_rn(y23, z23);
                 }
                 if (PASS == 1) {
                     dtsum += (dt01.x + dt01.y) + (dt23.x + dt23.y);
