@@ -36,14 +36,17 @@ namespace ss2d {
 constexpr int kWarp = 32;   // threads (= channels) per CTA
 // steps staged per chunk (B/C, u, delta); shorter chunks use less shared memory per CTA
 #ifndef SS2D_FWD_LC
-#define SS2D_FWD_LC 16
+#define SS2D_FWD_LC 8
 #endif
 constexpr int kLC = SS2D_FWD_LC;
 constexpr int kG = 4;       // steps per register group
 constexpr int kStateChunk = SS2D_CHUNK_LEN;
 
-// Resident CTAs (warps) per SM the forward kernel is compiled for; 21 puts the
-// headline problem's 3,072 warps in one wave on 148 SMs, fewer leaves more registers.
+// Resident CTAs (warps) per SM the forward kernel is compiled for.  16 keeps four
+// warps on each of the SM's four schedulers (13 or 21 would leave one scheduler a
+// warp more than the others) and leaves 128 registers per lane, enough for the
+// unrolled 16-state loop without spills; fewer registers (e.g. 96 for 20 warps)
+// spill and measured slower.
 #ifndef SS2D_FWD_MIN_BLOCKS
 #define SS2D_FWD_MIN_BLOCKS 16
 #endif
@@ -57,9 +60,9 @@ constexpr int kStateChunk = SS2D_CHUNK_LEN;
 #define SS2D_FWD_YSPLIT 0
 #endif
 // 1: A*log2(e) per (lane, state) lives in shared memory (fewer registers);
-// 0: in registers (fewer shared-memory loads)
+// 0: in registers for fp32 inputs (fewer shared-memory loads), shared memory for bf16
 #ifndef SS2D_FWD_A2_SMEM
-#define SS2D_FWD_A2_SMEM 1
+#define SS2D_FWD_A2_SMEM 0
 #endif
 
 struct FwdParams {
@@ -159,13 +162,12 @@ __device__ __forceinline__ void stage_chunk(FwdStage<Tin, NS> &st, const Tin *Bk
 template <int NS, typename Tin, typename Tout, bool IMG, int PASS, bool VEC>
 __global__ void __launch_bounds__(kWarp, SS2D_FWD_MIN_BLOCKS) scan_fwd_kernel(const FwdParams p) {
     __shared__ __align__(16) FwdStage<Tin, NS> stage[2];
-#if SS2D_FWD_A2_SMEM
-    __shared__ float A2s[NS][kWarp];  // A[c, n] * log2(e) of each lane's channel (kept out of registers)
-#define SS2D_A2(n) A2s[n][t]
-#else
+    // A[c, n] * log2(e) of each lane's channel: in registers for fp32 inputs, in shared memory
+    // for bf16 (whose conversions need the registers)
+    constexpr bool kA2Smem = SS2D_FWD_A2_SMEM || sizeof(Tin) < 4;
+    __shared__ float A2s[kA2Smem ? NS : 1][kWarp];
     float A2r[NS];
-#define SS2D_A2(n) A2r[n]
-#endif
+#define SS2D_A2(n) (kA2Smem ? A2s[n][t] : A2r[n])
 
     const int t = threadIdx.x;
     const int k = blockIdx.y;
@@ -182,7 +184,11 @@ __global__ void __launch_bounds__(kWarp, SS2D_FWD_MIN_BLOCKS) scan_fwd_kernel(co
     float h[NS];
 #pragma unroll
     for (int n = 0; n < NS; ++n) {
-        SS2D_A2(n) = (active && n < N) ? p.A[c * N + n] * kLog2e : 0.f;
+        const float a2v = (active && n < N) ? p.A[c * N + n] * kLog2e : 0.f;
+        if (kA2Smem)
+            A2s[n][t] = a2v;
+        else
+            A2r[n] = a2v;
         h[n] = 0.f;
     }
     const float Dc = (active && p.Dv) ? p.Dv[c] : 0.f;
