@@ -155,6 +155,45 @@ transpose_kernel(const T *__restrict__ x, T *__restrict__ xT, int64_t H, int64_t
     }
 }
 
+// x -> xT with 4-element vector accesses (H % 4 == 0 and W % 4 == 0): 256 threads per
+// 32x32 tile, 16-byte row loads (8-byte for bf16) and 16-byte column stores through
+// a padded shared tile.  bf16 values pass through fp32 unchanged (exact).
+template <typename T>
+__global__ void __launch_bounds__(256)
+transpose_vec_kernel(const T *__restrict__ x, T *__restrict__ xT, int64_t H, int64_t W, int64_t tiles_w,
+                     int64_t tiles_h) {
+    __shared__ float tile[kTile][kTile + 1];
+    int64_t blk = blockIdx.x;
+    const int64_t tw = blk % tiles_w;
+    blk /= tiles_w;
+    const int64_t th = blk % tiles_h;
+    const int64_t bd = blk / tiles_h;
+    const int64_t L = H * W;
+    const int64_t h0 = th * kTile, w0 = tw * kTile;
+    const int t = threadIdx.x;
+    {
+        const int row = t >> 3, wq = t & 7;
+        const int64_t h = h0 + row, w = w0 + 4 * wq;
+        if (h < H && w < W) {
+            float v[4];
+            ld4(x + bd * L + h * W + w, v);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) tile[row][4 * wq + e] = v[e];
+        }
+    }
+    __syncthreads();
+    {
+        const int col = t >> 3, hq = t & 7;
+        const int64_t w = w0 + col, h = h0 + 4 * hq;
+        if (w < W && h < H) {
+            float v[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) v[e] = tile[4 * hq + e][col];
+            st4(xT + bd * L + w * H + h, v);
+        }
+    }
+}
+
 // CrossMerge with 4-element vector accesses, for H % 4 == 0 and W % 4 == 0 (then
 // every 4-pixel run of a row or a column, and its mirror in a reversed path, is
 // aligned).  256 threads per 32x32 tile; each thread handles 4 pixels.
@@ -269,6 +308,15 @@ cudaError_t launch_transpose(const LaunchShape &s, ss2d_dtype_t dt, const void *
     }
     int64_t tw, th;
     dim3 grid = tile_grid(s.B * s.D, s.H, s.W, &tw, &th);
+    if ((s.H % 4) == 0 && (s.W % 4) == 0) {
+        if (dt == SS2D_F32)
+            transpose_vec_kernel<float><<<grid, 256, 0, stream>>>((const float *)x, (float *)xT, s.H, s.W, tw, th);
+        else
+            transpose_vec_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>((const __nv_bfloat16 *)x,
+                                                                        (__nv_bfloat16 *)xT, s.H, s.W, tw, th);
+        note_launch(stream);
+        return cudaGetLastError();
+    }
     dim3 block(kTile, kRows);
     if (dt == SS2D_F32)
         transpose_kernel<float><<<grid, block, 0, stream>>>((const float *)x, (float *)xT, s.H, s.W, tw, th);
