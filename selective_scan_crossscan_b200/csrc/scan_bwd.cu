@@ -37,6 +37,10 @@
 #include "common.cuh"
 #include "kernels.h"
 
+#ifndef SS2D_BWD_MIN_BLOCKS
+#define SS2D_BWD_MIN_BLOCKS 3  // CTAs per SM the register budget is held to
+#endif
+
 namespace ss2d {
 
 constexpr int kWarps = 4;                 // warps per CTA
@@ -70,6 +74,13 @@ struct BwdParams {
     int ntiles;
 };
 
+// B and C of a block are the same for every channel of one (b, k): the CTA stages them once.
+template <int NS>
+struct BwdCtaSmem {
+    float Bs[kBlk][NS + 4];  // B[., l] with the states contiguous (16-byte aligned rows)
+    float Cs[kBlk][NS + 4];
+};
+
 template <int NS>
 struct BwdWarpSmem {
     static constexpr int HS = NS / 2;  // states per lane
@@ -79,58 +90,94 @@ struct BwdWarpSmem {
     float DTU[kChPerWarp][kRow];
     float SG[kChPerWarp][kRow];  // delta, then d softplus / d delta, then ddelta
     float G[kChPerWarp][kRow];   // dout, then du
-    float Bs[kBlk][NS + 4];      // B[., l] with the states contiguous (16-byte aligned rows)
-    float Cs[kBlk][NS + 4];
-    float ck[32][kNSub][HS];     // per-lane state checkpoints
+    float2 ck[kNSub][HS / 2][32];  // per-lane state checkpoints, lanes fastest (conflict-free)
     float red[kChPerWarp][4 * NS + 4];  // [channel][output o][2 steps]
     float bct[kBlk][2 * NS];     // channel sums of this warp: [step][dB n | dC n]
 };
 
+template <int NS>
+constexpr size_t bwd_smem_bytes() {
+    return sizeof(BwdCtaSmem<NS>) + kWarps * sizeof(BwdWarpSmem<NS>);
+}
+
+// The warp's channels: u, delta, dout of 16 channels x 16 steps.  Every load is issued
+// before the first shared-memory store so that their latencies overlap.
 template <int NS, typename Tin, typename Tg, bool IMG>
-__device__ __forceinline__ void stage_block(BwdWarpSmem<NS> &sm, const BwdParams &p, int64_t b, int k,
-                                            int64_t dw0, int nch, int64_t l0, int len) {
+__device__ __forceinline__ void stage_channels(BwdWarpSmem<NS> &sm, const BwdParams &p, int64_t b, int k,
+                                               int64_t dw0, int nch, int64_t l0, int len) {
+    constexpr int kPer = kChPerWarp * kBlk / 32;
     const int lane = threadIdx.x & 31;
     const int64_t D = p.D, L = p.L, C4 = kPaths * p.D;
     const bool rev = IMG && k >= 2;
-    for (int idx = lane; idx < kChPerWarp * kBlk; idx += 32) {
+    float uv[kPer], dv[kPer], gv[kPer];
+#pragma unroll
+    for (int t = 0; t < kPer; ++t) {
+        const int idx = lane + 32 * t;
         const int ci = idx / kBlk, i = idx % kBlk;
-        float uv = 0.f, dv = 0.f, gv = 0.f;
+        uv[t] = dv[t] = gv[t] = 0.f;
         if (ci < nch && i < len) {
             const int64_t l = l0 + i;
             const int64_t cc = k * D + dw0 + ci;
-            dv = ld(static_cast<const Tin *>(p.delta) + (b * C4 + cc) * L + l);
+            dv[t] = ld(static_cast<const Tin *>(p.delta) + (b * C4 + cc) * L + l);
             if (IMG) {
                 const int64_t row = (b * D + dw0 + ci) * L;
                 const int64_t m = rev ? (L - 1 - l) : l;
                 const Tin *ub = static_cast<const Tin *>((k & 1) ? p.uT : p.u);
                 const Tg *gb = static_cast<const Tg *>((k & 1) ? p.doutT : p.dout);
-                uv = ld(ub + row + m);
-                gv = ld(gb + row + m);
+                uv[t] = ld(ub + row + m);
+                gv[t] = ld(gb + row + m);
             } else {
-                uv = ld(static_cast<const Tin *>(p.u) + (b * C4 + cc) * L + l);
-                gv = ld(static_cast<const Tg *>(p.dout) + (b * C4 + cc) * L + l);
+                uv[t] = ld(static_cast<const Tin *>(p.u) + (b * C4 + cc) * L + l);
+                gv[t] = ld(static_cast<const Tg *>(p.dout) + (b * C4 + cc) * L + l);
             }
         }
-        sm.U[ci][i] = uv;
-        sm.SG[ci][i] = dv;
-        sm.G[ci][i] = gv;
     }
+#pragma unroll
+    for (int t = 0; t < kPer; ++t) {
+        const int idx = lane + 32 * t;
+        const int ci = idx / kBlk, i = idx % kBlk;
+        sm.U[ci][i] = uv[t];
+        sm.SG[ci][i] = dv[t];
+        sm.G[ci][i] = gv[t];
+    }
+}
+
+// The block's B and C, staged once by all the CTA's threads.
+template <int NS, typename Tin>
+__device__ __forceinline__ void stage_bc(BwdCtaSmem<NS> &cs, const BwdParams &p, int64_t b, int k, int64_t l0,
+                                         int len) {
+    constexpr int kTot = NS * kBlk;
+    constexpr int kIt = (kTot + 32 * kWarps - 1) / (32 * kWarps);
+    const int64_t L = p.L;
     const Tin *Bk = static_cast<const Tin *>(p.Bm) + (b * kPaths + k) * p.N * L;
     const Tin *Ck = static_cast<const Tin *>(p.Cm) + (b * kPaths + k) * p.N * L;
-    for (int idx = lane; idx < NS * kBlk; idx += 32) {
+    float rb[kIt], rc[kIt];
+#pragma unroll
+    for (int t = 0; t < kIt; ++t) {
+        const int idx = threadIdx.x + 32 * kWarps * t;
         const int n = idx / kBlk, i = idx % kBlk;
-        const bool ok = n < p.N && i < len;
-        sm.Bs[i][n] = ok ? ld(Bk + (int64_t)n * L + l0 + i) : 0.f;
-        sm.Cs[i][n] = ok ? ld(Ck + (int64_t)n * L + l0 + i) : 0.f;
+        const bool ok = idx < kTot && n < p.N && i < len;
+        rb[t] = ok ? ld(Bk + (int64_t)n * L + l0 + i) : 0.f;
+        rc[t] = ok ? ld(Ck + (int64_t)n * L + l0 + i) : 0.f;
+    }
+#pragma unroll
+    for (int t = 0; t < kIt; ++t) {
+        const int idx = threadIdx.x + 32 * kWarps * t;
+        const int n = idx / kBlk, i = idx % kBlk;
+        if (idx < kTot) {
+            cs.Bs[i][n] = rb[t];
+            cs.Cs[i][n] = rc[t];
+        }
     }
 }
 
 template <int NS, typename Tin, typename Tg, typename Tdu, bool IMG>
-__global__ void __launch_bounds__(32 * kWarps) scan_bwd_kernel(const BwdParams p) {
+__global__ void __launch_bounds__(32 * kWarps, SS2D_BWD_MIN_BLOCKS) scan_bwd_kernel(const BwdParams p) {
     constexpr int HS = NS / 2;
     constexpr int HP = HS / 2;  // state pairs per lane
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    BwdWarpSmem<NS> *wsm = reinterpret_cast<BwdWarpSmem<NS> *>(smem_raw);
+    BwdCtaSmem<NS> &csm = *reinterpret_cast<BwdCtaSmem<NS> *>(smem_raw);
+    BwdWarpSmem<NS> *wsm = reinterpret_cast<BwdWarpSmem<NS> *>(smem_raw + sizeof(BwdCtaSmem<NS>));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     BwdWarpSmem<NS> &sm = wsm[warp];
 
@@ -168,46 +215,63 @@ __global__ void __launch_bounds__(32 * kWarps) scan_bwd_kernel(const BwdParams p
     for (int blk = nblk - 1; blk >= 0; --blk) {
         const int64_t l0 = (int64_t)blk * kBlk;
         const int len = (int)min((int64_t)kBlk, L - l0);
-        __syncwarp();
-        stage_block<NS, Tin, Tg, IMG>(sm, p, b, k, dw0, nch, l0, len);
-        __syncwarp();
-        // pre-pass: dt, dt*u, d softplus / d delta for each (channel, step), lanes hf split the steps
-        for (int i = hf * (kBlk / 2); i < (hf + 1) * (kBlk / 2); ++i) {
-            const float tt = sm.SG[ci][i] + bias;
-            float dt, sg;
-            if (p.softplus) {
-                const float z = ex2_sfu(-fabsf(tt) * kLog2e);  // e^{-|t|}
-                dt = softplus_f(tt);
-                const float r = __frcp_rn(1.f + z);
-                sg = tt >= 0.f ? r : z * r;  // sigmoid(t)
-            } else {
-                dt = tt;
-                sg = 1.f;
-            }
-            if (i >= len) dt = 0.f;  // past the end: decay 1, no input
-            sm.DT[ci][i] = dt;
-            sm.DTU[ci][i] = dt * sm.U[ci][i];
-            sm.SG[ci][i] = sg;
-        }
-        __syncwarp();
-
-        // level 1: checkpoint every kSub steps, from the state the forward saved before this block
+        // the state the forward saved before this block (loaded first, used after the staging)
+        float2 h0[HP];
         {
-            float2 h[HP];
             const float *src = (blk > 0 && active) ? p.cs + ((b * C4 + c) * p.nchunks + (blk - 1)) * N : nullptr;
 #pragma unroll
             for (int q = 0; q < HP; ++q) {
                 const int na = n0 + 2 * q;
-                h[q] = make_float2((src && na < N) ? src[na] : 0.f, (src && na + 1 < N) ? src[na + 1] : 0.f);
+                h0[q] = make_float2((src && na < N) ? src[na] : 0.f, (src && na + 1 < N) ? src[na + 1] : 0.f);
             }
+        }
+        stage_bc<NS, Tin>(csm, p, b, k, l0, len);
+        stage_channels<NS, Tin, Tg, IMG>(sm, p, b, k, dw0, nch, l0, len);
+        __syncthreads();  // B, C of the block are staged for all warps
+        // pre-pass: dt, dt*u, d softplus / d delta for each (channel, step), lanes hf split the steps
+        if (p.softplus) {
+#pragma unroll
+            for (int j = 0; j < kBlk / 2; ++j) {
+                const int i = hf * (kBlk / 2) + j;
+                const float tt = sm.SG[ci][i] + bias;
+                const float z = ex2_sfu(-fabsf(tt) * kLog2e);  // e^{-|t|}
+                const float r = __frcp_rn(1.f + z);
+                const float dt = i < len ? softplus_f(tt) : 0.f;  // past the end: decay 1, no input
+                sm.DT[ci][i] = dt;
+                sm.DTU[ci][i] = dt * sm.U[ci][i];
+                sm.SG[ci][i] = tt >= 0.f ? r : z * r;  // sigmoid(t)
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < kBlk / 2; ++j) {
+                const int i = hf * (kBlk / 2) + j;
+                const float dt = i < len ? sm.SG[ci][i] + bias : 0.f;
+                sm.DT[ci][i] = dt;
+                sm.DTU[ci][i] = dt * sm.U[ci][i];
+                sm.SG[ci][i] = 1.f;
+            }
+        }
+        __syncwarp();
+
+        // level 1: checkpoint every kSub steps, from the state the forward saved before this block.
+        // Steps past the end of the sequence have dt = 0 (decay 1, no input), so every sub-block
+        // runs its full kSub steps; the last sub-block's steps are not needed here.
+        {
+            float2 h[HP];
+#pragma unroll
+            for (int q = 0; q < HP; ++q) h[q] = h0[q];
+#pragma unroll
             for (int s = 0; s < kNSub; ++s) {
 #pragma unroll
-                for (int q = 0; q < HP; ++q) *reinterpret_cast<float2 *>(&sm.ck[lane][s][2 * q]) = h[q];
-                for (int i = s * kSub; i < s * kSub + kSub && i < len; ++i) {
+                for (int q = 0; q < HP; ++q) sm.ck[s][q][lane] = h[q];
+                if (s == kNSub - 1) break;
+#pragma unroll
+                for (int j = 0; j < kSub; ++j) {
+                    const int i = s * kSub + j;
                     const float dt = sm.DT[ci][i], dtu = sm.DTU[ci][i];
 #pragma unroll
                     for (int q = 0; q < HP; ++q) {
-                        const float2 bb = *reinterpret_cast<const float2 *>(&sm.Bs[i][n0 + 2 * q]);
+                        const float2 bb = *reinterpret_cast<const float2 *>(&csm.Bs[i][n0 + 2 * q]);
                         const float2 x = __fmul2_rn(make_float2(dt, dt), A2[q]);
                         const float2 a = make_float2(ex2_sfu(x.x), ex2_sfu(x.y));
                         h[q] = __ffma2_rn(a, h[q], __fmul2_rn(make_float2(dtu, dtu), bb));
@@ -225,14 +289,14 @@ __global__ void __launch_bounds__(32 * kWarps) scan_bwd_kernel(const BwdParams p
             {
                 float2 h[HP];
 #pragma unroll
-                for (int q = 0; q < HP; ++q) h[q] = *reinterpret_cast<const float2 *>(&sm.ck[lane][s][2 * q]);
+                for (int q = 0; q < HP; ++q) h[q] = sm.ck[s][q][lane];
 #pragma unroll
                 for (int j = 0; j < kSub; ++j) {
                     const int i = i0 + j;  // steps past the end have dt = 0: decay 1, no input
                     const float dt = sm.DT[ci][i], dtu = sm.DTU[ci][i];
 #pragma unroll
                     for (int q = 0; q < HP; ++q) {
-                        const float2 bb = *reinterpret_cast<const float2 *>(&sm.Bs[i][n0 + 2 * q]);
+                        const float2 bb = *reinterpret_cast<const float2 *>(&csm.Bs[i][n0 + 2 * q]);
                         const float2 x = __fmul2_rn(make_float2(dt, dt), A2[q]);
                         dec[j][q] = make_float2(ex2_sfu(x.x), ex2_sfu(x.y));
                         h[q] = __ffma2_rn(dec[j][q], h[q], __fmul2_rn(make_float2(dtu, dtu), bb));
@@ -240,54 +304,44 @@ __global__ void __launch_bounds__(32 * kWarps) scan_bwd_kernel(const BwdParams p
                     }
                 }
             }
-            // the adjoint, two steps at a time (jp, jp-1)
-            for (int jp = cnt - 1; jp >= 0; jp -= 2) {
-                float2 vb[2][HP], vc[2][HP];  // dB, dC contributions of the two steps
+            float2 vb[2][HP], vc[2][HP];
+            // one step of the adjoint walk; jj is the register-resident step, e the slot of
+            // the two-step reduction it fills
+            auto adjoint_step = [&](const int jj, const int e) {
+                const int i = i0 + jj;
+                const float g = sm.G[ci][i], dt = sm.DT[ci][i], dtu = sm.DTU[ci][i];
+                const float uv = sm.U[ci][i];
+                float2 ddt2 = make_float2(0.f, 0.f), du2 = make_float2(0.f, 0.f);
 #pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int j = jp - e;
-#pragma unroll
-                    for (int q = 0; q < HP; ++q) {
-                        vb[e][q] = make_float2(0.f, 0.f);
-                        vc[e][q] = make_float2(0.f, 0.f);
-                    }
-                    if (j < 0) continue;
-#pragma unroll
-                    for (int jj = 0; jj < kSub; ++jj) {
-                        if (jj != j) continue;  // registers need compile-time indices
-                        const int i = i0 + jj;
-                        const float g = sm.G[ci][i], dt = sm.DT[ci][i], dtu = sm.DTU[ci][i];
-                        const float uv = sm.U[ci][i];
-                        float2 ddt2 = make_float2(0.f, 0.f), du2 = make_float2(0.f, 0.f);
-#pragma unroll
-                        for (int q = 0; q < HP; ++q) {
-                            const float2 bb = *reinterpret_cast<const float2 *>(&sm.Bs[i][n0 + 2 * q]);
-                            const float2 cc = *reinterpret_cast<const float2 *>(&sm.Cs[i][n0 + 2 * q]);
-                            lam[q] = __ffma2_rn(cc, make_float2(g, g), lam[q]);
-                            const float2 bt = __fmul2_rn(make_float2(dtu, dtu), bb);  // as in the recompute
-                            const float2 ah = __ffma2_rn(bt, make_float2(-1.f, -1.f), hist[jj][q]);  // a_l h_{l-1}
-                            const float2 inner = __ffma2_rn(Aln[q], ah, __fmul2_rn(make_float2(uv, uv), bb));
-                            ddt2 = __ffma2_rn(lam[q], inner, ddt2);
-                            const float2 ldt = __fmul2_rn(lam[q], make_float2(dt, dt));
-                            dA[q] = __ffma2_rn(ldt, ah, dA[q]);
-                            du2 = __ffma2_rn(ldt, bb, du2);
-                            vb[e][q] = __fmul2_rn(lam[q], make_float2(dtu, dtu));
-                            vc[e][q] = __fmul2_rn(make_float2(g, g), hist[jj][q]);
-                            lam[q] = __fmul2_rn(lam[q], dec[jj][q]);
-                        }
-                        float ddt = ddt2.x + ddt2.y, dul = du2.x + du2.y;
-                        ddt += __shfl_xor_sync(0xffffffffu, ddt, 1);  // the other half of the states
-                        dul += __shfl_xor_sync(0xffffffffu, dul, 1);
-                        if (hf == 0 && active) {
-                            const float dd = ddt * sm.SG[ci][i];
-                            dbias += dd;
-                            dD = fmaf(g, uv, dD);
-                            sm.SG[ci][i] = dd;
-                            sm.G[ci][i] = fmaf(g, Dc, dul);
-                        }
-                    }
+                for (int q = 0; q < HP; ++q) {
+                    const float2 bb = *reinterpret_cast<const float2 *>(&csm.Bs[i][n0 + 2 * q]);
+                    const float2 cc = *reinterpret_cast<const float2 *>(&csm.Cs[i][n0 + 2 * q]);
+                    lam[q] = __ffma2_rn(cc, make_float2(g, g), lam[q]);
+                    const float2 bt = __fmul2_rn(make_float2(dtu, dtu), bb);  // as in the recompute
+                    const float2 ah = __ffma2_rn(bt, make_float2(-1.f, -1.f), hist[jj][q]);  // a_l h_{l-1}
+                    const float2 inner = __ffma2_rn(Aln[q], ah, __fmul2_rn(make_float2(uv, uv), bb));
+                    ddt2 = __ffma2_rn(lam[q], inner, ddt2);
+                    const float2 ldt = __fmul2_rn(lam[q], make_float2(dt, dt));
+                    dA[q] = __ffma2_rn(ldt, ah, dA[q]);
+                    du2 = __ffma2_rn(ldt, bb, du2);
+                    vb[e][q] = __fmul2_rn(lam[q], make_float2(dtu, dtu));
+                    vc[e][q] = __fmul2_rn(make_float2(g, g), hist[jj][q]);
+                    lam[q] = __fmul2_rn(lam[q], dec[jj][q]);
                 }
-                // transpose the two steps' contributions: red[ci][o][e], o = state (dB) or NS + state (dC)
+                float ddt = ddt2.x + ddt2.y, dul = du2.x + du2.y;
+                ddt += __shfl_xor_sync(0xffffffffu, ddt, 1);  // the other half of the states
+                dul += __shfl_xor_sync(0xffffffffu, dul, 1);
+                if (hf == 0 && active) {
+                    const float dd = ddt * sm.SG[ci][i];
+                    dbias += dd;
+                    dD = fmaf(g, uv, dD);
+                    sm.SG[ci][i] = dd;
+                    sm.G[ci][i] = fmaf(g, Dc, dul);
+                }
+            };
+            // transpose two steps' contributions, red[ci][o][e] (o = state for dB, NS + state for dC),
+            // and let lane o sum output o over the warp's channels for both steps at once
+            auto reduce_pair = [&](const int ia, const int ib) {
 #pragma unroll
                 for (int q = 0; q < HP; ++q) {
                     const int o = n0 + 2 * q;
@@ -297,15 +351,51 @@ __global__ void __launch_bounds__(32 * kWarps) scan_bwd_kernel(const BwdParams p
                         make_float4(vc[0][q].x, vc[1][q].x, vc[0][q].y, vc[1][q].y);
                 }
                 __syncwarp();
-                if (lane < 2 * NS) {  // lane = output o: sum over the warp's channels, both steps at once
-                    float2 acc = make_float2(0.f, 0.f);
+                if (lane < 2 * NS) {  // four interleaved partial sums, combined in a fixed order
+                    float2 acc[4];
 #pragma unroll
-                    for (int r = 0; r < kChPerWarp; ++r)
-                        acc = __fadd2_rn(acc, *reinterpret_cast<const float2 *>(&sm.red[r][2 * lane]));
-                    sm.bct[i0 + jp][lane] = acc.x;
-                    if (jp - 1 >= 0) sm.bct[i0 + jp - 1][lane] = acc.y;
+                    for (int r = 0; r < 4; ++r) acc[r] = *reinterpret_cast<const float2 *>(&sm.red[r][2 * lane]);
+#pragma unroll
+                    for (int r = 4; r < kChPerWarp; ++r)
+                        acc[r & 3] = __fadd2_rn(acc[r & 3], *reinterpret_cast<const float2 *>(&sm.red[r][2 * lane]));
+                    const float2 sum = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+                    sm.bct[ia][lane] = sum.x;
+                    if (ib >= 0) sm.bct[ib][lane] = sum.y;
                 }
                 __syncwarp();
+            };
+            if (cnt == kSub) {  // the common case: a full sub-block, steps 3, 2, 1, 0
+                adjoint_step(3, 0);
+                adjoint_step(2, 1);
+                reduce_pair(i0 + 3, i0 + 2);
+                adjoint_step(1, 0);
+                adjoint_step(0, 1);
+                reduce_pair(i0 + 1, i0);
+            } else {  // the last, partial sub-block of a sequence
+#pragma unroll
+                for (int q = 0; q < HP; ++q) {
+                    vb[1][q] = make_float2(0.f, 0.f);
+                    vc[1][q] = make_float2(0.f, 0.f);
+                }
+                if (cnt == 3) {
+                    adjoint_step(2, 0);
+                    adjoint_step(1, 1);
+                    reduce_pair(i0 + 2, i0 + 1);
+                    adjoint_step(0, 0);
+#pragma unroll
+                    for (int q = 0; q < HP; ++q) {
+                        vb[1][q] = make_float2(0.f, 0.f);
+                        vc[1][q] = make_float2(0.f, 0.f);
+                    }
+                    reduce_pair(i0, -1);
+                } else if (cnt == 2) {
+                    adjoint_step(1, 0);
+                    adjoint_step(0, 1);
+                    reduce_pair(i0 + 1, i0);
+                } else {
+                    adjoint_step(0, 0);
+                    reduce_pair(i0, -1);
+                }
             }
         }
         __syncthreads();  // all four warps' channel sums of this block are in shared memory
@@ -401,7 +491,7 @@ size_t scan_bwd_workspace_bytes(const LaunchShape &s) {
 
 template <int NS, typename Tin, typename Tg, typename Tdu, bool IMG>
 static cudaError_t launch_bwd_t(const LaunchShape &s, const BwdParams &p, cudaStream_t stream) {
-    const size_t smem = sizeof(BwdWarpSmem<NS>) * kWarps;
+    const size_t smem = bwd_smem_bytes<NS>();
     auto kern = scan_bwd_kernel<NS, Tin, Tg, Tdu, IMG>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
