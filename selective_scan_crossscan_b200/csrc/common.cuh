@@ -79,6 +79,13 @@ __device__ __forceinline__ int64_t path_pixel(int k, int64_t l, int64_t H, int64
 // ------------------------------------------------------------------ math --
 
 // 2^x on the SFU (MUFU.EX2); flushes subnormal results to zero.
+// 1 / x from the special-function unit (about 1 ulp; no IEEE special-case path)
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ float ex2_sfu(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

@@ -193,14 +193,13 @@ __global__ void __launch_bounds__(32 * kWarps, SS2D_BWD_MIN_BLOCKS) scan_bwd_ker
     const int N = p.N;
     const int n0 = hf * HS;  // first state of this lane
 
-    float2 A2[HP], Aln[HP], lam[HP], dA[HP];
+    float2 A2[HP], lam[HP], dA[HP];
 #pragma unroll
     for (int q = 0; q < HP; ++q) {
         const int na = n0 + 2 * q, nb = na + 1;
         const float aa = (active && na < N) ? p.A[c * N + na] : 0.f;
         const float ab = (active && nb < N) ? p.A[c * N + nb] : 0.f;
         A2[q] = make_float2(aa * kLog2e, ab * kLog2e);
-        Aln[q] = make_float2(aa, ab);
         lam[q] = make_float2(0.f, 0.f);
         dA[q] = make_float2(0.f, 0.f);
     }
@@ -235,7 +234,7 @@ __global__ void __launch_bounds__(32 * kWarps, SS2D_BWD_MIN_BLOCKS) scan_bwd_ker
                 const int i = hf * (kBlk / 2) + j;
                 const float tt = sm.SG[ci][i] + bias;
                 const float z = ex2_sfu(-fabsf(tt) * kLog2e);  // e^{-|t|}
-                const float r = __frcp_rn(1.f + z);
+                const float r = rcp_approx(1.f + z);  // 1 + z in [1, 2]
                 const float dt = i < len ? softplus_f(tt) : 0.f;  // past the end: decay 1, no input
                 sm.DT[ci][i] = dt;
                 sm.DTU[ci][i] = dt * sm.U[ci][i];
@@ -311,32 +310,37 @@ __global__ void __launch_bounds__(32 * kWarps, SS2D_BWD_MIN_BLOCKS) scan_bwd_ker
                 const int i = i0 + jj;
                 const float g = sm.G[ci][i], dt = sm.DT[ci][i], dtu = sm.DTU[ci][i];
                 const float uv = sm.U[ci][i];
-                float2 ddt2 = make_float2(0.f, 0.f), du2 = make_float2(0.f, 0.f);
+                // with t = lambda a_l h_{l-1}: dA += dt t, ddt = sum A t + u sum lambda B,
+                // du = g D + dt sum lambda B
+                float2 sA = make_float2(0.f, 0.f), sB = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int q = 0; q < HP; ++q) {
                     const float2 bb = *reinterpret_cast<const float2 *>(&csm.Bs[i][n0 + 2 * q]);
                     const float2 cc = *reinterpret_cast<const float2 *>(&csm.Cs[i][n0 + 2 * q]);
                     lam[q] = __ffma2_rn(cc, make_float2(g, g), lam[q]);
-                    const float2 bt = __fmul2_rn(make_float2(dtu, dtu), bb);  // as in the recompute
-                    const float2 ah = __ffma2_rn(bt, make_float2(-1.f, -1.f), hist[jj][q]);  // a_l h_{l-1}
-                    const float2 inner = __ffma2_rn(Aln[q], ah, __fmul2_rn(make_float2(uv, uv), bb));
-                    ddt2 = __ffma2_rn(lam[q], inner, ddt2);
-                    const float2 ldt = __fmul2_rn(lam[q], make_float2(dt, dt));
-                    dA[q] = __ffma2_rn(ldt, ah, dA[q]);
-                    du2 = __ffma2_rn(ldt, bb, du2);
+                    // a_l h_{l-1} = h_l - dt u B, with dt u B rounded as in the recompute (an add of the
+                    // rounded product could be contracted into an unrounded FFMA; as an FFMA's
+                    // multiplicand it cannot, so L = 1 gives dA = 0 exactly)
+                    const float2 bt = __fmul2_rn(make_float2(dtu, dtu), bb);
+                    const float2 ah = __ffma2_rn(bt, make_float2(-1.f, -1.f), hist[jj][q]);
+                    const float2 t = __fmul2_rn(lam[q], ah);
+                    dA[q] = __ffma2_rn(make_float2(dt, dt), t, dA[q]);
+                    sA = __ffma2_rn(A2[q], t, sA);
+                    sB = __ffma2_rn(lam[q], bb, sB);
                     vb[e][q] = __fmul2_rn(lam[q], make_float2(dtu, dtu));
                     vc[e][q] = __fmul2_rn(make_float2(g, g), hist[jj][q]);
                     lam[q] = __fmul2_rn(lam[q], dec[jj][q]);
                 }
-                float ddt = ddt2.x + ddt2.y, dul = du2.x + du2.y;
-                ddt += __shfl_xor_sync(0xffffffffu, ddt, 1);  // the other half of the states
-                dul += __shfl_xor_sync(0xffffffffu, dul, 1);
+                float sa = sA.x + sA.y, sb = sB.x + sB.y;
+                sa += __shfl_xor_sync(0xffffffffu, sa, 1);  // the other half of the states
+                sb += __shfl_xor_sync(0xffffffffu, sb, 1);
                 if (hf == 0 && active) {
+                    const float ddt = fmaf(kLn2, sa, uv * sb);  // A = A2 ln 2
                     const float dd = ddt * sm.SG[ci][i];
                     dbias += dd;
                     dD = fmaf(g, uv, dD);
                     sm.SG[ci][i] = dd;
-                    sm.G[ci][i] = fmaf(g, Dc, dul);
+                    sm.G[ci][i] = fmaf(g, Dc, dt * sb);
                 }
             };
             // transpose two steps' contributions, red[ci][o][e] (o = state for dB, NS + state for dC),
