@@ -59,9 +59,9 @@ def _load():
             lib.oracle_cross_scan.argtypes = [l, l, l, l, P, P]
             lib.oracle_cross_merge.argtypes = [l, l, l, l, P, P]
             lib.oracle_selective_scan_fwd.argtypes = [l, l, l, l, l, P, P, P, P, P, P, P,
-                                                      ctypes.c_int, P, P]
+                                                      ctypes.c_int, P, P, P]
             lib.oracle_selective_scan_bwd.argtypes = [l, l, l, l, l, P, P, P, P, P, P, P,
-                                                      ctypes.c_int, P, P, P, P, P, P, P, P]
+                                                      ctypes.c_int, P, P, P, P, P, P, P, P, P, P]
             lib.oracle_ss2d_forward.argtypes = [l, l, l, l, l, P, P, P, P, P, P, P, ctypes.c_int, P]
             lib.oracle_ss2d_backward.argtypes = [l, l, l, l, l, P, P, P, P, P, P, P, ctypes.c_int,
                                                  P, P, P, P, P, P, P, P]
@@ -114,27 +114,29 @@ def cross_merge(ys, H: int, W: int):
 
 
 def selective_scan_fwd(u, delta, A, B, C, D=None, delta_bias=None, delta_softplus=False,
-                       return_last_state=False):
-    """S6 forward.  u, delta (Bn, Ch, L); A (Ch, N); B, C (Bn, G, N, L); D, delta_bias (Ch)."""
+                       return_last_state=False, z=None):
+    """S6 forward.  u, delta (Bn, Ch, L); A (Ch, N); B, C (Bn, G, N, L); D, delta_bias (Ch);
+    z (Bn, Ch, L) gates the output with silu(z)."""
     u, delta, A, B, C = (_f64(t) for t in (u, delta, A, B, C))
-    D, delta_bias = _f64(D), _f64(delta_bias)
+    D, delta_bias, z = _f64(D), _f64(delta_bias), _f64(z)
     Bn, Ch, L = u.shape
     N = A.shape[1]
     G = B.shape[1]
     assert delta.shape == u.shape and A.shape == (Ch, N) and B.shape == (Bn, G, N, L)
     assert C.shape == B.shape and Ch % G == 0
+    assert z is None or z.shape == u.shape
     out = np.empty_like(u)
     last = np.empty((Bn, Ch, N), dtype=np.float64) if return_last_state else None
     _load().oracle_selective_scan_fwd(Bn, Ch, L, N, G, _ptr(u), _ptr(delta), _ptr(A), _ptr(B),
                                       _ptr(C), _ptr(D), _ptr(delta_bias), int(bool(delta_softplus)),
-                                      _ptr(out), _ptr(last))
+                                      _ptr(z), _ptr(out), _ptr(last))
     return (out, last) if return_last_state else out
 
 
-def selective_scan_bwd(u, delta, A, B, C, D, delta_bias, delta_softplus, dout):
-    """S6 backward.  Returns dict du, ddelta, dA, dB, dC, dD, ddelta_bias (None when absent)."""
+def selective_scan_bwd(u, delta, A, B, C, D, delta_bias, delta_softplus, dout, z=None):
+    """S6 backward.  Returns dict du, ddelta, dA, dB, dC, dD, ddelta_bias, dz (None when absent)."""
     u, delta, A, B, C, dout = (_f64(t) for t in (u, delta, A, B, C, dout))
-    D, delta_bias = _f64(D), _f64(delta_bias)
+    D, delta_bias, z = _f64(D), _f64(delta_bias), _f64(z)
     Bn, Ch, L = u.shape
     N = A.shape[1]
     G = B.shape[1]
@@ -145,11 +147,13 @@ def selective_scan_bwd(u, delta, A, B, C, D, delta_bias, delta_softplus, dout):
     dC = np.empty_like(C)
     dD = np.empty(Ch, dtype=np.float64) if D is not None else None
     dbias = np.empty(Ch, dtype=np.float64) if delta_bias is not None else None
+    dz = np.empty_like(u) if z is not None else None
+    assert z is None or z.shape == u.shape
     _load().oracle_selective_scan_bwd(Bn, Ch, L, N, G, _ptr(u), _ptr(delta), _ptr(A), _ptr(B),
                                       _ptr(C), _ptr(D), _ptr(delta_bias), int(bool(delta_softplus)),
-                                      _ptr(dout), _ptr(du), _ptr(ddelta), _ptr(dA), _ptr(dB),
-                                      _ptr(dC), _ptr(dD), _ptr(dbias))
-    return dict(du=du, ddelta=ddelta, dA=dA, dB=dB, dC=dC, dD=dD, ddelta_bias=dbias)
+                                      _ptr(z), _ptr(dout), _ptr(du), _ptr(ddelta), _ptr(dA), _ptr(dB),
+                                      _ptr(dC), _ptr(dD), _ptr(dbias), _ptr(dz))
+    return dict(du=du, ddelta=ddelta, dA=dA, dB=dB, dC=dC, dD=dD, ddelta_bias=dbias, dz=dz)
 
 
 def ss2d_forward(x, delta, A, B, C, D=None, delta_bias=None, delta_softplus=True):

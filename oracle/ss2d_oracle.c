@@ -21,6 +21,9 @@
  *    h = exp(delta*A) * h + delta * B * u starting from h = 0; the output is
  *    y = sum_n C[n] * h[n] + D * u.  B and C carry G groups and channel c uses
  *    group c / (channels / G) (the repeat "B G N L -> B (G H) N L").
+ *    When a gate z is given, the output is multiplied by silu(z) = z * sigmoid(z)
+ *    after the D * u term is added (the last lines of selective_scan_ref), and
+ *    the state after the last step can be returned (return_last_state).
  *
  *  - Backward: the same page gives only the signature of the CUDA backward
  *    (SelectiveScanFn.backward); the gradients here are the analytic
@@ -99,6 +102,19 @@ static double sigmoid_d(double t)
     return 1.0 / (1.0 + exp(-t));
 }
 
+/* silu(z) = z * sigmoid(z), the output gate of selective_scan_ref */
+static double silu_d(double z)
+{
+    return z * sigmoid_d(z);
+}
+
+/* d silu / dz = sigmoid(z) * (1 + z * (1 - sigmoid(z))) */
+static double silu_grad_d(double z)
+{
+    double s = sigmoid_d(z);
+    return s * (1.0 + z * (1.0 - s));
+}
+
 /* delta + bias, then softplus when asked (selective_scan_ref, first lines). */
 static double step_size(double delta, const double *bias, long c, int softplus, double *t_out)
 {
@@ -113,12 +129,14 @@ static double step_size(double delta, const double *bias, long c, int softplus, 
  *   A             : (Ch, N)
  *   Bm, Cm        : (Bn, G, N, L), channel c uses group c / (Ch / G)
  *   Dv, bias      : (Ch) or NULL
+ *   z             : (Bn, Ch, L) or NULL -- out = (y + D u) * silu(z)
  *   last_state    : (Bn, Ch, N) or NULL -- h after the last step
  */
 void oracle_selective_scan_fwd(long Bn, long Ch, long L, long N, long G,
                                const double *u, const double *delta, const double *A,
                                const double *Bm, const double *Cm, const double *Dv,
-                               const double *bias, int softplus, double *out, double *last_state)
+                               const double *bias, int softplus, const double *z, double *out,
+                               double *last_state)
 {
     long per_group = Ch / G;
 #pragma omp parallel for collapse(2) schedule(dynamic)
@@ -138,6 +156,7 @@ void oracle_selective_scan_fwd(long Bn, long Ch, long L, long N, long G,
                 for (long n = 0; n < N; ++n)
                     y += Cg[n * L + l] * h[n];
                 if (Dv) y += Dv[c] * uc[l];
+                if (z) y *= silu_d(z[(b * Ch + c) * L + l]);
                 out[(b * Ch + c) * L + l] = y;
             }
             if (last_state)
@@ -162,13 +181,16 @@ void oracle_selective_scan_fwd(long Bn, long Ch, long L, long N, long G,
  *   dB[n,l]  += lambda_n dt_l u_l
  *   du_l     += lambda_n dt_l B[n,l]   (+ g_l D[c])
  *   ddelta_l  = ddt_l * sigmoid(t_l) under softplus, else ddt_l
+ * With a gate z (out = o * silu(z), o = y + D u): g_l = dout_l * silu(z_l) is the
+ * gradient reaching o, and dz_l = dout_l * o_l * silu'(z_l), o_l rebuilt from the
+ * recomputed states.  dz: (Bn, Ch, L), written only when z is given.
  */
 void oracle_selective_scan_bwd(long Bn, long Ch, long L, long N, long G,
                                const double *u, const double *delta, const double *A,
                                const double *Bm, const double *Cm, const double *Dv,
-                               const double *bias, int softplus, const double *dout,
-                               double *du, double *ddelta, double *dA, double *dB, double *dC,
-                               double *dD, double *dbias)
+                               const double *bias, int softplus, const double *z,
+                               const double *dout, double *du, double *ddelta, double *dA,
+                               double *dB, double *dC, double *dD, double *dbias, double *dz)
 {
     long per_group = Ch / G;
     /* per-batch partials of the parameter gradients, summed in fixed order below */
@@ -210,6 +232,13 @@ void oracle_selective_scan_bwd(long Bn, long Ch, long L, long N, long G,
                 double t;
                 double dt = step_size(dc[l], bias, c, softplus, &t);
                 double g_l = gc[l];
+                if (z) {
+                    double zl = z[(b * Ch + c) * L + l];
+                    double o = Dv ? Dv[c] * uc[l] : 0.0;
+                    for (long n = 0; n < N; ++n) o += Cg[n * L + l] * hist[l * N + n];
+                    dz[(b * Ch + c) * L + l] = g_l * o * silu_grad_d(zl);
+                    g_l *= silu_d(zl);
+                }
                 double dul = Dv ? g_l * Dv[c] : 0.0;
                 double ddt = 0.0;
                 if (Dv) pD[b * Ch + c] += g_l * uc[l];
@@ -275,7 +304,7 @@ void oracle_ss2d_forward(long Bn, long Dn, long H, long W, long N,
     double *ys = (double *)malloc(sizeof(double) * seq);
     oracle_cross_scan(Bn, Dn, H, W, x, xs);
     oracle_selective_scan_fwd(Bn, K_PATHS * Dn, L, N, K_PATHS, xs, delta, A, Bm, Cm, Dv, bias,
-                              softplus, ys, NULL);
+                              softplus, NULL, ys, NULL);
     oracle_cross_merge(Bn, Dn, H, W, ys, y);
     free(xs);
     free(ys);
@@ -302,7 +331,7 @@ void oracle_ss2d_backward(long Bn, long Dn, long H, long W, long N,
     oracle_cross_scan(Bn, Dn, H, W, x, xs);
     oracle_cross_scan(Bn, Dn, H, W, dy, gs);
     oracle_selective_scan_bwd(Bn, K_PATHS * Dn, L, N, K_PATHS, xs, delta, A, Bm, Cm, Dv, bias,
-                              softplus, gs, dus, ddelta, dA, dB, dC, dD, dbias);
+                              softplus, NULL, gs, dus, ddelta, dA, dB, dC, dD, dbias, NULL);
     oracle_cross_merge(Bn, Dn, H, W, dus, dx);
     free(xs);
     free(gs);

@@ -9,7 +9,10 @@ Pins used: hand-tabulated traversal orders and hand-worked S6 values
 recurrence evaluated by brute force, special cases that reduce to library
 routines (cumulative sum, elementwise product), linearity, permutation and
 adjoint identities of the index maps, central finite differences and exact
-dot-product identities for the backward.
+dot-product identities for the backward.  The output gate (out times silu(z),
+the last lines of selective_scan_ref) is pinned by its special values, by
+scipy's logistic function and by central differences; the last state by
+reading it back through a one-hot C.
 """
 import json
 import math
@@ -383,6 +386,95 @@ def test_backward_of_scan_alone_matches_central_differences(oracle):
             fd = (lp - lm) / (2 * h)
             an = g[gname].reshape(-1)[i]
             assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (name, i, fd, an)
+
+
+# ------------------------------------------------------- gate and last state
+
+def test_gate_special_values(oracle):
+    # silu(0) = 0: a zero gate zeroes every output; silu(z) -> z as z grows (sigmoid(40) = 1 - 4e-18)
+    rng = _rng(41)
+    p = _random_problem(rng, 2, 3, 9, 4, 1)
+    plain = oracle.selective_scan_fwd(**p)
+    zero = oracle.selective_scan_fwd(**p, z=np.zeros_like(p["u"]))
+    assert np.all(zero == 0.0)
+    big = oracle.selective_scan_fwd(**p, z=np.full_like(p["u"], 40.0))
+    np.testing.assert_allclose(big, 40.0 * plain, rtol=1e-15, atol=0)
+
+
+def test_gate_matches_logistic_times_output(oracle):
+    # gated = ungated (including the D*u term) times z * expit(z), elementwise at the same (b, c, l)
+    from scipy.special import expit
+
+    rng = _rng(42)
+    p = _random_problem(rng, 2, 4, 11, 3, 2)
+    z = 2.0 * rng.standard_normal(p["u"].shape)
+    plain = oracle.selective_scan_fwd(**p)
+    gated = oracle.selective_scan_fwd(**p, z=z)
+    np.testing.assert_allclose(gated, plain * z * expit(z), rtol=1e-13, atol=1e-15)
+
+
+def test_gated_backward_matches_central_differences(oracle):
+    rng = _rng(43)
+    p = _random_problem(rng, 2, 4, 7, 3, 2)
+    z = 1.5 * rng.standard_normal(p["u"].shape)
+    dout = rng.standard_normal(p["u"].shape)
+    g = oracle.selective_scan_bwd(p["u"], p["delta"], p["A"], p["B"], p["C"], p["D"], p["delta_bias"],
+                                  True, dout, z=z)
+    q = dict(p, z=z)
+
+    def loss():
+        return float(np.sum(oracle.selective_scan_fwd(**q) * dout))
+
+    for name, gname in (("z", "dz"), ("u", "du"), ("delta", "ddelta"), ("A", "dA"), ("B", "dB"),
+                        ("C", "dC"), ("D", "dD"), ("delta_bias", "ddelta_bias")):
+        flat = q[name].reshape(-1)
+        for i in rng.choice(flat.size, size=min(flat.size, 8), replace=False):
+            theta = flat[i]
+            h = 1e-6 * max(1.0, abs(theta))
+            flat[i] = theta + h
+            lp = loss()
+            flat[i] = theta - h
+            lm = loss()
+            flat[i] = theta
+            fd = (lp - lm) / (2 * h)
+            an = g[gname].reshape(-1)[i]
+            assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (name, i, fd, an)
+
+
+def test_gate_at_zero_halves_the_output_gradient(oracle):
+    # silu'(0) = 1/2 and silu(0) = 0: dz = dout * o / 2 and nothing reaches the scan
+    rng = _rng(44)
+    p = _random_problem(rng, 1, 3, 6, 2, 1)
+    dout = rng.standard_normal(p["u"].shape)
+    g = oracle.selective_scan_bwd(p["u"], p["delta"], p["A"], p["B"], p["C"], p["D"], p["delta_bias"],
+                                  True, dout, z=np.zeros_like(p["u"]))
+    o = oracle.selective_scan_fwd(**p)
+    np.testing.assert_allclose(g["dz"], 0.5 * dout * o, rtol=1e-14, atol=1e-15)
+    assert np.all(g["du"] == 0.0) and np.all(g["dA"] == 0.0) and np.all(g["dB"] == 0.0)
+
+
+def test_last_state_read_back_through_one_hot_c(oracle):
+    # with D absent and C[., n, L-1] = e_m, the last output is h_{L-1}[m]
+    rng = _rng(45)
+    Bn, Ch, L, N, G = 2, 4, 13, 5, 2
+    p = _random_problem(rng, Bn, Ch, L, N, G, with_d=False)
+    _, last = oracle.selective_scan_fwd(**p, return_last_state=True)
+    assert last.shape == (Bn, Ch, N)
+    for m in range(N):
+        q = dict(p)
+        q["C"] = p["C"].copy()
+        q["C"][:, :, :, L - 1] = 0.0
+        q["C"][:, :, m, L - 1] = 1.0
+        y = oracle.selective_scan_fwd(**q)
+        np.testing.assert_array_equal(y[:, :, L - 1], last[:, :, m])
+
+
+def test_last_state_unaffected_by_gate(oracle):
+    rng = _rng(46)
+    p = _random_problem(rng, 1, 2, 8, 3, 1)
+    _, a = oracle.selective_scan_fwd(**p, return_last_state=True)
+    _, b = oracle.selective_scan_fwd(**p, return_last_state=True, z=rng.standard_normal(p["u"].shape))
+    np.testing.assert_array_equal(a, b)
 
 
 # --------------------------------------------------------- input generator
