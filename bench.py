@@ -2,6 +2,7 @@
 """SS2D forward throughput on B200: state-updates/s and HBM GB/s against the roofline.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload I] [--impl ss2d|reference]
+                    [--backward] [--gate]
 
 A step is one fused SS2D forward (CrossScan -> S6 -> CrossMerge) over one batch of
 the workload, with every input already resident in HBM.  The default workload is
@@ -14,6 +15,11 @@ collective on the data path -- only a barrier and a max over ranks of the timing
 
 Rank 0 prints one JSON line.  `--impl reference` times the fp64 CPU oracle on a
 bounded sample of the same workload instead (rank 0 only).
+
+`--backward` adds the fused backward to every step; `--gate` times the scan in its
+sequence form instead, u (B, 4D, L) with the output gate out * silu(z) and the last
+state (selective_scan_fn's z and return_last_state), plus its backward with dz
+under `--backward`.  Neither is the headline line.
 """
 from __future__ import annotations
 
@@ -57,6 +63,30 @@ def fwd_algorithmic_bytes(w) -> int:
     s = 4 if w.dtype == "f32" else 2
     Bn, Dn, L, N = w.batch, w.dim, w.L, w.d_state
     return s * (Bn * Dn * L + 4 * Bn * Dn * L + 8 * Bn * N * L) + s * Bn * Dn * L + 4 * 4 * Dn * (N + 2)
+
+
+def seq_fwd_algorithmic_bytes(w, gate: bool) -> int:
+    """The sequence-form forward: read u, delta (B, 4D, L), B, C, z if gated; write out and
+    the last state (B, 4D, N) fp32."""
+    s = 4 if w.dtype == "f32" else 2
+    Bn, Dn, L, N = w.batch, w.dim, w.L, w.d_state
+    seq = 4 * Bn * Dn * L
+    return s * (seq * (3 if gate else 2) + 8 * Bn * N * L) + s * seq + 4 * 4 * Bn * Dn * N + 4 * 4 * Dn * (N + 2)
+
+
+def bwd_algorithmic_bytes(w, gate: bool = False) -> int:
+    """Bytes the backward must move at least once.  Fused form: read x, delta, B, C, dy, write
+    dx, ddelta, dB, dC.  Sequence form: u, delta, B, C, dout (+ z) in, du, ddelta, dB, dC (+ dz)
+    out.  Plus the fp32 parameters and their gradients."""
+    s = 4 if w.dtype == "f32" else 2
+    Bn, Dn, L, N = w.batch, w.dim, w.L, w.d_state
+    img = Bn * Dn * L
+    bc = 8 * Bn * N * L
+    params = 2 * 4 * 4 * Dn * (N + 2)
+    if gate:
+        seq = 4 * img
+        return s * (seq * 2 + bc) + s * seq + s * (seq * 2 + bc) + 2 * s * seq + params
+    return s * (2 * img + 4 * img + bc) + s * (img + 4 * img + bc) + params
 
 
 def source_hash() -> str:
@@ -243,13 +273,29 @@ def run_gpu(args, world, rank, local):
     if args.batch:
         w = w.with_batch(args.batch)
     dev = torch.device("cuda", local)
-    inp = ss2d_inputs.make_inputs(w, seed=shard_seed(args.workload, rank), device=dev, with_dy=args.backward)
+    if args.gate:
+        inp = ss2d_inputs.make_scan_inputs(w, seed=shard_seed(args.workload, rank), device=dev,
+                                           with_dout=args.backward, with_z=True)
+    else:
+        inp = ss2d_inputs.make_inputs(w, seed=shard_seed(args.workload, rank), device=dev, with_dy=args.backward)
     y = torch.empty((w.batch, w.dim, w.height, w.width), dtype=w.torch_dtype, device=dev)
     nbytes = ss.workspace_bytes(w.batch, w.dim, w.height, w.width, w.d_state, ss.OP_FORWARD, w.torch_dtype)
     ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    if args.backward:
+    if args.gate:
+        seq_out = torch.empty((w.batch, 4 * w.dim, w.L), dtype=w.torch_dtype, device=dev)
+
+        def step():
+            # gated sequence-form forward (keeping the chunk states under --backward), then the
+            # gated backward from them
+            res = ss.selective_scan_fwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"],
+                                        inp["delta_bias"], True, out=seq_out, z=inp["z"], return_last_state=True,
+                                        return_chunk_states=args.backward)
+            if args.backward:
+                ss.selective_scan_bwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"],
+                                      inp["delta_bias"], True, inp["dout"], chunk_states=res[2], z=inp["z"])
+    elif args.backward:
         nb = ss.workspace_bytes(w.batch, w.dim, w.height, w.width, w.d_state, ss.OP_BACKWARD, w.torch_dtype)
         wsb = torch.empty(max(nb, 1), dtype=torch.uint8, device=dev)
         cs = torch.empty((w.batch, 4 * w.dim, -(-w.L // ss.CHUNK_LEN), w.d_state), dtype=torch.float32, device=dev)
@@ -317,7 +363,13 @@ def run_gpu(args, world, rank, local):
 
     peaks = load_peaks()
     clocks = sampler.summary() if sampler else None
-    alg_bytes = fwd_algorithmic_bytes(w)
+    # algorithmic bytes of the dominant kernel: the backward's when a backward runs in the step
+    if args.backward:
+        alg_bytes = bwd_algorithmic_bytes(w, gate=args.gate)
+    elif args.gate:
+        alg_bytes = seq_fwd_algorithmic_bytes(w, gate=True)
+    else:
+        alg_bytes = fwd_algorithmic_bytes(w)
     bytes_per_update = alg_bytes / w.updates
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     achieved_gbs = bytes_per_update * w.updates / (dom_ms / 1e3) / 1e9
@@ -326,7 +378,7 @@ def run_gpu(args, world, rank, local):
     sfu_achieved = w.updates / (dom_ms / 1e3) / 1e9  # one exp(dt*A) per state update
     traffic = recorded_traffic(w.name)
 
-    e2e = run_e2e(args, w, inp, dev, stream, world, rank) if not (args.no_e2e or args.backward) else None
+    e2e = run_e2e(args, w, inp, dev, stream, world, rank) if not (args.no_e2e or args.backward or args.gate) else None
 
     result = {
         "metric": METRIC,
@@ -344,7 +396,8 @@ def run_gpu(args, world, rank, local):
         "config": {"workload": w.name, "batch_per_gpu": w.batch, "global_batch": w.batch * world, "dim": w.dim,
                    "height": w.height, "width": w.width, "d_state": w.d_state, "paths": 4,
                    "parallelism": f"batch shards x{world}, no collective",
-                   "pass": "forward + backward" if args.backward else "forward",
+                   "pass": ("forward + backward" if args.backward else "forward")
+                   + (" (sequence form, gate z + last state)" if args.gate else ""),
                    "l2": f"inputs {alg_bytes / 1e9:.2f} GB > 126 MB L2, no flush needed"},
         "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved_gbs / hbm_peak, "traffic": traffic,
@@ -359,7 +412,8 @@ def run_gpu(args, world, rank, local):
         "clocks": clocks,
         "e2e": e2e,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    # the oracle sample times the fused forward, so it is reported beside the forward line only
+    if rank == 0 and world == 1 and not (args.no_cpu_baseline or args.backward or args.gate):
         result["cpu_baseline"] = time_oracle(w, seconds_budget=args.cpu_seconds)
     return result
 
@@ -440,6 +494,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ss2d", "reference"], default="ss2d")
     ap.add_argument("--backward", action="store_true",
                     help="time forward (keeping chunk states) + fused backward per step")
+    ap.add_argument("--gate", action="store_true",
+                    help="time the sequence-form scan with the output gate z and the last state instead")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="time budget of the CPU oracle sample")

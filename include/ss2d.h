@@ -155,6 +155,43 @@ SS2D_API ss2d_status_t ss2d_selective_scan_bwd(const ss2d_desc_t *desc, const vo
                                       void *workspace, size_t workspace_bytes,
                                       ss2d_stream_t stream);
 
+/*
+ * The same forward with the rest of selective_scan_fn's signature ("vision
+ * mamba-yolov8", section "2. Vmamba module code": the z and return_last_state
+ * arguments of SelectiveScanFn.forward and selective_scan_ref).
+ * z            : (B, 4D, L) in_dtype, or NULL.  When given, the output is gated after
+ *                the D*u term: out = (C.h + D u) * silu(z), silu(z) = z * sigmoid(z),
+ *                computed in fp32 and rounded once to out_dtype.
+ * last_state   : (B, 4D, N) fp32, or NULL: the state after the last step (h at l = L-1).
+ *                It carries no gradient (the pages leave it out of the backward).
+ * Other arguments, layouts and errors as for ss2d_selective_scan_fwd;
+ * ss2d_selective_scan_fwd(...) is this call with z = last_state = NULL.
+ */
+SS2D_API ss2d_status_t ss2d_selective_scan_fwd_ex(const ss2d_desc_t *desc, const void *u, const void *delta,
+                                                  const float *A, const void *Bm, const void *Cm,
+                                                  const float *D, const void *z, const float *delta_bias,
+                                                  int delta_softplus, void *out, float *last_state,
+                                                  float *chunk_states, ss2d_stream_t stream);
+
+/*
+ * Backward of ss2d_selective_scan_fwd_ex (the backward of SelectiveScanFn with z).
+ * z            : the forward's gate, or NULL.  dout is then the gradient of the gated
+ *                output: dout * silu(z) drives the scan's backward, and
+ *                dz = dout * silu'(z) * (C.h + D u), with C.h rebuilt from the
+ *                recomputed states (the caller does not keep the ungated output).
+ * dz           : (B, 4D, L) in_dtype; must be non-NULL exactly when z is.
+ * Other arguments, layouts, workspace (SS2D_OP_SELECTIVE_SCAN_BWD) and errors as for
+ * ss2d_selective_scan_bwd, which is this call with z = dz = NULL.
+ */
+SS2D_API ss2d_status_t ss2d_selective_scan_bwd_ex(const ss2d_desc_t *desc, const void *u, const void *delta,
+                                                  const float *A, const void *Bm, const void *Cm,
+                                                  const float *D, const void *z, const float *delta_bias,
+                                                  int delta_softplus, const void *dout,
+                                                  const float *chunk_states, void *du, void *ddelta, float *dA,
+                                                  void *dBm, void *dCm, float *dD, float *ddelta_bias, void *dz,
+                                                  void *workspace, size_t workspace_bytes,
+                                                  ss2d_stream_t stream);
+
 /* --------------------------------------------------------- fused SS2D -- */
 
 /*

@@ -12,8 +12,10 @@ visual data", Fig. 2; the S6 arithmetic follows selective_scan_ref on
 "vision mamba-yolov8", section "2. Vmamba module code"):
 
 * ``cross_scan(x)``: (B, D, H, W) -> (B, 4, D, L): row-major, column-major, both reversed
-* ``selective_scan_fwd(u, delta, A, B, C, ...)``: S6 forward over (B, 4D, L) sequences
-* ``selective_scan_bwd(...)``: its gradients
+* ``selective_scan_fwd(u, delta, A, B, C, ...)``: S6 forward over (B, 4D, L) sequences,
+  with the optional output gate ``z`` (out * silu(z)) and the last state
+* ``selective_scan_bwd(...)``: its gradients (and dz)
+* ``selective_scan_fn``: the differentiable scan with selective_scan_fn's arguments
 * ``cross_merge(ys, H, W)``: (B, 4, D, L) -> (B, D, H, W), (y0 + y2) + (y1 + y3)
 * ``ss2d_forward`` / ``ss2d_backward``: the fused SS2D forward and backward
 * ``SS2DFunction``: a torch.autograd.Function around the fused pair
@@ -27,7 +29,8 @@ import threading
 import torch
 
 __all__ = [
-    "SS2DError", "cross_scan", "cross_merge", "selective_scan_fwd", "selective_scan_bwd", "ss2d_forward",
+    "SS2DError", "cross_scan", "cross_merge", "selective_scan_fwd", "selective_scan_bwd", "selective_scan_fn",
+    "SelectiveScanFunction", "ss2d_forward",
     "ss2d_backward", "SS2DFunction", "ss2d", "workspace_bytes", "chunk_states_elems", "launch_count",
     "library_path", "CHUNK_LEN", "trace_events",
 ]
@@ -81,10 +84,13 @@ def _load():
         lib.ss2d_cross_merge.argtypes = [D, P, P, P]
         lib.ss2d_selective_scan_fwd.argtypes = [D, P, P, P, P, P, P, P, i, P, P, P]
         lib.ss2d_selective_scan_bwd.argtypes = [D, P, P, P, P, P, P, P, i, P, P, P, P, P, P, P, P, P, P, sz, P]
+        lib.ss2d_selective_scan_fwd_ex.argtypes = [D, P, P, P, P, P, P, P, P, i, P, P, P, P]
+        lib.ss2d_selective_scan_bwd_ex.argtypes = [D, P, P, P, P, P, P, P, P, i, P, P, P, P, P, P, P, P, P, P,
+                                                   P, sz, P]
         lib.ss2d_forward.argtypes = [D, P, P, P, P, P, P, P, i, P, P, P, sz, P]
         lib.ss2d_backward.argtypes = [D, P, P, P, P, P, P, P, i, P, P, P, P, P, P, P, P, P, P, sz, P]
         for name in ("ss2d_cross_scan", "ss2d_cross_merge", "ss2d_selective_scan_fwd", "ss2d_selective_scan_bwd",
-                     "ss2d_forward", "ss2d_backward"):
+                     "ss2d_selective_scan_fwd_ex", "ss2d_selective_scan_bwd_ex", "ss2d_forward", "ss2d_backward"):
             getattr(lib, name).restype = ctypes.c_int
         lib.ss2d_workspace_bytes.argtypes = [D, i]
         lib.ss2d_workspace_bytes.restype = sz
@@ -214,18 +220,22 @@ def _params(A, D, delta_bias):
 
 
 def selective_scan_fwd(u, delta, A, B, C, D=None, delta_bias=None, delta_softplus=False, out=None,
-                       out_dtype=None, return_chunk_states=False):
+                       out_dtype=None, return_chunk_states=False, z=None, return_last_state=False):
     """S6 forward over the 4*dim sequences of an SS2D problem.
 
-    u, delta (Bn, 4D, L); A (4D, N) fp32; B, C (Bn, 4, N, L); D, delta_bias (4D) fp32 or None.
-    Returns out (Bn, 4D, L) [, chunk_states (Bn, 4D, ceil(L/64), N) fp32].
+    u, delta (Bn, 4D, L); A (4D, N) fp32; B, C (Bn, 4, N, L); D, delta_bias (4D) fp32 or None;
+    z (Bn, 4D, L) or None gates the output: out = (C.h + D u) * silu(z).
+    Returns out (Bn, 4D, L), followed by last_state (Bn, 4D, N) fp32 if return_last_state and
+    chunk_states (Bn, 4D, ceil(L / CHUNK_LEN), N) fp32 if return_chunk_states.
     """
     u = _c(u)
-    delta, B, C = (_c(t, u.dtype) for t in (delta, B, C))
+    delta, B, C, z = (_c(t, u.dtype) for t in (delta, B, C, z))
     A, D, delta_bias = _params(A, D, delta_bias)
     Bn, Ch, L = u.shape
     if Ch % 4 or B.shape[1] != 4:
         raise ValueError("selective_scan_fwd: u must be (B, 4*dim, L) and B/C (B, 4, N, L)")
+    if z is not None and z.shape != u.shape:
+        raise ValueError("selective_scan_fwd: z must have u's shape")
     N = A.shape[1]
     out_dtype = out_dtype or u.dtype
     if out is None:
@@ -233,17 +243,21 @@ def selective_scan_fwd(u, delta, A, B, C, D=None, delta_bias=None, delta_softplu
     cs = None
     if return_chunk_states:
         cs = torch.empty((Bn, Ch, -(-L // CHUNK_LEN), N), dtype=torch.float32, device=u.device)
+    last = torch.empty((Bn, Ch, N), dtype=torch.float32, device=u.device) if return_last_state else None
     d = _desc(Bn, Ch // 4, 1, L, N, u.dtype, out.dtype)
-    st = _load().ss2d_selective_scan_fwd(ctypes.byref(d), _p(u), _p(delta), _p(A), _p(B), _p(C), _p(D),
-                                         _p(delta_bias), int(bool(delta_softplus)), _p(out), _p(cs), _stream(u))
-    _check(st, "ss2d_selective_scan_fwd")
-    return (out, cs) if return_chunk_states else out
+    st = _load().ss2d_selective_scan_fwd_ex(ctypes.byref(d), _p(u), _p(delta), _p(A), _p(B), _p(C), _p(D), _p(z),
+                                            _p(delta_bias), int(bool(delta_softplus)), _p(out), _p(last), _p(cs),
+                                            _stream(u))
+    _check(st, "ss2d_selective_scan_fwd_ex")
+    extra = ([last] if return_last_state else []) + ([cs] if return_chunk_states else [])
+    return (out, *extra) if extra else out
 
 
-def selective_scan_bwd(u, delta, A, B, C, D, delta_bias, delta_softplus, dout, chunk_states=None):
-    """Gradients of selective_scan_fwd.  Returns dict du, ddelta, dA, dB, dC, dD, ddelta_bias."""
+def selective_scan_bwd(u, delta, A, B, C, D, delta_bias, delta_softplus, dout, chunk_states=None, z=None):
+    """Gradients of selective_scan_fwd.  Returns dict du, ddelta, dA, dB, dC, dD, ddelta_bias, dz
+    (dD, ddelta_bias, dz are None when D, delta_bias, z are)."""
     u = _c(u)
-    delta, B, C = (_c(t, u.dtype) for t in (delta, B, C))
+    delta, B, C, z = (_c(t, u.dtype) for t in (delta, B, C, z))
     A, D, delta_bias = _params(A, D, delta_bias)
     dout = _c(dout)
     chunk_states = _c(chunk_states, torch.float32)
@@ -257,15 +271,49 @@ def selective_scan_bwd(u, delta, A, B, C, D, delta_bias, delta_softplus, dout, c
     dC = torch.empty_like(C)
     dD = torch.empty_like(D) if D is not None else None
     dbias = torch.empty_like(delta_bias) if delta_bias is not None else None
+    dz = torch.empty_like(u) if z is not None else None
     d = _desc(Bn, Ch // 4, 1, L, N, u.dtype, dout.dtype)
     lib = _load()
     nbytes = int(lib.ss2d_workspace_bytes(ctypes.byref(d), OP_SELECTIVE_SCAN_BWD))
     ws = _workspace(nbytes, dev)
-    st = lib.ss2d_selective_scan_bwd(ctypes.byref(d), _p(u), _p(delta), _p(A), _p(B), _p(C), _p(D), _p(delta_bias),
-                                     int(bool(delta_softplus)), _p(dout), _p(chunk_states), _p(du), _p(ddelta),
-                                     _p(dA), _p(dB), _p(dC), _p(dD), _p(dbias), _p(ws), nbytes, _stream(u))
-    _check(st, "ss2d_selective_scan_bwd")
-    return dict(du=du, ddelta=ddelta, dA=dA, dB=dB, dC=dC, dD=dD, ddelta_bias=dbias)
+    st = lib.ss2d_selective_scan_bwd_ex(ctypes.byref(d), _p(u), _p(delta), _p(A), _p(B), _p(C), _p(D), _p(z),
+                                        _p(delta_bias), int(bool(delta_softplus)), _p(dout), _p(chunk_states),
+                                        _p(du), _p(ddelta), _p(dA), _p(dB), _p(dC), _p(dD), _p(dbias), _p(dz),
+                                        _p(ws), nbytes, _stream(u))
+    _check(st, "ss2d_selective_scan_bwd_ex")
+    return dict(du=du, ddelta=ddelta, dA=dA, dB=dB, dC=dC, dD=dD, ddelta_bias=dbias, dz=dz)
+
+
+class SelectiveScanFunction(torch.autograd.Function):
+    """autograd wrapper of the scan with selective_scan_fn's arguments ("vision mamba-yolov8",
+    section "2. Vmamba module code", SelectiveScanFn): the forward keeps the chunk states, the
+    backward rebuilds the states from them; the last state carries no gradient."""
+
+    @staticmethod
+    def forward(ctx, u, delta, A, B, C, D, z, delta_bias, delta_softplus, return_last_state):
+        out, last, cs = selective_scan_fwd(u, delta, A, B, C, D, delta_bias, delta_softplus, z=z,
+                                           return_last_state=True, return_chunk_states=True)
+        ctx.save_for_backward(u, delta, A, B, C, D, z, delta_bias, cs)
+        ctx.delta_softplus = delta_softplus
+        if not return_last_state:
+            return out
+        ctx.mark_non_differentiable(last)
+        return out, last
+
+    @staticmethod
+    def backward(ctx, dout, *unused):
+        u, delta, A, B, C, D, z, delta_bias, cs = ctx.saved_tensors
+        g = selective_scan_bwd(u, delta, A, B, C, D, delta_bias, ctx.delta_softplus, dout.to(u.dtype),
+                               chunk_states=cs, z=z)
+        return (g["du"], g["ddelta"], g["dA"], g["dB"], g["dC"], g["dD"], g["dz"], g["ddelta_bias"], None, None)
+
+
+def selective_scan_fn(u, delta, A, B, C, D=None, z=None, delta_bias=None, delta_softplus=False,
+                      return_last_state=False):
+    """Differentiable S6 scan over the (Bn, 4*dim, L) sequences of an SS2D problem, with the
+    argument order of the pages' selective_scan_fn.  B and C carry the 4 path groups
+    (Bn, 4, N, L).  Returns out, or (out, last_state) with last_state (Bn, 4*dim, N) fp32."""
+    return SelectiveScanFunction.apply(u, delta, A, B, C, D, z, delta_bias, delta_softplus, return_last_state)
 
 
 # ------------------------------------------------------------------ fused --

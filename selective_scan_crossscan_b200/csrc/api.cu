@@ -193,12 +193,15 @@ static ss2d_status_t check_scan_inputs(const void *u, const void *delta, const f
     return SS2D_OK;
 }
 
-ss2d_status_t ss2d_selective_scan_fwd(const ss2d_desc_t *desc, const void *u, const void *delta, const float *A,
-                                      const void *Bm, const void *Cm, const float *D, const float *delta_bias,
-                                      int delta_softplus, void *out, float *chunk_states, ss2d_stream_t stream) {
+ss2d_status_t ss2d_selective_scan_fwd_ex(const ss2d_desc_t *desc, const void *u, const void *delta, const float *A,
+                                         const void *Bm, const void *Cm, const float *D, const void *z,
+                                         const float *delta_bias, int delta_softplus, void *out,
+                                         float *last_state, float *chunk_states, ss2d_stream_t stream) {
     SS2D_TRY(check_desc(desc));
     SS2D_TRY(check_scan_inputs(u, delta, A, Bm, Cm, D, delta_bias));
+    SS2D_TRY(optional(z));
     SS2D_TRY(need(out));
+    SS2D_TRY(optional(last_state));
     SS2D_TRY(optional(chunk_states));
     const LaunchShape s = shape_of(desc);
     SS2D_TRY(check_device());
@@ -213,6 +216,8 @@ ss2d_status_t ss2d_selective_scan_fwd(const ss2d_desc_t *desc, const void *u, co
     a.softplus = delta_softplus != 0;
     a.out = out;
     a.chunk_states = chunk_states;
+    a.z = z;
+    a.last_state = last_state;
     a.from_image = false;
     a.in_dtype = desc->in_dtype;
     a.out_dtype = desc->out_dtype;
@@ -220,14 +225,22 @@ ss2d_status_t ss2d_selective_scan_fwd(const ss2d_desc_t *desc, const void *u, co
     return from_cuda(launch_scan_fwd(s, a, nullptr, (cudaStream_t)stream));
 }
 
-ss2d_status_t ss2d_selective_scan_bwd(const ss2d_desc_t *desc, const void *u, const void *delta, const float *A,
+ss2d_status_t ss2d_selective_scan_fwd(const ss2d_desc_t *desc, const void *u, const void *delta, const float *A,
                                       const void *Bm, const void *Cm, const float *D, const float *delta_bias,
-                                      int delta_softplus, const void *dout, const float *chunk_states, void *du,
-                                      void *ddelta, float *dA, void *dBm, void *dCm, float *dD,
-                                      float *ddelta_bias, void *workspace, size_t workspace_bytes,
-                                      ss2d_stream_t stream) {
+                                      int delta_softplus, void *out, float *chunk_states, ss2d_stream_t stream) {
+    return ss2d_selective_scan_fwd_ex(desc, u, delta, A, Bm, Cm, D, nullptr, delta_bias, delta_softplus, out,
+                                      nullptr, chunk_states, stream);
+}
+
+ss2d_status_t ss2d_selective_scan_bwd_ex(const ss2d_desc_t *desc, const void *u, const void *delta, const float *A,
+                                         const void *Bm, const void *Cm, const float *D, const void *z,
+                                         const float *delta_bias, int delta_softplus, const void *dout,
+                                         const float *chunk_states, void *du, void *ddelta, float *dA, void *dBm,
+                                         void *dCm, float *dD, float *ddelta_bias, void *dz, void *workspace,
+                                         size_t workspace_bytes, ss2d_stream_t stream) {
     SS2D_TRY(check_desc(desc));
     SS2D_TRY(check_scan_inputs(u, delta, A, Bm, Cm, D, delta_bias));
+    SS2D_TRY(optional(z));
     SS2D_TRY(need(dout));
     SS2D_TRY(optional(chunk_states));
     SS2D_TRY(need(du));
@@ -237,8 +250,10 @@ ss2d_status_t ss2d_selective_scan_bwd(const ss2d_desc_t *desc, const void *u, co
     SS2D_TRY(need(dCm));
     if ((D == nullptr) != (dD == nullptr)) return SS2D_ERR_NULL;
     if ((delta_bias == nullptr) != (ddelta_bias == nullptr)) return SS2D_ERR_NULL;
+    if ((z == nullptr) != (dz == nullptr)) return SS2D_ERR_NULL;
     SS2D_TRY(optional(dD));
     SS2D_TRY(optional(ddelta_bias));
+    SS2D_TRY(optional(dz));
     const LaunchShape s = shape_of(desc);
     const size_t ws = scan_bwd_workspace_bytes(s);
     if (ws > 0 && (!workspace || workspace_bytes < ws)) return SS2D_ERR_WORKSPACE;
@@ -262,10 +277,23 @@ ss2d_status_t ss2d_selective_scan_bwd(const ss2d_desc_t *desc, const void *u, co
     a.dCm = dCm;
     a.dD = dD;
     a.dbias = ddelta_bias;
+    a.z = z;
+    a.dz = dz;
     a.from_image = false;
     a.in_dtype = desc->in_dtype;
     a.out_dtype = desc->out_dtype;
     return from_cuda(launch_scan_bwd(s, a, workspace, workspace_bytes, (cudaStream_t)stream));
+}
+
+ss2d_status_t ss2d_selective_scan_bwd(const ss2d_desc_t *desc, const void *u, const void *delta, const float *A,
+                                      const void *Bm, const void *Cm, const float *D, const float *delta_bias,
+                                      int delta_softplus, const void *dout, const float *chunk_states, void *du,
+                                      void *ddelta, float *dA, void *dBm, void *dCm, float *dD,
+                                      float *ddelta_bias, void *workspace, size_t workspace_bytes,
+                                      ss2d_stream_t stream) {
+    return ss2d_selective_scan_bwd_ex(desc, u, delta, A, Bm, Cm, D, nullptr, delta_bias, delta_softplus, dout,
+                                      chunk_states, du, ddelta, dA, dBm, dCm, dD, ddelta_bias, nullptr, workspace,
+                                      workspace_bytes, stream);
 }
 
 ss2d_status_t ss2d_forward(const ss2d_desc_t *desc, const void *x, const void *delta, const float *A,

@@ -172,10 +172,11 @@ __device__ __forceinline__ float2 ex2_poly2(float2 x) {
                        __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
 }
 
-// d softplus / dt = sigmoid(t)
-__device__ __forceinline__ float sigmoid_f(float t) {
-    return 1.f / (1.f + ex2_sfu(-t * kLog2e));
-}
+// sigmoid(t) = 1 / (1 + e^{-t}) (= d softplus / dt); for t -> -inf, e^{-t} -> inf and the result -> 0
+__device__ __forceinline__ float sigmoid_f(float t) { return rcp_approx(1.f + ex2_sfu(-t * kLog2e)); }
+
+// silu(z) = z * sigmoid(z), the output gate of the selective scan
+__device__ __forceinline__ float silu_f(float z) { return z * sigmoid_f(z); }
 
 __host__ __device__ __forceinline__ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 

@@ -36,7 +36,9 @@ struct ScanFwdArgs {
     const float *bias;   // (4D) or null
     int softplus;
     void *out;           // (B, 4D, L)
-    float *chunk_states; // (B, 4D, ceil(L/64), N) or null
+    float *chunk_states; // (B, 4D, ceil(L/SS2D_CHUNK_LEN), N) or null
+    const void *z = nullptr;      // (B, 4D, L) output gate, out *= silu(z); sequences only
+    float *last_state = nullptr;  // (B, 4D, N) state after the last step, or null
     bool from_image;     // read u along path k from the image (fused CrossScan)
     ss2d_dtype_t in_dtype, out_dtype;
     int max_segments = 32;  // 1 = never split a sequence (no workspace needed)
@@ -70,6 +72,8 @@ struct ScanBwdArgs {
     void *dCm;
     float *dD;
     float *dbias;
+    const void *z = nullptr;  // (B, 4D, L) output gate of the forward; sequences only
+    void *dz = nullptr;       // (B, 4D, L) in_dtype, written when z is given
     bool from_image;
     ss2d_dtype_t in_dtype, out_dtype;
 };

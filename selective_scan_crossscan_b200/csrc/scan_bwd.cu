@@ -34,6 +34,8 @@
 // and written as one partial per (b, k, 64-channel tile); a second kernel sums
 // the partials over tiles, and dA, dD, ddelta_bias over the batch, in a fixed
 // order -- no float atomics, deterministic results.
+#include <cstddef>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -63,8 +65,10 @@ struct BwdParams {
     const void *dout;   // (B, 4D, L), or image dy (B, D, H, W)
     const void *doutT;  // transposed dy (image mode, column paths)
     const float *cs;    // (B, 4D, nchunks, N)
+    const void *z;      // (B, 4D, L) output gate of the forward, or null (sequences only)
     void *du;
     void *ddelta;
+    void *dz;           // (B, 4D, L) in_dtype, when z is given
     float *part_bc;     // (B, 4, ntiles, 2N, L)
     float *part_p;      // (B, 4D, N + 2): dA (N), dD, ddelta_bias partials
     int64_t B, D, H, W, L;
@@ -81,40 +85,47 @@ struct BwdCtaSmem {
     float Cs[kBlk][NS + 4];
 };
 
-template <int NS>
-struct BwdWarpSmem {
+template <int NS, bool GATE>
+struct alignas(16) BwdWarpSmem {
     static constexpr int HS = NS / 2;  // states per lane
     static constexpr int kRow = kBlk + 1;
     float U[kChPerWarp][kRow];
     float DT[kChPerWarp][kRow];
     float DTU[kChPerWarp][kRow];
     float SG[kChPerWarp][kRow];  // delta, then d softplus / d delta, then ddelta
-    float G[kChPerWarp][kRow];   // dout, then du
+    float G[kChPerWarp][kRow];   // dout (times silu(z) under a gate), then du
+    float GZ[GATE ? kChPerWarp : 1][kRow];  // gate: z, then dout silu'(z), then dz
     float2 ck[kNSub][HS / 2][32];  // per-lane state checkpoints, lanes fastest (conflict-free)
-    float red[kChPerWarp][4 * NS + 4];  // [channel][output o][2 steps]
+    alignas(16) float red[kChPerWarp][4 * NS + 4];  // [channel][output o][2 steps]; 128-bit stores
     float bct[kBlk][2 * NS];     // channel sums of this warp: [step][dB n | dC n]
 };
 
-template <int NS>
+template <int NS, bool GATE>
 constexpr size_t bwd_smem_bytes() {
-    return sizeof(BwdCtaSmem<NS>) + kWarps * sizeof(BwdWarpSmem<NS>);
+    // the 128-bit stores into red need it 16-byte aligned in every warp's slice of the dynamic
+    // shared memory (which follows the CTA part)
+    using W = BwdWarpSmem<NS, GATE>;
+    static_assert(offsetof(W, red) % 16 == 0 && sizeof(W) % 16 == 0, "warp slice alignment");
+    static_assert(sizeof(BwdCtaSmem<NS>) % 16 == 0, "CTA part alignment");
+    return sizeof(BwdCtaSmem<NS>) + kWarps * sizeof(W);
 }
 
 // The warp's channels: u, delta, dout of 16 channels x 16 steps.  Every load is issued
 // before the first shared-memory store so that their latencies overlap.
-template <int NS, typename Tin, typename Tg, bool IMG>
-__device__ __forceinline__ void stage_channels(BwdWarpSmem<NS> &sm, const BwdParams &p, int64_t b, int k,
+template <int NS, typename Tin, typename Tg, bool IMG, bool GATE>
+__device__ __forceinline__ void stage_channels(BwdWarpSmem<NS, GATE> &sm, const BwdParams &p, int64_t b, int k,
                                                int64_t dw0, int nch, int64_t l0, int len) {
     constexpr int kPer = kChPerWarp * kBlk / 32;
     const int lane = threadIdx.x & 31;
     const int64_t D = p.D, L = p.L, C4 = kPaths * p.D;
     const bool rev = IMG && k >= 2;
-    float uv[kPer], dv[kPer], gv[kPer];
+    float uv[kPer], dv[kPer], gv[kPer], zv[GATE ? kPer : 1];
 #pragma unroll
     for (int t = 0; t < kPer; ++t) {
         const int idx = lane + 32 * t;
         const int ci = idx / kBlk, i = idx % kBlk;
         uv[t] = dv[t] = gv[t] = 0.f;
+        if (GATE) zv[t] = 0.f;
         if (ci < nch && i < len) {
             const int64_t l = l0 + i;
             const int64_t cc = k * D + dw0 + ci;
@@ -129,6 +140,7 @@ __device__ __forceinline__ void stage_channels(BwdWarpSmem<NS> &sm, const BwdPar
             } else {
                 uv[t] = ld(static_cast<const Tin *>(p.u) + (b * C4 + cc) * L + l);
                 gv[t] = ld(static_cast<const Tg *>(p.dout) + (b * C4 + cc) * L + l);
+                if (GATE) zv[t] = ld(static_cast<const Tin *>(p.z) + (b * C4 + cc) * L + l);
             }
         }
     }
@@ -139,6 +151,7 @@ __device__ __forceinline__ void stage_channels(BwdWarpSmem<NS> &sm, const BwdPar
         sm.U[ci][i] = uv[t];
         sm.SG[ci][i] = dv[t];
         sm.G[ci][i] = gv[t];
+        if (GATE) sm.GZ[ci][i] = zv[t];
     }
 }
 
@@ -171,15 +184,16 @@ __device__ __forceinline__ void stage_bc(BwdCtaSmem<NS> &cs, const BwdParams &p,
     }
 }
 
-template <int NS, typename Tin, typename Tg, typename Tdu, bool IMG>
+template <int NS, typename Tin, typename Tg, typename Tdu, bool IMG, bool GATE>
 __global__ void __launch_bounds__(32 * kWarps, SS2D_BWD_MIN_BLOCKS) scan_bwd_kernel(const BwdParams p) {
+    static_assert(!(IMG && GATE), "the output gate belongs to the sequence form");
     constexpr int HS = NS / 2;
     constexpr int HP = HS / 2;  // state pairs per lane
     extern __shared__ __align__(16) unsigned char smem_raw[];
     BwdCtaSmem<NS> &csm = *reinterpret_cast<BwdCtaSmem<NS> *>(smem_raw);
-    BwdWarpSmem<NS> *wsm = reinterpret_cast<BwdWarpSmem<NS> *>(smem_raw + sizeof(BwdCtaSmem<NS>));
+    BwdWarpSmem<NS, GATE> *wsm = reinterpret_cast<BwdWarpSmem<NS, GATE> *>(smem_raw + sizeof(BwdCtaSmem<NS>));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    BwdWarpSmem<NS> &sm = wsm[warp];
+    BwdWarpSmem<NS, GATE> &sm = wsm[warp];
 
     const int ci = lane >> 1, hf = lane & 1;  // channel within the warp, state half
     const int k = blockIdx.y;
@@ -225,8 +239,20 @@ __global__ void __launch_bounds__(32 * kWarps, SS2D_BWD_MIN_BLOCKS) scan_bwd_ker
             }
         }
         stage_bc<NS, Tin>(csm, p, b, k, l0, len);
-        stage_channels<NS, Tin, Tg, IMG>(sm, p, b, k, dw0, nch, l0, len);
+        stage_channels<NS, Tin, Tg, IMG, GATE>(sm, p, b, k, dw0, nch, l0, len);
         __syncthreads();  // B, C of the block are staged for all warps
+        // gate: the scan's output o reaches the loss as o * silu(z), so dout * silu(z) drives the
+        // adjoint and dz = dout * silu'(z) * o (o is rebuilt in the adjoint walk)
+        if (GATE) {
+#pragma unroll
+            for (int j = 0; j < kBlk / 2; ++j) {
+                const int i = hf * (kBlk / 2) + j;
+                const float zz = sm.GZ[ci][i], go = sm.G[ci][i];
+                const float sg = sigmoid_f(zz);
+                sm.G[ci][i] = go * (zz * sg);
+                sm.GZ[ci][i] = go * (sg * fmaf(zz, 1.f - sg, 1.f));
+            }
+        }
         // pre-pass: dt, dt*u, d softplus / d delta for each (channel, step), lanes hf split the steps
         if (p.softplus) {
 #pragma unroll
@@ -312,11 +338,12 @@ __global__ void __launch_bounds__(32 * kWarps, SS2D_BWD_MIN_BLOCKS) scan_bwd_ker
                 const float uv = sm.U[ci][i];
                 // with t = lambda a_l h_{l-1}: dA += dt t, ddt = sum A t + u sum lambda B,
                 // du = g D + dt sum lambda B
-                float2 sA = make_float2(0.f, 0.f), sB = make_float2(0.f, 0.f);
+                float2 sA = make_float2(0.f, 0.f), sB = make_float2(0.f, 0.f), so = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int q = 0; q < HP; ++q) {
                     const float2 bb = *reinterpret_cast<const float2 *>(&csm.Bs[i][n0 + 2 * q]);
                     const float2 cc = *reinterpret_cast<const float2 *>(&csm.Cs[i][n0 + 2 * q]);
+                    if (GATE) so = __ffma2_rn(cc, hist[jj][q], so);  // C_l . h_l
                     lam[q] = __ffma2_rn(cc, make_float2(g, g), lam[q]);
                     // a_l h_{l-1} = h_l - dt u B, with dt u B rounded as in the recompute (an add of the
                     // rounded product could be contracted into an unrounded FFMA; as an FFMA's
@@ -331,9 +358,10 @@ __global__ void __launch_bounds__(32 * kWarps, SS2D_BWD_MIN_BLOCKS) scan_bwd_ker
                     vc[e][q] = __fmul2_rn(make_float2(g, g), hist[jj][q]);
                     lam[q] = __fmul2_rn(lam[q], dec[jj][q]);
                 }
-                float sa = sA.x + sA.y, sb = sB.x + sB.y;
+                float sa = sA.x + sA.y, sb = sB.x + sB.y, yo = so.x + so.y;
                 sa += __shfl_xor_sync(0xffffffffu, sa, 1);  // the other half of the states
                 sb += __shfl_xor_sync(0xffffffffu, sb, 1);
+                if (GATE) yo += __shfl_xor_sync(0xffffffffu, yo, 1);
                 if (hf == 0 && active) {
                     const float ddt = fmaf(kLn2, sa, uv * sb);  // A = A2 ln 2
                     const float dd = ddt * sm.SG[ci][i];
@@ -341,6 +369,7 @@ __global__ void __launch_bounds__(32 * kWarps, SS2D_BWD_MIN_BLOCKS) scan_bwd_ker
                     dD = fmaf(g, uv, dD);
                     sm.SG[ci][i] = dd;
                     sm.G[ci][i] = fmaf(g, Dc, dt * sb);
+                    if (GATE) sm.GZ[ci][i] *= fmaf(Dc, uv, yo);  // dz = dout silu'(z) (C.h + D u)
                 }
             };
             // transpose two steps' contributions, red[ci][o][e] (o = state for dB, NS + state for dC),
@@ -411,6 +440,7 @@ __global__ void __launch_bounds__(32 * kWarps, SS2D_BWD_MIN_BLOCKS) scan_bwd_ker
                 const int64_t cc = k * D + dw0 + cw;
                 st(du_out + (b * C4 + cc) * L + l0 + i, sm.G[cw][i]);
                 st(dd_out + (b * C4 + cc) * L + l0 + i, sm.SG[cw][i]);
+                if (GATE) st(static_cast<Tin *>(p.dz) + (b * C4 + cc) * L + l0 + i, sm.GZ[cw][i]);
             }
         }
         float *pbc = p.part_bc + ((b * kPaths + k) * p.ntiles + blockIdx.x) * (int64_t)(2 * N) * L;
@@ -493,10 +523,10 @@ size_t scan_bwd_workspace_bytes(const LaunchShape &s) {
     return bytes;
 }
 
-template <int NS, typename Tin, typename Tg, typename Tdu, bool IMG>
+template <int NS, typename Tin, typename Tg, typename Tdu, bool IMG, bool GATE>
 static cudaError_t launch_bwd_t(const LaunchShape &s, const BwdParams &p, cudaStream_t stream) {
-    const size_t smem = bwd_smem_bytes<NS>();
-    auto kern = scan_bwd_kernel<NS, Tin, Tg, Tdu, IMG>;
+    const size_t smem = bwd_smem_bytes<NS, GATE>();
+    auto kern = scan_bwd_kernel<NS, Tin, Tg, Tdu, IMG, GATE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)bwd_tiles(s), kPaths, (unsigned)s.B);
@@ -505,11 +535,17 @@ static cudaError_t launch_bwd_t(const LaunchShape &s, const BwdParams &p, cudaSt
     return cudaGetLastError();
 }
 
+template <typename Tin, typename Tg, typename Tdu, bool IMG, bool GATE>
+static cudaError_t launch_bwd_gate(const LaunchShape &s, const BwdParams &p, cudaStream_t stream) {
+    if (s.N <= 4) return launch_bwd_t<4, Tin, Tg, Tdu, IMG, GATE>(s, p, stream);
+    if (s.N <= 8) return launch_bwd_t<8, Tin, Tg, Tdu, IMG, GATE>(s, p, stream);
+    return launch_bwd_t<16, Tin, Tg, Tdu, IMG, GATE>(s, p, stream);
+}
+
 template <typename Tin, typename Tg, typename Tdu, bool IMG>
 static cudaError_t launch_bwd_ns(const LaunchShape &s, const BwdParams &p, cudaStream_t stream) {
-    if (s.N <= 4) return launch_bwd_t<4, Tin, Tg, Tdu, IMG>(s, p, stream);
-    if (s.N <= 8) return launch_bwd_t<8, Tin, Tg, Tdu, IMG>(s, p, stream);
-    return launch_bwd_t<16, Tin, Tg, Tdu, IMG>(s, p, stream);
+    if (!IMG && p.z) return launch_bwd_gate<Tin, Tg, Tdu, false, true>(s, p, stream);
+    return launch_bwd_gate<Tin, Tg, Tdu, IMG, false>(s, p, stream);
 }
 
 template <typename Tin, typename Tg, bool IMG>
@@ -580,8 +616,10 @@ cudaError_t launch_scan_bwd(const LaunchShape &s, const ScanBwdArgs &a, void *wo
     p.dout = a.dout;
     p.doutT = a.doutT;
     p.cs = cs;
+    p.z = a.from_image ? nullptr : a.z;
     p.du = a.du;
     p.ddelta = a.ddelta;
+    p.dz = a.dz;
     p.part_bc = part_bc;
     p.part_p = part_p;
     p.B = s.B;

@@ -76,6 +76,8 @@ struct FwdParams {
     const float *bias;
     void *out;
     float *chunk_states;
+    const void *z;       // (B, 4D, L) output gate or null (sequence mode only)
+    float *last_state;   // (B, 4D, N) or null
     float *seg;  // (B, 4D, nseg, 2, N): decay product and end state of each segment
     int64_t B, D, H, W, L;
     int N;
@@ -341,7 +343,19 @@ __global__ void __launch_bounds__(kWarp, SS2D_FWD_MIN_BLOCKS) scan_fwd_kernel(co
                 if (PASS == 1) {
                     dtsum += (dt01.x + dt01.y) + (dt23.x + dt23.y);
                 } else {
-                    const float y[kG] = {y01.x, y01.y, y23.x, y23.y};
+                    float y[kG] = {y01.x, y01.y, y23.x, y23.y};
+                    if (!IMG && p.z) {  // output gate: y * silu(z), after the D u term
+                        const Tin *zrow = static_cast<const Tin *>(p.z) + (b * C4 + c) * L;
+                        float zv[kG];
+                        if (VEC) {
+                            ld4(zrow + l0, zv);
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < kG; ++j) zv[j] = j < nvalid ? ld(zrow + l0 + j) : 0.f;
+                        }
+#pragma unroll
+                        for (int j = 0; j < kG; ++j) y[j] *= silu_f(zv[j]);
+                    }
                     if (orow) {
                         if (VEC) {
                             st4(orow + l0, y);
@@ -364,6 +378,12 @@ __global__ void __launch_bounds__(kWarp, SS2D_FWD_MIN_BLOCKS) scan_fwd_kernel(co
         __syncwarp();  // every lane is done with this buffer before it is refilled
     }
 
+    if (!IMG && PASS != 1 && active && p.last_state && sgi == p.nseg - 1) {  // sequence mode only
+        float *ls = p.last_state + (b * C4 + c) * N;
+#pragma unroll
+        for (int n = 0; n < NS; ++n)
+            if (n < N) ls[n] = h[n];
+    }
     if (PASS == 1 && active) {
         float *sg = p.seg + ((b * C4 + c) * (int64_t)p.nseg + sgi) * 2 * N;
 #pragma unroll
@@ -451,6 +471,8 @@ cudaError_t launch_scan_fwd(const LaunchShape &s, const ScanFwdArgs &a, void *wo
     p.bias = a.bias;
     p.out = a.out;
     p.chunk_states = a.chunk_states;
+    p.z = a.from_image ? nullptr : a.z;
+    p.last_state = a.from_image ? nullptr : a.last_state;
     p.seg = static_cast<float *>(workspace);
     p.B = s.B;
     p.D = s.D;

@@ -141,9 +141,10 @@ def batch_slice(inputs: dict, idx) -> dict:
     return out
 
 
-def make_scan_inputs(w: Workload, seed: int = 0, device="cpu", with_dout: bool = False):
+def make_scan_inputs(w: Workload, seed: int = 0, device="cpu", with_dout: bool = False, with_z: bool = False):
     """Inputs for the standalone S6 scan in its sequence view: u (B, 4D, L) drawn directly
-    (N(0,1)) instead of an image, the other tensors as in make_inputs.  dout ~ N(0,1) if asked."""
+    (N(0,1)) instead of an image, the other tensors as in make_inputs.  dout ~ N(0,1) if asked;
+    the output gate z ~ N(0,1) (B, 4D, L) if asked, drawn last so the other tensors do not change."""
     g = torch.Generator(device=device)
     g.manual_seed(int(seed) + 1000)
     f32 = dict(dtype=torch.float32, device=device, generator=g)
@@ -154,8 +155,10 @@ def make_scan_inputs(w: Workload, seed: int = 0, device="cpu", with_dout: bool =
     out["u"] = u
     if with_dout:
         out["dout"] = torch.randn((w.batch, K_PATHS * w.dim, w.L), **f32)
+    if with_z:
+        out["z"] = torch.randn((w.batch, K_PATHS * w.dim, w.L), **f32)
     if w.dtype == "bf16":
-        for key in ("u", "dout"):
+        for key in ("u", "dout", "z"):
             if key in out:
                 out[key] = out[key].to(torch.bfloat16)
     return out

@@ -94,6 +94,25 @@ def test_backward_argument_errors(lib):
     assert ff(_d(), *args, None, None, 1, B16, None, A16, wsf - 1, None) == ERR_WORKSPACE
 
 
+def test_gated_scan_argument_errors(lib):
+    # ss2d_selective_scan_fwd_ex / _bwd_ex: z and last_state are optional but must be aligned;
+    # dz must be given exactly when z is
+    mis = ctypes.c_void_p(0x10004)
+    f = lib.ss2d_selective_scan_fwd_ex
+    args = [A16] * 5
+    assert f(_d(), *args, None, mis, None, 1, B16, None, None, None) == ERR_ALIGN  # z
+    assert f(_d(), *args, None, None, None, 1, B16, mis, None, None) == ERR_ALIGN  # last_state
+    assert f(_d(), *args, None, A16, None, 1, None, A16, None, None) == ERR_NULL   # out
+    g = lib.ss2d_selective_scan_bwd_ex
+    ws = lib.ss2d_workspace_bytes(_d(), ss.OP_SELECTIVE_SCAN_BWD)
+    grads = [A16] * 5  # du, ddelta, dA, dB, dC
+    assert g(_d(), *args, None, A16, None, 1, A16, None, *grads, None, None, None, A16, ws, None) == ERR_NULL
+    assert g(_d(), *args, None, None, None, 1, A16, None, *grads, None, None, A16, A16, ws, None) == ERR_NULL
+    assert g(_d(), *args, None, mis, None, 1, A16, None, *grads, None, None, A16, A16, ws, None) == ERR_ALIGN
+    assert g(_d(), *args, None, A16, None, 1, A16, None, *grads, None, None, A16, A16, ws - 1,
+             None) == ERR_WORKSPACE
+
+
 def test_valid_call_without_gpu_reports_device_error(lib):
     import torch
     if torch.cuda.is_available():

@@ -206,6 +206,109 @@ def test_selective_scan_bwd_without_optional():
         assert_rel_l2(g[name], ref[name], GRAD_TOL, name)
 
 
+# ------------------------------------------- output gate and last state
+
+def _gated_case(Bn, Dn, H, W, N, dtype="f32", seed=0):
+    w = ss2d_inputs.custom(Bn, Dn, H, W, N, dtype=dtype)
+    return w, ss2d_inputs.make_scan_inputs(w, seed=seed, with_dout=True, with_z=True)
+
+
+GATED_CASES = [(1, 8, 8, 8, 4), (2, 40, 5, 7, 16), (1, 3, 1, 1, 3), (1, 33, 4, 50, 8), (2, 4, 3, 43, 16)]
+
+
+@pytest.mark.parametrize("case", GATED_CASES)
+def test_selective_scan_fwd_gate_and_last_state(case):
+    w, inp = _gated_case(*case, seed=30)
+    d = _dev(inp)
+    out, last, cs = ss.selective_scan_fwd(d["u"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["delta_bias"], True,
+                                          z=d["z"], return_last_state=True, return_chunk_states=True)
+    ref, ref_last = oracle.selective_scan_fwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"],
+                                              inp["delta_bias"], True, return_last_state=True, z=inp["z"])
+    assert_rel_l2(out, ref, FWD_TOL, f"{case} out")
+    assert_rel_l2(last, ref_last, FWD_TOL, f"{case} last_state")
+    # the last state is the final chunk state, bit for bit
+    assert torch.equal(last, cs[:, :, -1, :])
+
+
+def test_last_state_without_gate_and_gate_without_last_state():
+    w, inp = _gated_case(2, 6, 7, 9, 16, seed=31)
+    d = _dev(inp)
+    plain = ss.selective_scan_fwd(d["u"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["delta_bias"], True)
+    out, last = ss.selective_scan_fwd(d["u"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["delta_bias"], True,
+                                      return_last_state=True)
+    assert torch.equal(out, plain)  # the last state changes nothing else
+    _, ref_last = oracle.selective_scan_fwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"],
+                                            inp["delta_bias"], True, return_last_state=True)
+    assert_rel_l2(last, ref_last, FWD_TOL, "last_state")
+    gated = ss.selective_scan_fwd(d["u"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["delta_bias"], True,
+                                  z=d["z"])
+    ref = oracle.selective_scan_fwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"],
+                                    inp["delta_bias"], True, z=inp["z"])
+    assert_rel_l2(gated, ref, FWD_TOL, "gated out")
+
+
+def test_gate_extremes():
+    # z = 0 gives exactly 0; very negative z gives (-)0, not NaN; large z passes the output through
+    w, inp = _gated_case(1, 4, 4, 16, 8, seed=32)
+    d = _dev(inp)
+    args = (d["u"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["delta_bias"], True)
+    plain = ss.selective_scan_fwd(*args)
+    assert torch.all(ss.selective_scan_fwd(*args, z=torch.zeros_like(d["u"])) == 0)
+    neg = ss.selective_scan_fwd(*args, z=torch.full_like(d["u"], -200.0))
+    assert torch.all(neg == 0) and not torch.isnan(neg).any()
+    big = ss.selective_scan_fwd(*args, z=torch.full_like(d["u"], 60.0))
+    torch.testing.assert_close(big, 60.0 * plain, rtol=2e-6, atol=0)
+
+
+GATED_BWD_NAMES = BWD_NAMES + [("dz", "dz")]
+
+
+@pytest.mark.parametrize("case", GATED_CASES)
+@pytest.mark.parametrize("with_states", [False, True])
+def test_selective_scan_bwd_gated_parity(case, with_states):
+    w, inp = _gated_case(*case, seed=33)
+    d = _dev(inp)
+    cs = None
+    if with_states:
+        _, cs = ss.selective_scan_fwd(d["u"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["delta_bias"], True,
+                                      z=d["z"], return_chunk_states=True)
+    g = ss.selective_scan_bwd(d["u"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["delta_bias"], True, d["dout"],
+                              chunk_states=cs, z=d["z"])
+    ref = oracle.selective_scan_bwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"],
+                                    inp["delta_bias"], True, inp["dout"], z=inp["z"])
+    for name, rname in GATED_BWD_NAMES:
+        assert_rel_l2(g[name], ref[rname], GRAD_TOL, f"{case} {name}")
+
+
+def test_gated_bwd_bf16():
+    w, inp = _gated_case(2, 8, 6, 20, 16, dtype="bf16", seed=34)
+    d = _dev(inp)
+    g = ss.selective_scan_bwd(d["u"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["delta_bias"], True, d["dout"],
+                              z=d["z"])
+    assert g["dz"].dtype == torch.bfloat16
+    ref = oracle.selective_scan_bwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"],
+                                    inp["delta_bias"], True, inp["dout"], z=inp["z"])
+    for name, rname in GATED_BWD_NAMES:
+        assert_rel_l2(g[name], ref[rname], BF16_TOL, name)
+
+
+def test_selective_scan_fn_autograd():
+    # the pages' selective_scan_fn call: gated output and last state; backward through autograd
+    w, inp = _gated_case(2, 5, 6, 13, 16, seed=35)
+    d = _dev(inp)
+    leaves = {k: d[k].clone().requires_grad_(True) for k in ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")}
+    out, last = ss.selective_scan_fn(leaves["u"], leaves["delta"], leaves["A"], leaves["B"], leaves["C"],
+                                     leaves["D"], z=leaves["z"], delta_bias=leaves["delta_bias"],
+                                     delta_softplus=True, return_last_state=True)
+    assert not last.requires_grad
+    out.backward(d["dout"])
+    ref = oracle.selective_scan_bwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"],
+                                    inp["delta_bias"], True, inp["dout"], z=inp["z"])
+    names = dict(u="du", delta="ddelta", A="dA", B="dB", C="dC", D="dD", z="dz", delta_bias="ddelta_bias")
+    for k, rname in names.items():
+        assert_rel_l2(leaves[k].grad, ref[rname], GRAD_TOL, k)
+
+
 # ------------------------------------------------------------- fused SS2D
 
 FUSED_CASES = [(1, 8, 8, 8, 4), (2, 6, 5, 9, 16), (1, 70, 12, 11, 16), (1, 8, 64, 64, 16), (2, 3, 1, 1, 2),
