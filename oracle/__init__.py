@@ -156,6 +156,54 @@ def selective_scan_bwd(u, delta, A, B, C, D, delta_bias, delta_softplus, dout, z
     return dict(du=du, ddelta=ddelta, dA=dA, dB=dB, dC=dC, dD=dD, ddelta_bias=dbias, dz=dz)
 
 
+def _flip(t):
+    return None if t is None else np.ascontiguousarray(np.flip(t, -1))
+
+
+def _group_axis(B):
+    """B or C given as (Bn, N, L) -> (Bn, 1, N, L); 4-D passes through."""
+    return None if B is None else (B[:, None] if B.ndim == 3 else B)
+
+
+def bimamba_forward(x, delta, A, A_b, B, C, D=None, z=None, delta_bias=None, delta_softplus=True):
+    """Bidirectional scan of bimamba_inner_ref ("vision mamba-yolov8", section "2. Vmamba module
+    code"): one scan over the sequence with A, one over the flipped sequence with A_b (delta, B,
+    C, z flipped too; D and delta_bias shared), the second output flipped back and added.
+
+    x, delta, z (Bn, D, L); A, A_b (D, N); B, C (Bn, N, L) or (Bn, 1, N, L); D, delta_bias (D).
+    """
+    x, delta, A, A_b, B, C = (_f64(t) for t in (x, delta, A, A_b, B, C))
+    D, delta_bias, z = _f64(D), _f64(delta_bias), _f64(z)
+    B4, C4 = _group_axis(B), _group_axis(C)
+    y = selective_scan_fwd(x, delta, A, B4, C4, D, delta_bias, delta_softplus, z=z)
+    y_b = selective_scan_fwd(_flip(x), _flip(delta), A_b, _flip(B4), _flip(C4), D, delta_bias, delta_softplus,
+                             z=_flip(z))
+    return y + _flip(y_b)
+
+
+def bimamba_backward(x, delta, A, A_b, B, C, D, z, delta_bias, delta_softplus, dy):
+    """Gradients of bimamba_forward: the two scans' backward passes, the flipped one's gradients
+    flipped back, shared inputs' gradients added.  Returns dict dx, ddelta, dA, dA_b, dB, dC, dD,
+    ddelta_bias, dz (dB, dC in B's and C's shapes; None where an input is None)."""
+    x, delta, A, A_b, B, C, dy = (_f64(t) for t in (x, delta, A, A_b, B, C, dy))
+    D, delta_bias, z = _f64(D), _f64(delta_bias), _f64(z)
+    B4, C4 = _group_axis(B), _group_axis(C)
+    gf = selective_scan_bwd(x, delta, A, B4, C4, D, delta_bias, delta_softplus, dy, z=z)
+    gb = selective_scan_bwd(_flip(x), _flip(delta), A_b, _flip(B4), _flip(C4), D, delta_bias, delta_softplus,
+                            _flip(dy), z=_flip(z))
+
+    def both(name):
+        return None if gf[name] is None else gf[name] + _flip(gb[name])
+
+    def total(name):
+        return None if gf[name] is None else gf[name] + gb[name]
+
+    dB, dC = both("dB"), both("dC")
+    return dict(dx=both("du"), ddelta=both("ddelta"), dA=gf["dA"], dA_b=gb["dA"],
+                dB=dB.reshape(B.shape), dC=dC.reshape(C.shape), dD=total("dD"),
+                ddelta_bias=total("ddelta_bias"), dz=both("dz"))
+
+
 def ss2d_forward(x, delta, A, B, C, D=None, delta_bias=None, delta_softplus=True):
     """Full SS2D forward.  x (Bn, D, H, W) -> y (Bn, D, H, W)."""
     x, delta, A, B, C = (_f64(t) for t in (x, delta, A, B, C))

@@ -9,7 +9,9 @@ Pins used: hand-tabulated traversal orders and hand-worked S6 values
 recurrence evaluated by brute force, special cases that reduce to library
 routines (cumulative sum, elementwise product), linearity, permutation and
 adjoint identities of the index maps, central finite differences and exact
-dot-product identities for the backward.  The output gate (out times silu(z),
+dot-product identities for the backward.  The bidirectional scan
+(bimamba_inner_ref) is pinned by its mirror symmetry and by the SS2D oracle on a
+one-row image, whose row-major paths are the sequence and its reverse.  The output gate (out times silu(z),
 the last lines of selective_scan_ref) is pinned by its special values, by
 scipy's logistic function and by central differences; the last state by
 reading it back through a one-hot C.
@@ -475,6 +477,75 @@ def test_last_state_unaffected_by_gate(oracle):
     _, a = oracle.selective_scan_fwd(**p, return_last_state=True)
     _, b = oracle.selective_scan_fwd(**p, return_last_state=True, z=rng.standard_normal(p["u"].shape))
     np.testing.assert_array_equal(a, b)
+
+
+# ------------------------------------------------------- bidirectional scan
+
+def _bimamba_problem(rng, Bn=2, Dn=3, L=9, N=4):
+    return dict(x=rng.standard_normal((Bn, Dn, L)), delta=0.3 * rng.standard_normal((Bn, Dn, L)),
+                A=-rng.uniform(0.2, 3.0, (Dn, N)), A_b=-rng.uniform(0.2, 3.0, (Dn, N)),
+                B=rng.standard_normal((Bn, N, L)), C=rng.standard_normal((Bn, N, L)),
+                D=rng.standard_normal(Dn), delta_bias=rng.uniform(-4.0, 0.0, Dn))
+
+
+def test_bimamba_mirror_symmetry(oracle):
+    # with A_b = A and mirror-symmetric inputs the two directions see the same sequence, so the
+    # output is mirror-symmetric; with A_b != A it is not
+    rng = _rng(51)
+    p = _bimamba_problem(rng)
+    for k in ("x", "delta", "B", "C"):
+        p[k] = p[k] + np.flip(p[k], -1)
+    z = rng.standard_normal(p["x"].shape)
+    z = z + np.flip(z, -1)
+    y = oracle.bimamba_forward(**dict(p, A_b=p["A"]), z=z)
+    np.testing.assert_allclose(y, np.flip(y, -1), rtol=1e-13, atol=1e-13)
+    y2 = oracle.bimamba_forward(**p, z=z)
+    assert np.abs(y2 - np.flip(y2, -1)).max() > 1e-3
+
+
+def test_bimamba_is_half_of_ss2d_on_one_row(oracle):
+    # a 1 x L image: SS2D's paths 0 and 1 are the sequence itself, 2 and 3 its reverse.  Give the
+    # reversed paths A_b and the reversed delta/B/C, and SS2D sums each direction twice.
+    rng = _rng(52)
+    Bn, Dn, L, N = 2, 3, 11, 4
+    p = _bimamba_problem(rng, Bn, Dn, L, N)
+    y = oracle.bimamba_forward(**p)
+    fl = lambda t: np.flip(t, -1)
+    delta4 = np.concatenate([p["delta"], p["delta"], fl(p["delta"]), fl(p["delta"])], axis=1)
+    A4 = np.concatenate([p["A"], p["A"], p["A_b"], p["A_b"]], axis=0)
+    B4 = np.stack([p["B"], p["B"], fl(p["B"]), fl(p["B"])], axis=1)
+    C4 = np.stack([p["C"], p["C"], fl(p["C"]), fl(p["C"])], axis=1)
+    y_img = oracle.ss2d_forward(p["x"].reshape(Bn, Dn, 1, L), delta4, A4, B4, C4, np.tile(p["D"], 4),
+                                np.tile(p["delta_bias"], 4), True)
+    np.testing.assert_allclose(y_img.reshape(Bn, Dn, L), 2.0 * y, rtol=1e-12, atol=1e-12)
+
+
+def test_bimamba_backward_matches_central_differences(oracle):
+    rng = _rng(53)
+    p = _bimamba_problem(rng, 2, 3, 7, 3)
+    p["z"] = 1.5 * rng.standard_normal(p["x"].shape)
+    dy = rng.standard_normal(p["x"].shape)
+    g = oracle.bimamba_backward(p["x"], p["delta"], p["A"], p["A_b"], p["B"], p["C"], p["D"], p["z"],
+                                p["delta_bias"], True, dy)
+
+    def loss():
+        return float(np.sum(oracle.bimamba_forward(**p) * dy))
+
+    names = dict(x="dx", delta="ddelta", A="dA", A_b="dA_b", B="dB", C="dC", D="dD", delta_bias="ddelta_bias",
+                 z="dz")
+    for name, gname in names.items():
+        flat = p[name].reshape(-1)
+        for i in rng.choice(flat.size, size=min(flat.size, 8), replace=False):
+            theta = flat[i]
+            h = 1e-6 * max(1.0, abs(theta))
+            flat[i] = theta + h
+            lp = loss()
+            flat[i] = theta - h
+            lm = loss()
+            flat[i] = theta
+            fd = (lp - lm) / (2 * h)
+            an = g[gname].reshape(-1)[i]
+            assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (name, i, fd, an)
 
 
 # --------------------------------------------------------- input generator
