@@ -16,6 +16,9 @@ collective on the data path -- only a barrier and a max over ranks of the timing
 Rank 0 prints one JSON line.  `--impl reference` times the fp64 CPU oracle on a
 bounded sample of the same workload instead (rank 0 only).
 
+`--workload 5` is the bidirectional scan of bimamba_inner_ref (Vim-T tokens, gated by
+silu(z)): a step is one bidirectional forward (plus its backward under `--backward`).
+
 `--backward` adds the fused backward to every step; `--gate` times the scan in its
 sequence form instead, u (B, 4D, L) with the output gate out * silu(z) and the last
 state (selective_scan_fn's z and return_last_state), plus its backward with dz
@@ -72,6 +75,19 @@ def seq_fwd_algorithmic_bytes(w, gate: bool) -> int:
     Bn, Dn, L, N = w.batch, w.dim, w.L, w.d_state
     seq = 4 * Bn * Dn * L
     return s * (seq * (3 if gate else 2) + 8 * Bn * N * L) + s * seq + 4 * 4 * Bn * Dn * N + 4 * 4 * Dn * (N + 2)
+
+
+def bidir_algorithmic_bytes(w, backward: bool) -> int:
+    """The bidirectional scan.  Forward: read x, delta, z (B, D, L), B, C (B, N, L); write y.
+    Backward: read x, delta, z, dy, B, C; write dx, ddelta, dz, dB, dC.  Plus A, A_b, D, bias
+    (and their gradients)."""
+    s = 4 if w.dtype == "f32" else 2
+    Bn, Dn, L, N = w.batch, w.dim, w.L, w.d_state
+    seq, bc = Bn * Dn * L, 2 * Bn * N * L
+    params = 4 * (2 * Dn * N + 2 * Dn)
+    if backward:
+        return s * (4 * seq + bc) + s * (3 * seq + bc) + 2 * params
+    return s * (3 * seq + bc) + s * seq + params
 
 
 def bwd_algorithmic_bytes(w, gate: bool = False) -> int:
@@ -273,7 +289,11 @@ def run_gpu(args, world, rank, local):
     if args.batch:
         w = w.with_batch(args.batch)
     dev = torch.device("cuda", local)
-    if args.gate:
+    bidir = w.kind == "bidir"
+    if bidir:
+        inp = ss2d_inputs.make_bimamba_inputs(w, seed=shard_seed(args.workload, rank), device=dev,
+                                              with_dy=args.backward, with_z=True)
+    elif args.gate:
         inp = ss2d_inputs.make_scan_inputs(w, seed=shard_seed(args.workload, rank), device=dev,
                                            with_dout=args.backward, with_z=True)
     else:
@@ -283,7 +303,21 @@ def run_gpu(args, world, rank, local):
     ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    if args.gate:
+    if bidir:
+        y_seq = torch.empty((w.batch, w.dim, w.L), dtype=w.torch_dtype, device=dev)
+        nbf = ss.workspace_bytes(w.batch, w.dim, 1, w.L, w.d_state, ss.OP_BIMAMBA_FORWARD, w.torch_dtype)
+        wsf = torch.empty(max(nbf, 1), dtype=torch.uint8, device=dev)
+        nbb = ss.workspace_bytes(w.batch, w.dim, 1, w.L, w.d_state, ss.OP_BIMAMBA_BACKWARD, w.torch_dtype)
+        wsb2 = torch.empty(max(nbb, 1), dtype=torch.uint8, device=dev)
+        bargs = (inp["x"], inp["delta"], inp["A"], inp["A_b"], inp["B"], inp["C"], inp["D"], inp["z"],
+                 inp["delta_bias"], True)
+
+        def step():
+            # bidirectional forward (keeping the chunk states under --backward), then its backward
+            res = ss.bimamba_forward(*bargs, out=y_seq, return_chunk_states=args.backward, workspace=wsf)
+            if args.backward:
+                ss.bimamba_backward(*bargs, inp["dy"], chunk_states=res[1], workspace=wsb2)
+    elif args.gate:
         seq_out = torch.empty((w.batch, 4 * w.dim, w.L), dtype=w.torch_dtype, device=dev)
 
         def step():
@@ -364,7 +398,9 @@ def run_gpu(args, world, rank, local):
     peaks = load_peaks()
     clocks = sampler.summary() if sampler else None
     # algorithmic bytes of the dominant kernel: the backward's when a backward runs in the step
-    if args.backward:
+    if bidir:
+        alg_bytes = bidir_algorithmic_bytes(w, args.backward)
+    elif args.backward:
         alg_bytes = bwd_algorithmic_bytes(w, gate=args.gate)
     elif args.gate:
         alg_bytes = seq_fwd_algorithmic_bytes(w, gate=True)
@@ -378,7 +414,9 @@ def run_gpu(args, world, rank, local):
     sfu_achieved = w.updates / (dom_ms / 1e3) / 1e9  # one exp(dt*A) per state update
     traffic = recorded_traffic(w.name)
 
-    e2e = run_e2e(args, w, inp, dev, stream, world, rank) if not (args.no_e2e or args.backward or args.gate) else None
+    e2e = None
+    if not (args.no_e2e or args.backward or args.gate or bidir):
+        e2e = run_e2e(args, w, inp, dev, stream, world, rank)
 
     result = {
         "metric": METRIC,
@@ -394,10 +432,11 @@ def run_gpu(args, world, rank, local):
         "dtype": "f32" if w.dtype == "f32" else "bf16",
         "data": "synthetic (seeded; VMamba init recipe for A, D, delta_bias)",
         "config": {"workload": w.name, "batch_per_gpu": w.batch, "global_batch": w.batch * world, "dim": w.dim,
-                   "height": w.height, "width": w.width, "d_state": w.d_state, "paths": 4,
+                   "height": w.height, "width": w.width, "d_state": w.d_state, "paths": w.paths,
                    "parallelism": f"batch shards x{world}, no collective",
                    "pass": ("forward + backward" if args.backward else "forward")
-                   + (" (sequence form, gate z + last state)" if args.gate else ""),
+                   + (" (sequence form, gate z + last state)" if args.gate else "")
+                   + (" (bidirectional, gate z)" if bidir else ""),
                    "l2": f"inputs {alg_bytes / 1e9:.2f} GB > 126 MB L2, no flush needed"},
         "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved_gbs / hbm_peak, "traffic": traffic,
@@ -413,7 +452,7 @@ def run_gpu(args, world, rank, local):
         "e2e": e2e,
     }
     # the oracle sample times the fused forward, so it is reported beside the forward line only
-    if rank == 0 and world == 1 and not (args.no_cpu_baseline or args.backward or args.gate):
+    if rank == 0 and world == 1 and not (args.no_cpu_baseline or args.backward or args.gate or bidir):
         result["cpu_baseline"] = time_oracle(w, seconds_budget=args.cpu_seconds)
     return result
 

@@ -85,7 +85,9 @@ typedef struct {
 typedef enum {
     SS2D_OP_SELECTIVE_SCAN_BWD = 1,
     SS2D_OP_FORWARD = 2,
-    SS2D_OP_BACKWARD = 3
+    SS2D_OP_BACKWARD = 3,
+    SS2D_OP_BIMAMBA_FORWARD = 4,
+    SS2D_OP_BIMAMBA_BACKWARD = 5
 } ss2d_op_t;
 
 /* Chunk length (steps) at which the forward saves scan states for the backward. */
@@ -227,6 +229,55 @@ SS2D_API ss2d_status_t ss2d_backward(const ss2d_desc_t *desc, const void *x, con
                             const float *chunk_states, void *dx, void *ddelta, float *dA,
                             void *dBm, void *dCm, float *dD, float *ddelta_bias,
                             void *workspace, size_t workspace_bytes, ss2d_stream_t stream);
+
+/* ------------------------------------------------- bidirectional scan -- */
+
+/*
+ * Bidirectional selective scan of bimamba_inner_ref ("vision mamba-yolov8",
+ * section "2. Vmamba module code"): one scan over the sequence with A, one over
+ * the reversed sequence with A_b (x, delta, B, C, z reversed with it; D and
+ * delta_bias shared), the second output reversed back and added:
+ *   y = S6(x, delta, A, B, C, D, z) + flip(S6(flip x, flip delta, A_b, flip B, flip C, D, flip z))
+ * Both directions are one launch; the reverse one reads its inputs backwards and
+ * writes at natural positions, and a merge adds the two in fp32 (gated by silu(z),
+ * which both directions share position by position) and rounds once.
+ * desc         : batch B, dim D, height 1, width L (a sequence), d_state N
+ * x, delta     : (B, D, L)  in_dtype
+ * A            : (2, D, N)  fp32: A, then A_b
+ * Bm, Cm       : (B, N, L)  in_dtype, shared by the two directions
+ * D, delta_bias: (D)        fp32 or NULL
+ * z            : (B, D, L)  in_dtype or NULL (output gate silu(z))
+ * y            : (B, D, L)  out_dtype
+ * chunk_states : (B, 2D, ceil(L / SS2D_CHUNK_LEN), N) fp32 or NULL, per direction in its own
+ *                step order (direction 1 counts steps from the end of the sequence)
+ * workspace    : ss2d_workspace_bytes(desc, SS2D_OP_BIMAMBA_FORWARD) bytes
+ * Errors: as for ss2d_forward; height != 1 is SS2D_ERR_SHAPE.
+ */
+SS2D_API ss2d_status_t ss2d_bimamba_forward(const ss2d_desc_t *desc, const void *x, const void *delta,
+                                            const float *A, const void *Bm, const void *Cm, const float *D,
+                                            const void *z, const float *delta_bias, int delta_softplus, void *y,
+                                            float *chunk_states, void *workspace, size_t workspace_bytes,
+                                            ss2d_stream_t stream);
+
+/*
+ * Gradients of ss2d_bimamba_forward.
+ * dy           : (B, D, L) out_dtype
+ * chunk_states : as written by ss2d_bimamba_forward, or NULL (recomputed)
+ * dx, ddelta   : (B, D, L) in_dtype (both directions' contributions added)
+ * dA           : (2, D, N) fp32: dA, then dA_b
+ * dBm, dCm     : (B, N, L) in_dtype
+ * dD, ddelta_bias: (D) fp32, non-NULL exactly when D / delta_bias are
+ * dz           : (B, D, L) in_dtype, non-NULL exactly when z is
+ * workspace    : ss2d_workspace_bytes(desc, SS2D_OP_BIMAMBA_BACKWARD) bytes
+ * Reductions are deterministic (fixed-order partial sums, no float atomics).
+ */
+SS2D_API ss2d_status_t ss2d_bimamba_backward(const ss2d_desc_t *desc, const void *x, const void *delta,
+                                             const float *A, const void *Bm, const void *Cm, const float *D,
+                                             const void *z, const float *delta_bias, int delta_softplus,
+                                             const void *dy, const float *chunk_states, void *dx, void *ddelta,
+                                             float *dA, void *dBm, void *dCm, float *dD, float *ddelta_bias,
+                                             void *dz, void *workspace, size_t workspace_bytes,
+                                             ss2d_stream_t stream);
 
 /*
  * S6 selective scan forward that allocates nothing and takes no workspace.

@@ -19,6 +19,8 @@ visual data", Fig. 2; the S6 arithmetic follows selective_scan_ref on
 * ``cross_merge(ys, H, W)``: (B, 4, D, L) -> (B, D, H, W), (y0 + y2) + (y1 + y3)
 * ``ss2d_forward`` / ``ss2d_backward``: the fused SS2D forward and backward
 * ``SS2DFunction``: a torch.autograd.Function around the fused pair
+* ``bimamba_forward`` / ``bimamba_backward`` / ``bimamba_scan``: the bidirectional scan of
+  bimamba_inner_ref (a sequence and its reverse with A and A_b, outputs added)
 """
 from __future__ import annotations
 
@@ -30,7 +32,8 @@ import torch
 
 __all__ = [
     "SS2DError", "cross_scan", "cross_merge", "selective_scan_fwd", "selective_scan_bwd", "selective_scan_fn",
-    "SelectiveScanFunction", "ss2d_forward",
+    "SelectiveScanFunction", "ss2d_forward", "bimamba_forward", "bimamba_backward", "BiMambaFunction",
+    "bimamba_scan",
     "ss2d_backward", "SS2DFunction", "ss2d", "workspace_bytes", "chunk_states_elems", "launch_count",
     "library_path", "CHUNK_LEN", "trace_events",
 ]
@@ -43,7 +46,7 @@ _lib = None
 
 CHUNK_LEN = 16  # SS2D_CHUNK_LEN
 F32, BF16 = 0, 1
-OP_SELECTIVE_SCAN_BWD, OP_FORWARD, OP_BACKWARD = 1, 2, 3
+OP_SELECTIVE_SCAN_BWD, OP_FORWARD, OP_BACKWARD, OP_BIMAMBA_FORWARD, OP_BIMAMBA_BACKWARD = 1, 2, 3, 4, 5
 _STATUS = {0: "SS2D_OK", 1: "SS2D_ERR_NULL", 2: "SS2D_ERR_SHAPE", 3: "SS2D_ERR_DTYPE", 4: "SS2D_ERR_ALIGN",
            5: "SS2D_ERR_WORKSPACE", 6: "SS2D_ERR_LAUNCH", 7: "SS2D_ERR_TIMEOUT", 8: "SS2D_ERR_DEVICE"}
 
@@ -88,9 +91,13 @@ def _load():
         lib.ss2d_selective_scan_bwd_ex.argtypes = [D, P, P, P, P, P, P, P, P, i, P, P, P, P, P, P, P, P, P, P,
                                                    P, sz, P]
         lib.ss2d_forward.argtypes = [D, P, P, P, P, P, P, P, i, P, P, P, sz, P]
+        lib.ss2d_bimamba_forward.argtypes = [D, P, P, P, P, P, P, P, P, i, P, P, P, sz, P]
+        lib.ss2d_bimamba_backward.argtypes = [D, P, P, P, P, P, P, P, P, i, P, P, P, P, P, P, P, P, P, P, P, sz,
+                                              P]
         lib.ss2d_backward.argtypes = [D, P, P, P, P, P, P, P, i, P, P, P, P, P, P, P, P, P, P, sz, P]
         for name in ("ss2d_cross_scan", "ss2d_cross_merge", "ss2d_selective_scan_fwd", "ss2d_selective_scan_bwd",
-                     "ss2d_selective_scan_fwd_ex", "ss2d_selective_scan_bwd_ex", "ss2d_forward", "ss2d_backward"):
+                     "ss2d_selective_scan_fwd_ex", "ss2d_selective_scan_bwd_ex", "ss2d_forward", "ss2d_backward",
+                     "ss2d_bimamba_forward", "ss2d_bimamba_backward"):
             getattr(lib, name).restype = ctypes.c_int
         lib.ss2d_workspace_bytes.argtypes = [D, i]
         lib.ss2d_workspace_bytes.restype = sz
@@ -396,3 +403,108 @@ class SS2DFunction(torch.autograd.Function):
 def ss2d(x, delta, A, B, C, D=None, delta_bias=None, delta_softplus=True):
     """Differentiable fused SS2D: y = CrossMerge(S6(CrossScan(x)))."""
     return SS2DFunction.apply(x, delta, A, B, C, D, delta_bias, delta_softplus)
+
+
+# ------------------------------------------------------------ bidirectional --
+
+def _bidir_params(A, A_b, D, delta_bias):
+    A2 = torch.stack([_c(A, torch.float32), _c(A_b, torch.float32)]).contiguous()  # (2, D, N)
+    return A2, _c(D, torch.float32), _c(delta_bias, torch.float32)
+
+
+def _bc3(t, dtype):
+    """B or C as (Bn, N, L); a (Bn, 1, N, L) tensor is accepted too"""
+    t = _c(t, dtype)
+    return t[:, 0] if t.dim() == 4 else t
+
+
+def bimamba_forward(x, delta, A, A_b, B, C, D=None, z=None, delta_bias=None, delta_softplus=True, out=None,
+                    out_dtype=None, return_chunk_states=False, workspace=None):
+    """Bidirectional scan of bimamba_inner_ref: S6 over the sequence with A plus S6 over the reversed
+    sequence with A_b, reversed back; gated by silu(z) when z is given.
+
+    x, delta, z (Bn, D, L); A, A_b (D, N) fp32; B, C (Bn, N, L); D, delta_bias (D) fp32 or None.
+    Returns y (Bn, D, L) [, chunk_states (Bn, 2D, ceil(L / CHUNK_LEN), N)].
+    """
+    x = _c(x)
+    delta, z = (_c(t, x.dtype) for t in (delta, z))
+    B, C = _bc3(B, x.dtype), _bc3(C, x.dtype)
+    A2, D, delta_bias = _bidir_params(A, A_b, D, delta_bias)
+    Bn, Dn, L = x.shape
+    N = A2.shape[2]
+    out_dtype = out_dtype or x.dtype
+    if out is None:
+        out = torch.empty((Bn, Dn, L), dtype=out_dtype, device=x.device)
+    cs = None
+    if return_chunk_states:
+        cs = torch.empty((Bn, 2 * Dn, -(-L // CHUNK_LEN), N), dtype=torch.float32, device=x.device)
+    d = _desc(Bn, Dn, 1, L, N, x.dtype, out.dtype)
+    lib = _load()
+    nbytes = int(lib.ss2d_workspace_bytes(ctypes.byref(d), OP_BIMAMBA_FORWARD))
+    if workspace is None or workspace.numel() < nbytes:
+        workspace = _workspace(nbytes, x.device)
+    st = lib.ss2d_bimamba_forward(ctypes.byref(d), _p(x), _p(delta), _p(A2), _p(B), _p(C), _p(D), _p(z),
+                                  _p(delta_bias), int(bool(delta_softplus)), _p(out), _p(cs), _p(workspace), nbytes,
+                                  _stream(x))
+    _check(st, "ss2d_bimamba_forward")
+    return (out, cs) if return_chunk_states else out
+
+
+def bimamba_backward(x, delta, A, A_b, B, C, D, z, delta_bias, delta_softplus, dy, chunk_states=None,
+                     workspace=None):
+    """Gradients of bimamba_forward.  Returns dict dx, ddelta, dA, dA_b, dB, dC, dD, ddelta_bias, dz
+    (dB, dC as (Bn, N, L); None where the input is None)."""
+    x = _c(x)
+    delta, z = (_c(t, x.dtype) for t in (delta, z))
+    B, C = _bc3(B, x.dtype), _bc3(C, x.dtype)
+    A2, D, delta_bias = _bidir_params(A, A_b, D, delta_bias)
+    dy = _c(dy)
+    chunk_states = _c(chunk_states, torch.float32)
+    Bn, Dn, L = x.shape
+    N = A2.shape[2]
+    dev = x.device
+    dx = torch.empty_like(x)
+    ddelta = torch.empty_like(delta)
+    dA2 = torch.empty_like(A2)
+    dB = torch.empty_like(B)
+    dC = torch.empty_like(C)
+    dD = torch.empty_like(D) if D is not None else None
+    dbias = torch.empty_like(delta_bias) if delta_bias is not None else None
+    dz = torch.empty_like(z) if z is not None else None
+    d = _desc(Bn, Dn, 1, L, N, x.dtype, dy.dtype)
+    lib = _load()
+    nbytes = int(lib.ss2d_workspace_bytes(ctypes.byref(d), OP_BIMAMBA_BACKWARD))
+    if workspace is None or workspace.numel() < nbytes:
+        workspace = _workspace(nbytes, dev)
+    st = lib.ss2d_bimamba_backward(ctypes.byref(d), _p(x), _p(delta), _p(A2), _p(B), _p(C), _p(D), _p(z),
+                                   _p(delta_bias), int(bool(delta_softplus)), _p(dy), _p(chunk_states), _p(dx),
+                                   _p(ddelta), _p(dA2), _p(dB), _p(dC), _p(dD), _p(dbias), _p(dz), _p(workspace),
+                                   nbytes, _stream(x))
+    _check(st, "ss2d_bimamba_backward")
+    return dict(dx=dx, ddelta=ddelta, dA=dA2[0], dA_b=dA2[1], dB=dB, dC=dC, dD=dD, ddelta_bias=dbias, dz=dz)
+
+
+class BiMambaFunction(torch.autograd.Function):
+    """autograd wrapper of the bidirectional scan: the forward keeps both directions' chunk states."""
+
+    @staticmethod
+    def forward(ctx, x, delta, A, A_b, B, C, D, z, delta_bias, delta_softplus):
+        y, cs = bimamba_forward(x, delta, A, A_b, B, C, D, z, delta_bias, delta_softplus, return_chunk_states=True)
+        ctx.save_for_backward(x, delta, A, A_b, B, C, D, z, delta_bias, cs)
+        ctx.delta_softplus = delta_softplus
+        ctx.bc4 = (B.dim() == 4, C.dim() == 4)
+        return y
+
+    @staticmethod
+    def backward(ctx, dy):
+        x, delta, A, A_b, B, C, D, z, delta_bias, cs = ctx.saved_tensors
+        g = bimamba_backward(x, delta, A, A_b, B, C, D, z, delta_bias, ctx.delta_softplus, dy.to(x.dtype),
+                             chunk_states=cs)
+        dB = g["dB"].unsqueeze(1) if ctx.bc4[0] else g["dB"]
+        dC = g["dC"].unsqueeze(1) if ctx.bc4[1] else g["dC"]
+        return g["dx"], g["ddelta"], g["dA"], g["dA_b"], dB, dC, g["dD"], g["dz"], g["ddelta_bias"], None
+
+
+def bimamba_scan(x, delta, A, A_b, B, C, D=None, z=None, delta_bias=None, delta_softplus=True):
+    """Differentiable bidirectional scan (the selective-scan part of bimamba_inner_ref)."""
+    return BiMambaFunction.apply(x, delta, A, A_b, B, C, D, z, delta_bias, delta_softplus)

@@ -114,6 +114,15 @@ static size_t bwd_fused_ws_bytes(const LaunchShape &s, ss2d_dtype_t in, ss2d_dty
            round64(scan_bwd_workspace_bytes(s));
 }
 
+// bidirectional forward workspace: [fp32 per-direction outputs (B,2,D,L)] [segment summaries]
+static size_t bidir_fwd_ws_bytes(const LaunchShape &s) {
+    return round64((size_t)s.B * 2 * s.D * s.L * sizeof(float)) + round64(scan_fwd_workspace_bytes(s, 2));
+}
+// bidirectional backward workspace: [fp32 per-direction du, ddelta, dz (B,2,D,L) each] [scan backward workspace]
+static size_t bidir_bwd_ws_bytes(const LaunchShape &s) {
+    return 3 * round64((size_t)s.B * 2 * s.D * s.L * sizeof(float)) + round64(scan_bwd_workspace_bytes(s, 2));
+}
+
 }  // namespace ss2d
 
 using namespace ss2d;
@@ -160,6 +169,8 @@ size_t ss2d_workspace_bytes(const ss2d_desc_t *desc, int op) {
         case SS2D_OP_SELECTIVE_SCAN_BWD: return scan_bwd_workspace_bytes(s);
         case SS2D_OP_FORWARD: return fwd_ws_bytes(s, desc->in_dtype);
         case SS2D_OP_BACKWARD: return bwd_fused_ws_bytes(s, desc->in_dtype, desc->out_dtype);
+        case SS2D_OP_BIMAMBA_FORWARD: return bidir_fwd_ws_bytes(s);
+        case SS2D_OP_BIMAMBA_BACKWARD: return bidir_bwd_ws_bytes(s);
         default: return (size_t)-1;
     }
 }
@@ -294,6 +305,108 @@ ss2d_status_t ss2d_selective_scan_bwd(const ss2d_desc_t *desc, const void *u, co
     return ss2d_selective_scan_bwd_ex(desc, u, delta, A, Bm, Cm, D, nullptr, delta_bias, delta_softplus, dout,
                                       chunk_states, du, ddelta, dA, dBm, dCm, dD, ddelta_bias, nullptr, workspace,
                                       workspace_bytes, stream);
+}
+
+ss2d_status_t ss2d_bimamba_forward(const ss2d_desc_t *desc, const void *x, const void *delta, const float *A,
+                                   const void *Bm, const void *Cm, const float *D, const void *z,
+                                   const float *delta_bias, int delta_softplus, void *y, float *chunk_states,
+                                   void *workspace, size_t workspace_bytes, ss2d_stream_t stream) {
+    SS2D_TRY(check_desc(desc));
+    if (desc->height != 1) return SS2D_ERR_SHAPE;
+    SS2D_TRY(check_scan_inputs(x, delta, A, Bm, Cm, D, delta_bias));
+    SS2D_TRY(optional(z));
+    SS2D_TRY(need(y));
+    SS2D_TRY(optional(chunk_states));
+    const LaunchShape s = shape_of(desc);
+    const size_t ws = bidir_fwd_ws_bytes(s);
+    if (!workspace || workspace_bytes < ws) return SS2D_ERR_WORKSPACE;
+    SS2D_TRY(optional(workspace));
+    SS2D_TRY(check_device());
+    float *ys = static_cast<float *>(workspace);
+    void *seg = static_cast<unsigned char *>(workspace) + round64((size_t)s.B * 2 * s.D * s.L * sizeof(float));
+    ScanFwdArgs a;
+    a.u = x;
+    a.delta = delta;
+    a.A = A;
+    a.Bm = Bm;
+    a.Cm = Cm;
+    a.Dv = D;
+    a.bias = delta_bias;
+    a.softplus = delta_softplus != 0;
+    a.out = ys;
+    a.chunk_states = chunk_states;
+    a.from_image = false;
+    a.bidir = true;
+    a.in_dtype = desc->in_dtype;
+    a.out_dtype = SS2D_F32;
+    cudaStream_t st = (cudaStream_t)stream;
+    SS2D_TRY(from_cuda(launch_scan_fwd(s, a, seg, st)));
+    return from_cuda(launch_bidir_sum(ys, z, desc->in_dtype, y, desc->out_dtype, s.B, s.D, s.L, st));
+}
+
+ss2d_status_t ss2d_bimamba_backward(const ss2d_desc_t *desc, const void *x, const void *delta, const float *A,
+                                    const void *Bm, const void *Cm, const float *D, const void *z,
+                                    const float *delta_bias, int delta_softplus, const void *dy,
+                                    const float *chunk_states, void *dx, void *ddelta, float *dA, void *dBm,
+                                    void *dCm, float *dD, float *ddelta_bias, void *dz, void *workspace,
+                                    size_t workspace_bytes, ss2d_stream_t stream) {
+    SS2D_TRY(check_desc(desc));
+    if (desc->height != 1) return SS2D_ERR_SHAPE;
+    SS2D_TRY(check_scan_inputs(x, delta, A, Bm, Cm, D, delta_bias));
+    SS2D_TRY(optional(z));
+    SS2D_TRY(need(dy));
+    SS2D_TRY(optional(chunk_states));
+    SS2D_TRY(need(dx));
+    SS2D_TRY(need(ddelta));
+    SS2D_TRY(need(dA));
+    SS2D_TRY(need(dBm));
+    SS2D_TRY(need(dCm));
+    if ((D == nullptr) != (dD == nullptr)) return SS2D_ERR_NULL;
+    if ((delta_bias == nullptr) != (ddelta_bias == nullptr)) return SS2D_ERR_NULL;
+    if ((z == nullptr) != (dz == nullptr)) return SS2D_ERR_NULL;
+    SS2D_TRY(optional(dD));
+    SS2D_TRY(optional(ddelta_bias));
+    SS2D_TRY(optional(dz));
+    const LaunchShape s = shape_of(desc);
+    const size_t ws = bidir_bwd_ws_bytes(s);
+    if (!workspace || workspace_bytes < ws) return SS2D_ERR_WORKSPACE;
+    SS2D_TRY(optional(workspace));
+    SS2D_TRY(check_device());
+    const size_t half = round64((size_t)s.B * 2 * s.D * s.L * sizeof(float));
+    unsigned char *w = static_cast<unsigned char *>(workspace);
+    float *du2 = reinterpret_cast<float *>(w);
+    float *dd2 = reinterpret_cast<float *>(w + half);
+    float *dz2 = reinterpret_cast<float *>(w + 2 * half);
+    ScanBwdArgs a;
+    a.u = x;
+    a.delta = delta;
+    a.A = A;
+    a.Bm = Bm;
+    a.Cm = Cm;
+    a.Dv = D;
+    a.bias = delta_bias;
+    a.softplus = delta_softplus != 0;
+    a.dout = dy;
+    a.chunk_states = chunk_states;
+    a.du = du2;
+    a.ddelta = dd2;
+    a.dA = dA;
+    a.dBm = dBm;
+    a.dCm = dCm;
+    a.dD = dD;
+    a.dbias = ddelta_bias;
+    a.z = z;
+    a.dz = z ? dz2 : nullptr;
+    a.from_image = false;
+    a.bidir = true;
+    a.in_dtype = desc->in_dtype;
+    a.out_dtype = desc->out_dtype;
+    cudaStream_t st = (cudaStream_t)stream;
+    SS2D_TRY(from_cuda(launch_scan_bwd(s, a, w + 3 * half, workspace_bytes - 3 * half, st)));
+    SS2D_TRY(from_cuda(launch_bidir_sum(du2, nullptr, SS2D_F32, dx, desc->in_dtype, s.B, s.D, s.L, st)));
+    SS2D_TRY(from_cuda(launch_bidir_sum(dd2, nullptr, SS2D_F32, ddelta, desc->in_dtype, s.B, s.D, s.L, st)));
+    if (z) SS2D_TRY(from_cuda(launch_bidir_sum(dz2, nullptr, SS2D_F32, dz, desc->in_dtype, s.B, s.D, s.L, st)));
+    return SS2D_OK;
 }
 
 ss2d_status_t ss2d_forward(const ss2d_desc_t *desc, const void *x, const void *delta, const float *A,

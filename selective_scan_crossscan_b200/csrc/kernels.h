@@ -25,6 +25,13 @@ cudaError_t launch_cross_merge(const LaunchShape &s, ss2d_dtype_t din, ss2d_dtyp
 
 // ---------------------------------------------------------------- forward --
 
+// How the scan kernels find a sequence's inputs:
+//  kModeSeq   -- (B, 4D, L) sequences, each path's data in its own sequence order;
+//  kModeImg   -- u read from the image along SS2D path k (fused CrossScan);
+//  kModeBidir -- a 1D sequence and its reverse (K = 2 directions) reading the same
+//                x, delta, B, C in natural order, the reverse direction backwards.
+enum ScanMode { kModeSeq = 0, kModeImg = 1, kModeBidir = 2 };
+
 struct ScanFwdArgs {
     const void *u;       // (B, 4D, L) sequences, or (B, D, H, W) image when from_image
     const void *uT = nullptr;  // (B, D, W, H) transposed image, read by the column paths when from_image
@@ -40,17 +47,24 @@ struct ScanFwdArgs {
     const void *z = nullptr;      // (B, 4D, L) output gate, out *= silu(z); sequences only
     float *last_state = nullptr;  // (B, 4D, N) state after the last step, or null
     bool from_image;     // read u along path k from the image (fused CrossScan)
+    bool bidir = false;  // kModeBidir: x (B, D, L), delta (B, D, L), B/C (B, 1, N, L), A (2D, N),
+                         // D/bias (D); out = per-direction outputs (B, 2, D, L) fp32 at natural positions
     ss2d_dtype_t in_dtype, out_dtype;
     int max_segments = 32;  // 1 = never split a sequence (no workspace needed)
 };
 
 // Number of sequence segments the forward scan is split into (1 = single pass).
-int scan_fwd_segments(const LaunchShape &s);
+int scan_fwd_segments(const LaunchShape &s, int paths = 4);
 // Workspace bytes for the forward scan's segment summaries.
-size_t scan_fwd_workspace_bytes(const LaunchShape &s);
+size_t scan_fwd_workspace_bytes(const LaunchShape &s, int paths = 4);
 cudaError_t launch_scan_fwd(const LaunchShape &s, const ScanFwdArgs &a, void *workspace, cudaStream_t stream);
 
 // --------------------------------------------------------------- backward --
+
+// Bidirectional scan: out[b, d, m] = (two[b, 0, d, m] + two[b, 1, d, m]) * (z ? silu(z[b, d, m]) : 1),
+// two (B, 2, D, L) fp32, z (B, D, L) z_dtype or null, out (B, D, L) out_dtype.
+cudaError_t launch_bidir_sum(const float *two, const void *z, ss2d_dtype_t z_dtype, void *out,
+                             ss2d_dtype_t out_dtype, int64_t B, int64_t D, int64_t L, cudaStream_t stream);
 
 struct ScanBwdArgs {
     const void *u;       // (B, 4D, L) sequences, or (B, D, H, W) image when from_image
@@ -75,10 +89,12 @@ struct ScanBwdArgs {
     const void *z = nullptr;  // (B, 4D, L) output gate of the forward; sequences only
     void *dz = nullptr;       // (B, 4D, L) in_dtype, written when z is given
     bool from_image;
+    bool bidir = false;       // kModeBidir: du, ddelta, dz are per-direction fp32 (B, 2, D, L) at natural
+                              // positions; dA (2D, N); dB/dC (B, 1, N, L); dD/dbias (D)
     ss2d_dtype_t in_dtype, out_dtype;
 };
 
-size_t scan_bwd_workspace_bytes(const LaunchShape &s);
+size_t scan_bwd_workspace_bytes(const LaunchShape &s, int paths = 4);
 
 // Helpers of the C-ABI layer (api.cu) for entry points defined in other files.
 ss2d_status_t check_scan_fwd_args(const ss2d_desc_t *desc, const void *u, const void *delta, const float *A,

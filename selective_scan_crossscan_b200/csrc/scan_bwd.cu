@@ -112,13 +112,14 @@ constexpr size_t bwd_smem_bytes() {
 
 // The warp's channels: u, delta, dout of 16 channels x 16 steps.  Every load is issued
 // before the first shared-memory store so that their latencies overlap.
-template <int NS, typename Tin, typename Tg, bool IMG, bool GATE>
+template <int NS, typename Tin, typename Tg, int MODE, bool GATE>
 __device__ __forceinline__ void stage_channels(BwdWarpSmem<NS, GATE> &sm, const BwdParams &p, int64_t b, int k,
                                                int64_t dw0, int nch, int64_t l0, int len) {
+    constexpr bool IMG = MODE == kModeImg, BIDIR = MODE == kModeBidir;
     constexpr int kPer = kChPerWarp * kBlk / 32;
     const int lane = threadIdx.x & 31;
     const int64_t D = p.D, L = p.L, C4 = kPaths * p.D;
-    const bool rev = IMG && k >= 2;
+    const bool rev = (IMG && k >= 2) || (BIDIR && k == 1);
     float uv[kPer], dv[kPer], gv[kPer], zv[GATE ? kPer : 1];
 #pragma unroll
     for (int t = 0; t < kPer; ++t) {
@@ -126,7 +127,15 @@ __device__ __forceinline__ void stage_channels(BwdWarpSmem<NS, GATE> &sm, const 
         const int ci = idx / kBlk, i = idx % kBlk;
         uv[t] = dv[t] = gv[t] = 0.f;
         if (GATE) zv[t] = 0.f;
-        if (ci < nch && i < len) {
+        if (ci < nch && i < len && BIDIR) {
+            // x, delta, dy, z in natural order, shared by the two directions
+            const int64_t row = (b * D + dw0 + ci) * L;
+            const int64_t m = rev ? (L - 1 - (l0 + i)) : l0 + i;
+            dv[t] = ld(static_cast<const Tin *>(p.delta) + row + m);
+            uv[t] = ld(static_cast<const Tin *>(p.u) + row + m);
+            gv[t] = ld(static_cast<const Tg *>(p.dout) + row + m);
+            if (GATE) zv[t] = ld(static_cast<const Tin *>(p.z) + row + m);
+        } else if (ci < nch && i < len) {
             const int64_t l = l0 + i;
             const int64_t cc = k * D + dw0 + ci;
             dv[t] = ld(static_cast<const Tin *>(p.delta) + (b * C4 + cc) * L + l);
@@ -156,22 +165,26 @@ __device__ __forceinline__ void stage_channels(BwdWarpSmem<NS, GATE> &sm, const 
 }
 
 // The block's B and C, staged once by all the CTA's threads.
-template <int NS, typename Tin>
+template <int NS, typename Tin, int MODE>
 __device__ __forceinline__ void stage_bc(BwdCtaSmem<NS> &cs, const BwdParams &p, int64_t b, int k, int64_t l0,
                                          int len) {
+    constexpr bool BIDIR = MODE == kModeBidir;
     constexpr int kTot = NS * kBlk;
     constexpr int kIt = (kTot + 32 * kWarps - 1) / (32 * kWarps);
     const int64_t L = p.L;
-    const Tin *Bk = static_cast<const Tin *>(p.Bm) + (b * kPaths + k) * p.N * L;
-    const Tin *Ck = static_cast<const Tin *>(p.Cm) + (b * kPaths + k) * p.N * L;
+    const int64_t grp = BIDIR ? b : b * kPaths + k;  // one B/C group per batch item in the bidirectional scan
+    const bool rev = BIDIR && k == 1;
+    const Tin *Bk = static_cast<const Tin *>(p.Bm) + grp * p.N * L;
+    const Tin *Ck = static_cast<const Tin *>(p.Cm) + grp * p.N * L;
     float rb[kIt], rc[kIt];
 #pragma unroll
     for (int t = 0; t < kIt; ++t) {
         const int idx = threadIdx.x + 32 * kWarps * t;
         const int n = idx / kBlk, i = idx % kBlk;
         const bool ok = idx < kTot && n < p.N && i < len;
-        rb[t] = ok ? ld(Bk + (int64_t)n * L + l0 + i) : 0.f;
-        rc[t] = ok ? ld(Ck + (int64_t)n * L + l0 + i) : 0.f;
+        const int64_t m = rev ? L - 1 - (l0 + i) : l0 + i;
+        rb[t] = ok ? ld(Bk + (int64_t)n * L + m) : 0.f;
+        rc[t] = ok ? ld(Ck + (int64_t)n * L + m) : 0.f;
     }
 #pragma unroll
     for (int t = 0; t < kIt; ++t) {
@@ -184,9 +197,10 @@ __device__ __forceinline__ void stage_bc(BwdCtaSmem<NS> &cs, const BwdParams &p,
     }
 }
 
-template <int NS, typename Tin, typename Tg, typename Tdu, bool IMG, bool GATE>
+template <int NS, typename Tin, typename Tg, typename Tdu, int MODE, bool GATE>
 __global__ void __launch_bounds__(32 * kWarps, SS2D_BWD_MIN_BLOCKS) scan_bwd_kernel(const BwdParams p) {
-    static_assert(!(IMG && GATE), "the output gate belongs to the sequence form");
+    constexpr bool IMG = MODE == kModeImg, BIDIR = MODE == kModeBidir;
+    static_assert(!(IMG && GATE), "the output gate belongs to the sequence forms");
     constexpr int HS = NS / 2;
     constexpr int HP = HS / 2;  // state pairs per lane
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -198,7 +212,9 @@ __global__ void __launch_bounds__(32 * kWarps, SS2D_BWD_MIN_BLOCKS) scan_bwd_ker
     const int ci = lane >> 1, hf = lane & 1;  // channel within the warp, state half
     const int k = blockIdx.y;
     const int64_t b = blockIdx.z;
-    const int64_t D = p.D, L = p.L, C4 = kPaths * p.D;
+    constexpr int K = BIDIR ? 2 : kPaths;  // paths (directions) per batch item
+    const int64_t D = p.D, L = p.L, C4 = K * p.D;
+    const bool rev = BIDIR && k == 1;  // the reverse direction stores at natural positions
     const int64_t dc0 = (int64_t)blockIdx.x * kChPerCta;  // first channel of the CTA
     const int64_t dw0 = dc0 + warp * kChPerWarp;           // first channel of this warp
     const int nch = (int)max((int64_t)0, min((int64_t)kChPerWarp, D - dw0));
@@ -217,8 +233,9 @@ __global__ void __launch_bounds__(32 * kWarps, SS2D_BWD_MIN_BLOCKS) scan_bwd_ker
         lam[q] = make_float2(0.f, 0.f);
         dA[q] = make_float2(0.f, 0.f);
     }
-    const float Dc = (active && p.Dv) ? p.Dv[c] : 0.f;
-    const float bias = (active && p.bias) ? p.bias[c] : 0.f;
+    const int64_t pc = BIDIR ? (active ? dw0 + ci : 0) : c;  // D and delta_bias are shared by the directions
+    const float Dc = (active && p.Dv) ? p.Dv[pc] : 0.f;
+    const float bias = (active && p.bias) ? p.bias[pc] : 0.f;
     float dD = 0.f, dbias = 0.f;
 
     Tdu *du_out = static_cast<Tdu *>(p.du);
@@ -238,8 +255,8 @@ __global__ void __launch_bounds__(32 * kWarps, SS2D_BWD_MIN_BLOCKS) scan_bwd_ker
                 h0[q] = make_float2((src && na < N) ? src[na] : 0.f, (src && na + 1 < N) ? src[na + 1] : 0.f);
             }
         }
-        stage_bc<NS, Tin>(csm, p, b, k, l0, len);
-        stage_channels<NS, Tin, Tg, IMG, GATE>(sm, p, b, k, dw0, nch, l0, len);
+        stage_bc<NS, Tin, MODE>(csm, p, b, k, l0, len);
+        stage_channels<NS, Tin, Tg, MODE, GATE>(sm, p, b, k, dw0, nch, l0, len);
         __syncthreads();  // B, C of the block are staged for all warps
         // gate: the scan's output o reaches the loss as o * silu(z), so dout * silu(z) drives the
         // adjoint and dz = dout * silu'(z) * o (o is rebuilt in the adjoint walk)
@@ -438,12 +455,19 @@ __global__ void __launch_bounds__(32 * kWarps, SS2D_BWD_MIN_BLOCKS) scan_bwd_ker
             const int cw = idx / kBlk, i = idx % kBlk;
             if (cw < nch && i < len) {
                 const int64_t cc = k * D + dw0 + cw;
-                st(du_out + (b * C4 + cc) * L + l0 + i, sm.G[cw][i]);
-                st(dd_out + (b * C4 + cc) * L + l0 + i, sm.SG[cw][i]);
-                if (GATE) st(static_cast<Tin *>(p.dz) + (b * C4 + cc) * L + l0 + i, sm.GZ[cw][i]);
+                if (BIDIR) {  // per-direction fp32 partials at natural positions, summed afterwards
+                    const int64_t o = (b * C4 + cc) * L + (rev ? L - 1 - (l0 + i) : l0 + i);
+                    static_cast<float *>(p.du)[o] = sm.G[cw][i];
+                    static_cast<float *>(p.ddelta)[o] = sm.SG[cw][i];
+                    if (GATE) static_cast<float *>(p.dz)[o] = sm.GZ[cw][i];
+                } else {
+                    st(du_out + (b * C4 + cc) * L + l0 + i, sm.G[cw][i]);
+                    st(dd_out + (b * C4 + cc) * L + l0 + i, sm.SG[cw][i]);
+                    if (GATE) st(static_cast<Tin *>(p.dz) + (b * C4 + cc) * L + l0 + i, sm.GZ[cw][i]);
+                }
             }
         }
-        float *pbc = p.part_bc + ((b * kPaths + k) * p.ntiles + blockIdx.x) * (int64_t)(2 * N) * L;
+        float *pbc = p.part_bc + ((b * K + k) * p.ntiles + blockIdx.x) * (int64_t)(2 * N) * L;
         for (int idx = threadIdx.x; idx < 2 * N * kBlk; idx += 32 * kWarps) {
             const int v = idx / kBlk, i = idx % kBlk;
             const int col = v < N ? v : NS + (v - N);
@@ -451,7 +475,7 @@ __global__ void __launch_bounds__(32 * kWarps, SS2D_BWD_MIN_BLOCKS) scan_bwd_ker
                 float s = 0.f;
 #pragma unroll
                 for (int w = 0; w < kWarps; ++w) s += wsm[w].bct[i][col];
-                pbc[(int64_t)v * L + l0 + i] = s;
+                pbc[(int64_t)v * L + (rev ? L - 1 - (l0 + i) : l0 + i)] = s;
             }
         }
         __syncthreads();  // bct is rewritten by the next block
@@ -473,10 +497,12 @@ __global__ void __launch_bounds__(32 * kWarps, SS2D_BWD_MIN_BLOCKS) scan_bwd_ker
 }
 
 // dB/dC = sum over tiles of the partials (fixed order); dA/dD/ddelta_bias = sum over the batch.
+// G groups per batch item; the bidirectional scan has one group whose "tiles" are both
+// directions' channel tiles (its partials are stored at natural positions).
 template <typename Tin>
 __global__ void bwd_reduce_bc_kernel(const float *__restrict__ part_bc, Tin *__restrict__ dB, Tin *__restrict__ dC,
-                                     int64_t B, int N, int64_t L, int ntiles) {
-    const int64_t total = B * kPaths * N * L;
+                                     int64_t B, int G, int N, int64_t L, int ntiles) {
+    const int64_t total = B * G * N * L;
     for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
          e += (int64_t)gridDim.x * blockDim.x) {
         const int64_t l = e % L;
@@ -493,15 +519,38 @@ __global__ void bwd_reduce_bc_kernel(const float *__restrict__ part_bc, Tin *__r
     }
 }
 
+// shared > 1: D and delta_bias are shared by `shared` directions (channels c, c + D, ...): their
+// gradients sum over those too, batch item by batch item in a fixed order.
 __global__ void bwd_reduce_params_kernel(const float *__restrict__ part_p, float *__restrict__ dA, float *__restrict__ dD,
-                                         float *__restrict__ dbias, int64_t B, int64_t C4, int N) {
+                                         float *__restrict__ dbias, int64_t B, int64_t C4, int N, int shared) {
     const int64_t total = C4 * (N + 2);
+    const int64_t Dsh = C4 / shared;
     for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
          e += (int64_t)gridDim.x * blockDim.x) {
         const int64_t c = e / (N + 2);
         const int v = (int)(e % (N + 2));
+        if (v >= N && c >= Dsh) continue;  // folded into channel c mod Dsh
+        const int reps = v < N ? 1 : shared;
+        const int64_t bstride = C4 * (N + 2);
+        const float *src = part_p + c * (N + 2) + v;
         float s = 0.f;
-        for (int64_t b = 0; b < B; ++b) s += part_p[(b * C4 + c) * (N + 2) + v];
+        int64_t b = 0;
+        const int64_t rstride = Dsh * (N + 2);
+        for (; b + 8 <= B; b += 8) {  // eight batch items' loads in flight, added in batch order
+            float t0[8], t1[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                t0[j] = src[(b + j) * bstride];
+                t1[j] = reps > 1 ? src[(b + j) * bstride + rstride] : 0.f;
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                s += t0[j];
+                if (reps > 1) s += t1[j];
+            }
+        }
+        for (; b < B; ++b)
+            for (int r = 0; r < reps; ++r) s += src[b * bstride + r * rstride];
         if (v < N) dA[c * N + v] = s;
         else if (v == N) { if (dD) dD[c] = s; }
         else if (dbias) dbias[c] = s;
@@ -512,61 +561,62 @@ __global__ void bwd_reduce_params_kernel(const float *__restrict__ part_p, float
 
 static int bwd_tiles(const LaunchShape &s) { return (int)ceil_div(s.D, kChPerCta); }
 
-size_t scan_bwd_workspace_bytes(const LaunchShape &s) {
+size_t scan_bwd_workspace_bytes(const LaunchShape &s, int paths) {
     const size_t nchunks = (size_t)ceil_div(s.L, kBlk);
     size_t bytes = 0;
     auto add = [&](size_t n) { bytes += (n + 63) / 64 * 64; };
-    add((size_t)s.B * kPaths * bwd_tiles(s) * 2 * s.N * s.L * sizeof(float));  // part_bc
-    add((size_t)s.B * kPaths * s.D * (s.N + 2) * sizeof(float));               // part_p
-    add((size_t)s.B * kPaths * s.D * nchunks * s.N * sizeof(float));            // recomputed chunk states
-    add(scan_fwd_workspace_bytes(s));                                           // forward segment summaries
+    add((size_t)s.B * paths * bwd_tiles(s) * 2 * s.N * s.L * sizeof(float));  // part_bc
+    add((size_t)s.B * paths * s.D * (s.N + 2) * sizeof(float));               // part_p
+    add((size_t)s.B * paths * s.D * nchunks * s.N * sizeof(float));            // recomputed chunk states
+    add(scan_fwd_workspace_bytes(s, paths));                                   // forward segment summaries
     return bytes;
 }
 
-template <int NS, typename Tin, typename Tg, typename Tdu, bool IMG, bool GATE>
+template <int NS, typename Tin, typename Tg, typename Tdu, int MODE, bool GATE>
 static cudaError_t launch_bwd_t(const LaunchShape &s, const BwdParams &p, cudaStream_t stream) {
     const size_t smem = bwd_smem_bytes<NS, GATE>();
-    auto kern = scan_bwd_kernel<NS, Tin, Tg, Tdu, IMG, GATE>;
+    auto kern = scan_bwd_kernel<NS, Tin, Tg, Tdu, MODE, GATE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)bwd_tiles(s), kPaths, (unsigned)s.B);
+    dim3 grid((unsigned)bwd_tiles(s), MODE == kModeBidir ? 2 : kPaths, (unsigned)s.B);
     kern<<<grid, 32 * kWarps, smem, stream>>>(p);
     note_launch(stream);
     return cudaGetLastError();
 }
 
-template <typename Tin, typename Tg, typename Tdu, bool IMG, bool GATE>
+template <typename Tin, typename Tg, typename Tdu, int MODE, bool GATE>
 static cudaError_t launch_bwd_gate(const LaunchShape &s, const BwdParams &p, cudaStream_t stream) {
-    if (s.N <= 4) return launch_bwd_t<4, Tin, Tg, Tdu, IMG, GATE>(s, p, stream);
-    if (s.N <= 8) return launch_bwd_t<8, Tin, Tg, Tdu, IMG, GATE>(s, p, stream);
-    return launch_bwd_t<16, Tin, Tg, Tdu, IMG, GATE>(s, p, stream);
+    if (s.N <= 4) return launch_bwd_t<4, Tin, Tg, Tdu, MODE, GATE>(s, p, stream);
+    if (s.N <= 8) return launch_bwd_t<8, Tin, Tg, Tdu, MODE, GATE>(s, p, stream);
+    return launch_bwd_t<16, Tin, Tg, Tdu, MODE, GATE>(s, p, stream);
 }
 
-template <typename Tin, typename Tg, typename Tdu, bool IMG>
+template <typename Tin, typename Tg, typename Tdu, int MODE>
 static cudaError_t launch_bwd_ns(const LaunchShape &s, const BwdParams &p, cudaStream_t stream) {
-    if (!IMG && p.z) return launch_bwd_gate<Tin, Tg, Tdu, false, true>(s, p, stream);
-    return launch_bwd_gate<Tin, Tg, Tdu, IMG, false>(s, p, stream);
+    if (MODE != kModeImg && p.z) return launch_bwd_gate<Tin, Tg, Tdu, MODE == kModeImg ? kModeSeq : MODE, true>(s, p, stream);
+    return launch_bwd_gate<Tin, Tg, Tdu, MODE, false>(s, p, stream);
 }
 
-template <typename Tin, typename Tg, bool IMG>
+template <typename Tin, typename Tg, int MODE>
 static cudaError_t launch_bwd_du(const LaunchShape &s, const BwdParams &p, cudaStream_t stream) {
-    // the fused backward keeps du in fp32 for the merge that follows
-    if (IMG) return launch_bwd_ns<Tin, Tg, float, IMG>(s, p, stream);
-    return launch_bwd_ns<Tin, Tg, Tin, IMG>(s, p, stream);
+    // the fused and bidirectional backward passes keep du in fp32 for the merge that follows
+    if (MODE != kModeSeq) return launch_bwd_ns<Tin, Tg, float, MODE>(s, p, stream);
+    return launch_bwd_ns<Tin, Tg, Tin, MODE>(s, p, stream);
 }
 
-template <bool IMG>
+template <int MODE>
 static cudaError_t launch_bwd_types(const LaunchShape &s, const BwdParams &p, ss2d_dtype_t din, ss2d_dtype_t dg,
                                     cudaStream_t stream) {
-    if (din == SS2D_F32 && dg == SS2D_F32) return launch_bwd_du<float, float, IMG>(s, p, stream);
-    if (din == SS2D_F32) return launch_bwd_du<float, __nv_bfloat16, IMG>(s, p, stream);
-    if (dg == SS2D_F32) return launch_bwd_du<__nv_bfloat16, float, IMG>(s, p, stream);
-    return launch_bwd_du<__nv_bfloat16, __nv_bfloat16, IMG>(s, p, stream);
+    if (din == SS2D_F32 && dg == SS2D_F32) return launch_bwd_du<float, float, MODE>(s, p, stream);
+    if (din == SS2D_F32) return launch_bwd_du<float, __nv_bfloat16, MODE>(s, p, stream);
+    if (dg == SS2D_F32) return launch_bwd_du<__nv_bfloat16, float, MODE>(s, p, stream);
+    return launch_bwd_du<__nv_bfloat16, __nv_bfloat16, MODE>(s, p, stream);
 }
 
 cudaError_t launch_scan_bwd(const LaunchShape &s, const ScanBwdArgs &a, void *workspace, size_t ws_bytes,
                             cudaStream_t stream) {
     (void)ws_bytes;
+    const int K = a.bidir ? 2 : kPaths;  // paths (directions) per batch item
     const int64_t nchunks = ceil_div(s.L, kBlk);
     unsigned char *ws = static_cast<unsigned char *>(workspace);
     size_t off = 0;
@@ -575,10 +625,10 @@ cudaError_t launch_scan_bwd(const LaunchShape &s, const ScanBwdArgs &a, void *wo
         off += (n + 63) / 64 * 64;
         return ptr;
     };
-    float *part_bc = (float *)take((size_t)s.B * kPaths * bwd_tiles(s) * 2 * s.N * s.L * sizeof(float));
-    float *part_p = (float *)take((size_t)s.B * kPaths * s.D * (s.N + 2) * sizeof(float));
-    float *cs_ws = (float *)take((size_t)s.B * kPaths * s.D * nchunks * s.N * sizeof(float));
-    void *fwd_ws = take(scan_fwd_workspace_bytes(s));
+    float *part_bc = (float *)take((size_t)s.B * K * bwd_tiles(s) * 2 * s.N * s.L * sizeof(float));
+    float *part_p = (float *)take((size_t)s.B * K * s.D * (s.N + 2) * sizeof(float));
+    float *cs_ws = (float *)take((size_t)s.B * K * s.D * nchunks * s.N * sizeof(float));
+    void *fwd_ws = take(scan_fwd_workspace_bytes(s, K));
 
     const float *cs = a.chunk_states;
     cudaError_t e;
@@ -597,6 +647,7 @@ cudaError_t launch_scan_bwd(const LaunchShape &s, const ScanBwdArgs &a, void *wo
         f.out = nullptr;
         f.chunk_states = cs_ws;
         f.from_image = a.from_image;
+        f.bidir = a.bidir;
         f.in_dtype = a.in_dtype;
         f.out_dtype = SS2D_F32;
         e = launch_scan_fwd(s, f, fwd_ws, stream);
@@ -616,7 +667,7 @@ cudaError_t launch_scan_bwd(const LaunchShape &s, const ScanBwdArgs &a, void *wo
     p.dout = a.dout;
     p.doutT = a.doutT;
     p.cs = cs;
-    p.z = a.from_image ? nullptr : a.z;
+    p.z = a.from_image ? nullptr : a.z;  // the fused SS2D path has no gate
     p.du = a.du;
     p.ddelta = a.ddelta;
     p.dz = a.dz;
@@ -631,24 +682,31 @@ cudaError_t launch_scan_bwd(const LaunchShape &s, const ScanBwdArgs &a, void *wo
     p.softplus = a.softplus;
     p.nchunks = nchunks;
     p.ntiles = bwd_tiles(s);
-    e = a.from_image ? launch_bwd_types<true>(s, p, a.in_dtype, a.out_dtype, stream)
-                     : launch_bwd_types<false>(s, p, a.in_dtype, a.out_dtype, stream);
+    if (a.bidir)
+        e = launch_bwd_types<kModeBidir>(s, p, a.in_dtype, a.out_dtype, stream);
+    else if (a.from_image)
+        e = launch_bwd_types<kModeImg>(s, p, a.in_dtype, a.out_dtype, stream);
+    else
+        e = launch_bwd_types<kModeSeq>(s, p, a.in_dtype, a.out_dtype, stream);
     if (e != cudaSuccess) return e;
 
+    // the bidirectional scan has one B/C group per batch item, reduced over both directions' tiles
+    const int G = a.bidir ? 1 : kPaths;
+    const int rtiles = a.bidir ? 2 * p.ntiles : p.ntiles;
     const int threads = 256;
-    const int64_t nbc = s.B * kPaths * s.N * s.L;
+    const int64_t nbc = s.B * G * s.N * s.L;
     const int64_t nblk = ceil_div(nbc, threads);
     const int blocks_bc = (int)(nblk < 148 * 16 ? nblk : 148 * 16);
     if (a.in_dtype == SS2D_F32)
         bwd_reduce_bc_kernel<float><<<blocks_bc, threads, 0, stream>>>(part_bc, (float *)a.dBm, (float *)a.dCm, s.B,
-                                                                     (int)s.N, s.L, p.ntiles);
+                                                                     G, (int)s.N, s.L, rtiles);
     else
         bwd_reduce_bc_kernel<__nv_bfloat16><<<blocks_bc, threads, 0, stream>>>(
-            part_bc, (__nv_bfloat16 *)a.dBm, (__nv_bfloat16 *)a.dCm, s.B, (int)s.N, s.L, p.ntiles);
+            part_bc, (__nv_bfloat16 *)a.dBm, (__nv_bfloat16 *)a.dCm, s.B, G, (int)s.N, s.L, rtiles);
     note_launch(stream);
-    const int64_t np = kPaths * s.D * (s.N + 2);
-    bwd_reduce_params_kernel<<<(int)ceil_div(np, threads), threads, 0, stream>>>(part_p, a.dA, a.dD, a.dbias, s.B,
-                                                                                kPaths * s.D, (int)s.N);
+    const int64_t np = K * s.D * (s.N + 2);
+    bwd_reduce_params_kernel<<<(int)ceil_div(np, threads), threads, 0, stream>>>(
+        part_p, a.dA, a.dD, a.dbias, s.B, K * s.D, (int)s.N, a.bidir ? 2 : 1);
     note_launch(stream);
     return cudaGetLastError();
 }

@@ -12,17 +12,19 @@
 // FMUL (dt * A*log2e), one MUFU.EX2, one FMUL (dt*u * B) and two FFMAs -- no
 // cross-thread scan arithmetic at all.
 //
-//  * A CTA is one warp: 32 channels of one (b, k).  The headline problem
-//    (98,304 sequences) then fits the GPU in a single wave (~21 warps per SM),
-//    so no SM idles while a second, nearly empty wave runs.
-//  * u and delta are read by each thread along its own sequence, four steps at
-//    a time (16-byte loads for fp32, 8-byte for bf16), one group ahead of use.
-//  * B[., l] and C[., l] are the same for all 32 threads (group k of batch b):
-//    they are staged in shared memory in 32-step chunks with cp.async, double
-//    buffered, and read as broadcast vector loads.
+//  * A CTA is one warp: 32 channels of one (b, k), 16 warps resident per SM
+//    (four per scheduler).
+//  * B[., l] and C[., l] are the same for all 32 threads (group k of batch b);
+//    each thread's u and delta rows are its own.  All of them are staged in
+//    shared memory in 8-step chunks with cp.async (16-byte pieces for fp32,
+//    8-byte for bf16), double buffered, and read as 4-step vector loads.
 //  * The fused SS2D forward reads u from the image along path k: row-major
 //    paths from x (k=2 backwards), column-major paths from a transposed copy
 //    of x (k=3 backwards), so every load stays sequential.
+//  * The bidirectional scan (bimamba_inner_ref) runs a sequence and its reverse
+//    as two directions of one launch; the reverse direction stages x, delta, B
+//    and C backwards (4-step pieces copied in memory order, read from the end)
+//    and stores its outputs at their natural positions.
 //
 // When a problem has too few sequences to fill the GPU, each sequence is cut
 // into segments: a summary pass computes, per segment, the state reached
@@ -115,9 +117,14 @@ struct FwdStage {
     Tin Dl[kWarp][kRow];
 };
 
-// Issue the copies of chunk [cbeg, cbeg+len).  VEC: 4-element cp.async pieces
-// (len is then a multiple of 4); else plain loads (synchronous).
-template <int NS, bool VEC, typename Tin>
+// Shared-memory slots are the same in every form: slot i of a row holds step cbeg+i,
+// or step cbeg+kLC-1-i for a reversed row, so the scan reads 4-step vectors.
+// Issue the copies of chunk [cbeg, cbeg+len):
+//  * VEC (rows 16-byte aligned, len a multiple of 4): 4-element cp.async pieces;
+//  * fp32 rows of any alignment: one 4-byte cp.async per element, slots past the end zeroed;
+//  * bf16 rows of any alignment: plain loads (synchronous), slots past the end zeroed.
+// REV: the chunk is walked backwards through delta, B and C as well (bidirectional scan).
+template <int NS, bool VEC, bool REV, typename Tin>
 __device__ __forceinline__ void stage_chunk(FwdStage<Tin, NS> &st, const Tin *Bk, const Tin *Ck, int N, int64_t L,
                                             const Tin *urow, bool urev, const Tin *drow, bool active, int64_t cbeg,
                                             int len) {
@@ -128,15 +135,23 @@ __device__ __forceinline__ void stage_chunk(FwdStage<Tin, NS> &st, const Tin *Bk
         for (int idx = t; idx < NS * q; idx += kWarp) {
             const int n = idx / q, i4 = (idx % q) * 4;
             if (n < N && i4 < len) {
-                cp_async_bytes(&st.B[n][i4], Bk + (int64_t)n * L + cbeg + i4, kBytes);
-                cp_async_bytes(&st.C[n][i4], Ck + (int64_t)n * L + cbeg + i4, kBytes);
+                if (!REV) {
+                    cp_async_bytes(&st.B[n][i4], Bk + (int64_t)n * L + cbeg + i4, kBytes);
+                    cp_async_bytes(&st.C[n][i4], Ck + (int64_t)n * L + cbeg + i4, kBytes);
+                } else {
+                    cp_async_bytes(&st.B[n][kLC - 4 - i4], Bk + (int64_t)n * L + (L - cbeg - 4 - i4), kBytes);
+                    cp_async_bytes(&st.C[n][kLC - 4 - i4], Ck + (int64_t)n * L + (L - cbeg - 4 - i4), kBytes);
+                }
             }
         }
         if (active) {
 #pragma unroll
             for (int i4 = 0; i4 < kLC; i4 += 4) {
                 if (i4 < len) {
-                    cp_async_bytes(&st.Dl[t][i4], drow + cbeg + i4, kBytes);
+                    if (!REV)
+                        cp_async_bytes(&st.Dl[t][i4], drow + cbeg + i4, kBytes);
+                    else
+                        cp_async_bytes(&st.Dl[t][kLC - 4 - i4], drow + (L - cbeg - 4 - i4), kBytes);
                     if (!urev)
                         cp_async_bytes(&st.U[t][i4], urow + cbeg + i4, kBytes);
                     else  // steps cbeg+i4 .. +3 live at memory L-1-cbeg-i4-3 .. L-1-cbeg-i4
@@ -144,30 +159,62 @@ __device__ __forceinline__ void stage_chunk(FwdStage<Tin, NS> &st, const Tin *Bk
                 }
             }
         }
+    } else if (sizeof(Tin) == 4) {
+        for (int idx = t; idx < NS * kLC; idx += kWarp) {
+            const int n = idx / kLC, i = idx % kLC;
+            const int slot = REV ? kLC - 1 - i : i;
+            if (n < N && i < len) {
+                const int64_t m = REV ? L - 1 - (cbeg + i) : cbeg + i;
+                cp_async_bytes(&st.B[n][slot], Bk + (int64_t)n * L + m, 4);
+                cp_async_bytes(&st.C[n][slot], Ck + (int64_t)n * L + m, 4);
+            } else {
+                st.B[n][slot] = Tin(0.f);
+                st.C[n][slot] = Tin(0.f);
+            }
+        }
+        for (int i = 0; i < kLC; ++i) {
+            const int64_t l = cbeg + i;
+            const int dslot = REV ? kLC - 1 - i : i, uslot = urev ? kLC - 1 - i : i;
+            if (active && i < len) {
+                cp_async_bytes(&st.Dl[t][dslot], drow + (REV ? L - 1 - l : l), 4);
+                cp_async_bytes(&st.U[t][uslot], urow + (urev ? L - 1 - l : l), 4);
+            } else {
+                st.Dl[t][dslot] = Tin(0.f);
+                st.U[t][uslot] = Tin(0.f);
+            }
+        }
     } else {
         for (int idx = t; idx < NS * kLC; idx += kWarp) {
             const int n = idx / kLC, i = idx % kLC;
             const bool ok = n < N && i < len;
-            st.B[n][i] = ok ? Bk[(int64_t)n * L + cbeg + i] : Tin(0.f);
-            st.C[n][i] = ok ? Ck[(int64_t)n * L + cbeg + i] : Tin(0.f);
+            const int64_t m = REV ? L - 1 - (cbeg + i) : cbeg + i;
+            const int slot = REV ? kLC - 1 - i : i;
+            st.B[n][slot] = ok ? Bk[(int64_t)n * L + m] : Tin(0.f);
+            st.C[n][slot] = ok ? Ck[(int64_t)n * L + m] : Tin(0.f);
         }
         for (int i = 0; i < kLC; ++i) {
             const bool ok = active && i < len;
             const int64_t l = cbeg + i;
-            st.Dl[t][i] = ok ? drow[l] : Tin(0.f);
+            st.Dl[t][REV ? kLC - 1 - i : i] = ok ? drow[REV ? L - 1 - l : l] : Tin(0.f);
             st.U[t][urev ? (kLC - 1 - i) : i] = ok ? urow[urev ? (L - 1 - l) : l] : Tin(0.f);
         }
     }
 }
 
-// PASS 0: single pass.  PASS 1: segment summaries only.  PASS 2: outputs with carries.
-template <int NS, typename Tin, typename Tout, bool IMG, int PASS, bool VEC>
-__global__ void __launch_bounds__(kWarp, SS2D_FWD_MIN_BLOCKS) scan_fwd_kernel(const FwdParams p) {
-    __shared__ __align__(16) FwdStage<Tin, NS> stage[2];
-    // A[c, n] * log2(e) of each lane's channel: in registers for fp32 inputs, in shared memory
-    // for bf16 (whose conversions need the registers)
-    constexpr bool kA2Smem = SS2D_FWD_A2_SMEM || sizeof(Tin) < 4;
-    __shared__ float A2s[kA2Smem ? NS : 1][kWarp];
+// A[c, n] * log2(e) of each lane's channel: in registers for fp32 inputs, in shared memory
+// for bf16 (whose conversions need the registers)
+template <typename Tin>
+__host__ __device__ constexpr bool a2_in_smem() {
+    return SS2D_FWD_A2_SMEM || sizeof(Tin) < 4;
+}
+
+// The scan of one CTA.  PASS 0: single pass.  PASS 1: segment summaries only.  PASS 2:
+// outputs with carries.  REV: the reverse direction of the bidirectional scan.
+template <int NS, typename Tin, typename Tout, int MODE, int PASS, bool VEC, bool REV>
+__device__ __forceinline__ void scan_fwd_body(const FwdParams &p, FwdStage<Tin, NS> (&stage)[2],
+                                              float (&A2s)[a2_in_smem<Tin>() ? NS : 1][kWarp]) {
+    constexpr bool IMG = MODE == kModeImg, BIDIR = MODE == kModeBidir, SEQ = MODE == kModeSeq;
+    constexpr bool kA2Smem = a2_in_smem<Tin>();
     float A2r[NS];
 #define SS2D_A2(n) (kA2Smem ? A2s[n][t] : A2r[n])
 
@@ -175,7 +222,7 @@ __global__ void __launch_bounds__(kWarp, SS2D_FWD_MIN_BLOCKS) scan_fwd_kernel(co
     const int k = blockIdx.y;
     const int64_t b = blockIdx.z / p.nseg;
     const int sgi = blockIdx.z % p.nseg;
-    const int64_t D = p.D, L = p.L, C4 = kPaths * p.D;
+    const int64_t D = p.D, L = p.L, C4 = (BIDIR ? 2 : kPaths) * p.D;
     const int64_t d = (int64_t)blockIdx.x * kWarp + t;
     const bool active = d < D;
     const int64_t c = k * D + (active ? d : 0);
@@ -193,8 +240,9 @@ __global__ void __launch_bounds__(kWarp, SS2D_FWD_MIN_BLOCKS) scan_fwd_kernel(co
             A2r[n] = a2v;
         h[n] = 0.f;
     }
-    const float Dc = (active && p.Dv) ? p.Dv[c] : 0.f;
-    const float bias = (active && p.bias) ? p.bias[c] : 0.f;
+    const int64_t pc = BIDIR ? (active ? d : 0) : c;  // D and delta_bias are shared by the two directions
+    const float Dc = (active && p.Dv) ? p.Dv[pc] : 0.f;
+    const float bias = (active && p.bias) ? p.bias[pc] : 0.f;
     if (PASS == 2 && active) {
         // carry into this segment: fold the summaries of the segments before it
         const float *sg = p.seg + (b * C4 + c) * (int64_t)p.nseg * 2 * N;
@@ -213,13 +261,17 @@ __global__ void __launch_bounds__(kWarp, SS2D_FWD_MIN_BLOCKS) scan_fwd_kernel(co
         const Tin *img = static_cast<const Tin *>((k & 1) ? p.uT : p.u);
         urow = img + (b * D + (active ? d : 0)) * L;
         urev = k >= 2;
+    } else if (BIDIR) {
+        urow = static_cast<const Tin *>(p.u) + (b * D + (active ? d : 0)) * L;
+        urev = REV;
     } else {
         urow = static_cast<const Tin *>(p.u) + (b * C4 + c) * L;
         urev = false;
     }
-    const Tin *drow = static_cast<const Tin *>(p.delta) + (b * C4 + c) * L;
-    const Tin *Bk = static_cast<const Tin *>(p.Bm) + (b * kPaths + k) * N * L;
-    const Tin *Ck = static_cast<const Tin *>(p.Cm) + (b * kPaths + k) * N * L;
+    const Tin *drow = static_cast<const Tin *>(p.delta) + (BIDIR ? b * D + (active ? d : 0) : b * C4 + c) * L;
+    const int64_t grp = BIDIR ? b : b * kPaths + k;  // the B/C group of this (b, k)
+    const Tin *Bk = static_cast<const Tin *>(p.Bm) + grp * N * L;
+    const Tin *Ck = static_cast<const Tin *>(p.Cm) + grp * N * L;
     Tout *orow = p.out ? static_cast<Tout *>(p.out) + (b * C4 + c) * L : nullptr;
 
     const int64_t nloc = lend - lbeg;
@@ -236,7 +288,7 @@ __global__ void __launch_bounds__(kWarp, SS2D_FWD_MIN_BLOCKS) scan_fwd_kernel(co
     }
     __syncwarp();
 
-    stage_chunk<NS, VEC>(stage[0], Bk, Ck, N, L, urow, urev, drow, active, lbeg, (int)min((int64_t)kLC, nloc));
+    stage_chunk<NS, VEC, REV>(stage[0], Bk, Ck, N, L, urow, urev, drow, active, lbeg, (int)min((int64_t)kLC, nloc));
     cp_async_commit();
 
     for (int ch = 0; ch < nchunk; ++ch) {
@@ -245,7 +297,7 @@ __global__ void __launch_bounds__(kWarp, SS2D_FWD_MIN_BLOCKS) scan_fwd_kernel(co
         const int buf = ch & 1;
         if (ch + 1 < nchunk) {
             const int64_t nbeg = cbeg + kLC;
-            stage_chunk<NS, VEC>(stage[buf ^ 1], Bk, Ck, N, L, urow, urev, drow, active, nbeg,
+            stage_chunk<NS, VEC, REV>(stage[buf ^ 1], Bk, Ck, N, L, urow, urev, drow, active, nbeg,
                                  (int)min((int64_t)kLC, lend - nbeg));
             cp_async_commit();
             cp_async_wait<1>();
@@ -260,8 +312,17 @@ __global__ void __launch_bounds__(kWarp, SS2D_FWD_MIN_BLOCKS) scan_fwd_kernel(co
                 const int64_t l0 = cbeg + g;
                 const int nvalid = (int)min((int64_t)kG, lend - l0);
                 float uv[kG], dv[kG];
-                if (VEC) {
-                    ld4(&sm.Dl[t][g], dv);
+                {  // slots hold 4-step groups in every staging form (see stage_chunk)
+                    if (!REV) {
+                        ld4(&sm.Dl[t][g], dv);
+                    } else {
+                        float w[kG];
+                        ld4(&sm.Dl[t][kLC - 4 - g], w);
+                        dv[0] = w[3];
+                        dv[1] = w[2];
+                        dv[2] = w[1];
+                        dv[3] = w[0];
+                    }
                     if (!urev) {
                         ld4(&sm.U[t][g], uv);
                     } else {
@@ -271,12 +332,6 @@ __global__ void __launch_bounds__(kWarp, SS2D_FWD_MIN_BLOCKS) scan_fwd_kernel(co
                         uv[1] = w[2];
                         uv[2] = w[1];
                         uv[3] = w[0];
-                    }
-                } else {
-#pragma unroll
-                    for (int j = 0; j < kG; ++j) {
-                        dv[j] = (g + j < kLC) ? ld(&sm.Dl[t][g + j]) : 0.f;
-                        uv[j] = (g + j < kLC) ? ld(&sm.U[t][urev ? (kLC - 1 - g - j) : (g + j)]) : 0.f;
                     }
                 }
                 // step pairs (0,1) and (2,3) ride the packed fp32 pipe (f32x2)
@@ -302,14 +357,17 @@ __global__ void __launch_bounds__(kWarp, SS2D_FWD_MIN_BLOCKS) scan_fwd_kernel(co
                     const float a2s = SS2D_A2(n);
                     const float2 a2 = make_float2(a2s, a2s);
                     float bq[kG], cq[kG];
-                    if (VEC) {
+                    if (!REV) {
                         ld4(&sm.B[n][g], bq);
                         ld4(&sm.C[n][g], cq);
                     } else {
+                        float wb[kG], wc[kG];
+                        ld4(&sm.B[n][kLC - 4 - g], wb);
+                        ld4(&sm.C[n][kLC - 4 - g], wc);
 #pragma unroll
                         for (int j = 0; j < kG; ++j) {
-                            bq[j] = (g + j < kLC) ? ld(&sm.B[n][g + j]) : 0.f;
-                            cq[j] = (g + j < kLC) ? ld(&sm.C[n][g + j]) : 0.f;
+                            bq[j] = wb[kG - 1 - j];
+                            cq[j] = wc[kG - 1 - j];
                         }
                     }
                     const float2 x01 = __fmul2_rn(dt01, a2), x23 = __fmul2_rn(dt23, a2);
@@ -344,7 +402,7 @@ __global__ void __launch_bounds__(kWarp, SS2D_FWD_MIN_BLOCKS) scan_fwd_kernel(co
                     dtsum += (dt01.x + dt01.y) + (dt23.x + dt23.y);
                 } else {
                     float y[kG] = {y01.x, y01.y, y23.x, y23.y};
-                    if (!IMG && p.z) {  // output gate: y * silu(z), after the D u term
+                    if (SEQ && p.z) {  // output gate: y * silu(z), after the D u term
                         const Tin *zrow = static_cast<const Tin *>(p.z) + (b * C4 + c) * L;
                         float zv[kG];
                         if (VEC) {
@@ -357,20 +415,28 @@ __global__ void __launch_bounds__(kWarp, SS2D_FWD_MIN_BLOCKS) scan_fwd_kernel(co
                         for (int j = 0; j < kG; ++j) y[j] *= silu_f(zv[j]);
                     }
                     if (orow) {
-                        if (VEC) {
+                        if (VEC && !REV) {
                             st4(orow + l0, y);
+                        } else if (VEC) {  // the reverse direction stores at the natural positions
+                            const float yr[kG] = {y[3], y[2], y[1], y[0]};
+                            st4(orow + (L - kG - l0), yr);
                         } else {
 #pragma unroll
                             for (int j = 0; j < kG; ++j)
-                                if (j < nvalid) st(orow + l0 + j, y[j]);
+                                if (j < nvalid) st(orow + (REV ? L - 1 - (l0 + j) : l0 + j), y[j]);
                         }
                     }
                     const int64_t llast = l0 + nvalid - 1;
                     if (p.chunk_states && (((llast + 1) % kStateChunk) == 0 || llast + 1 == L)) {
                         float *cs = p.chunk_states + ((b * C4 + c) * p.nchunks + llast / kStateChunk) * N;
+                        if (N == NS && NS % 4 == 0) {  // 16-byte aligned rows of N floats
 #pragma unroll
-                        for (int n = 0; n < NS; ++n)
-                            if (n < N) cs[n] = h[n];
+                            for (int n = 0; n < NS; n += 4) st4(cs + n, &h[n]);
+                        } else {
+#pragma unroll
+                            for (int n = 0; n < NS; ++n)
+                                if (n < N) cs[n] = h[n];
+                        }
                     }
                 }
             }
@@ -378,7 +444,7 @@ __global__ void __launch_bounds__(kWarp, SS2D_FWD_MIN_BLOCKS) scan_fwd_kernel(co
         __syncwarp();  // every lane is done with this buffer before it is refilled
     }
 
-    if (!IMG && PASS != 1 && active && p.last_state && sgi == p.nseg - 1) {  // sequence mode only
+    if (SEQ && PASS != 1 && active && p.last_state && sgi == p.nseg - 1) {  // sequence mode only
         float *ls = p.last_state + (b * C4 + c) * N;
 #pragma unroll
         for (int n = 0; n < NS; ++n)
@@ -397,11 +463,21 @@ __global__ void __launch_bounds__(kWarp, SS2D_FWD_MIN_BLOCKS) scan_fwd_kernel(co
 
 #undef SS2D_A2
 
+template <int NS, typename Tin, typename Tout, int MODE, int PASS, bool VEC>
+__global__ void __launch_bounds__(kWarp, SS2D_FWD_MIN_BLOCKS) scan_fwd_kernel(const FwdParams p) {
+    __shared__ __align__(16) FwdStage<Tin, NS> stage[2];
+    __shared__ float A2s[a2_in_smem<Tin>() ? NS : 1][kWarp];
+    if (MODE == kModeBidir && blockIdx.y == 1)
+        scan_fwd_body<NS, Tin, Tout, MODE, PASS, VEC, true>(p, stage, A2s);
+    else
+        scan_fwd_body<NS, Tin, Tout, MODE, PASS, VEC, false>(p, stage, A2s);
+}
+
 // Segment plan: how many segments each sequence is cut into, and their length
 // (a multiple of the state-chunk length).  One segment means a single pass.
-static void seg_plan(const LaunchShape &s, int max_segments, int *nseg_out, int64_t *seglen_out) {
+static void seg_plan(const LaunchShape &s, int paths, int max_segments, int *nseg_out, int64_t *seglen_out) {
     // aim for at least ~512 resident sequences (threads) per SM on 148 SMs
-    const int64_t seqs = s.B * kPaths * s.D;
+    const int64_t seqs = s.B * paths * s.D;
     const int64_t target = 148LL * 512;
     *nseg_out = 1;
     *seglen_out = s.L;
@@ -416,47 +492,47 @@ static void seg_plan(const LaunchShape &s, int max_segments, int *nseg_out, int6
     *nseg_out = (int)ceil_div(s.L, seglen);
 }
 
-int scan_fwd_segments(const LaunchShape &s) {
+int scan_fwd_segments(const LaunchShape &s, int paths) {
     int nseg;
     int64_t seglen;
-    seg_plan(s, 32, &nseg, &seglen);
+    seg_plan(s, paths, 32, &nseg, &seglen);
     return nseg;
 }
 
-size_t scan_fwd_workspace_bytes(const LaunchShape &s) {
-    const int nseg = scan_fwd_segments(s);
+size_t scan_fwd_workspace_bytes(const LaunchShape &s, int paths) {
+    const int nseg = scan_fwd_segments(s, paths);
     if (nseg <= 1) return 0;
-    return (size_t)s.B * kPaths * s.D * nseg * 2 * s.N * sizeof(float);
+    return (size_t)s.B * paths * s.D * nseg * 2 * s.N * sizeof(float);
 }
 
-template <int NS, typename Tin, typename Tout, bool IMG, bool VEC>
+template <int NS, typename Tin, typename Tout, int MODE, bool VEC>
 static cudaError_t launch_ns(const FwdParams &p, cudaStream_t stream) {
-    dim3 grid((unsigned)ceil_div(p.D, kWarp), kPaths, (unsigned)(p.B * p.nseg));
+    dim3 grid((unsigned)ceil_div(p.D, kWarp), MODE == kModeBidir ? 2 : kPaths, (unsigned)(p.B * p.nseg));
     if (p.nseg == 1) {
-        scan_fwd_kernel<NS, Tin, Tout, IMG, 0, VEC><<<grid, kWarp, 0, stream>>>(p);
+        scan_fwd_kernel<NS, Tin, Tout, MODE, 0, VEC><<<grid, kWarp, 0, stream>>>(p);
         note_launch(stream);
     } else {
-        scan_fwd_kernel<NS, Tin, Tout, IMG, 1, VEC><<<grid, kWarp, 0, stream>>>(p);
+        scan_fwd_kernel<NS, Tin, Tout, MODE, 1, VEC><<<grid, kWarp, 0, stream>>>(p);
         note_launch(stream);
-        scan_fwd_kernel<NS, Tin, Tout, IMG, 2, VEC><<<grid, kWarp, 0, stream>>>(p);
+        scan_fwd_kernel<NS, Tin, Tout, MODE, 2, VEC><<<grid, kWarp, 0, stream>>>(p);
         note_launch(stream);
     }
     return cudaGetLastError();
 }
 
-template <typename Tin, typename Tout, bool IMG, bool VEC>
+template <typename Tin, typename Tout, int MODE, bool VEC>
 static cudaError_t launch_types(const FwdParams &p, cudaStream_t stream) {
-    if (p.N <= 4) return launch_ns<4, Tin, Tout, IMG, VEC>(p, stream);
-    if (p.N <= 8) return launch_ns<8, Tin, Tout, IMG, VEC>(p, stream);
-    return launch_ns<16, Tin, Tout, IMG, VEC>(p, stream);
+    if (p.N <= 4) return launch_ns<4, Tin, Tout, MODE, VEC>(p, stream);
+    if (p.N <= 8) return launch_ns<8, Tin, Tout, MODE, VEC>(p, stream);
+    return launch_ns<16, Tin, Tout, MODE, VEC>(p, stream);
 }
 
-template <bool IMG, bool VEC>
-static cudaError_t launch_img(const FwdParams &p, ss2d_dtype_t din, ss2d_dtype_t dout, cudaStream_t stream) {
-    if (din == SS2D_F32 && dout == SS2D_F32) return launch_types<float, float, IMG, VEC>(p, stream);
-    if (din == SS2D_F32) return launch_types<float, __nv_bfloat16, IMG, VEC>(p, stream);
-    if (dout == SS2D_F32) return launch_types<__nv_bfloat16, float, IMG, VEC>(p, stream);
-    return launch_types<__nv_bfloat16, __nv_bfloat16, IMG, VEC>(p, stream);
+template <int MODE, bool VEC>
+static cudaError_t launch_mode(const FwdParams &p, ss2d_dtype_t din, ss2d_dtype_t dout, cudaStream_t stream) {
+    if (din == SS2D_F32 && dout == SS2D_F32) return launch_types<float, float, MODE, VEC>(p, stream);
+    if (din == SS2D_F32) return launch_types<float, __nv_bfloat16, MODE, VEC>(p, stream);
+    if (dout == SS2D_F32) return launch_types<__nv_bfloat16, float, MODE, VEC>(p, stream);
+    return launch_types<__nv_bfloat16, __nv_bfloat16, MODE, VEC>(p, stream);
 }
 
 cudaError_t launch_scan_fwd(const LaunchShape &s, const ScanFwdArgs &a, void *workspace, cudaStream_t stream) {
@@ -471,8 +547,9 @@ cudaError_t launch_scan_fwd(const LaunchShape &s, const ScanFwdArgs &a, void *wo
     p.bias = a.bias;
     p.out = a.out;
     p.chunk_states = a.chunk_states;
-    p.z = a.from_image ? nullptr : a.z;
-    p.last_state = a.from_image ? nullptr : a.last_state;
+    const bool seq = !a.from_image && !a.bidir;
+    p.z = seq ? a.z : nullptr;
+    p.last_state = seq ? a.last_state : nullptr;
     p.seg = static_cast<float *>(workspace);
     p.B = s.B;
     p.D = s.D;
@@ -481,15 +558,22 @@ cudaError_t launch_scan_fwd(const LaunchShape &s, const ScanFwdArgs &a, void *wo
     p.L = s.L;
     p.N = (int)s.N;
     p.softplus = a.softplus;
-    seg_plan(s, a.max_segments, &p.nseg, &p.seglen);
+    seg_plan(s, a.bidir ? 2 : kPaths, a.max_segments, &p.nseg, &p.seglen);
     p.nchunks = ceil_div(s.L, kStateChunk);
     // 4-step vector loads need every row start and step group 4-element aligned
     const bool vec = (s.L % 4) == 0;
+    if (a.bidir) {  // the merge that follows reads fp32 per-direction outputs
+        if (a.in_dtype == SS2D_F32)
+            return vec ? launch_types<float, float, kModeBidir, true>(p, stream)
+                       : launch_types<float, float, kModeBidir, false>(p, stream);
+        return vec ? launch_types<__nv_bfloat16, float, kModeBidir, true>(p, stream)
+                   : launch_types<__nv_bfloat16, float, kModeBidir, false>(p, stream);
+    }
     if (a.from_image)
-        return vec ? launch_img<true, true>(p, a.in_dtype, a.out_dtype, stream)
-                   : launch_img<true, false>(p, a.in_dtype, a.out_dtype, stream);
-    return vec ? launch_img<false, true>(p, a.in_dtype, a.out_dtype, stream)
-               : launch_img<false, false>(p, a.in_dtype, a.out_dtype, stream);
+        return vec ? launch_mode<kModeImg, true>(p, a.in_dtype, a.out_dtype, stream)
+                   : launch_mode<kModeImg, false>(p, a.in_dtype, a.out_dtype, stream);
+    return vec ? launch_mode<kModeSeq, true>(p, a.in_dtype, a.out_dtype, stream)
+               : launch_mode<kModeSeq, false>(p, a.in_dtype, a.out_dtype, stream);
 }
 
 }  // namespace ss2d

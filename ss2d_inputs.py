@@ -20,6 +20,15 @@ Draw order from one torch.Generator seeded with the workload index:
 u, delta, B, C, dt, dy.  The same seed on another device gives other values
 (torch's CPU and CUDA generators differ); every consumer receives the tensors
 themselves, so the oracle and the kernels always see identical numbers.
+
+The bidirectional scan (bimamba_inner_ref on the same page) takes a sequence of
+tokens.  Its workload follows the VisionMamba call printed on "Vision Mamba架构深入解析"
+(jsqmd.com), section "双向状态空间模型设计" (bidirectional state-space model design):
+img_size=224, patch_size=16, embed_dim=192, so 14 x 14 = 196 patch tokens plus
+a class token, L = 197, and an inner width of 2 x 192 = 384 channels (the
+Mamba block's default expansion of 2), d_state 16.  Its A and A_b both follow
+the S4D-real initialisation; tests may ask for A_b scaled elementwise by a
+seeded factor in [0.5, 1.5] so that the two directions differ.
 """
 from __future__ import annotations
 
@@ -43,19 +52,24 @@ class Workload:
     a_init: str       # "neg_index": A = -(n+1) exactly; "s4d_real": -exp(log(n+1)) in fp32
     backward: bool = False
     description: str = ""
+    kind: str = "ss2d"  # "ss2d": four paths over an H x W map; "bidir": a sequence and its reverse
 
     @property
     def L(self) -> int:
         return self.height * self.width
 
     @property
+    def paths(self) -> int:
+        return 2 if self.kind == "bidir" else K_PATHS
+
+    @property
     def channels(self) -> int:
-        return K_PATHS * self.dim
+        return self.paths * self.dim
 
     @property
     def updates(self) -> int:
-        """state updates of one forward: B * 4 * D * L * N"""
-        return self.batch * K_PATHS * self.dim * self.L * self.d_state
+        """state updates of one forward: B * paths * D * L * N"""
+        return self.batch * self.paths * self.dim * self.L * self.d_state
 
     @property
     def torch_dtype(self):
@@ -76,6 +90,8 @@ WORKLOADS = [
              description="high-resolution SS2D fwd, B=8 D=192 H=W=128 (L=16384) N=16, bf16 in / fp32 state"),
     Workload("vmamba_t_stage1_fwd_bwd_fp32", 32, 192, 56, 56, 16, "f32", "s4d_real", backward=True,
              description="SS2D fwd+bwd, B=32 D=192 H=W=56 N=16, fp32, dy ~ N(0,1)"),
+    Workload("vim_t_bidir_fp32", 128, 384, 1, 197, 16, "f32", "s4d_real", kind="bidir",
+             description="bidirectional scan (Vim-T tokens), B=128 D=384 L=197 N=16, fp32, gate z"),
 ]
 
 
@@ -88,9 +104,9 @@ def workload(index_or_name) -> Workload:
     raise KeyError(index_or_name)
 
 
-def custom(batch, dim, height, width, d_state, dtype="f32", a_init="neg_index", backward=True):
-    return Workload(f"custom_{batch}x{dim}x{height}x{width}_n{d_state}_{dtype}", batch, dim, height,
-                    width, d_state, dtype, a_init, backward)
+def custom(batch, dim, height, width, d_state, dtype="f32", a_init="neg_index", backward=True, kind="ss2d"):
+    return Workload(f"custom_{kind}_{batch}x{dim}x{height}x{width}_n{d_state}_{dtype}", batch, dim, height,
+                    width, d_state, dtype, a_init, backward, kind=kind)
 
 
 def make_inputs(w: Workload, seed: int = 0, device="cpu", with_dy: bool | None = None):
@@ -130,11 +146,46 @@ def make_inputs(w: Workload, seed: int = 0, device="cpu", with_dy: bool | None =
     return out
 
 
+def make_bimamba_inputs(w: Workload, seed: int = 0, device="cpu", with_dy: bool = False, with_z: bool = False,
+                        distinct_a_b: bool = False):
+    """Draw one bidirectional-scan problem (w.kind == "bidir", w.height == 1).  Returns x, delta,
+    z (B, D, L); A, A_b (D, N) fp32; B, C (B, N, L); D, delta_bias (D) fp32; dy (B, D, L) if asked.
+    Draw order: x, delta, B, C, dt, [z], [dy], [A_b factor]."""
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed) + 2000)
+    f32 = dict(dtype=torch.float32, device=device, generator=g)
+    Bn, Dn, L, N = w.batch, w.dim, w.L, w.d_state
+    x = torch.randn((Bn, Dn, L), **f32)
+    delta = torch.randn((Bn, Dn, L), **f32) * 0.1
+    Bm = torch.randn((Bn, N, L), **f32)
+    Cm = torch.randn((Bn, N, L), **f32)
+    dt_min, dt_max, dt_floor = 1e-3, 1e-1, 1e-4
+    dt = torch.exp(torch.rand((Dn,), **f32) * (math.log(dt_max) - math.log(dt_min))
+                   + math.log(dt_min)).clamp(min=dt_floor)
+    delta_bias = dt + torch.log(-torch.expm1(-dt))
+    n1 = torch.arange(1, N + 1, dtype=torch.float32, device=device)
+    A_row = -n1 if w.a_init == "neg_index" else -torch.exp(torch.log(n1))
+    A = A_row.unsqueeze(0).repeat(Dn, 1).contiguous()
+    out = dict(x=x, delta=delta, A=A, A_b=A.clone(), B=Bm, C=Cm, D=torch.ones(Dn, dtype=torch.float32, device=device),
+               delta_bias=delta_bias)
+    if with_z:
+        out["z"] = torch.randn((Bn, Dn, L), **f32)
+    if with_dy:
+        out["dy"] = torch.randn((Bn, Dn, L), **f32)
+    if distinct_a_b:
+        out["A_b"] = (A * (0.5 + torch.rand((Dn, N), **f32))).contiguous()
+    if w.dtype == "bf16":
+        for key in ("x", "delta", "B", "C", "z", "dy"):
+            if key in out:
+                out[key] = out[key].to(torch.bfloat16)
+    return out
+
+
 def batch_slice(inputs: dict, idx) -> dict:
     """Restrict batch-indexed tensors to batch items `idx` (a list); parameters are shared."""
     out = {}
     for k, v in inputs.items():
-        if k in ("x", "delta", "B", "C", "dy"):
+        if k in ("x", "delta", "B", "C", "dy", "z", "u", "dout"):
             out[k] = v[idx]
         else:
             out[k] = v

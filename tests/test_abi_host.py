@@ -113,6 +113,29 @@ def test_gated_scan_argument_errors(lib):
              None) == ERR_WORKSPACE
 
 
+def test_bimamba_argument_errors(lib):
+    f = lib.ss2d_bimamba_forward
+    wsf = lib.ss2d_workspace_bytes(_d(H=1, W=37), ss.OP_BIMAMBA_FORWARD)
+    wsb = lib.ss2d_workspace_bytes(_d(H=1, W=37), ss.OP_BIMAMBA_BACKWARD)
+    assert 0 < wsf < wsb
+    args = [A16] * 5  # x, delta, A, B, C
+    # a sequence is a 1 x L image
+    assert f(_d(H=2, W=37), *args, None, None, None, 1, B16, None, A16, wsf, None) == ERR_SHAPE
+    assert f(_d(H=1, W=37), *args, None, None, None, 1, None, None, A16, wsf, None) == ERR_NULL
+    assert f(_d(H=1, W=37), *args, None, None, None, 1, B16, None, A16, wsf - 1, None) == ERR_WORKSPACE
+    assert f(_d(H=1, W=37), *args, None, ctypes.c_void_p(0x10004), None, 1, B16, None, A16, wsf,
+             None) == ERR_ALIGN
+    g = lib.ss2d_bimamba_backward
+    grads = [A16] * 5  # dx, ddelta, dA, dB, dC
+    # z given but dz missing, and the reverse
+    assert g(_d(H=1, W=37), *args, None, A16, None, 1, A16, None, *grads, None, None, None, A16, wsb,
+             None) == ERR_NULL
+    assert g(_d(H=1, W=37), *args, None, None, None, 1, A16, None, *grads, None, None, A16, A16, wsb,
+             None) == ERR_NULL
+    assert g(_d(H=1, W=37), *args, None, A16, None, 1, A16, None, *grads, None, None, A16, A16, wsb - 1,
+             None) == ERR_WORKSPACE
+
+
 def test_valid_call_without_gpu_reports_device_error(lib):
     import torch
     if torch.cuda.is_available():

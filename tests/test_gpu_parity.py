@@ -309,6 +309,113 @@ def test_selective_scan_fn_autograd():
         assert_rel_l2(leaves[k].grad, ref[rname], GRAD_TOL, k)
 
 
+# ------------------------------------------------------- bidirectional scan
+
+def _bidir_case(Bn, Dn, L, N, dtype="f32", seed=0, with_z=True):
+    w = ss2d_inputs.custom(Bn, Dn, 1, L, N, dtype=dtype, a_init="s4d_real", kind="bidir")
+    return w, ss2d_inputs.make_bimamba_inputs(w, seed=seed, with_dy=True, with_z=with_z, distinct_a_b=True)
+
+
+# L = 1, ragged L (scalar staging), several 16-step blocks and 64-channel tiles, N < 16
+BIDIR_CASES = [(1, 8, 16, 4), (2, 40, 37, 16), (1, 3, 1, 3), (2, 70, 200, 16), (1, 5, 197, 8), (3, 33, 64, 16)]
+BIDIR_BWD_NAMES = ["dx", "ddelta", "dA", "dA_b", "dB", "dC", "dD", "ddelta_bias", "dz"]
+
+
+def _bidir_ref_fwd(inp, z=True):
+    return oracle.bimamba_forward(inp["x"], inp["delta"], inp["A"], inp["A_b"], inp["B"], inp["C"], inp["D"],
+                                  inp["z"] if z else None, inp["delta_bias"], True)
+
+
+@pytest.mark.parametrize("case", BIDIR_CASES)
+@pytest.mark.parametrize("gated", [True, False])
+def test_bimamba_forward_parity(case, gated):
+    w, inp = _bidir_case(*case, seed=40, with_z=gated)
+    d = _dev(inp)
+    y = ss.bimamba_forward(d["x"], d["delta"], d["A"], d["A_b"], d["B"], d["C"], d["D"], d.get("z"),
+                           d["delta_bias"], True)
+    assert_rel_l2(y, _bidir_ref_fwd(inp, gated), FWD_TOL, f"{case} y")
+
+
+@pytest.mark.parametrize("case", BIDIR_CASES)
+@pytest.mark.parametrize("with_states", [False, True])
+def test_bimamba_backward_parity(case, with_states):
+    w, inp = _bidir_case(*case, seed=41)
+    d = _dev(inp)
+    args = (d["x"], d["delta"], d["A"], d["A_b"], d["B"], d["C"], d["D"], d["z"], d["delta_bias"], True)
+    cs = None
+    if with_states:
+        _, cs = ss.bimamba_forward(*args, return_chunk_states=True)
+    g = ss.bimamba_backward(*args, d["dy"], chunk_states=cs)
+    ref = oracle.bimamba_backward(inp["x"], inp["delta"], inp["A"], inp["A_b"], inp["B"], inp["C"], inp["D"],
+                                  inp["z"], inp["delta_bias"], True, inp["dy"])
+    for name in BIDIR_BWD_NAMES:
+        assert_rel_l2(g[name], ref[name], GRAD_TOL, f"{case} {name}")
+
+
+def test_bimamba_without_optional_inputs():
+    w, inp = _bidir_case(2, 12, 45, 16, seed=42, with_z=False)
+    d = _dev(inp)
+    y = ss.bimamba_forward(d["x"], d["delta"], d["A"], d["A_b"], d["B"], d["C"])
+    ref = oracle.bimamba_forward(inp["x"], inp["delta"], inp["A"], inp["A_b"], inp["B"], inp["C"])
+    assert_rel_l2(y, ref, FWD_TOL, "y")
+    g = ss.bimamba_backward(d["x"], d["delta"], d["A"], d["A_b"], d["B"], d["C"], None, None, None, True, d["dy"])
+    assert g["dD"] is None and g["ddelta_bias"] is None and g["dz"] is None
+    r = oracle.bimamba_backward(inp["x"], inp["delta"], inp["A"], inp["A_b"], inp["B"], inp["C"], None, None, None,
+                                True, inp["dy"])
+    for name in ("dx", "ddelta", "dA", "dA_b", "dB", "dC"):
+        assert_rel_l2(g[name], r[name], GRAD_TOL, name)
+
+
+def test_bimamba_bf16():
+    w, inp = _bidir_case(2, 16, 60, 16, dtype="bf16", seed=43)
+    d = _dev(inp)
+    args = (d["x"], d["delta"], d["A"], d["A_b"], d["B"], d["C"], d["D"], d["z"], d["delta_bias"], True)
+    y = ss.bimamba_forward(*args)
+    assert y.dtype == torch.bfloat16
+    assert_rel_l2(y, _bidir_ref_fwd(inp), BF16_TOL, "y")
+    g = ss.bimamba_backward(*args, d["dy"])
+    ref = oracle.bimamba_backward(inp["x"], inp["delta"], inp["A"], inp["A_b"], inp["B"], inp["C"], inp["D"],
+                                  inp["z"], inp["delta_bias"], True, inp["dy"])
+    for name in BIDIR_BWD_NAMES:
+        assert_rel_l2(g[name], ref[name], BF16_TOL, name)
+
+
+def test_bimamba_autograd():
+    w, inp = _bidir_case(2, 6, 29, 16, seed=44)
+    d = _dev(inp)
+    names = ("x", "delta", "A", "A_b", "B", "C", "D", "z", "delta_bias")
+    leaves = {k: d[k].clone().requires_grad_(True) for k in names}
+    y = ss.bimamba_scan(leaves["x"], leaves["delta"], leaves["A"], leaves["A_b"], leaves["B"], leaves["C"],
+                        leaves["D"], leaves["z"], leaves["delta_bias"], True)
+    y.backward(d["dy"])
+    ref = oracle.bimamba_backward(inp["x"], inp["delta"], inp["A"], inp["A_b"], inp["B"], inp["C"], inp["D"],
+                                  inp["z"], inp["delta_bias"], True, inp["dy"])
+    gmap = dict(x="dx", delta="ddelta", A="dA", A_b="dA_b", B="dB", C="dC", D="dD", z="dz",
+                delta_bias="ddelta_bias")
+    for k, rname in gmap.items():
+        assert_rel_l2(leaves[k].grad, ref[rname], GRAD_TOL, k)
+
+
+def test_bimamba_full_vim_workload_sampled():
+    # the benchmark's bidirectional workload at full size, in the launch configuration bench.py
+    # times; batch items checked one by one against the oracle
+    w = ss2d_inputs.workload("vim_t_bidir_fp32")
+    inp = ss2d_inputs.make_bimamba_inputs(w, seed=5, with_dy=True, with_z=True, distinct_a_b=True)
+    d = _dev(inp)
+    args = (d["x"], d["delta"], d["A"], d["A_b"], d["B"], d["C"], d["D"], d["z"], d["delta_bias"], True)
+    y, cs = ss.bimamba_forward(*args, return_chunk_states=True)
+    g = ss.bimamba_backward(*args, d["dy"], chunk_states=cs)
+    for bi in (0, 77, w.batch - 1):
+        sl = ss2d_inputs.batch_slice(inp, [bi])
+        ref_y = oracle.bimamba_forward(sl["x"], sl["delta"], sl["A"], sl["A_b"], sl["B"], sl["C"], sl["D"],
+                                       sl["z"], sl["delta_bias"], True)
+        assert_rel_l2(y[bi:bi + 1], ref_y, FWD_TOL, f"y[{bi}]")
+        r = oracle.bimamba_backward(sl["x"], sl["delta"], sl["A"], sl["A_b"], sl["B"], sl["C"], sl["D"], sl["z"],
+                                    sl["delta_bias"], True, sl["dy"])
+        for name in ("dx", "ddelta", "dB", "dC", "dz"):
+            assert_rel_l2(g[name][bi:bi + 1], r[name], GRAD_TOL, f"{name}[{bi}]")
+
+
 # ------------------------------------------------------------- fused SS2D
 
 FUSED_CASES = [(1, 8, 8, 8, 4), (2, 6, 5, 9, 16), (1, 70, 12, 11, 16), (1, 8, 64, 64, 16), (2, 3, 1, 1, 2),
