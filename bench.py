@@ -48,6 +48,7 @@ UNIT = "state-updates/s"
 SM_COUNT = 148
 MUFU_EX2_PER_CLK_PER_SM = 16  # measured on this B200 pool: 16.00 MUFU.EX2 per clock per SM
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0, "source": "fallback"}
+REFERENCE_ITEMS_PER_STEP = 16
 
 
 def load_peaks():
@@ -105,20 +106,24 @@ def bwd_algorithmic_bytes(w, gate: bool = False) -> int:
     return s * (2 * img + 4 * img + bc) + s * (img + 4 * img + bc) + params
 
 
-def source_hash() -> str:
-    """Hash of the CUDA sources: ncu traffic figures are only reused for the exact same kernels."""
+# the files the recorded forward scan kernel is compiled from
+FWD_KERNEL_SOURCES = ("selective_scan_crossscan_b200/csrc/scan_fwd.cu", "selective_scan_crossscan_b200/csrc/common.cuh",
+                      "selective_scan_crossscan_b200/csrc/kernels.h", "include/ss2d.h")
+
+
+def source_hash(files=FWD_KERNEL_SOURCES) -> str:
+    """Hash of a kernel's source files: ncu traffic figures are only reused for the exact same kernel."""
     h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "selective_scan_crossscan_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode())
+    for rel in files:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(rel.encode())
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
 def recorded_traffic(workload_name: str):
     """dram read+write bytes per launch of the dominant kernel from a committed ncu capture, if the
-    kernels have not changed since it was taken; else None."""
+    kernel's sources have not changed since it was taken; else None."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
@@ -126,7 +131,13 @@ def recorded_traffic(workload_name: str):
     except (OSError, ValueError):
         return None
     entry = rec.get(workload_name)
-    if not entry or entry.get("source_hash") != source_hash():
+    if not entry:
+        return None
+    files = tuple(entry.get("sources") or FWD_KERNEL_SOURCES)
+    try:
+        if entry.get("source_hash") != source_hash(files):
+            return None
+    except OSError:
         return None
     return entry.get("traffic_bytes_per_launch")
 
@@ -248,31 +259,50 @@ def oracle_sample(w, seed: int, item: int):
     return ss2d_inputs.make_inputs(one, seed=seed + 7919 * item, device="cpu", with_dy=False)
 
 
-def time_oracle(w, seconds_budget: float = 20.0, steps: int = 1, warmup: int = 0):
-    """Time the fp64 oracle's SS2D forward on whole batch items of the workload (bounded sample)."""
+def _oracle_item(oracle, w, item: int) -> float:
+    """Seconds the fp64 oracle's SS2D forward takes on batch item `item` (inputs drawn untimed)."""
+    inp = oracle_sample(w, 0, item)
+    args = [oracle._f64(inp[k]) for k in ("x", "delta", "A", "B", "C", "D", "delta_bias")]
+    t0 = time.perf_counter()
+    oracle.ss2d_forward(*args, True)
+    return time.perf_counter() - t0
+
+
+def time_oracle(w, seconds_budget: float = 15.0, steps: int | None = None, warmup: int = 1,
+                items_per_step: int = 1):
+    """Time the fp64 oracle's SS2D forward on whole batch items of the workload (bounded sample).
+
+    steps=None: after `warmup` untimed items, time items one by one until `seconds_budget` seconds
+    of oracle time are spent or every batch item has run.  Otherwise: exactly `steps` steps of
+    `items_per_step` items each after the warm-up."""
     import oracle
     oracle.build()
-    samples = []
-    items_done = 0
-    t_total = 0.0
-    for i in range(warmup + steps):
-        inp = oracle_sample(w, 0, i)
-        args = [oracle._f64(inp[k]) for k in ("x", "delta", "A", "B", "C", "D", "delta_bias")]
-        t0 = time.perf_counter()
-        oracle.ss2d_forward(*args, True)
-        dt = time.perf_counter() - t0
-        if i >= warmup:
-            samples.append(dt)
+    for i in range(warmup):
+        _oracle_item(oracle, w, i)
+    items_done, t_total, step_s = 0, 0.0, []
+    item = warmup
+    if steps is None:
+        while items_done < w.batch and (items_done == 0 or t_total < seconds_budget):
+            t_total += _oracle_item(oracle, w, item % w.batch)
             items_done += 1
-            t_total += dt
-        if t_total > seconds_budget and i >= warmup:
-            break
+            item += 1
+    else:
+        for _ in range(steps):
+            t = 0.0
+            for _ in range(items_per_step):
+                t += _oracle_item(oracle, w, item % w.batch)
+                item += 1
+            step_s.append(t)
+            t_total += t
+            items_done += items_per_step
     per_item_updates = w.with_batch(1).updates
     value = items_done * per_item_updates / t_total
+    what = (f"{items_done} batch item(s) of {w.name} ({per_item_updates} updates each"
+            + (f", {items_per_step} per step" if steps is not None else "") + ")")
     return dict(value=value, unit=UNIT, cores=oracle.num_threads(), kind="oracle",
                 ms_per_item=1e3 * t_total / max(items_done, 1),
-                sample=f"{items_done} batch item(s) (1 of {w.batch} each, {per_item_updates} updates) of "
-                       f"{w.name}, fp64 C oracle with OpenMP over (batch, channel)",
+                ms_per_step=1e3 * t_total / len(step_s) if step_s else None,
+                sample=f"{what}, fp64 C oracle with OpenMP over (batch, channel)",
                 seconds=t_total)
 
 
@@ -412,7 +442,8 @@ def run_gpu(args, world, rank, local):
     sm_max = float(peaks.get("sm_max_mhz", FALLBACK_PEAKS["sm_max_mhz"]))
     sfu_peak = MUFU_EX2_PER_CLK_PER_SM * SM_COUNT * sm_max * 1e6 / 1e9  # G ex2/s at max clock
     sfu_achieved = w.updates / (dom_ms / 1e3) / 1e9  # one exp(dt*A) per state update
-    traffic = recorded_traffic(w.name)
+    # the traffic record is of the fused forward's scan kernel: other lines have no capture
+    traffic = recorded_traffic(w.name) if not (args.backward or args.gate or bidir) else None
 
     e2e = None
     if not (args.no_e2e or args.backward or args.gate or bidir):
@@ -499,7 +530,9 @@ def run_e2e(args, w, inp, dev, stream, world, rank):
 
 def run_reference(args, world, rank):
     w = ss2d_inputs.workload(args.workload)
-    base = time_oracle(w, seconds_budget=args.cpu_seconds, steps=args.steps, warmup=args.warmup)
+    # a step is a slice of REFERENCE_ITEMS_PER_STEP whole batch items (about half a second of oracle time
+    # for VMamba-T stage 1), so the default --steps/--warmup run takes well under a minute
+    base = time_oracle(w, steps=args.steps, warmup=args.warmup, items_per_step=REFERENCE_ITEMS_PER_STEP)
     return {
         "impl": "reference",
         "metric": METRIC,
@@ -508,7 +541,7 @@ def run_reference(args, world, rank):
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": base["ms_per_item"],
+        "ms_per_step": base["ms_per_step"],
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
