@@ -66,6 +66,12 @@ def _load():
             lib.oracle_ss2d_backward.argtypes = [l, l, l, l, l, P, P, P, P, P, P, P, ctypes.c_int,
                                                  P, P, P, P, P, P, P, P]
             lib.oracle_num_threads.restype = ctypes.c_int
+            LP = ctypes.POINTER(ctypes.c_long)
+            lib.oracle_cross_scan_table.argtypes = [l, l, l, LP, P, P]
+            lib.oracle_cross_merge_table.argtypes = [l, l, l, LP, P, P]
+            lib.oracle_ss2d_forward_table.argtypes = [l, l, l, l, LP, P, P, P, P, P, P, P, ctypes.c_int, P]
+            lib.oracle_ss2d_backward_table.argtypes = [l, l, l, l, LP, P, P, P, P, P, P, P, ctypes.c_int, P, P,
+                                                       P, P, P, P, P, P]
             _lib = lib
     return _lib
 
@@ -154,6 +160,89 @@ def selective_scan_bwd(u, delta, A, B, C, D, delta_bias, delta_softplus, dout, z
                                       _ptr(z), _ptr(dout), _ptr(du), _ptr(ddelta), _ptr(dA), _ptr(dB),
                                       _ptr(dC), _ptr(dD), _ptr(dbias), _ptr(dz))
     return dict(du=du, ddelta=ddelta, dA=dA, dB=dB, dC=dC, dD=dD, ddelta_bias=dbias, dz=dz)
+
+
+# ---------------------------------------------------------------- path sets
+
+def cross_paths(H: int, W: int):
+    """(4, H*W) table of the VMamba page's cross scan: row-major, column-major, both reversed."""
+    L = H * W
+    return np.array([[path_pixel(k, l, H, W) for l in range(L)] for k in range(K_PATHS)], dtype=np.int64)
+
+
+def diagonal_order(H: int, W: int, direction: int):
+    """Pixel order of the diagonal scans of "Visual Mamba实战从零开始搭建图像分类模型附PyTorch代码"
+    (section 3, SS2D._get_diagonal_indices): anti-diagonals s = 0 .. H+W-2 in turn, rows i ascending
+    within each; column j = s - i for direction > 0, j = (W-1) - (s - i) otherwise."""
+    order = []
+    for s in range(H + W - 1):
+        for i in range(max(0, s - W + 1), min(s + 1, H)):
+            j = s - i if direction > 0 else (W - 1) - (s - i)
+            order.append(i * W + j)
+    return np.array(order, dtype=np.int64)
+
+
+def diagonal_paths(H: int, W: int):
+    """(4, H*W) table: the two diagonal orders, then each of them reversed (paths 2, 3), the same
+    structure as the cross scan's path set."""
+    d0, d1 = diagonal_order(H, W, 1), diagonal_order(H, W, -1)
+    return np.stack([d0, d1, d0[::-1], d1[::-1]]).astype(np.int64)
+
+
+def _table(table, L):
+    t = np.ascontiguousarray(np.asarray(table, dtype=np.int64).reshape(K_PATHS, L))
+    return t, t.ctypes.data_as(ctypes.POINTER(ctypes.c_long))
+
+
+def cross_scan_table(x, table):
+    """x (B, D, H, W) -> xs (B, 4, D, L) along the four paths of `table` (4, L)."""
+    x = _f64(x)
+    Bn, Dn, H, W = x.shape
+    t, tp = _table(table, H * W)
+    xs = np.empty((Bn, K_PATHS, Dn, H * W), dtype=np.float64)
+    _load().oracle_cross_scan_table(Bn, Dn, H * W, tp, _ptr(x), _ptr(xs))
+    return xs
+
+
+def cross_merge_table(ys, H: int, W: int, table):
+    ys = _f64(ys)
+    Bn, K, Dn, L = ys.shape
+    t, tp = _table(table, L)
+    y = np.empty((Bn, Dn, H, W), dtype=np.float64)
+    _load().oracle_cross_merge_table(Bn, Dn, L, tp, _ptr(ys), _ptr(y))
+    return y
+
+
+def ss2d_forward_table(x, delta, A, B, C, D, delta_bias, delta_softplus, table):
+    """SS2D forward over the path set `table` (4, L)."""
+    x, delta, A, B, C = (_f64(t) for t in (x, delta, A, B, C))
+    D, delta_bias = _f64(D), _f64(delta_bias)
+    Bn, Dn, H, W = x.shape
+    N = A.shape[1]
+    t, tp = _table(table, H * W)
+    y = np.empty_like(x)
+    _load().oracle_ss2d_forward_table(Bn, Dn, H * W, N, tp, _ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C),
+                                      _ptr(D), _ptr(delta_bias), int(bool(delta_softplus)), _ptr(y))
+    return y
+
+
+def ss2d_backward_table(x, delta, A, B, C, D, delta_bias, delta_softplus, dy, table):
+    x, delta, A, B, C, dy = (_f64(t) for t in (x, delta, A, B, C, dy))
+    D, delta_bias = _f64(D), _f64(delta_bias)
+    Bn, Dn, H, W = x.shape
+    N = A.shape[1]
+    t, tp = _table(table, H * W)
+    dx = np.empty_like(x)
+    ddelta = np.empty_like(delta)
+    dA = np.empty_like(A)
+    dB = np.empty_like(B)
+    dC = np.empty_like(C)
+    dD = np.empty(K_PATHS * Dn, dtype=np.float64) if D is not None else None
+    dbias = np.empty(K_PATHS * Dn, dtype=np.float64) if delta_bias is not None else None
+    _load().oracle_ss2d_backward_table(Bn, Dn, H * W, N, tp, _ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C),
+                                       _ptr(D), _ptr(delta_bias), int(bool(delta_softplus)), _ptr(dy), _ptr(dx),
+                                       _ptr(ddelta), _ptr(dA), _ptr(dB), _ptr(dC), _ptr(dD), _ptr(dbias))
+    return dict(dx=dx, ddelta=ddelta, dA=dA, dB=dB, dC=dC, dD=dD, ddelta_bias=dbias)
 
 
 def _flip(t):

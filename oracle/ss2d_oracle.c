@@ -338,6 +338,76 @@ void oracle_ss2d_backward(long Bn, long Dn, long H, long W, long N,
     free(dus);
 }
 
+/* ---------------------------------------------------- path sets as data -- */
+
+/*
+ * The same three steps for any four paths given as a table: table[k * L + l]
+ * is the pixel visited at step l of path k (each row a permutation of 0..L-1).
+ * Row-major / column-major / reversed (the VMamba page's cross scan) is one
+ * such table; the diagonal scans of "Visual Mamba实战从零开始搭建图像分类模型
+ * 附PyTorch代码" (section 3, _get_diagonal_indices) give another.
+ */
+void oracle_cross_scan_table(long Bn, long Dn, long L, const long *table, const double *x, double *xs)
+{
+    for (long b = 0; b < Bn; ++b)
+        for (int k = 0; k < K_PATHS; ++k)
+            for (long d = 0; d < Dn; ++d)
+                for (long l = 0; l < L; ++l)
+                    xs[((b * K_PATHS + k) * Dn + d) * L + l] = x[(b * Dn + d) * L + table[k * L + l]];
+}
+
+/* y[b, d, p] = (t0[p] + t2[p]) + (t1[p] + t3[p]) where t_k[table[k][l]] = ys[b, k, d, l] */
+void oracle_cross_merge_table(long Bn, long Dn, long L, const long *table, const double *ys, double *y)
+{
+    double *t = (double *)malloc(sizeof(double) * (size_t)(K_PATHS * L));
+    for (long b = 0; b < Bn; ++b)
+        for (long d = 0; d < Dn; ++d) {
+            for (int k = 0; k < K_PATHS; ++k)
+                for (long l = 0; l < L; ++l)
+                    t[k * L + table[k * L + l]] = ys[((b * K_PATHS + k) * Dn + d) * L + l];
+            for (long p = 0; p < L; ++p)
+                y[(b * Dn + d) * L + p] = (t[0 * L + p] + t[2 * L + p]) + (t[1 * L + p] + t[3 * L + p]);
+        }
+    free(t);
+}
+
+void oracle_ss2d_forward_table(long Bn, long Dn, long L, long N, const long *table,
+                               const double *x, const double *delta, const double *A,
+                               const double *Bm, const double *Cm, const double *Dv,
+                               const double *bias, int softplus, double *y)
+{
+    size_t seq = (size_t)(Bn * K_PATHS * Dn * L);
+    double *xs = (double *)malloc(sizeof(double) * seq);
+    double *ys = (double *)malloc(sizeof(double) * seq);
+    oracle_cross_scan_table(Bn, Dn, L, table, x, xs);
+    oracle_selective_scan_fwd(Bn, K_PATHS * Dn, L, N, K_PATHS, xs, delta, A, Bm, Cm, Dv, bias,
+                              softplus, NULL, ys, NULL);
+    oracle_cross_merge_table(Bn, Dn, L, table, ys, y);
+    free(xs);
+    free(ys);
+}
+
+void oracle_ss2d_backward_table(long Bn, long Dn, long L, long N, const long *table,
+                                const double *x, const double *delta, const double *A,
+                                const double *Bm, const double *Cm, const double *Dv,
+                                const double *bias, int softplus, const double *dy,
+                                double *dx, double *ddelta, double *dA, double *dB, double *dC,
+                                double *dD, double *dbias)
+{
+    size_t seq = (size_t)(Bn * K_PATHS * Dn * L);
+    double *xs = (double *)malloc(sizeof(double) * seq);
+    double *gs = (double *)malloc(sizeof(double) * seq);
+    double *dus = (double *)malloc(sizeof(double) * seq);
+    oracle_cross_scan_table(Bn, Dn, L, table, x, xs);
+    oracle_cross_scan_table(Bn, Dn, L, table, dy, gs);
+    oracle_selective_scan_bwd(Bn, K_PATHS * Dn, L, N, K_PATHS, xs, delta, A, Bm, Cm, Dv, bias,
+                              softplus, NULL, gs, dus, ddelta, dA, dB, dC, dD, dbias, NULL);
+    oracle_cross_merge_table(Bn, Dn, L, table, dus, dx);
+    free(xs);
+    free(gs);
+    free(dus);
+}
+
 /* number of host threads OpenMP will use (reported by the CPU baseline) */
 int oracle_num_threads(void)
 {

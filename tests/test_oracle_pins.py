@@ -11,7 +11,12 @@ routines (cumulative sum, elementwise product), linearity, permutation and
 adjoint identities of the index maps, central finite differences and exact
 dot-product identities for the backward.  The bidirectional scan
 (bimamba_inner_ref) is pinned by its mirror symmetry and by the SS2D oracle on a
-one-row image, whose row-major paths are the sequence and its reverse.  The output gate (out times silu(z),
+one-row image, whose row-major paths are the sequence and its reverse.  Path
+sets given as tables (the diagonal scans of the mooersco page, section 3) are
+pinned by hand-tabulated diagonal orders (tests/golden/diagonal_paths.txt), the
+horizontal-flip identity between the two diagonal families, equality with the
+fixed cross-scan functions for the cross table, merge-of-scan = 4x, adjointness
+and central differences.  The output gate (out times silu(z),
 the last lines of selective_scan_ref) is pinned by its special values, by
 scipy's logistic function and by central differences; the last state by
 reading it back through a one-hot C.
@@ -534,6 +539,100 @@ def test_bimamba_backward_matches_central_differences(oracle):
     names = dict(x="dx", delta="ddelta", A="dA", A_b="dA_b", B="dB", C="dC", D="dD", delta_bias="ddelta_bias",
                  z="dz")
     for name, gname in names.items():
+        flat = p[name].reshape(-1)
+        for i in rng.choice(flat.size, size=min(flat.size, 8), replace=False):
+            theta = flat[i]
+            h = 1e-6 * max(1.0, abs(theta))
+            flat[i] = theta + h
+            lp = loss()
+            flat[i] = theta - h
+            lm = loss()
+            flat[i] = theta
+            fd = (lp - lm) / (2 * h)
+            an = g[gname].reshape(-1)[i]
+            assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (name, i, fd, an)
+
+
+# ------------------------------------------------------------ path tables
+
+def _golden_diagonals():
+    rows = []
+    with open(os.path.join(GOLDEN, "diagonal_paths.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            head, seq = line.split(":")
+            H, W, direction = (int(t) for t in head.split())
+            rows.append((H, W, direction, [int(t) for t in seq.split()]))
+    return rows
+
+
+def test_diagonal_orders_match_hand_tabulated(oracle):
+    rows = _golden_diagonals()
+    assert len(rows) == 8
+    for H, W, direction, seq in rows:
+        assert oracle.diagonal_order(H, W, direction).tolist() == seq, (H, W, direction)
+
+
+@pytest.mark.parametrize("H,W", [(1, 1), (1, 6), (5, 1), (3, 7), (8, 8), (6, 4)])
+def test_diagonal_paths_are_permutations_and_mirror_images(oracle, H, W):
+    t = oracle.diagonal_paths(H, W)
+    L = H * W
+    for k in range(4):
+        assert sorted(t[k].tolist()) == list(range(L))
+    assert t[2].tolist() == t[0][::-1].tolist() and t[3].tolist() == t[1][::-1].tolist()
+    # direction -1 is direction +1 on the horizontally flipped image: pixel (i, j) <-> (i, W-1-j)
+    i, j = t[0] // W, t[0] % W
+    assert t[1].tolist() == (i * W + (W - 1 - j)).tolist()
+    if H == 1:  # one row: the diagonal order is the row order, the other family its reverse
+        assert t[0].tolist() == list(range(L)) and t[1].tolist() == list(range(L))[::-1]
+
+
+def test_cross_table_reproduces_the_fixed_paths(oracle):
+    rng = _rng(61)
+    Bn, Dn, H, W, N = 2, 3, 4, 5, 3
+    x = rng.standard_normal((Bn, Dn, H, W))
+    t = oracle.cross_paths(H, W)
+    np.testing.assert_array_equal(oracle.cross_scan_table(x, t), oracle.cross_scan(x))
+    ys = rng.standard_normal((Bn, 4, Dn, H * W))
+    np.testing.assert_array_equal(oracle.cross_merge_table(ys, H, W, t), oracle.cross_merge(ys, H, W))
+    p = _ss2d_problem(62, Bn, Dn, H, W, N)
+    args = (p["x"], p["delta"], p["A"], p["B"], p["C"], p["D"], p["delta_bias"], True)
+    np.testing.assert_array_equal(oracle.ss2d_forward_table(*args, t), oracle.ss2d_forward(*args))
+    dy = rng.standard_normal(x.shape)
+    g1 = oracle.ss2d_backward_table(*args, dy, t)
+    g2 = oracle.ss2d_backward(*args, dy)
+    for name in g1:
+        np.testing.assert_array_equal(g1[name], g2[name])
+
+
+def test_diagonal_merge_of_scan_and_adjointness(oracle):
+    rng = _rng(63)
+    Bn, Dn, H, W = 2, 3, 5, 7
+    t = oracle.diagonal_paths(H, W)
+    x = rng.standard_normal((Bn, Dn, H, W))
+    np.testing.assert_array_equal(oracle.cross_merge_table(oracle.cross_scan_table(x, t), H, W, t), 4.0 * x)
+    ys = rng.standard_normal((Bn, 4, Dn, H * W))
+    lhs = float(np.sum(oracle.cross_merge_table(ys, H, W, t) * x))
+    rhs = float(np.sum(ys * oracle.cross_scan_table(x, t)))
+    assert abs(lhs - rhs) <= 1e-12 * max(1.0, abs(lhs))
+    # the diagonal set is not the cross set: the scans differ
+    assert np.abs(oracle.cross_scan_table(x, t) - oracle.cross_scan(x)).max() > 0.1
+
+
+def test_diagonal_backward_matches_central_differences(oracle):
+    p = _ss2d_problem(64, Bn=1, Dn=2, H=3, W=4, N=3)
+    t = oracle.diagonal_paths(3, 4)
+    rng = _rng(65)
+    dy = rng.standard_normal(p["x"].shape)
+    g = oracle.ss2d_backward_table(p["x"], p["delta"], p["A"], p["B"], p["C"], p["D"], p["delta_bias"], True, dy, t)
+
+    def loss():
+        y = oracle.ss2d_forward_table(p["x"], p["delta"], p["A"], p["B"], p["C"], p["D"], p["delta_bias"], True, t)
+        return float(np.sum(y * dy))
+
+    for name, gname in (("x", "dx"), ("delta", "ddelta"), ("A", "dA"), ("B", "dB"), ("C", "dC")):
         flat = p[name].reshape(-1)
         for i in rng.choice(flat.size, size=min(flat.size, 8), replace=False):
             theta = flat[i]
