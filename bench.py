@@ -19,6 +19,9 @@ bounded sample of the same workload instead (rank 0 only).
 `--workload 5` is the bidirectional scan of bimamba_inner_ref (Vim-T tokens, gated by
 silu(z)): a step is one bidirectional forward (plus its backward under `--backward`).
 
+`--paths diagonal` runs the fused forward (and backward) over the diagonal path set of
+"Visual Mamba实战从零开始搭建图像分类模型附PyTorch代码" (section 3) instead of the cross scan.
+
 `--backward` adds the fused backward to every step; `--gate` times the scan in its
 sequence form instead, u (B, 4D, L) with the output gate out * silu(z) and the last
 state (selective_scan_fn's z and return_last_state), plus its backward with dz
@@ -359,6 +362,25 @@ def run_gpu(args, world, rank, local):
             if args.backward:
                 ss.selective_scan_bwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"],
                                       inp["delta_bias"], True, inp["dout"], chunk_states=res[2], z=inp["z"])
+    elif args.paths == "diagonal":
+        tables = ss.path_tables(w.height, w.width, ss.PATHS_DIAGONAL, device=dev)
+        nf = ss.workspace_bytes(w.batch, w.dim, w.height, w.width, w.d_state, ss.OP_FORWARD_TABLE, w.torch_dtype)
+        wst = torch.empty(max(nf, 1), dtype=torch.uint8, device=dev)
+        cs = None
+        if args.backward:
+            nb = ss.workspace_bytes(w.batch, w.dim, w.height, w.width, w.d_state, ss.OP_BACKWARD_TABLE,
+                                    w.torch_dtype)
+            wsb = torch.empty(max(nb, 1), dtype=torch.uint8, device=dev)
+            cs = torch.empty((w.batch, 4 * w.dim, -(-w.L // ss.CHUNK_LEN), w.d_state), dtype=torch.float32,
+                             device=dev)
+        targs = (inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"], inp["delta_bias"], True)
+
+        def step():
+            if args.backward:
+                _, c = ss.ss2d_forward_table(*targs, tables, out=y, return_chunk_states=True, workspace=wst)
+                ss.ss2d_backward_table(*targs, inp["dy"], tables, chunk_states=c, workspace=wsb)
+            else:
+                ss.ss2d_forward_table(*targs, tables, out=y, workspace=wst)
     elif args.backward:
         nb = ss.workspace_bytes(w.batch, w.dim, w.height, w.width, w.d_state, ss.OP_BACKWARD, w.torch_dtype)
         wsb = torch.empty(max(nb, 1), dtype=torch.uint8, device=dev)
@@ -443,10 +465,10 @@ def run_gpu(args, world, rank, local):
     sfu_peak = MUFU_EX2_PER_CLK_PER_SM * SM_COUNT * sm_max * 1e6 / 1e9  # G ex2/s at max clock
     sfu_achieved = w.updates / (dom_ms / 1e3) / 1e9  # one exp(dt*A) per state update
     # the traffic record is of the fused forward's scan kernel: other lines have no capture
-    traffic = recorded_traffic(w.name) if not (args.backward or args.gate or bidir) else None
+    traffic = recorded_traffic(w.name) if not (args.backward or args.gate or bidir or args.paths != "cross") else None
 
     e2e = None
-    if not (args.no_e2e or args.backward or args.gate or bidir):
+    if not (args.no_e2e or args.backward or args.gate or bidir or args.paths != "cross"):
         e2e = run_e2e(args, w, inp, dev, stream, world, rank)
 
     result = {
@@ -467,7 +489,8 @@ def run_gpu(args, world, rank, local):
                    "parallelism": f"batch shards x{world}, no collective",
                    "pass": ("forward + backward" if args.backward else "forward")
                    + (" (sequence form, gate z + last state)" if args.gate else "")
-                   + (" (bidirectional, gate z)" if bidir else ""),
+                   + (" (bidirectional, gate z)" if bidir else "")
+                   + (f" ({args.paths} paths)" if args.paths != "cross" else ""),
                    "l2": f"inputs {alg_bytes / 1e9:.2f} GB > 126 MB L2, no flush needed"},
         "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved_gbs / hbm_peak, "traffic": traffic,
@@ -483,7 +506,8 @@ def run_gpu(args, world, rank, local):
         "e2e": e2e,
     }
     # the oracle sample times the fused forward, so it is reported beside the forward line only
-    if rank == 0 and world == 1 and not (args.no_cpu_baseline or args.backward or args.gate or bidir):
+    if rank == 0 and world == 1 and not (args.no_cpu_baseline or args.backward or args.gate or bidir
+                                         or args.paths != "cross"):
         result["cpu_baseline"] = time_oracle(w, seconds_budget=args.cpu_seconds)
     return result
 
@@ -568,6 +592,8 @@ def main(argv=None):
                     help="time forward (keeping chunk states) + fused backward per step")
     ap.add_argument("--gate", action="store_true",
                     help="time the sequence-form scan with the output gate z and the last state instead")
+    ap.add_argument("--paths", choices=["cross", "diagonal"], default="cross",
+                    help="path set of the fused SS2D (default: the cross scan)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="time budget of the CPU oracle sample")

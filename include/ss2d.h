@@ -87,8 +87,16 @@ typedef enum {
     SS2D_OP_FORWARD = 2,
     SS2D_OP_BACKWARD = 3,
     SS2D_OP_BIMAMBA_FORWARD = 4,
-    SS2D_OP_BIMAMBA_BACKWARD = 5
+    SS2D_OP_BIMAMBA_BACKWARD = 5,
+    SS2D_OP_FORWARD_TABLE = 6,
+    SS2D_OP_BACKWARD_TABLE = 7
 } ss2d_op_t;
+
+/* Path sets that ss2d_path_tables generates (paths 2 and 3 are always 0 and 1 walked backwards). */
+typedef enum {
+    SS2D_PATHS_CROSS = 0,    /* row-major, column-major (l = w*H + h): the cross scan of ss2d_forward */
+    SS2D_PATHS_DIAGONAL = 1  /* the two diagonal orders of SS2D._get_diagonal_indices (see ss2d_path_tables) */
+} ss2d_paths_t;
 
 /* Chunk length (steps) at which the forward saves scan states for the backward. */
 #define SS2D_CHUNK_LEN 16
@@ -229,6 +237,55 @@ SS2D_API ss2d_status_t ss2d_backward(const ss2d_desc_t *desc, const void *x, con
                             const float *chunk_states, void *dx, void *ddelta, float *dA,
                             void *dBm, void *dCm, float *dD, float *ddelta_bias,
                             void *workspace, size_t workspace_bytes, ss2d_stream_t stream);
+
+/* ------------------------------------------------------------ path sets -- */
+
+/*
+ * Fill a path table for a path set, on the device.  The table is int32 (4, L), L = H*W:
+ *   rows 0, 1: fwd_k[l] = pixel p = h*W + w visited at step l of path k;
+ *   rows 2, 3: inv_k[p] = the step at which path k visits pixel p.
+ * Paths 2 and 3 are paths 0 and 1 walked backwards.  SS2D_PATHS_DIAGONAL follows
+ * SS2D._get_diagonal_indices of "Visual Mamba实战从零开始搭建图像分类模型附PyTorch代码"
+ * (section 3): anti-diagonals s = h + w in turn, h ascending within each, with w = s - h
+ * (path 0) or w = (W-1) - (s - h) (path 1).
+ * tables : device, 16-byte aligned, 4*L int32, written.  L must be below 2^31.
+ * Errors: SS2D_ERR_SHAPE for an unknown path set or L >= 2^31.
+ */
+SS2D_API ss2d_status_t ss2d_path_tables(const ss2d_desc_t *desc, int paths, int32_t *tables, ss2d_stream_t stream);
+
+/*
+ * CrossScan and CrossMerge over the path set of a table (as ss2d_path_tables writes it,
+ * or the caller's own: every entry is bounds-checked; an entry outside [0, L) reads as
+ * zero, so a table that is not made of permutations gives wrong values, never a bad access).
+ *   ss2d_cross_scan_table : xs[b, k, d, l] = x[b, d, fwd_k[l]] (k = 2, 3: fwd_{k-2}[L-1-l])
+ *   ss2d_cross_merge_table: y[b, d, p] = round_out((t0 + t2) + (t1 + t3)), t_k = path k's
+ *                           value at pixel p, summed in fp32
+ * Layouts and dtypes as ss2d_cross_scan / ss2d_cross_merge.
+ */
+SS2D_API ss2d_status_t ss2d_cross_scan_table(const ss2d_desc_t *desc, const int32_t *tables, const void *x,
+                                             void *xs, ss2d_stream_t stream);
+SS2D_API ss2d_status_t ss2d_cross_merge_table(const ss2d_desc_t *desc, const int32_t *tables, const void *ys,
+                                              void *y, ss2d_stream_t stream);
+
+/*
+ * Fused SS2D forward and backward over the path set of a table.  Arguments, layouts and
+ * results are those of ss2d_forward / ss2d_backward with path k walking the table's order
+ * (delta, B, C, chunk states in each path's own step order).  The scan reads x along
+ * paths 0 and 1 from two path-order copies that the call makes in its workspace, as the
+ * cross path set reads x and its transpose.
+ * workspace: ss2d_workspace_bytes(desc, SS2D_OP_FORWARD_TABLE / SS2D_OP_BACKWARD_TABLE) bytes.
+ */
+SS2D_API ss2d_status_t ss2d_forward_table(const ss2d_desc_t *desc, const int32_t *tables, const void *x,
+                                          const void *delta, const float *A, const void *Bm, const void *Cm,
+                                          const float *D, const float *delta_bias, int delta_softplus, void *y,
+                                          float *chunk_states, void *workspace, size_t workspace_bytes,
+                                          ss2d_stream_t stream);
+SS2D_API ss2d_status_t ss2d_backward_table(const ss2d_desc_t *desc, const int32_t *tables, const void *x,
+                                           const void *delta, const float *A, const void *Bm, const void *Cm,
+                                           const float *D, const float *delta_bias, int delta_softplus,
+                                           const void *dy, const float *chunk_states, void *dx, void *ddelta,
+                                           float *dA, void *dBm, void *dCm, float *dD, float *ddelta_bias,
+                                           void *workspace, size_t workspace_bytes, ss2d_stream_t stream);
 
 /* ------------------------------------------------- bidirectional scan -- */
 

@@ -21,6 +21,8 @@ visual data", Fig. 2; the S6 arithmetic follows selective_scan_ref on
 * ``SS2DFunction``: a torch.autograd.Function around the fused pair
 * ``bimamba_forward`` / ``bimamba_backward`` / ``bimamba_scan``: the bidirectional scan of
   bimamba_inner_ref (a sequence and its reverse with A and A_b, outputs added)
+* ``path_tables`` and the ``*_table`` calls: the same steps over another path set, e.g. the
+  diagonal scans of "Visual Mamba实战从零开始搭建图像分类模型附PyTorch代码" (section 3)
 """
 from __future__ import annotations
 
@@ -33,7 +35,8 @@ import torch
 __all__ = [
     "SS2DError", "cross_scan", "cross_merge", "selective_scan_fwd", "selective_scan_bwd", "selective_scan_fn",
     "SelectiveScanFunction", "ss2d_forward", "bimamba_forward", "bimamba_backward", "BiMambaFunction",
-    "bimamba_scan",
+    "bimamba_scan", "path_tables", "cross_scan_table", "cross_merge_table", "ss2d_forward_table",
+    "ss2d_backward_table", "PATHS_CROSS", "PATHS_DIAGONAL",
     "ss2d_backward", "SS2DFunction", "ss2d", "workspace_bytes", "chunk_states_elems", "launch_count",
     "library_path", "CHUNK_LEN", "trace_events",
 ]
@@ -47,6 +50,8 @@ _lib = None
 CHUNK_LEN = 16  # SS2D_CHUNK_LEN
 F32, BF16 = 0, 1
 OP_SELECTIVE_SCAN_BWD, OP_FORWARD, OP_BACKWARD, OP_BIMAMBA_FORWARD, OP_BIMAMBA_BACKWARD = 1, 2, 3, 4, 5
+OP_FORWARD_TABLE, OP_BACKWARD_TABLE = 6, 7
+PATHS_CROSS, PATHS_DIAGONAL = 0, 1
 _STATUS = {0: "SS2D_OK", 1: "SS2D_ERR_NULL", 2: "SS2D_ERR_SHAPE", 3: "SS2D_ERR_DTYPE", 4: "SS2D_ERR_ALIGN",
            5: "SS2D_ERR_WORKSPACE", 6: "SS2D_ERR_LAUNCH", 7: "SS2D_ERR_TIMEOUT", 8: "SS2D_ERR_DEVICE"}
 
@@ -92,12 +97,18 @@ def _load():
                                                    P, sz, P]
         lib.ss2d_forward.argtypes = [D, P, P, P, P, P, P, P, i, P, P, P, sz, P]
         lib.ss2d_bimamba_forward.argtypes = [D, P, P, P, P, P, P, P, P, i, P, P, P, sz, P]
+        lib.ss2d_path_tables.argtypes = [D, i, P, P]
+        lib.ss2d_cross_scan_table.argtypes = [D, P, P, P, P]
+        lib.ss2d_cross_merge_table.argtypes = [D, P, P, P, P]
+        lib.ss2d_forward_table.argtypes = [D, P, P, P, P, P, P, P, P, i, P, P, P, sz, P]
+        lib.ss2d_backward_table.argtypes = [D, P, P, P, P, P, P, P, P, i, P, P, P, P, P, P, P, P, P, P, sz, P]
         lib.ss2d_bimamba_backward.argtypes = [D, P, P, P, P, P, P, P, P, i, P, P, P, P, P, P, P, P, P, P, P, sz,
                                               P]
         lib.ss2d_backward.argtypes = [D, P, P, P, P, P, P, P, i, P, P, P, P, P, P, P, P, P, P, sz, P]
         for name in ("ss2d_cross_scan", "ss2d_cross_merge", "ss2d_selective_scan_fwd", "ss2d_selective_scan_bwd",
                      "ss2d_selective_scan_fwd_ex", "ss2d_selective_scan_bwd_ex", "ss2d_forward", "ss2d_backward",
-                     "ss2d_bimamba_forward", "ss2d_bimamba_backward"):
+                     "ss2d_bimamba_forward", "ss2d_bimamba_backward", "ss2d_path_tables", "ss2d_cross_scan_table",
+                     "ss2d_cross_merge_table", "ss2d_forward_table", "ss2d_backward_table"):
             getattr(lib, name).restype = ctypes.c_int
         lib.ss2d_workspace_bytes.argtypes = [D, i]
         lib.ss2d_workspace_bytes.restype = sz
@@ -384,25 +395,35 @@ def ss2d_backward(x, delta, A, B, C, D, delta_bias, delta_softplus, dy, chunk_st
 
 
 class SS2DFunction(torch.autograd.Function):
-    """autograd wrapper: forward saves the chunk states, backward runs the fused backward."""
+    """autograd wrapper: forward saves the chunk states, backward runs the fused backward.
+    ``tables`` (from path_tables) selects another path set; None is the cross scan."""
 
     @staticmethod
-    def forward(ctx, x, delta, A, B, C, D, delta_bias, delta_softplus):
-        y, cs = ss2d_forward(x, delta, A, B, C, D, delta_bias, delta_softplus, return_chunk_states=True)
-        ctx.save_for_backward(x, delta, A, B, C, D, delta_bias, cs)
+    def forward(ctx, x, delta, A, B, C, D, delta_bias, delta_softplus, tables=None):
+        if tables is None:
+            y, cs = ss2d_forward(x, delta, A, B, C, D, delta_bias, delta_softplus, return_chunk_states=True)
+        else:
+            y, cs = ss2d_forward_table(x, delta, A, B, C, D, delta_bias, delta_softplus, tables,
+                                       return_chunk_states=True)
+        ctx.save_for_backward(x, delta, A, B, C, D, delta_bias, cs, tables)
         ctx.delta_softplus = delta_softplus
         return y
 
     @staticmethod
     def backward(ctx, dy):
-        x, delta, A, B, C, D, delta_bias, cs = ctx.saved_tensors
-        g = ss2d_backward(x, delta, A, B, C, D, delta_bias, ctx.delta_softplus, dy.to(x.dtype), chunk_states=cs)
-        return g["dx"], g["ddelta"], g["dA"], g["dB"], g["dC"], g["dD"], g["ddelta_bias"], None
+        x, delta, A, B, C, D, delta_bias, cs, tables = ctx.saved_tensors
+        if tables is None:
+            g = ss2d_backward(x, delta, A, B, C, D, delta_bias, ctx.delta_softplus, dy.to(x.dtype), chunk_states=cs)
+        else:
+            g = ss2d_backward_table(x, delta, A, B, C, D, delta_bias, ctx.delta_softplus, dy.to(x.dtype), tables,
+                                    chunk_states=cs)
+        return g["dx"], g["ddelta"], g["dA"], g["dB"], g["dC"], g["dD"], g["ddelta_bias"], None, None
 
 
-def ss2d(x, delta, A, B, C, D=None, delta_bias=None, delta_softplus=True):
-    """Differentiable fused SS2D: y = CrossMerge(S6(CrossScan(x)))."""
-    return SS2DFunction.apply(x, delta, A, B, C, D, delta_bias, delta_softplus)
+def ss2d(x, delta, A, B, C, D=None, delta_bias=None, delta_softplus=True, tables=None):
+    """Differentiable fused SS2D: y = CrossMerge(S6(CrossScan(x))) over the cross scan, or over
+    the path set of ``tables`` (see path_tables)."""
+    return SS2DFunction.apply(x, delta, A, B, C, D, delta_bias, delta_softplus, tables)
 
 
 # ------------------------------------------------------------ bidirectional --
@@ -508,3 +529,109 @@ class BiMambaFunction(torch.autograd.Function):
 def bimamba_scan(x, delta, A, A_b, B, C, D=None, z=None, delta_bias=None, delta_softplus=True):
     """Differentiable bidirectional scan (the selective-scan part of bimamba_inner_ref)."""
     return BiMambaFunction.apply(x, delta, A, A_b, B, C, D, z, delta_bias, delta_softplus)
+
+
+# ---------------------------------------------------------------- path sets --
+
+def path_tables(H, W, paths=PATHS_DIAGONAL, device=None):
+    """int32 (4, H*W) device table of a path set: rows 0, 1 the pixel at each step of paths 0
+    and 1, rows 2, 3 the step at each pixel (paths 2, 3 are 0, 1 backwards).  paths is
+    PATHS_CROSS (row-major, column-major) or PATHS_DIAGONAL (the two diagonal orders)."""
+    device = device or torch.device("cuda", torch.cuda.current_device())
+    t = torch.empty((4, H * W), dtype=torch.int32, device=device)
+    d = _desc(1, 1, H, W, 1, torch.float32, torch.float32)
+    _check(_load().ss2d_path_tables(ctypes.byref(d), int(paths), _p(t), _stream(t)), "ss2d_path_tables")
+    return t
+
+
+def _tab(tables, L):
+    t = _c(tables)
+    if t.dtype != torch.int32 or t.shape != (4, L):
+        raise ValueError(f"path tables must be int32 (4, {L})")
+    return t
+
+
+def cross_scan_table(x, tables, out=None):
+    """x (B, D, H, W) -> xs (B, 4, D, H*W) along the path set of ``tables``."""
+    x = _c(x)
+    Bn, Dn, H, W = x.shape
+    t = _tab(tables, H * W)
+    if out is None:
+        out = torch.empty((Bn, 4, Dn, H * W), dtype=x.dtype, device=x.device)
+    d = _desc(Bn, Dn, H, W, 1, x.dtype, x.dtype)
+    _check(_load().ss2d_cross_scan_table(ctypes.byref(d), _p(t), _p(x), _p(out), _stream(x)), "ss2d_cross_scan_table")
+    return out
+
+
+def cross_merge_table(ys, H, W, tables, out=None, out_dtype=None):
+    """ys (B, 4, D, H*W) -> y (B, D, H, W): each path's value at each pixel, (t0 + t2) + (t1 + t3) in fp32."""
+    ys = _c(ys)
+    Bn, K, Dn, L = ys.shape
+    if K != 4 or L != H * W:
+        raise ValueError("cross_merge_table: ys must be (B, 4, D, H*W)")
+    t = _tab(tables, L)
+    out_dtype = out_dtype or ys.dtype
+    if out is None:
+        out = torch.empty((Bn, Dn, H, W), dtype=out_dtype, device=ys.device)
+    d = _desc(Bn, Dn, H, W, 1, ys.dtype, out.dtype)
+    _check(_load().ss2d_cross_merge_table(ctypes.byref(d), _p(t), _p(ys), _p(out), _stream(ys)),
+           "ss2d_cross_merge_table")
+    return out
+
+
+def ss2d_forward_table(x, delta, A, B, C, D, delta_bias, delta_softplus, tables, out=None, out_dtype=None,
+                       return_chunk_states=False, workspace=None):
+    """Fused SS2D forward over the path set of ``tables``; arguments as ss2d_forward."""
+    x = _c(x)
+    delta, B, C = (_c(t, x.dtype) for t in (delta, B, C))
+    A, D, delta_bias = _params(A, D, delta_bias)
+    Bn, Dn, H, W = x.shape
+    N = A.shape[1]
+    t = _tab(tables, H * W)
+    out_dtype = out_dtype or x.dtype
+    if out is None:
+        out = torch.empty((Bn, Dn, H, W), dtype=out_dtype, device=x.device)
+    cs = None
+    if return_chunk_states:
+        cs = torch.empty((Bn, 4 * Dn, -(-(H * W) // CHUNK_LEN), N), dtype=torch.float32, device=x.device)
+    d = _desc(Bn, Dn, H, W, N, x.dtype, out.dtype)
+    lib = _load()
+    nbytes = int(lib.ss2d_workspace_bytes(ctypes.byref(d), OP_FORWARD_TABLE))
+    if workspace is None or workspace.numel() < nbytes:
+        workspace = _workspace(nbytes, x.device)
+    st = lib.ss2d_forward_table(ctypes.byref(d), _p(t), _p(x), _p(delta), _p(A), _p(B), _p(C), _p(D), _p(delta_bias),
+                                int(bool(delta_softplus)), _p(out), _p(cs), _p(workspace), nbytes, _stream(x))
+    _check(st, "ss2d_forward_table")
+    return (out, cs) if return_chunk_states else out
+
+
+def ss2d_backward_table(x, delta, A, B, C, D, delta_bias, delta_softplus, dy, tables, chunk_states=None,
+                        workspace=None):
+    """Fused SS2D backward over the path set of ``tables``.  Returns the dict of ss2d_backward."""
+    x = _c(x)
+    delta, B, C = (_c(t, x.dtype) for t in (delta, B, C))
+    A, D, delta_bias = _params(A, D, delta_bias)
+    dy = _c(dy)
+    chunk_states = _c(chunk_states, torch.float32)
+    Bn, Dn, H, W = x.shape
+    N = A.shape[1]
+    t = _tab(tables, H * W)
+    dev = x.device
+    dx = torch.empty_like(x)
+    ddelta = torch.empty_like(delta)
+    dA = torch.empty_like(A)
+    dB = torch.empty_like(B)
+    dC = torch.empty_like(C)
+    dD = torch.empty_like(D) if D is not None else None
+    dbias = torch.empty_like(delta_bias) if delta_bias is not None else None
+    d = _desc(Bn, Dn, H, W, N, x.dtype, dy.dtype)
+    lib = _load()
+    nbytes = int(lib.ss2d_workspace_bytes(ctypes.byref(d), OP_BACKWARD_TABLE))
+    if workspace is None or workspace.numel() < nbytes:
+        workspace = _workspace(nbytes, dev)
+    st = lib.ss2d_backward_table(ctypes.byref(d), _p(t), _p(x), _p(delta), _p(A), _p(B), _p(C), _p(D),
+                                 _p(delta_bias), int(bool(delta_softplus)), _p(dy), _p(chunk_states), _p(dx),
+                                 _p(ddelta), _p(dA), _p(dB), _p(dC), _p(dD), _p(dbias), _p(workspace), nbytes,
+                                 _stream(x))
+    _check(st, "ss2d_backward_table")
+    return dict(dx=dx, ddelta=ddelta, dA=dA, dB=dB, dC=dC, dD=dD, ddelta_bias=dbias)

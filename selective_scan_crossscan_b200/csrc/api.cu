@@ -123,6 +123,21 @@ static size_t bidir_bwd_ws_bytes(const LaunchShape &s) {
     return 3 * round64((size_t)s.B * 2 * s.D * s.L * sizeof(float)) + round64(scan_bwd_workspace_bytes(s, 2));
 }
 
+// table forward workspace: [fp32 per-path outputs (B,4D,L)] [x in path-0 order] [x in path-1 order] [segments]
+static size_t table_fwd_ws_bytes(const LaunchShape &s, ss2d_dtype_t in) {
+    const size_t img = round64((size_t)s.B * s.D * s.L * elem_size(in));
+    return round64((size_t)s.B * kPaths * s.D * s.L * sizeof(float)) + 2 * img + round64(scan_fwd_workspace_bytes(s));
+}
+// table backward workspace: [fp32 per-path du] [x copies 0, 1] [dy copies 0, 1] [scan backward workspace]
+static size_t table_bwd_ws_bytes(const LaunchShape &s, ss2d_dtype_t in, ss2d_dtype_t out) {
+    return round64((size_t)s.B * kPaths * s.D * s.L * sizeof(float)) +
+           2 * round64((size_t)s.B * s.D * s.L * elem_size(in)) + 2 * round64((size_t)s.B * s.D * s.L * elem_size(out)) +
+           round64(scan_bwd_workspace_bytes(s));
+}
+static ss2d_status_t check_table_shape(const ss2d_desc_t *desc) {
+    return desc->height * desc->width < ((int64_t)1 << 31) ? SS2D_OK : SS2D_ERR_SHAPE;
+}
+
 }  // namespace ss2d
 
 using namespace ss2d;
@@ -171,6 +186,8 @@ size_t ss2d_workspace_bytes(const ss2d_desc_t *desc, int op) {
         case SS2D_OP_BACKWARD: return bwd_fused_ws_bytes(s, desc->in_dtype, desc->out_dtype);
         case SS2D_OP_BIMAMBA_FORWARD: return bidir_fwd_ws_bytes(s);
         case SS2D_OP_BIMAMBA_BACKWARD: return bidir_bwd_ws_bytes(s);
+        case SS2D_OP_FORWARD_TABLE: return table_fwd_ws_bytes(s, desc->in_dtype);
+        case SS2D_OP_BACKWARD_TABLE: return table_bwd_ws_bytes(s, desc->in_dtype, desc->out_dtype);
         default: return (size_t)-1;
     }
 }
@@ -305,6 +322,146 @@ ss2d_status_t ss2d_selective_scan_bwd(const ss2d_desc_t *desc, const void *u, co
     return ss2d_selective_scan_bwd_ex(desc, u, delta, A, Bm, Cm, D, nullptr, delta_bias, delta_softplus, dout,
                                       chunk_states, du, ddelta, dA, dBm, dCm, dD, ddelta_bias, nullptr, workspace,
                                       workspace_bytes, stream);
+}
+
+ss2d_status_t ss2d_path_tables(const ss2d_desc_t *desc, int paths, int32_t *tables, ss2d_stream_t stream) {
+    SS2D_TRY(check_desc(desc));
+    SS2D_TRY(check_table_shape(desc));
+    if (paths != SS2D_PATHS_CROSS && paths != SS2D_PATHS_DIAGONAL) return SS2D_ERR_SHAPE;
+    SS2D_TRY(need(tables));
+    SS2D_TRY(check_device());
+    return from_cuda(launch_path_tables(paths, desc->height, desc->width, tables, (cudaStream_t)stream));
+}
+
+ss2d_status_t ss2d_cross_scan_table(const ss2d_desc_t *desc, const int32_t *tables, const void *x, void *xs,
+                                    ss2d_stream_t stream) {
+    SS2D_TRY(check_desc(desc));
+    SS2D_TRY(check_table_shape(desc));
+    SS2D_TRY(need(tables));
+    SS2D_TRY(need(x));
+    SS2D_TRY(need(xs));
+    SS2D_TRY(check_device());
+    return from_cuda(launch_cross_scan_table(shape_of(desc), desc->in_dtype, x, tables, xs, (cudaStream_t)stream));
+}
+
+ss2d_status_t ss2d_cross_merge_table(const ss2d_desc_t *desc, const int32_t *tables, const void *ys, void *y,
+                                     ss2d_stream_t stream) {
+    SS2D_TRY(check_desc(desc));
+    SS2D_TRY(check_table_shape(desc));
+    SS2D_TRY(need(tables));
+    SS2D_TRY(need(ys));
+    SS2D_TRY(need(y));
+    SS2D_TRY(check_device());
+    return from_cuda(launch_cross_merge_table(shape_of(desc), desc->in_dtype, desc->out_dtype, ys, tables, y,
+                                              (cudaStream_t)stream));
+}
+
+ss2d_status_t ss2d_forward_table(const ss2d_desc_t *desc, const int32_t *tables, const void *x, const void *delta,
+                                 const float *A, const void *Bm, const void *Cm, const float *D,
+                                 const float *delta_bias, int delta_softplus, void *y, float *chunk_states,
+                                 void *workspace, size_t workspace_bytes, ss2d_stream_t stream) {
+    SS2D_TRY(check_desc(desc));
+    SS2D_TRY(check_table_shape(desc));
+    SS2D_TRY(need(tables));
+    SS2D_TRY(check_scan_inputs(x, delta, A, Bm, Cm, D, delta_bias));
+    SS2D_TRY(need(y));
+    SS2D_TRY(optional(chunk_states));
+    const LaunchShape s = shape_of(desc);
+    if (!workspace || workspace_bytes < table_fwd_ws_bytes(s, desc->in_dtype)) return SS2D_ERR_WORKSPACE;
+    SS2D_TRY(optional(workspace));
+    SS2D_TRY(check_device());
+    const size_t img = round64((size_t)s.B * s.D * s.L * elem_size(desc->in_dtype));
+    unsigned char *w = static_cast<unsigned char *>(workspace);
+    float *ys = reinterpret_cast<float *>(w);
+    w += round64((size_t)s.B * kPaths * s.D * s.L * sizeof(float));
+    void *c0 = w;
+    void *c1 = w + img;
+    void *seg = w + 2 * img;
+    cudaStream_t st = (cudaStream_t)stream;
+    SS2D_TRY(from_cuda(launch_path_copies(s, desc->in_dtype, x, tables, c0, c1, st)));
+    ScanFwdArgs a;
+    a.u = c0;   // path 0 (and 2, backwards)
+    a.uT = c1;  // path 1 (and 3, backwards)
+    a.delta = delta;
+    a.A = A;
+    a.Bm = Bm;
+    a.Cm = Cm;
+    a.Dv = D;
+    a.bias = delta_bias;
+    a.softplus = delta_softplus != 0;
+    a.out = ys;
+    a.chunk_states = chunk_states;
+    a.from_image = true;
+    a.in_dtype = desc->in_dtype;
+    a.out_dtype = SS2D_F32;
+    SS2D_TRY(from_cuda(launch_scan_fwd(s, a, seg, st)));
+    return from_cuda(launch_cross_merge_table(s, SS2D_F32, desc->out_dtype, ys, tables, y, st));
+}
+
+ss2d_status_t ss2d_backward_table(const ss2d_desc_t *desc, const int32_t *tables, const void *x, const void *delta,
+                                  const float *A, const void *Bm, const void *Cm, const float *D,
+                                  const float *delta_bias, int delta_softplus, const void *dy,
+                                  const float *chunk_states, void *dx, void *ddelta, float *dA, void *dBm, void *dCm,
+                                  float *dD, float *ddelta_bias, void *workspace, size_t workspace_bytes,
+                                  ss2d_stream_t stream) {
+    SS2D_TRY(check_desc(desc));
+    SS2D_TRY(check_table_shape(desc));
+    SS2D_TRY(need(tables));
+    SS2D_TRY(check_scan_inputs(x, delta, A, Bm, Cm, D, delta_bias));
+    SS2D_TRY(need(dy));
+    SS2D_TRY(optional(chunk_states));
+    SS2D_TRY(need(dx));
+    SS2D_TRY(need(ddelta));
+    SS2D_TRY(need(dA));
+    SS2D_TRY(need(dBm));
+    SS2D_TRY(need(dCm));
+    if ((D == nullptr) != (dD == nullptr)) return SS2D_ERR_NULL;
+    if ((delta_bias == nullptr) != (ddelta_bias == nullptr)) return SS2D_ERR_NULL;
+    SS2D_TRY(optional(dD));
+    SS2D_TRY(optional(ddelta_bias));
+    const LaunchShape s = shape_of(desc);
+    if (!workspace || workspace_bytes < table_bwd_ws_bytes(s, desc->in_dtype, desc->out_dtype))
+        return SS2D_ERR_WORKSPACE;
+    SS2D_TRY(optional(workspace));
+    SS2D_TRY(check_device());
+    const size_t ximg = round64((size_t)s.B * s.D * s.L * elem_size(desc->in_dtype));
+    const size_t gimg = round64((size_t)s.B * s.D * s.L * elem_size(desc->out_dtype));
+    unsigned char *w = static_cast<unsigned char *>(workspace);
+    float *du_seq = reinterpret_cast<float *>(w);
+    w += round64((size_t)s.B * kPaths * s.D * s.L * sizeof(float));
+    void *x0 = w, *x1 = w + ximg;
+    w += 2 * ximg;
+    void *g0 = w, *g1 = w + gimg;
+    w += 2 * gimg;
+    void *inner = w;
+    cudaStream_t st = (cudaStream_t)stream;
+    SS2D_TRY(from_cuda(launch_path_copies(s, desc->in_dtype, x, tables, x0, x1, st)));
+    SS2D_TRY(from_cuda(launch_path_copies(s, desc->out_dtype, dy, tables, g0, g1, st)));
+    ScanBwdArgs a;
+    a.u = x0;
+    a.uT = x1;
+    a.dout = g0;
+    a.doutT = g1;
+    a.delta = delta;
+    a.A = A;
+    a.Bm = Bm;
+    a.Cm = Cm;
+    a.Dv = D;
+    a.bias = delta_bias;
+    a.softplus = delta_softplus != 0;
+    a.chunk_states = chunk_states;
+    a.du = du_seq;
+    a.ddelta = ddelta;
+    a.dA = dA;
+    a.dBm = dBm;
+    a.dCm = dCm;
+    a.dD = dD;
+    a.dbias = ddelta_bias;
+    a.from_image = true;
+    a.in_dtype = desc->in_dtype;
+    a.out_dtype = desc->out_dtype;
+    SS2D_TRY(from_cuda(launch_scan_bwd(s, a, inner, scan_bwd_workspace_bytes(s), st)));
+    return from_cuda(launch_cross_merge_table(s, SS2D_F32, desc->in_dtype, du_seq, tables, dx, st));
 }
 
 ss2d_status_t ss2d_bimamba_forward(const ss2d_desc_t *desc, const void *x, const void *delta, const float *A,

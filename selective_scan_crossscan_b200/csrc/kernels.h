@@ -61,6 +61,16 @@ cudaError_t launch_scan_fwd(const LaunchShape &s, const ScanFwdArgs &a, void *wo
 
 // --------------------------------------------------------------- backward --
 
+// Path sets as tables (int32 (4, L): fwd0, fwd1, inv0, inv1; paths 2/3 are 0/1 backwards).
+cudaError_t launch_path_tables(int kind, int64_t H, int64_t W, int32_t *tab, cudaStream_t stream);
+// c0[b, d, l] = x[b, d, fwd0[l]], c1[b, d, l] = x[b, d, fwd1[l]]
+cudaError_t launch_path_copies(const LaunchShape &s, ss2d_dtype_t dt, const void *x, const int32_t *tab, void *c0,
+                               void *c1, cudaStream_t stream);
+cudaError_t launch_cross_scan_table(const LaunchShape &s, ss2d_dtype_t dt, const void *x, const int32_t *tab,
+                                    void *xs, cudaStream_t stream);
+cudaError_t launch_cross_merge_table(const LaunchShape &s, ss2d_dtype_t din, ss2d_dtype_t dout, const void *ys,
+                                     const int32_t *tab, void *y, cudaStream_t stream);
+
 // Bidirectional scan: out[b, d, m] = (two[b, 0, d, m] + two[b, 1, d, m]) * (z ? silu(z[b, d, m]) : 1),
 // two (B, 2, D, L) fp32, z (B, D, L) z_dtype or null, out (B, D, L) out_dtype.
 cudaError_t launch_bidir_sum(const float *two, const void *z, ss2d_dtype_t z_dtype, void *out,

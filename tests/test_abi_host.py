@@ -136,6 +136,22 @@ def test_bimamba_argument_errors(lib):
              None) == ERR_WORKSPACE
 
 
+def test_path_table_argument_errors(lib):
+    mis = ctypes.c_void_p(0x10004)
+    assert lib.ss2d_path_tables(_d(), 2, A16, None) == ERR_SHAPE  # unknown path set
+    assert lib.ss2d_path_tables(_d(), 1, None, None) == ERR_NULL
+    assert lib.ss2d_path_tables(_d(), 1, mis, None) == ERR_ALIGN
+    assert lib.ss2d_cross_scan_table(_d(), None, A16, B16, None) == ERR_NULL
+    assert lib.ss2d_cross_merge_table(_d(), mis, A16, B16, None) == ERR_ALIGN
+    f = lib.ss2d_forward_table
+    wsf = lib.ss2d_workspace_bytes(_d(), ss.OP_FORWARD_TABLE)
+    wsb = lib.ss2d_workspace_bytes(_d(), ss.OP_BACKWARD_TABLE)
+    assert wsf > lib.ss2d_workspace_bytes(_d(), ss.OP_FORWARD) and wsb > lib.ss2d_workspace_bytes(_d(), ss.OP_BACKWARD)
+    args = [A16] * 5
+    assert f(_d(), A16, *args, None, None, 1, B16, None, A16, wsf - 1, None) == ERR_WORKSPACE
+    assert f(_d(), None, *args, None, None, 1, B16, None, A16, wsf, None) == ERR_NULL
+
+
 def test_valid_call_without_gpu_reports_device_error(lib):
     import torch
     if torch.cuda.is_available():

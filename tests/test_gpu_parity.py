@@ -416,6 +416,143 @@ def test_bimamba_full_vim_workload_sampled():
             assert_rel_l2(g[name][bi:bi + 1], r[name], GRAD_TOL, f"{name}[{bi}]")
 
 
+# ---------------------------------------------------- path sets as tables
+
+# ragged planes, one-row and one-column maps, a 14x14 plane, and a plane too large for the
+# shared-memory merge (100 x 100)
+TABLE_SHAPES = [(1, 2, 3, 4), (2, 3, 5, 7), (1, 2, 1, 9), (1, 3, 8, 1), (2, 4, 14, 14), (1, 2, 100, 100)]
+
+
+@pytest.mark.parametrize("H,W", [(3, 4), (1, 7), (6, 1), (14, 14), (13, 37), (56, 56)])
+@pytest.mark.parametrize("kind", ["cross", "diagonal"])
+def test_path_tables_match_oracle(H, W, kind):
+    t = ss.path_tables(H, W, ss.PATHS_DIAGONAL if kind == "diagonal" else ss.PATHS_CROSS)
+    ref = oracle.diagonal_paths(H, W) if kind == "diagonal" else oracle.cross_paths(H, W)
+    got = _np(t).astype(np.int64)
+    np.testing.assert_array_equal(got[0], ref[0])
+    np.testing.assert_array_equal(got[1], ref[1])
+    L = H * W
+    for k in range(2):  # rows 2, 3: inverse permutations
+        np.testing.assert_array_equal(got[2 + k][ref[k]], np.arange(L))
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("shape", TABLE_SHAPES)
+def test_cross_scan_table_bit_exact(shape, dtype):
+    Bn, Dn, H, W = shape
+    g = torch.Generator().manual_seed(11)
+    x = torch.randn(shape, generator=g).to(dtype)
+    t = ss.path_tables(H, W, ss.PATHS_DIAGONAL)
+    xs = ss.cross_scan_table(x.cuda(), t)
+    np.testing.assert_array_equal(_np(xs), oracle.cross_scan_table(x, oracle.diagonal_paths(H, W)))
+
+
+@pytest.mark.parametrize("shape", TABLE_SHAPES)
+def test_cross_merge_table_bit_exact(shape):
+    Bn, Dn, H, W = shape
+    g = torch.Generator().manual_seed(12)
+    ys = torch.randint(-1000, 1000, (Bn, 4, Dn, H * W), generator=g).float()
+    t = ss.path_tables(H, W, ss.PATHS_DIAGONAL)
+    y = ss.cross_merge_table(ys.cuda(), H, W, t)
+    np.testing.assert_array_equal(_np(y), oracle.cross_merge_table(ys, H, W, oracle.diagonal_paths(H, W)))
+    x = torch.randn((Bn, Dn, H, W), generator=g).cuda()
+    assert torch.equal(ss.cross_merge_table(ss.cross_scan_table(x, t), H, W, t), 4 * x)
+
+
+def test_cross_table_equals_the_fixed_cross_path():
+    # the table machinery over the cross set gives the fixed path's results bit for bit
+    Bn, Dn, H, W, N = 2, 6, 9, 11, 16
+    w = ss2d_inputs.custom(Bn, Dn, H, W, N)
+    inp = ss2d_inputs.make_inputs(w, seed=13, with_dy=True)
+    d = _dev(inp)
+    t = ss.path_tables(H, W, ss.PATHS_CROSS)
+    args = (d["x"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["delta_bias"], True)
+    assert torch.equal(ss.cross_scan_table(d["x"], t), ss.cross_scan(d["x"]))
+    assert torch.equal(ss.ss2d_forward_table(*args, t), ss.ss2d_forward(*args))
+    g1 = ss.ss2d_backward_table(*args, d["dy"], t)
+    g2 = ss.ss2d_backward(*args, d["dy"])
+    for name in g1:
+        assert torch.equal(g1[name], g2[name]), name
+
+
+DIAG_CASES = [(1, 8, 8, 8, 4), (2, 6, 5, 9, 16), (1, 70, 12, 11, 16), (2, 3, 1, 1, 2), (1, 4, 3, 100, 8),
+              (1, 2, 100, 100, 16)]
+
+
+@pytest.mark.parametrize("case", DIAG_CASES)
+def test_ss2d_forward_diagonal_parity(case):
+    Bn, Dn, H, W, N = case
+    w = ss2d_inputs.custom(Bn, Dn, H, W, N)
+    inp = ss2d_inputs.make_inputs(w, seed=14)
+    d = _dev(inp)
+    t = ss.path_tables(H, W, ss.PATHS_DIAGONAL)
+    y = ss.ss2d_forward_table(d["x"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["delta_bias"], True, t)
+    ref = oracle.ss2d_forward_table(inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"],
+                                    inp["delta_bias"], True, oracle.diagonal_paths(H, W))
+    assert_fwd_close(y, ref, f"{case} y")
+
+
+@pytest.mark.parametrize("case", DIAG_CASES[:5])
+@pytest.mark.parametrize("with_states", [False, True])
+def test_ss2d_backward_diagonal_parity(case, with_states):
+    Bn, Dn, H, W, N = case
+    w = ss2d_inputs.custom(Bn, Dn, H, W, N)
+    inp = ss2d_inputs.make_inputs(w, seed=15, with_dy=True)
+    d = _dev(inp)
+    t = ss.path_tables(H, W, ss.PATHS_DIAGONAL)
+    args = (d["x"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["delta_bias"], True)
+    cs = None
+    if with_states:
+        _, cs = ss.ss2d_forward_table(*args, t, return_chunk_states=True)
+    g = ss.ss2d_backward_table(*args, d["dy"], t, chunk_states=cs)
+    ref = oracle.ss2d_backward_table(inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"],
+                                     inp["delta_bias"], True, inp["dy"], oracle.diagonal_paths(H, W))
+    for name, rname in SS2D_BWD_NAMES:
+        assert_rel_l2(g[name], ref[rname], GRAD_TOL, f"{case} {name}")
+
+
+def test_ss2d_diagonal_bf16_and_autograd():
+    w = ss2d_inputs.custom(1, 8, 12, 12, 16, dtype="bf16", a_init="s4d_real")
+    inp = ss2d_inputs.make_inputs(w, seed=16, with_dy=True)
+    d = _dev(inp)
+    t = ss.path_tables(12, 12, ss.PATHS_DIAGONAL)
+    tab = oracle.diagonal_paths(12, 12)
+    y = ss.ss2d_forward_table(d["x"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["delta_bias"], True, t)
+    ref = oracle.ss2d_forward_table(inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"],
+                                    inp["delta_bias"], True, tab)
+    assert_rel_l2(y, ref, BF16_TOL, "y bf16")
+    # autograd through ss2d(..., tables=) in fp32
+    w = ss2d_inputs.custom(1, 4, 6, 7, 8)
+    inp = ss2d_inputs.make_inputs(w, seed=17, with_dy=True)
+    d = _dev(inp)
+    t = ss.path_tables(6, 7, ss.PATHS_DIAGONAL)
+    names = ("x", "delta", "A", "B", "C", "D", "delta_bias")
+    leaves = {k: d[k].clone().requires_grad_(True) for k in names}
+    y = ss.ss2d(leaves["x"], leaves["delta"], leaves["A"], leaves["B"], leaves["C"], leaves["D"],
+                leaves["delta_bias"], True, tables=t)
+    y.backward(d["dy"])
+    ref = oracle.ss2d_backward_table(inp["x"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"],
+                                     inp["delta_bias"], True, inp["dy"], oracle.diagonal_paths(6, 7))
+    gmap = dict(x="dx", delta="ddelta", A="dA", B="dB", C="dC", D="dD", delta_bias="ddelta_bias")
+    for k, rname in gmap.items():
+        assert_rel_l2(leaves[k].grad, ref[rname], GRAD_TOL, k)
+
+
+def test_ss2d_diagonal_full_stage1_sampled():
+    # VMamba-T stage-1 shapes over the diagonal path set, batch items checked one by one
+    w = ss2d_inputs.workload("vmamba_t_stage1_fp32")
+    inp = ss2d_inputs.make_inputs(w, seed=18)
+    d = _dev(inp)
+    t = ss.path_tables(w.height, w.width, ss.PATHS_DIAGONAL)
+    y = ss.ss2d_forward_table(d["x"], d["delta"], d["A"], d["B"], d["C"], d["D"], d["delta_bias"], True, t)
+    tab = oracle.diagonal_paths(w.height, w.width)
+    for bi in (0, 63, w.batch - 1):
+        sl = ss2d_inputs.batch_slice(inp, [bi])
+        ref = oracle.ss2d_forward_table(sl["x"], sl["delta"], sl["A"], sl["B"], sl["C"], sl["D"], sl["delta_bias"],
+                                        True, tab)
+        assert_fwd_close(y[bi:bi + 1], ref, f"y[{bi}]")
+
+
 # ------------------------------------------------------------- fused SS2D
 
 FUSED_CASES = [(1, 8, 8, 8, 4), (2, 6, 5, 9, 16), (1, 70, 12, 11, 16), (1, 8, 64, 64, 16), (2, 3, 1, 1, 2),
