@@ -162,6 +162,36 @@ def selective_scan_bwd(u, delta, A, B, C, D, delta_bias, delta_softplus, dout, z
     return dict(du=du, ddelta=ddelta, dA=dA, dB=dB, dC=dC, dD=dD, ddelta_bias=dbias, dz=dz)
 
 
+# ------------------------------------------------------- producer projections
+
+def path_projections(x, x_proj_weight, dt_proj_weight):
+    """The producer of the scan's inputs, per path, as in MambaInnerFn.forward ("vision
+    mamba-yolov8", section 2): x_dbl = x_proj(u) with R + 2N outputs per token,
+    delta = dt_proj.weight @ x_dbl[:R], B = x_dbl[R:R+N], C = x_dbl[R+N:].  SS2D gives every
+    path k its own projections; u is x read along path k (CrossScan).
+
+    x (Bn, D, H, W); x_proj_weight (4, R+2N, D); dt_proj_weight (4, D, R).
+    Returns delta (Bn, 4D, L), B, C (Bn, 4, N, L), x_dbl (Bn, 4, R+2N, L)."""
+    x, Wx, Wdt = _f64(x), _f64(x_proj_weight), _f64(dt_proj_weight)
+    Bn, Dn, H, W = x.shape
+    K, RN, _ = Wx.shape
+    R = Wdt.shape[2]
+    N = (RN - R) // 2
+    xs = cross_scan(x)                                         # (Bn, 4, D, L)
+    x_dbl = np.einsum("bkdl,kcd->bkcl", xs, Wx)                # (Bn, 4, R+2N, L)
+    delta = np.einsum("kdr,bkrl->bkdl", Wdt, x_dbl[:, :, :R])  # (Bn, 4, D, L)
+    Bm = np.ascontiguousarray(x_dbl[:, :, R:R + N])
+    Cm = np.ascontiguousarray(x_dbl[:, :, R + N:])
+    return delta.reshape(Bn, K * Dn, H * W), Bm, Cm, x_dbl
+
+
+def ss2d_forward_proj(x, x_proj_weight, dt_proj_weight, dt_proj_bias, A, D=None, delta_softplus=True):
+    """SS2D forward with its producer: path_projections, then the SS2D forward on those inputs
+    with dt_proj's bias as delta_bias."""
+    delta, Bm, Cm, _ = path_projections(x, x_proj_weight, dt_proj_weight)
+    return ss2d_forward(x, delta, A, Bm, Cm, D, dt_proj_bias, delta_softplus)
+
+
 # ---------------------------------------------------------------- path sets
 
 def cross_paths(H: int, W: int):

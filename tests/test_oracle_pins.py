@@ -16,7 +16,9 @@ sets given as tables (the diagonal scans of the mooersco page, section 3) are
 pinned by hand-tabulated diagonal orders (tests/golden/diagonal_paths.txt), the
 horizontal-flip identity between the two diagonal families, equality with the
 fixed cross-scan functions for the cross table, merge-of-scan = 4x, adjointness
-and central differences.  The output gate (out times silu(z),
+and central differences.  The producer projections (MambaInnerFn.forward) are
+pinned by per-token loops, by the B/C scale invariance of the output, and by
+the special cases dt_proj = 0 and x_proj's C rows = 0.  The output gate (out times silu(z),
 the last lines of selective_scan_ref) is pinned by its special values, by
 scipy's logistic function and by central differences; the last state by
 reading it back through a one-hot C.
@@ -645,6 +647,69 @@ def test_diagonal_backward_matches_central_differences(oracle):
             fd = (lp - lm) / (2 * h)
             an = g[gname].reshape(-1)[i]
             assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (name, i, fd, an)
+
+
+# ------------------------------------------------------ producer projections
+
+def _proj_problem(seed, Bn=2, Dn=3, H=3, W=4, N=3, R=2):
+    rng = _rng(seed)
+    return dict(x=rng.standard_normal((Bn, Dn, H, W)), Wx=rng.standard_normal((4, R + 2 * N, Dn)) / np.sqrt(Dn),
+                Wdt=rng.uniform(-1, 1, (4, Dn, R)) / np.sqrt(R), bias=rng.uniform(-4.0, -2.0, 4 * Dn),
+                A=-rng.uniform(0.3, 2.5, (4 * Dn, N)), D=rng.standard_normal(4 * Dn))
+
+
+def test_projections_match_per_token_loops(oracle):
+    p = _proj_problem(71)
+    x, Wx, Wdt = p["x"], p["Wx"], p["Wdt"]
+    Bn, Dn, H, W = x.shape
+    R, N = Wdt.shape[2], (Wx.shape[1] - Wdt.shape[2]) // 2
+    delta, Bm, Cm, _ = oracle.path_projections(x, Wx, Wdt)
+    for b in range(Bn):
+        for k in range(4):
+            for l in range(H * W):
+                pix = oracle.path_pixel(k, l, H, W)
+                u = [x[b, d, pix // W, pix % W] for d in range(Dn)]
+                row = [sum(Wx[k, c, d] * u[d] for d in range(Dn)) for c in range(R + 2 * N)]
+                for d in range(Dn):
+                    want = sum(Wdt[k, d, r] * row[r] for r in range(R))
+                    assert abs(delta[b, k * Dn + d, l] - want) <= 1e-12
+                for n in range(N):
+                    assert abs(Bm[b, k, n, l] - row[R + n]) <= 1e-12
+                    assert abs(Cm[b, k, n, l] - row[R + N + n]) <= 1e-12
+
+
+def test_projection_output_invariant_to_b_c_scaling(oracle):
+    # h is linear in B and y = C.h: scaling x_proj's B rows by s and its C rows by 1/s leaves y unchanged
+    p = _proj_problem(72)
+    R, N = p["Wdt"].shape[2], (p["Wx"].shape[1] - p["Wdt"].shape[2]) // 2
+    y = oracle.ss2d_forward_proj(p["x"], p["Wx"], p["Wdt"], p["bias"], p["A"], p["D"])
+    Wx2 = p["Wx"].copy()
+    Wx2[:, R:R + N] *= 4.0
+    Wx2[:, R + N:] /= 4.0
+    y2 = oracle.ss2d_forward_proj(p["x"], Wx2, p["Wdt"], p["bias"], p["A"], p["D"])
+    np.testing.assert_allclose(y2, y, rtol=1e-12, atol=1e-12)
+    Wx3 = p["Wx"].copy()
+    Wx3[:, R:R + N] *= 4.0  # B alone scaled: the state path scales, the skip term does not
+    y3 = oracle.ss2d_forward_proj(p["x"], Wx3, p["Wdt"], p["bias"], p["A"], None)
+    y0 = oracle.ss2d_forward_proj(p["x"], p["Wx"], p["Wdt"], p["bias"], p["A"], None)
+    np.testing.assert_allclose(y3, 4.0 * y0, rtol=1e-12, atol=1e-12)
+
+
+def test_projection_special_cases(oracle):
+    p = _proj_problem(73)
+    R, N = p["Wdt"].shape[2], (p["Wx"].shape[1] - p["Wdt"].shape[2]) // 2
+    Bn, Dn, H, W = p["x"].shape
+    # dt_proj = 0: delta = 0 and dt = softplus(bias)
+    y = oracle.ss2d_forward_proj(p["x"], p["Wx"], np.zeros_like(p["Wdt"]), p["bias"], p["A"], p["D"])
+    _, Bm, Cm, _ = oracle.path_projections(p["x"], p["Wx"], p["Wdt"])
+    ref = oracle.ss2d_forward(p["x"], np.zeros((Bn, 4 * Dn, H * W)), p["A"], Bm, Cm, p["D"], p["bias"], True)
+    np.testing.assert_allclose(y, ref, rtol=1e-13, atol=1e-13)
+    # C rows = 0: only the skip term remains, 4 D u summed over the paths
+    Wx = p["Wx"].copy()
+    Wx[:, R + N:] = 0.0
+    y = oracle.ss2d_forward_proj(p["x"], Wx, p["Wdt"], p["bias"], p["A"], p["D"])
+    Dk = p["D"].reshape(4, Dn)
+    np.testing.assert_allclose(y, Dk.sum(0)[None, :, None, None] * p["x"], rtol=1e-13, atol=1e-13)
 
 
 # --------------------------------------------------------- input generator
