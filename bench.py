@@ -22,6 +22,9 @@ silu(z)): a step is one bidirectional forward (plus its backward under `--backwa
 `--paths diagonal` runs the fused forward (and backward) over the diagonal path set of
 "Visual Mamba实战从零开始搭建图像分类模型附PyTorch代码" (section 3) instead of the cross scan.
 
+`--proj` times the fused forward with its producer: per-path x_proj, then the scan computing
+dt = softplus(dt_proj . x_dbl[:R] + bias) per step (MambaInnerFn.forward's projections).
+
 `--backward` adds the fused backward to every step; `--gate` times the scan in its
 sequence form instead, u (B, 4D, L) with the output gate out * silu(z) and the last
 state (selective_scan_fn's z and return_last_state), plus its backward with dz
@@ -92,6 +95,15 @@ def bidir_algorithmic_bytes(w, backward: bool) -> int:
     if backward:
         return s * (4 * seq + bc) + s * (3 * seq + bc) + 2 * params
     return s * (3 * seq + bc) + s * seq + params
+
+
+def proj_algorithmic_bytes(w, R: int) -> int:
+    """The fused forward with its producer: read x and the small weights once, write y and the
+    saved projections x_dbl (B, 4, R+2N, L); delta, B and C never go through HBM as inputs."""
+    s = 4 if w.dtype == "f32" else 2
+    Bn, Dn, L, N = w.batch, w.dim, w.L, w.d_state
+    weights = 4 * (4 * (R + 2 * N) * Dn + 4 * Dn * R + 4 * Dn * (N + 2))
+    return s * Bn * Dn * L + s * Bn * Dn * L + s * Bn * 4 * (R + 2 * N) * L + weights
 
 
 def bwd_algorithmic_bytes(w, gate: bool = False) -> int:
@@ -323,7 +335,9 @@ def run_gpu(args, world, rank, local):
         w = w.with_batch(args.batch)
     dev = torch.device("cuda", local)
     bidir = w.kind == "bidir"
-    if bidir:
+    if args.proj:
+        inp = ss2d_inputs.make_proj_inputs(w, seed=shard_seed(args.workload, rank), device=dev)
+    elif bidir:
         inp = ss2d_inputs.make_bimamba_inputs(w, seed=shard_seed(args.workload, rank), device=dev,
                                               with_dy=args.backward, with_z=True)
     elif args.gate:
@@ -336,7 +350,14 @@ def run_gpu(args, world, rank, local):
     ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    if bidir:
+    if args.proj:
+        R = inp["R"]
+        x_dbl = torch.empty((w.batch, 4, R + 2 * w.d_state, w.L), dtype=w.torch_dtype, device=dev)
+        pargs = (inp["x"], inp["x_proj_weight"], inp["dt_proj_weight"], inp["dt_proj_bias"], inp["A"], inp["D"])
+
+        def step():
+            ss.ss2d_forward_proj(*pargs, True, out=y, workspace=ws)
+    elif bidir:
         y_seq = torch.empty((w.batch, w.dim, w.L), dtype=w.torch_dtype, device=dev)
         nbf = ss.workspace_bytes(w.batch, w.dim, 1, w.L, w.d_state, ss.OP_BIMAMBA_FORWARD, w.torch_dtype)
         wsf = torch.empty(max(nbf, 1), dtype=torch.uint8, device=dev)
@@ -450,7 +471,9 @@ def run_gpu(args, world, rank, local):
     peaks = load_peaks()
     clocks = sampler.summary() if sampler else None
     # algorithmic bytes of the dominant kernel: the backward's when a backward runs in the step
-    if bidir:
+    if args.proj:
+        alg_bytes = proj_algorithmic_bytes(w, inp["R"])
+    elif bidir:
         alg_bytes = bidir_algorithmic_bytes(w, args.backward)
     elif args.backward:
         alg_bytes = bwd_algorithmic_bytes(w, gate=args.gate)
@@ -465,10 +488,11 @@ def run_gpu(args, world, rank, local):
     sfu_peak = MUFU_EX2_PER_CLK_PER_SM * SM_COUNT * sm_max * 1e6 / 1e9  # G ex2/s at max clock
     sfu_achieved = w.updates / (dom_ms / 1e3) / 1e9  # one exp(dt*A) per state update
     # the traffic record is of the fused forward's scan kernel: other lines have no capture
-    traffic = recorded_traffic(w.name) if not (args.backward or args.gate or bidir or args.paths != "cross") else None
+    traffic = (recorded_traffic(w.name)
+               if not (args.backward or args.gate or bidir or args.paths != "cross" or args.proj) else None)
 
     e2e = None
-    if not (args.no_e2e or args.backward or args.gate or bidir or args.paths != "cross"):
+    if not (args.no_e2e or args.backward or args.gate or bidir or args.paths != "cross" or args.proj):
         e2e = run_e2e(args, w, inp, dev, stream, world, rank)
 
     result = {
@@ -490,7 +514,8 @@ def run_gpu(args, world, rank, local):
                    "pass": ("forward + backward" if args.backward else "forward")
                    + (" (sequence form, gate z + last state)" if args.gate else "")
                    + (" (bidirectional, gate z)" if bidir else "")
-                   + (f" ({args.paths} paths)" if args.paths != "cross" else ""),
+                   + (f" ({args.paths} paths)" if args.paths != "cross" else "")
+                   + (" (with the per-path x_proj/dt_proj producer)" if args.proj else ""),
                    "l2": f"inputs {alg_bytes / 1e9:.2f} GB > 126 MB L2, no flush needed"},
         "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved_gbs / hbm_peak, "traffic": traffic,
@@ -507,7 +532,7 @@ def run_gpu(args, world, rank, local):
     }
     # the oracle sample times the fused forward, so it is reported beside the forward line only
     if rank == 0 and world == 1 and not (args.no_cpu_baseline or args.backward or args.gate or bidir
-                                         or args.paths != "cross"):
+                                         or args.paths != "cross" or args.proj):
         result["cpu_baseline"] = time_oracle(w, seconds_budget=args.cpu_seconds)
     return result
 
@@ -594,6 +619,8 @@ def main(argv=None):
                     help="time the sequence-form scan with the output gate z and the last state instead")
     ap.add_argument("--paths", choices=["cross", "diagonal"], default="cross",
                     help="path set of the fused SS2D (default: the cross scan)")
+    ap.add_argument("--proj", action="store_true",
+                    help="time the fused forward with its per-path x_proj/dt_proj producer instead")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="time budget of the CPU oracle sample")

@@ -238,6 +238,31 @@ SS2D_API ss2d_status_t ss2d_backward(const ss2d_desc_t *desc, const void *x, con
                             void *dBm, void *dCm, float *dD, float *ddelta_bias,
                             void *workspace, size_t workspace_bytes, ss2d_stream_t stream);
 
+/* ------------------------------------------------ producer projections -- */
+
+/*
+ * Fused SS2D forward with its producer: the scan's delta, B and C are made from x by
+ * per-path projections, as MambaInnerFn.forward makes them ("vision mamba-yolov8",
+ * section 2): x_dbl = x_proj(u_k), delta = dt_proj.weight @ x_dbl[:R], B and C the next N
+ * and the last N rows of x_dbl; dt_proj.bias is the delta bias.  Here delta is never
+ * written: the scan computes dt = softplus(W_dt . x_dbl[:R] + bias) at every step.
+ * dt_rank          : R, 1 <= R <= 32 (ceil(d_model / 16) for d_model <= 512)
+ * x                : (B, D, H, W)  in_dtype
+ * x_proj_weight    : (4, R + 2N, D) fp32, one projection per path
+ * dt_proj_weight   : (4, D, R)     fp32
+ * dt_proj_bias     : (4D)          fp32 or NULL
+ * A, D, delta_softplus, y, chunk_states: as for ss2d_forward
+ * x_dbl            : (B, 4, R + 2N, L) in_dtype, written (each path's step order): the saved
+ *                    activation a backward needs
+ * workspace        : ss2d_workspace_bytes(desc, SS2D_OP_FORWARD) bytes
+ * Errors: SS2D_ERR_SHAPE for dt_rank outside [1, 32]; otherwise as for ss2d_forward.
+ */
+SS2D_API ss2d_status_t ss2d_forward_proj(const ss2d_desc_t *desc, int dt_rank, const void *x,
+                                         const float *x_proj_weight, const float *dt_proj_weight,
+                                         const float *dt_proj_bias, const float *A, const float *D,
+                                         int delta_softplus, void *y, void *x_dbl, float *chunk_states,
+                                         void *workspace, size_t workspace_bytes, ss2d_stream_t stream);
+
 /* ------------------------------------------------------------ path sets -- */
 
 /*

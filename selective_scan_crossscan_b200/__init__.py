@@ -36,7 +36,7 @@ __all__ = [
     "SS2DError", "cross_scan", "cross_merge", "selective_scan_fwd", "selective_scan_bwd", "selective_scan_fn",
     "SelectiveScanFunction", "ss2d_forward", "bimamba_forward", "bimamba_backward", "BiMambaFunction",
     "bimamba_scan", "path_tables", "cross_scan_table", "cross_merge_table", "ss2d_forward_table",
-    "ss2d_backward_table", "PATHS_CROSS", "PATHS_DIAGONAL",
+    "ss2d_backward_table", "PATHS_CROSS", "PATHS_DIAGONAL", "ss2d_forward_proj",
     "ss2d_backward", "SS2DFunction", "ss2d", "workspace_bytes", "chunk_states_elems", "launch_count",
     "library_path", "CHUNK_LEN", "trace_events",
 ]
@@ -98,6 +98,7 @@ def _load():
         lib.ss2d_forward.argtypes = [D, P, P, P, P, P, P, P, i, P, P, P, sz, P]
         lib.ss2d_bimamba_forward.argtypes = [D, P, P, P, P, P, P, P, P, i, P, P, P, sz, P]
         lib.ss2d_path_tables.argtypes = [D, i, P, P]
+        lib.ss2d_forward_proj.argtypes = [D, i, P, P, P, P, P, P, i, P, P, P, P, sz, P]
         lib.ss2d_cross_scan_table.argtypes = [D, P, P, P, P]
         lib.ss2d_cross_merge_table.argtypes = [D, P, P, P, P]
         lib.ss2d_forward_table.argtypes = [D, P, P, P, P, P, P, P, P, i, P, P, P, sz, P]
@@ -108,7 +109,7 @@ def _load():
         for name in ("ss2d_cross_scan", "ss2d_cross_merge", "ss2d_selective_scan_fwd", "ss2d_selective_scan_bwd",
                      "ss2d_selective_scan_fwd_ex", "ss2d_selective_scan_bwd_ex", "ss2d_forward", "ss2d_backward",
                      "ss2d_bimamba_forward", "ss2d_bimamba_backward", "ss2d_path_tables", "ss2d_cross_scan_table",
-                     "ss2d_cross_merge_table", "ss2d_forward_table", "ss2d_backward_table"):
+                     "ss2d_cross_merge_table", "ss2d_forward_table", "ss2d_backward_table", "ss2d_forward_proj"):
             getattr(lib, name).restype = ctypes.c_int
         lib.ss2d_workspace_bytes.argtypes = [D, i]
         lib.ss2d_workspace_bytes.restype = sz
@@ -635,3 +636,40 @@ def ss2d_backward_table(x, delta, A, B, C, D, delta_bias, delta_softplus, dy, ta
                                  _stream(x))
     _check(st, "ss2d_backward_table")
     return dict(dx=dx, ddelta=ddelta, dA=dA, dB=dB, dC=dC, dD=dD, ddelta_bias=dbias)
+
+
+# ---------------------------------------------------------------- producer --
+
+def ss2d_forward_proj(x, x_proj_weight, dt_proj_weight, dt_proj_bias, A, D=None, delta_softplus=True, out=None,
+                      out_dtype=None, return_x_dbl=False, return_chunk_states=False, workspace=None):
+    """Fused SS2D forward with its per-path producer (MambaInnerFn.forward's x_proj and dt_proj):
+    x (Bn, D, H, W); x_proj_weight (4, R+2N, D); dt_proj_weight (4, D, R); dt_proj_bias (4D).
+    delta is never materialised: the scan computes softplus(W_dt . x_dbl[:R] + bias) per step.
+    Returns y [, x_dbl (Bn, 4, R+2N, L)] [, chunk_states]."""
+    x = _c(x)
+    Wx = _c(x_proj_weight, torch.float32)
+    Wdt = _c(dt_proj_weight, torch.float32)
+    A, D, bias = _params(A, D, dt_proj_bias)
+    Bn, Dn, H, W = x.shape
+    N = A.shape[1]
+    R = Wdt.shape[2]
+    if Wx.shape != (4, R + 2 * N, Dn) or Wdt.shape != (4, Dn, R):
+        raise ValueError("ss2d_forward_proj: x_proj_weight must be (4, R+2N, D) and dt_proj_weight (4, D, R)")
+    out_dtype = out_dtype or x.dtype
+    if out is None:
+        out = torch.empty((Bn, Dn, H, W), dtype=out_dtype, device=x.device)
+    x_dbl = torch.empty((Bn, 4, R + 2 * N, H * W), dtype=x.dtype, device=x.device)
+    cs = None
+    if return_chunk_states:
+        cs = torch.empty((Bn, 4 * Dn, -(-(H * W) // CHUNK_LEN), N), dtype=torch.float32, device=x.device)
+    d = _desc(Bn, Dn, H, W, N, x.dtype, out.dtype)
+    lib = _load()
+    nbytes = int(lib.ss2d_workspace_bytes(ctypes.byref(d), OP_FORWARD))
+    if workspace is None or workspace.numel() < nbytes:
+        workspace = _workspace(nbytes, x.device)
+    st = lib.ss2d_forward_proj(ctypes.byref(d), int(R), _p(x), _p(Wx), _p(Wdt), _p(bias), _p(A), _p(D),
+                               int(bool(delta_softplus)), _p(out), _p(x_dbl), _p(cs), _p(workspace), nbytes,
+                               _stream(x))
+    _check(st, "ss2d_forward_proj")
+    extra = ([x_dbl] if return_x_dbl else []) + ([cs] if return_chunk_states else [])
+    return (out, *extra) if extra else out

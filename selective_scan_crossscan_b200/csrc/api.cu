@@ -324,6 +324,58 @@ ss2d_status_t ss2d_selective_scan_bwd(const ss2d_desc_t *desc, const void *u, co
                                       workspace_bytes, stream);
 }
 
+ss2d_status_t ss2d_forward_proj(const ss2d_desc_t *desc, int dt_rank, const void *x, const float *x_proj_weight,
+                                const float *dt_proj_weight, const float *dt_proj_bias, const float *A,
+                                const float *D, int delta_softplus, void *y, void *x_dbl, float *chunk_states,
+                                void *workspace, size_t workspace_bytes, ss2d_stream_t stream) {
+    SS2D_TRY(check_desc(desc));
+    if (dt_rank < 1 || dt_rank > kProjRMax) return SS2D_ERR_SHAPE;
+    SS2D_TRY(need(x));
+    SS2D_TRY(need(x_proj_weight));
+    SS2D_TRY(need(dt_proj_weight));
+    SS2D_TRY(optional(dt_proj_bias));
+    SS2D_TRY(need(A));
+    SS2D_TRY(optional(D));
+    SS2D_TRY(need(y));
+    SS2D_TRY(need(x_dbl));
+    SS2D_TRY(optional(chunk_states));
+    const LaunchShape s = shape_of(desc);
+    const size_t ws = fwd_ws_bytes(s, desc->in_dtype);
+    if (ws > 0 && (!workspace || workspace_bytes < ws)) return SS2D_ERR_WORKSPACE;
+    SS2D_TRY(optional(workspace));
+    SS2D_TRY(check_device());
+    unsigned char *w = static_cast<unsigned char *>(workspace);
+    float *ys = reinterpret_cast<float *>(w);
+    w += round64((size_t)s.B * kPaths * s.D * s.L * sizeof(float));
+    void *xT = w;
+    w += round64((size_t)s.B * s.D * s.L * elem_size(desc->in_dtype));
+    void *seg = w;
+    cudaStream_t st = (cudaStream_t)stream;
+    SS2D_TRY(from_cuda(launch_transpose(s, desc->in_dtype, x, xT, st)));
+    const int RN = dt_rank + 2 * (int)s.N;
+    SS2D_TRY(from_cuda(launch_xproj(s, desc->in_dtype, x, xT, x_proj_weight, RN, x_dbl, st)));
+    ScanFwdArgs a;
+    a.u = x;
+    a.uT = xT;
+    a.delta = nullptr;
+    a.A = A;
+    a.Bm = nullptr;
+    a.Cm = nullptr;
+    a.Dv = D;
+    a.bias = dt_proj_bias;
+    a.softplus = delta_softplus != 0;
+    a.out = ys;
+    a.chunk_states = chunk_states;
+    a.from_image = true;
+    a.xdbl = x_dbl;
+    a.Wdt = dt_proj_weight;
+    a.R = dt_rank;
+    a.in_dtype = desc->in_dtype;
+    a.out_dtype = SS2D_F32;
+    SS2D_TRY(from_cuda(launch_scan_fwd(s, a, seg, st)));
+    return from_cuda(launch_cross_merge(s, SS2D_F32, desc->out_dtype, ys, y, st));
+}
+
 ss2d_status_t ss2d_path_tables(const ss2d_desc_t *desc, int paths, int32_t *tables, ss2d_stream_t stream) {
     SS2D_TRY(check_desc(desc));
     SS2D_TRY(check_table_shape(desc));

@@ -30,7 +30,12 @@ cudaError_t launch_cross_merge(const LaunchShape &s, ss2d_dtype_t din, ss2d_dtyp
 //  kModeImg   -- u read from the image along SS2D path k (fused CrossScan);
 //  kModeBidir -- a 1D sequence and its reverse (K = 2 directions) reading the same
 //                x, delta, B, C in natural order, the reverse direction backwards.
-enum ScanMode { kModeSeq = 0, kModeImg = 1, kModeBidir = 2 };
+//  kModeImgProj -- kModeImg with the producer fused in: B, C and the low-rank dt rows come from
+//                the per-path x_proj output, dt = softplus(W_dt . x_dbl[:R] + bias) in-kernel;
+//                kModeImgProjWide is the same for ranks above kProjRNarrow.
+enum ScanMode { kModeSeq = 0, kModeImg = 1, kModeBidir = 2, kModeImgProj = 3, kModeImgProjWide = 4 };
+constexpr int kProjRNarrow = 8;  // dt ranks up to this use the narrow (smaller) projection kernels
+constexpr int kProjRMax = 32;    // largest dt_rank the fused projection takes
 
 struct ScanFwdArgs {
     const void *u;       // (B, 4D, L) sequences, or (B, D, H, W) image when from_image
@@ -49,6 +54,9 @@ struct ScanFwdArgs {
     bool from_image;     // read u along path k from the image (fused CrossScan)
     bool bidir = false;  // kModeBidir: x (B, D, L), delta (B, D, L), B/C (B, 1, N, L), A (2D, N),
                          // D/bias (D); out = per-direction outputs (B, 2, D, L) fp32 at natural positions
+    const void *xdbl = nullptr;  // kModeImgProj (with from_image): x_proj outputs (B, 4, R+2N, L) in_dtype
+    const float *Wdt = nullptr;  // kModeImgProj: dt_proj weight (4D, R)
+    int R = 0;                   // kModeImgProj: dt rank
     ss2d_dtype_t in_dtype, out_dtype;
     int max_segments = 32;  // 1 = never split a sequence (no workspace needed)
 };
@@ -70,6 +78,11 @@ cudaError_t launch_cross_scan_table(const LaunchShape &s, ss2d_dtype_t dt, const
                                     void *xs, cudaStream_t stream);
 cudaError_t launch_cross_merge_table(const LaunchShape &s, ss2d_dtype_t din, ss2d_dtype_t dout, const void *ys,
                                      const int32_t *tab, void *y, cudaStream_t stream);
+
+// Per-path x_proj: xdbl[b, k, c, l] = sum_d W[k, c, d] u_k[d, l] (u_0/u_2 from x, u_1/u_3 from xT),
+// in each path's step order, RN = R + 2N <= 64 rows.
+cudaError_t launch_xproj(const LaunchShape &s, ss2d_dtype_t dt, const void *x, const void *xT, const float *W,
+                         int RN, void *xdbl, cudaStream_t stream);
 
 // Bidirectional scan: out[b, d, m] = (two[b, 0, d, m] + two[b, 1, d, m]) * (z ? silu(z[b, d, m]) : 1),
 // two (B, 2, D, L) fp32, z (B, D, L) z_dtype or null, out (B, D, L) out_dtype.

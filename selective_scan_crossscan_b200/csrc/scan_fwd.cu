@@ -81,6 +81,9 @@ struct FwdParams {
     const void *z;       // (B, 4D, L) output gate or null (sequence mode only)
     float *last_state;   // (B, 4D, N) or null
     float *seg;  // (B, 4D, nseg, 2, N): decay product and end state of each segment
+    const void *xdbl;    // projection mode: (B, 4, R+2N, L) per-path x_proj outputs, in_dtype
+    const float *Wdt;    // projection mode: (4D, R)
+    int R;
     int64_t B, D, H, W, L;
     int N;
     int softplus;
@@ -124,12 +127,30 @@ struct FwdStage {
 //  * fp32 rows of any alignment: one 4-byte cp.async per element, slots past the end zeroed;
 //  * bf16 rows of any alignment: plain loads (synchronous), slots past the end zeroed.
 // REV: the chunk is walked backwards through delta, B and C as well (bidirectional scan).
-template <int NS, bool VEC, bool REV, typename Tin>
+// PROJ: instead of each lane's delta row, the R <= RB low-rank dt rows of the group (dts, like B/C).
+template <int NS, bool VEC, bool REV, bool PROJ, int RB, typename Tin>
 __device__ __forceinline__ void stage_chunk(FwdStage<Tin, NS> &st, const Tin *Bk, const Tin *Ck, int N, int64_t L,
                                             const Tin *urow, bool urev, const Tin *drow, bool active, int64_t cbeg,
-                                            int len) {
+                                            int len, Tin (*dts)[kLC] = nullptr, const Tin *DTk = nullptr,
+                                            int R = 0) {
     const int t = threadIdx.x;
     constexpr int kBytes = 4 * (int)sizeof(Tin);
+    if (PROJ) {  // the group's dt rows, in the same slots as B/C
+        for (int idx = t; idx < RB * kLC; idx += kWarp) {
+            const int r = idx / kLC, i = idx % kLC;
+            if (VEC) {
+                if (i % 4 == 0 && r < R && i < len)
+                    cp_async_bytes(&dts[r][i], DTk + (int64_t)r * L + cbeg + i, kBytes);
+            } else if (sizeof(Tin) == 4) {
+                if (r < R && i < len)
+                    cp_async_bytes(&dts[r][i], DTk + (int64_t)r * L + cbeg + i, 4);
+                else
+                    dts[r][i] = Tin(0.f);
+            } else {
+                dts[r][i] = (r < R && i < len) ? DTk[(int64_t)r * L + cbeg + i] : Tin(0.f);
+            }
+        }
+    }
     if (VEC) {
         constexpr int q = kLC / 4;
         for (int idx = t; idx < NS * q; idx += kWarp) {
@@ -148,7 +169,9 @@ __device__ __forceinline__ void stage_chunk(FwdStage<Tin, NS> &st, const Tin *Bk
 #pragma unroll
             for (int i4 = 0; i4 < kLC; i4 += 4) {
                 if (i4 < len) {
-                    if (!REV)
+                    if (PROJ)
+                        ;  // no delta row: dt comes from the projection
+                    else if (!REV)
                         cp_async_bytes(&st.Dl[t][i4], drow + cbeg + i4, kBytes);
                     else
                         cp_async_bytes(&st.Dl[t][kLC - 4 - i4], drow + (L - cbeg - 4 - i4), kBytes);
@@ -176,7 +199,7 @@ __device__ __forceinline__ void stage_chunk(FwdStage<Tin, NS> &st, const Tin *Bk
             const int64_t l = cbeg + i;
             const int dslot = REV ? kLC - 1 - i : i, uslot = urev ? kLC - 1 - i : i;
             if (active && i < len) {
-                cp_async_bytes(&st.Dl[t][dslot], drow + (REV ? L - 1 - l : l), 4);
+                if (!PROJ) cp_async_bytes(&st.Dl[t][dslot], drow + (REV ? L - 1 - l : l), 4);
                 cp_async_bytes(&st.U[t][uslot], urow + (urev ? L - 1 - l : l), 4);
             } else {
                 st.Dl[t][dslot] = Tin(0.f);
@@ -195,7 +218,7 @@ __device__ __forceinline__ void stage_chunk(FwdStage<Tin, NS> &st, const Tin *Bk
         for (int i = 0; i < kLC; ++i) {
             const bool ok = active && i < len;
             const int64_t l = cbeg + i;
-            st.Dl[t][REV ? kLC - 1 - i : i] = ok ? drow[REV ? L - 1 - l : l] : Tin(0.f);
+            if (!PROJ) st.Dl[t][REV ? kLC - 1 - i : i] = ok ? drow[REV ? L - 1 - l : l] : Tin(0.f);
             st.U[t][urev ? (kLC - 1 - i) : i] = ok ? urow[urev ? (L - 1 - l) : l] : Tin(0.f);
         }
     }
@@ -210,10 +233,19 @@ __host__ __device__ constexpr bool a2_in_smem() {
 
 // The scan of one CTA.  PASS 0: single pass.  PASS 1: segment summaries only.  PASS 2:
 // outputs with carries.  REV: the reverse direction of the bidirectional scan.
+// dt ranks the projection modes' shared arrays are sized for
+template <int MODE>
+__host__ __device__ constexpr int proj_rank_bucket() {
+    return MODE == kModeImgProj ? kProjRNarrow : (MODE == kModeImgProjWide ? kProjRMax : 1);
+}
+
 template <int NS, typename Tin, typename Tout, int MODE, int PASS, bool VEC, bool REV>
 __device__ __forceinline__ void scan_fwd_body(const FwdParams &p, FwdStage<Tin, NS> (&stage)[2],
-                                              float (&A2s)[a2_in_smem<Tin>() ? NS : 1][kWarp]) {
-    constexpr bool IMG = MODE == kModeImg, BIDIR = MODE == kModeBidir, SEQ = MODE == kModeSeq;
+                                              float (&A2s)[a2_in_smem<Tin>() ? NS : 1][kWarp],
+                                              Tin (*dts)[proj_rank_bucket<MODE>()][kLC], float (*wsm)[kWarp]) {
+    constexpr bool PROJ = MODE == kModeImgProj || MODE == kModeImgProjWide;
+    constexpr int RB = proj_rank_bucket<MODE>();
+    constexpr bool IMG = MODE == kModeImg || PROJ, BIDIR = MODE == kModeBidir, SEQ = MODE == kModeSeq;
     constexpr bool kA2Smem = a2_in_smem<Tin>();
     float A2r[NS];
 #define SS2D_A2(n) (kA2Smem ? A2s[n][t] : A2r[n])
@@ -239,6 +271,10 @@ __device__ __forceinline__ void scan_fwd_body(const FwdParams &p, FwdStage<Tin, 
         else
             A2r[n] = a2v;
         h[n] = 0.f;
+    }
+    if (PROJ) {  // this lane's row of dt_proj, kept in shared memory (lanes fastest)
+#pragma unroll
+        for (int r = 0; r < RB; ++r) wsm[r][t] = (active && r < p.R) ? p.Wdt[c * p.R + r] : 0.f;
     }
     const int64_t pc = BIDIR ? (active ? d : 0) : c;  // D and delta_bias are shared by the two directions
     const float Dc = (active && p.Dv) ? p.Dv[pc] : 0.f;
@@ -268,10 +304,13 @@ __device__ __forceinline__ void scan_fwd_body(const FwdParams &p, FwdStage<Tin, 
         urow = static_cast<const Tin *>(p.u) + (b * C4 + c) * L;
         urev = false;
     }
-    const Tin *drow = static_cast<const Tin *>(p.delta) + (BIDIR ? b * D + (active ? d : 0) : b * C4 + c) * L;
+    const Tin *drow =
+        PROJ ? nullptr : static_cast<const Tin *>(p.delta) + (BIDIR ? b * D + (active ? d : 0) : b * C4 + c) * L;
     const int64_t grp = BIDIR ? b : b * kPaths + k;  // the B/C group of this (b, k)
-    const Tin *Bk = static_cast<const Tin *>(p.Bm) + grp * N * L;
-    const Tin *Ck = static_cast<const Tin *>(p.Cm) + grp * N * L;
+    // projection mode: the group's x_proj outputs are R dt rows, then N rows of B, then N of C
+    const Tin *DTk = PROJ ? static_cast<const Tin *>(p.xdbl) + grp * (p.R + 2 * N) * L : nullptr;
+    const Tin *Bk = PROJ ? DTk + (int64_t)p.R * L : static_cast<const Tin *>(p.Bm) + grp * N * L;
+    const Tin *Ck = PROJ ? Bk + (int64_t)N * L : static_cast<const Tin *>(p.Cm) + grp * N * L;
     Tout *orow = p.out ? static_cast<Tout *>(p.out) + (b * C4 + c) * L : nullptr;
 
     const int64_t nloc = lend - lbeg;
@@ -288,7 +327,8 @@ __device__ __forceinline__ void scan_fwd_body(const FwdParams &p, FwdStage<Tin, 
     }
     __syncwarp();
 
-    stage_chunk<NS, VEC, REV>(stage[0], Bk, Ck, N, L, urow, urev, drow, active, lbeg, (int)min((int64_t)kLC, nloc));
+    stage_chunk<NS, VEC, REV, PROJ, RB>(stage[0], Bk, Ck, N, L, urow, urev, drow, active, lbeg,
+                                    (int)min((int64_t)kLC, nloc), PROJ ? dts[0] : nullptr, DTk, p.R);
     cp_async_commit();
 
     for (int ch = 0; ch < nchunk; ++ch) {
@@ -297,8 +337,9 @@ __device__ __forceinline__ void scan_fwd_body(const FwdParams &p, FwdStage<Tin, 
         const int buf = ch & 1;
         if (ch + 1 < nchunk) {
             const int64_t nbeg = cbeg + kLC;
-            stage_chunk<NS, VEC, REV>(stage[buf ^ 1], Bk, Ck, N, L, urow, urev, drow, active, nbeg,
-                                 (int)min((int64_t)kLC, lend - nbeg));
+            stage_chunk<NS, VEC, REV, PROJ, RB>(stage[buf ^ 1], Bk, Ck, N, L, urow, urev, drow, active, nbeg,
+                                            (int)min((int64_t)kLC, lend - nbeg), PROJ ? dts[buf ^ 1] : nullptr, DTk,
+                                            p.R);
             cp_async_commit();
             cp_async_wait<1>();
         } else {
@@ -313,7 +354,23 @@ __device__ __forceinline__ void scan_fwd_body(const FwdParams &p, FwdStage<Tin, 
                 const int nvalid = (int)min((int64_t)kG, lend - l0);
                 float uv[kG], dv[kG];
                 {  // slots hold 4-step groups in every staging form (see stage_chunk)
-                    if (!REV) {
+                    if (PROJ) {  // delta = dt_proj . x_dbl[:R] for the four steps
+                        float2 a01 = make_float2(0.f, 0.f), a23 = make_float2(0.f, 0.f);
+#pragma unroll
+                        for (int r = 0; r < RB; ++r) {
+                            if (r < p.R) {
+                                const float w = wsm[r][t];
+                                float q[kG];
+                                ld4(&dts[buf][r][g], q);
+                                a01 = __ffma2_rn(make_float2(w, w), make_float2(q[0], q[1]), a01);
+                                a23 = __ffma2_rn(make_float2(w, w), make_float2(q[2], q[3]), a23);
+                            }
+                        }
+                        dv[0] = a01.x;
+                        dv[1] = a01.y;
+                        dv[2] = a23.x;
+                        dv[3] = a23.y;
+                    } else if (!REV) {
                         ld4(&sm.Dl[t][g], dv);
                     } else {
                         float w[kG];
@@ -467,10 +524,15 @@ template <int NS, typename Tin, typename Tout, int MODE, int PASS, bool VEC>
 __global__ void __launch_bounds__(kWarp, SS2D_FWD_MIN_BLOCKS) scan_fwd_kernel(const FwdParams p) {
     __shared__ __align__(16) FwdStage<Tin, NS> stage[2];
     __shared__ float A2s[a2_in_smem<Tin>() ? NS : 1][kWarp];
-    if (MODE == kModeBidir && blockIdx.y == 1)
-        scan_fwd_body<NS, Tin, Tout, MODE, PASS, VEC, true>(p, stage, A2s);
-    else
-        scan_fwd_body<NS, Tin, Tout, MODE, PASS, VEC, false>(p, stage, A2s);
+    if constexpr (MODE == kModeImgProj || MODE == kModeImgProjWide) {  // dt rows, each lane's dt_proj row
+        __shared__ __align__(16) Tin dts[2][proj_rank_bucket<MODE>()][kLC];
+        __shared__ float wsm[proj_rank_bucket<MODE>()][kWarp];
+        scan_fwd_body<NS, Tin, Tout, MODE, PASS, VEC, false>(p, stage, A2s, dts, wsm);
+    } else if (MODE == kModeBidir && blockIdx.y == 1) {
+        scan_fwd_body<NS, Tin, Tout, MODE, PASS, VEC, true>(p, stage, A2s, nullptr, nullptr);
+    } else {
+        scan_fwd_body<NS, Tin, Tout, MODE, PASS, VEC, false>(p, stage, A2s, nullptr, nullptr);
+    }
 }
 
 // Segment plan: how many segments each sequence is cut into, and their length
@@ -551,6 +613,9 @@ cudaError_t launch_scan_fwd(const LaunchShape &s, const ScanFwdArgs &a, void *wo
     p.z = seq ? a.z : nullptr;
     p.last_state = seq ? a.last_state : nullptr;
     p.seg = static_cast<float *>(workspace);
+    p.xdbl = a.xdbl;
+    p.Wdt = a.Wdt;
+    p.R = a.R;
     p.B = s.B;
     p.D = s.D;
     p.H = s.H;
@@ -568,6 +633,20 @@ cudaError_t launch_scan_fwd(const LaunchShape &s, const ScanFwdArgs &a, void *wo
                        : launch_types<float, float, kModeBidir, false>(p, stream);
         return vec ? launch_types<__nv_bfloat16, float, kModeBidir, true>(p, stream)
                    : launch_types<__nv_bfloat16, float, kModeBidir, false>(p, stream);
+    }
+    if (a.from_image && a.xdbl) {  // producer fused: fp32 per-path outputs for the merge
+        if (a.R <= kProjRNarrow) {
+            if (a.in_dtype == SS2D_F32)
+                return vec ? launch_types<float, float, kModeImgProj, true>(p, stream)
+                           : launch_types<float, float, kModeImgProj, false>(p, stream);
+            return vec ? launch_types<__nv_bfloat16, float, kModeImgProj, true>(p, stream)
+                       : launch_types<__nv_bfloat16, float, kModeImgProj, false>(p, stream);
+        }
+        if (a.in_dtype == SS2D_F32)
+            return vec ? launch_types<float, float, kModeImgProjWide, true>(p, stream)
+                       : launch_types<float, float, kModeImgProjWide, false>(p, stream);
+        return vec ? launch_types<__nv_bfloat16, float, kModeImgProjWide, true>(p, stream)
+                   : launch_types<__nv_bfloat16, float, kModeImgProjWide, false>(p, stream);
     }
     if (a.from_image)
         return vec ? launch_mode<kModeImg, true>(p, a.in_dtype, a.out_dtype, stream)

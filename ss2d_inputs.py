@@ -181,6 +181,42 @@ def make_bimamba_inputs(w: Workload, seed: int = 0, device="cpu", with_dy: bool 
     return out
 
 
+def dt_rank_of(dim: int) -> int:
+    """dt_rank = ceil(d_model / 16) (Mamba.__init__), with d_model = dim / 2 for SS2D's
+    expansion of 2 (VMamba-T: 192 channels, d_model 96, rank 6)."""
+    return max(1, math.ceil((dim // 2) / 16))
+
+
+def make_proj_inputs(w: Workload, seed: int = 0, device="cpu"):
+    """Inputs of the SS2D forward with its producer (x_proj, dt_proj per path), drawn as
+    Mamba.__init__ initialises them: x ~ N(0,1) (B, D, H, W); x_proj weight (4, R+2N, D)
+    ~ U(-1/sqrt(D), 1/sqrt(D)) (nn.Linear's default); dt_proj weight (4, D, R) ~
+    U(-R^-0.5, R^-0.5) (dt_init "random", dt_scale 1); dt_proj bias, A and D as in make_inputs.
+    Draw order: x, x_proj weight, dt_proj weight, dt."""
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed) + 3000)
+    f32 = dict(dtype=torch.float32, device=device, generator=g)
+    Bn, Dn, N = w.batch, w.dim, w.d_state
+    R = dt_rank_of(Dn)
+    x = torch.randn((Bn, Dn, w.height, w.width), **f32)
+    bx = 1.0 / math.sqrt(Dn)
+    Wx = (torch.rand((K_PATHS, R + 2 * N, Dn), **f32) * 2 - 1) * bx
+    bd = R ** -0.5
+    Wdt = (torch.rand((K_PATHS, Dn, R), **f32) * 2 - 1) * bd
+    dt_min, dt_max, dt_floor = 1e-3, 1e-1, 1e-4
+    dt = torch.exp(torch.rand((K_PATHS * Dn,), **f32) * (math.log(dt_max) - math.log(dt_min))
+                   + math.log(dt_min)).clamp(min=dt_floor)
+    bias = dt + torch.log(-torch.expm1(-dt))
+    n1 = torch.arange(1, N + 1, dtype=torch.float32, device=device)
+    A_row = -n1 if w.a_init == "neg_index" else -torch.exp(torch.log(n1))
+    A = A_row.unsqueeze(0).repeat(K_PATHS * Dn, 1).contiguous()
+    out = dict(x=x, x_proj_weight=Wx, dt_proj_weight=Wdt, dt_proj_bias=bias, A=A,
+               D=torch.ones(K_PATHS * Dn, dtype=torch.float32, device=device), R=R)
+    if w.dtype == "bf16":
+        out["x"] = out["x"].to(torch.bfloat16)
+    return out
+
+
 def batch_slice(inputs: dict, idx) -> dict:
     """Restrict batch-indexed tensors to batch items `idx` (a list); parameters are shared."""
     out = {}

@@ -152,6 +152,16 @@ def test_path_table_argument_errors(lib):
     assert f(_d(), None, *args, None, None, 1, B16, None, A16, wsf, None) == ERR_NULL
 
 
+def test_forward_proj_argument_errors(lib):
+    f = lib.ss2d_forward_proj
+    ws = lib.ss2d_workspace_bytes(_d(), ss.OP_FORWARD)
+    w = [A16, A16, A16, A16]  # x, x_proj_weight, dt_proj_weight, dt_proj_bias
+    assert f(_d(), 0, *w, A16, None, 1, B16, B16, None, A16, ws, None) == ERR_SHAPE   # dt_rank 0
+    assert f(_d(), 33, *w, A16, None, 1, B16, B16, None, A16, ws, None) == ERR_SHAPE  # dt_rank > 32
+    assert f(_d(), 2, *w, A16, None, 1, B16, None, None, A16, ws, None) == ERR_NULL   # x_dbl
+    assert f(_d(), 2, *w, A16, None, 1, B16, B16, None, A16, ws - 1, None) == ERR_WORKSPACE
+
+
 def test_valid_call_without_gpu_reports_device_error(lib):
     import torch
     if torch.cuda.is_available():

@@ -553,6 +553,63 @@ def test_ss2d_diagonal_full_stage1_sampled():
         assert_fwd_close(y[bi:bi + 1], ref, f"y[{bi}]")
 
 
+# ----------------------------------------------------- producer projections
+
+def _proj_case(Bn, Dn, H, W, N, dtype="f32", seed=0):
+    w = ss2d_inputs.custom(Bn, Dn, H, W, N, dtype=dtype, a_init="s4d_real")
+    return w, ss2d_inputs.make_proj_inputs(w, seed=seed)
+
+
+# R = ceil(D / 32): D = 8 -> 1, 70 -> 3, 192 -> 6, 512 -> 8; ragged and one-pixel maps, N < 16
+PROJ_CASES = [(1, 8, 8, 8, 4), (2, 70, 5, 9, 16), (1, 40, 12, 11, 8), (2, 6, 1, 1, 16), (1, 192, 14, 14, 16),
+              (1, 512, 4, 6, 16)]
+
+
+@pytest.mark.parametrize("case", PROJ_CASES)
+def test_ss2d_forward_proj_parity(case):
+    w, inp = _proj_case(*case, seed=50)
+    d = _dev({k: v for k, v in inp.items() if k != "R"})
+    y, x_dbl = ss.ss2d_forward_proj(d["x"], d["x_proj_weight"], d["dt_proj_weight"], d["dt_proj_bias"], d["A"],
+                                    d["D"], True, return_x_dbl=True)
+    _, _, _, ref_dbl = oracle.path_projections(inp["x"], inp["x_proj_weight"], inp["dt_proj_weight"])
+    assert_fwd_close(x_dbl, ref_dbl, f"{case} x_dbl")
+    ref = oracle.ss2d_forward_proj(inp["x"], inp["x_proj_weight"], inp["dt_proj_weight"], inp["dt_proj_bias"],
+                                   inp["A"], inp["D"], True)
+    assert_fwd_close(y, ref, f"{case} y")
+
+
+def test_ss2d_forward_proj_matches_materialised_delta():
+    # the in-kernel dt projection against the plain fused forward fed the same projections
+    w, inp = _proj_case(2, 24, 9, 10, 16, seed=51)
+    d = _dev({k: v for k, v in inp.items() if k != "R"})
+    y, x_dbl = ss.ss2d_forward_proj(d["x"], d["x_proj_weight"], d["dt_proj_weight"], d["dt_proj_bias"], d["A"],
+                                    d["D"], True, return_x_dbl=True)
+    R, N = inp["R"], w.d_state
+    xd = x_dbl.double()
+    delta = torch.einsum("kdr,bkrl->bkdl", d["dt_proj_weight"].double(), xd[:, :, :R]).reshape(2, 4 * 24, 90)
+    y2 = ss.ss2d_forward(d["x"], delta.float(), d["A"], x_dbl[:, :, R:R + N].contiguous(),
+                         x_dbl[:, :, R + N:].contiguous(), d["D"], d["dt_proj_bias"], True)
+    torch.testing.assert_close(y, y2, rtol=1e-5, atol=1e-5)
+
+
+def test_ss2d_forward_proj_bf16_and_full_stage1_sampled():
+    w, inp = _proj_case(2, 16, 12, 12, 16, dtype="bf16", seed=52)
+    d = _dev({k: v for k, v in inp.items() if k != "R"})
+    y = ss.ss2d_forward_proj(d["x"], d["x_proj_weight"], d["dt_proj_weight"], d["dt_proj_bias"], d["A"], d["D"])
+    ref = oracle.ss2d_forward_proj(inp["x"], inp["x_proj_weight"], inp["dt_proj_weight"], inp["dt_proj_bias"],
+                                   inp["A"], inp["D"], True)
+    assert_rel_l2(y, ref, BF16_TOL, "y bf16")
+    # VMamba-T stage-1 shapes in the launch configuration bench.py times, sampled batch items
+    w = ss2d_inputs.workload("vmamba_t_stage1_fp32")
+    inp = ss2d_inputs.make_proj_inputs(w, seed=53)
+    d = _dev({k: v for k, v in inp.items() if k != "R"})
+    y = ss.ss2d_forward_proj(d["x"], d["x_proj_weight"], d["dt_proj_weight"], d["dt_proj_bias"], d["A"], d["D"])
+    for bi in (0, w.batch - 1):
+        ref = oracle.ss2d_forward_proj(inp["x"][bi:bi + 1], inp["x_proj_weight"], inp["dt_proj_weight"],
+                                       inp["dt_proj_bias"], inp["A"], inp["D"], True)
+        assert_fwd_close(y[bi:bi + 1], ref, f"y[{bi}]")
+
+
 # ------------------------------------------------------------- fused SS2D
 
 FUSED_CASES = [(1, 8, 8, 8, 4), (2, 6, 5, 9, 16), (1, 70, 12, 11, 16), (1, 8, 64, 64, 16), (2, 3, 1, 1, 2),
