@@ -355,8 +355,11 @@ def run_gpu(args, world, rank, local):
         x_dbl = torch.empty((w.batch, 4, R + 2 * w.d_state, w.L), dtype=w.torch_dtype, device=dev)
         pargs = (inp["x"], inp["x_proj_weight"], inp["dt_proj_weight"], inp["dt_proj_bias"], inp["A"], inp["D"])
 
+        npj = ss.workspace_bytes(w.batch, w.dim, w.height, w.width, w.d_state, ss.OP_FORWARD_PROJ, w.torch_dtype)
+        wsp = torch.empty(max(npj, 1), dtype=torch.uint8, device=dev)
+
         def step():
-            ss.ss2d_forward_proj(*pargs, True, out=y, workspace=ws)
+            ss.ss2d_forward_proj(*pargs, True, out=y, workspace=wsp)
     elif bidir:
         y_seq = torch.empty((w.batch, w.dim, w.L), dtype=w.torch_dtype, device=dev)
         nbf = ss.workspace_bytes(w.batch, w.dim, 1, w.L, w.d_state, ss.OP_BIMAMBA_FORWARD, w.torch_dtype)

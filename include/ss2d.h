@@ -89,7 +89,8 @@ typedef enum {
     SS2D_OP_BIMAMBA_FORWARD = 4,
     SS2D_OP_BIMAMBA_BACKWARD = 5,
     SS2D_OP_FORWARD_TABLE = 6,
-    SS2D_OP_BACKWARD_TABLE = 7
+    SS2D_OP_BACKWARD_TABLE = 7,
+    SS2D_OP_FORWARD_PROJ = 8
 } ss2d_op_t;
 
 /* Path sets that ss2d_path_tables generates (paths 2 and 3 are always 0 and 1 walked backwards). */
@@ -244,8 +245,10 @@ SS2D_API ss2d_status_t ss2d_backward(const ss2d_desc_t *desc, const void *x, con
  * Fused SS2D forward with its producer: the scan's delta, B and C are made from x by
  * per-path projections, as MambaInnerFn.forward makes them ("vision mamba-yolov8",
  * section 2): x_dbl = x_proj(u_k), delta = dt_proj.weight @ x_dbl[:R], B and C the next N
- * and the last N rows of x_dbl; dt_proj.bias is the delta bias.  Here delta is never
- * written: the scan computes dt = softplus(W_dt . x_dbl[:R] + bias) at every step.
+ * and the last N rows of x_dbl; dt_proj.bias is the delta bias.  For dt_rank <= 8 delta is
+ * never written: the scan computes dt = softplus(W_dt . x_dbl[:R] + bias) at every step;
+ * for larger ranks delta is materialised in the workspace (R multiply-adds per step would
+ * cost the scan more than reading it).  B and C are read from x_dbl in both cases.
  * dt_rank          : R, 1 <= R <= 32 (ceil(d_model / 16) for d_model <= 512)
  * x                : (B, D, H, W)  in_dtype
  * x_proj_weight    : (4, R + 2N, D) fp32, one projection per path
@@ -254,7 +257,7 @@ SS2D_API ss2d_status_t ss2d_backward(const ss2d_desc_t *desc, const void *x, con
  * A, D, delta_softplus, y, chunk_states: as for ss2d_forward
  * x_dbl            : (B, 4, R + 2N, L) in_dtype, written (each path's step order): the saved
  *                    activation a backward needs
- * workspace        : ss2d_workspace_bytes(desc, SS2D_OP_FORWARD) bytes
+ * workspace        : ss2d_workspace_bytes(desc, SS2D_OP_FORWARD_PROJ) bytes
  * Errors: SS2D_ERR_SHAPE for dt_rank outside [1, 32]; otherwise as for ss2d_forward.
  */
 SS2D_API ss2d_status_t ss2d_forward_proj(const ss2d_desc_t *desc, int dt_rank, const void *x,

@@ -50,7 +50,7 @@ _lib = None
 CHUNK_LEN = 16  # SS2D_CHUNK_LEN
 F32, BF16 = 0, 1
 OP_SELECTIVE_SCAN_BWD, OP_FORWARD, OP_BACKWARD, OP_BIMAMBA_FORWARD, OP_BIMAMBA_BACKWARD = 1, 2, 3, 4, 5
-OP_FORWARD_TABLE, OP_BACKWARD_TABLE = 6, 7
+OP_FORWARD_TABLE, OP_BACKWARD_TABLE, OP_FORWARD_PROJ = 6, 7, 8
 PATHS_CROSS, PATHS_DIAGONAL = 0, 1
 _STATUS = {0: "SS2D_OK", 1: "SS2D_ERR_NULL", 2: "SS2D_ERR_SHAPE", 3: "SS2D_ERR_DTYPE", 4: "SS2D_ERR_ALIGN",
            5: "SS2D_ERR_WORKSPACE", 6: "SS2D_ERR_LAUNCH", 7: "SS2D_ERR_TIMEOUT", 8: "SS2D_ERR_DEVICE"}
@@ -644,7 +644,8 @@ def ss2d_forward_proj(x, x_proj_weight, dt_proj_weight, dt_proj_bias, A, D=None,
                       out_dtype=None, return_x_dbl=False, return_chunk_states=False, workspace=None):
     """Fused SS2D forward with its per-path producer (MambaInnerFn.forward's x_proj and dt_proj):
     x (Bn, D, H, W); x_proj_weight (4, R+2N, D); dt_proj_weight (4, D, R); dt_proj_bias (4D).
-    delta is never materialised: the scan computes softplus(W_dt . x_dbl[:R] + bias) per step.
+    For dt ranks up to 8 delta is never materialised: the scan computes softplus(W_dt . x_dbl[:R] +
+    bias) per step; larger ranks materialise delta in the workspace.
     Returns y [, x_dbl (Bn, 4, R+2N, L)] [, chunk_states]."""
     x = _c(x)
     Wx = _c(x_proj_weight, torch.float32)
@@ -664,7 +665,7 @@ def ss2d_forward_proj(x, x_proj_weight, dt_proj_weight, dt_proj_bias, A, D=None,
         cs = torch.empty((Bn, 4 * Dn, -(-(H * W) // CHUNK_LEN), N), dtype=torch.float32, device=x.device)
     d = _desc(Bn, Dn, H, W, N, x.dtype, out.dtype)
     lib = _load()
-    nbytes = int(lib.ss2d_workspace_bytes(ctypes.byref(d), OP_FORWARD))
+    nbytes = int(lib.ss2d_workspace_bytes(ctypes.byref(d), OP_FORWARD_PROJ))
     if workspace is None or workspace.numel() < nbytes:
         workspace = _workspace(nbytes, x.device)
     st = lib.ss2d_forward_proj(ctypes.byref(d), int(R), _p(x), _p(Wx), _p(Wdt), _p(bias), _p(A), _p(D),

@@ -187,6 +187,8 @@ size_t ss2d_workspace_bytes(const ss2d_desc_t *desc, int op) {
         case SS2D_OP_BIMAMBA_FORWARD: return bidir_fwd_ws_bytes(s);
         case SS2D_OP_BIMAMBA_BACKWARD: return bidir_bwd_ws_bytes(s);
         case SS2D_OP_FORWARD_TABLE: return table_fwd_ws_bytes(s, desc->in_dtype);
+        case SS2D_OP_FORWARD_PROJ:
+            return fwd_ws_bytes(s, desc->in_dtype) + round64((size_t)s.B * kPaths * s.D * s.L * elem_size(desc->in_dtype));
         case SS2D_OP_BACKWARD_TABLE: return table_bwd_ws_bytes(s, desc->in_dtype, desc->out_dtype);
         default: return (size_t)-1;
     }
@@ -340,11 +342,14 @@ ss2d_status_t ss2d_forward_proj(const ss2d_desc_t *desc, int dt_rank, const void
     SS2D_TRY(need(x_dbl));
     SS2D_TRY(optional(chunk_states));
     const LaunchShape s = shape_of(desc);
-    const size_t ws = fwd_ws_bytes(s, desc->in_dtype);
-    if (ws > 0 && (!workspace || workspace_bytes < ws)) return SS2D_ERR_WORKSPACE;
+    const size_t delta_bytes = round64((size_t)s.B * kPaths * s.D * s.L * elem_size(desc->in_dtype));
+    const size_t ws = fwd_ws_bytes(s, desc->in_dtype) + delta_bytes;
+    if (!workspace || workspace_bytes < ws) return SS2D_ERR_WORKSPACE;
     SS2D_TRY(optional(workspace));
     SS2D_TRY(check_device());
     unsigned char *w = static_cast<unsigned char *>(workspace);
+    void *delta = w;  // used for ranks above kProjRNarrow only
+    w += delta_bytes;
     float *ys = reinterpret_cast<float *>(w);
     w += round64((size_t)s.B * kPaths * s.D * s.L * sizeof(float));
     void *xT = w;
@@ -354,10 +359,12 @@ ss2d_status_t ss2d_forward_proj(const ss2d_desc_t *desc, int dt_rank, const void
     SS2D_TRY(from_cuda(launch_transpose(s, desc->in_dtype, x, xT, st)));
     const int RN = dt_rank + 2 * (int)s.N;
     SS2D_TRY(from_cuda(launch_xproj(s, desc->in_dtype, x, xT, x_proj_weight, RN, x_dbl, st)));
+    const bool materialise = dt_rank > kProjRNarrow;
+    if (materialise) SS2D_TRY(from_cuda(launch_dtproj(s, desc->in_dtype, x_dbl, dt_proj_weight, dt_rank, RN, delta, st)));
     ScanFwdArgs a;
     a.u = x;
     a.uT = xT;
-    a.delta = nullptr;
+    a.delta = materialise ? delta : nullptr;
     a.A = A;
     a.Bm = nullptr;
     a.Cm = nullptr;

@@ -32,7 +32,8 @@ cudaError_t launch_cross_merge(const LaunchShape &s, ss2d_dtype_t din, ss2d_dtyp
 //                x, delta, B, C in natural order, the reverse direction backwards.
 //  kModeImgProj -- kModeImg with the producer fused in: B, C and the low-rank dt rows come from
 //                the per-path x_proj output, dt = softplus(W_dt . x_dbl[:R] + bias) in-kernel;
-//                kModeImgProjWide is the same for ranks above kProjRNarrow.
+//  kModeImgProjWide -- B, C from the x_proj output, delta materialised (ranks above
+//                kProjRNarrow, where R multiply-adds per step cost more than reading delta).
 enum ScanMode { kModeSeq = 0, kModeImg = 1, kModeBidir = 2, kModeImgProj = 3, kModeImgProjWide = 4 };
 constexpr int kProjRNarrow = 8;  // dt ranks up to this use the narrow (smaller) projection kernels
 constexpr int kProjRMax = 32;    // largest dt_rank the fused projection takes
@@ -79,6 +80,9 @@ cudaError_t launch_cross_scan_table(const LaunchShape &s, ss2d_dtype_t dt, const
 cudaError_t launch_cross_merge_table(const LaunchShape &s, ss2d_dtype_t din, ss2d_dtype_t dout, const void *ys,
                                      const int32_t *tab, void *y, cudaStream_t stream);
 
+// delta[b, k*D + d, l] = sum_r Wdt[k*D + d, r] xdbl[b, k, r, l], in_dtype
+cudaError_t launch_dtproj(const LaunchShape &s, ss2d_dtype_t dt, const void *xdbl, const float *Wdt, int R, int RN,
+                          void *delta, cudaStream_t stream);
 // Per-path x_proj: xdbl[b, k, c, l] = sum_d W[k, c, d] u_k[d, l] (u_0/u_2 from x, u_1/u_3 from xT),
 // in each path's step order, RN = R + 2N <= 64 rows.
 cudaError_t launch_xproj(const LaunchShape &s, ss2d_dtype_t dt, const void *x, const void *xT, const float *W,

@@ -236,14 +236,15 @@ __host__ __device__ constexpr bool a2_in_smem() {
 // dt ranks the projection modes' shared arrays are sized for
 template <int MODE>
 __host__ __device__ constexpr int proj_rank_bucket() {
-    return MODE == kModeImgProj ? kProjRNarrow : (MODE == kModeImgProjWide ? kProjRMax : 1);
+    return MODE == kModeImgProj ? kProjRNarrow : 1;
 }
 
 template <int NS, typename Tin, typename Tout, int MODE, int PASS, bool VEC, bool REV>
 __device__ __forceinline__ void scan_fwd_body(const FwdParams &p, FwdStage<Tin, NS> (&stage)[2],
                                               float (&A2s)[a2_in_smem<Tin>() ? NS : 1][kWarp],
                                               Tin (*dts)[proj_rank_bucket<MODE>()][kLC], float (*wsm)[kWarp]) {
-    constexpr bool PROJ = MODE == kModeImgProj || MODE == kModeImgProjWide;
+    constexpr bool PROJ = MODE == kModeImgProj || MODE == kModeImgProjWide;  // B, C from x_dbl
+    constexpr bool DTIN = MODE == kModeImgProj;  // dt projected here, not read from delta
     constexpr int RB = proj_rank_bucket<MODE>();
     constexpr bool IMG = MODE == kModeImg || PROJ, BIDIR = MODE == kModeBidir, SEQ = MODE == kModeSeq;
     constexpr bool kA2Smem = a2_in_smem<Tin>();
@@ -272,7 +273,7 @@ __device__ __forceinline__ void scan_fwd_body(const FwdParams &p, FwdStage<Tin, 
             A2r[n] = a2v;
         h[n] = 0.f;
     }
-    if (PROJ) {  // this lane's row of dt_proj, kept in shared memory (lanes fastest)
+    if (DTIN) {  // this lane's row of dt_proj, kept in shared memory (lanes fastest)
 #pragma unroll
         for (int r = 0; r < RB; ++r) wsm[r][t] = (active && r < p.R) ? p.Wdt[c * p.R + r] : 0.f;
     }
@@ -305,7 +306,7 @@ __device__ __forceinline__ void scan_fwd_body(const FwdParams &p, FwdStage<Tin, 
         urev = false;
     }
     const Tin *drow =
-        PROJ ? nullptr : static_cast<const Tin *>(p.delta) + (BIDIR ? b * D + (active ? d : 0) : b * C4 + c) * L;
+        DTIN ? nullptr : static_cast<const Tin *>(p.delta) + (BIDIR ? b * D + (active ? d : 0) : b * C4 + c) * L;
     const int64_t grp = BIDIR ? b : b * kPaths + k;  // the B/C group of this (b, k)
     // projection mode: the group's x_proj outputs are R dt rows, then N rows of B, then N of C
     const Tin *DTk = PROJ ? static_cast<const Tin *>(p.xdbl) + grp * (p.R + 2 * N) * L : nullptr;
@@ -327,8 +328,8 @@ __device__ __forceinline__ void scan_fwd_body(const FwdParams &p, FwdStage<Tin, 
     }
     __syncwarp();
 
-    stage_chunk<NS, VEC, REV, PROJ, RB>(stage[0], Bk, Ck, N, L, urow, urev, drow, active, lbeg,
-                                    (int)min((int64_t)kLC, nloc), PROJ ? dts[0] : nullptr, DTk, p.R);
+    stage_chunk<NS, VEC, REV, DTIN, RB>(stage[0], Bk, Ck, N, L, urow, urev, drow, active, lbeg,
+                                    (int)min((int64_t)kLC, nloc), DTIN ? dts[0] : nullptr, DTk, p.R);
     cp_async_commit();
 
     for (int ch = 0; ch < nchunk; ++ch) {
@@ -337,8 +338,8 @@ __device__ __forceinline__ void scan_fwd_body(const FwdParams &p, FwdStage<Tin, 
         const int buf = ch & 1;
         if (ch + 1 < nchunk) {
             const int64_t nbeg = cbeg + kLC;
-            stage_chunk<NS, VEC, REV, PROJ, RB>(stage[buf ^ 1], Bk, Ck, N, L, urow, urev, drow, active, nbeg,
-                                            (int)min((int64_t)kLC, lend - nbeg), PROJ ? dts[buf ^ 1] : nullptr, DTk,
+            stage_chunk<NS, VEC, REV, DTIN, RB>(stage[buf ^ 1], Bk, Ck, N, L, urow, urev, drow, active, nbeg,
+                                            (int)min((int64_t)kLC, lend - nbeg), DTIN ? dts[buf ^ 1] : nullptr, DTk,
                                             p.R);
             cp_async_commit();
             cp_async_wait<1>();
@@ -354,7 +355,7 @@ __device__ __forceinline__ void scan_fwd_body(const FwdParams &p, FwdStage<Tin, 
                 const int nvalid = (int)min((int64_t)kG, lend - l0);
                 float uv[kG], dv[kG];
                 {  // slots hold 4-step groups in every staging form (see stage_chunk)
-                    if (PROJ) {  // delta = dt_proj . x_dbl[:R] for the four steps
+                    if (DTIN) {  // delta = dt_proj . x_dbl[:R] for the four steps
                         float2 a01 = make_float2(0.f, 0.f), a23 = make_float2(0.f, 0.f);
 #pragma unroll
                         for (int r = 0; r < RB; ++r) {
@@ -524,7 +525,7 @@ template <int NS, typename Tin, typename Tout, int MODE, int PASS, bool VEC>
 __global__ void __launch_bounds__(kWarp, SS2D_FWD_MIN_BLOCKS) scan_fwd_kernel(const FwdParams p) {
     __shared__ __align__(16) FwdStage<Tin, NS> stage[2];
     __shared__ float A2s[a2_in_smem<Tin>() ? NS : 1][kWarp];
-    if constexpr (MODE == kModeImgProj || MODE == kModeImgProjWide) {  // dt rows, each lane's dt_proj row
+    if constexpr (MODE == kModeImgProj) {  // dt rows, each lane's dt_proj row
         __shared__ __align__(16) Tin dts[2][proj_rank_bucket<MODE>()][kLC];
         __shared__ float wsm[proj_rank_bucket<MODE>()][kWarp];
         scan_fwd_body<NS, Tin, Tout, MODE, PASS, VEC, false>(p, stage, A2s, dts, wsm);
@@ -635,7 +636,7 @@ cudaError_t launch_scan_fwd(const LaunchShape &s, const ScanFwdArgs &a, void *wo
                    : launch_types<__nv_bfloat16, float, kModeBidir, false>(p, stream);
     }
     if (a.from_image && a.xdbl) {  // producer fused: fp32 per-path outputs for the merge
-        if (a.R <= kProjRNarrow) {
+        if (!a.delta) {  // dt projected in the scan
             if (a.in_dtype == SS2D_F32)
                 return vec ? launch_types<float, float, kModeImgProj, true>(p, stream)
                            : launch_types<float, float, kModeImgProj, false>(p, stream);

@@ -154,7 +154,8 @@ def test_path_table_argument_errors(lib):
 
 def test_forward_proj_argument_errors(lib):
     f = lib.ss2d_forward_proj
-    ws = lib.ss2d_workspace_bytes(_d(), ss.OP_FORWARD)
+    ws = lib.ss2d_workspace_bytes(_d(), ss.OP_FORWARD_PROJ)
+    assert ws > lib.ss2d_workspace_bytes(_d(), ss.OP_FORWARD)
     w = [A16, A16, A16, A16]  # x, x_proj_weight, dt_proj_weight, dt_proj_bias
     assert f(_d(), 0, *w, A16, None, 1, B16, B16, None, A16, ws, None) == ERR_SHAPE   # dt_rank 0
     assert f(_d(), 33, *w, A16, None, 1, B16, B16, None, A16, ws, None) == ERR_SHAPE  # dt_rank > 32
