@@ -520,14 +520,18 @@ def run_gpu(args, world, rank, local):
                    + (f" ({args.paths} paths)" if args.paths != "cross" else "")
                    + (" (with the per-path x_proj/dt_proj producer)" if args.proj else ""),
                    "l2": f"inputs {alg_bytes / 1e9:.2f} GB > 126 MB L2, no flush needed"},
-        "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": achieved_gbs / hbm_peak, "traffic": traffic,
+        # the dominant (scan) kernel is bound by its exponentials on the SFU: that is the roofline;
+        # the HBM view the metric names is reported beside it
+        "roofline": {"bound": "alu", "achieved": sfu_achieved, "peak": sfu_peak, "unit": "G ex2/s",
+                     "frac": sfu_achieved / sfu_peak, "traffic": traffic,
                      "kernel": f"launch {dom} of {launches_per_step} per step", "kernel_ms": dom_ms,
-                     "algorithmic_bytes_per_update": bytes_per_update,
-                     "peak_source": f"{peaks.get('source')} hbm_gbs (b.copy_ burst)"},
-        "sfu_roofline": {"bound": "alu", "achieved": sfu_achieved, "peak": sfu_peak, "unit": "G ex2/s",
-                         "frac": sfu_achieved / sfu_peak,
-                         "peak_derivation": "16 MUFU.EX2/clk/SM x 148 SMs x max SM clock"},
+                     "algorithmic_ex2_per_update": 1,
+                     "peak_source": "derived: 16 MUFU.EX2 per clock per SM (measured on this pool) x 148 SMs x "
+                                    f"{sm_max:.0f} MHz maximum SM clock"},
+        "hbm_roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": achieved_gbs / hbm_peak, "traffic": traffic,
+                         "algorithmic_bytes_per_update": bytes_per_update,
+                         "peak_source": f"{peaks.get('source')} hbm_gbs (b.copy_ burst)"},
         "kernel_ms": per_kernel,
         "gpu_launches": gpu_launches,
         "clocks": clocks,
