@@ -192,6 +192,32 @@ def ss2d_forward_proj(x, x_proj_weight, dt_proj_weight, dt_proj_bias, A, D=None,
     return ss2d_forward(x, delta, A, Bm, Cm, D, dt_proj_bias, delta_softplus)
 
 
+def ss2d_backward_proj(x, x_proj_weight, dt_proj_weight, dt_proj_bias, A, D, delta_softplus, dy):
+    """Gradients of ss2d_forward_proj, per path as MambaInnerFn.backward ("vision mamba-yolov8",
+    section 2) computes them: the scan's backward on the projected inputs, then
+    dx_dbl[:R] = dt_proj.weight^T @ ddelta, dx_dbl[R:] = (dB, dC),
+    d dt_proj.weight = ddelta @ x_dbl[:R]^T, d x_proj.weight = dx_dbl @ u^T and
+    du += x_proj.weight^T @ dx_dbl, with u and du taken along each path (CrossScan / CrossMerge).
+    Returns dict dx, dx_proj_weight, ddt_proj_weight, ddt_proj_bias, dA, dD."""
+    x, Wx, Wdt, dy = _f64(x), _f64(x_proj_weight), _f64(dt_proj_weight), _f64(dy)
+    D, bias, A = _f64(D), _f64(dt_proj_bias), _f64(A)
+    Bn, Dn, H, W = x.shape
+    R = Wdt.shape[2]
+    N = (Wx.shape[1] - R) // 2
+    L = H * W
+    delta, Bm, Cm, x_dbl = path_projections(x, Wx, Wdt)
+    g = ss2d_backward(x, delta, A, Bm, Cm, D, bias, delta_softplus, dy)
+    ddelta = g["ddelta"].reshape(Bn, K_PATHS, Dn, L)
+    dx_dbl = np.concatenate([np.einsum("kdr,bkdl->bkrl", Wdt, ddelta), g["dB"], g["dC"]], axis=2)
+    ddt_proj_weight = np.einsum("bkdl,bkrl->kdr", ddelta, x_dbl[:, :, :R])
+    xs = cross_scan(x)                                              # u along every path
+    dx_proj_weight = np.einsum("bkcl,bkdl->kcd", dx_dbl, xs)
+    dus = np.einsum("kcd,bkcl->bkdl", Wx, dx_dbl)                   # du along every path
+    dx = g["dx"] + cross_merge(dus, H, W)
+    return dict(dx=dx, dx_proj_weight=dx_proj_weight, ddt_proj_weight=ddt_proj_weight,
+                ddt_proj_bias=g["ddelta_bias"], dA=g["dA"], dD=g["dD"])
+
+
 # ---------------------------------------------------------------- path sets
 
 def cross_paths(H: int, W: int):

@@ -555,6 +555,31 @@ def test_bimamba_backward_matches_central_differences(oracle):
             assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (name, i, fd, an)
 
 
+def test_projection_backward_matches_central_differences(oracle):
+    p = _proj_problem(74, Bn=1, Dn=3, H=3, W=4, N=3, R=2)
+    rng = _rng(75)
+    dy = rng.standard_normal(p["x"].shape)
+    g = oracle.ss2d_backward_proj(p["x"], p["Wx"], p["Wdt"], p["bias"], p["A"], p["D"], True, dy)
+
+    def loss():
+        return float(np.sum(oracle.ss2d_forward_proj(p["x"], p["Wx"], p["Wdt"], p["bias"], p["A"], p["D"]) * dy))
+
+    names = dict(x="dx", Wx="dx_proj_weight", Wdt="ddt_proj_weight", bias="ddt_proj_bias", A="dA", D="dD")
+    for name, gname in names.items():
+        flat = p[name].reshape(-1)
+        for i in rng.choice(flat.size, size=min(flat.size, 8), replace=False):
+            theta = flat[i]
+            h = 1e-6 * max(1.0, abs(theta))
+            flat[i] = theta + h
+            lp = loss()
+            flat[i] = theta - h
+            lm = loss()
+            flat[i] = theta
+            fd = (lp - lm) / (2 * h)
+            an = g[gname].reshape(-1)[i]
+            assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (name, i, fd, an)
+
+
 # ------------------------------------------------------------ path tables
 
 def _golden_diagonals():
