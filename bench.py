@@ -23,7 +23,8 @@ silu(z)): a step is one bidirectional forward (plus its backward under `--backwa
 "Visual Mamba实战从零开始搭建图像分类模型附PyTorch代码" (section 3) instead of the cross scan.
 
 `--proj` times the fused forward with its producer: per-path x_proj, then the scan computing
-dt = softplus(dt_proj . x_dbl[:R] + bias) per step (MambaInnerFn.forward's projections).
+dt = softplus(dt_proj . x_dbl[:R] + bias) per step (MambaInnerFn.forward's projections);
+with `--backward` each step adds the backward through the scan and both projections.
 
 `--backward` adds the fused backward to every step; `--gate` times the scan in its
 sequence form instead, u (B, 4D, L) with the output gate out * silu(z) and the last
@@ -351,15 +352,27 @@ def run_gpu(args, world, rank, local):
     stream = torch.cuda.current_stream(dev)
 
     if args.proj:
-        R = inp["R"]
-        x_dbl = torch.empty((w.batch, 4, R + 2 * w.d_state, w.L), dtype=w.torch_dtype, device=dev)
         pargs = (inp["x"], inp["x_proj_weight"], inp["dt_proj_weight"], inp["dt_proj_bias"], inp["A"], inp["D"])
 
         npj = ss.workspace_bytes(w.batch, w.dim, w.height, w.width, w.d_state, ss.OP_FORWARD_PROJ, w.torch_dtype)
         wsp = torch.empty(max(npj, 1), dtype=torch.uint8, device=dev)
 
-        def step():
-            ss.ss2d_forward_proj(*pargs, True, out=y, workspace=wsp)
+        if args.backward:
+            gdy = torch.Generator(device=dev)
+            gdy.manual_seed(shard_seed(args.workload, rank) + 7000)
+            dy = torch.randn((w.batch, w.dim, w.height, w.width), generator=gdy, device=dev).to(w.torch_dtype)
+            nbp = ss.workspace_bytes(w.batch, w.dim, w.height, w.width, w.d_state, ss.OP_BACKWARD_PROJ,
+                                     w.torch_dtype)
+            wsbp = torch.empty(max(nbp, 1), dtype=torch.uint8, device=dev)
+
+            def step():
+                # forward keeping x_dbl and the chunk states, then the backward through scan and producer
+                _, xd, cs = ss.ss2d_forward_proj(*pargs, True, out=y, return_x_dbl=True, return_chunk_states=True,
+                                                 workspace=wsp)
+                ss.ss2d_backward_proj(*pargs, xd, dy, True, chunk_states=cs, workspace=wsbp)
+        else:
+            def step():
+                ss.ss2d_forward_proj(*pargs, True, out=y, workspace=wsp)
     elif bidir:
         y_seq = torch.empty((w.batch, w.dim, w.L), dtype=w.torch_dtype, device=dev)
         nbf = ss.workspace_bytes(w.batch, w.dim, 1, w.L, w.d_state, ss.OP_BIMAMBA_FORWARD, w.torch_dtype)
@@ -474,7 +487,7 @@ def run_gpu(args, world, rank, local):
     peaks = load_peaks()
     clocks = sampler.summary() if sampler else None
     # algorithmic bytes of the dominant kernel: the backward's when a backward runs in the step
-    if args.proj:
+    if args.proj and not args.backward:
         alg_bytes = proj_algorithmic_bytes(w, inp["R"])
     elif bidir:
         alg_bytes = bidir_algorithmic_bytes(w, args.backward)

@@ -90,7 +90,8 @@ typedef enum {
     SS2D_OP_BIMAMBA_BACKWARD = 5,
     SS2D_OP_FORWARD_TABLE = 6,
     SS2D_OP_BACKWARD_TABLE = 7,
-    SS2D_OP_FORWARD_PROJ = 8
+    SS2D_OP_FORWARD_PROJ = 8,
+    SS2D_OP_BACKWARD_PROJ = 9
 } ss2d_op_t;
 
 /* Path sets that ss2d_path_tables generates (paths 2 and 3 are always 0 and 1 walked backwards). */
@@ -265,6 +266,38 @@ SS2D_API ss2d_status_t ss2d_forward_proj(const ss2d_desc_t *desc, int dt_rank, c
                                          const float *dt_proj_bias, const float *A, const float *D,
                                          int delta_softplus, void *y, void *x_dbl, float *chunk_states,
                                          void *workspace, size_t workspace_bytes, ss2d_stream_t stream);
+
+/*
+ * Backward of ss2d_forward_proj: the gradients MambaInnerFn.backward ("vision mamba-yolov8",
+ * section 2) takes through the scan and then through the producer.  With ddelta, dB, dC the
+ * scan's gradients (as ss2d_backward gives them), per path k and token l:
+ *   dx_dbl[:R]        = dt_proj.weight^T ddelta,   dx_dbl[R:] = (dB, dC)
+ *   ddt_proj_weight   = sum over batch and tokens of ddelta (x) x_dbl[:R]
+ *   dx_proj_weight    = sum over batch and tokens of dx_dbl (x) u_k
+ *   dx                = the scan's du plus x_proj.weight^T dx_dbl, each merged along its path
+ * ddt_proj_bias is the scan's delta-bias gradient; dA and dD the scan's.  delta is made again
+ * from x_dbl (in in_dtype), B and C are read from x_dbl.  The sums over tokens and batch run
+ * in a fixed order (deterministic), in fp32.
+ * dt_rank, x, x_proj_weight, dt_proj_weight, dt_proj_bias, A, D, delta_softplus: as for
+ *                    ss2d_forward_proj
+ * x_dbl            : (B, 4, R + 2N, L) in_dtype, as ss2d_forward_proj wrote it
+ * chunk_states     : as ss2d_forward_proj wrote them, or NULL (recomputed)
+ * dy               : (B, D, H, W) out_dtype
+ * dx               : (B, D, H, W) in_dtype, written
+ * dx_proj_weight   : (4, R + 2N, D) fp32, written;  ddt_proj_weight: (4, D, R) fp32, written
+ * ddt_proj_bias    : (4D) fp32, written; NULL exactly when dt_proj_bias is NULL
+ * dA (4D, N) fp32, dD (4D) fp32 (NULL exactly when D is NULL): written
+ * workspace        : ss2d_workspace_bytes(desc, SS2D_OP_BACKWARD_PROJ) bytes (sized for the
+ *                    largest dt_rank, 32)
+ * Errors: SS2D_ERR_SHAPE for dt_rank outside [1, 32]; otherwise as for ss2d_backward.
+ */
+SS2D_API ss2d_status_t ss2d_backward_proj(const ss2d_desc_t *desc, int dt_rank, const void *x,
+                                          const float *x_proj_weight, const float *dt_proj_weight,
+                                          const float *dt_proj_bias, const float *A, const float *D,
+                                          int delta_softplus, const void *x_dbl, const float *chunk_states,
+                                          const void *dy, void *dx, float *dx_proj_weight,
+                                          float *ddt_proj_weight, float *ddt_proj_bias, float *dA, float *dD,
+                                          void *workspace, size_t workspace_bytes, ss2d_stream_t stream);
 
 /* ------------------------------------------------------------ path sets -- */
 

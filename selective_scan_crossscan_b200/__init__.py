@@ -36,7 +36,7 @@ __all__ = [
     "SS2DError", "cross_scan", "cross_merge", "selective_scan_fwd", "selective_scan_bwd", "selective_scan_fn",
     "SelectiveScanFunction", "ss2d_forward", "bimamba_forward", "bimamba_backward", "BiMambaFunction",
     "bimamba_scan", "path_tables", "cross_scan_table", "cross_merge_table", "ss2d_forward_table",
-    "ss2d_backward_table", "PATHS_CROSS", "PATHS_DIAGONAL", "ss2d_forward_proj",
+    "ss2d_backward_table", "PATHS_CROSS", "PATHS_DIAGONAL", "ss2d_forward_proj", "ss2d_backward_proj", "OP_BACKWARD_PROJ",
     "ss2d_backward", "SS2DFunction", "ss2d", "workspace_bytes", "chunk_states_elems", "launch_count",
     "library_path", "CHUNK_LEN", "trace_events",
 ]
@@ -50,7 +50,7 @@ _lib = None
 CHUNK_LEN = 16  # SS2D_CHUNK_LEN
 F32, BF16 = 0, 1
 OP_SELECTIVE_SCAN_BWD, OP_FORWARD, OP_BACKWARD, OP_BIMAMBA_FORWARD, OP_BIMAMBA_BACKWARD = 1, 2, 3, 4, 5
-OP_FORWARD_TABLE, OP_BACKWARD_TABLE, OP_FORWARD_PROJ = 6, 7, 8
+OP_FORWARD_TABLE, OP_BACKWARD_TABLE, OP_FORWARD_PROJ, OP_BACKWARD_PROJ = 6, 7, 8, 9
 PATHS_CROSS, PATHS_DIAGONAL = 0, 1
 _STATUS = {0: "SS2D_OK", 1: "SS2D_ERR_NULL", 2: "SS2D_ERR_SHAPE", 3: "SS2D_ERR_DTYPE", 4: "SS2D_ERR_ALIGN",
            5: "SS2D_ERR_WORKSPACE", 6: "SS2D_ERR_LAUNCH", 7: "SS2D_ERR_TIMEOUT", 8: "SS2D_ERR_DEVICE"}
@@ -99,6 +99,7 @@ def _load():
         lib.ss2d_bimamba_forward.argtypes = [D, P, P, P, P, P, P, P, P, i, P, P, P, sz, P]
         lib.ss2d_path_tables.argtypes = [D, i, P, P]
         lib.ss2d_forward_proj.argtypes = [D, i, P, P, P, P, P, P, i, P, P, P, P, sz, P]
+        lib.ss2d_backward_proj.argtypes = [D, i, P, P, P, P, P, P, i, P, P, P, P, P, P, P, P, P, P, sz, P]
         lib.ss2d_cross_scan_table.argtypes = [D, P, P, P, P]
         lib.ss2d_cross_merge_table.argtypes = [D, P, P, P, P]
         lib.ss2d_forward_table.argtypes = [D, P, P, P, P, P, P, P, P, i, P, P, P, sz, P]
@@ -109,7 +110,8 @@ def _load():
         for name in ("ss2d_cross_scan", "ss2d_cross_merge", "ss2d_selective_scan_fwd", "ss2d_selective_scan_bwd",
                      "ss2d_selective_scan_fwd_ex", "ss2d_selective_scan_bwd_ex", "ss2d_forward", "ss2d_backward",
                      "ss2d_bimamba_forward", "ss2d_bimamba_backward", "ss2d_path_tables", "ss2d_cross_scan_table",
-                     "ss2d_cross_merge_table", "ss2d_forward_table", "ss2d_backward_table", "ss2d_forward_proj"):
+                     "ss2d_cross_merge_table", "ss2d_forward_table", "ss2d_backward_table", "ss2d_forward_proj",
+                     "ss2d_backward_proj"):
             getattr(lib, name).restype = ctypes.c_int
         lib.ss2d_workspace_bytes.argtypes = [D, i]
         lib.ss2d_workspace_bytes.restype = sz
@@ -674,3 +676,42 @@ def ss2d_forward_proj(x, x_proj_weight, dt_proj_weight, dt_proj_bias, A, D=None,
     _check(st, "ss2d_forward_proj")
     extra = ([x_dbl] if return_x_dbl else []) + ([cs] if return_chunk_states else [])
     return (out, *extra) if extra else out
+
+
+def ss2d_backward_proj(x, x_proj_weight, dt_proj_weight, dt_proj_bias, A, D, x_dbl, dy, delta_softplus=True,
+                       chunk_states=None, workspace=None):
+    """Backward of ss2d_forward_proj (MambaInnerFn.backward's path through the scan and the producer).
+    x_dbl is the forward's (Bn, 4, R+2N, L) output; dy (Bn, D, H, W).  Returns a dict with dx,
+    dx_proj_weight (4, R+2N, D), ddt_proj_weight (4, D, R), ddt_proj_bias (4D, or None without a bias),
+    dA (4D, N) and dD (4D, or None without D); the weight, bias, A and D gradients are fp32."""
+    x = _c(x)
+    Wx = _c(x_proj_weight, torch.float32)
+    Wdt = _c(dt_proj_weight, torch.float32)
+    A, D, bias = _params(A, D, dt_proj_bias)
+    Bn, Dn, H, W = x.shape
+    N = A.shape[1]
+    R = Wdt.shape[2]
+    if Wx.shape != (4, R + 2 * N, Dn) or Wdt.shape != (4, Dn, R):
+        raise ValueError("ss2d_backward_proj: x_proj_weight must be (4, R+2N, D) and dt_proj_weight (4, D, R)")
+    x_dbl = _c(x_dbl, x.dtype)
+    if x_dbl.shape != (Bn, 4, R + 2 * N, H * W):
+        raise ValueError("ss2d_backward_proj: x_dbl must be (Bn, 4, R+2N, H*W) in x's dtype")
+    dy = _c(dy)
+    cs = _c(chunk_states, torch.float32) if chunk_states is not None else None
+    f32 = dict(dtype=torch.float32, device=x.device)
+    dx = torch.empty_like(x)
+    dWx = torch.empty((4, R + 2 * N, Dn), **f32)
+    dWdt = torch.empty((4, Dn, R), **f32)
+    dbias = torch.empty((4 * Dn,), **f32) if bias is not None else None
+    dA = torch.empty((4 * Dn, N), **f32)
+    dD = torch.empty((4 * Dn,), **f32) if D is not None else None
+    d = _desc(Bn, Dn, H, W, N, x.dtype, dy.dtype)
+    lib = _load()
+    nbytes = int(lib.ss2d_workspace_bytes(ctypes.byref(d), OP_BACKWARD_PROJ))
+    if workspace is None or workspace.numel() < nbytes:
+        workspace = _workspace(nbytes, x.device)
+    st = lib.ss2d_backward_proj(ctypes.byref(d), int(R), _p(x), _p(Wx), _p(Wdt), _p(bias), _p(A), _p(D),
+                                int(bool(delta_softplus)), _p(x_dbl), _p(cs), _p(dy), _p(dx), _p(dWx), _p(dWdt),
+                                _p(dbias), _p(dA), _p(dD), _p(workspace), nbytes, _stream(x))
+    _check(st, "ss2d_backward_proj")
+    return dict(dx=dx, dx_proj_weight=dWx, ddt_proj_weight=dWdt, ddt_proj_bias=dbias, dA=dA, dD=dD)

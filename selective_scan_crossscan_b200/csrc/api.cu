@@ -134,6 +134,18 @@ static size_t table_bwd_ws_bytes(const LaunchShape &s, ss2d_dtype_t in, ss2d_dty
            2 * round64((size_t)s.B * s.D * s.L * elem_size(in)) + 2 * round64((size_t)s.B * s.D * s.L * elem_size(out)) +
            round64(scan_bwd_workspace_bytes(s));
 }
+// producer backward workspace (sized for the largest dt rank):
+// [fp32 per-path du (B,4D,L)] [transposed x] [transposed dy] [delta] [ddelta] [B, C, dB, dC (B,4,N,L) each]
+// [fp32 dx_dbl (B,4,RN,L)] [fp32 weight-gradient partials] [scan backward workspace]
+static size_t proj_bwd_ws_bytes(const LaunchShape &s, ss2d_dtype_t in, ss2d_dtype_t out) {
+    const size_t seq = (size_t)s.B * kPaths * s.D * s.L, img = (size_t)s.B * s.D * s.L;
+    const size_t bc = (size_t)s.B * kPaths * s.N * s.L, rn = (size_t)kProjRMax + 2 * s.N;
+    return round64(seq * sizeof(float)) + round64(img * elem_size(in)) + round64(img * elem_size(out)) +
+           2 * round64(seq * elem_size(in)) + 4 * round64(bc * elem_size(in)) +
+           round64((size_t)s.B * kPaths * rn * s.L * sizeof(float)) +
+           round64((size_t)kPaths * s.B * proj_bwd_chunks(s) * rn * s.D * sizeof(float)) +
+           round64(scan_bwd_workspace_bytes(s));
+}
 static ss2d_status_t check_table_shape(const ss2d_desc_t *desc) {
     return desc->height * desc->width < ((int64_t)1 << 31) ? SS2D_OK : SS2D_ERR_SHAPE;
 }
@@ -190,6 +202,7 @@ size_t ss2d_workspace_bytes(const ss2d_desc_t *desc, int op) {
         case SS2D_OP_FORWARD_PROJ:
             return fwd_ws_bytes(s, desc->in_dtype) + round64((size_t)s.B * kPaths * s.D * s.L * elem_size(desc->in_dtype));
         case SS2D_OP_BACKWARD_TABLE: return table_bwd_ws_bytes(s, desc->in_dtype, desc->out_dtype);
+        case SS2D_OP_BACKWARD_PROJ: return proj_bwd_ws_bytes(s, desc->in_dtype, desc->out_dtype);
         default: return (size_t)-1;
     }
 }
@@ -381,6 +394,102 @@ ss2d_status_t ss2d_forward_proj(const ss2d_desc_t *desc, int dt_rank, const void
     a.out_dtype = SS2D_F32;
     SS2D_TRY(from_cuda(launch_scan_fwd(s, a, seg, st)));
     return from_cuda(launch_cross_merge(s, SS2D_F32, desc->out_dtype, ys, y, st));
+}
+
+ss2d_status_t ss2d_backward_proj(const ss2d_desc_t *desc, int dt_rank, const void *x, const float *x_proj_weight,
+                                 const float *dt_proj_weight, const float *dt_proj_bias, const float *A,
+                                 const float *D, int delta_softplus, const void *x_dbl, const float *chunk_states,
+                                 const void *dy, void *dx, float *dx_proj_weight, float *ddt_proj_weight,
+                                 float *ddt_proj_bias, float *dA, float *dD, void *workspace, size_t workspace_bytes,
+                                 ss2d_stream_t stream) {
+    SS2D_TRY(check_desc(desc));
+    if (dt_rank < 1 || dt_rank > kProjRMax) return SS2D_ERR_SHAPE;
+    SS2D_TRY(need(x));
+    SS2D_TRY(need(x_proj_weight));
+    SS2D_TRY(need(dt_proj_weight));
+    SS2D_TRY(optional(dt_proj_bias));
+    SS2D_TRY(need(A));
+    SS2D_TRY(optional(D));
+    SS2D_TRY(need(x_dbl));
+    SS2D_TRY(optional(chunk_states));
+    SS2D_TRY(need(dy));
+    SS2D_TRY(need(dx));
+    SS2D_TRY(need(dx_proj_weight));
+    SS2D_TRY(need(ddt_proj_weight));
+    SS2D_TRY(need(dA));
+    if ((D == nullptr) != (dD == nullptr)) return SS2D_ERR_NULL;
+    if ((dt_proj_bias == nullptr) != (ddt_proj_bias == nullptr)) return SS2D_ERR_NULL;
+    SS2D_TRY(optional(dD));
+    SS2D_TRY(optional(ddt_proj_bias));
+    const LaunchShape s = shape_of(desc);
+    const ss2d_dtype_t in = desc->in_dtype;
+    if (!workspace || workspace_bytes < proj_bwd_ws_bytes(s, in, desc->out_dtype)) return SS2D_ERR_WORKSPACE;
+    SS2D_TRY(optional(workspace));
+    SS2D_TRY(check_device());
+    const int R = dt_rank, RN = R + 2 * (int)s.N;
+    const size_t seq = (size_t)s.B * kPaths * s.D * s.L, img = (size_t)s.B * s.D * s.L;
+    const size_t bc = (size_t)s.B * kPaths * s.N * s.L, es = elem_size(in);
+    unsigned char *w = static_cast<unsigned char *>(workspace);
+    auto take = [&w](size_t bytes) {
+        void *p = w;
+        w += round64(bytes);
+        return p;
+    };
+    float *du_seq = static_cast<float *>(take(seq * sizeof(float)));
+    void *xT = take(img * es);
+    void *dyT = take(img * elem_size(desc->out_dtype));
+    void *delta = take(seq * es);
+    void *ddelta = take(seq * es);
+    void *Bm = take(bc * es);
+    void *Cm = take(bc * es);
+    void *dBm = take(bc * es);
+    void *dCm = take(bc * es);
+    float *dxdbl = static_cast<float *>(take((size_t)s.B * kPaths * (kProjRMax + 2 * s.N) * s.L * sizeof(float)));
+    float *part = static_cast<float *>(
+        take((size_t)kPaths * s.B * proj_bwd_chunks(s) * (kProjRMax + 2 * s.N) * s.D * sizeof(float)));
+    void *inner = w;
+    cudaStream_t st = (cudaStream_t)stream;
+    SS2D_TRY(from_cuda(launch_transpose(s, in, x, xT, st)));
+    SS2D_TRY(from_cuda(launch_transpose(s, desc->out_dtype, dy, dyT, st)));
+    SS2D_TRY(from_cuda(launch_dtproj(s, in, x_dbl, dt_proj_weight, R, RN, delta, st)));
+    // B and C: rows [R, R+N) and [R+N, R+2N) of every (b, k) block of x_dbl
+    const size_t row = (size_t)s.N * s.L * es, pitch = (size_t)RN * s.L * es, blocks = (size_t)s.B * kPaths;
+    const unsigned char *xd = static_cast<const unsigned char *>(x_dbl);
+    SS2D_TRY(from_cuda(cudaMemcpy2DAsync(Bm, row, xd + (size_t)R * s.L * es, pitch, row, blocks,
+                                         cudaMemcpyDeviceToDevice, st)));
+    SS2D_TRY(from_cuda(cudaMemcpy2DAsync(Cm, row, xd + (size_t)(R + s.N) * s.L * es, pitch, row, blocks,
+                                         cudaMemcpyDeviceToDevice, st)));
+    ScanBwdArgs a;
+    a.u = x;
+    a.uT = xT;
+    a.doutT = dyT;
+    a.delta = delta;
+    a.A = A;
+    a.Bm = Bm;
+    a.Cm = Cm;
+    a.Dv = D;
+    a.bias = dt_proj_bias;
+    a.softplus = delta_softplus != 0;
+    a.dout = dy;
+    a.chunk_states = chunk_states;
+    a.du = du_seq;
+    a.ddelta = ddelta;
+    a.dA = dA;
+    a.dBm = dBm;
+    a.dCm = dCm;
+    a.dD = dD;
+    a.dbias = ddt_proj_bias;
+    a.from_image = true;
+    a.in_dtype = in;
+    a.out_dtype = desc->out_dtype;
+    SS2D_TRY(from_cuda(launch_scan_bwd(s, a, inner, scan_bwd_workspace_bytes(s), st)));
+    SS2D_TRY(from_cuda(launch_proj_bwd_dtlow(s, in, ddelta, dt_proj_weight, R, RN, dxdbl, st)));
+    SS2D_TRY(from_cuda(launch_proj_bwd_copy_rows(s, in, dBm, (int)s.N, RN, R, dxdbl, st)));
+    SS2D_TRY(from_cuda(launch_proj_bwd_copy_rows(s, in, dCm, (int)s.N, RN, R + (int)s.N, dxdbl, st)));
+    SS2D_TRY(from_cuda(launch_proj_bwd_dwdt(s, in, ddelta, x_dbl, R, RN, part, ddt_proj_weight, st)));
+    SS2D_TRY(from_cuda(launch_proj_bwd_dwx(s, in, dxdbl, x, xT, RN, part, dx_proj_weight, st)));
+    SS2D_TRY(from_cuda(launch_proj_bwd_du(s, dxdbl, x_proj_weight, RN, du_seq, st)));
+    return from_cuda(launch_cross_merge(s, SS2D_F32, in, du_seq, dx, st));
 }
 
 ss2d_status_t ss2d_path_tables(const ss2d_desc_t *desc, int paths, int32_t *tables, ss2d_stream_t stream) {

@@ -88,6 +88,26 @@ cudaError_t launch_dtproj(const LaunchShape &s, ss2d_dtype_t dt, const void *xdb
 cudaError_t launch_xproj(const LaunchShape &s, ss2d_dtype_t dt, const void *x, const void *xT, const float *W,
                          int RN, void *xdbl, cudaStream_t stream);
 
+// Producer backward (proj_bwd.cu).  dx_dbl is fp32 (B, 4, RN, L) in each path's step order.
+constexpr int64_t kProjTokenChunk = 1024;  // tokens one CTA of a weight-gradient reduction sums
+int64_t proj_bwd_chunks(const LaunchShape &s);
+// dx_dbl[b, k, r, l] = sum_d Wdt[k*D + d, r] ddelta[b, k*D + d, l] for r < R
+cudaError_t launch_proj_bwd_dtlow(const LaunchShape &s, ss2d_dtype_t dt, const void *ddelta, const float *Wdt, int R,
+                                  int RN, float *dxdbl, cudaStream_t stream);
+// dx_dbl[b, k, off + r, l] = src[b, k, r, l], r < rows
+cudaError_t launch_proj_bwd_copy_rows(const LaunchShape &s, ss2d_dtype_t dt, const void *src, int rows, int RN,
+                                      int off, float *dxdbl, cudaStream_t stream);
+// du_seq[b, k*D + d, l] += sum_c Wx[k, c, d] dx_dbl[b, k, c, l]
+cudaError_t launch_proj_bwd_du(const LaunchShape &s, const float *dxdbl, const float *Wx, int RN, float *du_seq,
+                               cudaStream_t stream);
+// dWdt[k*D + d, r] = sum_{b,l} ddelta[b, k*D + d, l] xdbl[b, k, r, l]; part holds
+// 4 * B * proj_bwd_chunks(s) * D * R floats
+cudaError_t launch_proj_bwd_dwdt(const LaunchShape &s, ss2d_dtype_t dt, const void *ddelta, const void *xdbl, int R,
+                                 int RN, float *part, float *dWdt, cudaStream_t stream);
+// dWx[k, c, d] = sum_{b,l} dx_dbl[b, k, c, l] u_k[b, d, l]; part holds 4 * B * proj_bwd_chunks(s) * RN * D floats
+cudaError_t launch_proj_bwd_dwx(const LaunchShape &s, ss2d_dtype_t dt, const float *dxdbl, const void *x,
+                                const void *xT, int RN, float *part, float *dWx, cudaStream_t stream);
+
 // Bidirectional scan: out[b, d, m] = (two[b, 0, d, m] + two[b, 1, d, m]) * (z ? silu(z[b, d, m]) : 1),
 // two (B, 2, D, L) fp32, z (B, D, L) z_dtype or null, out (B, D, L) out_dtype.
 cudaError_t launch_bidir_sum(const float *two, const void *z, ss2d_dtype_t z_dtype, void *out,

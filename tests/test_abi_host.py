@@ -163,6 +163,21 @@ def test_forward_proj_argument_errors(lib):
     assert f(_d(), 2, *w, A16, None, 1, B16, B16, None, A16, ws - 1, None) == ERR_WORKSPACE
 
 
+def test_backward_proj_argument_errors(lib):
+    f = lib.ss2d_backward_proj
+    ws = lib.ss2d_workspace_bytes(_d(), ss.OP_BACKWARD_PROJ)
+    assert ws > lib.ss2d_workspace_bytes(_d(), ss.OP_BACKWARD)
+    w = [A16, A16, A16, A16, A16, A16]  # x, x_proj_weight, dt_proj_weight, dt_proj_bias, A, D
+    g = [B16, B16, B16, B16, B16, B16]  # dx, dx_proj_weight, ddt_proj_weight, ddt_proj_bias, dA, dD
+    ok = (1, A16, None, A16)            # softplus, x_dbl, chunk_states, dy
+    assert f(_d(), 0, *w, *ok, *g, A16, ws, None) == ERR_SHAPE    # dt_rank 0
+    assert f(_d(), 33, *w, *ok, *g, A16, ws, None) == ERR_SHAPE   # dt_rank > 32
+    assert f(_d(), 2, *w, 1, None, None, A16, *g, A16, ws, None) == ERR_NULL  # x_dbl
+    assert f(_d(), 2, *w, *ok, B16, B16, B16, None, B16, B16, A16, ws, None) == ERR_NULL  # bias without its grad
+    assert f(_d(), 2, *w[:5], None, *ok, *g, A16, ws, None) == ERR_NULL  # dD without D
+    assert f(_d(), 2, *w, *ok, *g, A16, ws - 1, None) == ERR_WORKSPACE
+
+
 def test_valid_call_without_gpu_reports_device_error(lib):
     import torch
     if torch.cuda.is_available():

@@ -610,6 +610,70 @@ def test_ss2d_forward_proj_bf16_and_full_stage1_sampled():
         assert_fwd_close(y[bi:bi + 1], ref, f"y[{bi}]")
 
 
+PROJ_BWD_CASES = [(1, 8, 8, 8, 4), (2, 70, 5, 9, 16), (2, 6, 1, 1, 16), (1, 40, 33, 35, 8), (1, 192, 14, 14, 16),
+                  (1, 512, 4, 6, 16)]
+
+
+@pytest.mark.parametrize("case", PROJ_BWD_CASES)
+def test_ss2d_backward_proj_parity(case):
+    w, inp = _proj_case(*case, seed=54)
+    d = _dev({k: v for k, v in inp.items() if k != "R"})
+    y, x_dbl = ss.ss2d_forward_proj(d["x"], d["x_proj_weight"], d["dt_proj_weight"], d["dt_proj_bias"], d["A"],
+                                    d["D"], True, return_x_dbl=True)
+    g = torch.Generator().manual_seed(55)
+    dy_np = torch.randn(tuple(y.shape), generator=g, dtype=torch.float32).double().numpy()
+    got = ss.ss2d_backward_proj(d["x"], d["x_proj_weight"], d["dt_proj_weight"], d["dt_proj_bias"], d["A"], d["D"],
+                                x_dbl, torch.as_tensor(dy_np, dtype=torch.float32, device="cuda"), True)
+    ref = oracle.ss2d_backward_proj(inp["x"], inp["x_proj_weight"], inp["dt_proj_weight"], inp["dt_proj_bias"],
+                                    inp["A"], inp["D"], True, dy_np)
+    for name in ("dx", "dx_proj_weight", "ddt_proj_weight", "ddt_proj_bias", "dA", "dD"):
+        assert_rel_l2(got[name], ref[name], GRAD_TOL, f"{case} {name}")
+
+
+def test_ss2d_backward_proj_wide_rank_bf16_and_chunk_states():
+    # dt rank 24 (d_model 384), more tokens than one weight-gradient chunk, forward chunk states reused
+    w, inp = _proj_case(1, 768, 36, 30, 16, seed=56)
+    d = _dev({k: v for k, v in inp.items() if k != "R"})
+    y, x_dbl, cs = ss.ss2d_forward_proj(d["x"], d["x_proj_weight"], d["dt_proj_weight"], d["dt_proj_bias"],
+                                        d["A"], d["D"], True, return_x_dbl=True, return_chunk_states=True)
+    dy = torch.randn(y.shape, generator=torch.Generator(device="cuda").manual_seed(57), device="cuda")
+    a = ss.ss2d_backward_proj(d["x"], d["x_proj_weight"], d["dt_proj_weight"], d["dt_proj_bias"], d["A"], d["D"],
+                              x_dbl, dy, True)
+    b = ss.ss2d_backward_proj(d["x"], d["x_proj_weight"], d["dt_proj_weight"], d["dt_proj_bias"], d["A"], d["D"],
+                              x_dbl, dy, True, chunk_states=cs)
+    for k in a:
+        torch.testing.assert_close(a[k], b[k], rtol=1e-5, atol=1e-6)
+    ref = oracle.ss2d_backward_proj(inp["x"], inp["x_proj_weight"], inp["dt_proj_weight"], inp["dt_proj_bias"],
+                                    inp["A"], inp["D"], True, dy.double().cpu().numpy())
+    for name in ("dx", "dx_proj_weight", "ddt_proj_weight", "ddt_proj_bias", "dA", "dD"):
+        assert_rel_l2(a[name], ref[name], GRAD_TOL, name)
+    # bf16 activations: relative L2 against the oracle on the bf16-rounded inputs
+    w, inp = _proj_case(2, 16, 12, 12, 16, dtype="bf16", seed=58)
+    d = _dev({k: v for k, v in inp.items() if k != "R"})
+    y, x_dbl = ss.ss2d_forward_proj(d["x"], d["x_proj_weight"], d["dt_proj_weight"], d["dt_proj_bias"], d["A"],
+                                    d["D"], True, return_x_dbl=True)
+    dy_np = torch.randn(tuple(y.shape), generator=torch.Generator().manual_seed(59), dtype=torch.float64)
+    dy_np = dy_np.to(torch.bfloat16).double().numpy()
+    got = ss.ss2d_backward_proj(d["x"], d["x_proj_weight"], d["dt_proj_weight"], d["dt_proj_bias"], d["A"], d["D"],
+                                x_dbl, torch.as_tensor(dy_np, device="cuda").to(torch.bfloat16), True)
+    ref = oracle.ss2d_backward_proj(inp["x"], inp["x_proj_weight"], inp["dt_proj_weight"], inp["dt_proj_bias"],
+                                    inp["A"], inp["D"], True, dy_np)
+    for name in ("dx", "dx_proj_weight", "ddt_proj_weight", "ddt_proj_bias", "dA", "dD"):
+        assert_rel_l2(got[name], ref[name], BF16_TOL, f"{name} bf16")
+
+
+def test_ss2d_backward_proj_deterministic():
+    w, inp = _proj_case(2, 64, 20, 24, 16, seed=60)
+    d = _dev({k: v for k, v in inp.items() if k != "R"})
+    y, x_dbl = ss.ss2d_forward_proj(d["x"], d["x_proj_weight"], d["dt_proj_weight"], d["dt_proj_bias"], d["A"],
+                                    d["D"], True, return_x_dbl=True)
+    dy = torch.randn(y.shape, generator=torch.Generator(device="cuda").manual_seed(61), device="cuda")
+    runs = [ss.ss2d_backward_proj(d["x"], d["x_proj_weight"], d["dt_proj_weight"], d["dt_proj_bias"], d["A"], d["D"],
+                                  x_dbl, dy, True) for _ in range(2)]
+    for k in runs[0]:
+        assert torch.equal(runs[0][k], runs[1][k]), k
+
+
 # ------------------------------------------------------------- fused SS2D
 
 FUSED_CASES = [(1, 8, 8, 8, 4), (2, 6, 5, 9, 16), (1, 70, 12, 11, 16), (1, 8, 64, 64, 16), (2, 3, 1, 1, 2),
