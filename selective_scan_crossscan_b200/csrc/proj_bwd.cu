@@ -9,71 +9,223 @@
 //     du_k           += x_proj.weight^T @ dx_dbl                (D x R+2N) . (R+2N x L)
 // u_k is x along path k (x or its transpose, paths 2 and 3 backwards).
 //
-// pp_gemm_kernel does the per-token contractions: a CTA computes a 64 x 64 tile (output rows
-// x tokens) of one (b, k) with 256 threads holding 4 x 4 outputs each, streaming the
-// contraction dimension through shared memory 16 at a time.  tr_gemm_kernel does the sums over
-// tokens: a CTA computes a 64 x 64 tile of a weight gradient over one chunk of one batch
-// item's tokens and writes it as a partial; reduce_partials_kernel adds the partials of every
-// (batch item, chunk) in a fixed order, so the result is deterministic.  All arithmetic is
-// fp32 on the FMA pipe.
+// The two contractions with R on one side are narrow (R <= 32) and bound by reading ddelta
+// once: dtlow_kernel gives each thread one token and its R sums; dwdt_kernel gives each
+// thread one channel's R sums over a quarter of a staged token tile.  du_kernel stages both
+// operands of a 64-channel x 128-token tile whole (the contraction is R + 2N <= 64 long).
+// tr_gemm_kernel (d x_proj.weight) holds all R + 2N (<= 64) rows of a 128-column tile per CTA
+// and stages tokens 32 at a time, double-buffered through registers.  The sums over tokens
+// are written per (batch item, token chunk) as partials that reduce_partials_kernel adds in
+// a fixed order, so every gradient is deterministic.  All arithmetic is fp32 on the FMA pipe.
 #include "common.cuh"
 #include "kernels.h"
 
 namespace ss2d {
 
-constexpr int kGT = 64;       // tile edge
-constexpr int kGK = 16;       // contraction slice per shared-memory pass
-constexpr int kGThreads = 256;
+// ------------------------------------------------------------ narrow: R sums --
 
-// out[g, m, l] (+)= sum_j M(k, m, j) in[g, j, l], g = b * 4 + k, M(k, m, j) = Mw[k*msk + m*sm + j*sj]
-template <typename Tin, typename Tout, bool ACC>
-__global__ void __launch_bounds__(kGThreads) pp_gemm_kernel(const Tin *__restrict__ in, int64_t in_gstride,
-                                                            const float *__restrict__ Mw, int64_t msk, int64_t sm,
-                                                            int64_t sj, Tout *__restrict__ out, int64_t out_gstride,
-                                                            int Mrows, int J, int64_t L, int nmt, int64_t nlt) {
-    __shared__ __align__(16) float As[kGK][kGT + 4];  // [j][m]
-    __shared__ __align__(16) float Bs[kGK][kGT + 4];  // [j][l]
-    const int t = threadIdx.x, tx = t % 16, ty = t / 16;
-    // one flat grid: output-row tiles fastest (they share the input tile, read once through L2), then tokens, then g
-    const int64_t bid = blockIdx.x, rest = bid / nmt, g = rest / nlt, k = g % kPaths;
-    const int64_t m0 = (bid % nmt) * kGT, l0 = (rest % nlt) * kGT;
-    const Tin *src = in + g * in_gstride;
-    float acc[4][4] = {};
-    for (int j0 = 0; j0 < J; j0 += kGK) {
+constexpr int kNarrowTok = 256;  // tokens (one per thread) of a dtlow_kernel CTA
+constexpr int kNarrowD = 64;     // channels per staged slice of dt_proj.weight
+
+// dx_dbl[g, r, l] = sum_d Wdt[k*D + d, r] ddelta[g, d, l], g = b * 4 + k; RB = R rounded up to 4
+template <typename Tin, int RB>
+__global__ void __launch_bounds__(kNarrowTok) dtlow_kernel(const Tin *__restrict__ ddelta,
+                                                           const float *__restrict__ Wdt, float *__restrict__ dxdbl,
+                                                           int64_t D, int64_t L, int R, int RN, int64_t nlt) {
+    __shared__ __align__(16) float Ws[kNarrowD][RB];
+    const int64_t bid = blockIdx.x, g = bid / nlt, k = g % kPaths;
+    const int64_t l = (bid % nlt) * kNarrowTok + threadIdx.x;
+    const bool live = l < L;
+    const Tin *src = ddelta + g * D * L + (live ? l : L - 1);  // dead threads re-read the last token
+    float acc[RB];
+#pragma unroll
+    for (int r = 0; r < RB; ++r) acc[r] = 0.f;
+    for (int64_t d0 = 0; d0 < D; d0 += kNarrowD) {
+        const int n = (int)(D - d0 < kNarrowD ? D - d0 : kNarrowD);
         __syncthreads();
-        for (int e = t; e < kGK * kGT; e += kGThreads) {
-            const int jj = e / kGT, mm = e % kGT;
-            const int64_t m = m0 + mm, j = j0 + jj, l = l0 + mm;
-            As[jj][mm] = (m < Mrows && j < J) ? Mw[k * msk + m * sm + j * sj] : 0.f;
-            Bs[jj][mm] = (j < J && l < L) ? ld(src + j * L + l) : 0.f;
+        for (int e = threadIdx.x; e < kNarrowD * RB; e += kNarrowTok) {
+            const int i = e / RB, r = e % RB;
+            Ws[i][r] = (i < n && r < R) ? Wdt[(k * D + d0 + i) * R + r] : 0.f;
         }
         __syncthreads();
+        const Tin *s = src + d0 * L;
+#pragma unroll 8
+        for (int i = 0; i < n; ++i) {
+            const float v = ld(s + i * L);
 #pragma unroll
-        for (int jj = 0; jj < kGK; ++jj) {
-            const float4 a = *reinterpret_cast<const float4 *>(&As[jj][4 * ty]);
-            const float4 b = *reinterpret_cast<const float4 *>(&Bs[jj][4 * tx]);
-            const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int q = 0; q < 4; ++q) acc[i][q] = fmaf(av[i], bv[q], acc[i][q]);
-        }
-    }
-    Tout *dst = out + g * out_gstride;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int64_t m = m0 + 4 * ty + i;
-        if (m >= Mrows) continue;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int64_t l = l0 + 4 * tx + q;
-            if (l < L) {
-                Tout *o = dst + m * L + l;
-                st(o, ACC ? ld(o) + acc[i][q] : acc[i][q]);
+            for (int q = 0; q < RB / 4; ++q) {
+                const float4 w = *reinterpret_cast<const float4 *>(&Ws[i][4 * q]);
+                acc[4 * q + 0] = fmaf(w.x, v, acc[4 * q + 0]);
+                acc[4 * q + 1] = fmaf(w.y, v, acc[4 * q + 1]);
+                acc[4 * q + 2] = fmaf(w.z, v, acc[4 * q + 2]);
+                acc[4 * q + 3] = fmaf(w.w, v, acc[4 * q + 3]);
             }
         }
     }
+    if (!live) return;
+#pragma unroll
+    for (int r = 0; r < RB; ++r)
+        if (r < R) dxdbl[(g * RN + r) * L + l] = acc[r];
 }
+
+constexpr int kDwD = 64;  // channels per dwdt_kernel CTA (4 threads each)
+constexpr int kDwT = 32;  // tokens per staged tile
+
+// part[(k*B + b)*nlc + lc][d][r] = sum over the chunk's tokens of ddelta[g, d, l] x_dbl[g, r, l].
+// Tiles are double-buffered: the next tile's loads are in registers while this one is summed.
+template <typename Tin, int RB>
+__global__ void __launch_bounds__(256, 2) dwdt_kernel(const Tin *__restrict__ ddelta, const Tin *__restrict__ xdbl,
+                                                   float *__restrict__ part, int64_t B, int64_t D, int64_t L, int R,
+                                                   int RN, int64_t lchunk, int nlc, int ndt) {
+    constexpr int SV = kDwD * kDwT / 256, XV = RB * kDwT / 256;  // staged values per thread
+    static_assert(kDwD * kDwT % 256 == 0 && RB * kDwT % 256 == 0, "tile sizes");
+    __shared__ __align__(16) float S[2][kDwD][kDwT + 4];  // [channel][token]
+    __shared__ __align__(16) float X[2][kDwT][RB + 4];    // [token][r]; the pad spreads the 4 rows a warp reads
+    const int t = threadIdx.x, dl = t / 4, q = t % 4;
+    // one flat grid: channel tiles fastest (they share the x_dbl tile), then (path, batch item, chunk)
+    const int64_t bid = blockIdx.x, z = bid / ndt, k = z % kPaths, rest = z / kPaths, b = rest / nlc,
+                  lc = rest % nlc;
+    const int64_t d0 = (bid % ndt) * kDwD, g = b * kPaths + k;
+    const int64_t lb = lc * lchunk, le = L < lb + lchunk ? L : lb + lchunk;
+    const Tin *s_src = ddelta + g * D * L;
+    const Tin *x_src = xdbl + g * RN * L;
+    float sv[SV], xv[XV];
+    auto fetch = [&](int64_t t0) {
+#pragma unroll
+        for (int v = 0; v < SV; ++v) {
+            const int e = t + 256 * v, i = e / kDwT, j = e % kDwT;
+            const int64_t d = d0 + i, l = t0 + j;
+            sv[v] = (d < D && l < le) ? ld(s_src + d * L + l) : 0.f;
+        }
+#pragma unroll
+        for (int v = 0; v < XV; ++v) {
+            const int e = t + 256 * v, r = e / kDwT, j = e % kDwT;
+            const int64_t l = t0 + j;
+            xv[v] = (r < R && l < le) ? ld(x_src + r * L + l) : 0.f;
+        }
+    };
+    auto park = [&](int buf) {
+#pragma unroll
+        for (int v = 0; v < SV; ++v) {
+            const int e = t + 256 * v;
+            S[buf][e / kDwT][e % kDwT] = sv[v];
+        }
+#pragma unroll
+        for (int v = 0; v < XV; ++v) {
+            const int e = t + 256 * v;
+            X[buf][e % kDwT][e / kDwT] = xv[v];
+        }
+    };
+    float acc[RB];
+#pragma unroll
+    for (int r = 0; r < RB; ++r) acc[r] = 0.f;
+    fetch(lb);
+    park(0);
+    __syncthreads();
+    int buf = 0;
+    for (int64_t t0 = lb; t0 < le; t0 += kDwT) {
+        const bool more = t0 + kDwT < le;
+        if (more) fetch(t0 + kDwT);
+#pragma unroll 4
+        for (int j = q; j < kDwT; j += 4) {
+            const float v = S[buf][dl][j];
+#pragma unroll
+            for (int qq = 0; qq < RB / 4; ++qq) {
+                const float4 x = *reinterpret_cast<const float4 *>(&X[buf][j][4 * qq]);
+                acc[4 * qq + 0] = fmaf(v, x.x, acc[4 * qq + 0]);
+                acc[4 * qq + 1] = fmaf(v, x.y, acc[4 * qq + 1]);
+                acc[4 * qq + 2] = fmaf(v, x.z, acc[4 * qq + 2]);
+                acc[4 * qq + 3] = fmaf(v, x.w, acc[4 * qq + 3]);
+            }
+        }
+        if (more) park(buf ^ 1);  // the other buffer was last read before the previous barrier
+        __syncthreads();
+        buf ^= 1;
+    }
+    // the 4 threads of a channel are adjacent lanes: fold them in a fixed order
+#pragma unroll
+    for (int r = 0; r < RB; ++r) {
+        acc[r] += __shfl_xor_sync(0xffffffffu, acc[r], 1);
+        acc[r] += __shfl_xor_sync(0xffffffffu, acc[r], 2);
+    }
+    const int64_t d = d0 + dl;
+    if (q != 0 || d >= D) return;
+    float *dst = part + ((k * B + b) * nlc + lc) * D * R + d * R;
+#pragma unroll
+    for (int r = 0; r < RB; ++r)
+        if (r < R) dst[r] = acc[r];
+}
+
+// ------------------------------------------------------------------------ du --
+
+constexpr int kDuM = 64;   // channels per du_kernel tile (8 thread rows x 8)
+constexpr int kDuL = 128;  // tokens per tile (32 thread columns x 4)
+
+// du[g, d, l] += sum_c Wx[k, c, d] dx_dbl[g, c, l] over a 64-channel x 128-token tile.  The
+// contraction is short (R + 2N <= 64), so both operands are staged whole and summed after one
+// barrier; thread (ty, tx) holds channels ty + 8i and tokens 4tx..4tx+3, so a warp's
+// read-modify-write of du covers 128 contiguous floats of one row.
+__global__ void __launch_bounds__(256) du_kernel(const float *__restrict__ dxdbl, const float *__restrict__ Wx,
+                                                 float *__restrict__ du, int64_t D, int64_t L, int RN, int nmt,
+                                                 int64_t nlt) {
+    constexpr int AS = kDuM + 4, BS = kDuL + 4;
+    extern __shared__ __align__(16) float du_smem[];
+    float *As = du_smem;            // [RN][AS]  Wx[k, c, d0 + .]
+    float *Bs = du_smem + RN * AS;  // [RN][BS]  dx_dbl[g, c, l0 + .]
+    const int t = threadIdx.x, ty = t / 32, tx = t % 32;
+    // one flat grid: channel tiles fastest (they share the dx_dbl tile, read once through L2)
+    const int64_t bid = blockIdx.x, rest = bid / nmt, g = rest / nlt, k = g % kPaths;
+    const int64_t d0 = (bid % nmt) * kDuM, l0 = (rest % nlt) * kDuL;
+    for (int e = t; e < RN * kDuM; e += 256) {
+        const int c = e / kDuM, dd = e % kDuM;
+        As[c * AS + dd] = d0 + dd < D ? Wx[(k * RN + c) * D + d0 + dd] : 0.f;
+    }
+    const float *src = dxdbl + g * RN * L + l0;
+    for (int e = t; e < RN * kDuL; e += 256) {
+        const int c = e / kDuL, ll = e % kDuL;
+        Bs[c * BS + ll] = l0 + ll < L ? src[c * L + ll] : 0.f;
+    }
+    __syncthreads();
+    float acc[8][4];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[i][q] = 0.f;
+#pragma unroll 4
+    for (int c = 0; c < RN; ++c) {
+        const float4 bq = *reinterpret_cast<const float4 *>(&Bs[c * BS + 4 * tx]);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float a = As[c * AS + ty + 8 * i];
+            acc[i][0] = fmaf(a, bq.x, acc[i][0]);
+            acc[i][1] = fmaf(a, bq.y, acc[i][1]);
+            acc[i][2] = fmaf(a, bq.z, acc[i][2]);
+            acc[i][3] = fmaf(a, bq.w, acc[i][3]);
+        }
+    }
+    const int64_t l = l0 + 4 * tx;
+    const bool vec = (L % 4 == 0) && l + 3 < L;  // rows start 16-byte aligned when L % 4 == 0
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int64_t d = d0 + ty + 8 * i;
+        if (d >= D) continue;
+        float *o = du + (g * D + d) * L + l;
+        if (vec) {
+            float4 v = *reinterpret_cast<float4 *>(o);
+            v.x += acc[i][0];
+            v.y += acc[i][1];
+            v.z += acc[i][2];
+            v.w += acc[i][3];
+            *reinterpret_cast<float4 *>(o) = v;
+        } else {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                if (l + q < L) o[q] += acc[i][q];
+        }
+    }
+}
+
+// ------------------------------------------------- token sums of outer products --
 
 // part[((k * B + b) * nlc + lc), m, n] = sum over l in chunk lc of A(b, k, m, l) * Bop(b, k, n, l),
 // A(b, k, m, l) = A[b*a_bs + k*a_ks + m*L + l], Bop(b, k, n, l) = Bp[k][b*b_bs + n*L + (rev_k ? L-1-l : l)]
@@ -87,50 +239,108 @@ struct TrArgs {
     int64_t B, L;
     int64_t lchunk;
     int nlc;
-    int nmt, nnt;  // tiles of M and of N
+    int nnt;  // tiles of N
     float *part;
 };
 
-template <typename TA, typename TB>
-__global__ void __launch_bounds__(kGThreads) tr_gemm_kernel(const TrArgs p) {
-    __shared__ __align__(16) float As[kGK][kGT + 4];  // [token][m]
-    __shared__ __align__(16) float Bs[kGK][kGT + 4];  // [token][n]
-    const int t = threadIdx.x, tx = t % 16, ty = t / 16;
-    // one flat grid: N tiles fastest, then M tiles, then (path, batch item, token chunk)
-    const int64_t bid = blockIdx.x, r1 = bid / p.nnt, z = r1 / p.nmt;
+constexpr int kTN = 128;  // tile columns: 32 thread columns of 4
+constexpr int kTS = 32;   // tokens per staged slice
+
+// Staging map of a warp's 32 loads: 8 consecutive tokens of 4 rows (full 32-byte sectors in
+// fp32), so the transposing store [token][row] of a row stride 4 (mod 8) words hits 32 banks.
+__device__ __forceinline__ void stage_index(int e, int &row, int &tok) {
+    const int j = e % 32, grp = e / 32;
+    tok = (grp % (kTS / 8)) * 8 + j % 8;
+    row = (grp / (kTS / 8)) * 4 + j / 8;
+}
+
+template <int TY>
+constexpr size_t tr_smem_bytes() { return (size_t)2 * kTS * ((8 * TY + 4) + (kTN + 4)) * sizeof(float); }
+
+// CTA tile TM = 8*TY rows (all of M) x 128 columns, 256 threads: thread (ty, tx) holds rows ty + 8i
+// (i < TY) and columns 4tx..4tx+3.  Slices are double-buffered: the next slice's loads are in
+// registers while this one is summed.
+template <typename TA, typename TB, int TY>
+__global__ void __launch_bounds__(256, 2) tr_gemm_kernel(const TrArgs p) {
+    constexpr int TM = 8 * TY, AS = TM + 4, BS = kTN + 4, AV = kTS * TM / 256, BV = kTS * kTN / 256;
+    static_assert(kTS * TM % 256 == 0 && kTS * kTN % 256 == 0, "tile sizes");
+    extern __shared__ __align__(16) float tr_smem[];
+    float *As = tr_smem;                // [2][kTS][AS]  [token][m]
+    float *Bs = tr_smem + 2 * kTS * AS;  // [2][kTS][BS]  [token][n]
+    const int t = threadIdx.x, ty = t / 32, tx = t % 32;
+    // one flat grid: N tiles fastest, then (path, batch item, token chunk)
+    const int64_t bid = blockIdx.x, z = bid / p.nnt;
     const int64_t k = z % kPaths, rest = z / kPaths, b = rest / p.nlc, lc = rest % p.nlc;
-    const int64_t n0 = (bid % p.nnt) * kGT, m0 = (r1 % p.nmt) * kGT;
-    const int64_t lb = lc * p.lchunk, le = min(p.L, lb + p.lchunk);
+    const int64_t n0 = (bid % p.nnt) * kTN;
+    const int64_t lb = lc * p.lchunk, le = p.L < lb + p.lchunk ? p.L : lb + p.lchunk;
     const TA *A = static_cast<const TA *>(p.A) + b * p.a_bs + k * p.a_ks;
     const void *bk = k == 0 ? p.Bp[0] : k == 1 ? p.Bp[1] : k == 2 ? p.Bp[2] : p.Bp[3];  // no local copy of p.Bp
     const TB *Bo = static_cast<const TB *>(bk) + b * p.b_bs;
     const bool rev = (p.rev_mask >> k) & 1;
-    float acc[4][4] = {};
-    for (int64_t t0 = lb; t0 < le; t0 += kGK) {
-        __syncthreads();
-        for (int e = t; e < kGK * kGT; e += kGThreads) {
-            const int rr = e / kGK, tt = e % kGK;  // row of the tile, token of the slice (tokens fastest)
-            const int64_t l = t0 + tt, m = m0 + rr, n = n0 + rr;
-            const bool ok = l < le;
-            As[tt][rr] = (ok && m < p.M) ? ld(A + m * p.L + l) : 0.f;
-            Bs[tt][rr] = (ok && n < p.N) ? ld(Bo + n * p.L + (rev ? p.L - 1 - l : l)) : 0.f;
+    float av[AV], bv[BV];
+    auto fetch = [&](int64_t t0) {
+#pragma unroll
+        for (int v = 0; v < AV; ++v) {
+            int rr, tt;
+            stage_index(t + 256 * v, rr, tt);
+            const int64_t l = t0 + tt;
+            av[v] = (l < le && rr < p.M) ? ld(A + rr * p.L + l) : 0.f;
         }
-        __syncthreads();
 #pragma unroll
-        for (int tt = 0; tt < kGK; ++tt) {
-            const float4 a = *reinterpret_cast<const float4 *>(&As[tt][4 * ty]);
-            const float4 bq = *reinterpret_cast<const float4 *>(&Bs[tt][4 * tx]);
-            const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {bq.x, bq.y, bq.z, bq.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int q = 0; q < 4; ++q) acc[i][q] = fmaf(av[i], bv[q], acc[i][q]);
+        for (int v = 0; v < BV; ++v) {
+            int rr, tt;
+            stage_index(t + 256 * v, rr, tt);
+            const int64_t l = t0 + tt, n = n0 + rr;
+            bv[v] = (l < le && n < p.N) ? ld(Bo + n * p.L + (rev ? p.L - 1 - l : l)) : 0.f;
         }
+    };
+    auto park = [&](int buf) {
+#pragma unroll
+        for (int v = 0; v < AV; ++v) {
+            int rr, tt;
+            stage_index(t + 256 * v, rr, tt);
+            As[(buf * kTS + tt) * AS + rr] = av[v];
+        }
+#pragma unroll
+        for (int v = 0; v < BV; ++v) {
+            int rr, tt;
+            stage_index(t + 256 * v, rr, tt);
+            Bs[(buf * kTS + tt) * BS + rr] = bv[v];
+        }
+    };
+    float acc[TY][4];
+#pragma unroll
+    for (int i = 0; i < TY; ++i)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[i][q] = 0.f;
+    fetch(lb);
+    park(0);
+    __syncthreads();
+    int buf = 0;
+    for (int64_t t0 = lb; t0 < le; t0 += kTS) {
+        const bool more = t0 + kTS < le;
+        if (more) fetch(t0 + kTS);
+        const float *as = As + buf * kTS * AS + ty, *bs = Bs + buf * kTS * BS + 4 * tx;
+#pragma unroll 4
+        for (int tt = 0; tt < kTS; ++tt) {
+            const float4 bq = *reinterpret_cast<const float4 *>(bs + tt * BS);
+#pragma unroll
+            for (int i = 0; i < TY; ++i) {
+                const float a = as[tt * AS + 8 * i];
+                acc[i][0] = fmaf(a, bq.x, acc[i][0]);
+                acc[i][1] = fmaf(a, bq.y, acc[i][1]);
+                acc[i][2] = fmaf(a, bq.z, acc[i][2]);
+                acc[i][3] = fmaf(a, bq.w, acc[i][3]);
+            }
+        }
+        if (more) park(buf ^ 1);  // the other buffer was last read before the previous barrier
+        __syncthreads();
+        buf ^= 1;
     }
     float *dst = p.part + ((k * p.B + b) * p.nlc + lc) * (int64_t)p.M * p.N;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int64_t m = m0 + 4 * ty + i;
+    for (int i = 0; i < TY; ++i) {
+        const int64_t m = ty + 8 * i;
         if (m >= p.M) continue;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -171,39 +381,52 @@ static int grid_cap(int64_t items, int threads) {
     return (int)(want < 148 * 16 ? (want > 0 ? want : 1) : 148 * 16);
 }
 
-template <typename Tin, typename Tout, bool ACC>
-static cudaError_t pp_gemm_t(const void *in, int64_t in_gs, const float *Mw, int64_t msk, int64_t sm, int64_t sj, void *out,
-                      int64_t out_gs, int Mrows, int J, int64_t L, int64_t groups, cudaStream_t stream) {
-    const int nmt = (int)ceil_div(Mrows, kGT);
-    const int64_t nlt = ceil_div(L, kGT), blocks = nmt * nlt * groups;
+template <typename Tin, int RB>
+static cudaError_t dtlow_t(const LaunchShape &s, const void *ddelta, const float *Wdt, int R, int RN, float *dxdbl,
+                           cudaStream_t stream) {
+    const int64_t nlt = ceil_div(s.L, kNarrowTok), blocks = nlt * s.B * kPaths;
     if (blocks > INT32_MAX) return cudaErrorInvalidConfiguration;
-    pp_gemm_kernel<Tin, Tout, ACC><<<(unsigned)blocks, kGThreads, 0, stream>>>(
-        static_cast<const Tin *>(in), in_gs, Mw, msk, sm, sj, static_cast<Tout *>(out), out_gs, Mrows, J, L, nmt, nlt);
+    dtlow_kernel<Tin, RB><<<(unsigned)blocks, kNarrowTok, 0, stream>>>(static_cast<const Tin *>(ddelta), Wdt, dxdbl,
+                                                                        s.D, s.L, R, RN, nlt);
     return cudaSuccess;
+}
+
+template <typename Tin>
+static cudaError_t dtlow_r(const LaunchShape &s, const void *ddelta, const float *Wdt, int R, int RN, float *dxdbl,
+                           cudaStream_t stream) {
+    if (R <= 8) return dtlow_t<Tin, 8>(s, ddelta, Wdt, R, RN, dxdbl, stream);
+    if (R <= 16) return dtlow_t<Tin, 16>(s, ddelta, Wdt, R, RN, dxdbl, stream);
+    if (R <= 24) return dtlow_t<Tin, 24>(s, ddelta, Wdt, R, RN, dxdbl, stream);
+    return dtlow_t<Tin, 32>(s, ddelta, Wdt, R, RN, dxdbl, stream);
 }
 
 // dx_dbl[:R] (fp32, group stride RN*L) = dt_proj.weight^T @ ddelta (in dtype, group stride D*L)
 cudaError_t launch_proj_bwd_dtlow(const LaunchShape &s, ss2d_dtype_t dt, const void *ddelta, const float *Wdt, int R,
                                   int RN, float *dxdbl, cudaStream_t stream) {
-    // M(k, m = r, j = d) = Wdt[(k*D + d)*R + r]
-    const cudaError_t e =
-        dt == SS2D_F32
-            ? pp_gemm_t<float, float, false>(ddelta, s.D * s.L, Wdt, s.D * R, 1, R, dxdbl, (int64_t)RN * s.L, R,
-                                             (int)s.D, s.L, s.B * kPaths, stream)
-            : pp_gemm_t<__nv_bfloat16, float, false>(ddelta, s.D * s.L, Wdt, s.D * R, 1, R, dxdbl, (int64_t)RN * s.L,
-                                                     R, (int)s.D, s.L, s.B * kPaths, stream);
+    if (R < 1 || R > kProjRMax) return cudaErrorInvalidValue;
+    const cudaError_t e = dt == SS2D_F32 ? dtlow_r<float>(s, ddelta, Wdt, R, RN, dxdbl, stream)
+                                         : dtlow_r<__nv_bfloat16>(s, ddelta, Wdt, R, RN, dxdbl, stream);
     if (e != cudaSuccess) return e;
     note_launch(stream);
     return cudaGetLastError();
 }
 
-// du_seq (fp32, (B, 4D, L)) += x_proj.weight^T @ dx_dbl (fp32, group stride RN*L)
+constexpr int kRNMax = kProjRMax + 2 * 16;  // rows of x_dbl: dt rank <= 32, d_state <= 16
+
+static size_t du_smem_bytes(int RN) { return (size_t)RN * ((kDuM + 4) + (kDuL + 4)) * sizeof(float); }
+
+// du_seq (fp32, (B, 4D, L)) += x_proj.weight^T @ dx_dbl (fp32, group stride RN*L); du_seq 16-byte aligned
 cudaError_t launch_proj_bwd_du(const LaunchShape &s, const float *dxdbl, const float *Wx, int RN, float *du_seq,
                                cudaStream_t stream) {
-    // M(k, m = d, j = c) = Wx[(k*RN + c)*D + d]
-    const cudaError_t e = pp_gemm_t<float, float, true>(dxdbl, (int64_t)RN * s.L, Wx, (int64_t)RN * s.D, 1, s.D, du_seq,
-                                                        s.D * s.L, (int)s.D, RN, s.L, s.B * kPaths, stream);
+    if (RN < 1 || RN > kRNMax) return cudaErrorInvalidValue;
+    // up to 64 * 200 * 4 = 51,200 bytes: opt in on the current device (cheap, and right on any device)
+    cudaError_t e = cudaFuncSetAttribute(du_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)du_smem_bytes(kRNMax));
     if (e != cudaSuccess) return e;
+    const int nmt = (int)ceil_div(s.D, kDuM);
+    const int64_t nlt = ceil_div(s.L, kDuL), blocks = nmt * nlt * s.B * kPaths;
+    if (blocks > INT32_MAX) return cudaErrorInvalidConfiguration;
+    du_kernel<<<(unsigned)blocks, 256, du_smem_bytes(RN), stream>>>(dxdbl, Wx, du_seq, s.D, s.L, RN, nmt, nlt);
     note_launch(stream);
     return cudaGetLastError();
 }
@@ -223,41 +446,69 @@ cudaError_t launch_proj_bwd_copy_rows(const LaunchShape &s, ss2d_dtype_t dt, con
 
 int64_t proj_bwd_chunks(const LaunchShape &s) { return ceil_div(s.L, kProjTokenChunk); }
 
-template <typename TA, typename TB>
-static cudaError_t token_reduce_t(const LaunchShape &s, TrArgs p, float *out, cudaStream_t stream) {
-    p.B = s.B;
-    p.L = s.L;
-    p.lchunk = kProjTokenChunk;
-    p.nlc = (int)proj_bwd_chunks(s);
-    p.nmt = (int)ceil_div(p.M, kGT);
-    p.nnt = (int)ceil_div(p.N, kGT);
-    const int64_t blocks = (int64_t)p.nmt * p.nnt * kPaths * s.B * p.nlc;
+static void reduce_partials(const LaunchShape &s, const float *part, float *out, int64_t MN, cudaStream_t stream) {
+    reduce_partials_kernel<<<grid_cap(kPaths * MN, 256), 256, 0, stream>>>(part, out, s.B * proj_bwd_chunks(s), MN);
+    note_launch(stream);
+}
+
+template <typename Tin, int RB>
+static cudaError_t dwdt_t(const LaunchShape &s, const void *ddelta, const void *xdbl, int R, int RN, float *part,
+                          cudaStream_t stream) {
+    const int nlc = (int)proj_bwd_chunks(s), ndt = (int)ceil_div(s.D, kDwD);
+    const int64_t blocks = (int64_t)ndt * kPaths * s.B * nlc;
     if (blocks > INT32_MAX) return cudaErrorInvalidConfiguration;
-    tr_gemm_kernel<TA, TB><<<(unsigned)blocks, kGThreads, 0, stream>>>(p);
-    note_launch(stream);
-    const int64_t MN = (int64_t)p.M * p.N;
-    reduce_partials_kernel<<<grid_cap(kPaths * MN, 256), 256, 0, stream>>>(p.part, out, s.B * p.nlc, MN);
-    note_launch(stream);
-    return cudaGetLastError();
+    dwdt_kernel<Tin, RB><<<(unsigned)blocks, 256, 0, stream>>>(static_cast<const Tin *>(ddelta),
+                                                               static_cast<const Tin *>(xdbl), part, s.B, s.D, s.L, R,
+                                                               RN, kProjTokenChunk, nlc, ndt);
+    return cudaSuccess;
+}
+
+template <typename Tin>
+static cudaError_t dwdt_r(const LaunchShape &s, const void *ddelta, const void *xdbl, int R, int RN, float *part,
+                          cudaStream_t stream) {
+    if (R <= 8) return dwdt_t<Tin, 8>(s, ddelta, xdbl, R, RN, part, stream);
+    if (R <= 16) return dwdt_t<Tin, 16>(s, ddelta, xdbl, R, RN, part, stream);
+    if (R <= 24) return dwdt_t<Tin, 24>(s, ddelta, xdbl, R, RN, part, stream);
+    return dwdt_t<Tin, 32>(s, ddelta, xdbl, R, RN, part, stream);
 }
 
 // d dt_proj.weight (4, D, R) = sum over tokens of ddelta (x) x_dbl[:R]
 cudaError_t launch_proj_bwd_dwdt(const LaunchShape &s, ss2d_dtype_t dt, const void *ddelta, const void *xdbl, int R,
                                  int RN, float *part, float *dWdt, cudaStream_t stream) {
-    TrArgs p{};
-    p.A = ddelta;
-    p.a_bs = kPaths * s.D * s.L;
-    p.a_ks = s.D * s.L;
-    const size_t es = dt == SS2D_F32 ? 4 : 2;
-    for (int k = 0; k < kPaths; ++k)
-        p.Bp[k] = static_cast<const unsigned char *>(xdbl) + (size_t)k * RN * s.L * es;
-    p.b_bs = (int64_t)kPaths * RN * s.L;
-    p.rev_mask = 0;
-    p.M = (int)s.D;
-    p.N = R;
-    p.part = part;
-    if (dt == SS2D_F32) return token_reduce_t<float, float>(s, p, dWdt, stream);
-    return token_reduce_t<__nv_bfloat16, __nv_bfloat16>(s, p, dWdt, stream);
+    if (R < 1 || R > kProjRMax) return cudaErrorInvalidValue;
+    const cudaError_t e = dt == SS2D_F32 ? dwdt_r<float>(s, ddelta, xdbl, R, RN, part, stream)
+                                         : dwdt_r<__nv_bfloat16>(s, ddelta, xdbl, R, RN, part, stream);
+    if (e != cudaSuccess) return e;
+    note_launch(stream);
+    reduce_partials(s, part, dWdt, s.D * R, stream);
+    return cudaGetLastError();
+}
+
+template <typename TB, int TY>
+static cudaError_t dwx_t(const LaunchShape &s, TrArgs p, cudaStream_t stream) {
+    const int64_t blocks = (int64_t)p.nnt * kPaths * s.B * p.nlc;
+    if (blocks > INT32_MAX) return cudaErrorInvalidConfiguration;
+    constexpr size_t smem = tr_smem_bytes<TY>();  // up to 2 * 32 * (68 + 132) * 4 = 51,200 bytes
+    const cudaError_t e =
+        cudaFuncSetAttribute(tr_gemm_kernel<float, TB, TY>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    tr_gemm_kernel<float, TB, TY><<<(unsigned)blocks, 256, smem, stream>>>(p);
+    return cudaSuccess;
+}
+
+template <typename TB>
+static cudaError_t dwx_ty(const LaunchShape &s, TrArgs p, cudaStream_t stream) {
+    switch ((int)ceil_div(p.M, 8)) {  // rows R + 2N, 3..64, in one tile of 8 * TY rows
+        case 1: return dwx_t<TB, 1>(s, p, stream);
+        case 2: return dwx_t<TB, 2>(s, p, stream);
+        case 3: return dwx_t<TB, 3>(s, p, stream);
+        case 4: return dwx_t<TB, 4>(s, p, stream);
+        case 5: return dwx_t<TB, 5>(s, p, stream);
+        case 6: return dwx_t<TB, 6>(s, p, stream);
+        case 7: return dwx_t<TB, 7>(s, p, stream);
+        case 8: return dwx_t<TB, 8>(s, p, stream);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 // d x_proj.weight (4, RN, D) = sum over tokens of dx_dbl (x) u_k, u_k = x / xT along path k
@@ -275,9 +526,17 @@ cudaError_t launch_proj_bwd_dwx(const LaunchShape &s, ss2d_dtype_t dt, const flo
     p.rev_mask = 0b1100;  // paths 2 and 3 walk their base order backwards
     p.M = RN;
     p.N = (int)s.D;
+    p.B = s.B;
+    p.L = s.L;
+    p.lchunk = kProjTokenChunk;
+    p.nlc = (int)proj_bwd_chunks(s);
+    p.nnt = (int)ceil_div(p.N, kTN);
     p.part = part;
-    if (dt == SS2D_F32) return token_reduce_t<float, float>(s, p, dWx, stream);
-    return token_reduce_t<float, __nv_bfloat16>(s, p, dWx, stream);
+    const cudaError_t e = dt == SS2D_F32 ? dwx_ty<float>(s, p, stream) : dwx_ty<__nv_bfloat16>(s, p, stream);
+    if (e != cudaSuccess) return e;
+    note_launch(stream);
+    reduce_partials(s, part, dWx, (int64_t)RN * s.D, stream);
+    return cudaGetLastError();
 }
 
 }  // namespace ss2d
