@@ -74,7 +74,7 @@ constexpr int kDwT = 32;  // tokens per staged tile
 // part[(k*B + b)*nlc + lc][d][r] = sum over the chunk's tokens of ddelta[g, d, l] x_dbl[g, r, l].
 // Tiles are double-buffered: the next tile's loads are in registers while this one is summed.
 template <typename Tin, int RB>
-__global__ void __launch_bounds__(256, 2) dwdt_kernel(const Tin *__restrict__ ddelta, const Tin *__restrict__ xdbl,
+__global__ void __launch_bounds__(256, 3) dwdt_kernel(const Tin *__restrict__ ddelta, const Tin *__restrict__ xdbl,
                                                    float *__restrict__ part, int64_t B, int64_t D, int64_t L, int R,
                                                    int RN, int64_t lchunk, int nlc, int ndt) {
     constexpr int SV = kDwD * kDwT / 256, XV = RB * kDwT / 256;  // staged values per thread
@@ -261,7 +261,7 @@ constexpr size_t tr_smem_bytes() { return (size_t)2 * kTS * ((8 * TY + 4) + (kTN
 // (i < TY) and columns 4tx..4tx+3.  Slices are double-buffered: the next slice's loads are in
 // registers while this one is summed.
 template <typename TA, typename TB, int TY>
-__global__ void __launch_bounds__(256, 2) tr_gemm_kernel(const TrArgs p) {
+__global__ void __launch_bounds__(256, 3) tr_gemm_kernel(const TrArgs p) {
     constexpr int TM = 8 * TY, AS = TM + 4, BS = kTN + 4, AV = kTS * TM / 256, BV = kTS * kTN / 256;
     static_assert(kTS * TM % 256 == 0 && kTS * kTN % 256 == 0, "tile sizes");
     extern __shared__ __align__(16) float tr_smem[];
@@ -358,7 +358,15 @@ __global__ void reduce_partials_kernel(const float *__restrict__ part, float *__
         const int64_t k = e / MN, mn = e - k * MN;
         const float *src = part + k * nparts * MN + mn;
         float s = 0.f;
-        for (int64_t i = 0; i < nparts; ++i) s += src[i * MN];
+        int64_t i = 0;
+        for (; i + 8 <= nparts; i += 8) {  // eight loads in flight, added in the same order
+            float v[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v[j] = src[(i + j) * MN];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) s += v[j];
+        }
+        for (; i < nparts; ++i) s += src[i * MN];
         out[e] = s;
     }
 }

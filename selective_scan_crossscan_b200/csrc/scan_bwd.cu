@@ -499,23 +499,55 @@ __global__ void __launch_bounds__(32 * kWarps, SS2D_BWD_MIN_BLOCKS) scan_bwd_ker
 // dB/dC = sum over tiles of the partials (fixed order); dA/dD/ddelta_bias = sum over the batch.
 // G groups per batch item; the bidirectional scan has one group whose "tiles" are both
 // directions' channel tiles (its partials are stored at natural positions).
+constexpr int kReduceBcTok = 1024;  // tokens per CTA of bwd_reduce_bc_kernel (4 per thread)
+
+template <typename Tin>
+__device__ __forceinline__ void store4(Tin *p, float a, float b, float c, float d);
+template <>
+__device__ __forceinline__ void store4<float>(float *p, float a, float b, float c, float d) {
+    *reinterpret_cast<float4 *>(p) = make_float4(a, b, c, d);
+}
+template <>
+__device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16 *p, float a, float b, float c, float d) {
+    __nv_bfloat162 lo = __floats2bfloat162_rn(a, b), hi = __floats2bfloat162_rn(c, d);
+    uint2 v;
+    v.x = *reinterpret_cast<uint32_t *>(&lo);
+    v.y = *reinterpret_cast<uint32_t *>(&hi);
+    *reinterpret_cast<uint2 *>(p) = v;
+}
+
+// One CTA per (row = (b*G + k)*N + n, 1024-token range); each thread sums 4 consecutive tokens
+// over the channel tiles in tile order (16-byte loads when L % 4 == 0, so rows stay aligned).
 template <typename Tin>
 __global__ void bwd_reduce_bc_kernel(const float *__restrict__ part_bc, Tin *__restrict__ dB, Tin *__restrict__ dC,
-                                     int64_t B, int G, int N, int64_t L, int ntiles) {
-    const int64_t total = B * G * N * L;
-    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
-         e += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t l = e % L;
-        const int64_t n = (e / L) % N;
-        const int64_t bk = e / (L * N);
+                                     int N, int64_t L, int ntiles, int64_t nlt) {
+    const int64_t row = blockIdx.x / nlt, bk = row / N, n = row - bk * N;
+    const int64_t l = (blockIdx.x % nlt) * kReduceBcTok + 4 * threadIdx.x;
+    if (l >= L) return;
+    const float *pb = part_bc + (bk * ntiles * 2 * N + n) * L + l;  // tile tl: + tl * 2N * L; C rows: + N * L
+    const int64_t tstride = 2 * (int64_t)N * L, cofs = (int64_t)N * L;
+    Tin *ob = dB + row * L + l, *oc = dC + row * L + l;
+    if (L % 4 == 0) {
+        float4 sb = make_float4(0.f, 0.f, 0.f, 0.f), sc = sb;
+        for (int tl = 0; tl < ntiles; ++tl) {
+            const float4 vb = *reinterpret_cast<const float4 *>(pb + tl * tstride);
+            const float4 vc = *reinterpret_cast<const float4 *>(pb + tl * tstride + cofs);
+            sb.x += vb.x; sb.y += vb.y; sb.z += vb.z; sb.w += vb.w;
+            sc.x += vc.x; sc.y += vc.y; sc.z += vc.z; sc.w += vc.w;
+        }
+        store4(ob, sb.x, sb.y, sb.z, sb.w);
+        store4(oc, sc.x, sc.y, sc.z, sc.w);
+        return;
+    }
+    const int m = L - l < 4 ? (int)(L - l) : 4;
+    for (int q = 0; q < m; ++q) {
         float sb = 0.f, sc = 0.f;
         for (int tl = 0; tl < ntiles; ++tl) {
-            const float *pt = part_bc + ((bk * ntiles + tl) * 2 * N) * L;
-            sb += pt[n * L + l];
-            sc += pt[(N + n) * L + l];
+            sb += pb[tl * tstride + q];
+            sc += pb[tl * tstride + cofs + q];
         }
-        st(dB + e, sb);
-        st(dC + e, sc);
+        st(ob + q, sb);
+        st(oc + q, sc);
     }
 }
 
@@ -695,14 +727,14 @@ cudaError_t launch_scan_bwd(const LaunchShape &s, const ScanBwdArgs &a, void *wo
     const int rtiles = a.bidir ? 2 * p.ntiles : p.ntiles;
     const int threads = 256;
     const int64_t nbc = s.B * G * s.N * s.L;
-    const int64_t nblk = ceil_div(nbc, threads);
-    const int blocks_bc = (int)(nblk < 148 * 16 ? nblk : 148 * 16);
+    const int64_t nlt = ceil_div(s.L, kReduceBcTok), blocks_bc = nbc / s.L * nlt;
+    if (blocks_bc > INT32_MAX) return cudaErrorInvalidConfiguration;
     if (a.in_dtype == SS2D_F32)
-        bwd_reduce_bc_kernel<float><<<blocks_bc, threads, 0, stream>>>(part_bc, (float *)a.dBm, (float *)a.dCm, s.B,
-                                                                     G, (int)s.N, s.L, rtiles);
+        bwd_reduce_bc_kernel<float><<<(unsigned)blocks_bc, kReduceBcTok / 4, 0, stream>>>(
+            part_bc, (float *)a.dBm, (float *)a.dCm, (int)s.N, s.L, rtiles, nlt);
     else
-        bwd_reduce_bc_kernel<__nv_bfloat16><<<blocks_bc, threads, 0, stream>>>(
-            part_bc, (__nv_bfloat16 *)a.dBm, (__nv_bfloat16 *)a.dCm, s.B, G, (int)s.N, s.L, rtiles);
+        bwd_reduce_bc_kernel<__nv_bfloat16><<<(unsigned)blocks_bc, kReduceBcTok / 4, 0, stream>>>(
+            part_bc, (__nv_bfloat16 *)a.dBm, (__nv_bfloat16 *)a.dCm, (int)s.N, s.L, rtiles, nlt);
     note_launch(stream);
     const int64_t np = K * s.D * (s.N + 2);
     bwd_reduce_params_kernel<<<(int)ceil_div(np, threads), threads, 0, stream>>>(
