@@ -14,13 +14,48 @@
 // thread one channel's R sums over a quarter of a staged token tile.  du_kernel stages both
 // operands of a 64-channel x 128-token tile whole (the contraction is R + 2N <= 64 long).
 // tr_gemm_kernel (d x_proj.weight) holds all R + 2N (<= 64) rows of a 128-column tile per CTA
-// and stages tokens 32 at a time, double-buffered through registers.  The sums over tokens
+// and streams tokens through a 3-stage cp.async ring, 4 tokens per step.  The sums over tokens
 // are written per (batch item, token chunk) as partials that reduce_partials_kernel adds in
 // a fixed order, so every gradient is deterministic.  All arithmetic is fp32 on the FMA pipe.
 #include "common.cuh"
 #include "kernels.h"
 
 namespace ss2d {
+
+constexpr int kTS = 32;     // tokens per pipeline stage
+constexpr int kStages = 3;  // cp.async ring depth
+
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"((unsigned)__cvta_generic_to_shared(dst)),
+                 "l"(src));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
+
+// copy / zero four consecutive elements (16 bytes fp32, 8 bytes bf16)
+__device__ __forceinline__ void cp_async_quad(float *dst, const float *src) { cp_async16(dst, src); }
+__device__ __forceinline__ void cp_async_quad(__nv_bfloat16 *dst, const __nv_bfloat16 *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"((unsigned)__cvta_generic_to_shared(dst)),
+                 "l"(src));
+}
+__device__ __forceinline__ void zero_quad(float *dst) {
+    *reinterpret_cast<float4 *>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+__device__ __forceinline__ void zero_quad(__nv_bfloat16 *dst) { *reinterpret_cast<uint2 *>(dst) = make_uint2(0u, 0u); }
+
+// four consecutive elements of a shared-memory row as floats (fp32: one 16-byte load; bf16: 8 bytes)
+__device__ __forceinline__ float4 ld4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+__device__ __forceinline__ float4 ld4(const __nv_bfloat16 *p) {
+    const uint2 v = *reinterpret_cast<const uint2 *>(p);
+    return make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u), __uint_as_float(v.y << 16),
+                       __uint_as_float(v.y & 0xffff0000u));
+}
+
+// shared-memory row pitch in elements: 16-byte aligned, and 4 words apart (mod 32) so that eight
+// consecutive rows read at one column fill distinct banks
+template <typename T>
+__host__ __device__ constexpr int row_pitch() { return sizeof(T) == 4 ? kTS + 4 : kTS + 8; }
 
 // ------------------------------------------------------------ narrow: R sums --
 
@@ -69,18 +104,22 @@ __global__ void __launch_bounds__(kNarrowTok) dtlow_kernel(const Tin *__restrict
 }
 
 constexpr int kDwD = 64;  // channels per dwdt_kernel CTA (4 threads each)
-constexpr int kDwT = 32;  // tokens per staged tile
+
+template <typename Tin, int RB>
+constexpr size_t dwdt_smem_bytes() { return (size_t)kStages * (kDwD + RB) * row_pitch<Tin>() * sizeof(Tin); }
 
 // part[(k*B + b)*nlc + lc][d][r] = sum over the chunk's tokens of ddelta[g, d, l] x_dbl[g, r, l].
-// Tiles are double-buffered: the next tile's loads are in registers while this one is summed.
-template <typename Tin, int RB>
-__global__ void __launch_bounds__(256, 3) dwdt_kernel(const Tin *__restrict__ ddelta, const Tin *__restrict__ xdbl,
-                                                   float *__restrict__ part, int64_t B, int64_t D, int64_t L, int R,
-                                                   int RN, int64_t lchunk, int nlc, int ndt) {
-    constexpr int SV = kDwD * kDwT / 256, XV = RB * kDwT / 256;  // staged values per thread
-    static_assert(kDwD * kDwT % 256 == 0 && RB * kDwT % 256 == 0, "tile sizes");
-    __shared__ __align__(16) float S[2][kDwD][kDwT + 4];  // [channel][token]
-    __shared__ __align__(16) float X[2][kDwT][RB + 4];    // [token][r]; the pad spreads the 4 rows a warp reads
+// ddelta and x_dbl's dt rows stream through a 3-stage cp.async ring of 32-token tiles in their
+// global [row][token] layout (plain loads when L % 4 != 0).  Thread (dl, q) sums channel dl over
+// tokens 8q..8q+7 of each tile, one quad at a time: 1 + RB quad loads feed 4*RB FMAs.
+template <typename Tin, int RB, bool VEC>
+__global__ void __launch_bounds__(256, 2) dwdt_kernel(const Tin *__restrict__ ddelta, const Tin *__restrict__ xdbl,
+                                                      float *__restrict__ part, int64_t B, int64_t D, int64_t L,
+                                                      int R, int RN, int64_t lchunk, int nlc, int ndt) {
+    constexpr int P = row_pitch<Tin>(), CS = kDwD * kTS / 4, CX = RB * kTS / 4;
+    extern __shared__ __align__(16) unsigned char dw_smem[];
+    Tin *S = reinterpret_cast<Tin *>(dw_smem);      // [kStages][kDwD][P]
+    Tin *X = S + (size_t)kStages * kDwD * P;        // [kStages][RB][P]
     const int t = threadIdx.x, dl = t / 4, q = t % 4;
     // one flat grid: channel tiles fastest (they share the x_dbl tile), then (path, batch item, chunk)
     const int64_t bid = blockIdx.x, z = bid / ndt, k = z % kPaths, rest = z / kPaths, b = rest / nlc,
@@ -89,58 +128,60 @@ __global__ void __launch_bounds__(256, 3) dwdt_kernel(const Tin *__restrict__ dd
     const int64_t lb = lc * lchunk, le = L < lb + lchunk ? L : lb + lchunk;
     const Tin *s_src = ddelta + g * D * L;
     const Tin *x_src = xdbl + g * RN * L;
-    float sv[SV], xv[XV];
-    auto fetch = [&](int64_t t0) {
-#pragma unroll
-        for (int v = 0; v < SV; ++v) {
-            const int e = t + 256 * v, i = e / kDwT, j = e % kDwT;
-            const int64_t d = d0 + i, l = t0 + j;
-            sv[v] = (d < D && l < le) ? ld(s_src + d * L + l) : 0.f;
-        }
-#pragma unroll
-        for (int v = 0; v < XV; ++v) {
-            const int e = t + 256 * v, r = e / kDwT, j = e % kDwT;
-            const int64_t l = t0 + j;
-            xv[v] = (r < R && l < le) ? ld(x_src + r * L + l) : 0.f;
-        }
-    };
-    auto park = [&](int buf) {
-#pragma unroll
-        for (int v = 0; v < SV; ++v) {
-            const int e = t + 256 * v;
-            S[buf][e / kDwT][e % kDwT] = sv[v];
-        }
-#pragma unroll
-        for (int v = 0; v < XV; ++v) {
-            const int e = t + 256 * v;
-            X[buf][e % kDwT][e / kDwT] = xv[v];
+    const int nst = (int)ceil_div(le - lb, kTS);
+    auto issue = [&](int st_) {
+        const int buf = st_ % kStages;
+        const int64_t t0 = lb + (int64_t)st_ * kTS;
+        const int nv = (int)(le - t0 < kTS ? le - t0 : kTS);
+        Tin *ss = S + (size_t)buf * kDwD * P, *xs = X + (size_t)buf * RB * P;
+        if (VEC) {
+            for (int c = t; c < CS + CX; c += 256) {
+                const bool sx = c < CS;
+                const int cc = sx ? c : c - CS, r = cc / (kTS / 4), j = 4 * (cc % (kTS / 4));
+                Tin *dst = (sx ? ss : xs) + r * P + j;
+                const bool ok = j < nv && (sx ? d0 + r < D : r < R);
+                if (ok) cp_async_quad(dst, (sx ? s_src + (d0 + r) * L : x_src + r * L) + t0 + j);
+                else zero_quad(dst);
+            }
+        } else {
+            for (int e = t; e < (kDwD + RB) * kTS; e += 256) {
+                const int r = e / kTS, j = e % kTS;
+                const bool sx = r < kDwD;
+                const int rr = sx ? r : r - kDwD;
+                const bool ok = j < nv && (sx ? d0 + rr < D : rr < R);
+                const float v = ok ? ld((sx ? s_src + (d0 + rr) * L : x_src + rr * L) + t0 + j) : 0.f;
+                st((sx ? ss : xs) + rr * P + j, v);
+            }
         }
     };
     float acc[RB];
 #pragma unroll
     for (int r = 0; r < RB; ++r) acc[r] = 0.f;
-    fetch(lb);
-    park(0);
-    __syncthreads();
-    int buf = 0;
-    for (int64_t t0 = lb; t0 < le; t0 += kDwT) {
-        const bool more = t0 + kDwT < le;
-        if (more) fetch(t0 + kDwT);
-#pragma unroll 4
-        for (int j = q; j < kDwT; j += 4) {
-            const float v = S[buf][dl][j];
 #pragma unroll
-            for (int qq = 0; qq < RB / 4; ++qq) {
-                const float4 x = *reinterpret_cast<const float4 *>(&X[buf][j][4 * qq]);
-                acc[4 * qq + 0] = fmaf(v, x.x, acc[4 * qq + 0]);
-                acc[4 * qq + 1] = fmaf(v, x.y, acc[4 * qq + 1]);
-                acc[4 * qq + 2] = fmaf(v, x.z, acc[4 * qq + 2]);
-                acc[4 * qq + 3] = fmaf(v, x.w, acc[4 * qq + 3]);
+    for (int st_ = 0; st_ < kStages - 1; ++st_) {
+        if (st_ < nst) issue(st_);
+        cp_async_commit();
+    }
+    for (int st_ = 0; st_ < nst; ++st_) {
+        cp_async_wait<kStages - 2>();
+        __syncthreads();  // tile st_ visible to all; every thread is done with tile st_ - 1's buffer
+        if (st_ + kStages - 1 < nst) issue(st_ + kStages - 1);
+        cp_async_commit();
+        const Tin *ss = S + (size_t)(st_ % kStages) * kDwD * P + dl * P, *xs = X + (size_t)(st_ % kStages) * RB * P;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int tq = 8 * q + 4 * h;
+            const float4 sv = ld4(ss + tq);
+#pragma unroll
+            for (int r = 0; r < RB; ++r) {
+                const float4 xv = ld4(xs + r * P + tq);
+                float a = acc[r];
+                a = fmaf(sv.x, xv.x, a);
+                a = fmaf(sv.y, xv.y, a);
+                a = fmaf(sv.z, xv.z, a);
+                acc[r] = fmaf(sv.w, xv.w, a);
             }
         }
-        if (more) park(buf ^ 1);  // the other buffer was last read before the previous barrier
-        __syncthreads();
-        buf ^= 1;
     }
     // the 4 threads of a channel are adjacent lanes: fold them in a fixed order
 #pragma unroll
@@ -162,28 +203,54 @@ constexpr int kDuM = 64;   // channels per du_kernel tile (8 thread rows x 8)
 constexpr int kDuL = 128;  // tokens per tile (32 thread columns x 4)
 
 // du[g, d, l] += sum_c Wx[k, c, d] dx_dbl[g, c, l] over a 64-channel x 128-token tile.  The
-// contraction is short (R + 2N <= 64), so both operands are staged whole and summed after one
-// barrier; thread (ty, tx) holds channels ty + 8i and tokens 4tx..4tx+3, so a warp's
-// read-modify-write of du covers 128 contiguous floats of one row.
+// contraction is short (R + 2N <= 64), so both operands and the du tile itself are staged whole
+// (one batch of 16-byte cp.async when L and D are multiples of 4, plain loads otherwise) and
+// summed after one barrier; thread (ty, tx) holds channels ty + 8i and tokens 4tx..4tx+3, so a
+// warp's write of du covers 128 contiguous floats of one row.
+template <bool VEC>
 __global__ void __launch_bounds__(256) du_kernel(const float *__restrict__ dxdbl, const float *__restrict__ Wx,
                                                  float *__restrict__ du, int64_t D, int64_t L, int RN, int nmt,
                                                  int64_t nlt) {
     constexpr int AS = kDuM + 4, BS = kDuL + 4;
     extern __shared__ __align__(16) float du_smem[];
-    float *As = du_smem;            // [RN][AS]  Wx[k, c, d0 + .]
-    float *Bs = du_smem + RN * AS;  // [RN][BS]  dx_dbl[g, c, l0 + .]
+    float *As = du_smem;             // [RN][AS]    Wx[k, c, d0 + .]
+    float *Bs = As + RN * AS;        // [RN][BS]    dx_dbl[g, c, l0 + .]
+    float *Us = Bs + RN * BS;        // [kDuM][BS]  du[g, d0 + ., l0 + .] (VEC only)
     const int t = threadIdx.x, ty = t / 32, tx = t % 32;
     // one flat grid: channel tiles fastest (they share the dx_dbl tile, read once through L2)
     const int64_t bid = blockIdx.x, rest = bid / nmt, g = rest / nlt, k = g % kPaths;
     const int64_t d0 = (bid % nmt) * kDuM, l0 = (rest % nlt) * kDuL;
-    for (int e = t; e < RN * kDuM; e += 256) {
-        const int c = e / kDuM, dd = e % kDuM;
-        As[c * AS + dd] = d0 + dd < D ? Wx[(k * RN + c) * D + d0 + dd] : 0.f;
-    }
     const float *src = dxdbl + g * RN * L + l0;
-    for (int e = t; e < RN * kDuL; e += 256) {
-        const int c = e / kDuL, ll = e % kDuL;
-        Bs[c * BS + ll] = l0 + ll < L ? src[c * L + ll] : 0.f;
+    float *out = du + g * D * L + l0;
+    if (VEC) {
+        const int ca = RN * (kDuM / 4), cb = RN * (kDuL / 4), cu = kDuM * (kDuL / 4);
+        for (int c = t; c < ca + cb + cu; c += 256) {
+            if (c < ca) {
+                const int r = c / (kDuM / 4), j = 4 * (c % (kDuM / 4));
+                float *dst = As + r * AS + j;
+                if (d0 + j < D) cp_async16(dst, Wx + (k * RN + r) * D + d0 + j);
+                else zero_quad(dst);
+            } else if (c < ca + cb) {
+                const int cc = c - ca, r = cc / (kDuL / 4), j = 4 * (cc % (kDuL / 4));
+                float *dst = Bs + r * BS + j;
+                if (l0 + j < L) cp_async16(dst, src + r * L + j);
+                else zero_quad(dst);
+            } else {
+                const int cc = c - ca - cb, r = cc / (kDuL / 4), j = 4 * (cc % (kDuL / 4));
+                if (d0 + r < D && l0 + j < L) cp_async16(Us + r * BS + j, out + (d0 + r) * L + j);
+            }
+        }
+        cp_async_commit();
+        cp_async_wait<0>();
+    } else {
+        for (int e = t; e < RN * kDuM; e += 256) {
+            const int c = e / kDuM, dd = e % kDuM;
+            As[c * AS + dd] = d0 + dd < D ? Wx[(k * RN + c) * D + d0 + dd] : 0.f;
+        }
+        for (int e = t; e < RN * kDuL; e += 256) {
+            const int c = e / kDuL, ll = e % kDuL;
+            Bs[c * BS + ll] = l0 + ll < L ? src[c * L + ll] : 0.f;
+        }
     }
     __syncthreads();
     float acc[8][4];
@@ -203,15 +270,15 @@ __global__ void __launch_bounds__(256) du_kernel(const float *__restrict__ dxdbl
             acc[i][3] = fmaf(a, bq.w, acc[i][3]);
         }
     }
-    const int64_t l = l0 + 4 * tx;
-    const bool vec = (L % 4 == 0) && l + 3 < L;  // rows start 16-byte aligned when L % 4 == 0
+    const int64_t l = 4 * tx;  // within the tile
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const int64_t d = d0 + ty + 8 * i;
         if (d >= D) continue;
-        float *o = du + (g * D + d) * L + l;
-        if (vec) {
-            float4 v = *reinterpret_cast<float4 *>(o);
+        float *o = out + d * L + l;
+        if (VEC) {
+            if (l0 + l >= L) continue;
+            float4 v = *reinterpret_cast<const float4 *>(&Us[(ty + 8 * i) * BS + l]);
             v.x += acc[i][0];
             v.y += acc[i][1];
             v.z += acc[i][2];
@@ -220,7 +287,7 @@ __global__ void __launch_bounds__(256) du_kernel(const float *__restrict__ dxdbl
         } else {
 #pragma unroll
             for (int q = 0; q < 4; ++q)
-                if (l + q < L) o[q] += acc[i][q];
+                if (l0 + l + q < L) o[q] += acc[i][q];
         }
     }
 }
@@ -243,69 +310,75 @@ struct TrArgs {
     float *part;
 };
 
-constexpr int kTN = 128;  // tile columns: 32 thread columns of 4
-constexpr int kTS = 32;   // tokens per staged slice
+constexpr int kTN = 128;  // tile columns: 32 lanes x 4, spaced 32 apart
 
-// Staging map of a warp's 32 loads: 8 consecutive tokens of 4 rows (full 32-byte sectors in
-// fp32), so the transposing store [token][row] of a row stride 4 (mod 8) words hits 32 banks.
-__device__ __forceinline__ void stage_index(int e, int &row, int &tok) {
-    const int j = e % 32, grp = e / 32;
-    tok = (grp % (kTS / 8)) * 8 + j % 8;
-    row = (grp / (kTS / 8)) * 4 + j / 8;
+template <typename TB, int TY>
+constexpr size_t tr_smem_bytes() {
+    return (size_t)kStages * (8 * TY * row_pitch<float>() * sizeof(float) + kTN * row_pitch<TB>() * sizeof(TB));
 }
 
-template <int TY>
-constexpr size_t tr_smem_bytes() { return (size_t)2 * kTS * ((8 * TY + 4) + (kTN + 4)) * sizeof(float); }
-
-// CTA tile TM = 8*TY rows (all of M) x 128 columns, 256 threads: thread (ty, tx) holds rows ty + 8i
-// (i < TY) and columns 4tx..4tx+3.  Slices are double-buffered: the next slice's loads are in
-// registers while this one is summed.
-template <typename TA, typename TB, int TY>
-__global__ void __launch_bounds__(256, 3) tr_gemm_kernel(const TrArgs p) {
-    constexpr int TM = 8 * TY, AS = TM + 4, BS = kTN + 4, AV = kTS * TM / 256, BV = kTS * kTN / 256;
-    static_assert(kTS * TM % 256 == 0 && kTS * kTN % 256 == 0, "tile sizes");
-    extern __shared__ __align__(16) float tr_smem[];
-    float *As = tr_smem;                // [2][kTS][AS]  [token][m]
-    float *Bs = tr_smem + 2 * kTS * AS;  // [2][kTS][BS]  [token][n]
+// CTA tile TM = 8*TY rows (all of M) x 128 columns over one token chunk, 256 threads: warp ty holds
+// rows ty + 8i (i < TY), lane tx columns tx + 32q (q < 4).  Both operands sit in shared memory as
+// [row][token] (their global layout), filled by 16-byte cp.async through a 3-stage ring when
+// VEC (L % 4 == 0; every chunk of 4 tokens is then wholly inside or outside the range), else by
+// plain loads.  Each step takes 4 tokens: TY row quads (broadcast in the warp) and 4 column quads
+// feed 16*TY FMAs.  A reversed path (rev) holds its tokens backwards in the row.
+template <typename TB, int TY, bool VEC>
+__global__ void __launch_bounds__(256, 2) tr_gemm_kernel(const TrArgs p) {
+    constexpr int TM = 8 * TY, PA = row_pitch<float>(), PB = row_pitch<TB>();
+    constexpr int CA = TM * kTS / 4, CB = kTN * kTS / 4;  // 4-token chunks per stage
+    extern __shared__ __align__(16) unsigned char tr_smem[];
+    float *As = reinterpret_cast<float *>(tr_smem);                                   // [kStages][TM][PA]
+    TB *Bs = reinterpret_cast<TB *>(tr_smem + (size_t)kStages * TM * PA * sizeof(float));  // [kStages][kTN][PB]
     const int t = threadIdx.x, ty = t / 32, tx = t % 32;
     // one flat grid: N tiles fastest, then (path, batch item, token chunk)
     const int64_t bid = blockIdx.x, z = bid / p.nnt;
     const int64_t k = z % kPaths, rest = z / kPaths, b = rest / p.nlc, lc = rest % p.nlc;
     const int64_t n0 = (bid % p.nnt) * kTN;
     const int64_t lb = lc * p.lchunk, le = p.L < lb + p.lchunk ? p.L : lb + p.lchunk;
-    const TA *A = static_cast<const TA *>(p.A) + b * p.a_bs + k * p.a_ks;
+    const float *A = static_cast<const float *>(p.A) + b * p.a_bs + k * p.a_ks;
     const void *bk = k == 0 ? p.Bp[0] : k == 1 ? p.Bp[1] : k == 2 ? p.Bp[2] : p.Bp[3];  // no local copy of p.Bp
     const TB *Bo = static_cast<const TB *>(bk) + b * p.b_bs;
     const bool rev = (p.rev_mask >> k) & 1;
-    float av[AV], bv[BV];
-    auto fetch = [&](int64_t t0) {
-#pragma unroll
-        for (int v = 0; v < AV; ++v) {
-            int rr, tt;
-            stage_index(t + 256 * v, rr, tt);
-            const int64_t l = t0 + tt;
-            av[v] = (l < le && rr < p.M) ? ld(A + rr * p.L + l) : 0.f;
-        }
-#pragma unroll
-        for (int v = 0; v < BV; ++v) {
-            int rr, tt;
-            stage_index(t + 256 * v, rr, tt);
-            const int64_t l = t0 + tt, n = n0 + rr;
-            bv[v] = (l < le && n < p.N) ? ld(Bo + n * p.L + (rev ? p.L - 1 - l : l)) : 0.f;
-        }
-    };
-    auto park = [&](int buf) {
-#pragma unroll
-        for (int v = 0; v < AV; ++v) {
-            int rr, tt;
-            stage_index(t + 256 * v, rr, tt);
-            As[(buf * kTS + tt) * AS + rr] = av[v];
-        }
-#pragma unroll
-        for (int v = 0; v < BV; ++v) {
-            int rr, tt;
-            stage_index(t + 256 * v, rr, tt);
-            Bs[(buf * kTS + tt) * BS + rr] = bv[v];
+    const int nst = (int)ceil_div(le - lb, kTS);
+
+    // stage s: tokens t0 = lb + s*kTS .. min(t0 + kTS, le); slot j of a B row holds token
+    // t0 + j, or t0 + kTS - 1 - j when rev.  Slots past the range hold zeros.
+    auto issue = [&](int s) {
+        const int buf = s % kStages;
+        const int64_t t0 = lb + (int64_t)s * kTS;
+        const int nv = (int)(le - t0 < kTS ? le - t0 : kTS);
+        float *as = As + (size_t)buf * TM * PA;
+        TB *bs = Bs + (size_t)buf * kTN * PB;
+        if (VEC) {
+            for (int c = t; c < CA; c += 256) {
+                const int r = c / (kTS / 4), j = 4 * (c % (kTS / 4));
+                float *dst = as + r * PA + j;
+                if (r < p.M && j < nv) cp_async16(dst, A + r * p.L + t0 + j);
+                else *reinterpret_cast<float4 *>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+            for (int c = t; c < CB; c += 256) {
+                const int r = c / (kTS / 4), j = 4 * (c % (kTS / 4));
+                TB *dst = bs + r * PB + j;
+                const int tok = rev ? kTS - 4 - j : j;  // first token of the slot quad, counted from t0
+                if (n0 + r < p.N && tok < nv) {
+                    const TB *src = Bo + (n0 + r) * p.L + (rev ? p.L - t0 - kTS + j : t0 + j);
+                    cp_async_quad(dst, src);
+                } else {
+                    zero_quad(dst);
+                }
+            }
+        } else {
+            for (int e = t; e < TM * kTS; e += 256) {
+                const int r = e / kTS, j = e % kTS;
+                as[r * PA + j] = (r < p.M && j < nv) ? A[r * p.L + t0 + j] : 0.f;
+            }
+            for (int e = t; e < kTN * kTS; e += 256) {
+                const int r = e / kTS, j = e % kTS, tok = rev ? kTS - 1 - j : j;
+                const float v = (n0 + r < p.N && tok < nv) ? ld(Bo + (n0 + r) * p.L + (rev ? p.L - 1 - t0 - tok : t0 + tok))
+                                                          : 0.f;
+                st(bs + r * PB + j, v);
+            }
         }
     };
     float acc[TY][4];
@@ -313,29 +386,38 @@ __global__ void __launch_bounds__(256, 3) tr_gemm_kernel(const TrArgs p) {
     for (int i = 0; i < TY; ++i)
 #pragma unroll
         for (int q = 0; q < 4; ++q) acc[i][q] = 0.f;
-    fetch(lb);
-    park(0);
-    __syncthreads();
-    int buf = 0;
-    for (int64_t t0 = lb; t0 < le; t0 += kTS) {
-        const bool more = t0 + kTS < le;
-        if (more) fetch(t0 + kTS);
-        const float *as = As + buf * kTS * AS + ty, *bs = Bs + buf * kTS * BS + 4 * tx;
-#pragma unroll 4
-        for (int tt = 0; tt < kTS; ++tt) {
-            const float4 bq = *reinterpret_cast<const float4 *>(bs + tt * BS);
 #pragma unroll
-            for (int i = 0; i < TY; ++i) {
-                const float a = as[tt * AS + 8 * i];
-                acc[i][0] = fmaf(a, bq.x, acc[i][0]);
-                acc[i][1] = fmaf(a, bq.y, acc[i][1]);
-                acc[i][2] = fmaf(a, bq.z, acc[i][2]);
-                acc[i][3] = fmaf(a, bq.w, acc[i][3]);
+    for (int s = 0; s < kStages - 1; ++s) {
+        if (s < nst) issue(s);
+        cp_async_commit();
+    }
+    for (int s = 0; s < nst; ++s) {
+        cp_async_wait<kStages - 2>();
+        __syncthreads();  // stage s visible to all; every thread is done with stage s - 1's buffer
+        if (s + kStages - 1 < nst) issue(s + kStages - 1);
+        cp_async_commit();
+        const float *as = As + (size_t)(s % kStages) * TM * PA + ty * PA;
+        const TB *bs = Bs + (size_t)(s % kStages) * kTN * PB + tx * PB;
+#pragma unroll 2
+        for (int tt = 0; tt < kTS; tt += 4) {
+            float4 av[TY];
+#pragma unroll
+            for (int i = 0; i < TY; ++i) av[i] = ld4(as + 8 * i * PA + tt);
+            const int jb = rev ? kTS - 4 - tt : tt;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                float4 bq = ld4(bs + 32 * q * PB + jb);
+                if (rev) bq = make_float4(bq.w, bq.z, bq.y, bq.x);
+#pragma unroll
+                for (int i = 0; i < TY; ++i) {
+                    float a = acc[i][q];
+                    a = fmaf(av[i].x, bq.x, a);
+                    a = fmaf(av[i].y, bq.y, a);
+                    a = fmaf(av[i].z, bq.z, a);
+                    acc[i][q] = fmaf(av[i].w, bq.w, a);
+                }
             }
         }
-        if (more) park(buf ^ 1);  // the other buffer was last read before the previous barrier
-        __syncthreads();
-        buf ^= 1;
     }
     float *dst = p.part + ((k * p.B + b) * p.nlc + lc) * (int64_t)p.M * p.N;
 #pragma unroll
@@ -344,7 +426,7 @@ __global__ void __launch_bounds__(256, 3) tr_gemm_kernel(const TrArgs p) {
         if (m >= p.M) continue;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            const int64_t n = n0 + 4 * tx + q;
+            const int64_t n = n0 + tx + 32 * q;
             if (n < p.N) dst[m * p.N + n] = acc[i][q];
         }
     }
@@ -421,20 +503,21 @@ cudaError_t launch_proj_bwd_dtlow(const LaunchShape &s, ss2d_dtype_t dt, const v
 
 constexpr int kRNMax = kProjRMax + 2 * 16;  // rows of x_dbl: dt rank <= 32, d_state <= 16
 
-static size_t du_smem_bytes(int RN) { return (size_t)RN * ((kDuM + 4) + (kDuL + 4)) * sizeof(float); }
+static size_t du_smem_bytes(int RN) { return ((size_t)RN * ((kDuM + 4) + (kDuL + 4)) + kDuM * (kDuL + 4)) * sizeof(float); }
 
 // du_seq (fp32, (B, 4D, L)) += x_proj.weight^T @ dx_dbl (fp32, group stride RN*L); du_seq 16-byte aligned
 cudaError_t launch_proj_bwd_du(const LaunchShape &s, const float *dxdbl, const float *Wx, int RN, float *du_seq,
                                cudaStream_t stream) {
     if (RN < 1 || RN > kRNMax) return cudaErrorInvalidValue;
-    // up to 64 * 200 * 4 = 51,200 bytes: opt in on the current device (cheap, and right on any device)
-    cudaError_t e = cudaFuncSetAttribute(du_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)du_smem_bytes(kRNMax));
+    // up to (64 * 200 + 64 * 132) * 4 = 84,992 bytes: opt in on the current device (cheap, right on any device)
+    const bool vec = s.L % 4 == 0 && s.D % 4 == 0;  // rows of du, dx_dbl and x_proj.weight 16-byte aligned
+    auto kern = vec ? du_kernel<true> : du_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)du_smem_bytes(kRNMax));
     if (e != cudaSuccess) return e;
     const int nmt = (int)ceil_div(s.D, kDuM);
     const int64_t nlt = ceil_div(s.L, kDuL), blocks = nmt * nlt * s.B * kPaths;
     if (blocks > INT32_MAX) return cudaErrorInvalidConfiguration;
-    du_kernel<<<(unsigned)blocks, 256, du_smem_bytes(RN), stream>>>(dxdbl, Wx, du_seq, s.D, s.L, RN, nmt, nlt);
+    kern<<<(unsigned)blocks, 256, du_smem_bytes(RN), stream>>>(dxdbl, Wx, du_seq, s.D, s.L, RN, nmt, nlt);
     note_launch(stream);
     return cudaGetLastError();
 }
@@ -465,9 +548,12 @@ static cudaError_t dwdt_t(const LaunchShape &s, const void *ddelta, const void *
     const int nlc = (int)proj_bwd_chunks(s), ndt = (int)ceil_div(s.D, kDwD);
     const int64_t blocks = (int64_t)ndt * kPaths * s.B * nlc;
     if (blocks > INT32_MAX) return cudaErrorInvalidConfiguration;
-    dwdt_kernel<Tin, RB><<<(unsigned)blocks, 256, 0, stream>>>(static_cast<const Tin *>(ddelta),
-                                                               static_cast<const Tin *>(xdbl), part, s.B, s.D, s.L, R,
-                                                               RN, kProjTokenChunk, nlc, ndt);
+    constexpr size_t smem = dwdt_smem_bytes<Tin, RB>();  // at most 3 * 96 * 36 * 4 = 41,472 bytes
+    auto kern = s.L % 4 == 0 ? dwdt_kernel<Tin, RB, true> : dwdt_kernel<Tin, RB, false>;
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<(unsigned)blocks, 256, smem, stream>>>(static_cast<const Tin *>(ddelta), static_cast<const Tin *>(xdbl),
+                                                  part, s.B, s.D, s.L, R, RN, kProjTokenChunk, nlc, ndt);
     return cudaSuccess;
 }
 
@@ -496,11 +582,12 @@ template <typename TB, int TY>
 static cudaError_t dwx_t(const LaunchShape &s, TrArgs p, cudaStream_t stream) {
     const int64_t blocks = (int64_t)p.nnt * kPaths * s.B * p.nlc;
     if (blocks > INT32_MAX) return cudaErrorInvalidConfiguration;
-    constexpr size_t smem = tr_smem_bytes<TY>();  // up to 2 * 32 * (68 + 132) * 4 = 51,200 bytes
-    const cudaError_t e =
-        cudaFuncSetAttribute(tr_gemm_kernel<float, TB, TY>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    constexpr size_t smem = tr_smem_bytes<TB, TY>();  // at most 3 * (64 + 128) * 36 * 4 = 82,944 bytes
+    const bool vec = s.L % 4 == 0;  // token quads then start 16-byte (fp32) / 8-byte (bf16) aligned
+    auto kern = vec ? tr_gemm_kernel<TB, TY, true> : tr_gemm_kernel<TB, TY, false>;
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    tr_gemm_kernel<float, TB, TY><<<(unsigned)blocks, 256, smem, stream>>>(p);
+    kern<<<(unsigned)blocks, 256, smem, stream>>>(p);
     return cudaSuccess;
 }
 
