@@ -218,6 +218,93 @@ def ss2d_backward_proj(x, x_proj_weight, dt_proj_weight, dt_proj_bias, A, D, del
                 ddt_proj_bias=g["ddelta_bias"], dA=g["dA"], dD=g["dD"])
 
 
+# --------------------------------------------- causal depthwise conv per path
+
+def path_conv(x, conv_weight, conv_bias=None):
+    """The causal depthwise conv with SiLU that MambaInnerFn.forward ("vision mamba-yolov8",
+    section 2) applies before x_proj (causal_conv1d_fwd(x, weight, bias, True)), taken along
+    every SS2D path, each path with its own weights, as the Visual Mamba page's SS2D runs one
+    Mamba block per scan direction:
+        pre_k[d, l] = bias[k, d] + sum_j w[k, d, j] * x_k[d, l - (W-1) + j]   (x_k = 0 before step 0)
+        u_k[d, l]   = silu(pre_k[d, l]) = pre / (1 + exp(-pre))
+    with x_k = x read along path k (CrossScan).  x (Bn, D, H, W); conv_weight (4, D, W);
+    conv_bias (4D) or None.  Returns u (Bn, 4, D, L) and pre (Bn, 4, D, L)."""
+    x, w, bias = _f64(x), _f64(conv_weight), _f64(conv_bias)
+    Bn, Dn, H, W = x.shape
+    Wc = w.shape[2]
+    L = H * W
+    xs = cross_scan(x)
+    pre = np.zeros_like(xs)
+    for j in range(Wc):
+        s = Wc - 1 - j                                         # tap j reads s steps back
+        pre[..., s:] += w[None, :, :, j, None] * xs[..., :L - s]
+    if bias is not None:
+        pre += bias.reshape(1, K_PATHS, Dn, 1)
+    return pre / (1.0 + np.exp(-pre)), pre
+
+
+def _seq_projections(us, Wx, Wdt):
+    """x_proj and dt_proj of per-path sequences us (Bn, 4, D, L), as path_projections."""
+    R = Wdt.shape[2]
+    N = (Wx.shape[1] - R) // 2
+    x_dbl = np.einsum("bkdl,kcd->bkcl", us, Wx)
+    delta = np.einsum("kdr,bkrl->bkdl", Wdt, x_dbl[:, :, :R])
+    return delta, np.ascontiguousarray(x_dbl[:, :, R:R + N]), np.ascontiguousarray(x_dbl[:, :, R + N:]), x_dbl
+
+
+def ss2d_forward_proj_conv(x, conv_weight, conv_bias, x_proj_weight, dt_proj_weight, dt_proj_bias, A, D=None,
+                           delta_softplus=True):
+    """SS2D forward with the whole per-path producer of MambaInnerFn.forward: u_k = path_conv,
+    x_dbl = x_proj(u_k), delta = dt_proj.weight @ x_dbl[:R], B, C from x_dbl, the S6 scan of
+    every path on u_k, and CrossMerge.  Returns y (Bn, D, H, W)."""
+    x, Wx, Wdt = _f64(x), _f64(x_proj_weight), _f64(dt_proj_weight)
+    Bn, Dn, H, W = x.shape
+    L = H * W
+    u, _ = path_conv(x, conv_weight, conv_bias)
+    delta, Bm, Cm, _ = _seq_projections(u, Wx, Wdt)
+    ys = selective_scan_fwd(u.reshape(Bn, K_PATHS * Dn, L), delta.reshape(Bn, K_PATHS * Dn, L), A, Bm, Cm, D,
+                            dt_proj_bias, delta_softplus)
+    return cross_merge(ys.reshape(Bn, K_PATHS, Dn, L), H, W)
+
+
+def ss2d_backward_proj_conv(x, conv_weight, conv_bias, x_proj_weight, dt_proj_weight, dt_proj_bias, A, D,
+                            delta_softplus, dy):
+    """Gradients of ss2d_forward_proj_conv, as MambaInnerFn.backward takes them: the scan's
+    backward on (u, delta, B, C) with dout = dy along every path; the projections' gradients as
+    ss2d_backward_proj; du_k = the scan's du + x_proj.weight^T dx_dbl; then the conv's backward
+    (causal_conv1d_bwd with SiLU): dpre = du * silu'(pre), d conv_weight[k, d, j] = sum over batch
+    and steps of dpre[l] x_k[l - (W-1) + j], d conv_bias = sum of dpre, and dx_k[m] =
+    sum_j w[k, d, j] dpre[m + (W-1) - j], merged along the paths.
+    Returns dict dx, dconv_weight, dconv_bias, dx_proj_weight, ddt_proj_weight, ddt_proj_bias, dA, dD."""
+    x, w, Wx, Wdt, dy = _f64(x), _f64(conv_weight), _f64(x_proj_weight), _f64(dt_proj_weight), _f64(dy)
+    Bn, Dn, H, W = x.shape
+    L = H * W
+    R = Wdt.shape[2]
+    Wc = w.shape[2]
+    u, pre = path_conv(x, conv_weight, conv_bias)
+    delta, Bm, Cm, x_dbl = _seq_projections(u, Wx, Wdt)
+    g = selective_scan_bwd(u.reshape(Bn, K_PATHS * Dn, L), delta.reshape(Bn, K_PATHS * Dn, L), A, Bm, Cm, D,
+                           dt_proj_bias, delta_softplus, cross_scan(dy).reshape(Bn, K_PATHS * Dn, L))
+    ddelta = g["ddelta"].reshape(Bn, K_PATHS, Dn, L)
+    dx_dbl = np.concatenate([np.einsum("kdr,bkdl->bkrl", Wdt, ddelta), g["dB"], g["dC"]], axis=2)
+    ddt_proj_weight = np.einsum("bkdl,bkrl->kdr", ddelta, x_dbl[:, :, :R])
+    dx_proj_weight = np.einsum("bkcl,bkdl->kcd", dx_dbl, u)
+    du = g["du"].reshape(Bn, K_PATHS, Dn, L) + np.einsum("kcd,bkcl->bkdl", Wx, dx_dbl)
+    sig = 1.0 / (1.0 + np.exp(-pre))
+    dpre = du * sig * (1.0 + pre * (1.0 - sig))                # silu'(p) = s (1 + p (1 - s))
+    xs = cross_scan(x)
+    dconv_weight = np.empty_like(w)
+    dxs = np.zeros_like(xs)
+    for j in range(Wc):
+        s = Wc - 1 - j
+        dconv_weight[:, :, j] = np.einsum("bkdl,bkdl->kd", dpre[..., s:], xs[..., :L - s])
+        dxs[..., :L - s] += w[None, :, :, j, None] * dpre[..., s:]
+    dconv_bias = dpre.sum(axis=(0, 3)).reshape(K_PATHS * Dn) if conv_bias is not None else None
+    return dict(dx=cross_merge(dxs, H, W), dconv_weight=dconv_weight, dconv_bias=dconv_bias,
+                dx_proj_weight=dx_proj_weight, ddt_proj_weight=ddt_proj_weight, ddt_proj_bias=g["ddelta_bias"],
+                dA=g["dA"], dD=g["dD"])
+
+
 # ---------------------------------------------------------------- path sets
 
 def cross_paths(H: int, W: int):

@@ -187,12 +187,14 @@ def dt_rank_of(dim: int) -> int:
     return max(1, math.ceil((dim // 2) / 16))
 
 
-def make_proj_inputs(w: Workload, seed: int = 0, device="cpu"):
+def make_proj_inputs(w: Workload, seed: int = 0, device="cpu", d_conv: int = 0):
     """Inputs of the SS2D forward with its producer (x_proj, dt_proj per path), drawn as
     Mamba.__init__ initialises them: x ~ N(0,1) (B, D, H, W); x_proj weight (4, R+2N, D)
     ~ U(-1/sqrt(D), 1/sqrt(D)) (nn.Linear's default); dt_proj weight (4, D, R) ~
     U(-R^-0.5, R^-0.5) (dt_init "random", dt_scale 1); dt_proj bias, A and D as in make_inputs.
-    Draw order: x, x_proj weight, dt_proj weight, dt."""
+    Draw order: x, x_proj weight, dt_proj weight, dt.  With d_conv > 0, the per-path causal
+    depthwise conv follows, as nn.Conv1d(D, D, d_conv, groups=D) initialises it: weight (4, D,
+    d_conv) and bias (4D), both ~ U(-1/sqrt(d_conv), 1/sqrt(d_conv)), drawn after the rest."""
     g = torch.Generator(device=device)
     g.manual_seed(int(seed) + 3000)
     f32 = dict(dtype=torch.float32, device=device, generator=g)
@@ -212,6 +214,10 @@ def make_proj_inputs(w: Workload, seed: int = 0, device="cpu"):
     A = A_row.unsqueeze(0).repeat(K_PATHS * Dn, 1).contiguous()
     out = dict(x=x, x_proj_weight=Wx, dt_proj_weight=Wdt, dt_proj_bias=bias, A=A,
                D=torch.ones(K_PATHS * Dn, dtype=torch.float32, device=device), R=R)
+    if d_conv > 0:
+        bc = 1.0 / math.sqrt(d_conv)
+        out["conv_weight"] = (torch.rand((K_PATHS, Dn, d_conv), **f32) * 2 - 1) * bc
+        out["conv_bias"] = (torch.rand((K_PATHS * Dn,), **f32) * 2 - 1) * bc
     if w.dtype == "bf16":
         out["x"] = out["x"].to(torch.bfloat16)
     return out

@@ -759,3 +759,82 @@ def test_input_recipe_statistics():
     again = ss2d_inputs.make_inputs(w, seed=0, with_dy=True)
     for k in inp:
         assert torch.equal(inp[k], again[k])
+
+
+# ------------------------------------------- causal depthwise conv per path
+
+def _conv_problem(seed, Bn=1, Dn=3, H=3, W=4, N=3, R=2, Wc=4):
+    p = _proj_problem(seed, Bn=Bn, Dn=Dn, H=H, W=W, N=N, R=R)
+    rng = _rng(seed + 1000)
+    p["cw"] = rng.standard_normal((4, Dn, Wc)) / np.sqrt(Wc)
+    p["cb"] = 0.3 * rng.standard_normal(4 * Dn)
+    return p
+
+
+def test_path_conv_matches_numpy_convolve(oracle):
+    from scipy.special import expit
+    p = _conv_problem(80, Bn=2, Dn=3, H=4, W=5)
+    u, pre = oracle.path_conv(p["x"], p["cw"], p["cb"])
+    xs = oracle.cross_scan(p["x"])
+    L = xs.shape[-1]
+    for b in range(2):
+        for k in range(4):
+            for d in range(3):
+                # causal cross-correlation = convolution with the reversed taps, first L outputs
+                ref = np.convolve(xs[b, k, d], p["cw"][k, d, ::-1])[:L] + p["cb"][k * 3 + d]
+                np.testing.assert_allclose(pre[b, k, d], ref, rtol=1e-13, atol=1e-13)
+                np.testing.assert_allclose(u[b, k, d], ref * expit(ref), rtol=1e-13, atol=1e-13)
+
+
+def test_path_conv_is_causal_along_each_path(oracle):
+    p = _conv_problem(81, Dn=2, H=3, W=5, Wc=3)
+    u0, _ = oracle.path_conv(p["x"], p["cw"], p["cb"])
+    H, W, L = 3, 5, 15
+    for pix in (0, 7, 14):
+        x = p["x"].copy()
+        x[0, 1, pix // W, pix % W] += 1.0
+        u1, _ = oracle.path_conv(x, p["cw"], p["cb"])
+        for k in range(4):
+            step = [oracle.path_pixel(k, l, H, W) for l in range(L)].index(pix)
+            changed = np.nonzero(np.abs(u1[0, k, 1] - u0[0, k, 1]) > 0)[0]
+            assert set(changed) <= set(range(step, min(L, step + 3))) and step in set(changed)
+            assert np.array_equal(u1[0, k, 0], u0[0, k, 0])  # other channels untouched
+
+
+def test_forward_proj_conv_with_last_tap_is_forward_proj_of_silu(oracle):
+    # one-hot weight on the newest tap and no bias: u_k = silu(x) read along path k
+    p = _conv_problem(82, Bn=2, Dn=3, H=3, W=4)
+    w = np.zeros_like(p["cw"])
+    w[:, :, -1] = 1.0
+    y = oracle.ss2d_forward_proj_conv(p["x"], w, None, p["Wx"], p["Wdt"], p["bias"], p["A"], p["D"], True)
+    xs = p["x"] / (1.0 + np.exp(-p["x"]))
+    ref = oracle.ss2d_forward_proj(xs, p["Wx"], p["Wdt"], p["bias"], p["A"], p["D"], True)
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_projection_conv_backward_matches_central_differences(oracle):
+    p = _conv_problem(83, Bn=1, Dn=2, H=3, W=3, N=2, R=2, Wc=3)
+    rng = _rng(84)
+    dy = rng.standard_normal(p["x"].shape)
+    g = oracle.ss2d_backward_proj_conv(p["x"], p["cw"], p["cb"], p["Wx"], p["Wdt"], p["bias"], p["A"], p["D"], True,
+                                       dy)
+
+    def loss():
+        return float(np.sum(oracle.ss2d_forward_proj_conv(p["x"], p["cw"], p["cb"], p["Wx"], p["Wdt"], p["bias"],
+                                                          p["A"], p["D"]) * dy))
+
+    names = dict(x="dx", cw="dconv_weight", cb="dconv_bias", Wx="dx_proj_weight", Wdt="ddt_proj_weight",
+                 bias="ddt_proj_bias", A="dA", D="dD")
+    for name, gname in names.items():
+        flat = p[name].reshape(-1)
+        for i in rng.choice(flat.size, size=min(flat.size, 8), replace=False):
+            theta = flat[i]
+            h = 1e-6 * max(1.0, abs(theta))
+            flat[i] = theta + h
+            lp = loss()
+            flat[i] = theta - h
+            lm = loss()
+            flat[i] = theta
+            fd = (lp - lm) / (2 * h)
+            an = g[gname].reshape(-1)[i]
+            assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (name, i, fd, an)
