@@ -25,6 +25,8 @@ silu(z)): a step is one bidirectional forward (plus its backward under `--backwa
 `--proj` times the fused forward with its producer: per-path x_proj, then the scan computing
 dt = softplus(dt_proj . x_dbl[:R] + bias) per step (MambaInnerFn.forward's projections);
 with `--backward` each step adds the backward through the scan and both projections.
+`--proj --conv 4` puts the per-path causal depthwise conv with SiLU (MambaInnerFn's
+causal_conv1d, width 4) in front of the producer; the scan then runs in sequence form.
 
 `--backward` adds the fused backward to every step; `--gate` times the scan in its
 sequence form instead, u (B, 4D, L) with the output gate out * silu(z) and the last
@@ -337,7 +339,7 @@ def run_gpu(args, world, rank, local):
     dev = torch.device("cuda", local)
     bidir = w.kind == "bidir"
     if args.proj:
-        inp = ss2d_inputs.make_proj_inputs(w, seed=shard_seed(args.workload, rank), device=dev)
+        inp = ss2d_inputs.make_proj_inputs(w, seed=shard_seed(args.workload, rank), device=dev, d_conv=args.conv)
     elif bidir:
         inp = ss2d_inputs.make_bimamba_inputs(w, seed=shard_seed(args.workload, rank), device=dev,
                                               with_dy=args.backward, with_z=True)
@@ -357,6 +359,11 @@ def run_gpu(args, world, rank, local):
         npj = ss.workspace_bytes(w.batch, w.dim, w.height, w.width, w.d_state, ss.OP_FORWARD_PROJ, w.torch_dtype)
         wsp = torch.empty(max(npj, 1), dtype=torch.uint8, device=dev)
 
+        if args.conv:
+            cargs = (inp["x"], inp["conv_weight"], inp["conv_bias"]) + pargs[1:]
+            npc = ss.workspace_bytes(w.batch, w.dim, w.height, w.width, w.d_state, ss.OP_FORWARD_PROJ_CONV,
+                                     w.torch_dtype)
+            wspc = torch.empty(max(npc, 1), dtype=torch.uint8, device=dev)
         if args.backward:
             gdy = torch.Generator(device=dev)
             gdy.manual_seed(shard_seed(args.workload, rank) + 7000)
@@ -365,11 +372,25 @@ def run_gpu(args, world, rank, local):
                                      w.torch_dtype)
             wsbp = torch.empty(max(nbp, 1), dtype=torch.uint8, device=dev)
 
+            if args.conv:
+                nbc = ss.workspace_bytes(w.batch, w.dim, w.height, w.width, w.d_state, ss.OP_BACKWARD_PROJ_CONV,
+                                         w.torch_dtype)
+                wsbc = torch.empty(max(nbc, 1), dtype=torch.uint8, device=dev)
+
+                def step():
+                    # the same with the per-path causal conv in front of the producer
+                    _, xd, cs = ss.ss2d_forward_proj_conv(*cargs, True, out=y, return_x_dbl=True,
+                                                          return_chunk_states=True, workspace=wspc)
+                    ss.ss2d_backward_proj_conv(*cargs, xd, dy, True, chunk_states=cs, workspace=wsbc)
+            else:
+                def step():
+                    # forward keeping x_dbl and the chunk states, then the backward through scan and producer
+                    _, xd, cs = ss.ss2d_forward_proj(*pargs, True, out=y, return_x_dbl=True,
+                                                     return_chunk_states=True, workspace=wsp)
+                    ss.ss2d_backward_proj(*pargs, xd, dy, True, chunk_states=cs, workspace=wsbp)
+        elif args.conv:
             def step():
-                # forward keeping x_dbl and the chunk states, then the backward through scan and producer
-                _, xd, cs = ss.ss2d_forward_proj(*pargs, True, out=y, return_x_dbl=True, return_chunk_states=True,
-                                                 workspace=wsp)
-                ss.ss2d_backward_proj(*pargs, xd, dy, True, chunk_states=cs, workspace=wsbp)
+                ss.ss2d_forward_proj_conv(*cargs, True, out=y, workspace=wspc)
         else:
             def step():
                 ss.ss2d_forward_proj(*pargs, True, out=y, workspace=wsp)
@@ -487,7 +508,9 @@ def run_gpu(args, world, rank, local):
     peaks = load_peaks()
     clocks = sampler.summary() if sampler else None
     # algorithmic bytes of the dominant kernel: the backward's when a backward runs in the step
-    if args.proj and not args.backward:
+    if args.proj and args.conv and not args.backward:
+        alg_bytes = seq_fwd_algorithmic_bytes(w, gate=False)  # the scan runs in sequence form on u
+    elif args.proj and not args.backward:
         alg_bytes = proj_algorithmic_bytes(w, inp["R"])
     elif bidir:
         alg_bytes = bidir_algorithmic_bytes(w, args.backward)
@@ -531,7 +554,8 @@ def run_gpu(args, world, rank, local):
                    + (" (sequence form, gate z + last state)" if args.gate else "")
                    + (" (bidirectional, gate z)" if bidir else "")
                    + (f" ({args.paths} paths)" if args.paths != "cross" else "")
-                   + (" (with the per-path x_proj/dt_proj producer)" if args.proj else ""),
+                   + (" (with the per-path x_proj/dt_proj producer)" if args.proj else "")
+                   + (f" (and its per-path causal conv, width {args.conv})" if args.proj and args.conv else ""),
                    "l2": f"inputs {alg_bytes / 1e9:.2f} GB > 126 MB L2, no flush needed"},
         # the dominant (scan) kernel is bound by its exponentials on the SFU: that is the roofline;
         # the HBM view the metric names is reported beside it
@@ -639,6 +663,8 @@ def main(argv=None):
                     help="time the sequence-form scan with the output gate z and the last state instead")
     ap.add_argument("--paths", choices=["cross", "diagonal"], default="cross",
                     help="path set of the fused SS2D (default: the cross scan)")
+    ap.add_argument("--conv", type=int, default=0, metavar="D_CONV",
+                    help="with --proj: put the per-path causal depthwise conv (width D_CONV, SiLU) in front")
     ap.add_argument("--proj", action="store_true",
                     help="time the fused forward with its per-path x_proj/dt_proj producer instead")
     ap.add_argument("--no-e2e", action="store_true")

@@ -91,7 +91,9 @@ typedef enum {
     SS2D_OP_FORWARD_TABLE = 6,
     SS2D_OP_BACKWARD_TABLE = 7,
     SS2D_OP_FORWARD_PROJ = 8,
-    SS2D_OP_BACKWARD_PROJ = 9
+    SS2D_OP_BACKWARD_PROJ = 9,
+    SS2D_OP_FORWARD_PROJ_CONV = 10,
+    SS2D_OP_BACKWARD_PROJ_CONV = 11
 } ss2d_op_t;
 
 /* Path sets that ss2d_path_tables generates (paths 2 and 3 are always 0 and 1 walked backwards). */
@@ -298,6 +300,53 @@ SS2D_API ss2d_status_t ss2d_backward_proj(const ss2d_desc_t *desc, int dt_rank, 
                                           const void *dy, void *dx, float *dx_proj_weight,
                                           float *ddt_proj_weight, float *ddt_proj_bias, float *dA, float *dD,
                                           void *workspace, size_t workspace_bytes, ss2d_stream_t stream);
+
+/*
+ * The producer with its causal depthwise conv: MambaInnerFn.forward ("vision mamba-yolov8",
+ * section 2) passes its input through causal_conv1d_fwd(x, weight, bias, True) (a depthwise conv
+ * of width d_conv over the current and previous steps, then SiLU) before x_proj.  As the Visual
+ * Mamba page's SS2D runs one Mamba block per scan direction, every path k convolves x read along
+ * its own step order with its own weights:
+ *   u_k[d, l] = silu(conv_bias[k*D + d] + sum_j conv_weight[k, d, j] x_k[d, l - (d_conv-1) + j])
+ * (x_k = 0 before step 0), then the producer of ss2d_forward_proj on u_k (x_proj, dt_proj, B and
+ * C from x_dbl), the S6 scan of every path on u_k, and CrossMerge.
+ * d_conv           : 1..4
+ * conv_weight      : (4, D, d_conv) fp32;  conv_bias: (4D) fp32 or NULL
+ * other arguments  : as for ss2d_forward_proj (x_dbl written, in each path's step order)
+ * workspace        : ss2d_workspace_bytes(desc, SS2D_OP_FORWARD_PROJ_CONV) bytes
+ * Errors: SS2D_ERR_SHAPE for dt_rank outside [1, 32] or d_conv outside [1, 4]; otherwise as for
+ * ss2d_forward_proj.
+ */
+SS2D_API ss2d_status_t ss2d_forward_proj_conv(const ss2d_desc_t *desc, int dt_rank, int d_conv, const void *x,
+                                              const float *conv_weight, const float *conv_bias,
+                                              const float *x_proj_weight, const float *dt_proj_weight,
+                                              const float *dt_proj_bias, const float *A, const float *D,
+                                              int delta_softplus, void *y, void *x_dbl, float *chunk_states,
+                                              void *workspace, size_t workspace_bytes, ss2d_stream_t stream);
+
+/*
+ * Backward of ss2d_forward_proj_conv (MambaInnerFn.backward with causal_conv1d_bwd): the scan's
+ * gradients, the producer's as in ss2d_backward_proj, then the conv's: dpre = du * silu'(pre),
+ * dconv_weight[k, d, j] = sum over batch and steps of dpre[l] x_k[l - (d_conv-1) + j],
+ * dconv_bias = sum of dpre, and dx = the per-path sum_j w[k, d, j] dpre[m + (d_conv-1) - j] merged
+ * along the paths.  u is made again from x; the sums run in a fixed order (deterministic), in fp32.
+ * x_dbl, chunk_states: as ss2d_forward_proj_conv wrote them (chunk_states may be NULL)
+ * dy (B, D, H, W) out_dtype;  dx (B, D, H, W) in_dtype, written
+ * dconv_weight (4, D, d_conv), dconv_bias (4D; NULL exactly when conv_bias is NULL), and the
+ * other gradients as for ss2d_backward_proj: fp32, written
+ * workspace        : ss2d_workspace_bytes(desc, SS2D_OP_BACKWARD_PROJ_CONV) bytes (sized for dt
+ *                    rank 32 and d_conv 4)
+ * Errors: as for ss2d_forward_proj_conv and ss2d_backward_proj.
+ */
+SS2D_API ss2d_status_t ss2d_backward_proj_conv(const ss2d_desc_t *desc, int dt_rank, int d_conv, const void *x,
+                                               const float *conv_weight, const float *conv_bias,
+                                               const float *x_proj_weight, const float *dt_proj_weight,
+                                               const float *dt_proj_bias, const float *A, const float *D,
+                                               int delta_softplus, const void *x_dbl, const float *chunk_states,
+                                               const void *dy, void *dx, float *dconv_weight, float *dconv_bias,
+                                               float *dx_proj_weight, float *ddt_proj_weight, float *ddt_proj_bias,
+                                               float *dA, float *dD, void *workspace, size_t workspace_bytes,
+                                               ss2d_stream_t stream);
 
 /* ------------------------------------------------------------ path sets -- */
 

@@ -37,6 +37,7 @@ __all__ = [
     "SelectiveScanFunction", "ss2d_forward", "bimamba_forward", "bimamba_backward", "BiMambaFunction",
     "bimamba_scan", "path_tables", "cross_scan_table", "cross_merge_table", "ss2d_forward_table",
     "ss2d_backward_table", "PATHS_CROSS", "PATHS_DIAGONAL", "ss2d_forward_proj", "ss2d_backward_proj", "OP_BACKWARD_PROJ",
+    "ss2d_forward_proj_conv", "ss2d_backward_proj_conv", "OP_FORWARD_PROJ_CONV", "OP_BACKWARD_PROJ_CONV",
     "ss2d_backward", "SS2DFunction", "ss2d", "workspace_bytes", "chunk_states_elems", "launch_count",
     "library_path", "CHUNK_LEN", "trace_events",
 ]
@@ -51,6 +52,7 @@ CHUNK_LEN = 16  # SS2D_CHUNK_LEN
 F32, BF16 = 0, 1
 OP_SELECTIVE_SCAN_BWD, OP_FORWARD, OP_BACKWARD, OP_BIMAMBA_FORWARD, OP_BIMAMBA_BACKWARD = 1, 2, 3, 4, 5
 OP_FORWARD_TABLE, OP_BACKWARD_TABLE, OP_FORWARD_PROJ, OP_BACKWARD_PROJ = 6, 7, 8, 9
+OP_FORWARD_PROJ_CONV, OP_BACKWARD_PROJ_CONV = 10, 11
 PATHS_CROSS, PATHS_DIAGONAL = 0, 1
 _STATUS = {0: "SS2D_OK", 1: "SS2D_ERR_NULL", 2: "SS2D_ERR_SHAPE", 3: "SS2D_ERR_DTYPE", 4: "SS2D_ERR_ALIGN",
            5: "SS2D_ERR_WORKSPACE", 6: "SS2D_ERR_LAUNCH", 7: "SS2D_ERR_TIMEOUT", 8: "SS2D_ERR_DEVICE"}
@@ -100,6 +102,9 @@ def _load():
         lib.ss2d_path_tables.argtypes = [D, i, P, P]
         lib.ss2d_forward_proj.argtypes = [D, i, P, P, P, P, P, P, i, P, P, P, P, sz, P]
         lib.ss2d_backward_proj.argtypes = [D, i, P, P, P, P, P, P, i, P, P, P, P, P, P, P, P, P, P, sz, P]
+        lib.ss2d_forward_proj_conv.argtypes = [D, i, i, P, P, P, P, P, P, P, P, i, P, P, P, P, sz, P]
+        lib.ss2d_backward_proj_conv.argtypes = [D, i, i, P, P, P, P, P, P, P, P, i, P, P, P, P, P, P, P, P, P, P,
+                                                P, P, sz, P]
         lib.ss2d_cross_scan_table.argtypes = [D, P, P, P, P]
         lib.ss2d_cross_merge_table.argtypes = [D, P, P, P, P]
         lib.ss2d_forward_table.argtypes = [D, P, P, P, P, P, P, P, P, i, P, P, P, sz, P]
@@ -111,7 +116,7 @@ def _load():
                      "ss2d_selective_scan_fwd_ex", "ss2d_selective_scan_bwd_ex", "ss2d_forward", "ss2d_backward",
                      "ss2d_bimamba_forward", "ss2d_bimamba_backward", "ss2d_path_tables", "ss2d_cross_scan_table",
                      "ss2d_cross_merge_table", "ss2d_forward_table", "ss2d_backward_table", "ss2d_forward_proj",
-                     "ss2d_backward_proj"):
+                     "ss2d_backward_proj", "ss2d_forward_proj_conv", "ss2d_backward_proj_conv"):
             getattr(lib, name).restype = ctypes.c_int
         lib.ss2d_workspace_bytes.argtypes = [D, i]
         lib.ss2d_workspace_bytes.restype = sz
@@ -715,3 +720,84 @@ def ss2d_backward_proj(x, x_proj_weight, dt_proj_weight, dt_proj_bias, A, D, x_d
                                 _p(dbias), _p(dA), _p(dD), _p(workspace), nbytes, _stream(x))
     _check(st, "ss2d_backward_proj")
     return dict(dx=dx, dx_proj_weight=dWx, ddt_proj_weight=dWdt, ddt_proj_bias=dbias, dA=dA, dD=dD)
+
+
+def _conv_args(x, conv_weight, conv_bias, x_proj_weight, dt_proj_weight, dt_proj_bias, A, D, what):
+    x = _c(x)
+    cw = _c(conv_weight, torch.float32)
+    cb = _c(conv_bias, torch.float32) if conv_bias is not None else None
+    Wx = _c(x_proj_weight, torch.float32)
+    Wdt = _c(dt_proj_weight, torch.float32)
+    A, D, bias = _params(A, D, dt_proj_bias)
+    Bn, Dn, H, W = x.shape
+    N = A.shape[1]
+    R = Wdt.shape[2]
+    if Wx.shape != (4, R + 2 * N, Dn) or Wdt.shape != (4, Dn, R):
+        raise ValueError(f"{what}: x_proj_weight must be (4, R+2N, D) and dt_proj_weight (4, D, R)")
+    if cw.dim() != 3 or cw.shape[:2] != (4, Dn) or (cb is not None and cb.shape != (4 * Dn,)):
+        raise ValueError(f"{what}: conv_weight must be (4, D, d_conv) and conv_bias (4D)")
+    return x, cw, cb, Wx, Wdt, A, D, bias, R, N
+
+
+def ss2d_forward_proj_conv(x, conv_weight, conv_bias, x_proj_weight, dt_proj_weight, dt_proj_bias, A, D=None,
+                           delta_softplus=True, out=None, out_dtype=None, return_x_dbl=False,
+                           return_chunk_states=False, workspace=None):
+    """SS2D forward with the whole per-path producer of MambaInnerFn.forward: a causal depthwise
+    conv of width d_conv with SiLU along every path (conv_weight (4, D, d_conv), conv_bias (4D)),
+    then x_proj, dt_proj, the scan of every path and CrossMerge.  Returns y [, x_dbl] [, chunk_states]."""
+    x, cw, cb, Wx, Wdt, A, D, bias, R, N = _conv_args(x, conv_weight, conv_bias, x_proj_weight, dt_proj_weight,
+                                                      dt_proj_bias, A, D, "ss2d_forward_proj_conv")
+    Bn, Dn, H, W = x.shape
+    out_dtype = out_dtype or x.dtype
+    if out is None:
+        out = torch.empty((Bn, Dn, H, W), dtype=out_dtype, device=x.device)
+    x_dbl = torch.empty((Bn, 4, R + 2 * N, H * W), dtype=x.dtype, device=x.device)
+    cs = None
+    if return_chunk_states:
+        cs = torch.empty((Bn, 4 * Dn, -(-(H * W) // CHUNK_LEN), N), dtype=torch.float32, device=x.device)
+    d = _desc(Bn, Dn, H, W, N, x.dtype, out.dtype)
+    lib = _load()
+    nbytes = int(lib.ss2d_workspace_bytes(ctypes.byref(d), OP_FORWARD_PROJ_CONV))
+    if workspace is None or workspace.numel() < nbytes:
+        workspace = _workspace(nbytes, x.device)
+    st = lib.ss2d_forward_proj_conv(ctypes.byref(d), int(R), int(cw.shape[2]), _p(x), _p(cw), _p(cb), _p(Wx),
+                                    _p(Wdt), _p(bias), _p(A), _p(D), int(bool(delta_softplus)), _p(out), _p(x_dbl),
+                                    _p(cs), _p(workspace), nbytes, _stream(x))
+    _check(st, "ss2d_forward_proj_conv")
+    extra = ([x_dbl] if return_x_dbl else []) + ([cs] if return_chunk_states else [])
+    return (out, *extra) if extra else out
+
+
+def ss2d_backward_proj_conv(x, conv_weight, conv_bias, x_proj_weight, dt_proj_weight, dt_proj_bias, A, D, x_dbl,
+                            dy, delta_softplus=True, chunk_states=None, workspace=None):
+    """Backward of ss2d_forward_proj_conv.  Returns a dict with dx, dconv_weight (4, D, d_conv),
+    dconv_bias (4D or None), dx_proj_weight, ddt_proj_weight, ddt_proj_bias, dA, dD (fp32 but dx)."""
+    x, cw, cb, Wx, Wdt, A, D, bias, R, N = _conv_args(x, conv_weight, conv_bias, x_proj_weight, dt_proj_weight,
+                                                      dt_proj_bias, A, D, "ss2d_backward_proj_conv")
+    Bn, Dn, H, W = x.shape
+    x_dbl = _c(x_dbl, x.dtype)
+    if x_dbl.shape != (Bn, 4, R + 2 * N, H * W):
+        raise ValueError("ss2d_backward_proj_conv: x_dbl must be (Bn, 4, R+2N, H*W) in x's dtype")
+    dy = _c(dy)
+    cs = _c(chunk_states, torch.float32) if chunk_states is not None else None
+    f32 = dict(dtype=torch.float32, device=x.device)
+    dx = torch.empty_like(x)
+    dcw = torch.empty(tuple(cw.shape), **f32)
+    dcb = torch.empty((4 * Dn,), **f32) if cb is not None else None
+    dWx = torch.empty((4, R + 2 * N, Dn), **f32)
+    dWdt = torch.empty((4, Dn, R), **f32)
+    dbias = torch.empty((4 * Dn,), **f32) if bias is not None else None
+    dA = torch.empty((4 * Dn, N), **f32)
+    dD = torch.empty((4 * Dn,), **f32) if D is not None else None
+    d = _desc(Bn, Dn, H, W, N, x.dtype, dy.dtype)
+    lib = _load()
+    nbytes = int(lib.ss2d_workspace_bytes(ctypes.byref(d), OP_BACKWARD_PROJ_CONV))
+    if workspace is None or workspace.numel() < nbytes:
+        workspace = _workspace(nbytes, x.device)
+    st = lib.ss2d_backward_proj_conv(ctypes.byref(d), int(R), int(cw.shape[2]), _p(x), _p(cw), _p(cb), _p(Wx),
+                                     _p(Wdt), _p(bias), _p(A), _p(D), int(bool(delta_softplus)), _p(x_dbl), _p(cs),
+                                     _p(dy), _p(dx), _p(dcw), _p(dcb), _p(dWx), _p(dWdt), _p(dbias), _p(dA), _p(dD),
+                                     _p(workspace), nbytes, _stream(x))
+    _check(st, "ss2d_backward_proj_conv")
+    return dict(dx=dx, dconv_weight=dcw, dconv_bias=dcb, dx_proj_weight=dWx, ddt_proj_weight=dWdt,
+                ddt_proj_bias=dbias, dA=dA, dD=dD)

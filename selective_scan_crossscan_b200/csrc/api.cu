@@ -1,5 +1,6 @@
 // api.cu -- the C ABI of libss2d (declared in include/ss2d.h): argument
 // validation on the host, workspace layout, and dispatch to the kernels.
+#include <algorithm>
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
@@ -146,6 +147,26 @@ static size_t proj_bwd_ws_bytes(const LaunchShape &s, ss2d_dtype_t in, ss2d_dtyp
            round64((size_t)kPaths * s.B * proj_bwd_chunks(s) * rn * s.D * sizeof(float)) +
            round64(scan_bwd_workspace_bytes(s));
 }
+// producer-with-conv forward workspace: [transposed x] [u (B,4D,L)] [delta] [B, C (B,4,N,L)]
+// [fp32 per-path outputs (B,4D,L)] [segment summaries]
+static size_t conv_fwd_ws_bytes(const LaunchShape &s, ss2d_dtype_t in) {
+    const size_t seq = (size_t)s.B * kPaths * s.D * s.L, img = (size_t)s.B * s.D * s.L;
+    const size_t bc = (size_t)s.B * kPaths * s.N * s.L;
+    return round64(img * elem_size(in)) + 2 * round64(seq * elem_size(in)) + 2 * round64(bc * elem_size(in)) +
+           round64(seq * sizeof(float)) + round64(scan_fwd_workspace_bytes(s));
+}
+// producer-with-conv backward workspace: [transposed x] [u] [dy along the paths] [delta] [ddelta]
+// [B, C, dB, dC] [fp32 du (B,4D,L)] [fp32 dx along the paths] [fp32 dx_dbl] [partials] [scan backward]
+// (sized for dt rank 32 and d_conv 4)
+static size_t conv_bwd_ws_bytes(const LaunchShape &s, ss2d_dtype_t in, ss2d_dtype_t out) {
+    const size_t seq = (size_t)s.B * kPaths * s.D * s.L, img = (size_t)s.B * s.D * s.L;
+    const size_t bc = (size_t)s.B * kPaths * s.N * s.L, rn = (size_t)kProjRMax + 2 * s.N;
+    const size_t part = std::max((size_t)kPaths * s.B * proj_bwd_chunks(s) * rn * s.D, path_conv_partial_floats(s, 4));
+    return round64(img * elem_size(in)) + round64(seq * elem_size(in)) + round64(seq * elem_size(out)) +
+           2 * round64(seq * elem_size(in)) + 4 * round64(bc * elem_size(in)) + 2 * round64(seq * sizeof(float)) +
+           round64((size_t)s.B * kPaths * rn * s.L * sizeof(float)) + round64(part * sizeof(float)) +
+           round64(scan_bwd_workspace_bytes(s));
+}
 static ss2d_status_t check_table_shape(const ss2d_desc_t *desc) {
     return desc->height * desc->width < ((int64_t)1 << 31) ? SS2D_OK : SS2D_ERR_SHAPE;
 }
@@ -203,6 +224,8 @@ size_t ss2d_workspace_bytes(const ss2d_desc_t *desc, int op) {
             return fwd_ws_bytes(s, desc->in_dtype) + round64((size_t)s.B * kPaths * s.D * s.L * elem_size(desc->in_dtype));
         case SS2D_OP_BACKWARD_TABLE: return table_bwd_ws_bytes(s, desc->in_dtype, desc->out_dtype);
         case SS2D_OP_BACKWARD_PROJ: return proj_bwd_ws_bytes(s, desc->in_dtype, desc->out_dtype);
+        case SS2D_OP_FORWARD_PROJ_CONV: return conv_fwd_ws_bytes(s, desc->in_dtype);
+        case SS2D_OP_BACKWARD_PROJ_CONV: return conv_bwd_ws_bytes(s, desc->in_dtype, desc->out_dtype);
         default: return (size_t)-1;
     }
 }
@@ -490,6 +513,181 @@ ss2d_status_t ss2d_backward_proj(const ss2d_desc_t *desc, int dt_rank, const voi
     SS2D_TRY(from_cuda(launch_proj_bwd_dwx(s, in, dxdbl, x, xT, RN, part, dx_proj_weight, st)));
     SS2D_TRY(from_cuda(launch_proj_bwd_du(s, dxdbl, x_proj_weight, RN, du_seq, st)));
     return from_cuda(launch_cross_merge(s, SS2D_F32, in, du_seq, dx, st));
+}
+
+ss2d_status_t ss2d_forward_proj_conv(const ss2d_desc_t *desc, int dt_rank, int d_conv, const void *x,
+                                     const float *conv_weight, const float *conv_bias, const float *x_proj_weight,
+                                     const float *dt_proj_weight, const float *dt_proj_bias, const float *A,
+                                     const float *D, int delta_softplus, void *y, void *x_dbl, float *chunk_states,
+                                     void *workspace, size_t workspace_bytes, ss2d_stream_t stream) {
+    SS2D_TRY(check_desc(desc));
+    if (dt_rank < 1 || dt_rank > kProjRMax || d_conv < 1 || d_conv > 4) return SS2D_ERR_SHAPE;
+    SS2D_TRY(need(x));
+    SS2D_TRY(need(conv_weight));
+    SS2D_TRY(optional(conv_bias));
+    SS2D_TRY(need(x_proj_weight));
+    SS2D_TRY(need(dt_proj_weight));
+    SS2D_TRY(optional(dt_proj_bias));
+    SS2D_TRY(need(A));
+    SS2D_TRY(optional(D));
+    SS2D_TRY(need(y));
+    SS2D_TRY(need(x_dbl));
+    SS2D_TRY(optional(chunk_states));
+    const LaunchShape s = shape_of(desc);
+    const ss2d_dtype_t in = desc->in_dtype;
+    if (!workspace || workspace_bytes < conv_fwd_ws_bytes(s, in)) return SS2D_ERR_WORKSPACE;
+    SS2D_TRY(optional(workspace));
+    SS2D_TRY(check_device());
+    const int R = dt_rank, RN = R + 2 * (int)s.N;
+    const size_t seq = (size_t)s.B * kPaths * s.D * s.L, img = (size_t)s.B * s.D * s.L;
+    const size_t bc = (size_t)s.B * kPaths * s.N * s.L, es = elem_size(in);
+    unsigned char *w = static_cast<unsigned char *>(workspace);
+    auto take = [&w](size_t bytes) {
+        void *p = w;
+        w += round64(bytes);
+        return p;
+    };
+    void *xT = take(img * es);
+    void *u = take(seq * es);
+    void *delta = take(seq * es);
+    void *Bm = take(bc * es);
+    void *Cm = take(bc * es);
+    float *ys = static_cast<float *>(take(seq * sizeof(float)));
+    void *seg = w;
+    cudaStream_t st = (cudaStream_t)stream;
+    SS2D_TRY(from_cuda(launch_transpose(s, in, x, xT, st)));
+    SS2D_TRY(from_cuda(launch_path_conv_fwd(s, in, x, xT, conv_weight, conv_bias, d_conv, u, st)));
+    SS2D_TRY(from_cuda(launch_xproj_seq(s, in, u, x_proj_weight, RN, x_dbl, st)));
+    SS2D_TRY(from_cuda(launch_dtproj(s, in, x_dbl, dt_proj_weight, R, RN, delta, st)));
+    const size_t row = (size_t)s.N * s.L * es, pitch = (size_t)RN * s.L * es, blocks = (size_t)s.B * kPaths;
+    const unsigned char *xd = static_cast<const unsigned char *>(x_dbl);
+    SS2D_TRY(from_cuda(cudaMemcpy2DAsync(Bm, row, xd + (size_t)R * s.L * es, pitch, row, blocks,
+                                         cudaMemcpyDeviceToDevice, st)));
+    SS2D_TRY(from_cuda(cudaMemcpy2DAsync(Cm, row, xd + (size_t)(R + s.N) * s.L * es, pitch, row, blocks,
+                                         cudaMemcpyDeviceToDevice, st)));
+    ScanFwdArgs a;
+    a.u = u;
+    a.delta = delta;
+    a.A = A;
+    a.Bm = Bm;
+    a.Cm = Cm;
+    a.Dv = D;
+    a.bias = dt_proj_bias;
+    a.softplus = delta_softplus != 0;
+    a.out = ys;
+    a.chunk_states = chunk_states;
+    a.from_image = false;
+    a.in_dtype = in;
+    a.out_dtype = SS2D_F32;
+    SS2D_TRY(from_cuda(launch_scan_fwd(s, a, seg, st)));
+    return from_cuda(launch_cross_merge(s, SS2D_F32, desc->out_dtype, ys, y, st));
+}
+
+ss2d_status_t ss2d_backward_proj_conv(const ss2d_desc_t *desc, int dt_rank, int d_conv, const void *x,
+                                      const float *conv_weight, const float *conv_bias, const float *x_proj_weight,
+                                      const float *dt_proj_weight, const float *dt_proj_bias, const float *A,
+                                      const float *D, int delta_softplus, const void *x_dbl,
+                                      const float *chunk_states, const void *dy, void *dx, float *dconv_weight,
+                                      float *dconv_bias, float *dx_proj_weight, float *ddt_proj_weight,
+                                      float *ddt_proj_bias, float *dA, float *dD, void *workspace,
+                                      size_t workspace_bytes, ss2d_stream_t stream) {
+    SS2D_TRY(check_desc(desc));
+    if (dt_rank < 1 || dt_rank > kProjRMax || d_conv < 1 || d_conv > 4) return SS2D_ERR_SHAPE;
+    SS2D_TRY(need(x));
+    SS2D_TRY(need(conv_weight));
+    SS2D_TRY(optional(conv_bias));
+    SS2D_TRY(need(x_proj_weight));
+    SS2D_TRY(need(dt_proj_weight));
+    SS2D_TRY(optional(dt_proj_bias));
+    SS2D_TRY(need(A));
+    SS2D_TRY(optional(D));
+    SS2D_TRY(need(x_dbl));
+    SS2D_TRY(optional(chunk_states));
+    SS2D_TRY(need(dy));
+    SS2D_TRY(need(dx));
+    SS2D_TRY(need(dconv_weight));
+    SS2D_TRY(need(dx_proj_weight));
+    SS2D_TRY(need(ddt_proj_weight));
+    SS2D_TRY(need(dA));
+    if ((D == nullptr) != (dD == nullptr)) return SS2D_ERR_NULL;
+    if ((dt_proj_bias == nullptr) != (ddt_proj_bias == nullptr)) return SS2D_ERR_NULL;
+    if ((conv_bias == nullptr) != (dconv_bias == nullptr)) return SS2D_ERR_NULL;
+    SS2D_TRY(optional(dD));
+    SS2D_TRY(optional(ddt_proj_bias));
+    SS2D_TRY(optional(dconv_bias));
+    const LaunchShape s = shape_of(desc);
+    const ss2d_dtype_t in = desc->in_dtype, out = desc->out_dtype;
+    if (!workspace || workspace_bytes < conv_bwd_ws_bytes(s, in, out)) return SS2D_ERR_WORKSPACE;
+    SS2D_TRY(optional(workspace));
+    SS2D_TRY(check_device());
+    const int R = dt_rank, RN = R + 2 * (int)s.N;
+    const size_t seq = (size_t)s.B * kPaths * s.D * s.L, img = (size_t)s.B * s.D * s.L;
+    const size_t bc = (size_t)s.B * kPaths * s.N * s.L, es = elem_size(in), rn = (size_t)kProjRMax + 2 * s.N;
+    unsigned char *w = static_cast<unsigned char *>(workspace);
+    auto take = [&w](size_t bytes) {
+        void *p = w;
+        w += round64(bytes);
+        return p;
+    };
+    void *xT = take(img * es);
+    void *u = take(seq * es);
+    void *g = take(seq * elem_size(out));
+    void *delta = take(seq * es);
+    void *ddelta = take(seq * es);
+    void *Bm = take(bc * es);
+    void *Cm = take(bc * es);
+    void *dBm = take(bc * es);
+    void *dCm = take(bc * es);
+    float *du = static_cast<float *>(take(seq * sizeof(float)));
+    float *dxs = static_cast<float *>(take(seq * sizeof(float)));
+    float *dxdbl = static_cast<float *>(take((size_t)s.B * kPaths * rn * s.L * sizeof(float)));
+    const size_t part_floats =
+        std::max((size_t)kPaths * s.B * proj_bwd_chunks(s) * rn * s.D, path_conv_partial_floats(s, 4));
+    float *part = static_cast<float *>(take(part_floats * sizeof(float)));
+    void *inner = w;
+    cudaStream_t st = (cudaStream_t)stream;
+    SS2D_TRY(from_cuda(launch_transpose(s, in, x, xT, st)));
+    SS2D_TRY(from_cuda(launch_path_conv_fwd(s, in, x, xT, conv_weight, conv_bias, d_conv, u, st)));
+    SS2D_TRY(from_cuda(launch_cross_scan(s, out, dy, g, st)));
+    SS2D_TRY(from_cuda(launch_dtproj(s, in, x_dbl, dt_proj_weight, R, RN, delta, st)));
+    const size_t row = (size_t)s.N * s.L * es, pitch = (size_t)RN * s.L * es, blocks = (size_t)s.B * kPaths;
+    const unsigned char *xd = static_cast<const unsigned char *>(x_dbl);
+    SS2D_TRY(from_cuda(cudaMemcpy2DAsync(Bm, row, xd + (size_t)R * s.L * es, pitch, row, blocks,
+                                         cudaMemcpyDeviceToDevice, st)));
+    SS2D_TRY(from_cuda(cudaMemcpy2DAsync(Cm, row, xd + (size_t)(R + s.N) * s.L * es, pitch, row, blocks,
+                                         cudaMemcpyDeviceToDevice, st)));
+    ScanBwdArgs a;
+    a.u = u;
+    a.delta = delta;
+    a.A = A;
+    a.Bm = Bm;
+    a.Cm = Cm;
+    a.Dv = D;
+    a.bias = dt_proj_bias;
+    a.softplus = delta_softplus != 0;
+    a.dout = g;
+    a.chunk_states = chunk_states;
+    a.du = du;
+    a.ddelta = ddelta;
+    a.dA = dA;
+    a.dBm = dBm;
+    a.dCm = dCm;
+    a.dD = dD;
+    a.dbias = ddt_proj_bias;
+    a.from_image = false;
+    a.du_f32 = true;
+    a.in_dtype = in;
+    a.out_dtype = out;
+    SS2D_TRY(from_cuda(launch_scan_bwd(s, a, inner, scan_bwd_workspace_bytes(s), st)));
+    SS2D_TRY(from_cuda(launch_proj_bwd_dtlow(s, in, ddelta, dt_proj_weight, R, RN, dxdbl, st)));
+    SS2D_TRY(from_cuda(launch_proj_bwd_copy_rows(s, in, dBm, (int)s.N, RN, R, dxdbl, st)));
+    SS2D_TRY(from_cuda(launch_proj_bwd_copy_rows(s, in, dCm, (int)s.N, RN, R + (int)s.N, dxdbl, st)));
+    SS2D_TRY(from_cuda(launch_proj_bwd_dwdt(s, in, ddelta, x_dbl, R, RN, part, ddt_proj_weight, st)));
+    SS2D_TRY(from_cuda(launch_proj_bwd_dwx_seq(s, in, dxdbl, u, RN, part, dx_proj_weight, st)));
+    SS2D_TRY(from_cuda(launch_proj_bwd_du(s, dxdbl, x_proj_weight, RN, du, st)));
+    SS2D_TRY(from_cuda(launch_path_conv_bwd(s, in, x, xT, conv_weight, conv_bias, d_conv, du, dxs, dconv_weight,
+                                            dconv_bias, part, st)));
+    return from_cuda(launch_cross_merge(s, SS2D_F32, in, dxs, dx, st));
 }
 
 ss2d_status_t ss2d_path_tables(const ss2d_desc_t *desc, int paths, int32_t *tables, ss2d_stream_t stream) {

@@ -108,6 +108,25 @@ cudaError_t launch_proj_bwd_dwdt(const LaunchShape &s, ss2d_dtype_t dt, const vo
 cudaError_t launch_proj_bwd_dwx(const LaunchShape &s, ss2d_dtype_t dt, const float *dxdbl, const void *x,
                                 const void *xT, int RN, float *part, float *dWx, cudaStream_t stream);
 
+// Causal depthwise conv with SiLU along every path (conv.cu): u[b, k*D + d, l] =
+// silu(bias[k*D + d] + sum_j w[k, d, j] x_k[d, l - (W-1) + j]), x_k = x (k = 0, 2) or xT (k = 1, 3)
+// read along path k; u in dt.  W = d_conv, 1..4; bias may be null.
+cudaError_t launch_path_conv_fwd(const LaunchShape &s, ss2d_dtype_t dt, const void *x, const void *xT,
+                                 const float *w, const float *bias, int W, void *u, cudaStream_t stream);
+// Its backward from du (fp32 (B, 4D, L), d loss / d u along the paths): dxs (fp32 (B, 4D, L), the
+// gradient of x read along each path, merged by the caller), dw (4, D, W) and dbias (4D, or null),
+// summed in a fixed order.  part holds path_conv_partial_floats(s, W) floats.
+size_t path_conv_partial_floats(const LaunchShape &s, int W);
+cudaError_t launch_path_conv_bwd(const LaunchShape &s, ss2d_dtype_t dt, const void *x, const void *xT,
+                                 const float *w, const float *bias, int W, const float *du, float *dxs, float *dw,
+                                 float *dbias, float *part, cudaStream_t stream);
+// d x_proj.weight for per-path sequences u (B, 4D, L) instead of the image read along the paths
+cudaError_t launch_proj_bwd_dwx_seq(const LaunchShape &s, ss2d_dtype_t dt, const float *dxdbl, const void *u, int RN,
+                                    float *part, float *dWx, cudaStream_t stream);
+// Per-path x_proj of sequences: xdbl[b, k, c, l] = sum_d W[k, c, d] u[b, k*D + d, l], RN <= 64
+cudaError_t launch_xproj_seq(const LaunchShape &s, ss2d_dtype_t dt, const void *u, const float *W, int RN,
+                             void *xdbl, cudaStream_t stream);
+
 // Bidirectional scan: out[b, d, m] = (two[b, 0, d, m] + two[b, 1, d, m]) * (z ? silu(z[b, d, m]) : 1),
 // two (B, 2, D, L) fp32, z (B, D, L) z_dtype or null, out (B, D, L) out_dtype.
 cudaError_t launch_bidir_sum(const float *two, const void *z, ss2d_dtype_t z_dtype, void *out,
@@ -138,6 +157,7 @@ struct ScanBwdArgs {
     bool from_image;
     bool bidir = false;       // kModeBidir: du, ddelta, dz are per-direction fp32 (B, 2, D, L) at natural
                               // positions; dA (2D, N); dB/dC (B, 1, N, L); dD/dbias (D)
+    bool du_f32 = false;      // sequence form: du written in fp32 whatever in_dtype
     ss2d_dtype_t in_dtype, out_dtype;
 };
 

@@ -10,7 +10,8 @@
 // u_k is x along path k (x or its transpose, paths 2 and 3 backwards).
 //
 // The two contractions with R on one side are narrow (R <= 32) and bound by reading ddelta
-// once: dtlow_kernel gives each thread one token and its R sums; dwdt_kernel gives each
+// once: rows_kernel gives each thread one token and its R sums (it also serves x_proj of
+// per-path sequences, R + 2N sums); dwdt_kernel gives each
 // thread one channel's R sums over a quarter of a staged token tile.  du_kernel stages both
 // operands of a 64-channel x 128-token tile whole (the contraction is R + 2N <= 64 long).
 // tr_gemm_kernel (d x_proj.weight) holds all R + 2N (<= 64) rows of a 128-column tile per CTA
@@ -62,16 +63,20 @@ __host__ __device__ constexpr int row_pitch() { return sizeof(T) == 4 ? kTS + 4 
 constexpr int kNarrowTok = 256;  // tokens (one per thread) of a dtlow_kernel CTA
 constexpr int kNarrowD = 64;     // channels per staged slice of dt_proj.weight
 
-// dx_dbl[g, r, l] = sum_d Wdt[k*D + d, r] ddelta[g, d, l], g = b * 4 + k; RB = R rounded up to 4
-template <typename Tin, int RB>
-__global__ void __launch_bounds__(kNarrowTok) dtlow_kernel(const Tin *__restrict__ ddelta,
-                                                           const float *__restrict__ Wdt, float *__restrict__ dxdbl,
-                                                           int64_t D, int64_t L, int R, int RN, int64_t nlt) {
+// out[g, r, l] = sum_d M(k, r, d) in[g, d, l] for r < R, g = b * 4 + k, M(k, r, d) =
+// Wm[k*w_ks + r*w_rs + d*w_ds]; in has D rows per group, out out_gs elements per group.  A thread
+// owns one token and its RB (R rounded up to 8) sums; M sits in shared memory 64 channels at a time.
+// Used for dx_dbl[:R] = dt_proj.weight^T ddelta and for x_proj of per-path sequences.
+template <typename Tin, typename Tout, int RB>
+__global__ void __launch_bounds__(kNarrowTok) rows_kernel(const Tin *__restrict__ in, const float *__restrict__ Wm,
+                                                          int64_t w_ks, int64_t w_rs, int64_t w_ds,
+                                                          Tout *__restrict__ out, int64_t out_gs, int64_t D,
+                                                          int64_t L, int R, int64_t nlt) {
     __shared__ __align__(16) float Ws[kNarrowD][RB];
     const int64_t bid = blockIdx.x, g = bid / nlt, k = g % kPaths;
     const int64_t l = (bid % nlt) * kNarrowTok + threadIdx.x;
     const bool live = l < L;
-    const Tin *src = ddelta + g * D * L + (live ? l : L - 1);  // dead threads re-read the last token
+    const Tin *src = in + g * D * L + (live ? l : L - 1);  // dead threads re-read the last token
     float acc[RB];
 #pragma unroll
     for (int r = 0; r < RB; ++r) acc[r] = 0.f;
@@ -80,13 +85,13 @@ __global__ void __launch_bounds__(kNarrowTok) dtlow_kernel(const Tin *__restrict
         __syncthreads();
         for (int e = threadIdx.x; e < kNarrowD * RB; e += kNarrowTok) {
             const int i = e / RB, r = e % RB;
-            Ws[i][r] = (i < n && r < R) ? Wdt[(k * D + d0 + i) * R + r] : 0.f;
+            Ws[i][r] = (i < n && r < R) ? Wm[k * w_ks + r * w_rs + (d0 + i) * w_ds] : 0.f;
         }
         __syncthreads();
-        const Tin *s = src + d0 * L;
+        const Tin *sp = src + d0 * L;
 #pragma unroll 8
         for (int i = 0; i < n; ++i) {
-            const float v = ld(s + i * L);
+            const float v = ld(sp + i * L);
 #pragma unroll
             for (int q = 0; q < RB / 4; ++q) {
                 const float4 w = *reinterpret_cast<const float4 *>(&Ws[i][4 * q]);
@@ -100,7 +105,7 @@ __global__ void __launch_bounds__(kNarrowTok) dtlow_kernel(const Tin *__restrict
     if (!live) return;
 #pragma unroll
     for (int r = 0; r < RB; ++r)
-        if (r < R) dxdbl[(g * RN + r) * L + l] = acc[r];
+        if (r < R) st(out + g * out_gs + r * L + l, acc[r]);
 }
 
 constexpr int kDwD = 64;  // channels per dwdt_kernel CTA (4 threads each)
@@ -471,31 +476,56 @@ static int grid_cap(int64_t items, int threads) {
     return (int)(want < 148 * 16 ? (want > 0 ? want : 1) : 148 * 16);
 }
 
-template <typename Tin, int RB>
-static cudaError_t dtlow_t(const LaunchShape &s, const void *ddelta, const float *Wdt, int R, int RN, float *dxdbl,
-                           cudaStream_t stream) {
+template <typename Tin, typename Tout, int RB>
+static cudaError_t rows_t(const LaunchShape &s, const void *in, const float *Wm, int64_t w_ks, int64_t w_rs,
+                          int64_t w_ds, void *out, int64_t out_gs, int R, cudaStream_t stream) {
     const int64_t nlt = ceil_div(s.L, kNarrowTok), blocks = nlt * s.B * kPaths;
     if (blocks > INT32_MAX) return cudaErrorInvalidConfiguration;
-    dtlow_kernel<Tin, RB><<<(unsigned)blocks, kNarrowTok, 0, stream>>>(static_cast<const Tin *>(ddelta), Wdt, dxdbl,
-                                                                        s.D, s.L, R, RN, nlt);
+    rows_kernel<Tin, Tout, RB><<<(unsigned)blocks, kNarrowTok, 0, stream>>>(
+        static_cast<const Tin *>(in), Wm, w_ks, w_rs, w_ds, static_cast<Tout *>(out), out_gs, s.D, s.L, R, nlt);
     return cudaSuccess;
 }
 
-template <typename Tin>
-static cudaError_t dtlow_r(const LaunchShape &s, const void *ddelta, const float *Wdt, int R, int RN, float *dxdbl,
-                           cudaStream_t stream) {
-    if (R <= 8) return dtlow_t<Tin, 8>(s, ddelta, Wdt, R, RN, dxdbl, stream);
-    if (R <= 16) return dtlow_t<Tin, 16>(s, ddelta, Wdt, R, RN, dxdbl, stream);
-    if (R <= 24) return dtlow_t<Tin, 24>(s, ddelta, Wdt, R, RN, dxdbl, stream);
-    return dtlow_t<Tin, 32>(s, ddelta, Wdt, R, RN, dxdbl, stream);
+template <typename Tin, typename Tout>
+static cudaError_t rows_r(const LaunchShape &s, const void *in, const float *Wm, int64_t w_ks, int64_t w_rs,
+                          int64_t w_ds, void *out, int64_t out_gs, int R, cudaStream_t stream) {
+    switch ((R + 7) / 8) {  // R rounded up to 8 sums per thread, R <= 64
+        case 1: return rows_t<Tin, Tout, 8>(s, in, Wm, w_ks, w_rs, w_ds, out, out_gs, R, stream);
+        case 2: return rows_t<Tin, Tout, 16>(s, in, Wm, w_ks, w_rs, w_ds, out, out_gs, R, stream);
+        case 3: return rows_t<Tin, Tout, 24>(s, in, Wm, w_ks, w_rs, w_ds, out, out_gs, R, stream);
+        case 4: return rows_t<Tin, Tout, 32>(s, in, Wm, w_ks, w_rs, w_ds, out, out_gs, R, stream);
+        case 5: return rows_t<Tin, Tout, 40>(s, in, Wm, w_ks, w_rs, w_ds, out, out_gs, R, stream);
+        case 6: return rows_t<Tin, Tout, 48>(s, in, Wm, w_ks, w_rs, w_ds, out, out_gs, R, stream);
+        case 7: return rows_t<Tin, Tout, 56>(s, in, Wm, w_ks, w_rs, w_ds, out, out_gs, R, stream);
+        case 8: return rows_t<Tin, Tout, 64>(s, in, Wm, w_ks, w_rs, w_ds, out, out_gs, R, stream);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 // dx_dbl[:R] (fp32, group stride RN*L) = dt_proj.weight^T @ ddelta (in dtype, group stride D*L)
 cudaError_t launch_proj_bwd_dtlow(const LaunchShape &s, ss2d_dtype_t dt, const void *ddelta, const float *Wdt, int R,
                                   int RN, float *dxdbl, cudaStream_t stream) {
     if (R < 1 || R > kProjRMax) return cudaErrorInvalidValue;
-    const cudaError_t e = dt == SS2D_F32 ? dtlow_r<float>(s, ddelta, Wdt, R, RN, dxdbl, stream)
-                                         : dtlow_r<__nv_bfloat16>(s, ddelta, Wdt, R, RN, dxdbl, stream);
+    // M(k, r, d) = Wdt[(k*D + d)*R + r]
+    const cudaError_t e =
+        dt == SS2D_F32
+            ? rows_r<float, float>(s, ddelta, Wdt, s.D * R, 1, R, dxdbl, (int64_t)RN * s.L, R, stream)
+            : rows_r<__nv_bfloat16, float>(s, ddelta, Wdt, s.D * R, 1, R, dxdbl, (int64_t)RN * s.L, R, stream);
+    if (e != cudaSuccess) return e;
+    note_launch(stream);
+    return cudaGetLastError();
+}
+
+// x_proj of per-path sequences: xdbl[b, k, c, l] = sum_d W[k, c, d] u[b, k*D + d, l] (in dtype)
+cudaError_t launch_xproj_seq(const LaunchShape &s, ss2d_dtype_t dt, const void *u, const float *W, int RN, void *xdbl,
+                             cudaStream_t stream) {
+    if (RN < 1 || RN > kProjRMax + 2 * 16) return cudaErrorInvalidValue;
+    // M(k, c, d) = W[(k*RN + c)*D + d]
+    const cudaError_t e =
+        dt == SS2D_F32
+            ? rows_r<float, float>(s, u, W, (int64_t)RN * s.D, s.D, 1, xdbl, (int64_t)RN * s.L, RN, stream)
+            : rows_r<__nv_bfloat16, __nv_bfloat16>(s, u, W, (int64_t)RN * s.D, s.D, 1, xdbl, (int64_t)RN * s.L, RN,
+                                                   stream);
     if (e != cudaSuccess) return e;
     note_launch(stream);
     return cudaGetLastError();
@@ -619,6 +649,33 @@ cudaError_t launch_proj_bwd_dwx(const LaunchShape &s, ss2d_dtype_t dt, const flo
     p.Bp[3] = xT;
     p.b_bs = s.D * s.L;
     p.rev_mask = 0b1100;  // paths 2 and 3 walk their base order backwards
+    p.M = RN;
+    p.N = (int)s.D;
+    p.B = s.B;
+    p.L = s.L;
+    p.lchunk = kProjTokenChunk;
+    p.nlc = (int)proj_bwd_chunks(s);
+    p.nnt = (int)ceil_div(p.N, kTN);
+    p.part = part;
+    const cudaError_t e = dt == SS2D_F32 ? dwx_ty<float>(s, p, stream) : dwx_ty<__nv_bfloat16>(s, p, stream);
+    if (e != cudaSuccess) return e;
+    note_launch(stream);
+    reduce_partials(s, part, dWx, (int64_t)RN * s.D, stream);
+    return cudaGetLastError();
+}
+
+
+// d x_proj.weight (4, RN, D) = sum over tokens of dx_dbl (x) u_k for per-path sequences u (B, 4D, L)
+cudaError_t launch_proj_bwd_dwx_seq(const LaunchShape &s, ss2d_dtype_t dt, const float *dxdbl, const void *u, int RN,
+                                    float *part, float *dWx, cudaStream_t stream) {
+    TrArgs p{};
+    p.A = dxdbl;
+    p.a_bs = (int64_t)kPaths * RN * s.L;
+    p.a_ks = (int64_t)RN * s.L;
+    const size_t es = dt == SS2D_F32 ? 4 : 2;
+    for (int k = 0; k < kPaths; ++k) p.Bp[k] = static_cast<const unsigned char *>(u) + (size_t)k * s.D * s.L * es;
+    p.b_bs = (int64_t)kPaths * s.D * s.L;
+    p.rev_mask = 0;
     p.M = RN;
     p.N = (int)s.D;
     p.B = s.B;

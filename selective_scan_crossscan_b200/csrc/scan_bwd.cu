@@ -76,6 +76,7 @@ struct BwdParams {
     int softplus;
     int64_t nchunks;
     int ntiles;
+    bool du_f32;        // sequence form: du written in fp32 whatever the input dtype
 };
 
 // B and C of a block are the same for every channel of one (b, k): the CTA stages them once.
@@ -631,8 +632,9 @@ static cudaError_t launch_bwd_ns(const LaunchShape &s, const BwdParams &p, cudaS
 
 template <typename Tin, typename Tg, int MODE>
 static cudaError_t launch_bwd_du(const LaunchShape &s, const BwdParams &p, cudaStream_t stream) {
-    // the fused and bidirectional backward passes keep du in fp32 for the merge that follows
-    if (MODE != kModeSeq) return launch_bwd_ns<Tin, Tg, float, MODE>(s, p, stream);
+    // the fused and bidirectional backward passes keep du in fp32 for the merge that follows,
+    // and so does a sequence-form caller that adds more to du before using it
+    if (MODE != kModeSeq || p.du_f32) return launch_bwd_ns<Tin, Tg, float, MODE>(s, p, stream);
     return launch_bwd_ns<Tin, Tg, Tin, MODE>(s, p, stream);
 }
 
@@ -700,6 +702,7 @@ cudaError_t launch_scan_bwd(const LaunchShape &s, const ScanBwdArgs &a, void *wo
     p.doutT = a.doutT;
     p.cs = cs;
     p.z = a.from_image ? nullptr : a.z;  // the fused SS2D path has no gate
+    p.du_f32 = a.du_f32;
     p.du = a.du;
     p.ddelta = a.ddelta;
     p.dz = a.dz;

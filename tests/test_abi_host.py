@@ -178,6 +178,23 @@ def test_backward_proj_argument_errors(lib):
     assert f(_d(), 2, *w, *ok, *g, A16, ws - 1, None) == ERR_WORKSPACE
 
 
+def test_proj_conv_argument_errors(lib):
+    f, g = lib.ss2d_forward_proj_conv, lib.ss2d_backward_proj_conv
+    wsf = lib.ss2d_workspace_bytes(_d(), ss.OP_FORWARD_PROJ_CONV)
+    wsb = lib.ss2d_workspace_bytes(_d(), ss.OP_BACKWARD_PROJ_CONV)
+    assert wsb > wsf > 0
+    w = [A16] * 8  # x, conv_weight, conv_bias, x_proj_weight, dt_proj_weight, dt_proj_bias, A, D
+    assert f(_d(), 0, 4, *w, 1, B16, B16, None, A16, wsf, None) == ERR_SHAPE   # dt_rank 0
+    assert f(_d(), 2, 0, *w, 1, B16, B16, None, A16, wsf, None) == ERR_SHAPE   # d_conv 0
+    assert f(_d(), 2, 5, *w, 1, B16, B16, None, A16, wsf, None) == ERR_SHAPE   # d_conv 5
+    assert f(_d(), 2, 4, A16, None, *w[2:], 1, B16, B16, None, A16, wsf, None) == ERR_NULL  # conv_weight
+    assert f(_d(), 2, 4, *w, 1, B16, B16, None, A16, wsf - 1, None) == ERR_WORKSPACE
+    gr = [B16] * 8  # dx, dconv_weight, dconv_bias, dx_proj_weight, ddt_proj_weight, ddt_proj_bias, dA, dD
+    assert g(_d(), 2, 4, *w, 1, A16, None, A16, *gr, A16, wsb - 1, None) == ERR_WORKSPACE
+    assert g(_d(), 2, 4, *w, 1, A16, None, A16, gr[0], gr[1], None, *gr[3:], A16, wsb, None) == ERR_NULL  # conv bias
+    assert g(_d(), 2, 5, *w, 1, A16, None, A16, *gr, A16, wsb, None) == ERR_SHAPE
+
+
 def test_valid_call_without_gpu_reports_device_error(lib):
     import torch
     if torch.cuda.is_available():

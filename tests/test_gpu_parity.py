@@ -674,6 +674,85 @@ def test_ss2d_backward_proj_deterministic():
         assert torch.equal(runs[0][k], runs[1][k]), k
 
 
+# ---------------------------------------- producer with its causal conv per path
+
+CONV_NAMES = ("dx", "dconv_weight", "dconv_bias", "dx_proj_weight", "ddt_proj_weight", "ddt_proj_bias", "dA", "dD")
+
+# (Bn, D, H, W, N, d_conv): L % 4 != 0 (plain-load paths), one-pixel maps, every conv width, wide rank
+CONV_CASES = [(1, 8, 8, 8, 4, 4), (2, 70, 5, 9, 16, 4), (2, 6, 1, 1, 16, 3), (1, 40, 12, 11, 8, 2),
+              (1, 192, 14, 14, 16, 4), (1, 16, 6, 7, 16, 1), (1, 768, 6, 8, 16, 4)]
+
+
+def _conv_case(Bn, Dn, H, W, N, d_conv, dtype="f32", seed=0):
+    w = ss2d_inputs.custom(Bn, Dn, H, W, N, dtype=dtype, a_init="s4d_real")
+    return w, ss2d_inputs.make_proj_inputs(w, seed=seed, d_conv=d_conv)
+
+
+def _conv_call_args(d):
+    return (d["x"], d["conv_weight"], d["conv_bias"], d["x_proj_weight"], d["dt_proj_weight"], d["dt_proj_bias"],
+            d["A"], d["D"])
+
+
+@pytest.mark.parametrize("case", CONV_CASES)
+def test_ss2d_proj_conv_forward_backward_parity(case):
+    w, inp = _conv_case(*case, seed=62)
+    d = _dev({k: v for k, v in inp.items() if k != "R"})
+    y, x_dbl = ss.ss2d_forward_proj_conv(*_conv_call_args(d), True, return_x_dbl=True)
+    ref = oracle.ss2d_forward_proj_conv(*_conv_call_args(inp), True)
+    assert_fwd_close(y, ref, f"{case} y")
+    u, _ = oracle.path_conv(inp["x"], inp["conv_weight"], inp["conv_bias"])
+    ref_dbl = np.einsum("bkdl,kcd->bkcl", u, inp["x_proj_weight"].double().numpy())
+    assert_fwd_close(x_dbl, ref_dbl, f"{case} x_dbl")
+    dy_np = torch.randn(tuple(y.shape), generator=torch.Generator().manual_seed(63),
+                        dtype=torch.float32).double().numpy()
+    got = ss.ss2d_backward_proj_conv(*_conv_call_args(d), x_dbl, torch.as_tensor(dy_np, dtype=torch.float32,
+                                                                                  device="cuda"), True)
+    refg = oracle.ss2d_backward_proj_conv(*_conv_call_args(inp), True, dy_np)
+    for name in CONV_NAMES:
+        assert_rel_l2(got[name], refg[name], GRAD_TOL, f"{case} {name}")
+
+
+def test_ss2d_proj_conv_without_bias_bf16_and_deterministic():
+    w, inp = _conv_case(2, 24, 9, 10, 16, 4, seed=64)
+    inp["conv_bias"] = None
+    d = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in inp.items() if k != "R"}
+    y, x_dbl, cs = ss.ss2d_forward_proj_conv(*_conv_call_args(d), True, return_x_dbl=True, return_chunk_states=True)
+    assert_fwd_close(y, oracle.ss2d_forward_proj_conv(*_conv_call_args(inp), True), "y without conv bias")
+    dy = torch.randn(y.shape, generator=torch.Generator(device="cuda").manual_seed(65), device="cuda")
+    runs = [ss.ss2d_backward_proj_conv(*_conv_call_args(d), x_dbl, dy, True, chunk_states=cs) for _ in range(2)]
+    assert runs[0]["dconv_bias"] is None
+    for k in runs[0]:
+        if runs[0][k] is not None:
+            assert torch.equal(runs[0][k], runs[1][k]), k
+    refg = oracle.ss2d_backward_proj_conv(*_conv_call_args(inp), True, dy.double().cpu().numpy())
+    for name in CONV_NAMES:
+        if name != "dconv_bias":
+            assert_rel_l2(runs[0][name], refg[name], GRAD_TOL, f"{name} without conv bias")
+    # bf16 activations against the oracle on the bf16-rounded inputs
+    w, inp = _conv_case(2, 16, 12, 12, 16, 4, dtype="bf16", seed=66)
+    d = _dev({k: v for k, v in inp.items() if k != "R"})
+    y, x_dbl = ss.ss2d_forward_proj_conv(*_conv_call_args(d), True, return_x_dbl=True)
+    assert_rel_l2(y, oracle.ss2d_forward_proj_conv(*_conv_call_args(inp), True), BF16_TOL, "y bf16")
+    dy_np = torch.randn(tuple(y.shape), generator=torch.Generator().manual_seed(67), dtype=torch.float64)
+    dy_np = dy_np.to(torch.bfloat16).double().numpy()
+    got = ss.ss2d_backward_proj_conv(*_conv_call_args(d), x_dbl,
+                                     torch.as_tensor(dy_np, device="cuda").to(torch.bfloat16), True)
+    refg = oracle.ss2d_backward_proj_conv(*_conv_call_args(inp), True, dy_np)
+    for name in CONV_NAMES:
+        assert_rel_l2(got[name], refg[name], BF16_TOL, f"{name} bf16")
+
+
+def test_ss2d_proj_conv_full_stage1_sampled():
+    # VMamba-T stage-1 shapes in the launch configuration bench.py times, sampled batch items
+    w = ss2d_inputs.workload("vmamba_t_stage1_fp32")
+    inp = ss2d_inputs.make_proj_inputs(w, seed=68, d_conv=4)
+    d = _dev({k: v for k, v in inp.items() if k != "R"})
+    y = ss.ss2d_forward_proj_conv(*_conv_call_args(d), True)
+    for bi in (0, w.batch - 1):
+        sl = dict(inp, x=inp["x"][bi:bi + 1])
+        assert_fwd_close(y[bi:bi + 1], oracle.ss2d_forward_proj_conv(*_conv_call_args(sl), True), f"y[{bi}]")
+
+
 # ------------------------------------------------------------- fused SS2D
 
 FUSED_CASES = [(1, 8, 8, 8, 4), (2, 6, 5, 9, 16), (1, 70, 12, 11, 16), (1, 8, 64, 64, 16), (2, 3, 1, 1, 2),
