@@ -12,16 +12,19 @@
 //     dpre = du * silu'(pre),  silu'(p) = s (1 + p (1 - s)),  s = sigmoid(p)
 //     dx_k[d, m] = sum_j w[k, d, j] dpre[m + (W-1) - j]
 //     dw[k, d, j] = sum over batch and steps of dpre[l] x_k[l - (W-1) + j],  dbias = sum of dpre
-// A CTA takes 256 steps of one (b, k, d) row, one per thread; the backward keeps the tile's dpre
-// and the W-1 steps after it in shared memory, reduces its weight and bias terms in a fixed
-// tree order, and a second kernel adds the per-(batch item, tile) partials in a fixed order.
+// A CTA takes 1024 steps of one (b, k, d) row, four consecutive ones per thread (the row is
+// decoded once per thread in 32-bit arithmetic); the backward keeps the tile's dpre and the
+// W-1 steps after it in shared memory, reduces its weight and bias terms in a fixed tree
+// order, and a second kernel adds the per-(batch item, tile) partials in a fixed order.
 // The work is a few multiply-adds per element: bound by HBM.
 #include "common.cuh"
 #include "kernels.h"
 
 namespace ss2d {
 
-constexpr int kConvTok = 256;  // steps per CTA, one per thread
+constexpr int kConvThreads = 256;
+constexpr int kConvPer = 4;                            // consecutive steps per thread
+constexpr int kConvTok = kConvThreads * kConvPer;      // steps per CTA
 constexpr int kConvWMax = 4;
 
 // step m of path k in a row of x (or xT): 0 before the first step
@@ -30,73 +33,110 @@ __device__ __forceinline__ float path_x(const Tin *row, bool rev, int64_t L, int
     return m < 0 ? 0.f : ld(row + (rev ? L - 1 - m : m));
 }
 
+// The CTA's row (b, k, d) and tile, decoded once in 32-bit arithmetic (the launcher checks the
+// row count fits), and the row's x (or xT) base, direction, weights and bias.
 template <typename Tin, int W>
-__global__ void __launch_bounds__(kConvTok) path_conv_fwd_kernel(const Tin *__restrict__ x, const Tin *__restrict__ xT,
-                                                                 const float *__restrict__ w,
-                                                                 const float *__restrict__ bias, Tin *__restrict__ u,
-                                                                 int64_t D, int64_t L, int64_t nlt) {
-    const int64_t bid = blockIdx.x, row = bid / nlt;  // row = (b * 4 + k) * D + d
-    const int64_t l = (bid % nlt) * kConvTok + threadIdx.x;
-    if (l >= L) return;
-    const int64_t d = row % D, bk = row / D, k = bk % kPaths, b = bk / kPaths;
-    const Tin *xr = ((k & 1) ? xT : x) + (b * D + d) * L;
-    const bool rev = k >= 2;
-    const float *wk = w + (k * D + d) * W;
-    float pre = bias ? bias[k * D + d] : 0.f;
+struct ConvRow {
+    int64_t row, l0;
+    const Tin *xr;
+    bool rev;
+    float w[W], b0;
+    __device__ __forceinline__ ConvRow(const Tin *x, const Tin *xT, const float *wt, const float *bias, uint32_t D,
+                                       uint32_t nlt, int64_t L) {
+        const uint32_t bid = blockIdx.x, r = bid / nlt, d = r % D, bk = r / D, k = bk % kPaths, b = bk / kPaths;
+        row = r;
+        l0 = (int64_t)(bid - r * nlt) * kConvTok;
+        xr = ((k & 1) ? xT : x) + ((int64_t)b * D + d) * L;
+        rev = k >= 2;
 #pragma unroll
-    for (int j = 0; j < W; ++j) pre = fmaf(wk[j], path_x(xr, rev, L, l - (W - 1) + j), pre);
-    st(u + row * L + l, silu_f(pre));
+        for (int j = 0; j < W; ++j) w[j] = wt[((int64_t)k * D + d) * W + j];
+        b0 = bias ? bias[(int64_t)k * D + d] : 0.f;
+    }
+    // x_k at steps l - (W-1) .. l + kConvPer - 1: the windows of kConvPer consecutive outputs
+    __device__ __forceinline__ void window(int64_t l, int64_t L, float (&xv)[kConvPer + W - 1]) const {
+#pragma unroll
+        for (int i = 0; i < kConvPer + W - 1; ++i) {
+            const int64_t m = l - (W - 1) + i;
+            xv[i] = m < L ? path_x(xr, rev, L, m) : 0.f;
+        }
+    }
+    __device__ __forceinline__ float pre(const float (&xv)[kConvPer + W - 1], int q) const {
+        float p = b0;
+#pragma unroll
+        for (int j = 0; j < W; ++j) p = fmaf(w[j], xv[q + j], p);
+        return p;
+    }
+};
+
+template <typename Tin, int W>
+__global__ void __launch_bounds__(kConvThreads) path_conv_fwd_kernel(const Tin *__restrict__ x, const Tin *__restrict__ xT,
+                                                                     const float *__restrict__ w,
+                                                                     const float *__restrict__ bias,
+                                                                     Tin *__restrict__ u, uint32_t D, int64_t L,
+                                                                     uint32_t nlt) {
+    const ConvRow<Tin, W> cr(x, xT, w, bias, D, nlt, L);
+    const int64_t l = cr.l0 + kConvPer * threadIdx.x;
+    if (l >= L) return;
+    float xv[kConvPer + W - 1];
+    cr.window(l, L, xv);
+    Tin *o = u + cr.row * L + l;
+#pragma unroll
+    for (int q = 0; q < kConvPer; ++q)
+        if (l + q < L) st(o + q, silu_f(cr.pre(xv, q)));
 }
 
 template <typename Tin, int W>
-__global__ void __launch_bounds__(kConvTok) path_conv_bwd_kernel(const Tin *__restrict__ x, const Tin *__restrict__ xT,
-                                                                 const float *__restrict__ w,
-                                                                 const float *__restrict__ bias,
-                                                                 const float *__restrict__ du, float *__restrict__ dxs,
-                                                                 float *__restrict__ part, int64_t D, int64_t L,
-                                                                 int64_t nlt) {
-    __shared__ float dp[kConvTok + kConvWMax];      // dpre of the tile's steps and of the W-1 after it
-    __shared__ float red[kConvTok / 32][W + 1];     // per-warp sums of the weight and bias terms
+__global__ void __launch_bounds__(kConvThreads) path_conv_bwd_kernel(const Tin *__restrict__ x, const Tin *__restrict__ xT,
+                                                                     const float *__restrict__ w,
+                                                                     const float *__restrict__ bias,
+                                                                     const float *__restrict__ du,
+                                                                     float *__restrict__ dxs, float *__restrict__ part,
+                                                                     uint32_t D, int64_t L, uint32_t nlt) {
+    __shared__ float dp[kConvTok + kConvWMax];          // dpre of the tile's steps and of the W-1 after it
+    __shared__ float red[kConvThreads / 32][W + 1];     // per-warp sums of the weight and bias terms
     const int t = threadIdx.x;
-    const int64_t bid = blockIdx.x, row = bid / nlt, tile = bid % nlt;
-    const int64_t l0 = tile * kConvTok, l = l0 + t;
-    const int64_t d = row % D, bk = row / D, k = bk % kPaths, b = bk / kPaths;
-    const Tin *xr = ((k & 1) ? xT : x) + (b * D + d) * L;
-    const bool rev = k >= 2;
-    const float *wk = w + (k * D + d) * W;
-    const float b0 = bias ? bias[k * D + d] : 0.f;
-    const float *dur = du + row * L;
-    auto dpre_of = [&](const float (&xin)[W], int64_t m) {
-        float pre = b0;
-#pragma unroll
-        for (int j = 0; j < W; ++j) pre = fmaf(wk[j], xin[j], pre);
-        const float sg = sigmoid_f(pre);
-        return dur[m] * sg * fmaf(pre, 1.f - sg, 1.f);
+    const ConvRow<Tin, W> cr(x, xT, w, bias, D, nlt, L);
+    const int64_t l = cr.l0 + kConvPer * t;
+    const float *dur = du + cr.row * L;
+    auto dpre_of = [&](float p, int64_t m) {
+        const float sg = sigmoid_f(p);
+        return dur[m] * sg * fmaf(p, 1.f - sg, 1.f);
     };
-    float xin[W];
+    float xv[kConvPer + W - 1];
+    cr.window(l, L, xv);
+    float dpl[kConvPer];
 #pragma unroll
-    for (int j = 0; j < W; ++j) xin[j] = l < L ? path_x(xr, rev, L, l - (W - 1) + j) : 0.f;
-    const float dpl = l < L ? dpre_of(xin, l) : 0.f;
-    dp[t] = dpl;
-    if (t < W - 1) {
-        const int64_t m = l0 + kConvTok + t;
-        float xh[W];
+    for (int q = 0; q < kConvPer; ++q) {
+        dpl[q] = l + q < L ? dpre_of(cr.pre(xv, q), l + q) : 0.f;
+        dp[kConvPer * t + q] = dpl[q];
+    }
+    if (t < W - 1) {  // the halo: dpre of the W-1 steps after the tile
+        const int64_t m = cr.l0 + kConvTok + t;
+        float p = cr.b0;
 #pragma unroll
-        for (int j = 0; j < W; ++j) xh[j] = m < L ? path_x(xr, rev, L, m - (W - 1) + j) : 0.f;
-        dp[kConvTok + t] = m < L ? dpre_of(xh, m) : 0.f;
+        for (int j = 0; j < W; ++j) p = fmaf(cr.w[j], m < L ? path_x(cr.xr, cr.rev, L, m - (W - 1) + j) : 0.f, p);
+        dp[kConvTok + t] = m < L ? dpre_of(p, m) : 0.f;
     }
     __syncthreads();
-    if (l < L) {
+#pragma unroll
+    for (int q = 0; q < kConvPer; ++q) {
+        if (l + q >= L) break;
         float acc = 0.f;
 #pragma unroll
-        for (int j = 0; j < W; ++j) acc = fmaf(wk[j], dp[t + (W - 1) - j], acc);
-        dxs[row * L + l] = acc;
+        for (int j = 0; j < W; ++j) acc = fmaf(cr.w[j], dp[kConvPer * t + q + (W - 1) - j], acc);
+        dxs[cr.row * L + l + q] = acc;
     }
-    // weight and bias terms of this tile: a fixed shuffle tree per warp, then the warps in order
+    // weight and bias terms: this thread's steps in order, a fixed shuffle tree per warp, then the
+    // warps in order
     float v[W + 1];
 #pragma unroll
-    for (int j = 0; j < W; ++j) v[j] = dpl * xin[j];
-    v[W] = dpl;
+    for (int j = 0; j <= W; ++j) v[j] = 0.f;
+#pragma unroll
+    for (int q = 0; q < kConvPer; ++q) {
+#pragma unroll
+        for (int j = 0; j < W; ++j) v[j] = fmaf(dpl[q], xv[q + j], v[j]);
+        v[W] += dpl[q];
+    }
 #pragma unroll
     for (int j = 0; j <= W; ++j)
 #pragma unroll
@@ -108,8 +148,8 @@ __global__ void __launch_bounds__(kConvTok) path_conv_bwd_kernel(const Tin *__re
     if (t <= W) {
         float s = 0.f;
 #pragma unroll
-        for (int i = 0; i < kConvTok / 32; ++i) s += red[i][t];
-        part[(row * nlt + tile) * (W + 1) + t] = s;
+        for (int i = 0; i < kConvThreads / 32; ++i) s += red[i][t];
+        part[(int64_t)blockIdx.x * (W + 1) + t] = s;
     }
 }
 
@@ -143,9 +183,10 @@ template <typename Tin, int W>
 static cudaError_t conv_fwd_t(const LaunchShape &s, const void *x, const void *xT, const float *w, const float *bias,
                               void *u, cudaStream_t stream) {
     const int64_t nlt = ceil_div(s.L, kConvTok), blocks = s.B * kPaths * s.D * nlt;
-    if (blocks > INT32_MAX) return cudaErrorInvalidConfiguration;
-    path_conv_fwd_kernel<Tin, W><<<(unsigned)blocks, kConvTok, 0, stream>>>(
-        static_cast<const Tin *>(x), static_cast<const Tin *>(xT), w, bias, static_cast<Tin *>(u), s.D, s.L, nlt);
+    if (blocks > INT32_MAX) return cudaErrorInvalidConfiguration;  // also keeps the 32-bit row decode exact
+    path_conv_fwd_kernel<Tin, W><<<(unsigned)blocks, kConvThreads, 0, stream>>>(
+        static_cast<const Tin *>(x), static_cast<const Tin *>(xT), w, bias, static_cast<Tin *>(u), (uint32_t)s.D,
+        s.L, (uint32_t)nlt);
     return cudaSuccess;
 }
 
@@ -174,9 +215,10 @@ template <typename Tin, int W>
 static cudaError_t conv_bwd_t(const LaunchShape &s, const void *x, const void *xT, const float *w, const float *bias,
                               const float *du, float *dxs, float *part, cudaStream_t stream) {
     const int64_t nlt = ceil_div(s.L, kConvTok), blocks = s.B * kPaths * s.D * nlt;
-    if (blocks > INT32_MAX) return cudaErrorInvalidConfiguration;
-    path_conv_bwd_kernel<Tin, W><<<(unsigned)blocks, kConvTok, 0, stream>>>(
-        static_cast<const Tin *>(x), static_cast<const Tin *>(xT), w, bias, du, dxs, part, s.D, s.L, nlt);
+    if (blocks > INT32_MAX) return cudaErrorInvalidConfiguration;  // also keeps the 32-bit row decode exact
+    path_conv_bwd_kernel<Tin, W><<<(unsigned)blocks, kConvThreads, 0, stream>>>(
+        static_cast<const Tin *>(x), static_cast<const Tin *>(xT), w, bias, du, dxs, part, (uint32_t)s.D, s.L,
+        (uint32_t)nlt);
     return cudaSuccess;
 }
 
