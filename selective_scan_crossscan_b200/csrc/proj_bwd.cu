@@ -65,24 +65,21 @@ constexpr int kNarrowD = 64;     // channels per staged slice of dt_proj.weight
 
 // out[g, r, l] = sum_d M(k, r, d) in[g, d, l] for r < R, g = b * 4 + k, M(k, r, d) =
 // Wm[k*w_ks + r*w_rs + d*w_ds]; in has D rows per group, out out_gs elements per group.  A thread
-// owns TOK tokens (t and t + 256) and their RB (R rounded up to 8) sums, as packed pairs when
-// TOK = 2 (one FFMA2 per r for both tokens); M sits in shared memory 64 channels at a time.
+// owns one token and its RB (R rounded up to 8) sums; M sits in shared memory 64 channels at a time.
 // Used for dx_dbl[:R] = dt_proj.weight^T ddelta and for x_proj of per-path sequences.
-template <typename Tin, typename Tout, int RB, int TOK>
+template <typename Tin, typename Tout, int RB>
 __global__ void __launch_bounds__(kNarrowTok) rows_kernel(const Tin *__restrict__ in, const float *__restrict__ Wm,
                                                           int64_t w_ks, int64_t w_rs, int64_t w_ds,
                                                           Tout *__restrict__ out, int64_t out_gs, int64_t D,
                                                           int64_t L, int R, int64_t nlt) {
-    static_assert(TOK == 1 || TOK == 2, "one or two tokens per thread");
     __shared__ __align__(16) float Ws[kNarrowD][RB];
     const int64_t bid = blockIdx.x, g = bid / nlt, k = g % kPaths;
-    const int64_t la = (bid % nlt) * (kNarrowTok * TOK) + threadIdx.x, lb = la + kNarrowTok;
-    const bool live_a = la < L, live_b = TOK == 2 && lb < L;
-    const Tin *src = in + g * D * L;
-    const int64_t oa = live_a ? la : L - 1, ob = live_b ? lb : L - 1;  // dead slots re-read the last token
-    float2 acc[RB];
+    const int64_t l = (bid % nlt) * kNarrowTok + threadIdx.x;
+    const bool live = l < L;
+    const Tin *src = in + g * D * L + (live ? l : L - 1);  // dead threads re-read the last token
+    float acc[RB];
 #pragma unroll
-    for (int r = 0; r < RB; ++r) acc[r] = make_float2(0.f, 0.f);
+    for (int r = 0; r < RB; ++r) acc[r] = 0.f;
     for (int64_t d0 = 0; d0 < D; d0 += kNarrowD) {
         const int n = (int)(D - d0 < kNarrowD ? D - d0 : kNarrowD);
         __syncthreads();
@@ -92,35 +89,23 @@ __global__ void __launch_bounds__(kNarrowTok) rows_kernel(const Tin *__restrict_
         }
         __syncthreads();
         const Tin *sp = src + d0 * L;
-#pragma unroll 4
+#pragma unroll 8
         for (int i = 0; i < n; ++i) {
-            const float va = ld(sp + i * L + oa);
-            const float vb = TOK == 2 ? ld(sp + i * L + ob) : 0.f;
-            const float2 v2 = make_float2(va, vb);
+            const float v = ld(sp + i * L);
 #pragma unroll
             for (int q = 0; q < RB / 4; ++q) {
                 const float4 w = *reinterpret_cast<const float4 *>(&Ws[i][4 * q]);
-                if (TOK == 2) {
-                    acc[4 * q + 0] = __ffma2_rn(v2, make_float2(w.x, w.x), acc[4 * q + 0]);
-                    acc[4 * q + 1] = __ffma2_rn(v2, make_float2(w.y, w.y), acc[4 * q + 1]);
-                    acc[4 * q + 2] = __ffma2_rn(v2, make_float2(w.z, w.z), acc[4 * q + 2]);
-                    acc[4 * q + 3] = __ffma2_rn(v2, make_float2(w.w, w.w), acc[4 * q + 3]);
-                } else {
-                    acc[4 * q + 0].x = fmaf(w.x, va, acc[4 * q + 0].x);
-                    acc[4 * q + 1].x = fmaf(w.y, va, acc[4 * q + 1].x);
-                    acc[4 * q + 2].x = fmaf(w.z, va, acc[4 * q + 2].x);
-                    acc[4 * q + 3].x = fmaf(w.w, va, acc[4 * q + 3].x);
-                }
+                acc[4 * q + 0] = fmaf(w.x, v, acc[4 * q + 0]);
+                acc[4 * q + 1] = fmaf(w.y, v, acc[4 * q + 1]);
+                acc[4 * q + 2] = fmaf(w.z, v, acc[4 * q + 2]);
+                acc[4 * q + 3] = fmaf(w.w, v, acc[4 * q + 3]);
             }
         }
     }
-    Tout *o = out + g * out_gs;
+    if (!live) return;
 #pragma unroll
-    for (int r = 0; r < RB; ++r) {
-        if (r >= R) continue;
-        if (live_a) st(o + r * L + la, acc[r].x);
-        if (live_b) st(o + r * L + lb, acc[r].y);
-    }
+    for (int r = 0; r < RB; ++r)
+        if (r < R) st(out + g * out_gs + r * L + l, acc[r]);
 }
 
 constexpr int kDwD = 64;  // channels per dwdt_kernel CTA (4 threads each)
@@ -494,10 +479,9 @@ static int grid_cap(int64_t items, int threads) {
 template <typename Tin, typename Tout, int RB>
 static cudaError_t rows_t(const LaunchShape &s, const void *in, const float *Wm, int64_t w_ks, int64_t w_rs,
                           int64_t w_ds, void *out, int64_t out_gs, int R, cudaStream_t stream) {
-    constexpr int TOK = RB <= 24 ? 2 : 1;  // packed pairs while their accumulators fit 128 registers
-    const int64_t nlt = ceil_div(s.L, kNarrowTok * TOK), blocks = nlt * s.B * kPaths;
+    const int64_t nlt = ceil_div(s.L, kNarrowTok), blocks = nlt * s.B * kPaths;
     if (blocks > INT32_MAX) return cudaErrorInvalidConfiguration;
-    rows_kernel<Tin, Tout, RB, TOK><<<(unsigned)blocks, kNarrowTok, 0, stream>>>(
+    rows_kernel<Tin, Tout, RB><<<(unsigned)blocks, kNarrowTok, 0, stream>>>(
         static_cast<const Tin *>(in), Wm, w_ks, w_rs, w_ds, static_cast<Tout *>(out), out_gs, s.D, s.L, R, nlt);
     return cudaSuccess;
 }
