@@ -204,61 +204,4 @@ cudaError_t launch_xproj(const LaunchShape &s, ss2d_dtype_t dt, const void *x, c
     return cudaGetLastError();
 }
 
-// dt_proj for ranks where the scan would spend more on R multiply-adds per step than on
-// reading delta: delta[b, k*D + d, l] = sum_r Wdt[k*D + d, r] * xdbl[b, k, r, l].  A CTA takes
-// 128 tokens of one path of one batch item and 32 channels; each thread keeps its token's 32
-// channel sums in registers and walks the ranks, so the multiply-adds are 32 independent
-// chains; the weights (rank-major in shared memory) are 128-bit broadcast loads, and each
-// channel's row of delta is written contiguously along the tokens.
-constexpr int kDtTok = 128, kDtCh = 32;
-
-template <typename Tin>
-__global__ void __launch_bounds__(kDtTok) dtproj_kernel(const Tin *__restrict__ xdbl, const float *__restrict__ Wdt,
-                                                        Tin *__restrict__ delta, int64_t D, int64_t L, int R,
-                                                        int RN) {
-    __shared__ __align__(16) float Wt[kProjRMax][kDtCh];
-    const int t = threadIdx.x;
-    const int64_t bk = blockIdx.z, k = bk % kPaths, d0 = (int64_t)blockIdx.y * kDtCh;
-    const int64_t l = (int64_t)blockIdx.x * kDtTok + t;
-    for (int e = t; e < kDtCh * kProjRMax; e += kDtTok) {
-        const int dd = e / kProjRMax, r = e % kProjRMax;
-        Wt[r][dd] = (d0 + dd < D && r < R) ? Wdt[(k * D + d0 + dd) * R + r] : 0.f;
-    }
-    __syncthreads();
-    if (l >= L) return;
-    const Tin *src = xdbl + bk * RN * L + l;
-    float acc[kDtCh];
-#pragma unroll
-    for (int dd = 0; dd < kDtCh; ++dd) acc[dd] = 0.f;
-    for (int r = 0; r < R; ++r) {
-        const float xv = ld(src + (int64_t)r * L);
-#pragma unroll
-        for (int dd = 0; dd < kDtCh; dd += 4) {
-            const float4 w = *reinterpret_cast<const float4 *>(&Wt[r][dd]);
-            acc[dd] = fmaf(w.x, xv, acc[dd]);
-            acc[dd + 1] = fmaf(w.y, xv, acc[dd + 1]);
-            acc[dd + 2] = fmaf(w.z, xv, acc[dd + 2]);
-            acc[dd + 3] = fmaf(w.w, xv, acc[dd + 3]);
-        }
-    }
-    Tin *dst = delta + (bk * D + d0) * L + l;
-#pragma unroll
-    for (int dd = 0; dd < kDtCh; ++dd)
-        if (d0 + dd < D) st(dst + (int64_t)dd * L, acc[dd]);
-}
-
-cudaError_t launch_dtproj(const LaunchShape &s, ss2d_dtype_t dt, const void *xdbl, const float *Wdt, int R, int RN,
-                          void *delta, cudaStream_t stream) {
-    dim3 grid((unsigned)ceil_div(s.L, kDtTok), (unsigned)ceil_div(s.D, kDtCh), (unsigned)(s.B * kPaths));
-    if (dt == SS2D_F32)
-        dtproj_kernel<float><<<grid, kDtTok, 0, stream>>>(static_cast<const float *>(xdbl), Wdt,
-                                                          static_cast<float *>(delta), s.D, s.L, R, RN);
-    else
-        dtproj_kernel<__nv_bfloat16><<<grid, kDtTok, 0, stream>>>(static_cast<const __nv_bfloat16 *>(xdbl), Wdt,
-                                                                  static_cast<__nv_bfloat16 *>(delta), s.D, s.L, R,
-                                                                  RN);
-    note_launch(stream);
-    return cudaGetLastError();
-}
-
 }  // namespace ss2d

@@ -12,8 +12,9 @@
 // The two contractions with R on one side are narrow (R <= 32) and bound by reading ddelta
 // once: rows_kernel gives each thread one token and its R sums (it also serves x_proj of
 // per-path sequences, R + 2N sums); dwdt_kernel gives each
-// thread one channel's R sums over a quarter of a staged token tile.  du_kernel stages both
-// operands of a 64-channel x 128-token tile whole (the contraction is R + 2N <= 64 long).
+// thread one channel's R sums over a quarter of a staged token tile.  chan_kernel stages both
+// operands of a 64-channel x 128-token tile whole (the contraction is R + 2N <= 64 long); it
+// also makes delta from x_dbl[:R] (dt_proj) for the backward and for wide ranks.
 // tr_gemm_kernel (d x_proj.weight) holds all R + 2N (<= 64) rows of a 128-column tile per CTA
 // and streams tokens through a 3-stage cp.async ring, 4 tokens per step.  The sums over tokens
 // are written per (batch item, token chunk) as partials that reduce_partials_kernel adds in
@@ -44,6 +45,14 @@ __device__ __forceinline__ void zero_quad(float *dst) {
     *reinterpret_cast<float4 *>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 __device__ __forceinline__ void zero_quad(__nv_bfloat16 *dst) { *reinterpret_cast<uint2 *>(dst) = make_uint2(0u, 0u); }
+
+// four consecutive outputs (16 bytes fp32, 8 bytes bf16, aligned)
+__device__ __forceinline__ void store4(float *p, float4 v) { *reinterpret_cast<float4 *>(p) = v; }
+__device__ __forceinline__ void store4(__nv_bfloat16 *p, float4 v) {
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
+    *reinterpret_cast<uint2 *>(p) = make_uint2(*reinterpret_cast<const uint32_t *>(&lo),
+                                               *reinterpret_cast<const uint32_t *>(&hi));
+}
 
 // four consecutive elements of a shared-memory row as floats (fp32: one 16-byte load; bf16: 8 bytes)
 __device__ __forceinline__ float4 ld4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
@@ -207,56 +216,68 @@ __global__ void __launch_bounds__(256, 2) dwdt_kernel(const Tin *__restrict__ dd
 constexpr int kDuM = 64;   // channels per du_kernel tile (8 thread rows x 8)
 constexpr int kDuL = 128;  // tokens per tile (32 thread columns x 4)
 
-// du[g, d, l] += sum_c Wx[k, c, d] dx_dbl[g, c, l] over a 64-channel x 128-token tile.  The
-// contraction is short (R + 2N <= 64), so both operands and the du tile itself are staged whole
-// (one batch of 16-byte cp.async when L and D are multiples of 4, plain loads otherwise) and
-// summed after one barrier; thread (ty, tx) holds channels ty + 8i and tokens 4tx..4tx+3, so a
-// warp's write of du covers 128 contiguous floats of one row.
-template <bool VEC>
-__global__ void __launch_bounds__(256) du_kernel(const float *__restrict__ dxdbl, const float *__restrict__ Wx,
-                                                 float *__restrict__ du, int64_t D, int64_t L, int RN, int nmt,
-                                                 int64_t nlt) {
+// out[g, d, l] (+)= sum_{c < C} M(k, d, c) in[g, c, l] over a 64-channel x 128-token tile, with
+// M(k, d, c) = Wm[k*w_ks + d*w_ds + c*w_cs], in in_gs elements per group (rows of L), out D rows of L
+// per group.  The contraction is short (C <= 64), so both operands (and, when ACC, the out tile
+// itself) are staged whole and summed after one barrier; thread (ty, tx) holds channels ty + 8i
+// and tokens 4tx..4tx+3, so a warp's write covers 128 contiguous elements of one row.  Token rows
+// are copied with 16-byte cp.async when VEC (L % 4 == 0) and fp32, else with plain loads.
+//   du:    du_seq += x_proj.weight^T dx_dbl   (fp32, ACC; M(k, d, c) = Wx[(k*RN + c)*D + d])
+//   delta: delta   = dt_proj.weight x_dbl[:R] (in dtype; M(k, d, c) = Wdt[(k*D + d)*R + c])
+template <typename Tin, typename Tout, bool ACC, bool VEC>
+__global__ void __launch_bounds__(256) chan_kernel(const Tin *__restrict__ in, int64_t in_gs,
+                                                   const float *__restrict__ Wm, int64_t w_ks, int64_t w_ds,
+                                                   int64_t w_cs, Tout *__restrict__ out, int64_t D, int64_t L, int C,
+                                                   int nmt, int64_t nlt) {
+    static_assert(!ACC || sizeof(Tout) == 4, "accumulation is in fp32");
     constexpr int AS = kDuM + 4, BS = kDuL + 4;
+    constexpr bool kAsyncIn = VEC && sizeof(Tin) == 4;
     extern __shared__ __align__(16) float du_smem[];
-    float *As = du_smem;             // [RN][AS]    Wx[k, c, d0 + .]
-    float *Bs = As + RN * AS;        // [RN][BS]    dx_dbl[g, c, l0 + .]
-    float *Us = Bs + RN * BS;        // [kDuM][BS]  du[g, d0 + ., l0 + .] (VEC only)
+    float *As = du_smem;        // [C][AS]    M(k, d0 + ., c)
+    float *Bs = As + C * AS;    // [C][BS]    in[g, c, l0 + .]
+    float *Us = Bs + C * BS;    // [kDuM][BS] out[g, d0 + ., l0 + .] (ACC and VEC only)
     const int t = threadIdx.x, ty = t / 32, tx = t % 32;
-    // one flat grid: channel tiles fastest (they share the dx_dbl tile, read once through L2)
+    // one flat grid: channel tiles fastest (they share the input tile, read once through L2)
     const int64_t bid = blockIdx.x, rest = bid / nmt, g = rest / nlt, k = g % kPaths;
     const int64_t d0 = (bid % nmt) * kDuM, l0 = (rest % nlt) * kDuL;
-    const float *src = dxdbl + g * RN * L + l0;
-    float *out = du + g * D * L + l0;
-    if (VEC) {
-        const int ca = RN * (kDuM / 4), cb = RN * (kDuL / 4), cu = kDuM * (kDuL / 4);
-        for (int c = t; c < ca + cb + cu; c += 256) {
-            if (c < ca) {
-                const int r = c / (kDuM / 4), j = 4 * (c % (kDuM / 4));
-                float *dst = As + r * AS + j;
-                if (d0 + j < D) cp_async16(dst, Wx + (k * RN + r) * D + d0 + j);
-                else zero_quad(dst);
-            } else if (c < ca + cb) {
-                const int cc = c - ca, r = cc / (kDuL / 4), j = 4 * (cc % (kDuL / 4));
+    const Tin *src = in + g * in_gs + l0;
+    Tout *o0 = out + g * D * L + l0;
+    // weights contiguous along the channels (w_ds = 1) and 16-byte aligned quads: cp.async too
+    const bool async_w = VEC && w_ds == 1 && D % 4 == 0 && w_cs % 4 == 0 && w_ks % 4 == 0;
+    if (async_w) {
+        for (int e = t; e < C * (kDuM / 4); e += 256) {
+            const int c = e / (kDuM / 4), j = 4 * (e % (kDuM / 4));
+            float *dst = As + c * AS + j;
+            if (d0 + j < D) cp_async16(dst, Wm + k * w_ks + d0 + j + c * w_cs);
+            else zero_quad(dst);
+        }
+    } else {
+        for (int e = t; e < C * kDuM; e += 256) {
+            const int c = e / kDuM, dd = e % kDuM;
+            As[c * AS + dd] = d0 + dd < D ? Wm[k * w_ks + (d0 + dd) * w_ds + c * w_cs] : 0.f;
+        }
+    }
+    if (kAsyncIn || (ACC && VEC) || async_w) {
+        const int cb = kAsyncIn ? C * (kDuL / 4) : 0, cu = (ACC && VEC) ? kDuM * (kDuL / 4) : 0;
+        for (int c = t; c < cb + cu; c += 256) {
+            if (c < cb) {
+                const int r = c / (kDuL / 4), j = 4 * (c % (kDuL / 4));
                 float *dst = Bs + r * BS + j;
-                if (l0 + j < L) cp_async16(dst, src + r * L + j);
+                if (l0 + j < L) cp_async16(dst, reinterpret_cast<const float *>(src) + r * L + j);
                 else zero_quad(dst);
             } else {
-                const int cc = c - ca - cb, r = cc / (kDuL / 4), j = 4 * (cc % (kDuL / 4));
-                if (d0 + r < D && l0 + j < L) cp_async16(Us + r * BS + j, out + (d0 + r) * L + j);
+                const int cc = c - cb, r = cc / (kDuL / 4), j = 4 * (cc % (kDuL / 4));
+                if (d0 + r < D && l0 + j < L) cp_async16(Us + r * BS + j, o0 + (d0 + r) * L + j);
             }
         }
         cp_async_commit();
-        cp_async_wait<0>();
-    } else {
-        for (int e = t; e < RN * kDuM; e += 256) {
-            const int c = e / kDuM, dd = e % kDuM;
-            As[c * AS + dd] = d0 + dd < D ? Wx[(k * RN + c) * D + d0 + dd] : 0.f;
-        }
-        for (int e = t; e < RN * kDuL; e += 256) {
-            const int c = e / kDuL, ll = e % kDuL;
-            Bs[c * BS + ll] = l0 + ll < L ? src[c * L + ll] : 0.f;
-        }
     }
+    if (!kAsyncIn)
+        for (int e = t; e < C * kDuL; e += 256) {
+            const int c = e / kDuL, ll = e % kDuL;
+            Bs[c * BS + ll] = l0 + ll < L ? ld(src + c * L + ll) : 0.f;
+        }
+    if (kAsyncIn || (ACC && VEC) || async_w) cp_async_wait<0>();
     __syncthreads();
     float acc[8][4];
 #pragma unroll
@@ -264,7 +285,7 @@ __global__ void __launch_bounds__(256) du_kernel(const float *__restrict__ dxdbl
 #pragma unroll
         for (int q = 0; q < 4; ++q) acc[i][q] = 0.f;
 #pragma unroll 4
-    for (int c = 0; c < RN; ++c) {
+    for (int c = 0; c < C; ++c) {
         const float4 bq = *reinterpret_cast<const float4 *>(&Bs[c * BS + 4 * tx]);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -279,20 +300,19 @@ __global__ void __launch_bounds__(256) du_kernel(const float *__restrict__ dxdbl
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const int64_t d = d0 + ty + 8 * i;
-        if (d >= D) continue;
-        float *o = out + d * L + l;
-        if (VEC) {
-            if (l0 + l >= L) continue;
-            float4 v = *reinterpret_cast<const float4 *>(&Us[(ty + 8 * i) * BS + l]);
-            v.x += acc[i][0];
-            v.y += acc[i][1];
-            v.z += acc[i][2];
-            v.w += acc[i][3];
-            *reinterpret_cast<float4 *>(o) = v;
+        if (d >= D || l0 + l >= L) continue;
+        Tout *o = o0 + d * L + l;
+        if (VEC) {  // the whole quad is inside the row (L % 4 == 0)
+            float4 v = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+            if (ACC) {
+                const float4 u = *reinterpret_cast<const float4 *>(&Us[(ty + 8 * i) * BS + l]);
+                v = make_float4(u.x + v.x, u.y + v.y, u.z + v.z, u.w + v.w);
+            }
+            store4(o, v);
         } else {
 #pragma unroll
             for (int q = 0; q < 4; ++q)
-                if (l0 + l + q < L) o[q] += acc[i][q];
+                if (l0 + l + q < L) st(o + q, ACC ? ld(o + q) + acc[i][q] : acc[i][q]);
         }
     }
 }
@@ -533,21 +553,51 @@ cudaError_t launch_xproj_seq(const LaunchShape &s, ss2d_dtype_t dt, const void *
 
 constexpr int kRNMax = kProjRMax + 2 * 16;  // rows of x_dbl: dt rank <= 32, d_state <= 16
 
-static size_t du_smem_bytes(int RN) { return ((size_t)RN * ((kDuM + 4) + (kDuL + 4)) + kDuM * (kDuL + 4)) * sizeof(float); }
+static size_t chan_smem_bytes(int C, bool acc) {
+    return ((size_t)C * ((kDuM + 4) + (kDuL + 4)) + (acc ? kDuM * (kDuL + 4) : 0)) * sizeof(float);
+}
 
-// du_seq (fp32, (B, 4D, L)) += x_proj.weight^T @ dx_dbl (fp32, group stride RN*L); du_seq 16-byte aligned
-cudaError_t launch_proj_bwd_du(const LaunchShape &s, const float *dxdbl, const float *Wx, int RN, float *du_seq,
-                               cudaStream_t stream) {
-    if (RN < 1 || RN > kRNMax) return cudaErrorInvalidValue;
+template <typename Tin, typename Tout, bool ACC>
+static cudaError_t chan_t(const LaunchShape &s, const void *in, int64_t in_gs, const float *Wm, int64_t w_ks,
+                          int64_t w_ds, int64_t w_cs, void *out, int C, cudaStream_t stream) {
+    if (C < 1 || C > kRNMax) return cudaErrorInvalidValue;
+    const bool vec = s.L % 4 == 0;  // token rows, and the out rows, 16-byte (fp32) / 8-byte (bf16) aligned
+    auto kern = vec ? chan_kernel<Tin, Tout, ACC, true> : chan_kernel<Tin, Tout, ACC, false>;
     // up to (64 * 200 + 64 * 132) * 4 = 84,992 bytes: opt in on the current device (cheap, right on any device)
-    const bool vec = s.L % 4 == 0 && s.D % 4 == 0;  // rows of du, dx_dbl and x_proj.weight 16-byte aligned
-    auto kern = vec ? du_kernel<true> : du_kernel<false>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)du_smem_bytes(kRNMax));
+    const cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)chan_smem_bytes(kRNMax, ACC));
     if (e != cudaSuccess) return e;
     const int nmt = (int)ceil_div(s.D, kDuM);
     const int64_t nlt = ceil_div(s.L, kDuL), blocks = nmt * nlt * s.B * kPaths;
     if (blocks > INT32_MAX) return cudaErrorInvalidConfiguration;
-    kern<<<(unsigned)blocks, 256, du_smem_bytes(RN), stream>>>(dxdbl, Wx, du_seq, s.D, s.L, RN, nmt, nlt);
+    kern<<<(unsigned)blocks, 256, chan_smem_bytes(C, ACC), stream>>>(static_cast<const Tin *>(in), in_gs, Wm, w_ks,
+                                                                     w_ds, w_cs, static_cast<Tout *>(out), s.D, s.L,
+                                                                     C, nmt, nlt);
+    return cudaSuccess;
+}
+
+// du_seq (fp32, (B, 4D, L)) += x_proj.weight^T @ dx_dbl (fp32, group stride RN*L); du_seq 16-byte aligned
+cudaError_t launch_proj_bwd_du(const LaunchShape &s, const float *dxdbl, const float *Wx, int RN, float *du_seq,
+                               cudaStream_t stream) {
+    // M(k, d, c) = Wx[(k*RN + c)*D + d]
+    const cudaError_t e = chan_t<float, float, true>(s, dxdbl, (int64_t)RN * s.L, Wx, (int64_t)RN * s.D, 1, s.D,
+                                                     du_seq, RN, stream);
+    if (e != cudaSuccess) return e;
+    note_launch(stream);
+    return cudaGetLastError();
+}
+
+// delta[b, k*D + d, l] = sum_r Wdt[k*D + d, r] xdbl[b, k, r, l] (in dtype): dt_proj for ranks where
+// the scan would spend more on R multiply-adds per step than on reading delta, and for the backward
+cudaError_t launch_dtproj(const LaunchShape &s, ss2d_dtype_t dt, const void *xdbl, const float *Wdt, int R, int RN,
+                          void *delta, cudaStream_t stream) {
+    if (R < 1 || R > kProjRMax) return cudaErrorInvalidValue;
+    // M(k, d, c) = Wdt[(k*D + d)*R + c]
+    const cudaError_t e =
+        dt == SS2D_F32 ? chan_t<float, float, false>(s, xdbl, (int64_t)RN * s.L, Wdt, s.D * R, R, 1, delta, R, stream)
+                       : chan_t<__nv_bfloat16, __nv_bfloat16, false>(s, xdbl, (int64_t)RN * s.L, Wdt, s.D * R, R, 1,
+                                                                     delta, R, stream);
+    if (e != cudaSuccess) return e;
     note_launch(stream);
     return cudaGetLastError();
 }
