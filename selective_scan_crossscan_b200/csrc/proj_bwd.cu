@@ -10,9 +10,10 @@
 // u_k is x along path k (x or its transpose, paths 2 and 3 backwards).
 //
 // The two contractions with R on one side are narrow (R <= 32) and bound by reading ddelta
-// once: rows_kernel gives each thread one token and its R sums (it also serves x_proj of
-// per-path sequences, R + 2N sums); dwdt_kernel gives each
-// thread one channel's R sums over a quarter of a staged token tile.  chan_kernel stages both
+// once: rows_kernel gives each thread one token and its R sums; dwdt_kernel gives each
+// thread one channel's R sums over a quarter of a staged token tile.  xseq_kernel (x_proj of the
+// per-path sequences the conv makes) streams the channels through a cp.async ring into an all-rows
+// x 128-token tile.  chan_kernel stages both
 // operands of a 64-channel x 128-token tile whole (the contraction is R + 2N <= 64 long); it
 // also makes delta from x_dbl[:R] (dt_proj) for the backward and for wide ranks.
 // tr_gemm_kernel (d x_proj.weight) holds all R + 2N (<= 64) rows of a 128-column tile per CTA
@@ -209,6 +210,109 @@ __global__ void __launch_bounds__(256, 2) dwdt_kernel(const Tin *__restrict__ dd
 #pragma unroll
     for (int r = 0; r < RB; ++r)
         if (r < R) dst[r] = acc[r];
+}
+
+// -------------------------------------------------- x_proj of per-path sequences --
+
+constexpr int kXsL = 128;  // tokens per CTA (32 lanes x 4)
+constexpr int kXsK = 16;   // channels per pipeline stage
+
+template <typename Tin, int TY>
+constexpr size_t xseq_smem_bytes() {
+    return (size_t)kStages * (8 * TY * (kXsK + 4) * sizeof(float) +
+                              kXsK * (sizeof(Tin) == 4 ? kXsL + 4 : kXsL + 8) * sizeof(Tin));
+}
+
+// xdbl[g, c, l] = sum_d W[k, c, d] u[g, d, l] for c < RN (g = b * 4 + k): all RN rows of a 128-token
+// tile per CTA, the channels streamed 16 at a time through a 3-stage cp.async ring (plain loads
+// when L or D is not a multiple of 4).  Warp ty holds rows ty + 8i (i < TY), lane tx tokens
+// 4tx..4tx+3 as two packed pairs: one 16-byte token load and TY broadcast weight loads feed 2*TY
+// FFMA2 per channel.
+template <typename Tin, int TY, bool VEC>
+__global__ void __launch_bounds__(256) xseq_kernel(const Tin *__restrict__ u, const float *__restrict__ W,
+                                                   Tin *__restrict__ xdbl, int64_t D, int64_t L, int RN,
+                                                   int64_t nlt) {
+    constexpr int TM = 8 * TY, PA = kXsK + 4, PB = sizeof(Tin) == 4 ? kXsL + 4 : kXsL + 8;
+    extern __shared__ __align__(16) unsigned char xs_smem[];
+    float *As = reinterpret_cast<float *>(xs_smem);                                        // [kStages][TM][PA]
+    Tin *Bs = reinterpret_cast<Tin *>(xs_smem + (size_t)kStages * TM * PA * sizeof(float));  // [kStages][kXsK][PB]
+    const int t = threadIdx.x, ty = t / 32, tx = t % 32;
+    const int64_t bid = blockIdx.x, g = bid / nlt, k = g % kPaths, l0 = (bid % nlt) * kXsL;
+    const Tin *src = u + g * D * L + l0;
+    const float *Wk = W + k * RN * D;
+    const int nst = (int)ceil_div(D, kXsK);
+    auto issue = [&](int st_) {
+        const int buf = st_ % kStages;
+        const int64_t d0 = (int64_t)st_ * kXsK;
+        float *as = As + (size_t)buf * TM * PA;
+        Tin *bs = Bs + (size_t)buf * kXsK * PB;
+        if (VEC) {  // D % 4 == 0 and L % 4 == 0: every quad is wholly inside or outside
+            for (int c = t; c < TM * (kXsK / 4); c += 256) {
+                const int r = c / (kXsK / 4), j = 4 * (c % (kXsK / 4));
+                float *dst = as + r * PA + j;
+                if (r < RN && d0 + j < D) cp_async16(dst, Wk + r * D + d0 + j);
+                else zero_quad(dst);
+            }
+            for (int c = t; c < kXsK * (kXsL / 4); c += 256) {
+                const int r = c / (kXsL / 4), j = 4 * (c % (kXsL / 4));
+                Tin *dst = bs + r * PB + j;
+                if (d0 + r < D && l0 + j < L) cp_async_quad(dst, src + (d0 + r) * L + j);
+                else zero_quad(dst);
+            }
+        } else {
+            for (int e = t; e < TM * kXsK; e += 256) {
+                const int r = e / kXsK, j = e % kXsK;
+                as[r * PA + j] = (r < RN && d0 + j < D) ? Wk[r * D + d0 + j] : 0.f;
+            }
+            for (int e = t; e < kXsK * kXsL; e += 256) {
+                const int r = e / kXsL, j = e % kXsL;
+                st(bs + r * PB + j, (d0 + r < D && l0 + j < L) ? ld(src + (d0 + r) * L + j) : 0.f);
+            }
+        }
+    };
+    float2 acc[TY][2];
+#pragma unroll
+    for (int i = 0; i < TY; ++i) acc[i][0] = acc[i][1] = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int st_ = 0; st_ < kStages - 1; ++st_) {
+        if (st_ < nst) issue(st_);
+        cp_async_commit();
+    }
+    for (int st_ = 0; st_ < nst; ++st_) {
+        cp_async_wait<kStages - 2>();
+        __syncthreads();  // stage st_ visible to all; every thread is done with stage st_ - 1's buffer
+        if (st_ + kStages - 1 < nst) issue(st_ + kStages - 1);
+        cp_async_commit();
+        const float *as = As + (size_t)(st_ % kStages) * TM * PA + ty * PA;
+        const Tin *bs = Bs + (size_t)(st_ % kStages) * kXsK * PB + 4 * tx;
+#pragma unroll
+        for (int dd = 0; dd < kXsK; ++dd) {
+            const float4 b = ld4(bs + dd * PB);
+            const float2 b01 = make_float2(b.x, b.y), b23 = make_float2(b.z, b.w);
+#pragma unroll
+            for (int i = 0; i < TY; ++i) {
+                const float a = as[8 * i * PA + dd];
+                acc[i][0] = __ffma2_rn(make_float2(a, a), b01, acc[i][0]);
+                acc[i][1] = __ffma2_rn(make_float2(a, a), b23, acc[i][1]);
+            }
+        }
+    }
+    const int64_t l = l0 + 4 * tx;
+    if (l >= L) return;
+    Tin *o = xdbl + g * RN * L + l;
+#pragma unroll
+    for (int i = 0; i < TY; ++i) {
+        const int c = ty + 8 * i;
+        if (c >= RN) continue;
+        const float v[4] = {acc[i][0].x, acc[i][0].y, acc[i][1].x, acc[i][1].y};
+        if (VEC) {  // the quad is inside the row and 16-byte (fp32) / 8-byte (bf16) aligned
+            store4(o + (int64_t)c * L, make_float4(v[0], v[1], v[2], v[3]));
+        } else {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                if (l + q < L) st(o + (int64_t)c * L + q, v[q]);
+        }
+    }
 }
 
 // ------------------------------------------------------------------------ du --
@@ -536,16 +640,41 @@ cudaError_t launch_proj_bwd_dtlow(const LaunchShape &s, ss2d_dtype_t dt, const v
     return cudaGetLastError();
 }
 
+template <typename Tin, int TY>
+static cudaError_t xseq_t(const LaunchShape &s, const void *u, const float *W, int RN, void *xdbl,
+                          cudaStream_t stream) {
+    const int64_t nlt = ceil_div(s.L, kXsL), blocks = nlt * s.B * kPaths;
+    if (blocks > INT32_MAX) return cudaErrorInvalidConfiguration;
+    const bool vec = s.L % 4 == 0 && s.D % 4 == 0;  // token and weight quads 16-byte (8-byte bf16) aligned
+    auto kern = vec ? xseq_kernel<Tin, TY, true> : xseq_kernel<Tin, TY, false>;
+    constexpr size_t smem = xseq_smem_bytes<Tin, TY>();  // at most 3 * (64 * 20 + 16 * 132) * 4 = 40,704 bytes
+    kern<<<(unsigned)blocks, 256, smem, stream>>>(static_cast<const Tin *>(u), W, static_cast<Tin *>(xdbl), s.D,
+                                                  s.L, RN, nlt);
+    return cudaSuccess;
+}
+
+template <typename Tin>
+static cudaError_t xseq_ty(const LaunchShape &s, const void *u, const float *W, int RN, void *xdbl,
+                           cudaStream_t stream) {
+    switch ((RN + 7) / 8) {  // rows R + 2N, 3..64, in one tile of 8 * TY rows
+        case 1: return xseq_t<Tin, 1>(s, u, W, RN, xdbl, stream);
+        case 2: return xseq_t<Tin, 2>(s, u, W, RN, xdbl, stream);
+        case 3: return xseq_t<Tin, 3>(s, u, W, RN, xdbl, stream);
+        case 4: return xseq_t<Tin, 4>(s, u, W, RN, xdbl, stream);
+        case 5: return xseq_t<Tin, 5>(s, u, W, RN, xdbl, stream);
+        case 6: return xseq_t<Tin, 6>(s, u, W, RN, xdbl, stream);
+        case 7: return xseq_t<Tin, 7>(s, u, W, RN, xdbl, stream);
+        case 8: return xseq_t<Tin, 8>(s, u, W, RN, xdbl, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
 // x_proj of per-path sequences: xdbl[b, k, c, l] = sum_d W[k, c, d] u[b, k*D + d, l] (in dtype)
 cudaError_t launch_xproj_seq(const LaunchShape &s, ss2d_dtype_t dt, const void *u, const float *W, int RN, void *xdbl,
                              cudaStream_t stream) {
     if (RN < 1 || RN > kProjRMax + 2 * 16) return cudaErrorInvalidValue;
-    // M(k, c, d) = W[(k*RN + c)*D + d]
-    const cudaError_t e =
-        dt == SS2D_F32
-            ? rows_r<float, float>(s, u, W, (int64_t)RN * s.D, s.D, 1, xdbl, (int64_t)RN * s.L, RN, stream)
-            : rows_r<__nv_bfloat16, __nv_bfloat16>(s, u, W, (int64_t)RN * s.D, s.D, 1, xdbl, (int64_t)RN * s.L, RN,
-                                                   stream);
+    const cudaError_t e = dt == SS2D_F32 ? xseq_ty<float>(s, u, W, RN, xdbl, stream)
+                                         : xseq_ty<__nv_bfloat16>(s, u, W, RN, xdbl, stream);
     if (e != cudaSuccess) return e;
     note_launch(stream);
     return cudaGetLastError();
