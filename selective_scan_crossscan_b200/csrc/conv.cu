@@ -33,6 +33,20 @@ __device__ __forceinline__ float path_x(const Tin *row, bool rev, int64_t L, int
     return m < 0 ? 0.f : ld(row + (rev ? L - 1 - m : m));
 }
 
+// four consecutive elements as floats / from floats (16 bytes fp32, 8 bytes bf16; aligned)
+__device__ __forceinline__ float4 ld4v(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+__device__ __forceinline__ float4 ld4v(const __nv_bfloat16 *p) {
+    const uint2 v = *reinterpret_cast<const uint2 *>(p);
+    return make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u), __uint_as_float(v.y << 16),
+                       __uint_as_float(v.y & 0xffff0000u));
+}
+__device__ __forceinline__ void st4v(float *p, float4 v) { *reinterpret_cast<float4 *>(p) = v; }
+__device__ __forceinline__ void st4v(__nv_bfloat16 *p, float4 v) {
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
+    *reinterpret_cast<uint2 *>(p) = make_uint2(*reinterpret_cast<const uint32_t *>(&lo),
+                                               *reinterpret_cast<const uint32_t *>(&hi));
+}
+
 // The CTA's row (b, k, d) and tile, decoded once in 32-bit arithmetic (the launcher checks the
 // row count fits), and the row's x (or xT) base, direction, weights and bias.
 template <typename Tin, int W>
@@ -52,12 +66,31 @@ struct ConvRow {
         for (int j = 0; j < W; ++j) w[j] = wt[((int64_t)k * D + d) * W + j];
         b0 = bias ? bias[(int64_t)k * D + d] : 0.f;
     }
-    // x_k at steps l - (W-1) .. l + kConvPer - 1: the windows of kConvPer consecutive outputs
+    // x_k at steps l - (W-1) .. l + kConvPer - 1: the windows of kConvPer consecutive outputs.
+    // VEC (L % 4 == 0, l % 4 == 0): two aligned quads of the row, steps l-4..l-1 and l..l+3, read
+    // backwards on the reversed paths (row positions L-l..L+3-l and L-4-l..L-1-l).
+    template <bool VEC>
     __device__ __forceinline__ void window(int64_t l, int64_t L, float (&xv)[kConvPer + W - 1]) const {
+        if (VEC) {
+            static_assert(kConvPer == 4, "quads");
+            float cat[8];  // x_k[l - 4 + j]
+            const float4 hi = ld4v(xr + (rev ? L - 4 - l : l));
+            const float4 lo = l >= 4 ? ld4v(xr + (rev ? L - l : l - 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
+            if (rev) {
+                cat[0] = lo.w; cat[1] = lo.z; cat[2] = lo.y; cat[3] = lo.x;
+                cat[4] = hi.w; cat[5] = hi.z; cat[6] = hi.y; cat[7] = hi.x;
+            } else {
+                cat[0] = lo.x; cat[1] = lo.y; cat[2] = lo.z; cat[3] = lo.w;
+                cat[4] = hi.x; cat[5] = hi.y; cat[6] = hi.z; cat[7] = hi.w;
+            }
 #pragma unroll
-        for (int i = 0; i < kConvPer + W - 1; ++i) {
-            const int64_t m = l - (W - 1) + i;
-            xv[i] = m < L ? path_x(xr, rev, L, m) : 0.f;
+            for (int i = 0; i < kConvPer + W - 1; ++i) xv[i] = cat[4 - (W - 1) + i];
+        } else {
+#pragma unroll
+            for (int i = 0; i < kConvPer + W - 1; ++i) {
+                const int64_t m = l - (W - 1) + i;
+                xv[i] = m < L ? path_x(xr, rev, L, m) : 0.f;
+            }
         }
     }
     __device__ __forceinline__ float pre(const float (&xv)[kConvPer + W - 1], int q) const {
@@ -68,7 +101,7 @@ struct ConvRow {
     }
 };
 
-template <typename Tin, int W>
+template <typename Tin, int W, bool VEC>
 __global__ void __launch_bounds__(kConvThreads) path_conv_fwd_kernel(const Tin *__restrict__ x, const Tin *__restrict__ xT,
                                                                      const float *__restrict__ w,
                                                                      const float *__restrict__ bias,
@@ -78,14 +111,19 @@ __global__ void __launch_bounds__(kConvThreads) path_conv_fwd_kernel(const Tin *
     const int64_t l = cr.l0 + kConvPer * threadIdx.x;
     if (l >= L) return;
     float xv[kConvPer + W - 1];
-    cr.window(l, L, xv);
+    cr.template window<VEC>(l, L, xv);
     Tin *o = u + cr.row * L + l;
+    if (VEC) {
+        st4v(o, make_float4(silu_f(cr.pre(xv, 0)), silu_f(cr.pre(xv, 1)), silu_f(cr.pre(xv, 2)),
+                            silu_f(cr.pre(xv, 3))));
+        return;
+    }
 #pragma unroll
     for (int q = 0; q < kConvPer; ++q)
         if (l + q < L) st(o + q, silu_f(cr.pre(xv, q)));
 }
 
-template <typename Tin, int W>
+template <typename Tin, int W, bool VEC>
 __global__ void __launch_bounds__(kConvThreads) path_conv_bwd_kernel(const Tin *__restrict__ x, const Tin *__restrict__ xT,
                                                                      const float *__restrict__ w,
                                                                      const float *__restrict__ bias,
@@ -103,13 +141,30 @@ __global__ void __launch_bounds__(kConvThreads) path_conv_bwd_kernel(const Tin *
         return dur[m] * sg * fmaf(p, 1.f - sg, 1.f);
     };
     float xv[kConvPer + W - 1];
-    cr.window(l, L, xv);
     float dpl[kConvPer];
+    if (VEC) {
+        if (l < L) {
+            cr.template window<true>(l, L, xv);
+            const float4 g4 = ld4v(dur + l);
+            const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
 #pragma unroll
-    for (int q = 0; q < kConvPer; ++q) {
-        dpl[q] = l + q < L ? dpre_of(cr.pre(xv, q), l + q) : 0.f;
-        dp[kConvPer * t + q] = dpl[q];
+            for (int q = 0; q < kConvPer; ++q) {
+                const float p = cr.pre(xv, q), sg = sigmoid_f(p);
+                dpl[q] = gv[q] * sg * fmaf(p, 1.f - sg, 1.f);
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < kConvPer + W - 1; ++i) xv[i] = 0.f;
+#pragma unroll
+            for (int q = 0; q < kConvPer; ++q) dpl[q] = 0.f;
+        }
+    } else {
+        cr.template window<false>(l, L, xv);
+#pragma unroll
+        for (int q = 0; q < kConvPer; ++q) dpl[q] = l + q < L ? dpre_of(cr.pre(xv, q), l + q) : 0.f;
     }
+#pragma unroll
+    for (int q = 0; q < kConvPer; ++q) dp[kConvPer * t + q] = dpl[q];
     if (t < W - 1) {  // the halo: dpre of the W-1 steps after the tile
         const int64_t m = cr.l0 + kConvTok + t;
         float p = cr.b0;
@@ -118,13 +173,24 @@ __global__ void __launch_bounds__(kConvThreads) path_conv_bwd_kernel(const Tin *
         dp[kConvTok + t] = m < L ? dpre_of(p, m) : 0.f;
     }
     __syncthreads();
+    if (VEC && l < L) {
+        float a[kConvPer];
 #pragma unroll
-    for (int q = 0; q < kConvPer; ++q) {
-        if (l + q >= L) break;
-        float acc = 0.f;
+        for (int q = 0; q < kConvPer; ++q) {
+            a[q] = 0.f;
 #pragma unroll
-        for (int j = 0; j < W; ++j) acc = fmaf(cr.w[j], dp[kConvPer * t + q + (W - 1) - j], acc);
-        dxs[cr.row * L + l + q] = acc;
+            for (int j = 0; j < W; ++j) a[q] = fmaf(cr.w[j], dp[kConvPer * t + q + (W - 1) - j], a[q]);
+        }
+        st4v(dxs + cr.row * L + l, make_float4(a[0], a[1], a[2], a[3]));
+    } else if (!VEC) {
+#pragma unroll
+        for (int q = 0; q < kConvPer; ++q) {
+            if (l + q >= L) break;
+            float acc = 0.f;
+#pragma unroll
+            for (int j = 0; j < W; ++j) acc = fmaf(cr.w[j], dp[kConvPer * t + q + (W - 1) - j], acc);
+            dxs[cr.row * L + l + q] = acc;
+        }
     }
     // weight and bias terms: this thread's steps in order, a fixed shuffle tree per warp, then the
     // warps in order
@@ -184,9 +250,11 @@ static cudaError_t conv_fwd_t(const LaunchShape &s, const void *x, const void *x
                               void *u, cudaStream_t stream) {
     const int64_t nlt = ceil_div(s.L, kConvTok), blocks = s.B * kPaths * s.D * nlt;
     if (blocks > INT32_MAX) return cudaErrorInvalidConfiguration;  // also keeps the 32-bit row decode exact
-    path_conv_fwd_kernel<Tin, W><<<(unsigned)blocks, kConvThreads, 0, stream>>>(
-        static_cast<const Tin *>(x), static_cast<const Tin *>(xT), w, bias, static_cast<Tin *>(u), (uint32_t)s.D,
-        s.L, (uint32_t)nlt);
+    // quads of 4 steps are aligned (16 bytes fp32, 8 bytes bf16) when L % 4 == 0
+    auto kern = s.L % 4 == 0 ? path_conv_fwd_kernel<Tin, W, true> : path_conv_fwd_kernel<Tin, W, false>;
+    kern<<<(unsigned)blocks, kConvThreads, 0, stream>>>(static_cast<const Tin *>(x), static_cast<const Tin *>(xT), w,
+                                                        bias, static_cast<Tin *>(u), (uint32_t)s.D, s.L,
+                                                        (uint32_t)nlt);
     return cudaSuccess;
 }
 
@@ -216,9 +284,9 @@ static cudaError_t conv_bwd_t(const LaunchShape &s, const void *x, const void *x
                               const float *du, float *dxs, float *part, cudaStream_t stream) {
     const int64_t nlt = ceil_div(s.L, kConvTok), blocks = s.B * kPaths * s.D * nlt;
     if (blocks > INT32_MAX) return cudaErrorInvalidConfiguration;  // also keeps the 32-bit row decode exact
-    path_conv_bwd_kernel<Tin, W><<<(unsigned)blocks, kConvThreads, 0, stream>>>(
-        static_cast<const Tin *>(x), static_cast<const Tin *>(xT), w, bias, du, dxs, part, (uint32_t)s.D, s.L,
-        (uint32_t)nlt);
+    auto kern = s.L % 4 == 0 ? path_conv_bwd_kernel<Tin, W, true> : path_conv_bwd_kernel<Tin, W, false>;
+    kern<<<(unsigned)blocks, kConvThreads, 0, stream>>>(static_cast<const Tin *>(x), static_cast<const Tin *>(xT), w,
+                                                        bias, du, dxs, part, (uint32_t)s.D, s.L, (uint32_t)nlt);
     return cudaSuccess;
 }
 
