@@ -315,10 +315,10 @@ __global__ void __launch_bounds__(256) xseq_kernel(const Tin *__restrict__ u, co
     }
 }
 
-// ------------------------------------------------------------------------ du --
+// ------------------------------------------------ short contractions (du, delta) --
 
-constexpr int kDuM = 64;   // channels per du_kernel tile (8 thread rows x 8)
-constexpr int kDuL = 128;  // tokens per tile (32 thread columns x 4)
+constexpr int kChM = 64;   // channels per chan_kernel tile (8 thread rows x 8)
+constexpr int kChL = 128;  // tokens per tile (32 thread columns x 4)
 
 // out[g, d, l] (+)= sum_{c < C} M(k, d, c) in[g, c, l] over a 64-channel x 128-token tile, with
 // M(k, d, c) = Wm[k*w_ks + d*w_ds + c*w_cs], in in_gs elements per group (rows of L), out D rows of L
@@ -334,51 +334,51 @@ __global__ void __launch_bounds__(256) chan_kernel(const Tin *__restrict__ in, i
                                                    int64_t w_cs, Tout *__restrict__ out, int64_t D, int64_t L, int C,
                                                    int nmt, int64_t nlt) {
     static_assert(!ACC || sizeof(Tout) == 4, "accumulation is in fp32");
-    constexpr int AS = kDuM + 4, BS = kDuL + 4;
+    constexpr int AS = kChM + 4, BS = kChL + 4;
     constexpr bool kAsyncIn = VEC && sizeof(Tin) == 4;
-    extern __shared__ __align__(16) float du_smem[];
-    float *As = du_smem;        // [C][AS]    M(k, d0 + ., c)
+    extern __shared__ __align__(16) float chan_smem[];
+    float *As = chan_smem;      // [C][AS]    M(k, d0 + ., c)
     float *Bs = As + C * AS;    // [C][BS]    in[g, c, l0 + .]
-    float *Us = Bs + C * BS;    // [kDuM][BS] out[g, d0 + ., l0 + .] (ACC and VEC only)
+    float *Us = Bs + C * BS;    // [kChM][BS] out[g, d0 + ., l0 + .] (ACC and VEC only)
     const int t = threadIdx.x, ty = t / 32, tx = t % 32;
     // one flat grid: channel tiles fastest (they share the input tile, read once through L2)
     const int64_t bid = blockIdx.x, rest = bid / nmt, g = rest / nlt, k = g % kPaths;
-    const int64_t d0 = (bid % nmt) * kDuM, l0 = (rest % nlt) * kDuL;
+    const int64_t d0 = (bid % nmt) * kChM, l0 = (rest % nlt) * kChL;
     const Tin *src = in + g * in_gs + l0;
     Tout *o0 = out + g * D * L + l0;
     // weights contiguous along the channels (w_ds = 1) and 16-byte aligned quads: cp.async too
     const bool async_w = VEC && w_ds == 1 && D % 4 == 0 && w_cs % 4 == 0 && w_ks % 4 == 0;
     if (async_w) {
-        for (int e = t; e < C * (kDuM / 4); e += 256) {
-            const int c = e / (kDuM / 4), j = 4 * (e % (kDuM / 4));
+        for (int e = t; e < C * (kChM / 4); e += 256) {
+            const int c = e / (kChM / 4), j = 4 * (e % (kChM / 4));
             float *dst = As + c * AS + j;
             if (d0 + j < D) cp_async16(dst, Wm + k * w_ks + d0 + j + c * w_cs);
             else zero_quad(dst);
         }
     } else {
-        for (int e = t; e < C * kDuM; e += 256) {
-            const int c = e / kDuM, dd = e % kDuM;
+        for (int e = t; e < C * kChM; e += 256) {
+            const int c = e / kChM, dd = e % kChM;
             As[c * AS + dd] = d0 + dd < D ? Wm[k * w_ks + (d0 + dd) * w_ds + c * w_cs] : 0.f;
         }
     }
     if (kAsyncIn || (ACC && VEC) || async_w) {
-        const int cb = kAsyncIn ? C * (kDuL / 4) : 0, cu = (ACC && VEC) ? kDuM * (kDuL / 4) : 0;
+        const int cb = kAsyncIn ? C * (kChL / 4) : 0, cu = (ACC && VEC) ? kChM * (kChL / 4) : 0;
         for (int c = t; c < cb + cu; c += 256) {
             if (c < cb) {
-                const int r = c / (kDuL / 4), j = 4 * (c % (kDuL / 4));
+                const int r = c / (kChL / 4), j = 4 * (c % (kChL / 4));
                 float *dst = Bs + r * BS + j;
                 if (l0 + j < L) cp_async16(dst, reinterpret_cast<const float *>(src) + r * L + j);
                 else zero_quad(dst);
             } else {
-                const int cc = c - cb, r = cc / (kDuL / 4), j = 4 * (cc % (kDuL / 4));
+                const int cc = c - cb, r = cc / (kChL / 4), j = 4 * (cc % (kChL / 4));
                 if (d0 + r < D && l0 + j < L) cp_async16(Us + r * BS + j, o0 + (d0 + r) * L + j);
             }
         }
         cp_async_commit();
     }
     if (!kAsyncIn)
-        for (int e = t; e < C * kDuL; e += 256) {
-            const int c = e / kDuL, ll = e % kDuL;
+        for (int e = t; e < C * kChL; e += 256) {
+            const int c = e / kChL, ll = e % kChL;
             Bs[c * BS + ll] = l0 + ll < L ? ld(src + c * L + ll) : 0.f;
         }
     if (kAsyncIn || (ACC && VEC) || async_w) cp_async_wait<0>();
@@ -683,7 +683,7 @@ cudaError_t launch_xproj_seq(const LaunchShape &s, ss2d_dtype_t dt, const void *
 constexpr int kRNMax = kProjRMax + 2 * 16;  // rows of x_dbl: dt rank <= 32, d_state <= 16
 
 static size_t chan_smem_bytes(int C, bool acc) {
-    return ((size_t)C * ((kDuM + 4) + (kDuL + 4)) + (acc ? kDuM * (kDuL + 4) : 0)) * sizeof(float);
+    return ((size_t)C * ((kChM + 4) + (kChL + 4)) + (acc ? kChM * (kChL + 4) : 0)) * sizeof(float);
 }
 
 template <typename Tin, typename Tout, bool ACC>
@@ -696,8 +696,8 @@ static cudaError_t chan_t(const LaunchShape &s, const void *in, int64_t in_gs, c
     const cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)chan_smem_bytes(kRNMax, ACC));
     if (e != cudaSuccess) return e;
-    const int nmt = (int)ceil_div(s.D, kDuM);
-    const int64_t nlt = ceil_div(s.L, kDuL), blocks = nmt * nlt * s.B * kPaths;
+    const int nmt = (int)ceil_div(s.D, kChM);
+    const int64_t nlt = ceil_div(s.L, kChL), blocks = nmt * nlt * s.B * kPaths;
     if (blocks > INT32_MAX) return cudaErrorInvalidConfiguration;
     kern<<<(unsigned)blocks, 256, chan_smem_bytes(C, ACC), stream>>>(static_cast<const Tin *>(in), in_gs, Wm, w_ks,
                                                                      w_ds, w_cs, static_cast<Tout *>(out), s.D, s.L,
