@@ -86,3 +86,29 @@ def test_algorithmic_bytes_match_the_stated_figure():
     # read u (308.3 MB), delta (1233.1 MB), B and C (102.8 MB each), write y (308.3 MB) in fp32
     assert abs(bench.fwd_algorithmic_bytes(w) / 1e6 - 2055.3) < 0.5
     assert w.updates == 4_932_501_504
+
+
+def test_backward_and_producer_bytes():
+    import bench
+    import ss2d_inputs
+    w = ss2d_inputs.workload(4)  # B=32 stage-1 shapes, fp32
+    # forward 513.9 MB; backward reads x, delta, B, C, dy and writes dx, ddelta, dB, dC: 950.6 MB
+    assert abs(bench.fwd_algorithmic_bytes(w) / 1e6 - 513.9) < 0.5
+    assert abs(bench.bwd_algorithmic_bytes(w) / 1e6 - 950.6) < 0.5
+    w1 = ss2d_inputs.workload(1)
+    R = ss2d_inputs.dt_rank_of(w1.dim)
+    # x read, y written (308.3 MB each), x_dbl (B, 4, R+2N, L) written, the small weights
+    img = w1.batch * w1.dim * w1.L * 4
+    xdbl = w1.batch * 4 * (R + 2 * w1.d_state) * w1.L * 4
+    weights = 4 * (4 * (R + 2 * w1.d_state) * w1.dim + 4 * w1.dim * R + 4 * w1.dim * (w1.d_state + 2))
+    assert bench.proj_algorithmic_bytes(w1, R) == 2 * img + xdbl + weights
+
+
+def test_recorded_traffic_needs_the_captured_sources(monkeypatch):
+    import bench
+    rec = bench.recorded_traffic("vmamba_t_stage1_fp32")
+    assert rec is None or rec > bench.fwd_algorithmic_bytes(__import__("ss2d_inputs").workload(1))
+    # any change to the hashed kernel sources invalidates the record
+    monkeypatch.setattr(bench, "source_hash", lambda files=None: "0" * 16)
+    assert bench.recorded_traffic("vmamba_t_stage1_fp32") is None
+    assert bench.recorded_traffic("no such workload") is None
