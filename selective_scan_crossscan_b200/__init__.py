@@ -38,6 +38,7 @@ __all__ = [
     "bimamba_scan", "path_tables", "cross_scan_table", "cross_merge_table", "ss2d_forward_table",
     "ss2d_backward_table", "PATHS_CROSS", "PATHS_DIAGONAL", "ss2d_forward_proj", "ss2d_backward_proj", "OP_BACKWARD_PROJ",
     "ss2d_forward_proj_conv", "ss2d_backward_proj_conv", "OP_FORWARD_PROJ_CONV", "OP_BACKWARD_PROJ_CONV",
+    "ss2d_proj", "SS2DProjFunction",
     "ss2d_backward", "SS2DFunction", "ss2d", "workspace_bytes", "chunk_states_elems", "launch_count",
     "library_path", "CHUNK_LEN", "trace_events",
 ]
@@ -801,3 +802,44 @@ def ss2d_backward_proj_conv(x, conv_weight, conv_bias, x_proj_weight, dt_proj_we
     _check(st, "ss2d_backward_proj_conv")
     return dict(dx=dx, dconv_weight=dcw, dconv_bias=dcb, dx_proj_weight=dWx, ddt_proj_weight=dWdt,
                 ddt_proj_bias=dbias, dA=dA, dD=dD)
+
+
+class SS2DProjFunction(torch.autograd.Function):
+    """autograd wrapper of the SS2D forward with its per-path producer (MambaInnerFn's x_proj and
+    dt_proj, and with conv_weight its causal depthwise conv + SiLU): the forward keeps x_dbl and
+    the chunk states, the backward runs ss2d_backward_proj(_conv)."""
+
+    @staticmethod
+    def forward(ctx, x, x_proj_weight, dt_proj_weight, dt_proj_bias, A, D, conv_weight, conv_bias, delta_softplus):
+        if conv_weight is None:
+            y, xd, cs = ss2d_forward_proj(x, x_proj_weight, dt_proj_weight, dt_proj_bias, A, D, delta_softplus,
+                                          return_x_dbl=True, return_chunk_states=True)
+        else:
+            y, xd, cs = ss2d_forward_proj_conv(x, conv_weight, conv_bias, x_proj_weight, dt_proj_weight,
+                                               dt_proj_bias, A, D, delta_softplus, return_x_dbl=True,
+                                               return_chunk_states=True)
+        ctx.save_for_backward(x, x_proj_weight, dt_proj_weight, dt_proj_bias, A, D, conv_weight, conv_bias, xd, cs)
+        ctx.delta_softplus = delta_softplus
+        return y
+
+    @staticmethod
+    def backward(ctx, dy):
+        x, Wx, Wdt, bias, A, D, cw, cb, xd, cs = ctx.saved_tensors
+        dy = dy.contiguous()
+        if cw is None:
+            g = ss2d_backward_proj(x, Wx, Wdt, bias, A, D, xd, dy, ctx.delta_softplus, chunk_states=cs)
+            dcw = dcb = None
+        else:
+            g = ss2d_backward_proj_conv(x, cw, cb, Wx, Wdt, bias, A, D, xd, dy, ctx.delta_softplus, chunk_states=cs)
+            dcw, dcb = g["dconv_weight"], g["dconv_bias"]
+        return (g["dx"], g["dx_proj_weight"], g["ddt_proj_weight"], g["ddt_proj_bias"], g["dA"], g["dD"], dcw, dcb,
+                None)
+
+
+def ss2d_proj(x, x_proj_weight, dt_proj_weight, dt_proj_bias, A, D=None, conv_weight=None, conv_bias=None,
+              delta_softplus=True):
+    """Differentiable SS2D with its per-path producer: y = ss2d_forward_proj(...) or, with conv_weight
+    (4, D, d_conv), ss2d_forward_proj_conv(...).  Gradients reach x, both projection weights, the
+    dt_proj bias, A, D and the conv weight and bias."""
+    return SS2DProjFunction.apply(x, x_proj_weight, dt_proj_weight, dt_proj_bias, A, D, conv_weight, conv_bias,
+                                  delta_softplus)

@@ -933,3 +933,27 @@ def test_full_size_fwd_bwd_fp32():
     g3 = ss.ss2d_backward(sl["x"], sl["delta"], sl["A"], sl["B"], sl["C"], sl["D"], sl["delta_bias"], True, sl["dy"])
     for name in ("dA", "dD", "ddelta_bias"):
         assert_rel_l2(g3[name], ref[name], GRAD_TOL, f"c4 items {name}")
+
+
+@pytest.mark.parametrize("d_conv", [0, 4])
+def test_ss2d_proj_autograd(d_conv):
+    # the differentiable producer path against the oracle's gradients, with and without the conv
+    w, inp = _conv_case(1, 24, 6, 8, 16, 4, seed=70)
+    names = ("x", "x_proj_weight", "dt_proj_weight", "dt_proj_bias", "A", "D", "conv_weight", "conv_bias")
+    lv = {k: inp[k].cuda().requires_grad_(True) for k in names}
+    cw, cb = (lv["conv_weight"], lv["conv_bias"]) if d_conv else (None, None)
+    y = ss.ss2d_proj(lv["x"], lv["x_proj_weight"], lv["dt_proj_weight"], lv["dt_proj_bias"], lv["A"], lv["D"], cw, cb)
+    dy = torch.randn(y.shape, generator=torch.Generator(device="cuda").manual_seed(71), device="cuda")
+    y.backward(dy)
+    dy_np = dy.double().cpu().numpy()
+    if d_conv:
+        ref = oracle.ss2d_backward_proj_conv(*_conv_call_args(inp), True, dy_np)
+        pairs = dict(x="dx", conv_weight="dconv_weight", conv_bias="dconv_bias", x_proj_weight="dx_proj_weight",
+                     dt_proj_weight="ddt_proj_weight", dt_proj_bias="ddt_proj_bias", A="dA", D="dD")
+    else:
+        ref = oracle.ss2d_backward_proj(inp["x"], inp["x_proj_weight"], inp["dt_proj_weight"], inp["dt_proj_bias"],
+                                        inp["A"], inp["D"], True, dy_np)
+        pairs = dict(x="dx", x_proj_weight="dx_proj_weight", dt_proj_weight="ddt_proj_weight",
+                     dt_proj_bias="ddt_proj_bias", A="dA", D="dD")
+    for leaf, rname in pairs.items():
+        assert_rel_l2(lv[leaf].grad, ref[rname], GRAD_TOL, f"{leaf} (d_conv {d_conv})")
