@@ -223,8 +223,8 @@ def ss2d_backward_proj(x, x_proj_weight, dt_proj_weight, dt_proj_bias, A, D, del
 def path_conv(x, conv_weight, conv_bias=None):
     """The causal depthwise conv with SiLU that MambaInnerFn.forward ("vision mamba-yolov8",
     section 2) applies before x_proj (causal_conv1d_fwd(x, weight, bias, True)), taken along
-    every SS2D path, each path with its own weights, as the Visual Mamba page's SS2D runs one
-    Mamba block per scan direction:
+    every SS2D path, each path with its own weights, as the SS2D of "Visual Mamba实战从零开始搭建
+    图像分类模型附PyTorch代码" (section 3) runs one Mamba block per scan direction:
         pre_k[d, l] = bias[k, d] + sum_j w[k, d, j] * x_k[d, l - (W-1) + j]   (x_k = 0 before step 0)
         u_k[d, l]   = silu(pre_k[d, l]) = pre / (1 + exp(-pre))
     with x_k = x read along path k (CrossScan).  x (Bn, D, H, W); conv_weight (4, D, W);

@@ -2,9 +2,9 @@
 //
 // MambaInnerFn.forward ("vision mamba-yolov8", section 2) passes its input through
 // causal_conv1d_fwd(x, weight, bias, True) before x_proj: a depthwise conv of width W over the
-// sequence, reading the current and the W-1 previous steps, then SiLU.  The Visual Mamba page's
-// SS2D runs one Mamba block per scan direction, so here every path k has its own weights and
-// convolves x read along its own step order:
+// sequence, reading the current and the W-1 previous steps, then SiLU.  The SS2D of "Visual
+// Mamba实战从零开始搭建图像分类模型附PyTorch代码" (section 3) runs one Mamba block per scan direction,
+// so here every path k has its own weights and convolves x read along its own step order:
 //     pre_k[d, l] = bias[k, d] + sum_j w[k, d, j] x_k[d, l - (W-1) + j]     (x_k = 0 before step 0)
 //     u_k[d, l]   = silu(pre_k[d, l])
 // x_k is x (k = 0) or its transpose (k = 1) read forwards, or backwards (k = 2, 3).
